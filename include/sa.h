@@ -1,0 +1,243 @@
+/*
+ * sa.h -- C ABI of libsa: learned top-k sparse attention on B200 (sm_100a).
+ *
+ * The hot path has three stages (token sparse attention, "Latent Sparse
+ * Attention", paperpeel 2610.42147, section 2 and 2.1):
+ *   (1) indexer:   score(t,s) = sum_h w[t,h] * ReLU(q_idx[t,h] . k_idx[s]), s <= t
+ *   (2) top-k:     the k visible keys of largest score (ties: lower key index)
+ *   (3) attention: softmax attention over the selected keys of one shared KV
+ *                  head, one index set shared by every query head (section 3.2)
+ * plus an optional two-stage indexer that first keeps the best mean-pooled key
+ * blocks and runs (1)-(2) only inside them (HISA, theflow "related" page;
+ * block score by the mean of its keys, LSA section 2.2).
+ *
+ * Conventions (all calls):
+ *  - Every pointer argument is DEVICE memory unless marked "host". The caller
+ *    owns every buffer; the library never allocates, and never synchronises
+ *    the host except where a call says so.
+ *  - Tensors are row-major and contiguous; the innermost row of every index
+ *    tensor (q_idx, k_idx) must start on a 16-byte boundary (TMA operand).
+ *  - Calls are ordered on `stream` and reentrant; there is no global mutable
+ *    state. Argument validation is synchronous and happens before any launch;
+ *    a failed validation launches nothing.
+ *  - Index rows ("J", appendix F.1 "Attention kernels") are int32 key
+ *    positions (KV-cache slots) in UNSPECIFIED order, padded with -1 at the
+ *    tail when fewer than k keys are visible. The attention does not depend on
+ *    their order (appendix F.1, "Selection by threshold").
+ *  - Errors: SA_ERR_INVALID_ARGUMENT (bad sizes, null pointers, misaligned
+ *    rows), SA_ERR_UNSUPPORTED (a valid shape this build does not implement),
+ *    SA_ERR_WORKSPACE_TOO_SMALL, SA_ERR_CUDA (a launch failed; the stream
+ *    state is whatever CUDA reports), SA_ERR_TIMEOUT is reported only through
+ *    the device status word (a bounded wait inside a kernel gave up).
+ */
+#ifndef SA_H_
+#define SA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARGUMENT = 1,
+  SA_ERR_UNSUPPORTED = 2,
+  SA_ERR_WORKSPACE_TOO_SMALL = 3,
+  SA_ERR_CUDA = 4,
+  SA_ERR_TIMEOUT = 5,
+  SA_ERR_INTERNAL = 6
+} sa_status;
+
+typedef enum {
+  SA_BF16 = 0,      /* bfloat16 */
+  SA_FP8_E4M3 = 1,  /* OCP e4m3 ("fn": no inf, 0x7F/0xFF NaN), one fp32 scale per row */
+  SA_F32 = 2
+} sa_dtype;
+
+typedef enum { SA_MODE_FLAT = 0, SA_MODE_TWO_STAGE = 1 } sa_mode;
+
+typedef enum {
+  SA_OP_INDEX_SCORES = 0,
+  SA_OP_TOPK = 1,
+  SA_OP_SPARSE_ATTN = 2,
+  SA_OP_PREFILL = 3,
+  SA_OP_DECODE = 4
+} sa_op;
+
+/*
+ * Indexer operands (stage 1 of the path; the lightweight indexer "with fewer
+ * heads, smaller dimension, lower precision", LSA section 2.1).
+ *
+ * Prefill (batch == 0): query row i sits at absolute position q_pos0 + i and
+ *   sees keys s <= q_pos0 + i, s < n_k.
+ *     q        [n_q, n_heads, d_idx]  (fp8 bytes or bf16)
+ *     q_scale  [n_q, n_heads] fp32    (fp8 only; NULL for bf16)
+ *     k        [n_k, d_idx]
+ *     k_scale  [n_k] fp32             (fp8 only; NULL for bf16)
+ *     w        [n_q, n_heads] fp32    head weights, expected >= 0
+ *   FP8 values are q_scale * e4m3(q) and k_scale * e4m3(k).
+ * Decode (batch > 0): sequence b has ONE query (n_q must equal batch) and its
+ *   own cache of capacity n_k keys; the query sees keys s < seq_lens[b]
+ *   (its own key is the cache's last row).
+ *     q [batch, n_heads, d_idx], q_scale [batch, n_heads], w [batch, n_heads]
+ *     k [batch, n_k, d_idx], k_scale [batch, n_k]
+ *     seq_lens [batch] int32 device, each in [1, n_k]; NULL means n_k for all.
+ * Supported (else SA_ERR_UNSUPPORTED): fp8 with d_idx = 128 and n_heads in
+ *            {32, 64}; bf16 with d_idx = 32 and n_heads in {4, 8} (prefill only).
+ */
+typedef struct {
+  int32_t n_q;
+  int32_t n_k;
+  int32_t q_pos0;
+  int32_t n_heads;
+  int32_t d_idx;
+  sa_dtype dtype;
+  const void* q;
+  const float* q_scale;
+  const void* k;
+  const float* k_scale;
+  const float* w;
+  int32_t batch;
+  const int32_t* seq_lens;
+} sa_indexer_in;
+
+/*
+ * Attention operands (stage 3): one shared KV head (MQA).
+ *   q       [n_q, n_q_heads, head_dim] bf16
+ *   k_cache [n_k, head_dim] bf16 (decode: [batch, n_k, head_dim])
+ *   v_cache [n_k, head_dim] bf16 (decode: [batch, n_k, head_dim])
+ *   head_dim in {64, 128}; n_q_heads in {8, 16}.
+ *   softmax_scale: logits are scale * q . k; 0 means 1/sqrt(head_dim).
+ */
+typedef struct {
+  int32_t n_q;
+  int32_t n_k;
+  int32_t n_q_heads;
+  int32_t head_dim;
+  float softmax_scale;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  int32_t batch;
+} sa_attn_in;
+
+/* Device-side status word, written by sa_prefill / sa_decode when non-NULL.
+ * Read it after synchronising the stream. */
+typedef struct {
+  uint32_t error;          /* 0 = ok; SA_ERR_TIMEOUT if a bounded wait gave up */
+  uint32_t timeout_site;   /* which wait gave up (diagnostic) */
+  uint32_t fallback_rows;  /* rows re-selected from their whole score row */
+  uint32_t overflow_rows;  /* rows whose candidate list overflowed */
+} sa_device_status;
+
+typedef struct {
+  int32_t k;             /* top-k budget, 1..4096 */
+  sa_mode mode;          /* FLAT or TWO_STAGE */
+  int32_t block_size;    /* two-stage key block (64) */
+  int32_t keep_blocks;   /* two-stage kept blocks per query (>= 2, <= 64) */
+  int32_t chunk_rows;    /* query rows per chunk (0 = library default) */
+  sa_device_status* status;  /* device, nullable; zeroed by the call */
+  int32_t test_hook;     /* 0 in production; see SA_HOOK_* */
+} sa_prefill_opts;
+
+typedef struct {
+  int32_t k;
+  sa_device_status* status;  /* device, nullable; zeroed by the call */
+  int32_t test_hook;
+} sa_decode_opts;
+
+/* test hooks: force the threshold of the streaming selector */
+#define SA_HOOK_NONE 0
+#define SA_HOOK_THETA_POS_INF 1   /* every row misses low -> whole-row fallback */
+#define SA_HOOK_THETA_NEG_INF 2   /* every key is a candidate -> overflow path */
+#define SA_HOOK_STALL_WAIT 3      /* a device wait that never completes -> SA_ERR_TIMEOUT */
+
+/* Human-readable name of a status code (host, static storage). */
+const char* sa_status_string(sa_status s);
+
+/*
+ * sa_index_scores: writes the causal indexer score table (stage 1).
+ *   scores[i * ld + s] = score(q_pos0 + i, s) for s <= q_pos0 + i, -inf for
+ *   the other s < n_k; columns >= n_k are not touched. ld >= n_k.
+ * Prefill only (batch == 0). Needs no workspace (ws may be NULL, ws_bytes 0).
+ * This is the pages' short-context path that writes S with one matrix product
+ * (LSA appendix F.1, "Flat prefill": below 32,768 buckets S is written).
+ * Returns SA_ERR_UNSUPPORTED if n_q * ld exceeds 2^34 entries.
+ */
+sa_status sa_index_scores(const sa_indexer_in* in, float* scores, int64_t ld,
+                          void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * sa_topk: exact top-k of each row of a score table (stage 2).
+ *   Row i considers columns s < min(n_k, q_pos0 + i + 1) and writes to
+ *   idx[i * k ...] the min(k, that count) columns of largest score, ties to
+ *   the lower column, in unspecified order, then -1 padding. Selection is the
+ *   radix select over packed keys of LSA appendix F.1 (score bits above the
+ *   inverted id). NaN scores order above +inf (by sign) and are not expected.
+ * Workspace: none (ws may be NULL).
+ */
+sa_status sa_topk(const float* scores, int32_t n_q, int32_t n_k, int64_t ld, int32_t q_pos0,
+                  int32_t k, int32_t* idx, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * sa_sparse_attn: softmax attention over given index rows (stage 3).
+ *   idx [n_q, k] int32 (decode: [batch, k], positions in that sequence's
+ *   cache); entries < 0 are skipped, entries must be < n_k.
+ *   out [n_q, n_q_heads, head_dim] bf16; lse [n_q, n_q_heads] fp32 (natural
+ *   log, nullable). A row with no valid index gets out = 0, lse = -inf.
+ * Workspace: sa_workspace_size(SA_OP_SPARSE_ATTN, ...) bytes (decode splits).
+ */
+sa_status sa_sparse_attn(const sa_attn_in* in, const int32_t* idx, int32_t k, void* out, float* lse,
+                         void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * sa_prefill: the fused prefill path (indexer -> top-k -> attention).
+ *   idx_out [n_q, k] int32 (nullable: then held in the workspace),
+ *   out [n_q, n_q_heads, head_dim] bf16, lse [n_q, n_q_heads] fp32 (nullable).
+ * FLAT: the token indexer over all visible keys. With a small table it writes
+ *   S and selects rows (LSA appendix F.1, "Flat prefill", short context);
+ *   above that it never writes S: each query keeps a threshold and a
+ *   candidate list filled in the indexer's epilogue, then selects exactly
+ *   (LSA appendix F.1, "Selection by threshold"; HyTopK's on-the-fly exact
+ *   top-k). Rows whose list misses are re-selected from their whole row.
+ * TWO_STAGE: block keys = mean of each block's dequantised keys (stored as
+ *   e4m3 with one scale per block); stage 1 scores complete blocks b <
+ *   floor(p / block_size) and keeps block 0, the current block and the best
+ *   keep_blocks - 2 others; stage 2 scores the visible keys of the kept
+ *   blocks; then top-k and attention.
+ * Requires in->n_k == n_k of attn, q_pos0 + n_q <= n_k.
+ * Host synchronisation: FLAT mode above the table size reads one counter per
+ * chunk back to the host (the miss count, as the pages do in prefill).
+ */
+sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* attn, const sa_prefill_opts* opts,
+                     int32_t* idx_out, void* out, float* lse, void* ws, size_t ws_bytes,
+                     cudaStream_t stream);
+
+/*
+ * sa_decode: one decode step for `batch` sequences (one new query each).
+ *   in->batch == attn->batch > 0. Keys visible to sequence b: s < seq_lens[b].
+ *   idx_out [batch, k] int32 (nullable), out [batch, n_q_heads, head_dim]
+ *   bf16, lse [batch, n_q_heads] (nullable).
+ * No host synchronisation and no allocation: the call can be captured in a
+ * CUDA graph (shapes are fixed by n_k; seq_lens are read on the device).
+ */
+sa_status sa_decode(const sa_indexer_in* in, const sa_attn_in* attn, const sa_decode_opts* opts,
+                    int32_t* idx_out, void* out, float* lse, void* ws, size_t ws_bytes,
+                    cudaStream_t stream);
+
+/*
+ * sa_workspace_size: bytes of device workspace `op` needs for these operands
+ * (host call, no device work). opts points to sa_prefill_opts (PREFILL),
+ * sa_decode_opts (DECODE), an int32_t k (TOPK, SPARSE_ATTN) or NULL.
+ * Workspace must be 256-byte aligned.
+ */
+sa_status sa_workspace_size(sa_op op, const sa_indexer_in* in, const sa_attn_in* attn,
+                            const void* opts, size_t* bytes);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SA_H_ */

@@ -1,0 +1,239 @@
+"""Python binding of libsa (include/sa.h): argument marshalling only.
+
+Every step of the sparse-attention path runs in the CUDA library; this module
+passes torch tensors' device pointers and the current CUDA stream through the
+C ABI and turns status codes into exceptions. There is no fallback: if the
+library is missing, importing the binding fails.
+
+    import indexer_selected_top_b200 as sa
+    idx = sa.topk(scores, k=64)                 # exact top-k of each row
+    out, lse = sa.prefill(inp, k=2048, mode="two_stage")
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libsa.so not built ({LIB_PATH}); run python -m indexer_selected_top_b200.build")
+_lib = ctypes.CDLL(LIB_PATH)
+
+# ----------------------------------------------------------------- constants
+SA_OK, SA_ERR_INVALID_ARGUMENT, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE_TOO_SMALL, SA_ERR_CUDA, SA_ERR_TIMEOUT, \
+    SA_ERR_INTERNAL = range(7)
+SA_BF16, SA_FP8_E4M3, SA_F32 = 0, 1, 2
+SA_MODE_FLAT, SA_MODE_TWO_STAGE = 0, 1
+SA_OP_INDEX_SCORES, SA_OP_TOPK, SA_OP_SPARSE_ATTN, SA_OP_PREFILL, SA_OP_DECODE = range(5)
+SA_HOOK_NONE, SA_HOOK_THETA_POS_INF, SA_HOOK_THETA_NEG_INF, SA_HOOK_STALL_WAIT = range(4)
+
+EXPORTS = ("sa_status_string", "sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode",
+           "sa_workspace_size")
+
+
+class IndexerIn(ctypes.Structure):
+    _fields_ = [("n_q", ctypes.c_int32), ("n_k", ctypes.c_int32), ("q_pos0", ctypes.c_int32),
+                ("n_heads", ctypes.c_int32), ("d_idx", ctypes.c_int32), ("dtype", ctypes.c_int),
+                ("q", ctypes.c_void_p), ("q_scale", ctypes.c_void_p), ("k", ctypes.c_void_p),
+                ("k_scale", ctypes.c_void_p), ("w", ctypes.c_void_p), ("batch", ctypes.c_int32),
+                ("seq_lens", ctypes.c_void_p)]
+
+
+class AttnIn(ctypes.Structure):
+    _fields_ = [("n_q", ctypes.c_int32), ("n_k", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("softmax_scale", ctypes.c_float), ("q", ctypes.c_void_p),
+                ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p), ("batch", ctypes.c_int32)]
+
+
+class PrefillOpts(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_int32), ("mode", ctypes.c_int), ("block_size", ctypes.c_int32),
+                ("keep_blocks", ctypes.c_int32), ("chunk_rows", ctypes.c_int32), ("status", ctypes.c_void_p),
+                ("test_hook", ctypes.c_int32)]
+
+
+class DecodeOpts(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_int32), ("status", ctypes.c_void_p), ("test_hook", ctypes.c_int32)]
+
+
+_P = ctypes.c_void_p
+_lib.sa_status_string.restype = ctypes.c_char_p
+_lib.sa_status_string.argtypes = [ctypes.c_int]
+_lib.sa_index_scores.argtypes = [ctypes.POINTER(IndexerIn), _P, ctypes.c_int64, _P, ctypes.c_size_t, _P]
+_lib.sa_topk.argtypes = [_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P, _P,
+                         ctypes.c_size_t, _P]
+_lib.sa_sparse_attn.argtypes = [ctypes.POINTER(AttnIn), _P, ctypes.c_int32, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.sa_prefill.argtypes = [ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), ctypes.POINTER(PrefillOpts), _P, _P,
+                            _P, _P, ctypes.c_size_t, _P]
+_lib.sa_decode.argtypes = [ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), ctypes.POINTER(DecodeOpts), _P, _P,
+                           _P, _P, ctypes.c_size_t, _P]
+_lib.sa_workspace_size.argtypes = [ctypes.c_int, ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), _P,
+                                   ctypes.POINTER(ctypes.c_size_t)]
+for _f in ("sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode", "sa_workspace_size"):
+    getattr(_lib, _f).restype = ctypes.c_int
+
+
+class SaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {_lib.sa_status_string(code).decode()}")
+
+
+def _check(code: int, where: str):
+    if code != SA_OK:
+        raise SaError(code, where)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def status_string(code: int) -> str:
+    return _lib.sa_status_string(code).decode()
+
+
+# ------------------------------------------------------------- descriptors
+def indexer_in(q, q_scale, k, k_scale, w, q_pos0=0, seq_lens=None) -> IndexerIn:
+    """q [n_q, H, d] (uint8 e4m3 bytes or bf16), k [n_k, d] (decode: q [B, H, d],
+    k [B, L, d] with seq_lens [B] int32 or None)."""
+    decode = k.dim() == 3
+    dt = SA_FP8_E4M3 if q.dtype == torch.uint8 else SA_BF16
+    return IndexerIn(n_q=q.shape[0], n_k=k.shape[-2], q_pos0=q_pos0, n_heads=q.shape[1], d_idx=q.shape[2], dtype=dt,
+                     q=_ptr(q), q_scale=_ptr(q_scale), k=_ptr(k), k_scale=_ptr(k_scale), w=_ptr(w),
+                     batch=k.shape[0] if decode else 0, seq_lens=_ptr(seq_lens))
+
+
+def attn_in(Q, K, V, softmax_scale=0.0) -> AttnIn:
+    """Q [n_q, Hq, dh] bf16, K/V [n_k, dh] (decode: [B, L, dh]) bf16."""
+    decode = K.dim() == 3
+    return AttnIn(n_q=Q.shape[0], n_k=K.shape[-2], n_q_heads=Q.shape[1], head_dim=Q.shape[2],
+                  softmax_scale=softmax_scale, q=_ptr(Q), k_cache=_ptr(K), v_cache=_ptr(V),
+                  batch=K.shape[0] if decode else 0)
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(nbytes, 256) + 256, dtype=torch.uint8, device=device)
+
+
+def _aligned(ws: torch.Tensor) -> int:
+    p = ws.data_ptr()
+    return (p + 255) & ~255
+
+
+def workspace_size(op: int, ind=None, att=None, opts=None) -> int:
+    n = ctypes.c_size_t(0)
+    o = None
+    if isinstance(opts, int):
+        o = ctypes.cast(ctypes.pointer(ctypes.c_int32(opts)), ctypes.c_void_p)
+    elif opts is not None:
+        o = ctypes.cast(ctypes.pointer(opts), ctypes.c_void_p)
+    _check(_lib.sa_workspace_size(op, ctypes.byref(ind) if ind is not None else None,
+                                  ctypes.byref(att) if att is not None else None, o, ctypes.byref(n)),
+           "sa_workspace_size")
+    return n.value
+
+
+# ------------------------------------------------------------------- calls
+def index_scores(q, q_scale, k, k_scale, w, q_pos0=0, out=None, stream=None):
+    """Causal score table [n_q, n_k] fp32 (-inf where invisible)."""
+    ind = indexer_in(q, q_scale, k, k_scale, w, q_pos0)
+    if out is None:
+        out = torch.empty((q.shape[0], k.shape[0]), dtype=torch.float32, device=q.device)
+    _check(_lib.sa_index_scores(ctypes.byref(ind), _ptr(out), out.stride(0), None, 0, _stream(stream)),
+           "sa_index_scores")
+    return out
+
+
+def topk(scores, k: int, q_pos0: int = 0, n_k=None, out=None, stream=None):
+    """Exact top-k of each row over columns s <= q_pos0 + row (unspecified
+    order within a row, -1 padded)."""
+    n_q = scores.shape[0]
+    n_k = scores.shape[1] if n_k is None else n_k
+    if out is None:
+        out = torch.empty((n_q, k), dtype=torch.int32, device=scores.device)
+    _check(_lib.sa_topk(_ptr(scores), n_q, n_k, scores.stride(0), q_pos0, k, _ptr(out), None, 0, _stream(stream)),
+           "sa_topk")
+    return out
+
+
+def sparse_attn(Q, K, V, idx, softmax_scale=0.0, out=None, lse=None, stream=None, want_lse=True):
+    att = attn_in(Q, K, V, softmax_scale)
+    k = idx.shape[1]
+    if out is None:
+        out = torch.empty_like(Q)
+    if lse is None and want_lse:
+        lse = torch.empty(Q.shape[:2], dtype=torch.float32, device=Q.device)
+    nws = workspace_size(SA_OP_SPARSE_ATTN, att=att, opts=k)
+    ws = _workspace(nws, Q.device)
+    _check(_lib.sa_sparse_attn(ctypes.byref(att), _ptr(idx), k, _ptr(out), _ptr(lse), _aligned(ws), nws,
+                               _stream(stream)), "sa_sparse_attn")
+    return out, lse
+
+
+class Prefill:
+    """A prepared sa_prefill call: descriptors and workspace built once, so a
+    timed loop runs only the library call."""
+
+    def __init__(self, q, q_scale, k, k_scale, w, Q, K, V, k_top: int, mode: str = "flat", block_size=64,
+                 keep_blocks=64, chunk_rows=0, q_pos0=0, softmax_scale=0.0, want_idx=True, want_lse=True,
+                 status=None, test_hook=0):
+        self.ind = indexer_in(q, q_scale, k, k_scale, w, q_pos0)
+        self.att = attn_in(Q, K, V, softmax_scale)
+        self.opts = PrefillOpts(k=k_top, mode=SA_MODE_TWO_STAGE if mode == "two_stage" else SA_MODE_FLAT,
+                                block_size=block_size, keep_blocks=keep_blocks, chunk_rows=chunk_rows,
+                                status=_ptr(status), test_hook=test_hook)
+        self.nws = workspace_size(SA_OP_PREFILL, self.ind, self.att, self.opts)
+        self.ws = _workspace(self.nws, Q.device)
+        self.idx = torch.empty((Q.shape[0], k_top), dtype=torch.int32, device=Q.device) if want_idx else None
+        self.out = torch.empty_like(Q)
+        self.lse = torch.empty(Q.shape[:2], dtype=torch.float32, device=Q.device) if want_lse else None
+        self._keep = (q, q_scale, k, k_scale, w, Q, K, V, status)
+
+    def __call__(self, stream=None):
+        _check(_lib.sa_prefill(ctypes.byref(self.ind), ctypes.byref(self.att), ctypes.byref(self.opts),
+                               _ptr(self.idx), _ptr(self.out), _ptr(self.lse), _aligned(self.ws), self.nws,
+                               _stream(stream)), "sa_prefill")
+        return self.out, self.lse, self.idx
+
+
+def prefill(q, q_scale, k, k_scale, w, Q, K, V, k_top: int, mode: str = "flat", **kw):
+    return Prefill(q, q_scale, k, k_scale, w, Q, K, V, k_top, mode, **kw)()
+
+
+class Decode:
+    """A prepared sa_decode call (one decode step of a batch of sequences)."""
+
+    def __init__(self, q, q_scale, k, k_scale, w, Q, K, V, seq_lens, k_top: int, softmax_scale=0.0,
+                 want_idx=True, want_lse=True, status=None, test_hook=0):
+        self.ind = indexer_in(q, q_scale, k, k_scale, w, 0, seq_lens)
+        self.att = attn_in(Q, K, V, softmax_scale)
+        self.opts = DecodeOpts(k=k_top, status=_ptr(status), test_hook=test_hook)
+        self.nws = workspace_size(SA_OP_DECODE, self.ind, self.att, self.opts)
+        self.ws = _workspace(self.nws, Q.device)
+        self.idx = torch.empty((Q.shape[0], k_top), dtype=torch.int32, device=Q.device) if want_idx else None
+        self.out = torch.empty_like(Q)
+        self.lse = torch.empty(Q.shape[:2], dtype=torch.float32, device=Q.device) if want_lse else None
+        self._keep = (q, q_scale, k, k_scale, w, Q, K, V, seq_lens, status)
+
+    def __call__(self, stream=None):
+        _check(_lib.sa_decode(ctypes.byref(self.ind), ctypes.byref(self.att), ctypes.byref(self.opts),
+                              _ptr(self.idx), _ptr(self.out), _ptr(self.lse), _aligned(self.ws), self.nws,
+                              _stream(stream)), "sa_decode")
+        return self.out, self.lse, self.idx
+
+
+def decode(q, q_scale, k, k_scale, w, Q, K, V, seq_lens, k_top: int, **kw):
+    return Decode(q, q_scale, k, k_scale, w, Q, K, V, seq_lens, k_top, **kw)()
+
+
+def new_status(device) -> torch.Tensor:
+    """A zeroed device sa_device_status (4 x uint32, as int32)."""
+    return torch.zeros(4, dtype=torch.int32, device=device)

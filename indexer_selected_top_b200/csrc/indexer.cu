@@ -1,0 +1,414 @@
+// indexer.cu -- the lightweight indexer on tcgen05 tensor cores.
+//
+// score(t, s) = sk[s] * sum_h w'[t,h] * ReLU(acc[s, (t,h)]),  w' = w * sq
+// acc[s, (t,h)] = e4m3(k[s]) . e4m3(q[t,h])  (or bf16), fp32 in TMEM.
+//
+// Token sparse attention's indexer (Latent Sparse Attention section 2.1)
+// scores every visible key of every query. The contraction over d runs on the
+// tensor cores with KEYS on the MMA M dimension (128 TMEM lanes = 128 keys)
+// and (query, head) pairs on N, so each epilogue thread owns one key and the
+// ReLU + head-weighted reduction is a thread-local loop over TMEM columns
+// (no cross-lane reduction). The scales factor out of the ReLU because they
+// are positive: ReLU(sq*sk*a) = sq*sk*ReLU(a).
+//
+// Roles (320 threads): warp 0 = TMA producer (one lane), warp 1 = MMA issuer
+// (one lane) and TMEM owner, warps 2..9 = two epilogue teams of 4 warps, one
+// per TMEM accumulator buffer (2 x 256 fp32 columns), so the epilogue of one
+// accumulator overlaps the MMAs into the other (the pages' bucket scan also
+// overlaps its epilogue with its products: appendix F.1, "Flat prefill").
+//
+// Key sources (template MODE):
+//   IDX_PREFILL  keys [0, lim] of one sequence, NQ consecutive query rows per
+//                CTA in G sub-tiles of QS queries (N = QS*H <= 256)
+//   IDX_DECODE   one query per sequence, a span of that sequence's key tiles
+//   IDX_GATHER   per query, the 64-key blocks it kept (two-stage stage 2);
+//                a tile = two kept blocks, N = H
+// Output: the fp32 score of every (row, key) of the processed tiles, -inf
+// where the key is not visible, into a row-major table.
+#include <cstdio>
+
+#include "ptx.cuh"
+#include "sa_internal.h"
+
+namespace sa {
+
+template <int H, int D, bool FP8, int MODE>
+struct IdxCfg {
+  static constexpr int ESZ = FP8 ? 1 : 2;
+  static constexpr int ROWB = D * ESZ;                       // bytes per index row
+  static constexpr int QS = (MODE == IDX_PREFILL) ? (256 / H) : 1;
+  static constexpr int N = QS * H;                           // MMA N
+  static constexpr int G = (MODE == IDX_PREFILL) ? 2 : 1;    // sub-tiles per CTA
+  static constexpr int NQ = (MODE == IDX_PREFILL) ? QS * G : (MODE == IDX_GATHER ? 4 : 1);
+  static constexpr int QBYTES = NQ * H * ROWB;
+  static constexpr int KBYTES = 128 * ROWB;
+  static constexpr int NS = (MODE == IDX_DECODE) ? 8 : 6;    // key-tile stages
+  static constexpr int KSTEPS = ROWB / 32;                   // 32-byte K slices per MMA
+  static constexpr int SMEM_USED = 1024 + QBYTES + NS * KBYTES + NQ * H * 4 + (2 * NS + 8) * 8 + 16;
+  // at least 120 KB: one CTA per SM, so two CTAs never contend for TMEM
+  static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
+  static_assert(N <= 256 && N % 16 == 0, "MMA N");
+  static_assert(N % 32 == 0, "epilogue loads 32 columns at a time");
+};
+
+__device__ __forceinline__ int vis_limit(int t, const IdxArgs& a) {
+  const int p = a.q_pos0 + t;
+  return (a.div == 1) ? (p - a.off) : (p / a.div - a.off);
+}
+
+// Walks the (query, pair-of-kept-blocks) jobs of a gather CTA in order; every
+// role advances its own copy identically. Queries without kept blocks (a
+// leading -1) are skipped, so a job never names block -1.
+struct GatherCursor {
+  const int* kept;
+  int keep, q0, nq, ql, pair;
+  __device__ void init(const int* k_, int keep_, int q0_, int nq_) {
+    kept = k_;
+    keep = keep_;
+    q0 = q0_;
+    nq = nq_;
+    ql = 0;
+    pair = 0;
+    skip_empty();
+  }
+  __device__ const int* row() const { return kept + (long long)(q0 + ql) * keep; }
+  __device__ void skip_empty() {
+    while (ql < nq && row()[0] < 0) ++ql;
+  }
+  __device__ void next() {
+    ++pair;
+    if (2 * pair >= keep || row()[2 * pair] < 0) {
+      pair = 0;
+      ++ql;
+      skip_empty();
+    }
+  }
+};
+
+template <int H, int D, bool FP8, int MODE>
+__global__ void __launch_bounds__(320, 1)
+    indexer_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                   const IdxArgs a) {
+  using C = IdxCfg<H, D, FP8, MODE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + C::QBYTES;
+  float* sW = reinterpret_cast<float*>(sK + C::NS * C::KBYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sW + C::NQ * H);
+  uint64_t* kfull = bars;
+  uint64_t* kempty = bars + C::NS;
+  uint64_t* qfull = bars + 2 * C::NS;
+  uint64_t* tfull = qfull + 1;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---------------- work unit (identical in every role) ----------------
+  int q0 = 0, nq = 0, seq = 0, tile0 = 0, ntiles = 0, geff = 1, njobs = 0, seq_len = a.n_k;
+  if constexpr (MODE == IDX_PREFILL) {
+    const int unit = gridDim.x - 1 - blockIdx.x;            // heaviest (latest rows) first
+    q0 = unit * C::NQ;
+    nq = min(C::NQ, a.n_q - q0);
+    geff = (nq + C::QS - 1) / C::QS;
+    const int lim = min(vis_limit(q0 + nq - 1, a), a.n_k - 1);
+    ntiles = (lim < 0) ? 0 : (lim / 128 + 1);
+    njobs = ntiles * geff;
+  } else if constexpr (MODE == IDX_DECODE) {
+    seq = blockIdx.y;
+    q0 = seq;
+    nq = 1;
+    seq_len = a.seq_lens ? min(a.seq_lens[seq], a.n_k) : a.n_k;
+    const int total = (seq_len + 127) / 128;
+    tile0 = blockIdx.x * a.tiles_per_cta;
+    ntiles = max(0, min(a.tiles_per_cta, total - tile0));
+    njobs = ntiles;
+  } else {
+    q0 = blockIdx.x * C::NQ;
+    nq = min(C::NQ, a.n_q - q0);
+    for (int ql = 0; ql < nq; ++ql) {
+      int nb = 0;
+      while (nb < a.keep && a.kept[(long long)(q0 + ql) * a.keep + nb] >= 0) ++nb;
+      njobs += (nb + 1) / 2;
+    }
+    ntiles = njobs;
+  }
+
+  // ---------------- setup ----------------
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(&kfull[s], 1);
+      mbar_init(&kempty[s], 1);
+    }
+    mbar_init(qfull, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc<512>(tmem_slot);
+  for (int i = threadIdx.x; i < C::NQ * H; i += blockDim.x) {
+    const int ql = i / H, h = i % H;
+    float v = 0.f;
+    if (ql < nq) {
+      const long long r = (long long)(q0 + ql) * H + h;
+      v = a.w[r] * (a.q_scale ? a.q_scale[r] : 1.f);
+    }
+    sW[i] = v;
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtx wc{abort_flag, a.status, a.budget};
+
+  if (warp == 0) {
+    // ======================= TMA producer =======================
+    if (lane == 0 && njobs > 0) {
+      prefetch_tmap(&qmap);
+      prefetch_tmap(&kmap);
+      if constexpr (MODE == IDX_PREFILL) {
+        mbar_arrive_expect_tx(qfull, geff * C::QS * H * C::ROWB);
+        for (int g = 0; g < geff; ++g)
+          tma_load_2d(sQ + g * C::QS * H * C::ROWB, &qmap, qfull, 0, (q0 + g * C::QS) * H);
+      } else {
+        mbar_arrive_expect_tx(qfull, nq * H * C::ROWB);
+        for (int ql = 0; ql < nq; ++ql) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, (q0 + ql) * H);
+      }
+      GatherCursor gc;
+      if constexpr (MODE == IDX_GATHER) gc.init(a.kept, a.keep, q0, nq);
+      int issued = 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int st = i % C::NS, u = i / C::NS;
+        if (!mbar_wait(&kempty[st], (u & 1) ^ 1, wc, 1)) break;
+        ++issued;
+        uint8_t* dst = sK + st * C::KBYTES;
+        if constexpr (MODE == IDX_PREFILL) {
+          mbar_arrive_expect_tx(&kfull[st], C::KBYTES);
+          tma_load_2d(dst, &kmap, &kfull[st], 0, i * 128);
+        } else if constexpr (MODE == IDX_DECODE) {
+          mbar_arrive_expect_tx(&kfull[st], C::KBYTES);
+          tma_load_2d(dst, &kmap, &kfull[st], 0, seq * a.n_k + (tile0 + i) * 128);
+        } else {
+          const int* kr = gc.row();
+          const int b0 = kr[2 * gc.pair];
+          const int b1 = (2 * gc.pair + 1 < a.keep) ? kr[2 * gc.pair + 1] : -1;
+          mbar_arrive_expect_tx(&kfull[st], (b1 >= 0 ? 2 : 1) * 64 * C::ROWB);
+          tma_load_2d(dst, &kmap, &kfull[st], 0, b0 * 64);
+          if (b1 >= 0) tma_load_2d(dst + 64 * C::ROWB, &kmap, &kfull[st], 0, b1 * 64);
+          gc.next();
+        }
+      }
+      // never leave with copies in flight (matters only after an abort):
+      // wait, bounded and regardless of the abort flag, for the last loads
+      const WaitCtx drain{abort_flag, nullptr, a.budget};
+      for (int i = max(0, issued - C::NS); i < issued; ++i)
+        mbar_wait_drain(&kfull[i % C::NS], (i / C::NS) & 1, drain);
+      mbar_wait_drain(qfull, 0, drain);
+    }
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================
+    if (lane == 0 && njobs > 0) {
+      constexpr uint32_t idesc = umma_idesc<FP8 ? 0 : 1, 128, C::N>();
+      if (mbar_wait(qfull, 0, wc, 2)) {
+        tc_fence_after();
+        GatherCursor gc;
+        if constexpr (MODE == IDX_GATHER) gc.init(a.kept, a.keep, q0, nq);
+        for (int j = 0; j < njobs; ++j) {
+          int tile, g;
+          if constexpr (MODE == IDX_PREFILL) {
+            tile = j / geff;
+            g = j % geff;
+          } else {
+            tile = j;
+            g = (MODE == IDX_GATHER) ? gc.ql : 0;
+          }
+          const int st = tile % C::NS;
+          const int buf = j & 1, ub = j >> 1;
+          if (g == 0 || MODE != IDX_PREFILL) {
+            if (!mbar_wait(&kfull[st], (tile / C::NS) & 1, wc, 3)) break;
+          }
+          if (!mbar_wait(&tempty[buf], (ub & 1) ^ 1, wc, 4)) break;
+          tc_fence_after();
+          if (a.hook == SA_HOOK_STALL_WAIT && j == 0) {            // test hook: never signal job 0
+            if constexpr (MODE == IDX_GATHER) gc.next();
+            continue;
+          }
+          const uint32_t a_base = smem_u32(sK + st * C::KBYTES);
+          const uint32_t b_base = smem_u32(sQ + g * (C::N * C::ROWB));
+          const uint32_t d_tmem = tmem_base + buf * 256;
+#pragma unroll
+          for (int ks = 0; ks < C::KSTEPS; ++ks) {
+            const uint64_t ad = umma_smem_desc<C::ROWB>(a_base + ks * 32);
+            const uint64_t bd = umma_smem_desc<C::ROWB>(b_base + ks * 32);
+            if constexpr (FP8)
+              mma_f8(d_tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
+            else
+              mma_bf16(d_tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
+          }
+          mma_commit(&tfull[buf]);
+          if (MODE != IDX_PREFILL || g == geff - 1) mma_commit(&kempty[st]);
+          if constexpr (MODE == IDX_GATHER) gc.next();
+        }
+      }
+    }
+  } else {
+    // ======================= epilogue teams =======================
+    const int team = (warp - 2) >> 2;
+    const int lq = warp & 3;                 // TMEM lane quarter this warp may access
+    const int row = lq * 32 + lane;          // key row of the tile (TMEM lane)
+    GatherCursor gc;                         // gather: job -> (query, pair)
+    int jq = 0;
+    if constexpr (MODE == IDX_GATHER) gc.init(a.kept, a.keep, q0, nq);
+    for (int j = team; j < njobs; j += 2) {
+      if constexpr (MODE == IDX_GATHER) {
+        while (jq < j) {
+          gc.next();
+          ++jq;
+        }
+      }
+      const int ql = gc.ql, pair = gc.pair;
+      const int buf = j & 1, ub = j >> 1;
+      if (!mbar_wait(&tfull[buf], ub & 1, wc, 5)) break;
+      tc_fence_after();
+      int tile, g;
+      if constexpr (MODE == IDX_PREFILL) {
+        tile = j / geff;
+        g = j % geff;
+      } else {
+        tile = j;
+        g = (MODE == IDX_GATHER) ? ql : 0;
+      }
+      // key of this thread
+      int s;
+      bool kvalid;
+      int col;
+      if constexpr (MODE == IDX_GATHER) {
+        const int slot = 2 * pair + (row >> 6);
+        const int* kr = a.kept + (long long)(q0 + ql) * a.keep;
+        const int blk = (slot < a.keep) ? kr[slot] : -1;
+        s = blk * 64 + (row & 63);
+        kvalid = blk >= 0;
+        col = pair * 128 + row;
+      } else if constexpr (MODE == IDX_DECODE) {
+        s = (tile0 + tile) * 128 + row;
+        kvalid = s < seq_len;
+        col = s;
+      } else {
+        s = tile * 128 + row;
+        kvalid = s < a.n_k;
+        col = s;
+      }
+      float sk = 1.f;
+      if (a.k_scale != nullptr && kvalid) sk = a.k_scale[(long long)seq * a.n_k * (MODE == IDX_DECODE) + s];
+
+      float acc[C::QS];
+#pragma unroll
+      for (int qq = 0; qq < C::QS; ++qq) acc[qq] = 0.f;
+      const uint32_t t_addr = tmem_base + (uint32_t(lq * 32) << 16) + buf * 256;
+      const float* wrow = sW + g * C::N;
+#pragma unroll
+      for (int c = 0; c < C::N / 32; ++c) {
+        float v[32];
+        tmem_ld32(t_addr + c * 32, v);
+        tmem_ld_wait();
+        if (c == C::N / 32 - 1) {
+          // all columns are in registers: hand the accumulator back to the MMA
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
+        }
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 w4 = *reinterpret_cast<const float4*>(wrow + c * 32 + e4 * 4);
+          const int qq = (c * 32 + e4 * 4) / H;
+          acc[qq] = fmaf(w4.x, fmaxf(v[e4 * 4 + 0], 0.f), acc[qq]);
+          acc[qq] = fmaf(w4.y, fmaxf(v[e4 * 4 + 1], 0.f), acc[qq]);
+          acc[qq] = fmaf(w4.z, fmaxf(v[e4 * 4 + 2], 0.f), acc[qq]);
+          acc[qq] = fmaf(w4.w, fmaxf(v[e4 * 4 + 3], 0.f), acc[qq]);
+        }
+      }
+      // outputs
+#pragma unroll
+      for (int qq = 0; qq < C::QS; ++qq) {
+        int t;
+        if constexpr (MODE == IDX_PREFILL)
+          t = q0 + g * C::QS + qq;
+        else if constexpr (MODE == IDX_DECODE)
+          t = seq;
+        else
+          t = q0 + ql;
+        if (t >= a.n_q) continue;
+        bool vis;
+        if constexpr (MODE == IDX_DECODE)
+          vis = kvalid;
+        else
+          vis = kvalid && s <= vis_limit(t, a);
+        const float score = vis ? acc[qq] * sk : -__int_as_float(0x7f800000);
+        if constexpr (MODE == IDX_GATHER) {
+          a.out[(long long)t * a.ld + col] = score;
+        } else {
+          if (col < a.n_k) a.out[(long long)t * a.ld + col] = score;
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc<512>(tmem_base);
+  }
+}
+
+// ----------------------------------------------------------------- host side
+template <int H, int D, bool FP8, int MODE>
+static cudaError_t launch_t(const void* q, const void* k, int q_rows, long long k_rows, const IdxArgs& a,
+                            cudaStream_t st) {
+  using C = IdxCfg<H, D, FP8, MODE>;
+  CUtensorMap qm, km;
+  const CUtensorMapDataType dt = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapSwizzle sw = (C::ROWB == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const uint32_t qbox = (MODE == IDX_PREFILL) ? C::QS * H : H;
+  const uint32_t kbox = (MODE == IDX_GATHER) ? 64 : 128;
+  if (!make_tmap_2d(&qm, q, dt, D, (uint64_t)q_rows * H, C::ROWB, D, qbox, sw)) return cudaErrorInvalidValue;
+  if (!make_tmap_2d(&km, k, dt, D, (uint64_t)k_rows, C::ROWB, D, kbox, sw)) return cudaErrorInvalidValue;
+  auto kern = indexer_kernel<H, D, FP8, MODE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  dim3 grid;
+  if constexpr (MODE == IDX_PREFILL)
+    grid = dim3((a.n_q + C::NQ - 1) / C::NQ);
+  else if constexpr (MODE == IDX_DECODE)
+    grid = dim3(((a.n_k + 127) / 128 + a.tiles_per_cta - 1) / a.tiles_per_cta, a.n_q);
+  else
+    grid = dim3((a.n_q + C::NQ - 1) / C::NQ);
+  if (grid.x == 0 || grid.y == 0) return cudaSuccess;
+  kern<<<grid, 320, C::SMEM, st>>>(qm, km, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_indexer(int mode, int heads, int d, sa_dtype dt, const void* q, const void* k, int q_rows,
+                           long long k_rows, const IdxArgs& a, cudaStream_t st) {
+#define SA_IDX_CASE(H_, D_, F_)                                                                   \
+  if (heads == H_ && d == D_ && (dt == SA_FP8_E4M3) == F_) {                                       \
+    if (mode == IDX_PREFILL) return launch_t<H_, D_, F_, IDX_PREFILL>(q, k, q_rows, k_rows, a, st); \
+    if (mode == IDX_DECODE) return launch_t<H_, D_, F_, IDX_DECODE>(q, k, q_rows, k_rows, a, st);   \
+    if (mode == IDX_GATHER) return launch_t<H_, D_, F_, IDX_GATHER>(q, k, q_rows, k_rows, a, st);   \
+  }
+#define SA_IDX_CASE_PREFILL(H_, D_, F_)                                                            \
+  if (heads == H_ && d == D_ && (dt == SA_FP8_E4M3) == F_ && mode == IDX_PREFILL)                  \
+    return launch_t<H_, D_, F_, IDX_PREFILL>(q, k, q_rows, k_rows, a, st);
+  SA_IDX_CASE(64, 128, true)
+  SA_IDX_CASE(32, 128, true)
+  SA_IDX_CASE_PREFILL(4, 32, false)
+  SA_IDX_CASE_PREFILL(8, 32, false)
+#undef SA_IDX_CASE_PREFILL
+#undef SA_IDX_CASE
+  return cudaErrorNotSupported;
+}
+
+}  // namespace sa

@@ -1,0 +1,415 @@
+// sa_api.cu -- the C ABI (include/sa.h): validation, workspace layout and
+// the launch sequences of the sparse-attention hot path.
+#include <cmath>
+#include <cstring>
+
+#include "sa_internal.h"
+
+namespace sa {
+
+// ------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;   // resolved once; read-only afterwards
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t rows,
+                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr || rows == 0) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------ validation
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static bool idx_supported(const sa_indexer_in* in) {
+  if (in->dtype == SA_FP8_E4M3) return in->d_idx == 128 && (in->n_heads == 64 || in->n_heads == 32);
+  if (in->dtype == SA_BF16) return in->batch == 0 && in->d_idx == 32 && (in->n_heads == 4 || in->n_heads == 8);
+  return false;
+}
+
+static sa_status check_indexer(const sa_indexer_in* in, bool decode) {
+  if (in == nullptr) return SA_ERR_INVALID_ARGUMENT;
+  if (in->n_q < 0 || in->n_k <= 0 || in->n_heads <= 0 || in->d_idx <= 0 || in->q_pos0 < 0)
+    return SA_ERR_INVALID_ARGUMENT;
+  if (decode != (in->batch > 0)) return SA_ERR_INVALID_ARGUMENT;
+  if (decode && in->n_q != in->batch) return SA_ERR_INVALID_ARGUMENT;
+  if (in->n_q > 0 && (in->q == nullptr || in->k == nullptr || in->w == nullptr)) return SA_ERR_INVALID_ARGUMENT;
+  if (in->dtype == SA_FP8_E4M3 && in->n_q > 0 && (in->q_scale == nullptr || in->k_scale == nullptr))
+    return SA_ERR_INVALID_ARGUMENT;
+  if (!aligned16(in->q) || !aligned16(in->k)) return SA_ERR_INVALID_ARGUMENT;
+  if (in->d_idx % 32 != 0 || in->d_idx > 128) return SA_ERR_INVALID_ARGUMENT;
+  if (!idx_supported(in)) return SA_ERR_UNSUPPORTED;
+  return SA_OK;
+}
+
+static sa_status check_attn(const sa_attn_in* at, bool decode) {
+  if (at == nullptr) return SA_ERR_INVALID_ARGUMENT;
+  if (at->n_q < 0 || at->n_k <= 0) return SA_ERR_INVALID_ARGUMENT;
+  if (decode != (at->batch > 0)) return SA_ERR_INVALID_ARGUMENT;
+  if (decode && at->n_q != at->batch) return SA_ERR_INVALID_ARGUMENT;
+  if (at->n_q > 0 && (at->q == nullptr || at->k_cache == nullptr || at->v_cache == nullptr))
+    return SA_ERR_INVALID_ARGUMENT;
+  if (!aligned16(at->q) || !aligned16(at->k_cache) || !aligned16(at->v_cache)) return SA_ERR_INVALID_ARGUMENT;
+  if (!(at->head_dim == 64 || at->head_dim == 128)) return SA_ERR_UNSUPPORTED;
+  if (!(at->n_q_heads == 16 || at->n_q_heads == 8)) return SA_ERR_UNSUPPORTED;
+  if (!(at->softmax_scale >= 0.f) || std::isinf(at->softmax_scale)) return SA_ERR_INVALID_ARGUMENT;
+  return SA_OK;
+}
+
+static float attn_scale(const sa_attn_in* at) {
+  return at->softmax_scale > 0.f ? at->softmax_scale : 1.0f / std::sqrt((float)at->head_dim);
+}
+
+static sa_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SA_OK;
+  if (e == cudaErrorNotSupported) return SA_ERR_UNSUPPORTED;
+  return SA_ERR_CUDA;
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+constexpr long long kWaitBudget = 4000000000ll;     // ~2 s of SM clock
+constexpr long long kHookBudget = 20000000ll;       // ~10 ms: the stall hook
+constexpr int kDecodeSplitKeys = 256;               // keys per decode attention split
+constexpr int kDecodeTilesPerCta = 16;              // 2048 keys per decode indexer CTA
+constexpr int kMaxBlocks = 16384;                   // two-stage: blocks per sequence
+
+static int decode_splits(int k) { return std::max(1, (k + kDecodeSplitKeys - 1) / kDecodeSplitKeys); }
+
+// ------------------------------------------------------------ workspace plans
+struct PrefillPlan {
+  int R;           // rows per chunk
+  int nb;          // two-stage: complete blocks
+  size_t off_table, off_idx, off_blk, off_blks, off_bsc, off_kept, off_cand, total;
+};
+
+static bool plan_prefill(const sa_indexer_in* in, const sa_prefill_opts* o, PrefillPlan* p) {
+  const long long nq = std::max(in->n_q, 1);
+  int R = o->chunk_rows > 0 ? o->chunk_rows : 32768;
+  R = (int)std::min<long long>(R, nq);
+  std::memset(p, 0, sizeof(*p));
+  size_t off = 0;
+  if (o->mode == SA_MODE_FLAT) {
+    // score table of one chunk; shrink the chunk so the table stays <= 4 GiB
+    while (R > 1 && (long long)R * in->n_k * 4ll > (4ll << 30)) R = (R + 1) / 2;
+    p->off_table = off;
+    off += align256((size_t)R * in->n_k * 4);
+  } else {
+    const int nb = in->n_k / o->block_size;
+    p->nb = nb;
+    p->off_blk = off;
+    off += align256((size_t)std::max(nb, 1) * in->d_idx);
+    p->off_blks = off;
+    off += align256((size_t)std::max(nb, 1) * 4);
+    p->off_bsc = off;
+    off += align256((size_t)R * std::max(nb, 1) * 4);
+    p->off_kept = off;
+    off += align256((size_t)R * o->keep_blocks * 4);
+    p->off_cand = off;
+    off += align256((size_t)R * o->keep_blocks * o->block_size * 4);
+  }
+  p->off_idx = off;
+  off += align256((size_t)R * o->k * 4);
+  p->R = R;
+  p->total = off;
+  return true;
+}
+
+struct DecodePlan {
+  size_t off_scores, off_idx, off_po, off_pl, total;
+  int splits;
+};
+
+static void plan_decode(const sa_indexer_in* in, const sa_attn_in* at, int k, DecodePlan* p) {
+  size_t off = 0;
+  p->splits = decode_splits(k);
+  p->off_scores = off;
+  off += align256((size_t)in->batch * in->n_k * 4);
+  p->off_idx = off;
+  off += align256((size_t)in->batch * k * 4);
+  p->off_po = off;
+  off += align256((size_t)in->batch * p->splits * at->n_q_heads * at->head_dim * 4);
+  p->off_pl = off;
+  off += align256((size_t)in->batch * p->splits * at->n_q_heads * 4);
+  p->total = off;
+}
+
+static size_t attn_ws(const sa_attn_in* at, int k) {
+  if (at->batch == 0) return 0;
+  const int sp = decode_splits(k);
+  return align256((size_t)at->batch * sp * at->n_q_heads * at->head_dim * 4) +
+         align256((size_t)at->batch * sp * at->n_q_heads * 4);
+}
+
+static IdxArgs base_args(const sa_indexer_in* in, uint32_t* status, int hook) {
+  IdxArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.n_q = in->n_q;
+  a.n_k = in->n_k;
+  a.q_pos0 = in->q_pos0;
+  a.div = 1;
+  a.off = 0;
+  a.q_scale = in->q_scale;
+  a.k_scale = in->k_scale;
+  a.w = in->w;
+  a.seq_lens = in->seq_lens;
+  a.status = status;
+  a.budget = hook == SA_HOOK_STALL_WAIT ? kHookBudget : kWaitBudget;
+  a.hook = hook;
+  return a;
+}
+
+static size_t esize(sa_dtype d) { return d == SA_FP8_E4M3 ? 1 : 2; }
+
+}  // namespace sa
+
+using namespace sa;
+
+extern "C" {
+
+const char* sa_status_string(sa_status s) {
+  switch (s) {
+    case SA_OK: return "SA_OK";
+    case SA_ERR_INVALID_ARGUMENT: return "SA_ERR_INVALID_ARGUMENT";
+    case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED";
+    case SA_ERR_WORKSPACE_TOO_SMALL: return "SA_ERR_WORKSPACE_TOO_SMALL";
+    case SA_ERR_CUDA: return "SA_ERR_CUDA";
+    case SA_ERR_TIMEOUT: return "SA_ERR_TIMEOUT";
+    case SA_ERR_INTERNAL: return "SA_ERR_INTERNAL";
+  }
+  return "SA_ERR_UNKNOWN";
+}
+
+sa_status sa_workspace_size(sa_op op, const sa_indexer_in* in, const sa_attn_in* at, const void* opts,
+                            size_t* bytes) {
+  if (bytes == nullptr) return SA_ERR_INVALID_ARGUMENT;
+  *bytes = 0;
+  switch (op) {
+    case SA_OP_INDEX_SCORES:
+    case SA_OP_TOPK:
+      return SA_OK;
+    case SA_OP_SPARSE_ATTN: {
+      if (at == nullptr || opts == nullptr) return SA_ERR_INVALID_ARGUMENT;
+      *bytes = attn_ws(at, *static_cast<const int32_t*>(opts));
+      return SA_OK;
+    }
+    case SA_OP_PREFILL: {
+      if (in == nullptr || opts == nullptr) return SA_ERR_INVALID_ARGUMENT;
+      const sa_prefill_opts* o = static_cast<const sa_prefill_opts*>(opts);
+      if (o->k <= 0 || o->block_size <= 0 || o->keep_blocks <= 0) return SA_ERR_INVALID_ARGUMENT;
+      PrefillPlan p;
+      plan_prefill(in, o, &p);
+      *bytes = p.total;
+      return SA_OK;
+    }
+    case SA_OP_DECODE: {
+      if (in == nullptr || at == nullptr || opts == nullptr) return SA_ERR_INVALID_ARGUMENT;
+      const sa_decode_opts* o = static_cast<const sa_decode_opts*>(opts);
+      if (o->k <= 0 || in->batch <= 0) return SA_ERR_INVALID_ARGUMENT;
+      DecodePlan p;
+      plan_decode(in, at, o->k, &p);
+      *bytes = p.total;
+      return SA_OK;
+    }
+  }
+  return SA_ERR_INVALID_ARGUMENT;
+}
+
+sa_status sa_index_scores(const sa_indexer_in* in, float* scores, int64_t ld, void* ws, size_t ws_bytes,
+                          cudaStream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  sa_status s = check_indexer(in, false);
+  if (s != SA_OK) return s;
+  if (scores == nullptr || ld < in->n_k) return SA_ERR_INVALID_ARGUMENT;
+  if (in->n_q == 0) return SA_OK;
+  if ((long long)in->n_q * ld > (1ll << 34)) return SA_ERR_UNSUPPORTED;
+  IdxArgs a = base_args(in, nullptr, 0);
+  a.out = scores;
+  a.ld = ld;
+  cudaError_t e = launch_indexer(IDX_PREFILL, in->n_heads, in->d_idx, in->dtype, in->q, in->k, in->n_q, in->n_k, a,
+                                 stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  return cuda_status(launch_fill_upper(scores, in->n_q, in->n_k, ld, in->q_pos0, stream));
+}
+
+sa_status sa_topk(const float* scores, int32_t n_q, int32_t n_k, int64_t ld, int32_t q_pos0, int32_t k,
+                  int32_t* idx, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (n_q < 0 || n_k <= 0 || ld < n_k || q_pos0 < 0 || k <= 0) return SA_ERR_INVALID_ARGUMENT;
+  if (n_q == 0) return SA_OK;
+  if (scores == nullptr || idx == nullptr) return SA_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_topk_table(scores, n_q, n_k, ld, q_pos0, k, idx, 0, nullptr, 0, nullptr, stream));
+}
+
+sa_status sa_sparse_attn(const sa_attn_in* at, const int32_t* idx, int32_t k, void* out, float* lse, void* ws,
+                         size_t ws_bytes, cudaStream_t stream) {
+  sa_status s = check_attn(at, at != nullptr && at->batch > 0);
+  if (s != SA_OK) return s;
+  if (k <= 0 || (at->n_q > 0 && (idx == nullptr || out == nullptr))) return SA_ERR_INVALID_ARGUMENT;
+  if (at->n_q == 0) return SA_OK;
+  const size_t need = attn_ws(at, k);
+  if (ws_bytes < need || (need > 0 && ws == nullptr)) return SA_ERR_WORKSPACE_TOO_SMALL;
+  int splits = 1;
+  float *po = nullptr, *pl = nullptr;
+  if (at->batch > 0) {
+    splits = decode_splits(k);
+    po = static_cast<float*>(ws);
+    pl = reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                  align256((size_t)at->batch * splits * at->n_q_heads * at->head_dim * 4));
+  }
+  return cuda_status(launch_attention(at->q, at->k_cache, at->v_cache, idx, at->n_q, k, at->n_k, at->n_q_heads,
+                                      at->head_dim, attn_scale(at), at->batch, out, lse, po, pl, splits, stream));
+}
+
+sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_prefill_opts* o, int32_t* idx_out,
+                     void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  sa_status s = check_indexer(in, false);
+  if (s != SA_OK) return s;
+  s = check_attn(at, false);
+  if (s != SA_OK) return s;
+  if (o == nullptr || o->k <= 0 || o->k > 4096) return SA_ERR_INVALID_ARGUMENT;
+  if (at->n_q != in->n_q || at->n_k != in->n_k || in->q_pos0 + (long long)in->n_q > in->n_k)
+    return SA_ERR_INVALID_ARGUMENT;
+  if (in->n_q > 0 && out == nullptr) return SA_ERR_INVALID_ARGUMENT;
+  if (o->mode != SA_MODE_FLAT && o->mode != SA_MODE_TWO_STAGE) return SA_ERR_INVALID_ARGUMENT;
+  if (o->mode == SA_MODE_TWO_STAGE) {
+    if (o->block_size != 64) return SA_ERR_UNSUPPORTED;
+    if (o->keep_blocks < 2 || o->keep_blocks > 64) return SA_ERR_INVALID_ARGUMENT;
+    if (in->dtype != SA_FP8_E4M3) return SA_ERR_UNSUPPORTED;
+    if ((in->q_pos0 + in->n_q - 1) / o->block_size >= kMaxBlocks) return SA_ERR_UNSUPPORTED;
+  }
+  if (in->n_q == 0) return SA_OK;
+  PrefillPlan p;
+  plan_prefill(in, o, &p);
+  if (ws == nullptr || ws_bytes < p.total) return SA_ERR_WORKSPACE_TOO_SMALL;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return SA_ERR_INVALID_ARGUMENT;
+  char* w = static_cast<char*>(ws);
+  uint32_t* status = o->status ? reinterpret_cast<uint32_t*>(o->status) : nullptr;
+  if (status && cudaMemsetAsync(status, 0, sizeof(sa_device_status), stream) != cudaSuccess) return SA_ERR_CUDA;
+  const float scale = attn_scale(at);
+  const size_t qrow = (size_t)in->n_heads * in->d_idx * esize(in->dtype);
+  cudaError_t e = cudaSuccess;
+
+  if (o->mode == SA_MODE_TWO_STAGE) {
+    uint8_t* blk = reinterpret_cast<uint8_t*>(w + p.off_blk);
+    float* blks = reinterpret_cast<float*>(w + p.off_blks);
+    e = launch_pool_blocks(static_cast<const uint8_t*>(in->k), in->k_scale, p.nb, o->block_size, blk, blks, stream);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+
+  for (int r0 = 0; r0 < in->n_q; r0 += p.R) {
+    const int R = std::min(p.R, in->n_q - r0);
+    sa_indexer_in ci = *in;
+    ci.n_q = R;
+    ci.q_pos0 = in->q_pos0 + r0;
+    ci.q = static_cast<const char*>(in->q) + (size_t)r0 * qrow;
+    ci.q_scale = in->q_scale ? in->q_scale + (size_t)r0 * in->n_heads : nullptr;
+    ci.w = in->w + (size_t)r0 * in->n_heads;
+    int32_t* idx = idx_out ? idx_out + (size_t)r0 * o->k : reinterpret_cast<int32_t*>(w + p.off_idx);
+    if (o->mode == SA_MODE_FLAT) {
+      float* table = reinterpret_cast<float*>(w + p.off_table);
+      IdxArgs a = base_args(&ci, status, o->test_hook);
+      a.out = table;
+      a.ld = in->n_k;
+      e = launch_indexer(IDX_PREFILL, in->n_heads, in->d_idx, in->dtype, ci.q, in->k, R, in->n_k, a, stream);
+      if (e != cudaSuccess) return cuda_status(e);
+      e = launch_topk_table(table, R, in->n_k, in->n_k, ci.q_pos0, o->k, idx, 0, nullptr, 0, nullptr, stream);
+      if (e != cudaSuccess) return cuda_status(e);
+    } else {
+      const uint8_t* blk = reinterpret_cast<const uint8_t*>(w + p.off_blk);
+      const float* blks = reinterpret_cast<const float*>(w + p.off_blks);
+      float* bsc = reinterpret_cast<float*>(w + p.off_bsc);
+      int* kept = reinterpret_cast<int*>(w + p.off_kept);
+      float* cand = reinterpret_cast<float*>(w + p.off_cand);
+      const int ncand = o->keep_blocks * o->block_size;
+      // stage 1: complete blocks b < floor(p / block) (the current block is forced)
+      if (p.nb > 0) {
+        sa_indexer_in bi = ci;
+        bi.n_k = p.nb;
+        bi.k = blk;
+        bi.k_scale = blks;
+        IdxArgs a = base_args(&bi, status, o->test_hook);
+        a.div = o->block_size;
+        a.off = 1;
+        a.out = bsc;
+        a.ld = p.nb;
+        e = launch_indexer(IDX_PREFILL, in->n_heads, in->d_idx, in->dtype, ci.q, blk, R, p.nb, a, stream);
+        if (e != cudaSuccess) return cuda_status(e);
+      }
+      e = launch_block_select(bsc, R, p.nb, std::max(p.nb, 1), ci.q_pos0, o->block_size, o->keep_blocks, kept,
+                              stream);
+      if (e != cudaSuccess) return cuda_status(e);
+      // stage 2: the visible keys of the kept blocks
+      IdxArgs a = base_args(&ci, status, o->test_hook);
+      a.out = cand;
+      a.ld = ncand;
+      a.kept = kept;
+      a.keep = o->keep_blocks;
+      e = launch_indexer(IDX_GATHER, in->n_heads, in->d_idx, in->dtype, ci.q, in->k, R, in->n_k, a, stream);
+      if (e != cudaSuccess) return cuda_status(e);
+      e = launch_topk_table(cand, R, ncand, ncand, ci.q_pos0, o->k, idx, 2, kept, o->keep_blocks, nullptr, stream);
+      if (e != cudaSuccess) return cuda_status(e);
+    }
+    const void* qa = static_cast<const char*>(at->q) + (size_t)r0 * at->n_q_heads * at->head_dim * 2;
+    void* oa = static_cast<char*>(out) + (size_t)r0 * at->n_q_heads * at->head_dim * 2;
+    float* la = lse ? lse + (size_t)r0 * at->n_q_heads : nullptr;
+    e = launch_attention(qa, at->k_cache, at->v_cache, idx, R, o->k, at->n_k, at->n_q_heads, at->head_dim, scale, 0,
+                         oa, la, nullptr, nullptr, 1, stream);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  return SA_OK;
+}
+
+sa_status sa_decode(const sa_indexer_in* in, const sa_attn_in* at, const sa_decode_opts* o, int32_t* idx_out,
+                    void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  sa_status s = check_indexer(in, true);
+  if (s != SA_OK) return s;
+  s = check_attn(at, true);
+  if (s != SA_OK) return s;
+  if (o == nullptr || o->k <= 0 || o->k > 4096) return SA_ERR_INVALID_ARGUMENT;
+  if (at->batch != in->batch || at->n_k != in->n_k || out == nullptr) return SA_ERR_INVALID_ARGUMENT;
+  DecodePlan p;
+  plan_decode(in, at, o->k, &p);
+  if (ws == nullptr || ws_bytes < p.total) return SA_ERR_WORKSPACE_TOO_SMALL;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return SA_ERR_INVALID_ARGUMENT;
+  char* w = static_cast<char*>(ws);
+  uint32_t* status = o->status ? reinterpret_cast<uint32_t*>(o->status) : nullptr;
+  if (status && cudaMemsetAsync(status, 0, sizeof(sa_device_status), stream) != cudaSuccess) return SA_ERR_CUDA;
+  float* rows = reinterpret_cast<float*>(w + p.off_scores);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + p.off_idx);
+  IdxArgs a = base_args(in, status, o->test_hook);
+  a.out = rows;
+  a.ld = in->n_k;
+  a.tiles_per_cta = kDecodeTilesPerCta;
+  cudaError_t e = launch_indexer(IDX_DECODE, in->n_heads, in->d_idx, in->dtype, in->q, in->k, in->batch,
+                                 (long long)in->batch * in->n_k, a, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  e = launch_topk_table(rows, in->batch, in->n_k, in->n_k, 0, o->k, idx, 1, nullptr, 0, in->seq_lens, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  e = launch_attention(at->q, at->k_cache, at->v_cache, idx, in->batch, o->k, at->n_k, at->n_q_heads, at->head_dim,
+                       attn_scale(at), in->batch, out, lse, reinterpret_cast<float*>(w + p.off_po),
+                       reinterpret_cast<float*>(w + p.off_pl), p.splits, stream);
+  return cuda_status(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,57 @@
+// sa_internal.h -- declarations shared by the library's translation units.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/sa.h"
+
+namespace sa {
+
+enum IdxMode { IDX_PREFILL = 0, IDX_DECODE = 1, IDX_GATHER = 2 };
+
+// Arguments of the indexer kernel (plain device pointers and sizes).
+struct IdxArgs {
+  int n_q;               // query rows (prefill / gather) or sequences (decode)
+  int n_k;               // keys per sequence (table width for prefill)
+  int q_pos0;            // absolute position of query row 0
+  int div, off;          // key s visible to row t iff s <= (q_pos0 + t) / div - off
+  const float* q_scale;  // [n_q, H] or null (bf16)
+  const float* k_scale;  // [n_k] / [batch, n_k] or null
+  const float* w;        // [n_q, H]
+  float* out;            // score table (row stride ld)
+  long long ld;
+  const int* seq_lens;   // decode: [batch] or null (= n_k)
+  int tiles_per_cta;     // decode: key tiles per CTA
+  const int* kept;       // gather: [n_q, keep] kept block ids, ascending, -1 padded
+  int keep;
+  uint32_t* status;      // device [error, site] or null
+  long long budget;      // wait budget in clock cycles
+  int hook;
+};
+
+// Host launchers (return cudaError_t of the launch).
+cudaError_t launch_indexer(int mode, int heads, int d, sa_dtype dt, const void* q, const void* k, int q_rows,
+                           long long k_rows, const IdxArgs& a, cudaStream_t st);
+
+cudaError_t launch_topk_table(const float* scores, int n_rows, int n_cols, long long ld, int q_pos0, int k,
+                              int32_t* idx, int vis_mode, const int* kept, int keep, const int* seq_lens,
+                              cudaStream_t st);
+
+cudaError_t launch_block_select(const float* bscores, int n_q, int nb, long long ld, int q_pos0, int block,
+                                int keep, int* kept, cudaStream_t st);
+
+cudaError_t launch_pool_blocks(const uint8_t* k, const float* k_scale, int n_blocks, int block,
+                               uint8_t* blk, float* blk_scale, cudaStream_t st);
+
+cudaError_t launch_attention(const void* q, const void* kc, const void* vc, const int32_t* idx, int n_q, int k,
+                             int n_k, int hq, int dh, float scale, int batch, void* out, float* lse,
+                             float* part_o, float* part_lse, int splits, cudaStream_t st);
+
+cudaError_t launch_fill_upper(float* scores, int n_q, int n_k, long long ld, int q_pos0, cudaStream_t st);
+
+// Encodes a 2-D TMA descriptor (rows x inner elements, row-major).
+bool make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t rows,
+                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw);
+
+}  // namespace sa

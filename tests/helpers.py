@@ -1,0 +1,70 @@
+"""Comparison rules shared by the parity tests (CUDA path vs oracle).
+
+Top-k ("tie band"): theta = the oracle's k-th score of the row, M = the row
+max, band = 1e-4 * M. The GPU set passes iff every key scoring > theta + band
+is in it, no key scoring < theta - band is, it has min(k, visible) distinct
+visible keys, and -1 appears only after them. Sets are compared, not orders
+(the order of an index row is unspecified).
+
+Scores: normwise per row, max_s |g - o| <= tol * max_s |o| over visible keys,
+with the contract tolerance (2e-2 FP8, 2e-3 bf16) and an internal gate of
+1e-5 (fp32 accumulation only; it has to stay well inside the 1e-4 band).
+
+Attention: max |g - o| <= 1e-2 against fp64 over the same indices (the
+contract) and the internal gate max |g - o| <= 1e-2 * max |o| + 1e-6.
+"""
+import numpy as np
+
+BAND = 1e-4
+SCORE_GATE = 1e-5
+
+
+def check_topk_row(gpu_row, cand, scores, k, where=""):
+    """gpu_row: int array [k] (-1 padded); cand: candidate key ids; scores:
+    their fp32 oracle scores (same order)."""
+    g = np.asarray(gpu_row, dtype=np.int64)
+    n_vis = len(cand)
+    want = min(k, n_vis)
+    valid = g[g >= 0]
+    assert len(valid) == want, f"{where}: {len(valid)} valid entries, want {want}"
+    assert (g[:want] >= 0).all() and (g[want:] == -1).all(), f"{where}: -1 not at the tail"
+    assert len(set(valid.tolist())) == want, f"{where}: duplicate indices"
+    pos = {int(c): i for i, c in enumerate(cand)}
+    missing = [int(x) for x in valid if int(x) not in pos]
+    assert not missing, f"{where}: invisible keys {missing[:5]}"
+    if want == n_vis:
+        return
+    s = np.asarray(scores, dtype=np.float64)
+    order = np.lexsort((np.arange(n_vis), -s))
+    theta = s[order[want - 1]]
+    band = BAND * max(np.abs(s).max(), 1e-30)
+    sel = np.zeros(n_vis, dtype=bool)
+    sel[[pos[int(x)] for x in valid]] = True
+    must = s > theta + band
+    never = s < theta - band
+    assert not (must & ~sel).any(), f"{where}: {int((must & ~sel).sum())} keys above the band missing"
+    assert not (never & sel).any(), f"{where}: {int((never & sel).sum())} keys below the band selected"
+
+
+def check_scores_row(gpu, ref, tol, where=""):
+    g = np.asarray(gpu, dtype=np.float64)
+    o = np.asarray(ref, dtype=np.float64)
+    m = np.abs(o).max() if o.size else 0.0
+    err = np.abs(g - o).max() if o.size else 0.0
+    assert err <= tol * max(m, 1e-30), f"{where}: normwise err {err / max(m, 1e-30):.3e} > {tol}"
+    return err / max(m, 1e-30)
+
+
+def check_attention_row(o_gpu, o_ref, lse_gpu=None, lse_ref=None, where=""):
+    g = np.asarray(o_gpu, dtype=np.float64)
+    r = np.asarray(o_ref, dtype=np.float64)
+    err = np.abs(g - r).max()
+    assert err <= 1e-2, f"{where}: max-abs err {err}"
+    assert err <= 1e-2 * np.abs(r).max() + 1e-6, f"{where}: err {err} vs max|o| {np.abs(r).max()}"
+    if lse_gpu is not None:
+        lg, lr = np.asarray(lse_gpu, dtype=np.float64), np.asarray(lse_ref, dtype=np.float64)
+        fin = np.isfinite(lr)
+        assert np.array_equal(np.isfinite(lg), fin), f"{where}: lse finiteness"
+        if fin.any():
+            assert np.abs(lg[fin] - lr[fin]).max() <= 1e-4, f"{where}: lse err {np.abs(lg[fin] - lr[fin]).max()}"
+    return err

@@ -1,0 +1,93 @@
+"""The C ABI without a GPU: the library loads, exports every symbol that
+include/sa.h declares, and validates arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def sa():
+    from indexer_selected_top_b200.build import build
+    build()
+    import indexer_selected_top_b200 as m
+    return m
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "sa.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:sa_status|const char\*)\s+(sa_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode", "sa_workspace_size",
+              "sa_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(sa):
+    lib = ctypes.CDLL(sa.LIB_PATH)
+    for n in _declared():
+        assert hasattr(lib, n), n
+    assert set(_declared()) <= set(sa.EXPORTS) | {"sa_status_string"}
+
+
+def test_status_strings(sa):
+    assert sa.status_string(0) == "SA_OK"
+    assert sa.status_string(3) == "SA_ERR_WORKSPACE_TOO_SMALL"
+    assert sa.status_string(99) == "SA_ERR_UNKNOWN"
+
+
+def test_host_validation_rejects_before_launch(sa):
+    lib = sa._lib
+    # sa_topk: bad sizes
+    assert lib.sa_topk(None, 4, 0, 0, 0, 8, None, None, 0, None) == sa.SA_ERR_INVALID_ARGUMENT
+    assert lib.sa_topk(None, 4, 10, 5, 0, 8, None, None, 0, None) == sa.SA_ERR_INVALID_ARGUMENT
+    assert lib.sa_topk(None, 4, 10, 10, 0, 8, None, None, 0, None) == sa.SA_ERR_INVALID_ARGUMENT  # null ptrs
+    assert lib.sa_topk(None, 0, 10, 10, 0, 8, None, None, 0, None) == sa.SA_OK                   # empty
+    # indexer: unsupported head count / dtype, misaligned pointer
+    ind = sa.IndexerIn(n_q=4, n_k=16, q_pos0=0, n_heads=7, d_idx=128, dtype=sa.SA_FP8_E4M3, q=256, q_scale=512,
+                       k=1024, k_scale=2048, w=4096, batch=0, seq_lens=None)
+    assert lib.sa_index_scores(ctypes.byref(ind), 8192, 16, None, 0, None) == sa.SA_ERR_UNSUPPORTED
+    ind.n_heads = 64
+    ind.q = 257
+    assert lib.sa_index_scores(ctypes.byref(ind), 8192, 16, None, 0, None) == sa.SA_ERR_INVALID_ARGUMENT
+    ind.q = 256
+    assert lib.sa_index_scores(ctypes.byref(ind), 8192, 8, None, 0, None) == sa.SA_ERR_INVALID_ARGUMENT  # ld < n_k
+    ind.q_scale = None
+    assert lib.sa_index_scores(ctypes.byref(ind), 8192, 16, None, 0, None) == sa.SA_ERR_INVALID_ARGUMENT
+    # attention: unsupported head_dim
+    att = sa.AttnIn(n_q=4, n_k=16, n_q_heads=16, head_dim=96, softmax_scale=0.0, q=256, k_cache=512, v_cache=768,
+                    batch=0)
+    assert lib.sa_sparse_attn(ctypes.byref(att), 1024, 8, 2048, None, None, 0, None) == sa.SA_ERR_UNSUPPORTED
+
+
+def test_workspace_sizes_and_too_small(sa):
+    ind = sa.IndexerIn(n_q=65536, n_k=65536, q_pos0=0, n_heads=64, d_idx=128, dtype=sa.SA_FP8_E4M3, q=256,
+                       q_scale=512, k=1024, k_scale=2048, w=4096, batch=0, seq_lens=None)
+    att = sa.AttnIn(n_q=65536, n_k=65536, n_q_heads=16, head_dim=128, softmax_scale=0.0, q=256, k_cache=512,
+                    v_cache=768, batch=0)
+    two = sa.PrefillOpts(k=2048, mode=sa.SA_MODE_TWO_STAGE, block_size=64, keep_blocks=64, chunk_rows=0,
+                         status=None, test_hook=0)
+    n_two = sa.workspace_size(sa.SA_OP_PREFILL, ind, att, two)
+    # per 32768-row chunk: block scores + kept + candidate scores + index rows, plus pooled keys
+    assert n_two >= 32768 * (1024 * 4 + 64 * 4 + 4096 * 4 + 2048 * 4)
+    flat = sa.PrefillOpts(k=2048, mode=sa.SA_MODE_FLAT, block_size=64, keep_blocks=64, chunk_rows=0, status=None,
+                          test_hook=0)
+    n_flat = sa.workspace_size(sa.SA_OP_PREFILL, ind, att, flat)
+    assert n_flat >= 16384 * 65536 * 4 and n_flat <= (4 << 30) + 32768 * 2048 * 4 + 4096
+    r = sa._lib.sa_prefill(ctypes.byref(ind), ctypes.byref(att), ctypes.byref(two), None, 4096, None, 256, 1024,
+                           None)
+    assert r == sa.SA_ERR_WORKSPACE_TOO_SMALL
+    dind = sa.IndexerIn(n_q=64, n_k=131072, q_pos0=0, n_heads=64, d_idx=128, dtype=sa.SA_FP8_E4M3, q=256,
+                        q_scale=512, k=1024, k_scale=2048, w=4096, batch=64, seq_lens=None)
+    datt = sa.AttnIn(n_q=64, n_k=131072, n_q_heads=16, head_dim=128, softmax_scale=0.0, q=256, k_cache=512,
+                     v_cache=768, batch=64)
+    dopts = sa.DecodeOpts(k=2048, status=None, test_hook=0)
+    assert sa.workspace_size(sa.SA_OP_DECODE, dind, datt, dopts) >= 64 * 131072 * 4
+    assert sa.workspace_size(sa.SA_OP_SPARSE_ATTN, att=datt, opts=2048) > 0
+    assert sa.workspace_size(sa.SA_OP_SPARSE_ATTN, att=att, opts=2048) == 0

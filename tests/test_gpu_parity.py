@@ -1,0 +1,306 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle on the
+same seeded inputs. Needs a B200."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle.topk import topk_row
+from oracle.pipeline import attention_rows, decode_attention_row
+from workloads import WORKLOADS, PrefillInputs, DecodeInputs, sample_rows
+from helpers import check_topk_row, check_scores_row, check_attention_row, SCORE_GATE
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from indexer_selected_top_b200.build import build
+    build()
+    import indexer_selected_top_b200 as m
+    return m
+
+
+def _gpu(t):
+    return None if t is None else t.cuda()
+
+
+# ------------------------------------------------------------------ indexer
+def _check_table(sa, wl, seed, rows=None, q_pos0=0, n_q=None, tol=2e-2):
+    inp = PrefillInputs(wl, "cuda", seed=seed)
+    host = inp.to_host()
+    T = wl.T
+    n_q = T - q_pos0 if n_q is None else n_q
+    q = inp.q_idx[q_pos0:q_pos0 + n_q]
+    qs = None if inp.q_scale is None else inp.q_scale[q_pos0:q_pos0 + n_q]
+    w = inp.w[q_pos0:q_pos0 + n_q]
+    table = sa.index_scores(q, qs, inp.k_idx, inp.k_scale, w, q_pos0=q_pos0)
+    torch.cuda.synchronize()
+    tab = table.cpu().numpy()
+    rows = range(n_q) if rows is None else rows
+    ref = oracle.scores_rows(host, [q_pos0 + r for r in rows])
+    worst = 0.0
+    for r in rows:
+        p = q_pos0 + r
+        o = ref[p]
+        g = tab[r, :p + 1]
+        worst = max(worst, check_scores_row(g, o, tol, f"row {p}"))
+        check_scores_row(g, o, SCORE_GATE, f"row {p} (gate)")
+        assert np.isneginf(tab[r, p + 1:]).all(), f"row {p}: invisible entries not -inf"
+    return tab, ref, worst
+
+
+def test_index_scores_bf16_tiny(sa):
+    _check_table(sa, WORKLOADS["tiny_t512"], seed=0, tol=2e-3)
+
+
+def test_index_scores_fp8_ragged(sa):
+    wl = WORKLOADS["prefill_t16k"].with_(T=1000)
+    _check_table(sa, wl, seed=1, tol=2e-2)
+
+
+def test_index_scores_fp8_offset_rows(sa):
+    wl = WORKLOADS["prefill_t16k"].with_(T=1000)
+    _check_table(sa, wl, seed=2, q_pos0=700, n_q=300, tol=2e-2)
+
+
+# -------------------------------------------------------------------- top-k
+def _topk_exact(sa, table, k, q_pos0=0):
+    t = torch.from_numpy(table).cuda()
+    idx = sa.topk(t, k, q_pos0=q_pos0).cpu().numpy()
+    for r in range(table.shape[0]):
+        n = min(table.shape[1], q_pos0 + r + 1)
+        want = topk_row(table[r, :n], k)
+        got = idx[r][idx[r] >= 0]
+        assert sorted(got.tolist()) == sorted(want.tolist()), f"row {r}"
+        assert (idx[r][len(got):] == -1).all()
+
+
+def test_topk_exact_with_ties(sa):
+    rng = np.random.default_rng(0)
+    tab = rng.integers(0, 50, size=(37, 1000)).astype(np.float32)
+    _topk_exact(sa, tab, 100)
+    _topk_exact(sa, tab, 1)
+    _topk_exact(sa, tab, 999, q_pos0=500)
+
+
+def test_topk_large_rows_bucket_paths(sa):
+    rng = np.random.default_rng(1)
+    n = 131072
+    rows = [
+        rng.standard_normal(n).astype(np.float32),                     # distinct values
+        rng.integers(0, 4, size=n).astype(np.float32),                 # huge ties at the cut
+        np.full(n, 7.0, dtype=np.float32),                             # all equal
+        np.where(rng.random(n) < 0.5, 0.0, -0.0).astype(np.float32),   # +0 / -0 equal
+        (rng.standard_normal(n) * 1e-3 + 5).astype(np.float32),        # narrow band
+    ]
+    tab = np.stack(rows)
+    _topk_exact(sa, tab, 2048, q_pos0=n)
+    _topk_exact(sa, tab, 20000, q_pos0=n)
+
+
+# ---------------------------------------------------------------- attention
+def _attn_case(sa, n_q, n_k, hq, dh, k, seed, std=None, decode=False):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    std = std or 1.0 / np.sqrt(dh)
+    if decode:
+        K = (torch.randn(n_q, n_k, dh, generator=g, device="cuda") * std).bfloat16()
+        V = (torch.randn(n_q, n_k, dh, generator=g, device="cuda") * std).bfloat16()
+    else:
+        K = (torch.randn(n_k, dh, generator=g, device="cuda") * std).bfloat16()
+        V = (torch.randn(n_k, dh, generator=g, device="cuda") * std).bfloat16()
+    Q = (torch.randn(n_q, hq, dh, generator=g, device="cuda") * std).bfloat16()
+    rng = np.random.default_rng(seed)
+    idx = np.full((n_q, k), -1, dtype=np.int32)
+    for t in range(n_q):
+        m = int(rng.integers(0, k + 1)) if t % 3 == 0 else k
+        m = min(m, n_k)
+        idx[t, :m] = rng.choice(n_k, size=m, replace=False)
+        rng.shuffle(idx[t])          # -1 anywhere: the kernel must skip them
+    out, lse = sa.sparse_attn(Q, K, V, torch.from_numpy(idx).cuda())
+    torch.cuda.synchronize()
+    out, lse = out.float().cpu().numpy(), lse.cpu().numpy()
+    Qh = Q.double().cpu().numpy()
+    Kh, Vh = K.double().cpu().numpy(), V.double().cpu().numpy()
+    for t in range(n_q):
+        if decode:
+            o, l = oracle.sparse_attention_row(Qh[t], Kh[t], Vh[t], idx[t])
+        else:
+            o, l = oracle.sparse_attention_row(Qh[t], Kh, Vh, idx[t])
+        check_attention_row(out[t], o, lse[t], l, f"row {t}")
+
+
+def test_sparse_attn_prefill_shapes(sa):
+    _attn_case(sa, 40, 3000, 16, 128, 2048, seed=0)
+    _attn_case(sa, 40, 500, 8, 64, 64, seed=1)
+    _attn_case(sa, 9, 100, 16, 64, 37, seed=2)
+
+
+def test_sparse_attn_sharp_softmax(sa):
+    # unscaled N(0,1) Q/K: logits of order 10, exercises the running-max rescale
+    _attn_case(sa, 24, 4000, 16, 128, 2048, seed=3, std=1.0)
+
+
+def test_sparse_attn_decode_splits(sa):
+    _attn_case(sa, 5, 3000, 16, 128, 2048, seed=4, decode=True)
+    _attn_case(sa, 3, 700, 16, 128, 600, seed=5, decode=True, std=1.0)
+
+
+# ------------------------------------------------------------------ prefill
+def _check_prefill(sa, wl, seed, rows, mode="flat", k=None, keep=64, chunk_rows=0):
+    k = k or wl.k
+    inp = PrefillInputs(wl, "cuda", seed=seed)
+    host = inp.to_host()
+    pre = sa.Prefill(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, k, mode=mode,
+                     keep_blocks=keep, chunk_rows=chunk_rows)
+    out, lse, idx = pre()
+    torch.cuda.synchronize()
+    out, lse, idx = out.float().cpu().numpy(), lse.cpu().numpy(), idx.cpu().numpy()
+    ref = oracle.prefill_rows(host, rows, k, mode=mode, keep=keep, attention=False)
+    for t in rows:
+        r = ref[t]
+        check_topk_row(idx[t], r["cand"], r["scores"], k, f"row {t}")
+    att = attention_rows(host, {t: idx[t] for t in rows})
+    for t in rows:
+        check_attention_row(out[t], att[t][0], lse[t], att[t][1], f"row {t}")
+    return inp, host, idx, ref
+
+
+def test_prefill_flat_tiny_all_rows(sa):
+    wl = WORKLOADS["tiny_t512"]
+    _check_prefill(sa, wl, 0, range(wl.T))
+
+
+def test_prefill_flat_fp8_ragged(sa):
+    wl = WORKLOADS["prefill_t16k"].with_(T=2500)
+    rows = sample_rows(wl.T, 120, seed=1, k=256)
+    _check_prefill(sa, wl, 1, rows, k=256)
+
+
+def test_prefill_flat_fp8_chunked(sa):
+    wl = WORKLOADS["prefill_t16k"].with_(T=1300)
+    rows = sample_rows(wl.T, 60, seed=2, k=300, extra=(499, 500, 501, 999, 1000))
+    _check_prefill(sa, wl, 2, rows, k=300, chunk_rows=500)
+
+
+def _two_stage_kept_sets(sa, inp, k_all):
+    """Kept blocks of every row, read through the public API: with k = keep *
+    64 every visible key of the kept blocks is selected."""
+    pre = sa.Prefill(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, k_all,
+                     mode="two_stage", keep_blocks=k_all // 64)
+    _, _, idx = pre()
+    torch.cuda.synchronize()
+    idx = idx.cpu().numpy()
+    return [np.unique(r[r >= 0] // 64) for r in idx]
+
+
+def _check_two_stage(sa, wl, seed, rows, k, keep=64):
+    inp = PrefillInputs(wl, "cuda", seed=seed)
+    host = inp.to_host()
+    kept_gpu = _two_stage_kept_sets(sa, inp, keep * 64)
+    ref = oracle.prefill_rows(host, rows, k, mode="two_stage", keep=keep, attention=False)
+    n_diff = 0
+    for t in rows:
+        ko = ref[t]["kept"]
+        kg = kept_gpu[t]
+        if not np.array_equal(ko, kg):
+            # several results are correct: differing blocks must sit at the cut
+            bs = ref[t]["bscores"].astype(np.float64)
+            cur = t // 64
+            others = np.arange(1, cur)
+            srt = np.sort(bs[1:cur])[::-1]
+            cut = srt[keep - 3]
+            for b in set(ko.tolist()) ^ set(kg.tolist()):
+                assert b not in (0, cur), f"row {t}: forced block {b} differs"
+                assert abs(bs[b] - cut) <= 2e-3 * np.abs(bs[:cur]).max(), f"row {t}: block {b} far from the cut"
+            n_diff += 1
+    assert n_diff <= max(2, len(rows) // 20)
+    pre = sa.Prefill(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, k,
+                     mode="two_stage", keep_blocks=keep)
+    out, lse, idx = pre()
+    torch.cuda.synchronize()
+    out, lse, idx = out.float().cpu().numpy(), lse.cpu().numpy(), idx.cpu().numpy()
+    ii = oracle.indexer.IndexerInputs(host)
+    for t in rows:
+        # stage 2 judged against the oracle's token scores over the GPU's kept blocks
+        cand = oracle.two_stage_candidates(kept_gpu[t], t, 64)
+        sc = oracle.scores_row(oracle.indexer.dequant(ii.q[t]), ii.sq[t], ii.kv[cand], ii.sk[cand], ii.w[t])
+        check_topk_row(idx[t], cand, sc, k, f"row {t}")
+    att = attention_rows(host, {t: idx[t] for t in rows})
+    for t in rows:
+        check_attention_row(out[t], att[t][0], lse[t], att[t][1], f"row {t}")
+
+
+def test_prefill_two_stage_small(sa):
+    wl = WORKLOADS["two_stage_t64k"].with_(T=6000, k=512)
+    rows = sample_rows(wl.T, 80, seed=3, k=512, extra=(63, 64, 4095, 4096, 5999))
+    _check_two_stage(sa, wl, 3, rows, k=512)
+
+
+def test_prefill_two_stage_equals_flat_below_64_blocks(sa):
+    wl = WORKLOADS["two_stage_t64k"].with_(T=3000, k=256, topic_run=256)
+    inp = PrefillInputs(wl, "cuda", seed=4)
+    a = sa.Prefill(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, 256, mode="flat")()
+    b = sa.Prefill(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, 256,
+                   mode="two_stage")()
+    torch.cuda.synchronize()
+    ia, ib = a[2].cpu().numpy(), b[2].cpu().numpy()
+    for t in range(wl.T):
+        assert sorted(ia[t].tolist()) == sorted(ib[t].tolist()), f"row {t}"
+
+
+# ------------------------------------------------------------------- decode
+def _check_decode(sa, wl, seed, seqs=None, seq_lens=None, k=None):
+    k = k or wl.k
+    inp = DecodeInputs(wl, "cuda", seed=seed)
+    if seq_lens is not None:
+        inp.seq_lens = torch.tensor(seq_lens, dtype=torch.int32, device="cuda")
+    host = inp.to_host()
+    dec = sa.Decode(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, inp.seq_lens, k)
+    out, lse, idx = dec()
+    torch.cuda.synchronize()
+    out, lse, idx = out.float().cpu().numpy(), lse.cpu().numpy(), idx.cpu().numpy()
+    seqs = range(wl.batch) if seqs is None else seqs
+    ref = oracle.decode_rows(host, seqs, k, attention=False)
+    for b in seqs:
+        check_topk_row(idx[b], ref[b]["cand"], ref[b]["scores"], k, f"seq {b}")
+        o, l = decode_attention_row(host, b, idx[b])
+        check_attention_row(out[b], o, lse[b], l, f"seq {b}")
+
+
+def test_decode_ragged_lengths(sa):
+    wl = WORKLOADS["decode_b64_l128k"].with_(batch=4, L=5000)
+    _check_decode(sa, wl, 0, seq_lens=[5000, 4097, 130, 2048], k=512)
+
+
+def test_decode_equals_prefill_last_row(sa):
+    wl = WORKLOADS["prefill_t16k"].with_(T=3000, k=512)
+    inp = PrefillInputs(wl, "cuda", seed=6)
+    T = wl.T
+    pre = sa.Prefill(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, 512)()
+    dec = sa.Decode(inp.q_idx[T - 1:T], inp.q_scale[T - 1:T], inp.k_idx[None], inp.k_scale[None], inp.w[T - 1:T],
+                    inp.Q[T - 1:T], inp.K[None], inp.V[None], torch.tensor([T], dtype=torch.int32, device="cuda"),
+                    512)()
+    torch.cuda.synchronize()
+    assert sorted(pre[2][T - 1].tolist()) == sorted(dec[2][0].tolist())
+    assert torch.equal(pre[0][T - 1], dec[0][0]) or (pre[0][T - 1].float() - dec[0][0].float()).abs().max() < 1e-2
+
+
+# ------------------------------------------------- full sizes, sampled rows
+def test_full_prefill_t16k_sampled(sa):
+    wl = WORKLOADS["prefill_t16k"]
+    rows = sample_rows(wl.T, 256, seed=10, k=wl.k)
+    _check_prefill(sa, wl, 0, rows)
+
+
+def test_full_two_stage_t64k_sampled(sa):
+    wl = WORKLOADS["two_stage_t64k"]
+    rows = sample_rows(wl.T, 256, seed=11, k=wl.k, extra=(63, 64, 4095, 4096))
+    _check_two_stage(sa, wl, 0, rows, k=wl.k)
+
+
+def test_full_decode_b64_l128k(sa):
+    wl = WORKLOADS["decode_b64_l128k"]
+    _check_decode(sa, wl, 0)
