@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""Benchmark of the learned top-k sparse-attention hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+  * a two-stage prefill of T = 65,536 tokens (block keys, stage-1 block
+    scores + keep, stage-2 token indexer, exact top-k = 2048, sparse MQA
+    attention over 16 heads x 128) -- the headline prefill tokens/s, and
+  * one decode step of 64 sequences x 131,072 cached keys (indexer, exact
+    top-2048, split-K attention) -- decode microseconds per token.
+L2 (126 MB) is flushed before every timed step by writing a 512 MB buffer
+outside the timed events. Inputs are seeded and synthetic (workloads module).
+
+  python bench.py --gpus N --steps K --warmup W [--impl reference]
+
+Under torchrun (N > 1) every rank runs its own independent copy of the
+workload (weak scaling; no collective on the data path); the reported time is
+the max over ranks.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn prefill tokens/s (indexer+top-k+attn) @64K k=2048; decode µs/token"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                rows.append(f)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows if _isnum(r[3])), default=None)}
+
+
+def _isnum(s):
+    try:
+        float(s)
+        return True
+    except ValueError:
+        return False
+
+
+# ------------------------------------------------------- algorithmic work
+def two_stage_work(wl):
+    """Data-independent algorithmic counts of the two-stage prefill."""
+    T, H, d, B, keep, k = wl.T, wl.H, wl.d, wl.block_size, wl.keep_blocks, wl.k
+    t = list(range(T))
+    blocks_scored = sum(p // B for p in t)                       # blocks [0, cur) per query
+    cand = sum(min(p + 1, (keep - 1) * B + p % B + 1) for p in t)  # visible keys of the kept blocks
+    pairs = sum(min(k, p + 1) for p in t)                        # selected keys attended
+    return {
+        "stage1_flops": 2.0 * H * d * blocks_scored,
+        "stage2_flops": 2.0 * H * d * cand,
+        "cand": cand,
+        "attn_pairs": pairs,
+        "attn_bytes": pairs * 2 * wl.dh * 2,                     # gathered K+V rows (bf16)
+        "attn_flops": 4.0 * wl.Hq * wl.dh * pairs,
+        "topk_bytes": cand * 4 + T * k * 4,                      # candidate scores read + index rows written
+    }
+
+
+def decode_work(wd):
+    B, L, d = wd.batch, wd.L, wd.d
+    return {
+        "indexer_bytes": B * L * (d + 4) + B * L * 4,            # FP8 keys + scales read, row scores written
+        "indexer_flops": 2.0 * wd.H * d * B * L,
+        "topk_bytes": B * L * 4,
+        "attn_bytes": B * min(wd.k, L) * 2 * wd.dh * 2,          # gathered K+V rows from HBM
+    }
+
+
+# ------------------------------------------------------------- CPU oracle
+def oracle_two_stage_sample(host, wl, n_rows: int, seed: int):
+    """Times the oracle on pooling (all blocks) + n_rows stratified rows of
+    the two-stage prefill; returns (tokens/s extrapolated to T rows, info)."""
+    import oracle
+    from oracle.two_stage import pool_block_keys
+    from workloads import sample_rows
+    rows = sample_rows(wl.T, n_rows, seed=seed, k=wl.k)
+    t0 = time.perf_counter()
+    blocks = pool_block_keys(host["k_idx"].numpy(), host["k_scale"].numpy(), wl.block_size)
+    t1 = time.perf_counter()
+    oracle.prefill_rows(host, rows, wl.k, mode="two_stage", keep=wl.keep_blocks, blocks=blocks)
+    t2 = time.perf_counter()
+    per_row = (t2 - t1) / len(rows)
+    full_s = (t1 - t0) + per_row * wl.T
+    return wl.T / full_s, {"pool_s": t1 - t0, "rows": len(rows), "rows_s": t2 - t1, "extrapolated_s": full_s}
+
+
+def oracle_decode_sample(hostd, wd, n_seq: int):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.decode_rows(hostd, range(n_seq), wd.k)
+    dt = time.perf_counter() - t0
+    return dt / n_seq * wd.batch * 1e6, dt        # µs per decode step of the full batch
+
+
+def blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max(i.get("num_threads", 1) for i in info if i.get("user_api") == "blas")
+    except Exception:
+        return os.cpu_count()
+
+
+# --------------------------------------------------------------- arms
+def run_reference(args):
+    """The oracle as the reference arm: rank 0 only, on host cores."""
+    import torch
+    from workloads import WORKLOADS, PrefillInputs, DecodeInputs
+    wl = WORKLOADS[args.workload]
+    wd = WORKLOADS["decode_b64_l128k"]
+    inp = PrefillInputs(wl, "cpu", seed=args.seed)
+    host = inp.to_host()
+    dinp = DecodeInputs(wd.with_(batch=2), "cpu", seed=args.seed)
+    hostd = dinp.to_host()
+    for i in range(args.warmup):
+        oracle_two_stage_sample(host, wl, args.ref_rows, seed=100 + i)
+    vals, infos = [], []
+    for i in range(args.steps):
+        v, info = oracle_two_stage_sample(host, wl, args.ref_rows, seed=200 + i)
+        vals.append(v)
+        infos.append(info)
+    dec_us, _ = oracle_decode_sample(hostd, wd.with_(batch=2), 1)
+    dec_us = dec_us / 2 * wd.batch
+    value = statistics.mean(vals)
+    sec_per_step = statistics.mean(x["extrapolated_s"] for x in infos)
+    sample = (f"per step: mean-pooling of all {wl.T // wl.block_size} blocks + {args.ref_rows} stratified "
+              f"query rows (both indexer stages, top-k, attention), extrapolated to {wl.T} rows")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(sec_per_step * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "k": wl.k, "mode": "two_stage", "block": wl.block_size,
+                   "keep_blocks": wl.keep_blocks, "seed": args.seed},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "decode": {"us_per_step": round(dec_us, 1), "us_per_token": round(dec_us / wd.batch, 2),
+                   "sample": "1 sequence of 131072 keys, scaled to the 64-sequence step"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_native(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from indexer_selected_top_b200.build import build
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    import indexer_selected_top_b200 as sa
+    from workloads import WORKLOADS, PrefillInputs, DecodeInputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[args.workload]
+    wd = WORKLOADS["decode_b64_l128k"]
+    seed = args.seed + 1000 * rank
+    inp = PrefillInputs(wl, dev, seed=seed)
+    ptimer = sa.StageTimer(sa.PREFILL_STAGES[wl.mode])
+    pre = sa.Prefill(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, wl.k, mode=wl.mode,
+                     keep_blocks=wl.keep_blocks, chunk_rows=wl.T, timer=ptimer)
+    dec = None
+    if not args.no_decode:
+        dinp = DecodeInputs(wd, dev, seed=seed)
+        dtimer = sa.StageTimer(sa.DECODE_STAGES)
+        dec = sa.Decode(dinp.q_idx, dinp.q_scale, dinp.k_idx, dinp.k_scale, dinp.w, dinp.Q, dinp.K, dinp.V,
+                        dinp.seq_lens, wd.k, timer=dtimer)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(timed):
+        flush.fill_(1)                                   # evict L2, outside the timed events
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        pre()
+        e1.record(stream)
+        if dec is not None:
+            dec()
+        e2.record(stream)
+        return e0, e1, e2
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    recs = []
+    stage_ms = {n: 0.0 for n in ptimer.names}
+    dstage_ms = {n: 0.0 for n in sa.DECODE_STAGES}
+    for _ in range(args.steps):
+        recs.append(step(True))
+        torch.cuda.synchronize()                         # read this step's stage events
+        for n, v in ptimer.ms().items():
+            stage_ms[n] += v
+        if dec is not None:
+            for n, v in dtimer.ms().items():
+                dstage_ms[n] += v
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    pre_ms = sum(a.elapsed_time(b) for a, b, _ in recs)
+    dec_ms = sum(b.elapsed_time(c) for _, b, c in recs)
+    tot = torch.tensor([pre_ms, dec_ms, pre_ms + dec_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
+    pre_ms, dec_ms, all_ms = (float(x) for x in tot.cpu())
+    K = args.steps
+
+    # ---------------- roofline of the dominant prefill kernel ----------------
+    peaks, peak_src = load_peaks()
+    fp8_peak = 2.0 * peaks["bf16_tflops"]                # dense FP8 = 2 x measured bf16 (nominal ratio)
+    work = two_stage_work(wl)
+    avg = {n: v / K for n, v in stage_ms.items()}
+    stages = {}
+    for n, ms in avg.items():
+        s = ms * 1e-3
+        if n == "stage2_indexer":
+            stages[n] = {"ms": round(ms, 4), "bound": "tensor", "achieved": work["stage2_flops"] / s / 1e12,
+                         "peak": fp8_peak, "unit": "TFLOP/s"}
+        elif n == "stage1_indexer":
+            stages[n] = {"ms": round(ms, 4), "bound": "tensor", "achieved": work["stage1_flops"] / s / 1e12,
+                         "peak": fp8_peak, "unit": "TFLOP/s"}
+        elif n == "attention":
+            stages[n] = {"ms": round(ms, 4), "bound": "hbm", "achieved": work["attn_bytes"] / s / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        elif n == "topk":
+            stages[n] = {"ms": round(ms, 4), "bound": "hbm", "achieved": work["topk_bytes"] / s / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        else:
+            stages[n] = {"ms": round(ms, 4)}
+    for v in stages.values():
+        if "achieved" in v:
+            v["achieved"] = round(v["achieved"], 2)
+            v["frac"] = round(v["achieved"] / v["peak"], 4)
+    dom = max((n for n in stages if "achieved" in stages[n]), key=lambda n: stages[n]["ms"])
+    roof = dict(stages[dom])
+    roof.pop("ms")
+    roof["kernel"] = dom
+    roof["traffic"] = None
+    roof["peak_source"] = (f"{peak_src}: " + ("2 x bf16 burst (nominal FP8/bf16 ratio)" if roof["unit"] == "TFLOP/s"
+                                              else "HBM copy"))
+
+    decode = None
+    if dec is not None:
+        dw = decode_work(wd)
+        davg = {n: v / K for n, v in dstage_ms.items()}
+        us = dec_ms / K * 1e3
+        decode = {"us_per_step": round(us, 1), "us_per_token": round(us / wd.batch, 3), "batch": wd.batch,
+                  "L": wd.L, "k": wd.k, "stages_ms": {n: round(v, 4) for n, v in davg.items()},
+                  "indexer_hbm_frac": round(dw["indexer_bytes"] / (davg["indexer"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                            4),
+                  "gather_hbm_frac": round(dw["attn_bytes"] / (davg["attention"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                           4),
+                  "step_hbm_frac": round((dw["indexer_bytes"] + dw["topk_bytes"] + dw["attn_bytes"]) /
+                                         (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)}
+
+    # ---------------- end to end through host buffers ----------------
+    e2e = None
+    if not args.skip_e2e:
+        names = ("q_idx", "q_scale", "k_idx", "k_scale", "w", "Q", "K", "V")
+        hbuf = {n: getattr(inp, n).cpu().pin_memory() for n in names}
+        hout = torch.empty(pre.out.shape, dtype=pre.out.dtype).pin_memory()
+        hlse = torch.empty(pre.lse.shape, dtype=pre.lse.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in hbuf.values())
+        d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
+        ne = max(1, min(args.steps, args.e2e_steps))
+
+        def e2e_step():
+            for n in names:
+                getattr(inp, n).copy_(hbuf[n], non_blocking=True)
+            pre()
+            hout.copy_(pre.out, non_blocking=True)
+            hlse.copy_(pre.lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(ne):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        t_e2e = torch.tensor([a.elapsed_time(b) / ne], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
+        e2e = {"value": round(world * wl.T / (float(t_e2e) * 1e-3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ne}
+
+    # ---------------- CPU oracle baseline (rank 0, N = 1) ----------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+        host = inp.to_host()
+        v, info = oracle_two_stage_sample(host, wl, args.cpu_rows, seed=7)
+        cpu = {"value": round(v, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"mean-pooling of all {wl.T // wl.block_size} blocks ({info['pool_s']:.1f} s) + "
+                         f"{info['rows']} stratified rows ({info['rows_s']:.1f} s: both indexer stages, top-k, "
+                         f"attention), extrapolated to {wl.T} rows"}
+
+    launches_per_step = 6 + (4 if dec is not None else 0)
+    line = {
+        "metric": METRIC,
+        "value": round(world * K * wl.T / (pre_ms * 1e-3), 1),
+        "unit": "tokens/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(all_ms / K, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8-e4m3 indexer (f32 accumulate), bf16 attention (f32 softmax)",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "d_idx": wl.d, "k": wl.k, "mode": wl.mode,
+                   "block": wl.block_size, "keep_blocks": wl.keep_blocks, "Hq": wl.Hq, "head_dim": wl.dh,
+                   "decode": None if dec is None else {"workload": wd.name, "batch": wd.batch, "L": wd.L},
+                   "parallelism": f"replicas x{world}", "l2": "flushed (512 MB write) before every step",
+                   "prefill_ms_per_step": round(pre_ms / K, 4)},
+        "roofline": roof,
+        "stages": stages,
+        "decode": decode,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * K,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("native", "reference"), default="native")
+    ap.add_argument("--workload", default="two_stage_t64k")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=96)
+    ap.add_argument("--ref-rows", type=int, default=12)
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_native(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

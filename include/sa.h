@@ -133,6 +133,18 @@ typedef struct {
   uint32_t overflow_rows;  /* rows whose candidate list overflowed */
 } sa_device_status;
 
+/* Optional stage timing: when stage_events is non-NULL the call records
+ * stage_events[i] on `stream` before stage i of its FIRST chunk and
+ * stage_events[n] after its last stage (n_stage_events must be >= n + 1).
+ * Stages (n): FLAT = indexer, top-k, attention (3); TWO_STAGE = pooling,
+ * stage-1 indexer, block keep, stage-2 indexer, top-k, attention (6);
+ * decode = indexer, top-k, attention (3). Events are created by the caller;
+ * an event that cannot be recorded makes the call return
+ * SA_ERR_INVALID_ARGUMENT after its work has been queued. */
+#define SA_PREFILL_FLAT_STAGES 3
+#define SA_PREFILL_TWO_STAGE_STAGES 6
+#define SA_DECODE_STAGES 3
+
 typedef struct {
   int32_t k;             /* top-k budget, 1..4096 */
   sa_mode mode;          /* FLAT or TWO_STAGE */
@@ -141,12 +153,16 @@ typedef struct {
   int32_t chunk_rows;    /* query rows per chunk (0 = library default) */
   sa_device_status* status;  /* device, nullable; zeroed by the call */
   int32_t test_hook;     /* 0 in production; see SA_HOOK_* */
+  cudaEvent_t* stage_events;  /* host array, nullable (see above) */
+  int32_t n_stage_events;
 } sa_prefill_opts;
 
 typedef struct {
   int32_t k;
   sa_device_status* status;  /* device, nullable; zeroed by the call */
   int32_t test_hook;
+  cudaEvent_t* stage_events;  /* host array, nullable (see above) */
+  int32_t n_stage_events;
 } sa_decode_opts;
 
 /* test hooks: force the threshold of the streaming selector */

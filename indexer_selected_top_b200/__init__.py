@@ -52,11 +52,36 @@ class AttnIn(ctypes.Structure):
 class PrefillOpts(ctypes.Structure):
     _fields_ = [("k", ctypes.c_int32), ("mode", ctypes.c_int), ("block_size", ctypes.c_int32),
                 ("keep_blocks", ctypes.c_int32), ("chunk_rows", ctypes.c_int32), ("status", ctypes.c_void_p),
-                ("test_hook", ctypes.c_int32)]
+                ("test_hook", ctypes.c_int32), ("stage_events", ctypes.c_void_p), ("n_stage_events", ctypes.c_int32)]
 
 
 class DecodeOpts(ctypes.Structure):
-    _fields_ = [("k", ctypes.c_int32), ("status", ctypes.c_void_p), ("test_hook", ctypes.c_int32)]
+    _fields_ = [("k", ctypes.c_int32), ("status", ctypes.c_void_p), ("test_hook", ctypes.c_int32),
+                ("stage_events", ctypes.c_void_p), ("n_stage_events", ctypes.c_int32)]
+
+
+PREFILL_STAGES = {"flat": ("indexer", "topk", "attention"),
+                  "two_stage": ("pool", "stage1_indexer", "block_keep", "stage2_indexer", "topk", "attention")}
+DECODE_STAGES = ("indexer", "topk", "attention")
+
+
+class StageTimer:
+    """torch.cuda.Events handed to the library; stage i runs between events i
+    and i+1 (first chunk only)."""
+
+    def __init__(self, names):
+        self.names = names
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+        for e in self.events:          # torch creates the CUDA event on first record
+            e.record()
+        self._arr = (ctypes.c_void_p * len(self.events))(*[e.cuda_event for e in self.events])
+
+    @property
+    def ptr(self):
+        return ctypes.cast(self._arr, ctypes.c_void_p)
+
+    def ms(self) -> dict:
+        return {n: self.events[i].elapsed_time(self.events[i + 1]) for i, n in enumerate(self.names)}
 
 
 _P = ctypes.c_void_p
@@ -184,12 +209,15 @@ class Prefill:
 
     def __init__(self, q, q_scale, k, k_scale, w, Q, K, V, k_top: int, mode: str = "flat", block_size=64,
                  keep_blocks=64, chunk_rows=0, q_pos0=0, softmax_scale=0.0, want_idx=True, want_lse=True,
-                 status=None, test_hook=0):
+                 status=None, test_hook=0, timer: "StageTimer" = None):
         self.ind = indexer_in(q, q_scale, k, k_scale, w, q_pos0)
         self.att = attn_in(Q, K, V, softmax_scale)
         self.opts = PrefillOpts(k=k_top, mode=SA_MODE_TWO_STAGE if mode == "two_stage" else SA_MODE_FLAT,
                                 block_size=block_size, keep_blocks=keep_blocks, chunk_rows=chunk_rows,
-                                status=_ptr(status), test_hook=test_hook)
+                                status=_ptr(status), test_hook=test_hook,
+                                stage_events=timer.ptr if timer else None,
+                                n_stage_events=len(timer.events) if timer else 0)
+        self.timer = timer
         self.nws = workspace_size(SA_OP_PREFILL, self.ind, self.att, self.opts)
         self.ws = _workspace(self.nws, Q.device)
         self.idx = torch.empty((Q.shape[0], k_top), dtype=torch.int32, device=Q.device) if want_idx else None
@@ -212,10 +240,13 @@ class Decode:
     """A prepared sa_decode call (one decode step of a batch of sequences)."""
 
     def __init__(self, q, q_scale, k, k_scale, w, Q, K, V, seq_lens, k_top: int, softmax_scale=0.0,
-                 want_idx=True, want_lse=True, status=None, test_hook=0):
+                 want_idx=True, want_lse=True, status=None, test_hook=0, timer: "StageTimer" = None):
         self.ind = indexer_in(q, q_scale, k, k_scale, w, 0, seq_lens)
         self.att = attn_in(Q, K, V, softmax_scale)
-        self.opts = DecodeOpts(k=k_top, status=_ptr(status), test_hook=test_hook)
+        self.opts = DecodeOpts(k=k_top, status=_ptr(status), test_hook=test_hook,
+                               stage_events=timer.ptr if timer else None,
+                               n_stage_events=len(timer.events) if timer else 0)
+        self.timer = timer
         self.nws = workspace_size(SA_OP_DECODE, self.ind, self.att, self.opts)
         self.ws = _workspace(self.nws, Q.device)
         self.idx = torch.empty((Q.shape[0], k_top), dtype=torch.int32, device=Q.device) if want_idx else None

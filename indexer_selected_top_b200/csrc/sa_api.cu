@@ -179,6 +179,20 @@ static IdxArgs base_args(const sa_indexer_in* in, uint32_t* status, int hook) {
 
 static size_t esize(sa_dtype d) { return d == SA_FP8_E4M3 ? 1 : 2; }
 
+// Records stage_events[i] (first chunk only) when the caller asked for them.
+struct StageMarks {
+  cudaEvent_t* ev;
+  int n;
+  bool on;
+  bool ok = true;
+  void mark(int i, cudaStream_t st) {
+    if (on && ev != nullptr && i < n && cudaEventRecord(ev[i], st) != cudaSuccess) {
+      (void)cudaGetLastError();   // do not let a bad event handle surface as a launch error
+      ok = false;
+    }
+  }
+};
+
 }  // namespace sa
 
 using namespace sa;
@@ -310,9 +324,14 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
   const size_t qrow = (size_t)in->n_heads * in->d_idx * esize(in->dtype);
   cudaError_t e = cudaSuccess;
 
+  const int n_stages = o->mode == SA_MODE_FLAT ? SA_PREFILL_FLAT_STAGES : SA_PREFILL_TWO_STAGE_STAGES;
+  if (o->stage_events != nullptr && o->n_stage_events < n_stages + 1) return SA_ERR_INVALID_ARGUMENT;
+  StageMarks sm{o->stage_events, o->n_stage_events, true};
+
   if (o->mode == SA_MODE_TWO_STAGE) {
     uint8_t* blk = reinterpret_cast<uint8_t*>(w + p.off_blk);
     float* blks = reinterpret_cast<float*>(w + p.off_blks);
+    sm.mark(0, stream);
     e = launch_pool_blocks(static_cast<const uint8_t*>(in->k), in->k_scale, p.nb, o->block_size, blk, blks, stream);
     if (e != cudaSuccess) return cuda_status(e);
   }
@@ -326,13 +345,16 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
     ci.q_scale = in->q_scale ? in->q_scale + (size_t)r0 * in->n_heads : nullptr;
     ci.w = in->w + (size_t)r0 * in->n_heads;
     int32_t* idx = idx_out ? idx_out + (size_t)r0 * o->k : reinterpret_cast<int32_t*>(w + p.off_idx);
+    sm.on = (r0 == 0);
     if (o->mode == SA_MODE_FLAT) {
       float* table = reinterpret_cast<float*>(w + p.off_table);
       IdxArgs a = base_args(&ci, status, o->test_hook);
       a.out = table;
       a.ld = in->n_k;
+      sm.mark(0, stream);
       e = launch_indexer(IDX_PREFILL, in->n_heads, in->d_idx, in->dtype, ci.q, in->k, R, in->n_k, a, stream);
       if (e != cudaSuccess) return cuda_status(e);
+      sm.mark(1, stream);
       e = launch_topk_table(table, R, in->n_k, in->n_k, ci.q_pos0, o->k, idx, 0, nullptr, 0, nullptr, stream);
       if (e != cudaSuccess) return cuda_status(e);
     } else {
@@ -343,6 +365,7 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
       float* cand = reinterpret_cast<float*>(w + p.off_cand);
       const int ncand = o->keep_blocks * o->block_size;
       // stage 1: complete blocks b < floor(p / block) (the current block is forced)
+      sm.mark(1, stream);
       if (p.nb > 0) {
         sa_indexer_in bi = ci;
         bi.n_k = p.nb;
@@ -356,10 +379,12 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
         e = launch_indexer(IDX_PREFILL, in->n_heads, in->d_idx, in->dtype, ci.q, blk, R, p.nb, a, stream);
         if (e != cudaSuccess) return cuda_status(e);
       }
+      sm.mark(2, stream);
       e = launch_block_select(bsc, R, p.nb, std::max(p.nb, 1), ci.q_pos0, o->block_size, o->keep_blocks, kept,
                               stream);
       if (e != cudaSuccess) return cuda_status(e);
       // stage 2: the visible keys of the kept blocks
+      sm.mark(3, stream);
       IdxArgs a = base_args(&ci, status, o->test_hook);
       a.out = cand;
       a.ld = ncand;
@@ -367,17 +392,20 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
       a.keep = o->keep_blocks;
       e = launch_indexer(IDX_GATHER, in->n_heads, in->d_idx, in->dtype, ci.q, in->k, R, in->n_k, a, stream);
       if (e != cudaSuccess) return cuda_status(e);
+      sm.mark(4, stream);
       e = launch_topk_table(cand, R, ncand, ncand, ci.q_pos0, o->k, idx, 2, kept, o->keep_blocks, nullptr, stream);
       if (e != cudaSuccess) return cuda_status(e);
     }
     const void* qa = static_cast<const char*>(at->q) + (size_t)r0 * at->n_q_heads * at->head_dim * 2;
     void* oa = static_cast<char*>(out) + (size_t)r0 * at->n_q_heads * at->head_dim * 2;
     float* la = lse ? lse + (size_t)r0 * at->n_q_heads : nullptr;
+    sm.mark(n_stages - 1, stream);
     e = launch_attention(qa, at->k_cache, at->v_cache, idx, R, o->k, at->n_k, at->n_q_heads, at->head_dim, scale, 0,
                          oa, la, nullptr, nullptr, 1, stream);
     if (e != cudaSuccess) return cuda_status(e);
+    sm.mark(n_stages, stream);
   }
-  return SA_OK;
+  return sm.ok ? SA_OK : SA_ERR_INVALID_ARGUMENT;
 }
 
 sa_status sa_decode(const sa_indexer_in* in, const sa_attn_in* at, const sa_decode_opts* o, int32_t* idx_out,
@@ -395,21 +423,28 @@ sa_status sa_decode(const sa_indexer_in* in, const sa_attn_in* at, const sa_deco
   char* w = static_cast<char*>(ws);
   uint32_t* status = o->status ? reinterpret_cast<uint32_t*>(o->status) : nullptr;
   if (status && cudaMemsetAsync(status, 0, sizeof(sa_device_status), stream) != cudaSuccess) return SA_ERR_CUDA;
+  if (o->stage_events != nullptr && o->n_stage_events < SA_DECODE_STAGES + 1) return SA_ERR_INVALID_ARGUMENT;
+  StageMarks sm{o->stage_events, o->n_stage_events, true};
   float* rows = reinterpret_cast<float*>(w + p.off_scores);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + p.off_idx);
   IdxArgs a = base_args(in, status, o->test_hook);
   a.out = rows;
   a.ld = in->n_k;
   a.tiles_per_cta = kDecodeTilesPerCta;
+  sm.mark(0, stream);
   cudaError_t e = launch_indexer(IDX_DECODE, in->n_heads, in->d_idx, in->dtype, in->q, in->k, in->batch,
                                  (long long)in->batch * in->n_k, a, stream);
   if (e != cudaSuccess) return cuda_status(e);
+  sm.mark(1, stream);
   e = launch_topk_table(rows, in->batch, in->n_k, in->n_k, 0, o->k, idx, 1, nullptr, 0, in->seq_lens, stream);
   if (e != cudaSuccess) return cuda_status(e);
+  sm.mark(2, stream);
   e = launch_attention(at->q, at->k_cache, at->v_cache, idx, in->batch, o->k, at->n_k, at->n_q_heads, at->head_dim,
                        attn_scale(at), in->batch, out, lse, reinterpret_cast<float*>(w + p.off_po),
                        reinterpret_cast<float*>(w + p.off_pl), p.splits, stream);
-  return cuda_status(e);
+  if (e != cudaSuccess) return cuda_status(e);
+  sm.mark(3, stream);
+  return sm.ok ? SA_OK : SA_ERR_INVALID_ARGUMENT;
 }
 
 }  // extern "C"
