@@ -199,9 +199,13 @@ def run_reference(args):
 def run_native(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
-    from indexer_selected_top_b200.build import build
     if rank == 0:
-        build()
+        import importlib.util
+        spec = importlib.util.spec_from_file_location("_sa_build", os.path.join(ROOT, "indexer_selected_top_b200",
+                                                                                "build.py"))
+        mod = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(mod)
+        mod.build()
     if world > 1:
         dist.barrier()
     import indexer_selected_top_b200 as sa

@@ -11,8 +11,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def sa():
-    from indexer_selected_top_b200.build import build
-    build()
+    from conftest import ensure_built
+    ensure_built()
     import indexer_selected_top_b200 as m
     return m
 

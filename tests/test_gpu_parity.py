@@ -17,8 +17,8 @@ pytestmark = pytest.mark.gpu
 def sa():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    from indexer_selected_top_b200.build import build
-    build()
+    from conftest import ensure_built
+    ensure_built()
     import indexer_selected_top_b200 as m
     return m
 
