@@ -245,6 +245,28 @@ sa_status sa_decode(const sa_indexer_in* in, const sa_attn_in* attn, const sa_de
                     cudaStream_t stream);
 
 /*
+ * sa_sparse_attn_decode_noalloc: the decode form of sa_sparse_attn (batch >
+ * 0) for callers that cannot provide device workspace -- for example a plugin
+ * in a serving engine that owns all device memory and passes only inputs and
+ * outputs, or a decode loop whose memory is fixed after start-up and which
+ * must not call the CUDA allocator (cudaMalloc / cudaFree may synchronise the
+ * device). The pages have no counterpart; this is a deployment convenience.
+ *   Arguments and results as sa_sparse_attn with batch > 0, without ws.
+ *   The per-split partial results live in one fixed array inside the library
+ *   (8 MiB + 512 KiB of device memory on every GPU that loads it, held until
+ *   the process exits): batch * ceil(k / 256) * n_q_heads * head_dim must be
+ *   <= 2^21 and batch * ceil(k / 256) * n_q_heads <= 2^17, otherwise the call
+ *   returns SA_ERR_WORKSPACE_TOO_SMALL and launches nothing (64 sequences x
+ *   k = 2048 x 16 heads x 128 fits).
+ *   The first call on a device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   Every call uses the same array, so calls that overlap on the GPU (other
+ *   streams, other host threads) race: order them. Calls allocate nothing.
+ */
+sa_status sa_sparse_attn_decode_noalloc(const sa_attn_in* in, const int32_t* idx, int32_t k, void* out,
+                                        float* lse, cudaStream_t stream);
+
+/*
  * sa_workspace_size: bytes of device workspace `op` needs for these operands
  * (host call, no device work). opts points to sa_prefill_opts (PREFILL),
  * sa_decode_opts (DECODE), an int32_t k (TOPK, SPARSE_ATTN) or NULL.

@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsa.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libsa.so not built ({LIB_PATH}); run python -m indexer_selected_top_b200.build")
+    raise ImportError(f"libsa.so not built ({LIB_PATH}); run python indexer_selected_top_b200/build.py")
 _lib = ctypes.CDLL(LIB_PATH)
 
 # ----------------------------------------------------------------- constants
@@ -32,7 +32,7 @@ SA_OP_INDEX_SCORES, SA_OP_TOPK, SA_OP_SPARSE_ATTN, SA_OP_PREFILL, SA_OP_DECODE =
 SA_HOOK_NONE, SA_HOOK_THETA_POS_INF, SA_HOOK_THETA_NEG_INF, SA_HOOK_STALL_WAIT = range(4)
 
 EXPORTS = ("sa_status_string", "sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode",
-           "sa_workspace_size")
+           "sa_workspace_size", "sa_sparse_attn_decode_noalloc")
 
 
 class IndexerIn(ctypes.Structure):
@@ -97,7 +97,9 @@ _lib.sa_decode.argtypes = [ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), ct
                            _P, _P, ctypes.c_size_t, _P]
 _lib.sa_workspace_size.argtypes = [ctypes.c_int, ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), _P,
                                    ctypes.POINTER(ctypes.c_size_t)]
-for _f in ("sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode", "sa_workspace_size"):
+_lib.sa_sparse_attn_decode_noalloc.argtypes = [ctypes.POINTER(AttnIn), _P, ctypes.c_int32, _P, _P, _P]
+for _f in ("sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode", "sa_workspace_size",
+           "sa_sparse_attn_decode_noalloc"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -200,6 +202,19 @@ def sparse_attn(Q, K, V, idx, softmax_scale=0.0, out=None, lse=None, stream=None
     ws = _workspace(nws, Q.device)
     _check(_lib.sa_sparse_attn(ctypes.byref(att), _ptr(idx), k, _ptr(out), _ptr(lse), _aligned(ws), nws,
                                _stream(stream)), "sa_sparse_attn")
+    return out, lse
+
+
+def sparse_attn_decode_noalloc(Q, K, V, idx, softmax_scale=0.0, out=None, lse=None, stream=None):
+    """Decode attention (K/V [B, L, dh]) that takes no workspace: for callers
+    that cannot allocate device memory around the call (see sa.h)."""
+    att = attn_in(Q, K, V, softmax_scale)
+    if out is None:
+        out = torch.empty_like(Q)
+    if lse is None:
+        lse = torch.empty(Q.shape[:2], dtype=torch.float32, device=Q.device)
+    _check(_lib.sa_sparse_attn_decode_noalloc(ctypes.byref(att), _ptr(idx), idx.shape[1], _ptr(out), _ptr(lse),
+                                              _stream(stream)), "sa_sparse_attn_decode_noalloc")
     return out, lse
 
 

@@ -1,5 +1,8 @@
 """Builds libsa.so (the CUDA library behind include/sa.h) in-tree with nvcc
-for sm_100a. Usage: python -m indexer_selected_top_b200.build"""
+for sm_100a. Usage: python indexer_selected_top_b200/build.py [--force]
+
+Run it by path (or load it with load_build below): importing the package
+itself loads libsa.so, which must already exist."""
 import os
 import subprocess
 import sys
@@ -7,7 +10,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["sa_api.cu", "indexer.cu", "topk.cu", "attn.cu", "pool.cu"]
+SOURCES = ["sa_api.cu", "indexer.cu", "topk.cu", "attn.cu", "pool.cu", "noalloc.cu"]
 LIB = os.path.join(HERE, "libsa.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
