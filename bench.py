@@ -214,6 +214,8 @@ def run_native(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     wl = WORKLOADS[args.workload]
+    if args.T:
+        wl = wl.with_(T=args.T)
     wd = WORKLOADS["decode_b64_l128k"]
     seed = args.seed + 1000 * rank
     inp = PrefillInputs(wl, dev, seed=seed)
@@ -400,6 +402,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("native", "reference"), default="native")
     ap.add_argument("--workload", default="two_stage_t64k")
+    ap.add_argument("--T", type=int, default=0, help="override the prefill length (profiling runs)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")

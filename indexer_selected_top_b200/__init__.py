@@ -17,7 +17,8 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsa.so")
+# SA_LIB may name another build of the same library (e.g. a tuning variant)
+LIB_PATH = os.environ.get("SA_LIB") or os.path.join(_HERE, "libsa.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libsa.so not built ({LIB_PATH}); run python indexer_selected_top_b200/build.py")

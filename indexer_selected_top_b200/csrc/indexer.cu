@@ -12,9 +12,10 @@
 // are positive: ReLU(sq*sk*a) = sq*sk*ReLU(a).
 //
 // Roles (320 threads): warp 0 = TMA producer (one lane), warp 1 = MMA issuer
-// (one lane) and TMEM owner, warps 2..9 = two epilogue teams of 4 warps, one
-// per TMEM accumulator buffer (2 x 256 fp32 columns), so the epilogue of one
-// accumulator overlaps the MMAs into the other (the pages' bucket scan also
+// (one lane) and TMEM owner, warps 2..9 = two epilogue teams of 4 warps. The
+// 512 TMEM columns hold 512 / N fp32 accumulators (2 at N = 256, 8 at N = 64)
+// used as a ring; team b % 2 drains buffer b, so the epilogue of one
+// accumulator overlaps the MMAs into the others (the pages' bucket scan also
 // overlaps its epilogue with its products: appendix F.1, "Flat prefill").
 //
 // Key sources (template MODE):
@@ -32,6 +33,14 @@
 
 namespace sa {
 
+// Tuning knobs (compile-time): queries per gather CTA and key-tile ring depth.
+#ifndef SA_IDX_GATHER_NQ
+#define SA_IDX_GATHER_NQ 8
+#endif
+#ifndef SA_IDX_STAGES
+#define SA_IDX_STAGES 6
+#endif
+
 template <int H, int D, bool FP8, int MODE>
 struct IdxCfg {
   static constexpr int ESZ = FP8 ? 1 : 2;
@@ -39,12 +48,16 @@ struct IdxCfg {
   static constexpr int QS = (MODE == IDX_PREFILL) ? (256 / H) : 1;
   static constexpr int N = QS * H;                           // MMA N
   static constexpr int G = (MODE == IDX_PREFILL) ? 2 : 1;    // sub-tiles per CTA
-  static constexpr int NQ = (MODE == IDX_PREFILL) ? QS * G : (MODE == IDX_GATHER ? 4 : 1);
+  static constexpr int NQ = (MODE == IDX_PREFILL) ? QS * G : (MODE == IDX_GATHER ? SA_IDX_GATHER_NQ : 1);
+  static constexpr int NBUF = 512 / N;                       // TMEM accumulator buffers (fp32 columns)
   static constexpr int QBYTES = NQ * H * ROWB;
   static constexpr int KBYTES = 128 * ROWB;
-  static constexpr int NS = (MODE == IDX_DECODE) ? 8 : 6;    // key-tile stages
+  static constexpr int NS = (MODE == IDX_DECODE) ? 8 : SA_IDX_STAGES;    // key-tile stages
   static constexpr int KSTEPS = ROWB / 32;                   // 32-byte K slices per MMA
-  static constexpr int SMEM_USED = 1024 + QBYTES + NS * KBYTES + NQ * H * 4 + (2 * NS + 8) * 8 + 16;
+  static constexpr int KEEPMAX = 64;                          // gather: kept blocks per query
+  static constexpr int KEPT_BYTES = (MODE == IDX_GATHER) ? NQ * KEEPMAX * 4 : 0;
+  static constexpr int SMEM_USED =
+      1024 + QBYTES + NS * KBYTES + NQ * H * 4 + KEPT_BYTES + (2 * NS + 1 + 2 * NBUF) * 8 + 16;
   // at least 120 KB: one CTA per SM, so two CTAs never contend for TMEM
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   static_assert(N <= 256 && N % 16 == 0, "MMA N");
@@ -95,13 +108,14 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + C::QBYTES;
   float* sW = reinterpret_cast<float*>(sK + C::NS * C::KBYTES);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sW + C::NQ * H);
+  int* sKept = reinterpret_cast<int*>(sW + C::NQ * H);         // gather: [NQ][KEEPMAX], -1 padded
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sKept) + C::KEPT_BYTES);
   uint64_t* kfull = bars;
   uint64_t* kempty = bars + C::NS;
   uint64_t* qfull = bars + 2 * C::NS;
   uint64_t* tfull = qfull + 1;
-  uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* tempty = tfull + C::NBUF;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + C::NBUF);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -127,13 +141,7 @@ __global__ void __launch_bounds__(320, 1)
     njobs = ntiles;
   } else {
     q0 = blockIdx.x * C::NQ;
-    nq = min(C::NQ, a.n_q - q0);
-    for (int ql = 0; ql < nq; ++ql) {
-      int nb = 0;
-      while (nb < a.keep && a.kept[(long long)(q0 + ql) * a.keep + nb] >= 0) ++nb;
-      njobs += (nb + 1) / 2;
-    }
-    ntiles = njobs;
+    nq = min(C::NQ, a.n_q - q0);   // jobs are counted from the staged kept lists below
   }
 
   // ---------------- setup ----------------
@@ -143,7 +151,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&kempty[s], 1);
     }
     mbar_init(qfull, 1);
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::NBUF; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 4);
     }
@@ -160,7 +168,22 @@ __global__ void __launch_bounds__(320, 1)
     }
     sW[i] = v;
   }
+  if constexpr (MODE == IDX_GATHER) {
+    // the CTA's kept-block lists, staged once: every role walks them per job
+    for (int i = threadIdx.x; i < C::NQ * C::KEEPMAX; i += blockDim.x) {
+      const int ql = i / C::KEEPMAX, j = i % C::KEEPMAX;
+      sKept[i] = (ql < nq && j < a.keep) ? a.kept[(long long)(q0 + ql) * a.keep + j] : -1;
+    }
+  }
   __syncthreads();
+  if constexpr (MODE == IDX_GATHER) {
+    for (int ql = 0; ql < nq; ++ql) {
+      int nb = 0;
+      while (nb < C::KEEPMAX && sKept[ql * C::KEEPMAX + nb] >= 0) ++nb;
+      njobs += (nb + 1) / 2;
+    }
+    ntiles = njobs;
+  }
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const WaitCtx wc{abort_flag, a.status, a.budget};
@@ -179,7 +202,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int ql = 0; ql < nq; ++ql) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, (q0 + ql) * H);
       }
       GatherCursor gc;
-      if constexpr (MODE == IDX_GATHER) gc.init(a.kept, a.keep, q0, nq);
+      if constexpr (MODE == IDX_GATHER) gc.init(sKept, C::KEEPMAX, 0, nq);
       int issued = 0;
       for (int i = 0; i < ntiles; ++i) {
         const int st = i % C::NS, u = i / C::NS;
@@ -195,7 +218,7 @@ __global__ void __launch_bounds__(320, 1)
         } else {
           const int* kr = gc.row();
           const int b0 = kr[2 * gc.pair];
-          const int b1 = (2 * gc.pair + 1 < a.keep) ? kr[2 * gc.pair + 1] : -1;
+          const int b1 = kr[2 * gc.pair + 1];
           mbar_arrive_expect_tx(&kfull[st], (b1 >= 0 ? 2 : 1) * 64 * C::ROWB);
           tma_load_2d(dst, &kmap, &kfull[st], 0, b0 * 64);
           if (b1 >= 0) tma_load_2d(dst + 64 * C::ROWB, &kmap, &kfull[st], 0, b1 * 64);
@@ -216,7 +239,7 @@ __global__ void __launch_bounds__(320, 1)
       if (mbar_wait(qfull, 0, wc, 2)) {
         tc_fence_after();
         GatherCursor gc;
-        if constexpr (MODE == IDX_GATHER) gc.init(a.kept, a.keep, q0, nq);
+        if constexpr (MODE == IDX_GATHER) gc.init(sKept, C::KEEPMAX, 0, nq);
         for (int j = 0; j < njobs; ++j) {
           int tile, g;
           if constexpr (MODE == IDX_PREFILL) {
@@ -227,7 +250,7 @@ __global__ void __launch_bounds__(320, 1)
             g = (MODE == IDX_GATHER) ? gc.ql : 0;
           }
           const int st = tile % C::NS;
-          const int buf = j & 1, ub = j >> 1;
+          const int buf = j % C::NBUF, ub = j / C::NBUF;
           if (g == 0 || MODE != IDX_PREFILL) {
             if (!mbar_wait(&kfull[st], (tile / C::NS) & 1, wc, 3)) break;
           }
@@ -239,7 +262,7 @@ __global__ void __launch_bounds__(320, 1)
           }
           const uint32_t a_base = smem_u32(sK + st * C::KBYTES);
           const uint32_t b_base = smem_u32(sQ + g * (C::N * C::ROWB));
-          const uint32_t d_tmem = tmem_base + buf * 256;
+          const uint32_t d_tmem = tmem_base + buf * C::N;
 #pragma unroll
           for (int ks = 0; ks < C::KSTEPS; ++ks) {
             const uint64_t ad = umma_smem_desc<C::ROWB>(a_base + ks * 32);
@@ -262,7 +285,7 @@ __global__ void __launch_bounds__(320, 1)
     const int row = lq * 32 + lane;          // key row of the tile (TMEM lane)
     GatherCursor gc;                         // gather: job -> (query, pair)
     int jq = 0;
-    if constexpr (MODE == IDX_GATHER) gc.init(a.kept, a.keep, q0, nq);
+    if constexpr (MODE == IDX_GATHER) gc.init(sKept, C::KEEPMAX, 0, nq);
     for (int j = team; j < njobs; j += 2) {
       if constexpr (MODE == IDX_GATHER) {
         while (jq < j) {
@@ -271,9 +294,7 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       const int ql = gc.ql, pair = gc.pair;
-      const int buf = j & 1, ub = j >> 1;
-      if (!mbar_wait(&tfull[buf], ub & 1, wc, 5)) break;
-      tc_fence_after();
+      const int buf = j % C::NBUF, ub = j / C::NBUF;    // buffer buf is always drained by team buf % 2
       int tile, g;
       if constexpr (MODE == IDX_PREFILL) {
         tile = j / geff;
@@ -282,14 +303,14 @@ __global__ void __launch_bounds__(320, 1)
         tile = j;
         g = (MODE == IDX_GATHER) ? ql : 0;
       }
-      // key of this thread
+      // key of this thread; its scale is loaded before waiting for the
+      // accumulator so the global-load latency hides behind the MMA
       int s;
       bool kvalid;
       int col;
       if constexpr (MODE == IDX_GATHER) {
         const int slot = 2 * pair + (row >> 6);
-        const int* kr = a.kept + (long long)(q0 + ql) * a.keep;
-        const int blk = (slot < a.keep) ? kr[slot] : -1;
+        const int blk = sKept[ql * C::KEEPMAX + slot];
         s = blk * 64 + (row & 63);
         kvalid = blk >= 0;
         col = pair * 128 + row;
@@ -304,11 +325,19 @@ __global__ void __launch_bounds__(320, 1)
       }
       float sk = 1.f;
       if (a.k_scale != nullptr && kvalid) sk = a.k_scale[(long long)seq * a.n_k * (MODE == IDX_DECODE) + s];
+      if (!mbar_wait(&tfull[buf], ub & 1, wc, 5)) break;
+      tc_fence_after();
 
-      float acc[C::QS];
+      // sum_h w'[h] * ReLU(acc[h]) in NP independent partial sums per query
+      // (a single running sum would be a dependent FMA chain of H links)
+      constexpr int NPMAX = (C::QS > 1) ? 4 : 8;
+      constexpr int NP = (H / 4 < NPMAX) ? H / 4 : NPMAX;
+      float acc[C::QS][NP];
 #pragma unroll
-      for (int qq = 0; qq < C::QS; ++qq) acc[qq] = 0.f;
-      const uint32_t t_addr = tmem_base + (uint32_t(lq * 32) << 16) + buf * 256;
+      for (int qq = 0; qq < C::QS; ++qq)
+#pragma unroll
+        for (int p = 0; p < NP; ++p) acc[qq][p] = 0.f;
+      const uint32_t t_addr = tmem_base + (uint32_t(lq * 32) << 16) + buf * C::N;
       const float* wrow = sW + g * C::N;
 #pragma unroll
       for (int c = 0; c < C::N / 32; ++c) {
@@ -324,11 +353,15 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
           const float4 w4 = *reinterpret_cast<const float4*>(wrow + c * 32 + e4 * 4);
-          const int qq = (c * 32 + e4 * 4) / H;
-          acc[qq] = fmaf(w4.x, fmaxf(v[e4 * 4 + 0], 0.f), acc[qq]);
-          acc[qq] = fmaf(w4.y, fmaxf(v[e4 * 4 + 1], 0.f), acc[qq]);
-          acc[qq] = fmaf(w4.z, fmaxf(v[e4 * 4 + 2], 0.f), acc[qq]);
-          acc[qq] = fmaf(w4.w, fmaxf(v[e4 * 4 + 3], 0.f), acc[qq]);
+          const int col0 = c * 32 + e4 * 4;
+          const int qq = col0 / H;
+          const int p = ((col0 % H) / 4) % NP;
+          float a4 = acc[qq][p];
+          a4 = fmaf(w4.x, fmaxf(v[e4 * 4 + 0], 0.f), a4);
+          a4 = fmaf(w4.y, fmaxf(v[e4 * 4 + 1], 0.f), a4);
+          a4 = fmaf(w4.z, fmaxf(v[e4 * 4 + 2], 0.f), a4);
+          a4 = fmaf(w4.w, fmaxf(v[e4 * 4 + 3], 0.f), a4);
+          acc[qq][p] = a4;
         }
       }
       // outputs
@@ -347,7 +380,10 @@ __global__ void __launch_bounds__(320, 1)
           vis = kvalid;
         else
           vis = kvalid && s <= vis_limit(t, a);
-        const float score = vis ? acc[qq] * sk : -__int_as_float(0x7f800000);
+        float sum = 0.f;
+#pragma unroll
+        for (int p = 0; p < NP; ++p) sum += acc[qq][p];
+        const float score = vis ? sum * sk : -__int_as_float(0x7f800000);
         if constexpr (MODE == IDX_GATHER) {
           a.out[(long long)t * a.ld + col] = score;
         } else {

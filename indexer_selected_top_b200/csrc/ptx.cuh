@@ -59,7 +59,7 @@ struct WaitCtx {
   long long budget;               // cycles
 };
 
-__device__ __noinline__ void record_timeout(const WaitCtx& w, uint32_t site) {
+static __device__ __noinline__ void record_timeout(const WaitCtx& w, uint32_t site) {
   *w.abort_flag = 1u;
   if (w.status != nullptr) {
     atomicCAS(w.status, 0u, 5u /* SA_ERR_TIMEOUT */);

@@ -5,6 +5,12 @@
 
 #include "sa_internal.h"
 
+// Tuning knob: select the two-stage candidates with one CTA per row (1) or
+// one warp per row (0).
+#ifndef SA_STAGE2_TOPK_CTA
+#define SA_STAGE2_TOPK_CTA 1
+#endif
+
 namespace sa {
 
 // ------------------------------------------------------------ tensor maps
@@ -272,7 +278,10 @@ sa_status sa_topk(const float* scores, int32_t n_q, int32_t n_k, int64_t ld, int
   if (n_q < 0 || n_k <= 0 || ld < n_k || q_pos0 < 0 || k <= 0) return SA_ERR_INVALID_ARGUMENT;
   if (n_q == 0) return SA_OK;
   if (scores == nullptr || idx == nullptr) return SA_ERR_INVALID_ARGUMENT;
-  return cuda_status(launch_topk_table(scores, n_q, n_k, ld, q_pos0, k, idx, 0, nullptr, 0, nullptr, stream));
+  cudaError_t e = launch_topk_rows_warp(scores, n_q, ld, n_k, q_pos0, nullptr, 0, k, idx, stream);
+  if (e == cudaErrorNotSupported)   // rows longer than a warp holds in shared memory
+    e = launch_topk_table(scores, n_q, n_k, ld, q_pos0, k, idx, 0, nullptr, 0, nullptr, stream);
+  return cuda_status(e);
 }
 
 sa_status sa_sparse_attn(const sa_attn_in* at, const int32_t* idx, int32_t k, void* out, float* lse, void* ws,
@@ -355,7 +364,9 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
       e = launch_indexer(IDX_PREFILL, in->n_heads, in->d_idx, in->dtype, ci.q, in->k, R, in->n_k, a, stream);
       if (e != cudaSuccess) return cuda_status(e);
       sm.mark(1, stream);
-      e = launch_topk_table(table, R, in->n_k, in->n_k, ci.q_pos0, o->k, idx, 0, nullptr, 0, nullptr, stream);
+      e = launch_topk_rows_warp(table, R, in->n_k, in->n_k, ci.q_pos0, nullptr, 0, o->k, idx, stream);
+      if (e == cudaErrorNotSupported)
+        e = launch_topk_table(table, R, in->n_k, in->n_k, ci.q_pos0, o->k, idx, 0, nullptr, 0, nullptr, stream);
       if (e != cudaSuccess) return cuda_status(e);
     } else {
       const uint8_t* blk = reinterpret_cast<const uint8_t*>(w + p.off_blk);
@@ -380,8 +391,10 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
         if (e != cudaSuccess) return cuda_status(e);
       }
       sm.mark(2, stream);
-      e = launch_block_select(bsc, R, p.nb, std::max(p.nb, 1), ci.q_pos0, o->block_size, o->keep_blocks, kept,
-                              stream);
+      e = launch_block_keep_warp(bsc, R, std::max(p.nb, 1), ci.q_pos0, o->block_size, o->keep_blocks, kept, stream);
+      if (e == cudaErrorNotSupported)   // more blocks than a warp keeps in shared memory
+        e = launch_block_select(bsc, R, p.nb, std::max(p.nb, 1), ci.q_pos0, o->block_size, o->keep_blocks, kept,
+                                stream);
       if (e != cudaSuccess) return cuda_status(e);
       // stage 2: the visible keys of the kept blocks
       sm.mark(3, stream);
@@ -393,7 +406,11 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
       e = launch_indexer(IDX_GATHER, in->n_heads, in->d_idx, in->dtype, ci.q, in->k, R, in->n_k, a, stream);
       if (e != cudaSuccess) return cuda_status(e);
       sm.mark(4, stream);
+#if SA_STAGE2_TOPK_CTA
       e = launch_topk_table(cand, R, ncand, ncand, ci.q_pos0, o->k, idx, 2, kept, o->keep_blocks, nullptr, stream);
+#else
+      e = launch_topk_rows_warp(cand, R, ncand, ncand, 0, kept, o->keep_blocks, o->k, idx, stream);
+#endif
       if (e != cudaSuccess) return cuda_status(e);
     }
     const void* qa = static_cast<const char*>(at->q) + (size_t)r0 * at->n_q_heads * at->head_dim * 2;
@@ -401,7 +418,7 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
     float* la = lse ? lse + (size_t)r0 * at->n_q_heads : nullptr;
     sm.mark(n_stages - 1, stream);
     e = launch_attention(qa, at->k_cache, at->v_cache, idx, R, o->k, at->n_k, at->n_q_heads, at->head_dim, scale, 0,
-                         oa, la, nullptr, nullptr, 1, stream);
+                         oa, la, nullptr, nullptr, 1, stream, status);
     if (e != cudaSuccess) return cuda_status(e);
     sm.mark(n_stages, stream);
   }
@@ -441,7 +458,7 @@ sa_status sa_decode(const sa_indexer_in* in, const sa_attn_in* at, const sa_deco
   sm.mark(2, stream);
   e = launch_attention(at->q, at->k_cache, at->v_cache, idx, in->batch, o->k, at->n_k, at->n_q_heads, at->head_dim,
                        attn_scale(at), in->batch, out, lse, reinterpret_cast<float*>(w + p.off_po),
-                       reinterpret_cast<float*>(w + p.off_pl), p.splits, stream);
+                       reinterpret_cast<float*>(w + p.off_pl), p.splits, stream, status);
   if (e != cudaSuccess) return cuda_status(e);
   sm.mark(3, stream);
   return sm.ok ? SA_OK : SA_ERR_INVALID_ARGUMENT;

@@ -41,12 +41,19 @@ cudaError_t launch_topk_table(const float* scores, int n_rows, int n_cols, long 
 cudaError_t launch_block_select(const float* bscores, int n_q, int nb, long long ld, int q_pos0, int block,
                                 int keep, int* kept, cudaStream_t st);
 
+cudaError_t launch_topk_rows_warp(const float* scores, int n_rows, long long ld, int n_cols, int q_pos0,
+                                  const int* kept, int keep, int k, int32_t* idx, cudaStream_t st);
+
+cudaError_t launch_block_keep_warp(const float* bscores, int n_q, long long ld, int q_pos0, int block, int keep,
+                                   int* kept, cudaStream_t st);
+
 cudaError_t launch_pool_blocks(const uint8_t* k, const float* k_scale, int n_blocks, int block,
                                uint8_t* blk, float* blk_scale, cudaStream_t st);
 
 cudaError_t launch_attention(const void* q, const void* kc, const void* vc, const int32_t* idx, int n_q, int k,
                              int n_k, int hq, int dh, float scale, int batch, void* out, float* lse,
-                             float* part_o, float* part_lse, int splits, cudaStream_t st);
+                             float* part_o, float* part_lse, int splits, cudaStream_t st,
+                             uint32_t* status = nullptr);
 
 cudaError_t launch_fill_upper(float* scores, int n_q, int n_k, long long ld, int q_pos0, cudaStream_t st);
 
