@@ -155,7 +155,18 @@ typedef struct {
   int32_t test_hook;     /* 0 in production; see SA_HOOK_* */
   cudaEvent_t* stage_events;  /* host array, nullable (see above) */
   int32_t n_stage_events;
+  int32_t flat_path;     /* FLAT mode: SA_FLAT_AUTO, SA_FLAT_TABLE or SA_FLAT_STREAM */
 } sa_prefill_opts;
+
+/* FLAT prefill paths. TABLE writes each chunk's score table and selects its
+ * rows; STREAM never writes the table: a sampled threshold per row, the
+ * indexer's epilogue appends the keys at or above it to the row's candidate
+ * list (capacity 4k), an exact select ranks the list, and rows whose list
+ * missed are re-selected from their whole row. AUTO takes TABLE while the
+ * keys number at most 65536, STREAM beyond. */
+#define SA_FLAT_AUTO 0
+#define SA_FLAT_TABLE 1
+#define SA_FLAT_STREAM 2
 
 typedef struct {
   int32_t k;

@@ -53,7 +53,12 @@ class AttnIn(ctypes.Structure):
 class PrefillOpts(ctypes.Structure):
     _fields_ = [("k", ctypes.c_int32), ("mode", ctypes.c_int), ("block_size", ctypes.c_int32),
                 ("keep_blocks", ctypes.c_int32), ("chunk_rows", ctypes.c_int32), ("status", ctypes.c_void_p),
-                ("test_hook", ctypes.c_int32), ("stage_events", ctypes.c_void_p), ("n_stage_events", ctypes.c_int32)]
+                ("test_hook", ctypes.c_int32), ("stage_events", ctypes.c_void_p), ("n_stage_events", ctypes.c_int32),
+                ("flat_path", ctypes.c_int32)]
+
+
+SA_FLAT_AUTO, SA_FLAT_TABLE, SA_FLAT_STREAM = 0, 1, 2
+FLAT_PATHS = {"auto": SA_FLAT_AUTO, "table": SA_FLAT_TABLE, "stream": SA_FLAT_STREAM}
 
 
 class DecodeOpts(ctypes.Structure):
@@ -225,14 +230,15 @@ class Prefill:
 
     def __init__(self, q, q_scale, k, k_scale, w, Q, K, V, k_top: int, mode: str = "flat", block_size=64,
                  keep_blocks=64, chunk_rows=0, q_pos0=0, softmax_scale=0.0, want_idx=True, want_lse=True,
-                 status=None, test_hook=0, timer: "StageTimer" = None):
+                 status=None, test_hook=0, timer: "StageTimer" = None, flat_path: str = "auto"):
         self.ind = indexer_in(q, q_scale, k, k_scale, w, q_pos0)
         self.att = attn_in(Q, K, V, softmax_scale)
         self.opts = PrefillOpts(k=k_top, mode=SA_MODE_TWO_STAGE if mode == "two_stage" else SA_MODE_FLAT,
                                 block_size=block_size, keep_blocks=keep_blocks, chunk_rows=chunk_rows,
                                 status=_ptr(status), test_hook=test_hook,
                                 stage_events=timer.ptr if timer else None,
-                                n_stage_events=len(timer.events) if timer else 0)
+                                n_stage_events=len(timer.events) if timer else 0,
+                                flat_path=FLAT_PATHS[flat_path])
         self.timer = timer
         self.nws = workspace_size(SA_OP_PREFILL, self.ind, self.att, self.opts)
         self.ws = _workspace(self.nws, Q.device)

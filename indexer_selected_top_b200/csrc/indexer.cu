@@ -55,7 +55,8 @@ struct IdxCfg {
   static constexpr int NS = (MODE == IDX_DECODE) ? 8 : SA_IDX_STAGES;    // key-tile stages
   static constexpr int KSTEPS = ROWB / 32;                   // 32-byte K slices per MMA
   static constexpr int KEEPMAX = 64;                          // gather: kept blocks per query
-  static constexpr int KEPT_BYTES = (MODE == IDX_GATHER) ? NQ * KEEPMAX * 4 : 0;
+  // gather: kept lists; other modes: the rows' thetas (candidate mode); 16-byte multiple
+  static constexpr int KEPT_BYTES = (MODE == IDX_GATHER) ? NQ * KEEPMAX * 4 : (NQ * 4 + 15) / 16 * 16;
   static constexpr int SMEM_USED =
       1024 + QBYTES + NS * KBYTES + NQ * H * 4 + KEPT_BYTES + (2 * NS + 1 + 2 * NBUF) * 8 + 16;
   // at least 120 KB: one CTA per SM, so two CTAs never contend for TMEM
@@ -65,7 +66,7 @@ struct IdxCfg {
 };
 
 __device__ __forceinline__ int vis_limit(int t, const IdxArgs& a) {
-  const int p = a.q_pos0 + t;
+  const int p = a.row_pos ? a.row_pos[t] : a.q_pos0 + t;
   return (a.div == 1) ? (p - a.off) : (p / a.div - a.off);
 }
 
@@ -109,6 +110,7 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sK = sQ + C::QBYTES;
   float* sW = reinterpret_cast<float*>(sK + C::NS * C::KBYTES);
   int* sKept = reinterpret_cast<int*>(sW + C::NQ * H);         // gather: [NQ][KEEPMAX], -1 padded
+  float* sTheta = reinterpret_cast<float*>(sKept);            // candidate mode: theta of the CTA's rows
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sKept) + C::KEPT_BYTES);
   uint64_t* kfull = bars;
   uint64_t* kempty = bars + C::NS;
@@ -167,6 +169,10 @@ __global__ void __launch_bounds__(320, 1)
       v = a.w[r] * (a.q_scale ? a.q_scale[r] : 1.f);
     }
     sW[i] = v;
+  }
+  if constexpr (MODE == IDX_PREFILL) {
+    if (a.cand != nullptr)
+      for (int i = threadIdx.x; i < C::NQ; i += blockDim.x) sTheta[i] = (i < nq) ? a.theta[q0 + i] : 0.f;
   }
   if constexpr (MODE == IDX_GATHER) {
     // the CTA's kept-block lists, staged once: every role walks them per job
@@ -283,48 +289,62 @@ __global__ void __launch_bounds__(320, 1)
     const int team = (warp - 2) >> 2;
     const int lq = warp & 3;                 // TMEM lane quarter this warp may access
     const int row = lq * 32 + lane;          // key row of the tile (TMEM lane)
-    GatherCursor gc;                         // gather: job -> (query, pair)
+    // job -> (tile, sub-tile / query, this thread's key, its scale); the scale
+    // of the team's next job is loaded one job ahead so its global-load
+    // latency hides behind the current job
+    struct JobKey {
+      int tile, g, ql, pair, s, col;
+      bool kvalid;
+      float sk;
+    };
+    GatherCursor gc;                         // gather: cursor at the job being loaded
     int jq = 0;
     if constexpr (MODE == IDX_GATHER) gc.init(sKept, C::KEEPMAX, 0, nq);
-    for (int j = team; j < njobs; j += 2) {
+    auto job_key = [&](int jj) {
+      JobKey k;
       if constexpr (MODE == IDX_GATHER) {
-        while (jq < j) {
+        while (jq < jj) {
           gc.next();
           ++jq;
         }
       }
-      const int ql = gc.ql, pair = gc.pair;
-      const int buf = j % C::NBUF, ub = j / C::NBUF;    // buffer buf is always drained by team buf % 2
-      int tile, g;
+      k.ql = gc.ql;
+      k.pair = gc.pair;
       if constexpr (MODE == IDX_PREFILL) {
-        tile = j / geff;
-        g = j % geff;
+        k.tile = jj / geff;
+        k.g = jj % geff;
       } else {
-        tile = j;
-        g = (MODE == IDX_GATHER) ? ql : 0;
+        k.tile = jj;
+        k.g = (MODE == IDX_GATHER) ? k.ql : 0;
       }
-      // key of this thread; its scale is loaded before waiting for the
-      // accumulator so the global-load latency hides behind the MMA
-      int s;
-      bool kvalid;
-      int col;
       if constexpr (MODE == IDX_GATHER) {
-        const int slot = 2 * pair + (row >> 6);
-        const int blk = sKept[ql * C::KEEPMAX + slot];
-        s = blk * 64 + (row & 63);
-        kvalid = blk >= 0;
-        col = pair * 128 + row;
+        const int slot = 2 * k.pair + (row >> 6);
+        const int blk = (k.ql < nq) ? sKept[k.ql * C::KEEPMAX + slot] : -1;
+        k.s = blk * 64 + (row & 63);
+        k.kvalid = blk >= 0;
+        k.col = k.pair * 128 + row;
       } else if constexpr (MODE == IDX_DECODE) {
-        s = (tile0 + tile) * 128 + row;
-        kvalid = s < seq_len;
-        col = s;
+        k.s = (tile0 + k.tile) * 128 + row;
+        k.kvalid = k.s < seq_len;
+        k.col = k.s;
       } else {
-        s = tile * 128 + row;
-        kvalid = s < a.n_k;
-        col = s;
+        k.s = k.tile * 128 + row;
+        k.kvalid = k.s < a.n_k;
+        k.col = k.s;
       }
-      float sk = 1.f;
-      if (a.k_scale != nullptr && kvalid) sk = a.k_scale[(long long)seq * a.n_k * (MODE == IDX_DECODE) + s];
+      k.sk = 1.f;
+      if (jj < njobs && a.k_scale != nullptr && k.kvalid)
+        k.sk = a.k_scale[(long long)seq * a.n_k * (MODE == IDX_DECODE) + k.s];
+      return k;
+    };
+    JobKey nxt = job_key(team);
+    for (int j = team; j < njobs; j += 2) {
+      const JobKey cur = nxt;
+      nxt = job_key(j + 2);
+      const int ql = cur.ql, g = cur.g, s = cur.s, col = cur.col;
+      const bool kvalid = cur.kvalid;
+      const float sk = cur.sk;
+      const int buf = j % C::NBUF, ub = j / C::NBUF;    // buffer buf is always drained by team buf % 2
       if (!mbar_wait(&tfull[buf], ub & 1, wc, 5)) break;
       tc_fence_after();
 
@@ -332,6 +352,7 @@ __global__ void __launch_bounds__(320, 1)
       // (a single running sum would be a dependent FMA chain of H links)
       constexpr int NPMAX = (C::QS > 1) ? 4 : 8;
       constexpr int NP = (H / 4 < NPMAX) ? H / 4 : NPMAX;
+      constexpr int NCH = C::N / 32;
       float acc[C::QS][NP];
 #pragma unroll
       for (int qq = 0; qq < C::QS; ++qq)
@@ -339,17 +360,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int p = 0; p < NP; ++p) acc[qq][p] = 0.f;
       const uint32_t t_addr = tmem_base + (uint32_t(lq * 32) << 16) + buf * C::N;
       const float* wrow = sW + g * C::N;
-#pragma unroll
-      for (int c = 0; c < C::N / 32; ++c) {
-        float v[32];
-        tmem_ld32(t_addr + c * 32, v);
-        tmem_ld_wait();
-        if (c == C::N / 32 - 1) {
-          // all columns are in registers: hand the accumulator back to the MMA
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[buf]);
-        }
+      auto consume = [&](const float (&v)[32], int c) {
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
           const float4 w4 = *reinterpret_cast<const float4*>(wrow + c * 32 + e4 * 4);
@@ -362,6 +373,34 @@ __global__ void __launch_bounds__(320, 1)
           a4 = fmaf(w4.z, fmaxf(v[e4 * 4 + 2], 0.f), a4);
           a4 = fmaf(w4.w, fmaxf(v[e4 * 4 + 3], 0.f), a4);
           acc[qq][p] = a4;
+        }
+      };
+      auto release = [&]() {   // every column of this accumulator is in registers
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf]);
+      };
+      // double-buffered TMEM loads: chunk c + 1 is in flight while chunk c is
+      // consumed (one wait::ld covers it)
+      float va[32], vb[32];
+      tmem_ld32(t_addr, va);
+      tmem_ld_wait();
+      tmem_regs_ready(va);
+#pragma unroll
+      for (int c = 0; c < NCH; c += 2) {
+        if (c + 1 < NCH) tmem_ld32(t_addr + (c + 1) * 32, vb);
+        if (c + 1 >= NCH) release();
+        consume(va, c);
+        if (c + 1 < NCH) {
+          tmem_ld_wait();
+          tmem_regs_ready(vb);
+          if (c + 2 < NCH) tmem_ld32(t_addr + (c + 2) * 32, va);
+          if (c + 2 >= NCH) release();
+          consume(vb, c + 1);
+          if (c + 2 < NCH) {
+            tmem_ld_wait();
+            tmem_regs_ready(va);
+          }
         }
       }
       // outputs
@@ -384,6 +423,26 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int p = 0; p < NP; ++p) sum += acc[qq][p];
         const float score = vis ? sum * sk : -__int_as_float(0x7f800000);
+        if constexpr (MODE == IDX_PREFILL) {
+          if (a.cand != nullptr) {
+            // candidate mode: warp-aggregated append of keys at or above theta
+            const bool take = vis && score >= sTheta[t - q0];
+            const unsigned bal = __ballot_sync(0xffffffffu, take);
+            if (bal != 0u) {
+              int base = 0;
+              if (lane == 0) base = atomicAdd(&a.cand_cnt[t], __popc(bal));
+              base = __shfl_sync(0xffffffffu, base, 0);
+              const int pos = base + __popc(bal & ((1u << lane) - 1u));
+              if (take && pos < a.cap) {
+                uint32_t b = __float_as_uint(score);
+                if (b == 0x80000000u) b = 0u;
+                const uint32_t key = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+                a.cand[(long long)t * a.cap + pos] = ((unsigned long long)key << 32) | (uint32_t)(~(uint32_t)s);
+              }
+            }
+            continue;
+          }
+        }
         if constexpr (MODE == IDX_GATHER) {
           a.out[(long long)t * a.ld + col] = score;
         } else {

@@ -176,6 +176,16 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// After tmem_ld_wait: marks the loaded registers as (re)defined here, so no
+// use of them can be scheduled above the wait.
+__device__ __forceinline__ void tmem_regs_ready(float (&v)[32]) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+  for (int i = 0; i < 32; i += 8)
+    asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]),
+                 "+r"(r[i + 6]), "+r"(r[i + 7]));
+}
+
 // --------------------------------------------------------- UMMA descriptors
 // Shared-memory matrix descriptor (sm_100 "version 1"), K-major operand laid
 // out by TMA with a 128-byte (rows of 128 B) or 64-byte (rows of 64 B) swizzle:

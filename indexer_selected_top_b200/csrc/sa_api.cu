@@ -104,8 +104,23 @@ static int decode_splits(int k) { return std::max(1, (k + kDecodeSplitKeys - 1) 
 struct PrefillPlan {
   int R;           // rows per chunk
   int nb;          // two-stage: complete blocks
+  bool stream;     // FLAT without a score table
+  int m, n_s, cap, fb;   // stream: sample stride and count, list capacity, fallback rows per batch
   size_t off_table, off_idx, off_blk, off_blks, off_bsc, off_kept, off_cand, total;
+  size_t off_ks, off_kss, off_stab, off_theta, off_cnt, off_list, off_miss, off_rows, off_count, off_pos;
+  size_t off_fq, off_fqs, off_fw, off_ftab;
 };
+
+constexpr int kStreamSamples = 16384;      // sampled keys per row for the threshold (at most)
+constexpr float kStreamGamma = 2.0f;       // target list length = gamma * k
+constexpr int kTableMaxKeys = 65536;       // FLAT auto: table path up to this many keys
+
+static bool flat_streams(const sa_indexer_in* in, const sa_prefill_opts* o) {
+  if (o->mode != SA_MODE_FLAT) return false;
+  if (o->flat_path == SA_FLAT_STREAM) return true;
+  if (o->flat_path == SA_FLAT_TABLE) return false;
+  return in->n_k > kTableMaxKeys;
+}
 
 static bool plan_prefill(const sa_indexer_in* in, const sa_prefill_opts* o, PrefillPlan* p) {
   const long long nq = std::max(in->n_q, 1);
@@ -113,7 +128,45 @@ static bool plan_prefill(const sa_indexer_in* in, const sa_prefill_opts* o, Pref
   R = (int)std::min<long long>(R, nq);
   std::memset(p, 0, sizeof(*p));
   size_t off = 0;
-  if (o->mode == SA_MODE_FLAT) {
+  if (o->mode == SA_MODE_FLAT && flat_streams(in, o)) {
+    p->stream = true;
+    p->m = std::max(1, (in->n_k + kStreamSamples - 1) / kStreamSamples);
+    p->n_s = (in->n_k + p->m - 1) / p->m;
+    p->cap = (4 * o->k + 63) / 64 * 64;
+    if (o->chunk_rows <= 0) R = std::min(R, 16384);
+    while (R > 1 && ((long long)R * p->n_s * 4ll > (2ll << 30) || (long long)R * p->cap * 8ll > (2ll << 30)))
+      R = (R + 1) / 2;
+    p->fb = (int)std::max<long long>(1, std::min<long long>(R, (1ll << 30) / ((long long)in->n_k * 4)));
+    const size_t qrow = (size_t)in->n_heads * in->d_idx * (in->dtype == SA_FP8_E4M3 ? 1 : 2);
+    p->off_ks = off;
+    off += align256((size_t)p->n_s * in->d_idx * (in->dtype == SA_FP8_E4M3 ? 1 : 2));
+    p->off_kss = off;
+    off += align256((size_t)p->n_s * 4);
+    p->off_stab = off;
+    off += align256((size_t)R * p->n_s * 4);
+    p->off_theta = off;
+    off += align256((size_t)R * 4);
+    p->off_cnt = off;
+    off += align256((size_t)R * 4);
+    p->off_list = off;
+    off += align256((size_t)R * p->cap * 8);
+    p->off_miss = off;
+    off += align256((size_t)R * 4);
+    p->off_rows = off;
+    off += align256((size_t)R * 4);
+    p->off_count = off;
+    off += 256;
+    p->off_pos = off;
+    off += align256((size_t)R * 4);
+    p->off_fq = off;
+    off += align256((size_t)p->fb * qrow);
+    p->off_fqs = off;
+    off += align256((size_t)p->fb * in->n_heads * 4);
+    p->off_fw = off;
+    off += align256((size_t)p->fb * in->n_heads * 4);
+    p->off_ftab = off;
+    off += align256((size_t)p->fb * in->n_k * 4);
+  } else if (o->mode == SA_MODE_FLAT) {
     // score table of one chunk; shrink the chunk so the table stays <= 4 GiB
     while (R > 1 && (long long)R * in->n_k * 4ll > (4ll << 30)) R = (R + 1) / 2;
     p->off_table = off;
@@ -198,6 +251,100 @@ struct StageMarks {
     }
   }
 };
+
+// Streaming FLAT selection of one chunk (rows ci->q_pos0 ...): sampled
+// thresholds, the appending scan, the exact list select, then the whole-row
+// fallback for the rows whose list missed (one counter read on the host).
+static sa_status stream_select_chunk(const sa_indexer_in* in, const sa_indexer_in* ci, const sa_prefill_opts* o,
+                                     const PrefillPlan& p, char* w, bool first, int32_t* idx, uint32_t* status,
+                                     cudaStream_t stream) {
+  const int R = ci->n_q;
+  const size_t esz = esize(in->dtype);
+  const int krow = in->d_idx * (int)esz;
+  const int qrow = in->n_heads * in->d_idx * (int)esz;
+  uint8_t* ks = reinterpret_cast<uint8_t*>(w + p.off_ks);
+  float* kss = reinterpret_cast<float*>(w + p.off_kss);
+  float* stab = reinterpret_cast<float*>(w + p.off_stab);
+  float* theta = reinterpret_cast<float*>(w + p.off_theta);
+  int* cnt = reinterpret_cast<int*>(w + p.off_cnt);
+  auto* list = reinterpret_cast<unsigned long long*>(w + p.off_list);
+  int* miss = reinterpret_cast<int*>(w + p.off_miss);
+  int* rows = reinterpret_cast<int*>(w + p.off_rows);
+  int* count = reinterpret_cast<int*>(w + p.off_count);
+  int* pos = reinterpret_cast<int*>(w + p.off_pos);
+  cudaError_t e = cudaSuccess;
+  if (first) {   // the sample: every m-th key (and its scale)
+    e = launch_gather_rows(in->k, ks, nullptr, p.n_s, krow, p.m, krow, stream);
+    if (e == cudaSuccess && in->k_scale)
+      e = launch_gather_rows(in->k_scale, kss, nullptr, p.n_s, 4, p.m, 4, stream);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  // 1. sample scores: sample i (key m*i) is visible to row t iff m*i <= p
+  {
+    sa_indexer_in si = *ci;
+    si.n_k = p.n_s;
+    si.k = ks;
+    si.k_scale = in->k_scale ? kss : nullptr;
+    IdxArgs a = base_args(&si, status, o->test_hook);
+    a.div = p.m;
+    a.off = 0;
+    a.out = stab;
+    a.ld = p.n_s;
+    e = launch_indexer(IDX_PREFILL, in->n_heads, in->d_idx, in->dtype, ci->q, ks, R, p.n_s, a, stream);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  // 2. thresholds
+  e = launch_theta(stab, R, p.n_s, p.n_s, ci->q_pos0, p.m, in->n_k, o->k, p.cap, kStreamGamma, o->test_hook, theta,
+                   stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  // 3. the scan appends candidates
+  if (cudaMemsetAsync(cnt, 0, (size_t)R * 4, stream) != cudaSuccess) return SA_ERR_CUDA;
+  {
+    IdxArgs a = base_args(ci, status, o->test_hook);
+    a.theta = theta;
+    a.cand = list;
+    a.cand_cnt = cnt;
+    a.cap = p.cap;
+    e = launch_indexer(IDX_PREFILL, in->n_heads, in->d_idx, in->dtype, ci->q, in->k, R, in->n_k, a, stream);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  // 4. exact select of each list; flag the misses
+  e = launch_select_cand(list, cnt, theta, R, p.cap, ci->q_pos0, in->n_k, o->k, idx, miss, status, stream);
+  if (e == cudaSuccess) e = launch_compact_rows(miss, R, rows, count, ci->q_pos0, pos, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  int n_miss = 0;
+  if (cudaMemcpyAsync(&n_miss, count, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return SA_ERR_CUDA;
+  // 5. whole-row fallback of the missed rows, in batches
+  uint8_t* fq = reinterpret_cast<uint8_t*>(w + p.off_fq);
+  float* fqs = reinterpret_cast<float*>(w + p.off_fqs);
+  float* fw = reinterpret_cast<float*>(w + p.off_fw);
+  float* ftab = reinterpret_cast<float*>(w + p.off_ftab);
+  for (int b0 = 0; b0 < n_miss; b0 += p.fb) {
+    const int nb = std::min(p.fb, n_miss - b0);
+    e = launch_gather_rows(ci->q, fq, rows + b0, nb, qrow, 0, qrow, stream);
+    if (e == cudaSuccess && ci->q_scale)
+      e = launch_gather_rows(ci->q_scale, fqs, rows + b0, nb, in->n_heads * 4, 0, in->n_heads * 4, stream);
+    if (e == cudaSuccess) e = launch_gather_rows(ci->w, fw, rows + b0, nb, in->n_heads * 4, 0, in->n_heads * 4, stream);
+    if (e != cudaSuccess) return cuda_status(e);
+    sa_indexer_in fi = *ci;
+    fi.n_q = nb;
+    fi.q = fq;
+    fi.q_scale = ci->q_scale ? fqs : nullptr;
+    fi.w = fw;
+    IdxArgs a = base_args(&fi, status, o->test_hook);
+    a.row_pos = pos + b0;
+    a.out = ftab;
+    a.ld = in->n_k;
+    e = launch_indexer(IDX_PREFILL, in->n_heads, in->d_idx, in->dtype, fq, in->k, nb, in->n_k, a, stream);
+    if (e == cudaSuccess)
+      e = launch_topk_table(ftab, nb, in->n_k, in->n_k, 0, o->k, idx, 0, nullptr, 0, nullptr, stream, pos + b0,
+                            rows + b0);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  return SA_OK;
+}
 
 }  // namespace sa
 
@@ -355,7 +502,12 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
     ci.w = in->w + (size_t)r0 * in->n_heads;
     int32_t* idx = idx_out ? idx_out + (size_t)r0 * o->k : reinterpret_cast<int32_t*>(w + p.off_idx);
     sm.on = (r0 == 0);
-    if (o->mode == SA_MODE_FLAT) {
+    if (o->mode == SA_MODE_FLAT && p.stream) {
+      sm.mark(0, stream);
+      sa_status fs = stream_select_chunk(in, &ci, o, p, w, r0 == 0, idx, status, stream);
+      if (fs != SA_OK) return fs;
+      sm.mark(1, stream);
+    } else if (o->mode == SA_MODE_FLAT) {
       float* table = reinterpret_cast<float*>(w + p.off_table);
       IdxArgs a = base_args(&ci, status, o->test_hook);
       a.out = table;

@@ -4,7 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "../../include/sa.h"
+#include "sa.h"
 
 namespace sa {
 
@@ -28,6 +28,16 @@ struct IdxArgs {
   uint32_t* status;      // device [error, site] or null
   long long budget;      // wait budget in clock cycles
   int hook;
+  // prefill: absolute position of every query row (ascending), overriding
+  // q_pos0 + t when non-null
+  const int* row_pos;
+  // candidate mode (prefill): instead of writing the table, append every
+  // visible key with score >= theta[t] to row t's list as the packed key
+  // (order-preserving score bits << 32 | ~key); counts may exceed cap
+  const float* theta;
+  unsigned long long* cand;
+  int* cand_cnt;
+  int cap;
 };
 
 // Host launchers (return cudaError_t of the launch).
@@ -36,7 +46,18 @@ cudaError_t launch_indexer(int mode, int heads, int d, sa_dtype dt, const void* 
 
 cudaError_t launch_topk_table(const float* scores, int n_rows, int n_cols, long long ld, int q_pos0, int k,
                               int32_t* idx, int vis_mode, const int* kept, int keep, const int* seq_lens,
-                              cudaStream_t st);
+                              cudaStream_t st, const int* row_pos = nullptr, const int* out_rows = nullptr);
+
+// ---- streaming selector (stream.cu) ----
+cudaError_t launch_gather_rows(const void* src, void* dst, const int* rows, int n_rows, long long src_stride,
+                               int m_stride, int row_bytes, cudaStream_t st);
+cudaError_t launch_theta(const float* stab, int n_rows, int n_s, long long ld, int q_pos0, int m, int n_k, int k,
+                         int cap, float gamma, int hook, float* theta, cudaStream_t st);
+cudaError_t launch_select_cand(const unsigned long long* cand, const int* cnt, const float* theta, int n_rows,
+                               int cap, int q_pos0, int n_k, int k, int32_t* idx, int* miss_flag, uint32_t* status,
+                               cudaStream_t st);
+cudaError_t launch_compact_rows(const int* flags, int n_rows, int* rows, int* count, int q_pos0, int* pos,
+                                cudaStream_t st);
 
 cudaError_t launch_block_select(const float* bscores, int n_q, int nb, long long ld, int q_pos0, int block,
                                 int keep, int* kept, cudaStream_t st);

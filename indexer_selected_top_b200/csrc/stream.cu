@@ -1,0 +1,187 @@
+// stream.cu -- the streaming exact selector: top-k without a score table.
+//
+// Latent Sparse Attention appendix F.1 ("Selection by threshold", "Flat
+// prefill"): before the scan, set a threshold theta_t per query from a
+// sample of its row; the scan compares each score with theta_t once and
+// appends the keys at or above it to the query's list L_t as packed 64-bit
+// keys; only L_t is then ranked (radix select). When L_t holds every key
+// with score >= theta_t and at least k of them, the top-k is inside it. A
+// query the estimate misses -- fewer than k listed, or more than the list
+// holds -- falls back to its whole row (done here by the table path on the
+// missed rows only). HyScale's HyTopK also computes each query's exact top-k
+// on the fly without a full score table (theflow "related" page).
+//
+// theta_t: the sample holds every m-th key (key m*i); query t sees the
+// n_vs = min(n_s, p / m + 1) samples at positions <= p. To list about
+// gamma * k of its n_vis = p + 1 keys it takes the n_theta-th largest sample
+// score, n_theta = round(gamma * k * n_vs / n_vis). Rows whose visible keys
+// all fit in the list take theta = -inf.
+#include "radix.cuh"
+#include "sa_internal.h"
+
+namespace sa {
+
+// dst row i = src row rows[i] (or row i * m_stride when rows is null)
+__global__ void gather_rows_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, const int* rows,
+                                   long long src_stride, int m_stride, int row_bytes) {
+  const int i = blockIdx.x;
+  const long long r = rows ? (long long)rows[i] : (long long)i * m_stride;
+  const uint32_t* s = reinterpret_cast<const uint32_t*>(src + r * src_stride);
+  uint32_t* d = reinterpret_cast<uint32_t*>(dst + (long long)i * row_bytes);
+  for (int j = threadIdx.x; j < row_bytes / 4; j += blockDim.x) d[j] = s[j];
+}
+
+cudaError_t launch_gather_rows(const void* src, void* dst, const int* rows, int n_rows, long long src_stride,
+                               int m_stride, int row_bytes, cudaStream_t st) {
+  if (n_rows <= 0) return cudaSuccess;
+  if (row_bytes % 4 != 0) return cudaErrorInvalidValue;
+  gather_rows_kernel<<<n_rows, 128, 0, st>>>(static_cast<const uint8_t*>(src), static_cast<uint8_t*>(dst), rows,
+                                             src_stride, m_stride, row_bytes);
+  return cudaGetLastError();
+}
+
+static __device__ __forceinline__ float key_to_float(uint32_t key) {
+  const uint32_t b = (key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key;
+  return __uint_as_float(b);
+}
+
+// theta[t] for chunk row t (absolute position q_pos0 + t); stab row t holds
+// the scores of samples 0..n_s-1 (entries beyond the visible ones unused)
+__global__ void __launch_bounds__(TK_THREADS, 1)
+    theta_kernel(const float* __restrict__ stab, int n_s, long long ld, int q_pos0, int m, int n_k, int k, int cap,
+                 float gamma, int hook, float* __restrict__ theta) {
+  extern __shared__ uint8_t th_raw[];
+  TkShared& sh = *reinterpret_cast<TkShared*>(th_raw);
+  const int t = blockIdx.x, tid = threadIdx.x;
+  const int p = q_pos0 + t;
+  const int n_vis = min(n_k, p + 1);
+  float th;
+  if (hook == SA_HOOK_THETA_POS_INF) {
+    th = INFINITY;
+  } else if (hook == SA_HOOK_THETA_NEG_INF || n_vis <= cap) {
+    th = -INFINITY;
+  } else {
+    const int n_vs = min(n_s, p / m + 1);
+    const long long want = llrintf(gamma * (float)k * (float)n_vs / (float)n_vis);
+    int need = (int)max(1ll, min((long long)n_vs, want));
+    const float* row = stab + (long long)t * ld;
+    uint32_t prefix = 0;
+    int pbits = 0;
+    while (pbits < 32) {                    // 12 + 12 + 8 bits: the exact n_theta-th key
+      const int db = (pbits == 24) ? 8 : TK_HBITS;
+      const int nbins = 1 << db;
+      for (int b = tid; b < nbins; b += TK_THREADS) sh.hist[b] = 0;
+      __syncthreads();
+      const int sdig = 32 - pbits - db;
+      for (int j = tid; j < n_vs; j += TK_THREADS) {
+        const uint32_t key = score_key(row[j]);
+        if (pbits == 0 || (key >> (32 - pbits)) == prefix) atomicAdd(&sh.hist[(key >> sdig) & (nbins - 1)], 1u);
+      }
+      __syncthreads();
+      find_bucket(sh, nbins, need);
+      need -= sh.above;
+      prefix = (prefix << db) | (uint32_t)sh.bucket;
+      pbits += db;
+      __syncthreads();
+    }
+    th = key_to_float(prefix);
+  }
+  if (tid == 0) theta[t] = th;
+}
+
+cudaError_t launch_theta(const float* stab, int n_rows, int n_s, long long ld, int q_pos0, int m, int n_k, int k,
+                         int cap, float gamma, int hook, float* theta, cudaStream_t st) {
+  if (n_rows <= 0) return cudaSuccess;
+  const int smem = (int)sizeof(TkShared);
+  cudaError_t e = cudaFuncSetAttribute(theta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  theta_kernel<<<n_rows, TK_THREADS, smem, st>>>(stab, n_s, ld, q_pos0, m, n_k, k, cap, gamma, hook, theta);
+  return cudaGetLastError();
+}
+
+// Exact top-k of each row's candidate list; rows whose list missed (fewer
+// than min(k, visible) candidates, or more than cap) are flagged for the
+// whole-row fallback and their index rows left to it.
+__global__ void __launch_bounds__(TK_THREADS, 1)
+    select_cand_kernel(const unsigned long long* __restrict__ cand, const int* __restrict__ cnt, int cap,
+                       int q_pos0, int n_k, int k, int32_t* __restrict__ idx, int* __restrict__ miss,
+                       uint32_t* status) {
+  extern __shared__ uint8_t sc_raw[];
+  TkShared& sh = *reinterpret_cast<TkShared*>(sc_raw);
+  const int t = blockIdx.x, tid = threadIdx.x;
+  const int n_vis = min(n_k, q_pos0 + t + 1);
+  const int need = min(k, n_vis);
+  const int c = cnt[t];
+  const bool ok = c <= cap && c >= need;
+  if (tid == 0) {
+    miss[t] = ok ? 0 : 1;
+    if (status != nullptr) {
+      if (!ok) atomicAdd(status + 2, 1u);
+      if (c > cap) atomicAdd(status + 3, 1u);
+    }
+    sh.n_out = 0;
+  }
+  if (!ok) return;
+  const unsigned long long* row = cand + (long long)t * cap;
+  for (int j = tid; j < c; j += TK_THREADS) sh.cand[j] = row[j];
+  __syncthreads();
+  int32_t* out = idx + (long long)t * k;
+  smem_select64(sh, c, need, [&](uint64_t key) {
+    out[atomicAdd(&sh.n_out, 1)] = (int32_t)(~(uint32_t)(key & 0xFFFFFFFFu));
+  });
+  for (int j = need + tid; j < k; j += TK_THREADS) out[j] = -1;
+}
+
+cudaError_t launch_select_cand(const unsigned long long* cand, const int* cnt, const float* theta, int n_rows,
+                               int cap, int q_pos0, int n_k, int k, int32_t* idx, int* miss_flag, uint32_t* status,
+                               cudaStream_t st) {
+  (void)theta;
+  if (n_rows <= 0) return cudaSuccess;
+  if (cap > TK_CAP) return cudaErrorNotSupported;
+  const int smem = (int)sizeof(TkShared);
+  cudaError_t e = cudaFuncSetAttribute(select_cand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  select_cand_kernel<<<n_rows, TK_THREADS, smem, st>>>(cand, cnt, cap, q_pos0, n_k, k, idx, miss_flag, status);
+  return cudaGetLastError();
+}
+
+// Ordered compaction of the flagged rows: rows[] ascending, count[0], and
+// pos[i] = q_pos0 + rows[i] (their absolute positions). One CTA.
+__global__ void __launch_bounds__(1024) compact_rows_kernel(const int* __restrict__ flags, int n_rows,
+                                                            int* __restrict__ rows, int* __restrict__ count,
+                                                            int q_pos0, int* __restrict__ pos) {
+  __shared__ int red[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (n_rows + 1023) / 1024;
+  const int lo = min(n_rows, tid * per), hi = min(n_rows, lo + per);
+  int mine = 0;
+  for (int i = lo; i < hi; ++i) mine += flags[i] != 0;
+  int x = mine;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) red[warp] = x;
+  __syncthreads();
+  int base = 0, tot = 0;
+  for (int w = 0; w < 32; ++w) {
+    if (w < warp) base += red[w];
+    tot += red[w];
+  }
+  int o = base + x - mine;
+  for (int i = lo; i < hi; ++i)
+    if (flags[i] != 0) {
+      rows[o] = i;
+      pos[o] = q_pos0 + i;
+      ++o;
+    }
+  if (tid == 0) count[0] = tot;
+}
+
+cudaError_t launch_compact_rows(const int* flags, int n_rows, int* rows, int* count, int q_pos0, int* pos,
+                                cudaStream_t st) {
+  compact_rows_kernel<<<1, 1024, 0, st>>>(flags, n_rows, rows, count, q_pos0, pos);
+  return cudaGetLastError();
+}
+
+}  // namespace sa

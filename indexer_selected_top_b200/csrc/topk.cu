@@ -14,21 +14,10 @@
 // and gathers the bucket's (key, index) pairs, which a shared-memory radix
 // select over the packed 64-bit keys finishes. A bucket of identical scores
 // larger than shared memory is resolved by an ordered scan (lowest indices).
+#include "radix.cuh"
 #include "sa_internal.h"
 
 namespace sa {
-
-constexpr int TK_THREADS = 512;
-constexpr int TK_CAP = 12288;          // (key, index) pairs kept in shared memory
-constexpr int TK_HBITS = 12;
-constexpr int TK_HBINS = 1 << TK_HBITS;
-constexpr uint32_t KEY_NEG_INF = 0x007FFFFFu;   // score key of -inf
-
-__device__ __forceinline__ uint32_t score_key(float x) {
-  uint32_t b = __float_as_uint(x);
-  if (b == 0x80000000u) b = 0u;                    // -0 sorts with +0
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
 
 // Row description: column c of the row holds the score of key key_of(c);
 // only columns [0, ncols) exist; invalid columns are skipped.
@@ -40,114 +29,6 @@ struct RowView {
   __device__ __forceinline__ bool valid_key(uint32_t key) const { return vis_mode != 2 || key != KEY_NEG_INF; }
   __device__ __forceinline__ int key_of(int c) const { return vis_mode == 2 ? kept[c >> 6] * 64 + (c & 63) : c; }
 };
-
-struct TkShared {
-  uint32_t hist[TK_HBINS];
-  unsigned long long cand[TK_CAP];
-  int n_out;
-  int n_cand;
-  int bucket;
-  int above;
-  int total;
-  int red[TK_THREADS / 32];
-};
-
-// block-wide sum
-__device__ int block_sum(int v, int* red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  int r = 0;
-  for (int i = 0; i < TK_THREADS / 32; ++i) r += red[i];
-  __syncthreads();
-  return r;
-}
-
-// block-wide exclusive prefix sum (threads in order)
-__device__ int block_excl_scan(int v, int* red, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  __syncthreads();
-  if (lane == 31) red[warp] = x;
-  __syncthreads();
-  int base = 0, tot = 0;
-  for (int i = 0; i < TK_THREADS / 32; ++i) {
-    if (i < warp) base += red[i];
-    tot += red[i];
-  }
-  __syncthreads();
-  *total = tot;
-  return base + x - v;
-}
-
-// Find, in hist[0..nbins), the bucket b with sum(hist[b+1..]) < need <= sum(hist[b..]).
-// Sets sh.bucket and sh.above (count strictly above the bucket).
-__device__ void find_bucket(TkShared& sh, int nbins, int need) {
-  // each thread owns a contiguous range of bins (from the top)
-  const int per = (nbins + TK_THREADS - 1) / TK_THREADS;
-  const int hi = nbins - threadIdx.x * per;              // exclusive upper bin of this thread
-  const int lo = max(0, hi - per);
-  int mine = 0;
-  for (int b = lo; b < hi; ++b) mine += sh.hist[b];
-  int tot;
-  const int before = block_excl_scan(mine, sh.red, &tot);  // bins above this thread's range
-  if (before < need && before + mine >= need) {
-    int acc = before;
-    for (int b = hi - 1; b >= lo; --b) {
-      if (acc + (int)sh.hist[b] >= need) {
-        sh.bucket = b;
-        sh.above = acc;
-        break;
-      }
-      acc += sh.hist[b];
-    }
-  }
-  __syncthreads();
-}
-
-// Select the `need` largest of sh.cand[0..cnt) (unique 64-bit keys) and emit them.
-template <class Emit>
-__device__ void smem_select64(TkShared& sh, int cnt, int need, Emit emit) {
-  uint64_t hi = 0;
-  int nb = 0;
-  uint64_t cut = 0;
-  if (need >= cnt) {
-    cut = 0;
-  } else {
-    while (true) {
-      for (int b = threadIdx.x; b < 256; b += TK_THREADS) sh.hist[b] = 0;
-      __syncthreads();
-      const int sh_digit = 64 - nb - 8;
-      for (int j = threadIdx.x; j < cnt; j += TK_THREADS) {
-        const uint64_t key = sh.cand[j];
-        if (nb == 0 || (key >> (64 - nb)) == hi) atomicAdd(&sh.hist[(key >> sh_digit) & 255u], 1u);
-      }
-      __syncthreads();
-      find_bucket(sh, 256, need);
-      const int d = sh.bucket;
-      need -= sh.above;
-      hi = (hi << 8) | (uint64_t)d;
-      nb += 8;
-      const int inb = sh.hist[d];
-      __syncthreads();
-      if (inb == need || nb == 64) {
-        cut = hi << (64 - nb);
-        break;
-      }
-    }
-  }
-  for (int j = threadIdx.x; j < cnt; j += TK_THREADS) {
-    const uint64_t key = sh.cand[j];
-    if (key >= cut) emit(key);
-  }
-  __syncthreads();
-}
 
 __device__ void topk_row(TkShared& sh, const RowView& rv, int k, int32_t* out) {
   const int tid = threadIdx.x;
@@ -245,7 +126,8 @@ __device__ void topk_row(TkShared& sh, const RowView& rv, int k, int32_t* out) {
 
 __global__ void __launch_bounds__(TK_THREADS, 1)
     topk_table_kernel(const float* scores, int n_rows, int n_cols, long long ld, int q_pos0, int k, int32_t* idx,
-                      int vis_mode, const int* kept, int keep, const int* seq_lens) {
+                      int vis_mode, const int* kept, int keep, const int* seq_lens, const int* row_pos,
+                      const int* out_rows) {
   extern __shared__ uint8_t tk_raw[];
   TkShared& sh = *reinterpret_cast<TkShared*>(tk_raw);
   const int row = blockIdx.x;
@@ -254,7 +136,8 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
   rv.vis_mode = vis_mode;
   rv.kept = nullptr;
   if (vis_mode == 0) {
-    rv.ncols = max(0, min(n_cols, q_pos0 + row + 1));
+    rv.ncols = max(0, min(n_cols, (row_pos ? row_pos[row] : q_pos0 + row) + 1));
+    rv.vis_mode = 0;
   } else if (vis_mode == 1) {
     rv.ncols = seq_lens ? min(n_cols, seq_lens[row]) : n_cols;
   } else {
@@ -263,18 +146,18 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
     while (nb < keep && rv.kept[nb] >= 0) ++nb;
     rv.ncols = min(n_cols, nb * 64);
   }
-  topk_row(sh, rv, k, idx + (long long)row * k);
+  topk_row(sh, rv, k, idx + (long long)(out_rows ? out_rows[row] : row) * k);
 }
 
 cudaError_t launch_topk_table(const float* scores, int n_rows, int n_cols, long long ld, int q_pos0, int k,
                               int32_t* idx, int vis_mode, const int* kept, int keep, const int* seq_lens,
-                              cudaStream_t st) {
+                              cudaStream_t st, const int* row_pos, const int* out_rows) {
   if (n_rows <= 0) return cudaSuccess;
   const int smem = (int)sizeof(TkShared);
   cudaError_t e = cudaFuncSetAttribute(topk_table_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   topk_table_kernel<<<n_rows, TK_THREADS, smem, st>>>(scores, n_rows, n_cols, ld, q_pos0, k, idx, vis_mode, kept,
-                                                       keep, seq_lens);
+                                                       keep, seq_lens, row_pos, out_rows);
   return cudaGetLastError();
 }
 

@@ -149,12 +149,13 @@ def test_sparse_attn_decode_splits(sa):
 
 
 # ------------------------------------------------------------------ prefill
-def _check_prefill(sa, wl, seed, rows, mode="flat", k=None, keep=64, chunk_rows=0):
+def _check_prefill(sa, wl, seed, rows, mode="flat", k=None, keep=64, chunk_rows=0, flat_path="auto", hook=0,
+                   status=None, inp=None):
     k = k or wl.k
-    inp = PrefillInputs(wl, "cuda", seed=seed)
+    inp = inp or PrefillInputs(wl, "cuda", seed=seed)
     host = inp.to_host()
     pre = sa.Prefill(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, k, mode=mode,
-                     keep_blocks=keep, chunk_rows=chunk_rows)
+                     keep_blocks=keep, chunk_rows=chunk_rows, flat_path=flat_path, test_hook=hook, status=status)
     out, lse, idx = pre()
     torch.cuda.synchronize()
     out, lse, idx = out.float().cpu().numpy(), lse.cpu().numpy(), idx.cpu().numpy()
@@ -183,6 +184,33 @@ def test_prefill_flat_fp8_chunked(sa):
     wl = WORKLOADS["prefill_t16k"].with_(T=1300)
     rows = sample_rows(wl.T, 60, seed=2, k=300, extra=(499, 500, 501, 999, 1000))
     _check_prefill(sa, wl, 2, rows, k=300, chunk_rows=500)
+
+
+def test_prefill_flat_streaming_ragged(sa):
+    # no score table: sampled thresholds, appending scan, exact list select
+    wl = WORKLOADS["prefill_t16k"].with_(T=40000, k=256)
+    rows = sample_rows(wl.T, 96, seed=5, k=256, extra=(1023, 1024, 1025, 39999))
+    st = sa.new_status("cuda")
+    _check_prefill(sa, wl, 5, rows, k=256, flat_path="stream", chunk_rows=16000, status=st)
+    s = st.cpu().tolist()
+    assert s[0] == 0, s
+    assert s[2] <= 40, f"too many whole-row fallbacks: {s}"
+
+
+def test_prefill_flat_streaming_forced_fallbacks(sa):
+    # theta = +inf: every list misses low, every row takes the whole-row fallback
+    wl = WORKLOADS["prefill_t16k"].with_(T=3000, k=128)
+    rows = sample_rows(wl.T, 48, seed=6, k=128)
+    inp = PrefillInputs(wl, "cuda", seed=6)
+    st = sa.new_status("cuda")
+    _check_prefill(sa, wl, 6, rows, k=128, flat_path="stream", hook=sa.SA_HOOK_THETA_POS_INF, status=st, inp=inp)
+    assert st.cpu().tolist()[2] == wl.T
+    # theta = -inf: every key is listed; rows with more than 4k = 512 visible
+    # keys overflow their list and fall back
+    st = sa.new_status("cuda")
+    _check_prefill(sa, wl, 6, rows, k=128, flat_path="stream", hook=sa.SA_HOOK_THETA_NEG_INF, status=st, inp=inp)
+    s = st.cpu().tolist()
+    assert s[3] == wl.T - 512 and s[2] == wl.T - 512, s
 
 
 def _two_stage_kept_sets(sa, inp, k_all):
