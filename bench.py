@@ -111,6 +111,20 @@ def two_stage_work(wl):
     }
 
 
+def flat_work(wl, streaming: bool):
+    """Algorithmic counts of the flat prefill (every visible key scored)."""
+    T, H, d, k = wl.T, wl.H, wl.d, wl.k
+    scores = T * (T + 1) // 2                                    # sum over t of (t + 1)
+    pairs = sum(min(k, p + 1) for p in range(T))
+    return {
+        "indexer_flops": 2.0 * H * d * scores,
+        "attn_pairs": pairs,
+        "attn_bytes": pairs * 2 * wl.dh * 2,
+        # table path: the score table is read once by the selector (+ index rows written)
+        "topk_bytes": 0 if streaming else scores * 4 + T * k * 4,
+    }
+
+
 def decode_work(wd):
     B, L, d = wd.batch, wd.L, wd.d
     return {
@@ -220,8 +234,10 @@ def run_native(args, rank, world, local_rank):
     seed = args.seed + 1000 * rank
     inp = PrefillInputs(wl, dev, seed=seed)
     ptimer = sa.StageTimer(sa.PREFILL_STAGES[wl.mode])
+    # one chunk for the two-stage and table paths (stage events cover the whole step)
+    chunk = wl.T if (wl.mode == "two_stage" or wl.T <= 65536) else 0
     pre = sa.Prefill(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, wl.k, mode=wl.mode,
-                     keep_blocks=wl.keep_blocks, chunk_rows=wl.T, timer=ptimer)
+                     keep_blocks=wl.keep_blocks, chunk_rows=chunk, timer=ptimer)
     dec = None
     if not args.no_decode:
         dinp = DecodeInputs(wd, dev, seed=seed)
@@ -279,21 +295,19 @@ def run_native(args, rank, world, local_rank):
     # ---------------- roofline of the dominant prefill kernel ----------------
     peaks, peak_src = load_peaks()
     fp8_peak = 2.0 * peaks["bf16_tflops"]                # dense FP8 = 2 x measured bf16 (nominal ratio)
-    work = two_stage_work(wl)
+    work = two_stage_work(wl) if wl.mode == "two_stage" else flat_work(wl, wl.T > 65536)
     avg = {n: v / K for n, v in stage_ms.items()}
+    flop_stage = {"stage2_indexer": "stage2_flops", "stage1_indexer": "stage1_flops", "indexer": "indexer_flops"}
     stages = {}
     for n, ms in avg.items():
-        s = ms * 1e-3
-        if n == "stage2_indexer":
-            stages[n] = {"ms": round(ms, 4), "bound": "tensor", "achieved": work["stage2_flops"] / s / 1e12,
-                         "peak": fp8_peak, "unit": "TFLOP/s"}
-        elif n == "stage1_indexer":
-            stages[n] = {"ms": round(ms, 4), "bound": "tensor", "achieved": work["stage1_flops"] / s / 1e12,
+        s = max(ms, 1e-9) * 1e-3
+        if n in flop_stage:
+            stages[n] = {"ms": round(ms, 4), "bound": "tensor", "achieved": work[flop_stage[n]] / s / 1e12,
                          "peak": fp8_peak, "unit": "TFLOP/s"}
         elif n == "attention":
             stages[n] = {"ms": round(ms, 4), "bound": "hbm", "achieved": work["attn_bytes"] / s / 1e9,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s"}
-        elif n == "topk":
+        elif n == "topk" and work["topk_bytes"] > 0:
             stages[n] = {"ms": round(ms, 4), "bound": "hbm", "achieved": work["topk_bytes"] / s / 1e9,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s"}
         else:
@@ -368,7 +382,14 @@ def run_native(args, rank, world, local_rank):
                          f"{info['rows']} stratified rows ({info['rows_s']:.1f} s: both indexer stages, top-k, "
                          f"attention), extrapolated to {wl.T} rows"}
 
-    launches_per_step = 6 + (4 if dec is not None else 0)
+    if wl.mode == "two_stage":
+        pre_launches = 6                       # pool, stage 1, keep, stage 2, top-k, attention
+    elif wl.T <= 65536:
+        pre_launches = 3                       # indexer (table), top-k, attention
+    else:                                      # streaming: sample gathers once; per chunk sample scores,
+        n_chunks = -(-wl.T // 16384)           # thresholds, scan, list select, compaction, attention
+        pre_launches = 2 + 6 * n_chunks        # (+ 5 per fallback batch, normally none)
+    launches_per_step = pre_launches + (4 if dec is not None else 0)
     line = {
         "metric": METRIC,
         "value": round(world * K * wl.T / (pre_ms * 1e-3), 1),

@@ -11,10 +11,10 @@
 // (no cross-lane reduction). The scales factor out of the ReLU because they
 // are positive: ReLU(sq*sk*a) = sq*sk*ReLU(a).
 //
-// Roles (320 threads): warp 0 = TMA producer (one lane), warp 1 = MMA issuer
-// (one lane) and TMEM owner, warps 2..9 = two epilogue teams of 4 warps. The
-// 512 TMEM columns hold 512 / N fp32 accumulators (2 at N = 256, 8 at N = 64)
-// used as a ring; team b % 2 drains buffer b, so the epilogue of one
+// Roles: warp 0 = TMA producer (one lane), warp 1 = MMA issuer (one lane)
+// and TMEM owner, warps 2.. = TEAMS epilogue teams of 4 warps. The 512 TMEM
+// columns hold 512 / N fp32 accumulators (2 at N = 256, 8 at N = 64) used as
+// a ring; team b % TEAMS drains buffer b, so the epilogue of one
 // accumulator overlaps the MMAs into the others (the pages' bucket scan also
 // overlaps its epilogue with its products: appendix F.1, "Flat prefill").
 //
@@ -40,16 +40,31 @@ namespace sa {
 #ifndef SA_IDX_STAGES
 #define SA_IDX_STAGES 6
 #endif
+// epilogue teams of 4 warps (2 or 4) and the prefill MMA N (256 or 128); a
+// team count above 2 needs N <= 128 so every team owns an accumulator
+#ifndef SA_IDX_TEAMS
+#define SA_IDX_TEAMS 2
+#endif
+#ifndef SA_IDX_PREFILL_N
+#define SA_IDX_PREFILL_N 256
+#endif
+// epilogue math: 1 = (w/2) * (a + |a|) accumulated with packed f32x2 FMAs
+#ifndef SA_IDX_EPI_PACKED
+#define SA_IDX_EPI_PACKED 1
+#endif
 
 template <int H, int D, bool FP8, int MODE>
 struct IdxCfg {
   static constexpr int ESZ = FP8 ? 1 : 2;
   static constexpr int ROWB = D * ESZ;                       // bytes per index row
-  static constexpr int QS = (MODE == IDX_PREFILL) ? (256 / H) : 1;
+  static constexpr int QS = (MODE == IDX_PREFILL) ? (SA_IDX_PREFILL_N / H) : 1;
   static constexpr int N = QS * H;                           // MMA N
-  static constexpr int G = (MODE == IDX_PREFILL) ? 2 : 1;    // sub-tiles per CTA
+  static constexpr int G = (MODE == IDX_PREFILL) ? (QS * 2 < 8 ? 8 / QS : 2) : 1;    // sub-tiles per CTA
   static constexpr int NQ = (MODE == IDX_PREFILL) ? QS * G : (MODE == IDX_GATHER ? SA_IDX_GATHER_NQ : 1);
   static constexpr int NBUF = 512 / N;                       // TMEM accumulator buffers (fp32 columns)
+  static constexpr int TEAMS = SA_IDX_TEAMS;
+  static constexpr int THREADS = 64 + 128 * TEAMS;
+  static_assert(NBUF % TEAMS == 0, "every team owns whole accumulators");
   static constexpr int QBYTES = NQ * H * ROWB;
   static constexpr int KBYTES = 128 * ROWB;
   static constexpr int NS = (MODE == IDX_DECODE) ? 8 : SA_IDX_STAGES;    // key-tile stages
@@ -100,7 +115,7 @@ struct GatherCursor {
 };
 
 template <int H, int D, bool FP8, int MODE>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                    const IdxArgs a) {
   using C = IdxCfg<H, D, FP8, MODE>;
@@ -168,7 +183,7 @@ __global__ void __launch_bounds__(320, 1)
       const long long r = (long long)(q0 + ql) * H + h;
       v = a.w[r] * (a.q_scale ? a.q_scale[r] : 1.f);
     }
-    sW[i] = v;
+    sW[i] = SA_IDX_EPI_PACKED ? 0.5f * v : v;   // packed math sums (w / 2) * (a + |a|)
   }
   if constexpr (MODE == IDX_PREFILL) {
     if (a.cand != nullptr)
@@ -286,7 +301,7 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else {
     // ======================= epilogue teams =======================
-    const int team = (warp - 2) >> 2;
+    const int team = (warp - 2) >> 2;        // jobs j with j % TEAMS == team
     const int lq = warp & 3;                 // TMEM lane quarter this warp may access
     const int row = lq * 32 + lane;          // key row of the tile (TMEM lane)
     // job -> (tile, sub-tile / query, this thread's key, its scale); the scale
@@ -297,7 +312,7 @@ __global__ void __launch_bounds__(320, 1)
       bool kvalid;
       float sk;
     };
-    GatherCursor gc;                         // gather: cursor at the job being loaded
+    GatherCursor gc = {};                    // gather: cursor at the job being loaded
     int jq = 0;
     if constexpr (MODE == IDX_GATHER) gc.init(sKept, C::KEEPMAX, 0, nq);
     auto job_key = [&](int jj) {
@@ -338,13 +353,13 @@ __global__ void __launch_bounds__(320, 1)
       return k;
     };
     JobKey nxt = job_key(team);
-    for (int j = team; j < njobs; j += 2) {
+    for (int j = team; j < njobs; j += C::TEAMS) {
       const JobKey cur = nxt;
-      nxt = job_key(j + 2);
+      nxt = job_key(j + C::TEAMS);
       const int ql = cur.ql, g = cur.g, s = cur.s, col = cur.col;
       const bool kvalid = cur.kvalid;
       const float sk = cur.sk;
-      const int buf = j % C::NBUF, ub = j / C::NBUF;    // buffer buf is always drained by team buf % 2
+      const int buf = j % C::NBUF, ub = j / C::NBUF;    // buffer buf is always drained by team buf % TEAMS
       if (!mbar_wait(&tfull[buf], ub & 1, wc, 5)) break;
       tc_fence_after();
 
@@ -360,6 +375,30 @@ __global__ void __launch_bounds__(320, 1)
         for (int p = 0; p < NP; ++p) acc[qq][p] = 0.f;
       const uint32_t t_addr = tmem_base + (uint32_t(lq * 32) << 16) + buf * C::N;
       const float* wrow = sW + g * C::N;
+#if SA_IDX_EPI_PACKED
+      // w * ReLU(a) = (w / 2) * (a + |a|): a + |a| is exact (2a or +0) and one
+      // FADD; the halved weights sit in sW, pairs accumulate with f32x2 FMAs
+      float2 acc2[C::QS][NP];
+#pragma unroll
+      for (int qq = 0; qq < C::QS; ++qq)
+#pragma unroll
+        for (int p = 0; p < NP; ++p) acc2[qq][p] = make_float2(0.f, 0.f);
+      auto consume = [&](const float (&v)[32], int c) {
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 w4 = *reinterpret_cast<const float4*>(wrow + c * 32 + e4 * 4);
+          const int col0 = c * 32 + e4 * 4;
+          const int qq = col0 / H;
+          const int p = ((col0 % H) / 4) % NP;
+          const float2 r01 = make_float2(v[e4 * 4 + 0] + fabsf(v[e4 * 4 + 0]), v[e4 * 4 + 1] + fabsf(v[e4 * 4 + 1]));
+          const float2 r23 = make_float2(v[e4 * 4 + 2] + fabsf(v[e4 * 4 + 2]), v[e4 * 4 + 3] + fabsf(v[e4 * 4 + 3]));
+          float2 a2 = acc2[qq][p];
+          a2 = __ffma2_rn(make_float2(w4.x, w4.y), r01, a2);
+          a2 = __ffma2_rn(make_float2(w4.z, w4.w), r23, a2);
+          acc2[qq][p] = a2;
+        }
+      };
+#else
       auto consume = [&](const float (&v)[32], int c) {
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
@@ -375,6 +414,7 @@ __global__ void __launch_bounds__(320, 1)
           acc[qq][p] = a4;
         }
       };
+#endif
       auto release = [&]() {   // every column of this accumulator is in registers
         tc_fence_before();
         __syncwarp();
@@ -420,8 +460,13 @@ __global__ void __launch_bounds__(320, 1)
         else
           vis = kvalid && s <= vis_limit(t, a);
         float sum = 0.f;
+#if SA_IDX_EPI_PACKED
+#pragma unroll
+        for (int p = 0; p < NP; ++p) sum += acc2[qq][p].x + acc2[qq][p].y;
+#else
 #pragma unroll
         for (int p = 0; p < NP; ++p) sum += acc[qq][p];
+#endif
         const float score = vis ? sum * sk : -__int_as_float(0x7f800000);
         if constexpr (MODE == IDX_PREFILL) {
           if (a.cand != nullptr) {
@@ -482,7 +527,7 @@ static cudaError_t launch_t(const void* q, const void* k, int q_rows, long long 
   else
     grid = dim3((a.n_q + C::NQ - 1) / C::NQ);
   if (grid.x == 0 || grid.y == 0) return cudaSuccess;
-  kern<<<grid, 320, C::SMEM, st>>>(qm, km, a);
+  kern<<<grid, C::THREADS, C::SMEM, st>>>(qm, km, a);
   return cudaGetLastError();
 }
 

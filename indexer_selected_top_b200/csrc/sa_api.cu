@@ -5,12 +5,6 @@
 
 #include "sa_internal.h"
 
-// Tuning knob: select the two-stage candidates with one CTA per row (1) or
-// one warp per row (0).
-#ifndef SA_STAGE2_TOPK_CTA
-#define SA_STAGE2_TOPK_CTA 1
-#endif
-
 namespace sa {
 
 // ------------------------------------------------------------ tensor maps
@@ -425,8 +419,8 @@ sa_status sa_topk(const float* scores, int32_t n_q, int32_t n_k, int64_t ld, int
   if (n_q < 0 || n_k <= 0 || ld < n_k || q_pos0 < 0 || k <= 0) return SA_ERR_INVALID_ARGUMENT;
   if (n_q == 0) return SA_OK;
   if (scores == nullptr || idx == nullptr) return SA_ERR_INVALID_ARGUMENT;
-  cudaError_t e = launch_topk_rows_warp(scores, n_q, ld, n_k, q_pos0, nullptr, 0, k, idx, stream);
-  if (e == cudaErrorNotSupported)   // rows longer than a warp holds in shared memory
+  cudaError_t e = launch_topk_fast(scores, n_q, ld, n_k, q_pos0, nullptr, nullptr, 0, k, idx, stream);
+  if (e == cudaErrorNotSupported)   // rows longer than one CTA holds in registers
     e = launch_topk_table(scores, n_q, n_k, ld, q_pos0, k, idx, 0, nullptr, 0, nullptr, stream);
   return cuda_status(e);
 }
@@ -516,7 +510,7 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
       e = launch_indexer(IDX_PREFILL, in->n_heads, in->d_idx, in->dtype, ci.q, in->k, R, in->n_k, a, stream);
       if (e != cudaSuccess) return cuda_status(e);
       sm.mark(1, stream);
-      e = launch_topk_rows_warp(table, R, in->n_k, in->n_k, ci.q_pos0, nullptr, 0, o->k, idx, stream);
+      e = launch_topk_fast(table, R, in->n_k, in->n_k, ci.q_pos0, nullptr, nullptr, 0, o->k, idx, stream);
       if (e == cudaErrorNotSupported)
         e = launch_topk_table(table, R, in->n_k, in->n_k, ci.q_pos0, o->k, idx, 0, nullptr, 0, nullptr, stream);
       if (e != cudaSuccess) return cuda_status(e);
@@ -558,11 +552,9 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
       e = launch_indexer(IDX_GATHER, in->n_heads, in->d_idx, in->dtype, ci.q, in->k, R, in->n_k, a, stream);
       if (e != cudaSuccess) return cuda_status(e);
       sm.mark(4, stream);
-#if SA_STAGE2_TOPK_CTA
-      e = launch_topk_table(cand, R, ncand, ncand, ci.q_pos0, o->k, idx, 2, kept, o->keep_blocks, nullptr, stream);
-#else
-      e = launch_topk_rows_warp(cand, R, ncand, ncand, 0, kept, o->keep_blocks, o->k, idx, stream);
-#endif
+      e = launch_topk_fast(cand, R, ncand, ncand, 0, nullptr, kept, o->keep_blocks, o->k, idx, stream);
+      if (e == cudaErrorNotSupported)
+        e = launch_topk_table(cand, R, ncand, ncand, ci.q_pos0, o->k, idx, 2, kept, o->keep_blocks, nullptr, stream);
       if (e != cudaSuccess) return cuda_status(e);
     }
     const void* qa = static_cast<const char*>(at->q) + (size_t)r0 * at->n_q_heads * at->head_dim * 2;

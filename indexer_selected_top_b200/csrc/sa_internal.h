@@ -48,6 +48,9 @@ cudaError_t launch_topk_table(const float* scores, int n_rows, int n_cols, long 
                               int32_t* idx, int vis_mode, const int* kept, int keep, const int* seq_lens,
                               cudaStream_t st, const int* row_pos = nullptr, const int* out_rows = nullptr);
 
+cudaError_t launch_topk_fast(const float* scores, int n_rows, long long ld, int n_cols, int q_pos0, const int* row_pos,
+                             const int* kept, int keep, int k, int32_t* idx, cudaStream_t st);
+
 // ---- streaming selector (stream.cu) ----
 cudaError_t launch_gather_rows(const void* src, void* dst, const int* rows, int n_rows, long long src_stride,
                                int m_stride, int row_bytes, cudaStream_t st);
