@@ -41,6 +41,27 @@ def load_peaks():
     return PEAKS_FALLBACK, "fallback"
 
 
+# --------------------------------------------------------- multi-rank plumbing
+def rank_seed(base: int, rank: int) -> int:
+    """Every rank runs its own independent copy of the workload (weak scaling)."""
+    return base + 1000 * rank
+
+
+def reduce_max(values, device=None):
+    """Max over ranks of per-rank device-timed values (no-op on one rank)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def weak_scaling_value(world: int, steps: int, units_per_rank_step: int, max_ms: float) -> float:
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    return world * steps * units_per_rank_step / (max_ms * 1e-3)
+
+
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -231,7 +252,7 @@ def run_native(args, rank, world, local_rank):
     if args.T:
         wl = wl.with_(T=args.T)
     wd = WORKLOADS["decode_b64_l128k"]
-    seed = args.seed + 1000 * rank
+    seed = rank_seed(args.seed, rank)
     inp = PrefillInputs(wl, dev, seed=seed)
     ptimer = sa.StageTimer(sa.PREFILL_STAGES[wl.mode])
     # one chunk for the two-stage and table paths (stage events cover the whole step)
@@ -286,10 +307,7 @@ def run_native(args, rank, world, local_rank):
     clk = clocks.stop()
     pre_ms = sum(a.elapsed_time(b) for a, b, _ in recs)
     dec_ms = sum(b.elapsed_time(c) for _, b, c in recs)
-    tot = torch.tensor([pre_ms, dec_ms, pre_ms + dec_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
-    pre_ms, dec_ms, all_ms = (float(x) for x in tot.cpu())
+    pre_ms, dec_ms, all_ms = reduce_max([pre_ms, dec_ms, pre_ms + dec_ms], device=dev)
     K = args.steps
 
     # ---------------- roofline of the dominant prefill kernel ----------------
@@ -366,10 +384,8 @@ def run_native(args, rank, world, local_rank):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        t_e2e = torch.tensor([a.elapsed_time(b) / ne], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
-        e2e = {"value": round(world * wl.T / (float(t_e2e) * 1e-3), 1), "unit": "tokens/s",
+        t_e2e = reduce_max([a.elapsed_time(b) / ne], device=dev)[0]
+        e2e = {"value": round(weak_scaling_value(world, 1, wl.T, t_e2e), 1), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ne}
 
     # ---------------- CPU oracle baseline (rank 0, N = 1) ----------------
@@ -392,7 +408,7 @@ def run_native(args, rank, world, local_rank):
     launches_per_step = pre_launches + (4 if dec is not None else 0)
     line = {
         "metric": METRIC,
-        "value": round(world * K * wl.T / (pre_ms * 1e-3), 1),
+        "value": round(weak_scaling_value(world, K, wl.T, pre_ms), 1),
         "unit": "tokens/s",
         "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": round(all_ms / K, 4),

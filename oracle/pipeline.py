@@ -17,14 +17,16 @@ from .two_stage import block_scores_row, keep_blocks_row, pool_block_keys, two_s
 
 
 def prefill_rows(host, rows, k: int, mode: str = "flat", block: int = 64, keep: int = 64,
-                 pos0: int = 0, scale=None, attention: bool = True, blocks=None):
+                 pos0: int = 0, scale=None, attention: bool = True, blocks=None, positions=None):
     """Oracle results for the given query rows of a prefill input.
 
     Per row: idx (int64 [k], -1 padded), cand (candidate key indices), scores
     (fp32 scores of the candidates, same order), and for two-stage kept
     (kept blocks) and bscores (block scores of blocks [0, cur)); O / lse
     (fp64 attention over idx) unless attention=False. ``blocks`` may carry
-    precomputed (bytes, scale) block keys."""
+    precomputed (bytes, scale) block keys. ``positions`` (same length as
+    rows) gives each row's absolute position when the host tensors hold only
+    the sampled query rows (default pos0 + t)."""
     ii = IndexerInputs(host)
     n_k = ii.kv.shape[0]
     K = as_numpy(host["K"]) if attention else None
@@ -35,9 +37,9 @@ def prefill_rows(host, rows, k: int, mode: str = "flat", block: int = 64, keep: 
         blk_vals = e4m3_decode(blocks[0])
         blk_scale = blocks[1].astype(np.float64)
     out = {}
-    for t in rows:
+    for i, t in enumerate(rows):
         t = int(t)
-        p = pos0 + t
+        p = pos0 + t if positions is None else int(positions[i])
         n_vis = min(n_k, p + 1)
         r = {}
         q_t = dequant(ii.q[t])

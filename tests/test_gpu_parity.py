@@ -332,3 +332,29 @@ def test_full_two_stage_t64k_sampled(sa):
 def test_full_decode_b64_l128k(sa):
     wl = WORKLOADS["decode_b64_l128k"]
     _check_decode(sa, wl, 0)
+
+
+def test_full_prefill_t1m_streaming_sampled(sa):
+    # 2^20 tokens: FLAT prefill without a score table; 256 stratified rows
+    # checked against the oracle (host copies of the sampled query rows only)
+    wl = WORKLOADS["prefill_t1m"]
+    inp = PrefillInputs(wl, "cuda", seed=0)
+    st = sa.new_status("cuda")
+    out, lse, idx = sa.Prefill(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, wl.k,
+                               status=st, want_lse=True)()
+    torch.cuda.synchronize()
+    s = st.cpu().tolist()
+    assert s[0] == 0, s
+    rows = sample_rows(wl.T, 256, seed=12, k=wl.k, extra=(8191, 8192, 16383, 16384))
+    r_t = torch.as_tensor(rows, device="cuda")
+    host = {"q_idx": inp.q_idx[r_t].cpu(), "q_scale": inp.q_scale[r_t].cpu(), "w": inp.w[r_t].cpu(),
+            "Q": inp.Q[r_t].cpu(), "k_idx": inp.k_idx.cpu(), "k_scale": inp.k_scale.cpu(),
+            "K": inp.K.cpu(), "V": inp.V.cpu()}
+    ref = oracle.prefill_rows(host, range(len(rows)), wl.k, attention=False, positions=rows)
+    gi = idx[r_t].cpu().numpy()
+    go, gl = out[r_t].float().cpu().numpy(), lse[r_t].cpu().numpy()
+    att = attention_rows(host, {i: gi[i] for i in range(len(rows))})
+    for i, t in enumerate(rows):
+        check_topk_row(gi[i], ref[i]["cand"], ref[i]["scores"], wl.k, f"row {t}")
+        check_attention_row(go[i], att[i][0], gl[i], att[i][1], f"row {t}")
+    assert s[2] <= wl.T // 1000, f"whole-row fallbacks: {s}"
