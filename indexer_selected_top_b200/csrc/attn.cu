@@ -326,25 +326,24 @@ __global__ void __launch_bounds__(AT_WARPS * 32)
   }
 }
 
+// merge of the splits: one CTA per (sequence, head), one thread per column
 template <int HQ, int DH>
-__global__ void attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse, int n_q,
-                                    int splits, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
-  const int t = blockIdx.x;
-  for (int e = threadIdx.x; e < HQ * DH; e += blockDim.x) {
-    const int h = e / DH, col = e % DH;
-    float M = -INFINITY;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, part_lse[((long long)t * splits + s) * HQ + h]);
-    float L = 0.f, acc = 0.f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < splits; ++s) {
-        const float f = __expf(part_lse[((long long)t * splits + s) * HQ + h] - M);
-        L += f;
-        acc += f * part_o[(((long long)t * splits + s) * HQ + h) * DH + col];
-      }
+__global__ void __launch_bounds__(DH) attn_combine_kernel(const float* __restrict__ part_o,
+                                                          const float* __restrict__ part_lse, int n_q, int splits,
+                                                          __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  const int t = blockIdx.x / HQ, h = blockIdx.x % HQ, col = threadIdx.x;
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, part_lse[((long long)t * splits + s) * HQ + h]);
+  float L = 0.f, acc = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < splits; ++s) {
+      const float f = __expf(part_lse[((long long)t * splits + s) * HQ + h] - M);
+      L += f;
+      acc += f * part_o[(((long long)t * splits + s) * HQ + h) * DH + col];
     }
-    out[((long long)t * HQ + h) * DH + col] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
-    if (lse != nullptr && col == 0) lse[(long long)t * HQ + h] = (L > 0.f) ? M + logf(L) : -INFINITY;
   }
+  out[((long long)t * HQ + h) * DH + col] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+  if (lse != nullptr && col == 0) lse[(long long)t * HQ + h] = (L > 0.f) ? M + logf(L) : -INFINITY;
 }
 
 template <int HQ, int DH>
@@ -365,7 +364,7 @@ static cudaError_t launch_attn_t(const void* q, const void* kc, const void* vc, 
       batch, (__nv_bfloat16*)out, lse, part_o, part_lse, splits, status);
   e = cudaGetLastError();
   if (e != cudaSuccess || splits == 1) return e;
-  attn_combine_kernel<HQ, DH><<<n_q, 256, 0, st>>>(part_o, part_lse, n_q, splits, (__nv_bfloat16*)out, lse);
+  attn_combine_kernel<HQ, DH><<<n_q * HQ, DH, 0, st>>>(part_o, part_lse, n_q, splits, (__nv_bfloat16*)out, lse);
   return cudaGetLastError();
 }
 

@@ -60,7 +60,7 @@ extern "C" sa_status sa_sparse_attn_decode_noalloc(const sa_attn_in* at, const i
   if (!(at->head_dim == 64 || at->head_dim == 128) || !(at->n_q_heads == 16 || at->n_q_heads == 8))
     return SA_ERR_UNSUPPORTED;
   if (!(at->softmax_scale >= 0.f) || at->softmax_scale > 3.0e38f) return SA_ERR_INVALID_ARGUMENT;
-  // same split as sa_sparse_attn: one split per 256 selected keys
+  // one split per 256 selected keys (the fixed array is sized for that)
   const int splits = (k + 255) / 256;
   const size_t n_part = (size_t)at->batch * splits * at->n_q_heads * at->head_dim;
   const size_t n_lse = (size_t)at->batch * splits * at->n_q_heads;

@@ -89,7 +89,8 @@ static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 constexpr long long kWaitBudget = 4000000000ll;     // ~2 s of SM clock
 constexpr long long kHookBudget = 20000000ll;       // ~10 ms: the stall hook
 constexpr int kDecodeSplitKeys = 256;               // keys per decode attention split
-constexpr int kDecodeTilesPerCta = 16;              // 2048 keys per decode indexer CTA
+constexpr int kDecodeTilesPerCta = 64;              // 8192 keys per decode indexer CTA
+constexpr int kDecodeSamples = 8192;                // sampled scores per sequence for the decode threshold
 constexpr int kMaxBlocks = 16384;                   // two-stage: blocks per sequence
 
 static int decode_splits(int k) { return std::max(1, (k + kDecodeSplitKeys - 1) / kDecodeSplitKeys); }
@@ -188,16 +189,27 @@ static bool plan_prefill(const sa_indexer_in* in, const sa_prefill_opts* o, Pref
 
 struct DecodePlan {
   size_t off_scores, off_idx, off_po, off_pl, total;
-  int splits;
+  size_t off_theta, off_cnt, off_list, off_miss;
+  int splits, cap, m;
 };
 
 static void plan_decode(const sa_indexer_in* in, const sa_attn_in* at, int k, DecodePlan* p) {
   size_t off = 0;
   p->splits = decode_splits(k);
+  p->cap = (4 * k + 63) / 64 * 64;
+  p->m = std::max(1, (in->n_k + kDecodeSamples - 1) / kDecodeSamples);
   p->off_scores = off;
   off += align256((size_t)in->batch * in->n_k * 4);
   p->off_idx = off;
   off += align256((size_t)in->batch * k * 4);
+  p->off_theta = off;
+  off += align256((size_t)in->batch * 4);
+  p->off_cnt = off;
+  off += align256((size_t)in->batch * 4);
+  p->off_list = off;
+  off += align256((size_t)in->batch * p->cap * 8);
+  p->off_miss = off;
+  off += align256((size_t)in->batch * 4);
   p->off_po = off;
   off += align256((size_t)in->batch * p->splits * at->n_q_heads * at->head_dim * 4);
   p->off_pl = off;
@@ -596,9 +608,29 @@ sa_status sa_decode(const sa_indexer_in* in, const sa_attn_in* at, const sa_deco
   cudaError_t e = launch_indexer(IDX_DECODE, in->n_heads, in->d_idx, in->dtype, in->q, in->k, in->batch,
                                  (long long)in->batch * in->n_k, a, stream);
   if (e != cudaSuccess) return cuda_status(e);
+  // selection from the written rows (LSA appendix F.1, "Flat decode"): a
+  // threshold from every m-th score, the scores at or above it listed, the
+  // lists ranked exactly; a sequence whose list missed is re-selected from
+  // its whole written row (device-side, no host synchronisation)
   sm.mark(1, stream);
-  e = launch_topk_table(rows, in->batch, in->n_k, in->n_k, 0, o->k, idx, 1, nullptr, 0, in->seq_lens, stream);
-  if (e != cudaSuccess) return cuda_status(e);
+  {
+    float* theta = reinterpret_cast<float*>(w + p.off_theta);
+    int* cnt = reinterpret_cast<int*>(w + p.off_cnt);
+    auto* list = reinterpret_cast<unsigned long long*>(w + p.off_list);
+    int* miss = reinterpret_cast<int*>(w + p.off_miss);
+    e = launch_theta(rows, in->batch, 0, in->n_k, 0, p.m, in->n_k, o->k, p.cap, kStreamGamma, o->test_hook, theta,
+                     stream, 1, in->seq_lens);
+    if (e == cudaSuccess && cudaMemsetAsync(cnt, 0, (size_t)in->batch * 4, stream) != cudaSuccess) e = cudaErrorUnknown;
+    if (e == cudaSuccess)
+      e = launch_collect_cand(rows, in->batch, in->n_k, in->n_k, in->seq_lens, theta, list, cnt, p.cap, stream);
+    if (e == cudaSuccess)
+      e = launch_select_cand(list, cnt, theta, in->batch, p.cap, 0, in->n_k, o->k, idx, miss, status, stream, 1,
+                             in->seq_lens);
+    if (e == cudaSuccess)
+      e = launch_topk_table(rows, in->batch, in->n_k, in->n_k, 0, o->k, idx, 1, nullptr, 0, in->seq_lens, stream,
+                            nullptr, nullptr, miss);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
   sm.mark(2, stream);
   e = launch_attention(at->q, at->k_cache, at->v_cache, idx, in->batch, o->k, at->n_k, at->n_q_heads, at->head_dim,
                        attn_scale(at), in->batch, out, lse, reinterpret_cast<float*>(w + p.off_po),

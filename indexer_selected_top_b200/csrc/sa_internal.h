@@ -46,7 +46,8 @@ cudaError_t launch_indexer(int mode, int heads, int d, sa_dtype dt, const void* 
 
 cudaError_t launch_topk_table(const float* scores, int n_rows, int n_cols, long long ld, int q_pos0, int k,
                               int32_t* idx, int vis_mode, const int* kept, int keep, const int* seq_lens,
-                              cudaStream_t st, const int* row_pos = nullptr, const int* out_rows = nullptr);
+                              cudaStream_t st, const int* row_pos = nullptr, const int* out_rows = nullptr,
+                              const int* only_flagged = nullptr);
 
 cudaError_t launch_topk_fast(const float* scores, int n_rows, long long ld, int n_cols, int q_pos0, const int* row_pos,
                              const int* kept, int keep, int k, int32_t* idx, cudaStream_t st);
@@ -55,10 +56,13 @@ cudaError_t launch_topk_fast(const float* scores, int n_rows, long long ld, int 
 cudaError_t launch_gather_rows(const void* src, void* dst, const int* rows, int n_rows, long long src_stride,
                                int m_stride, int row_bytes, cudaStream_t st);
 cudaError_t launch_theta(const float* stab, int n_rows, int n_s, long long ld, int q_pos0, int m, int n_k, int k,
-                         int cap, float gamma, int hook, float* theta, cudaStream_t st);
+                         int cap, float gamma, int hook, float* theta, cudaStream_t st, int decode = 0,
+                         const int* seq_lens = nullptr);
 cudaError_t launch_select_cand(const unsigned long long* cand, const int* cnt, const float* theta, int n_rows,
                                int cap, int q_pos0, int n_k, int k, int32_t* idx, int* miss_flag, uint32_t* status,
-                               cudaStream_t st);
+                               cudaStream_t st, int decode = 0, const int* seq_lens = nullptr);
+cudaError_t launch_collect_cand(const float* rows, int batch, long long ld, int n_k, const int* seq_lens,
+                                const float* theta, unsigned long long* cand, int* cnt, int cap, cudaStream_t st);
 cudaError_t launch_compact_rows(const int* flags, int n_rows, int* rows, int* count, int q_pos0, int* pos,
                                 cudaStream_t st);
 

@@ -47,21 +47,24 @@ static __device__ __forceinline__ float key_to_float(uint32_t key) {
 
 // theta[t] for chunk row t (absolute position q_pos0 + t); stab row t holds
 // the scores of samples 0..n_s-1 (entries beyond the visible ones unused)
+// Decode (decode != 0): row t is sequence t's written score row; its samples
+// are every m-th visible score (n_vis = seq_lens[t], or n_k).
 __global__ void __launch_bounds__(TK_THREADS, 1)
     theta_kernel(const float* __restrict__ stab, int n_s, long long ld, int q_pos0, int m, int n_k, int k, int cap,
-                 float gamma, int hook, float* __restrict__ theta) {
+                 float gamma, int hook, float* __restrict__ theta, int decode, const int* seq_lens) {
   extern __shared__ uint8_t th_raw[];
   TkShared& sh = *reinterpret_cast<TkShared*>(th_raw);
   const int t = blockIdx.x, tid = threadIdx.x;
-  const int p = q_pos0 + t;
+  const int p = decode ? ((seq_lens ? min(seq_lens[t], n_k) : n_k) - 1) : q_pos0 + t;
   const int n_vis = min(n_k, p + 1);
+  const int sstride = decode ? m : 1;
   float th;
   if (hook == SA_HOOK_THETA_POS_INF) {
     th = INFINITY;
   } else if (hook == SA_HOOK_THETA_NEG_INF || n_vis <= cap) {
     th = -INFINITY;
   } else {
-    const int n_vs = min(n_s, p / m + 1);
+    const int n_vs = decode ? (n_vis + m - 1) / m : min(n_s, p / m + 1);
     const long long want = llrintf(gamma * (float)k * (float)n_vs / (float)n_vis);
     int need = (int)max(1ll, min((long long)n_vs, want));
     const float* row = stab + (long long)t * ld;
@@ -74,7 +77,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
       __syncthreads();
       const int sdig = 32 - pbits - db;
       for (int j = tid; j < n_vs; j += TK_THREADS) {
-        const uint32_t key = score_key(row[j]);
+        const uint32_t key = score_key(row[(long long)j * sstride]);
         if (pbits == 0 || (key >> (32 - pbits)) == prefix) atomicAdd(&sh.hist[(key >> sdig) & (nbins - 1)], 1u);
       }
       __syncthreads();
@@ -90,12 +93,14 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
 }
 
 cudaError_t launch_theta(const float* stab, int n_rows, int n_s, long long ld, int q_pos0, int m, int n_k, int k,
-                         int cap, float gamma, int hook, float* theta, cudaStream_t st) {
+                         int cap, float gamma, int hook, float* theta, cudaStream_t st, int decode,
+                         const int* seq_lens) {
   if (n_rows <= 0) return cudaSuccess;
   const int smem = (int)sizeof(TkShared);
   cudaError_t e = cudaFuncSetAttribute(theta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  theta_kernel<<<n_rows, TK_THREADS, smem, st>>>(stab, n_s, ld, q_pos0, m, n_k, k, cap, gamma, hook, theta);
+  theta_kernel<<<n_rows, TK_THREADS, smem, st>>>(stab, n_s, ld, q_pos0, m, n_k, k, cap, gamma, hook, theta, decode,
+                                                 seq_lens);
   return cudaGetLastError();
 }
 
@@ -105,11 +110,11 @@ cudaError_t launch_theta(const float* stab, int n_rows, int n_s, long long ld, i
 __global__ void __launch_bounds__(TK_THREADS, 1)
     select_cand_kernel(const unsigned long long* __restrict__ cand, const int* __restrict__ cnt, int cap,
                        int q_pos0, int n_k, int k, int32_t* __restrict__ idx, int* __restrict__ miss,
-                       uint32_t* status) {
+                       uint32_t* status, int decode, const int* seq_lens) {
   extern __shared__ uint8_t sc_raw[];
   TkShared& sh = *reinterpret_cast<TkShared*>(sc_raw);
   const int t = blockIdx.x, tid = threadIdx.x;
-  const int n_vis = min(n_k, q_pos0 + t + 1);
+  const int n_vis = decode ? (seq_lens ? min(seq_lens[t], n_k) : n_k) : min(n_k, q_pos0 + t + 1);
   const int need = min(k, n_vis);
   const int c = cnt[t];
   const bool ok = c <= cap && c >= need;
@@ -134,14 +139,56 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
 
 cudaError_t launch_select_cand(const unsigned long long* cand, const int* cnt, const float* theta, int n_rows,
                                int cap, int q_pos0, int n_k, int k, int32_t* idx, int* miss_flag, uint32_t* status,
-                               cudaStream_t st) {
+                               cudaStream_t st, int decode, const int* seq_lens) {
   (void)theta;
   if (n_rows <= 0) return cudaSuccess;
   if (cap > TK_CAP) return cudaErrorNotSupported;
   const int smem = (int)sizeof(TkShared);
   cudaError_t e = cudaFuncSetAttribute(select_cand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  select_cand_kernel<<<n_rows, TK_THREADS, smem, st>>>(cand, cnt, cap, q_pos0, n_k, k, idx, miss_flag, status);
+  select_cand_kernel<<<n_rows, TK_THREADS, smem, st>>>(cand, cnt, cap, q_pos0, n_k, k, idx, miss_flag, status,
+                                                       decode, seq_lens);
+  return cudaGetLastError();
+}
+
+// Decode lists from the written score rows: every visible score >= theta[b]
+// of sequence b is appended to b's list, packed as in the indexer's candidate
+// mode. Grid: (row chunks of COLLECT_CHUNK scores, sequences). A CTA gathers
+// its hits in shared memory and reserves their place in the list with one
+// global atomic (a global atomic per warp contends on the 64 counters).
+constexpr int COLLECT_CHUNK = 4096;
+
+__global__ void __launch_bounds__(256)
+    collect_cand_kernel(const float* __restrict__ rows, long long ld, int n_k, const int* __restrict__ seq_lens,
+                        const float* __restrict__ theta, unsigned long long* __restrict__ cand, int* __restrict__ cnt,
+                        int cap) {
+  __shared__ unsigned long long hits[COLLECT_CHUNK];
+  __shared__ int n_hit, base;
+  const int b = blockIdx.y;
+  const int n_vis = seq_lens ? min(seq_lens[b], n_k) : n_k;
+  const float th = theta[b];
+  const float* row = rows + (long long)b * ld;
+  const int lo = blockIdx.x * COLLECT_CHUNK, hi = min(n_vis, lo + COLLECT_CHUNK);
+  if (threadIdx.x == 0) n_hit = 0;
+  __syncthreads();
+  for (int s = lo + threadIdx.x; s < hi; s += 256) {
+    const float sc = row[s];
+    if (sc >= th) hits[atomicAdd(&n_hit, 1)] = ((unsigned long long)score_key(sc) << 32) | (uint32_t)(~(uint32_t)s);
+  }
+  __syncthreads();
+  const int n = n_hit;
+  if (n == 0) return;
+  if (threadIdx.x == 0) base = atomicAdd(&cnt[b], n);
+  __syncthreads();
+  for (int j = threadIdx.x; j < n; j += 256)
+    if (base + j < cap) cand[(long long)b * cap + base + j] = hits[j];
+}
+
+cudaError_t launch_collect_cand(const float* rows, int batch, long long ld, int n_k, const int* seq_lens,
+                                const float* theta, unsigned long long* cand, int* cnt, int cap, cudaStream_t st) {
+  if (batch <= 0) return cudaSuccess;
+  const int chunks = (n_k + COLLECT_CHUNK - 1) / COLLECT_CHUNK;
+  collect_cand_kernel<<<dim3(chunks, batch), 256, 0, st>>>(rows, ld, n_k, seq_lens, theta, cand, cnt, cap);
   return cudaGetLastError();
 }
 

@@ -280,13 +280,14 @@ def test_prefill_two_stage_equals_flat_below_64_blocks(sa):
 
 
 # ------------------------------------------------------------------- decode
-def _check_decode(sa, wl, seed, seqs=None, seq_lens=None, k=None):
+def _check_decode(sa, wl, seed, seqs=None, seq_lens=None, k=None, hook=0, status=None):
     k = k or wl.k
     inp = DecodeInputs(wl, "cuda", seed=seed)
     if seq_lens is not None:
         inp.seq_lens = torch.tensor(seq_lens, dtype=torch.int32, device="cuda")
     host = inp.to_host()
-    dec = sa.Decode(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, inp.seq_lens, k)
+    dec = sa.Decode(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, inp.seq_lens, k,
+                    test_hook=hook, status=status)
     out, lse, idx = dec()
     torch.cuda.synchronize()
     out, lse, idx = out.float().cpu().numpy(), lse.cpu().numpy(), idx.cpu().numpy()
@@ -301,6 +302,20 @@ def _check_decode(sa, wl, seed, seqs=None, seq_lens=None, k=None):
 def test_decode_ragged_lengths(sa):
     wl = WORKLOADS["decode_b64_l128k"].with_(batch=4, L=5000)
     _check_decode(sa, wl, 0, seq_lens=[5000, 4097, 130, 2048], k=512)
+
+
+def test_decode_forced_fallbacks(sa):
+    # theta = +inf: every list is empty, every sequence falls back to its row;
+    # theta = -inf: every visible score is listed and the 3000-key rows
+    # overflow their 4k = 512 list, then fall back
+    wl = WORKLOADS["decode_b64_l128k"].with_(batch=3, L=3000)
+    st = sa.new_status("cuda")
+    _check_decode(sa, wl, 1, k=128, hook=sa.SA_HOOK_THETA_POS_INF, status=st)
+    assert st.cpu().tolist()[2] == 3
+    st = sa.new_status("cuda")
+    _check_decode(sa, wl, 1, k=128, hook=sa.SA_HOOK_THETA_NEG_INF, status=st)
+    s = st.cpu().tolist()
+    assert s[2] == 3 and s[3] == 3, s
 
 
 def test_decode_equals_prefill_last_row(sa):
