@@ -176,11 +176,14 @@ typedef struct {
   int32_t n_stage_events;
 } sa_decode_opts;
 
-/* test hooks: force the threshold of the streaming selector */
+/* test hooks: force the threshold of the streaming selector, a stalled wait,
+ * or the per-query schedule of the grouped prefill attention */
 #define SA_HOOK_NONE 0
 #define SA_HOOK_THETA_POS_INF 1   /* every row misses low -> whole-row fallback */
 #define SA_HOOK_THETA_NEG_INF 2   /* every key is a candidate -> overflow path */
 #define SA_HOOK_STALL_WAIT 3      /* a device wait that never completes -> SA_ERR_TIMEOUT */
+#define SA_HOOK_ATTN_UNGROUPED 4  /* prefill attention takes one query at a time, as for a group whose union of
+                                     selected keys does not fit the kernel's tables */
 
 /* Human-readable name of a status code (host, static storage). */
 const char* sa_status_string(sa_status s);

@@ -1,0 +1,561 @@
+// group.cu -- attention over the keys a group of queries selected together.
+//
+// The plain prefill attention (attn.cu) gathers every query's selected K/V
+// rows on its own: at 2048 keys of 512 bytes per query that is 1 MiB of
+// scattered reads per query, and the kernel runs at the L2 gather rate.
+// Queries that attend to nearly the same keys can share those reads. In the
+// two-stage method the queries that keep the same key blocks (HISA section 3)
+// select mostly the same keys; the grouping kernel below sorts every window
+// of GW consecutive queries by a MinHash of its kept-block set, so runs of GA
+// queries in that order tend to keep the same blocks. The grouped kernel then
+// takes GA queries per CTA (one warp each), forms the union of their index
+// sets with a per-key mask of the queries that chose the key, gathers each
+// union key once into a ring shared by the CTA, and lets every warp attend
+// over the union with its own mask. Each query still attends exactly to its
+// own index set (softmax does not depend on the order of the keys, Latent
+// Sparse Attention section 3.2); the grouping only changes the schedule.
+//
+// A group whose union does not fit the CTA's tables (more than GU_MAX key
+// blocks of 64, more than GL_MAX keys, or n_k above GK_MAX) is processed one
+// query at a time instead, with the query's keys split over the warps and the
+// warp states merged, which is the plain kernel's schedule.
+#include <cuda_bf16.h>
+
+#include "attn_common.cuh"
+#include "ptx.cuh"
+#include "sa_internal.h"
+
+namespace sa {
+
+constexpr int GW = 2048;             // queries per grouping window
+constexpr int GA = kGroupQueries;    // queries per attention group (one warp each)
+constexpr int GT = GA * 32;          // threads per grouped CTA
+constexpr int GCH = 64;              // keys per ring stage
+constexpr int GST = 3;               // ring stages
+constexpr int GU_MAX = 512;          // union blocks of 64 keys
+constexpr int GL_MAX = 16384;        // union keys
+constexpr int GK_MAX = 1 << 20;      // keys per cache covered by the block bitmap
+constexpr int GK_WORDS = GK_MAX / 2048;
+
+// ---------------------------------------------------------------- grouping
+static __device__ __forceinline__ uint32_t block_hash(uint32_t b) {
+  uint32_t x = b * 0x9E3779B1u;
+  x ^= x >> 15;
+  x *= 0x2C1B3C6Du;
+  x ^= x >> 12;
+  return x;
+}
+
+// perm[w * GW + i] = the query at rank i of window w in (signature, query)
+// order, -1 past n_q. The signature is the smallest hash over the query's
+// kept blocks, leaving out block 0 and the query's own block, which every
+// query keeps (HISA section 3: the first and the local block are always in).
+__global__ void __launch_bounds__(1024) group_queries_kernel(const int* __restrict__ kept, int keep, int n_q,
+                                                             int q_pos0, int block, int* __restrict__ perm) {
+  __shared__ unsigned long long key[GW];
+  const int w0 = blockIdx.x * GW;
+  for (int i = threadIdx.x; i < GW; i += 1024) {
+    const int t = w0 + i;
+    unsigned long long k = ~0ull;
+    if (t < n_q) {
+      const int cur = (q_pos0 + t) / block;
+      uint32_t h = 0xFFFFFFFFu;
+      const int* kr = kept + (long long)t * keep;
+      for (int j = 0; j < keep; ++j) {
+        const int b = kr[j];
+        if (b < 0) break;
+        if (b != 0 && b != cur) h = min(h, block_hash((uint32_t)b));
+      }
+      k = ((unsigned long long)h << 32) | (uint32_t)t;
+    }
+    key[i] = k;
+  }
+  __syncthreads();
+  // bitonic sort, ascending
+  for (int size = 2; size <= GW; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < GW / 2; i += 1024) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const unsigned long long a = key[lo], b = key[hi];
+        if ((a > b) == up) {
+          key[lo] = b;
+          key[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < GW; i += 1024) {
+    const unsigned long long k = key[i];
+    perm[w0 + i] = (k == ~0ull) ? -1 : (int)(uint32_t)(k & 0xFFFFFFFFu);
+  }
+}
+
+int group_perm_len(int n_q) { return (n_q + GW - 1) / GW * GW; }
+
+cudaError_t launch_group_queries(const int* kept, int keep, int n_q, int q_pos0, int block, int* perm,
+                                 cudaStream_t st) {
+  if (n_q <= 0) return cudaSuccess;
+  if (keep <= 0 || block <= 0) return cudaErrorInvalidValue;
+  group_queries_kernel<<<(n_q + GW - 1) / GW, 1024, 0, st>>>(kept, keep, n_q, q_pos0, block, perm);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------- grouped attention
+template <int DH>
+struct GaCfg {
+  static constexpr int ROWB = DH * 2;
+  static constexpr int SEGS = ROWB / 16;
+  static constexpr int STAGE_BYTES = 2 * GCH * ROWB;                 // K rows, then V rows
+  static constexpr int RING = GST * STAGE_BYTES;
+  static constexpr int MERGE_BYTES = GA * (16 * DH + 32) * 4;
+  // the union build borrows the ring for the per-key masks and the bitmap
+  static constexpr int MASK_BYTES = GU_MAX * 64;
+  static constexpr int BUILD_BYTES = MASK_BYTES + 2 * GK_WORDS * 4;
+  static_assert(RING >= MERGE_BYTES && RING >= BUILD_BYTES, "ring too small for its other uses");
+  static constexpr int OFF_LIST = RING;
+  static constexpr int OFF_LMASK = OFF_LIST + GL_MAX * 4;
+  static constexpr int OFF_UB = OFF_LMASK + GL_MAX;
+  static constexpr int OFF_MISC = OFF_UB + GU_MAX * 4;
+  static constexpr int SMEM = OFF_MISC + 64 * 4;
+};
+
+template <int HQ, int DH>
+__global__ void __launch_bounds__(GT, 1)
+    grouped_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
+                        const __nv_bfloat16* __restrict__ vc, const int32_t* __restrict__ idx,
+                        const int* __restrict__ perm, int n_q, int k, int n_k, float scale_log2,
+                        __nv_bfloat16* __restrict__ out, float* __restrict__ lse, bool ungrouped) {
+  using C = GaCfg<DH>;
+  using W = AttnWarp<HQ, DH, 1>;
+  extern __shared__ __align__(128) uint8_t ga_smem[];
+  uint32_t* maskw = reinterpret_cast<uint32_t*>(ga_smem);                       // [GU_MAX * 16]  (build only)
+  uint32_t* bits = reinterpret_cast<uint32_t*>(ga_smem + C::MASK_BYTES);       // [GK_WORDS]     (build only)
+  int* wpre = reinterpret_cast<int*>(ga_smem + C::MASK_BYTES + GK_WORDS * 4);  // [GK_WORDS]     (build only)
+  int* list = reinterpret_cast<int*>(ga_smem + C::OFF_LIST);                   // union keys, ascending
+  uint8_t* lmask = ga_smem + C::OFF_LMASK;                                      // their query masks
+  int* ub2blk = reinterpret_cast<int*>(ga_smem + C::OFF_UB);                   // union block -> block
+  int* misc = reinterpret_cast<int*>(ga_smem + C::OFF_MISC);
+  int* qt = misc;                  // [GA] the group's queries (-1: none)
+  int* red = misc + GA;            // [GA] scan partials
+  int& n_ub = misc[2 * GA];
+  int& n_list = misc[2 * GA + 1];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid < GA) {
+    const int j = blockIdx.x * GA + tid;
+    const int t = perm ? perm[j] : j;
+    qt[tid] = (t >= 0 && t < n_q) ? t : -1;
+  }
+  __syncthreads();
+  bool any = false;
+#pragma unroll
+  for (int w = 0; w < GA; ++w) any |= qt[w] >= 0;
+  if (!any) return;
+
+  // ---- union of the group's index sets ----
+  bool grouped = n_k <= GK_MAX && !ungrouped;
+  const int nwords = (n_k + 2047) / 2048;
+  // the group's index rows, staged in the list area (which the union
+  // overwrites only after its last read of them) when they fit; a row read
+  // from global memory entry by entry would leave every thread waiting on
+  // one dependent load per entry
+  const bool staged = (long long)GA * k <= GL_MAX;
+  auto row_at = [&](int qi, int j) -> int {
+    return staged ? list[qi * k + j] : idx[(long long)qt[qi] * k + j];
+  };
+  if (grouped) {
+    if (staged) {
+      const bool vec = (k & 3) == 0 && (reinterpret_cast<uintptr_t>(idx) & 15u) == 0;
+      for (int qi = 0; qi < GA; ++qi) {
+        const int t = qt[qi];
+        int* dst = list + qi * k;
+        if (t >= 0 && vec) {
+          const int32_t* row = idx + (long long)t * k;
+          for (int j = tid * 4; j < k; j += GT * 4) cp_async16(smem_u32(dst + j), row + j);
+        } else {
+          for (int j = tid; j < k; j += GT) dst[j] = t >= 0 ? idx[(long long)t * k + j] : -1;
+        }
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+    }
+    for (int i = tid; i < nwords; i += GT) bits[i] = 0u;
+    __syncthreads();
+    // pass 1: which 64-key blocks hold a selected key
+    for (int qi = 0; qi < GA; ++qi) {
+      if (qt[qi] < 0) continue;
+      for (int j = tid; j < k; j += GT) {
+        const int s = row_at(qi, j);
+        if (s >= 0 && s < n_k) atomicOr(&bits[s >> 11], 1u << ((s >> 6) & 31));
+      }
+    }
+    __syncthreads();
+    // union block numbering in ascending block order
+    if (warp == 0) {
+      const int per = (nwords + 31) / 32;
+      const int lo = min(nwords, lane * per), hi = min(nwords, lo + per);
+      int cnt = 0;
+      for (int i = lo; i < hi; ++i) cnt += __popc(bits[i]);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int p = incl - cnt;
+      for (int i = lo; i < hi; ++i) {
+        wpre[i] = p;
+        uint32_t b = bits[i];
+        while (b) {
+          const int bit = __ffs(b) - 1;
+          b &= b - 1;
+          if (p < GU_MAX) ub2blk[p] = i * 32 + bit;
+          ++p;
+        }
+      }
+      if (lane == 31) n_ub = incl;
+    }
+    __syncthreads();
+    grouped = n_ub <= GU_MAX;
+  }
+  if (grouped) {
+    for (int i = tid; i < n_ub * 16; i += GT) maskw[i] = 0u;
+    __syncthreads();
+    // pass 2: per-key masks of the queries that selected the key
+    for (int qi = 0; qi < GA; ++qi) {
+      if (qt[qi] < 0) continue;
+      for (int j = tid; j < k; j += GT) {
+        const int s = row_at(qi, j);
+        if (s < 0 || s >= n_k) continue;
+        const int wi = s >> 11, b = (s >> 6) & 31;
+        const int ub = wpre[wi] + __popc(bits[wi] & ((1u << b) - 1u));
+        const int slot = ub * 64 + (s & 63);
+        atomicOr(&maskw[slot >> 2], (1u << qi) << (8 * (slot & 3)));
+      }
+    }
+    __syncthreads();
+    // ordered compaction of the selected union keys
+    const int n_slot = n_ub * 64;
+    const int per = (n_slot + GT - 1) / GT;
+    const int lo = min(n_slot, tid * per), hi = min(n_slot, lo + per);
+    const uint8_t* mb = reinterpret_cast<const uint8_t*>(maskw);
+    int cnt = 0;
+    for (int i = lo; i < hi; ++i) cnt += mb[i] != 0;
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) red[warp] = incl;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < GA; ++w) {
+      before += (w < warp) ? red[w] : 0;
+      total += red[w];
+    }
+    if (total <= GL_MAX) {
+      int p = before + incl - cnt;
+      for (int i = lo; i < hi; ++i) {
+        const uint8_t m = mb[i];
+        if (m) {
+          list[p] = ub2blk[i >> 6] * 64 + (i & 63);
+          lmask[p] = m;
+          ++p;
+        }
+      }
+      for (int i = total + tid; i < (total + GCH - 1) / GCH * GCH; i += GT) {
+        list[i] = -1;
+        lmask[i] = 0;
+      }
+    }
+    grouped = total <= GL_MAX;
+    if (tid == 0) n_list = total;
+    __syncthreads();   // the masks (in the ring) are consumed; the list is complete
+  }
+
+  // ---- the ring loop over a key list ----
+  // grouped: every warp takes the 16-key chunks holding one of its keys;
+  // single: the chunks go round-robin over the warps, every listed key valid
+  constexpr int SEGS = C::SEGS;
+  constexpr int RPP = GT / SEGS;        // rows per loader pass
+  auto issue = [&](int stage, int slot) {
+    const uint32_t kdst = smem_u32(ga_smem + slot * C::STAGE_BYTES);
+    const uint32_t vdst = kdst + GCH * C::ROWB;
+    const int seg = tid % SEGS;
+#pragma unroll
+    for (int i = 0; i < GCH / RPP; ++i) {
+      const int r = i * RPP + tid / SEGS;
+      const int s = list[stage * GCH + r];
+      const long long off = (long long)(s >= 0 ? s : 0) * DH + seg * 8;
+      cp_async16(kdst + W::off(r, seg), kc + off);
+      cp_async16(vdst + W::off(r, seg), vc + off);
+    }
+  };
+  uint32_t qa[W::KK][4];
+  float o[W::NT][4], m_r[2], l_r[2];
+  auto run = [&](int n_ent, bool by_mask) {
+    const int n_st = (n_ent + GCH - 1) / GCH;
+#pragma unroll
+    for (int i = 0; i < GST - 1; ++i) {
+      if (i < n_st) issue(i, i);
+      cp_async_commit();
+    }
+    for (int i = 0; i < n_st; ++i) {
+      cp_async_wait<GST - 2>();
+      __syncthreads();
+      if (i + GST - 1 < n_st) issue(i + GST - 1, (i + GST - 1) % GST);
+      cp_async_commit();
+      const uint32_t base = smem_u32(ga_smem + (i % GST) * C::STAGE_BYTES);
+#pragma unroll
+      for (int sub = 0; sub < GCH / AT_CHUNK; ++sub) {
+        const int c = i * (GCH / AT_CHUNK) + sub;
+        if (c * AT_CHUNK >= n_ent) break;
+        const int e = c * AT_CHUNK + (lane & (AT_CHUNK - 1));
+        uint32_t valid;
+        if (by_mask) {
+          valid = __ballot_sync(0xffffffffu, lane < AT_CHUNK && ((lmask[e] >> warp) & 1u));
+        } else {
+          if (c % GA != warp) continue;
+          valid = __ballot_sync(0xffffffffu, lane < AT_CHUNK && list[e] >= 0);
+        }
+        if (valid == 0u) continue;
+        W::step(qa, base + sub * AT_CHUNK * C::ROWB, base + GCH * C::ROWB + sub * AT_CHUNK * C::ROWB, valid, lane,
+                scale_log2, o, m_r, l_r);
+      }
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+  };
+
+  if (grouped) {
+    const int t = qt[warp];
+    W::load_q(q, t, lane, qa);
+    W::init(o, m_r, l_r);
+    run(n_list, true);
+    W::reduce_l(l_r);
+    if (t >= 0) W::store(out + (long long)t * HQ * DH, lse ? lse + (long long)t * HQ : nullptr, lane, o, m_r, l_r);
+    return;
+  }
+
+  // one query at a time, its keys split over the warps
+  for (int qi = 0; qi < GA; ++qi) {
+    const int t = qt[qi];
+    if (t < 0) continue;
+    W::load_q(q, t, lane, qa);
+    W::init(o, m_r, l_r);
+    const int32_t* row = idx + (long long)t * k;
+    for (int j0 = 0; j0 < k; j0 += GL_MAX) {
+      const int n = min(GL_MAX, k - j0);
+      for (int j = tid; j < (n + GCH - 1) / GCH * GCH; j += GT) {
+        const int s = j < n ? row[j0 + j] : -1;
+        list[j] = (s >= 0 && s < n_k) ? s : -1;
+      }
+      __syncthreads();
+      run(n, false);
+    }
+    W::reduce_l(l_r);
+    float* slots = reinterpret_cast<float*>(ga_smem);
+    W::to_slot(slots + warp * (16 * DH + 32), lane, o, m_r, l_r);
+    __syncthreads();
+    for (int e = tid; e < HQ * DH; e += GT) {
+      const int h = e / DH, col = e % DH;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < GA; ++w) M = fmaxf(M, slots[w * (16 * DH + 32) + 16 * DH + h]);
+      const float Ms = (M == -INFINITY) ? 0.f : M;
+      float L = 0.f, acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < GA; ++w) {
+        const float* bw = slots + w * (16 * DH + 32);
+        const float f = exp2f(bw[16 * DH + h] - Ms);
+        L += bw[16 * DH + 16 + h] * f;
+        acc += bw[h * DH + col] * f;
+      }
+      out[((long long)t * HQ + h) * DH + col] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+      if (lse != nullptr && col == 0)
+        lse[(long long)t * HQ + h] = L > 0.f ? (Ms + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    }
+    __syncthreads();
+  }
+}
+
+template <int HQ, int DH>
+static cudaError_t launch_grouped_t(const void* q, const void* kc, const void* vc, const int32_t* idx,
+                                   const int* perm, int n_groups, int n_q, int k, int n_k, float scale, void* out,
+                                   float* lse, bool ungrouped, cudaStream_t st) {
+  using C = GaCfg<DH>;
+  auto kern = grouped_attn_kernel<HQ, DH>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<n_groups, GT, C::SMEM, st>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)kc, (const __nv_bfloat16*)vc,
+                                      idx, perm, n_q, k, n_k, scale * 1.4426950408889634f, (__nv_bfloat16*)out, lse,
+                                      ungrouped);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attention_grouped(const void* q, const void* kc, const void* vc, const int32_t* idx,
+                                     const int* perm, int n_perm, int n_q, int k, int n_k, int hq, int dh,
+                                     float scale, void* out, float* lse, bool ungrouped, cudaStream_t st) {
+  if (n_q <= 0) return cudaSuccess;
+  const int n_groups = ((perm ? n_perm : n_q) + GA - 1) / GA;
+  if (hq == 16 && dh == 128)
+    return launch_grouped_t<16, 128>(q, kc, vc, idx, perm, n_groups, n_q, k, n_k, scale, out, lse, ungrouped, st);
+  if (hq == 8 && dh == 128)
+    return launch_grouped_t<8, 128>(q, kc, vc, idx, perm, n_groups, n_q, k, n_k, scale, out, lse, ungrouped, st);
+  if (hq == 16 && dh == 64)
+    return launch_grouped_t<16, 64>(q, kc, vc, idx, perm, n_groups, n_q, k, n_k, scale, out, lse, ungrouped, st);
+  if (hq == 8 && dh == 64)
+    return launch_grouped_t<8, 64>(q, kc, vc, idx, perm, n_groups, n_q, k, n_k, scale, out, lse, ungrouped, st);
+  return cudaErrorNotSupported;
+}
+
+}  // namespace sa
+
+namespace sa {
+
+// ------------------------------------------------------ union of a group
+// Two-stage rows: a query's selected keys are the set bits of its selection
+// bitmap over its kept blocks' candidates (column c = 64 * slot + offset).
+// The union of the group is built block-wise: the group's kept blocks in
+// ascending order (a bitmap over all blocks, ranked by popcount), a table of
+// each query's slot of every union block, then one mask byte per union key.
+int group_union_cap(int k) { return (GA * k + 63) / 64 * 64; }
+
+__global__ void __launch_bounds__(256) group_union_kernel(const int* __restrict__ kept, int keep,
+                                                          const uint32_t* __restrict__ sel, const int* __restrict__ perm,
+                                                          int n_q, int n_k, int cap, int* __restrict__ list,
+                                                          uint8_t* __restrict__ lmask, int* __restrict__ n_list) {
+  constexpr int KB = 64;                         // kept blocks per query (at most)
+  __shared__ int qt[GA];
+  __shared__ int kb[GA][KB];
+  __shared__ uint32_t sw[GA][2 * KB];
+  __shared__ uint32_t bits[GK_WORDS];
+  __shared__ int wpre[GK_WORDS];
+  __shared__ signed char slot[GA][GA * KB];
+  __shared__ int ub2blk[GA * KB];
+  __shared__ int red[8];
+  __shared__ int s_nub;
+  const int g = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid < GA) {
+    const int j = g * GA + tid;
+    const int t = perm ? perm[j] : j;
+    qt[tid] = (t >= 0 && t < n_q) ? t : -1;
+  }
+  const int nwords = ((n_k + 63) / 64 + 31) / 32;
+  for (int i = tid; i < nwords; i += 256) bits[i] = 0u;
+  __syncthreads();
+  const int words = 2 * keep;
+  for (int i = tid; i < GA * KB; i += 256) {
+    const int qi = i / KB, c = i % KB, t = qt[qi];
+    kb[qi][c] = (t >= 0 && c < keep) ? kept[(long long)t * keep + c] : -1;
+  }
+  for (int i = tid; i < GA * 2 * KB; i += 256) {
+    const int qi = i / (2 * KB), w = i % (2 * KB), t = qt[qi];
+    sw[qi][w] = (t >= 0 && w < words) ? sel[(long long)t * words + w] : 0u;
+  }
+  __syncthreads();
+  for (int i = tid; i < GA * KB; i += 256) {
+    const int b = kb[i / KB][i % KB];
+    if (b >= 0) atomicOr(&bits[b >> 5], 1u << (b & 31));
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int per = (nwords + 31) / 32;
+    const int lo = min(nwords, lane * per), hi = min(nwords, lo + per);
+    int cnt = 0;
+    for (int i = lo; i < hi; ++i) cnt += __popc(bits[i]);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int p = incl - cnt;
+    for (int i = lo; i < hi; ++i) {
+      wpre[i] = p;
+      uint32_t b = bits[i];
+      while (b) {
+        const int bit = __ffs(b) - 1;
+        b &= b - 1;
+        ub2blk[p++] = i * 32 + bit;
+      }
+    }
+    if (lane == 31) s_nub = incl;
+  }
+  __syncthreads();
+  const int n_ub = s_nub;                         // <= GA * KB: every union block is some query's kept block
+  for (int i = tid; i < GA * GA * KB; i += 256) (&slot[0][0])[i] = -1;
+  __syncthreads();
+  for (int i = tid; i < GA * KB; i += 256) {
+    const int qi = i / KB, c = i % KB, b = kb[qi][c];
+    if (b >= 0) slot[qi][wpre[b >> 5] + __popc(bits[b >> 5] & ((1u << (b & 31)) - 1u))] = (signed char)c;
+  }
+  __syncthreads();
+  auto mask_of = [&](int e) -> uint32_t {
+    const int u = e >> 6, j = e & 63;
+    uint32_t m = 0u;
+#pragma unroll
+    for (int qi = 0; qi < GA; ++qi) {
+      const int s = slot[qi][u];
+      if (s >= 0) {
+        const int c = s * 64 + j;
+        m |= ((sw[qi][c >> 5] >> (c & 31)) & 1u) << qi;
+      }
+    }
+    return m;
+  };
+  const int n_slot = n_ub * 64;
+  const int per = (n_slot + 255) / 256;
+  const int lo = min(n_slot, tid * per), hi = min(n_slot, lo + per);
+  int cnt = 0;
+  for (int e = lo; e < hi; ++e) cnt += mask_of(e) != 0u;
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) red[warp] = incl;
+  __syncthreads();
+  int before = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    before += (w < warp) ? red[w] : 0;
+    total += red[w];
+  }
+  total = min(total, cap);                        // cannot bind: each query selects at most k keys
+  int* gl = list + (long long)g * cap;
+  uint8_t* gm = lmask + (long long)g * cap;
+  int p = before + incl - cnt;
+  for (int e = lo; e < hi; ++e) {
+    const uint32_t m = mask_of(e);
+    if (m != 0u) {
+      if (p < cap) {
+        gl[p] = ub2blk[e >> 6] * 64 + (e & 63);
+        gm[p] = (uint8_t)m;
+      }
+      ++p;
+    }
+  }
+  for (int i = total + tid; i < (total + 63) / 64 * 64; i += 256) {
+    gl[i] = -1;
+    gm[i] = 0;
+  }
+  if (tid == 0) n_list[g] = total;
+}
+
+cudaError_t launch_group_union(const int* kept, int keep, const uint32_t* sel, const int* perm, int n_perm, int n_q,
+                               int n_k, int cap, int* list, uint8_t* lmask, int* n_list, cudaStream_t st) {
+  if (n_q <= 0) return cudaSuccess;
+  if (keep <= 0 || keep > 64 || n_k > GK_MAX || cap % 64 != 0) return cudaErrorNotSupported;
+  const int n_groups = ((perm ? n_perm : n_q) + GA - 1) / GA;
+  group_union_kernel<<<n_groups, 256, 0, st>>>(kept, keep, sel, perm, n_q, n_k, cap, list, lmask, n_list);
+  return cudaGetLastError();
+}
+
+}  // namespace sa

@@ -172,6 +172,23 @@ __device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4]) {
                : "r"(taddr));
 }
 
+// 32 lanes x 32 consecutive 32-bit columns <- 32 registers per thread.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  const uint32_t* r = reinterpret_cast<const uint32_t*>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
+      "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+      "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -204,6 +221,21 @@ __device__ __forceinline__ uint64_t umma_smem_desc(uint32_t saddr) {
   return d;
 }
 
+// Descriptor of a 128-byte-swizzled operand with explicit strides (bytes):
+// for a K-major operand lbo is unused and sbo is the distance between 8-row
+// groups; for an MN-major operand (the contiguous 128-byte rows run along M
+// or N, one row per K index) lbo is the distance between 64-element column
+// blocks along M/N and sbo the distance between groups of 8 K rows.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  d |= 2ull << 61;
+  return d;
+}
+
 // Instruction descriptor: D f32, A/B K-major, dense.
 // fmt: 0 = e4m3 (kind::f8f6f4), 1 = bf16 (kind::f16).
 template <int FMT, int M, int N>
@@ -215,6 +247,12 @@ __host__ __device__ constexpr uint32_t umma_idesc() {
          | (uint32_t(FMT) << 10)         // B format
          | (uint32_t(N >> 3) << 17)      // N / 8
          | (uint32_t(M >> 4) << 24);     // M / 16
+}
+
+// The same with B read MN-major (bit 16: B transposed relative to K-major).
+template <int FMT, int M, int N>
+__host__ __device__ constexpr uint32_t umma_idesc_bmn() {
+  return umma_idesc<FMT, M, N>() | (1u << 16);
 }
 
 }  // namespace sa

@@ -101,7 +101,9 @@ struct PrefillPlan {
   int nb;          // two-stage: complete blocks
   bool stream;     // FLAT without a score table
   int m, n_s, cap, fb;   // stream: sample stride and count, list capacity, fallback rows per batch
-  size_t off_table, off_idx, off_blk, off_blks, off_bsc, off_kept, off_cand, total;
+  size_t off_table, off_idx, off_blk, off_blks, off_bsc, off_kept, off_cand, off_perm, total;
+  size_t off_sel, off_ulist, off_umask, off_unl;   // two-stage: group union lists
+  int n_groups, ucap;
   size_t off_ks, off_kss, off_stab, off_theta, off_cnt, off_list, off_miss, off_rows, off_count, off_pos;
   size_t off_fq, off_fqs, off_fw, off_ftab;
 };
@@ -109,6 +111,7 @@ struct PrefillPlan {
 constexpr int kStreamSamples = 16384;      // sampled keys per row for the threshold (at most)
 constexpr float kStreamGamma = 2.0f;       // target list length = gamma * k
 constexpr int kTableMaxKeys = 65536;       // FLAT auto: table path up to this many keys
+constexpr int kUnionMaxKeys = 1 << 20;     // block bitmap of the group union kernel
 
 static bool flat_streams(const sa_indexer_in* in, const sa_prefill_opts* o) {
   if (o->mode != SA_MODE_FLAT) return false;
@@ -179,6 +182,19 @@ static bool plan_prefill(const sa_indexer_in* in, const sa_prefill_opts* o, Pref
     off += align256((size_t)R * o->keep_blocks * 4);
     p->off_cand = off;
     off += align256((size_t)R * o->keep_blocks * o->block_size * 4);
+    p->off_perm = off;
+    off += align256((size_t)group_perm_len(R) * 4);
+    // tensor-core attention of the groups' union lists
+    p->n_groups = group_perm_len(R) / kGroupQueries;
+    p->ucap = group_union_cap(o->k);
+    p->off_sel = off;
+    off += align256((size_t)R * o->keep_blocks * 2 * 4);
+    p->off_ulist = off;
+    off += align256((size_t)p->n_groups * p->ucap * 4);
+    p->off_umask = off;
+    off += align256((size_t)p->n_groups * p->ucap);
+    p->off_unl = off;
+    off += align256((size_t)p->n_groups * 4);
   }
   p->off_idx = off;
   off += align256((size_t)R * o->k * 4);
@@ -554,6 +570,10 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
         e = launch_block_select(bsc, R, p.nb, std::max(p.nb, 1), ci.q_pos0, o->block_size, o->keep_blocks, kept,
                                 stream);
       if (e != cudaSuccess) return cuda_status(e);
+      // attention groups: queries that keep the same blocks side by side
+      e = launch_group_queries(kept, o->keep_blocks, R, ci.q_pos0, o->block_size,
+                               reinterpret_cast<int*>(w + p.off_perm), stream);
+      if (e != cudaSuccess) return cuda_status(e);
       // stage 2: the visible keys of the kept blocks
       sm.mark(3, stream);
       IdxArgs a = base_args(&ci, status, o->test_hook);
@@ -564,17 +584,34 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
       e = launch_indexer(IDX_GATHER, in->n_heads, in->d_idx, in->dtype, ci.q, in->k, R, in->n_k, a, stream);
       if (e != cudaSuccess) return cuda_status(e);
       sm.mark(4, stream);
-      e = launch_topk_fast(cand, R, ncand, ncand, 0, nullptr, kept, o->keep_blocks, o->k, idx, stream);
-      if (e == cudaErrorNotSupported)
-        e = launch_topk_table(cand, R, ncand, ncand, ci.q_pos0, o->k, idx, 2, kept, o->keep_blocks, nullptr, stream);
-      if (e != cudaSuccess) return cuda_status(e);
+      uint32_t* sel = reinterpret_cast<uint32_t*>(w + p.off_sel);
+      e = launch_topk_fast(cand, R, ncand, ncand, 0, nullptr, kept, o->keep_blocks, o->k, idx, stream, sel);
+      if (e != cudaSuccess) return cuda_status(e);   // keep_blocks <= 64: at most 4096 candidates
     }
     const void* qa = static_cast<const char*>(at->q) + (size_t)r0 * at->n_q_heads * at->head_dim * 2;
     void* oa = static_cast<char*>(out) + (size_t)r0 * at->n_q_heads * at->head_dim * 2;
     float* la = lse ? lse + (size_t)r0 * at->n_q_heads : nullptr;
     sm.mark(n_stages - 1, stream);
-    e = launch_attention(qa, at->k_cache, at->v_cache, idx, R, o->k, at->n_k, at->n_q_heads, at->head_dim, scale, 0,
-                         oa, la, nullptr, nullptr, 1, stream, status);
+    // grouped attention: two-stage groups by kept blocks (tensor cores over
+    // each group's union of keys), FLAT groups by query order
+    const int* perm = o->mode == SA_MODE_TWO_STAGE ? reinterpret_cast<const int*>(w + p.off_perm) : nullptr;
+    const bool ungrouped = o->test_hook == SA_HOOK_ATTN_UNGROUPED;
+    if (o->mode == SA_MODE_TWO_STAGE && !ungrouped && tc_attention_supported(at->n_q_heads, at->head_dim) &&
+        in->n_k <= kUnionMaxKeys) {
+      int* list = reinterpret_cast<int*>(w + p.off_ulist);
+      uint8_t* lmask = reinterpret_cast<uint8_t*>(w + p.off_umask);
+      int* nlist = reinterpret_cast<int*>(w + p.off_unl);
+      e = launch_group_union(reinterpret_cast<const int*>(w + p.off_kept), o->keep_blocks,
+                             reinterpret_cast<const uint32_t*>(w + p.off_sel), perm, group_perm_len(R), R, in->n_k,
+                             p.ucap, list, lmask, nlist, stream);
+      if (e != cudaSuccess) return cuda_status(e);
+      e = launch_attention_tc(qa, at->k_cache, at->v_cache, list, lmask, nlist, perm, p.n_groups, R, p.ucap, scale,
+                              oa, la, status, o->test_hook == SA_HOOK_STALL_WAIT ? kHookBudget : kWaitBudget,
+                              stream);
+    } else {
+      e = launch_attention_grouped(qa, at->k_cache, at->v_cache, idx, perm, group_perm_len(R), R, o->k, at->n_k,
+                                   at->n_q_heads, at->head_dim, scale, oa, la, ungrouped, stream);
+    }
     if (e != cudaSuccess) return cuda_status(e);
     sm.mark(n_stages, stream);
   }

@@ -49,8 +49,11 @@ cudaError_t launch_topk_table(const float* scores, int n_rows, int n_cols, long 
                               cudaStream_t st, const int* row_pos = nullptr, const int* out_rows = nullptr,
                               const int* only_flagged = nullptr);
 
+// sel (gathered rows only, nullable): per row keep * 2 words, bit c of the
+// row's bitmap set iff candidate column c was selected
 cudaError_t launch_topk_fast(const float* scores, int n_rows, long long ld, int n_cols, int q_pos0, const int* row_pos,
-                             const int* kept, int keep, int k, int32_t* idx, cudaStream_t st);
+                             const int* kept, int keep, int k, int32_t* idx, cudaStream_t st,
+                             uint32_t* sel = nullptr);
 
 // ---- streaming selector (stream.cu) ----
 cudaError_t launch_gather_rows(const void* src, void* dst, const int* rows, int n_rows, long long src_stride,
@@ -82,6 +85,29 @@ cudaError_t launch_attention(const void* q, const void* kc, const void* vc, cons
                              int n_k, int hq, int dh, float scale, int batch, void* out, float* lse,
                              float* part_o, float* part_lse, int splits, cudaStream_t st,
                              uint32_t* status = nullptr);
+
+// grouped prefill attention (group.cu): perm orders the queries so that runs
+// of kGroupQueries share keys (nullptr: query order); n_perm = its length
+constexpr int kGroupQueries = 8;
+int group_perm_len(int n_q);
+cudaError_t launch_group_queries(const int* kept, int keep, int n_q, int q_pos0, int block, int* perm,
+                                 cudaStream_t st);
+cudaError_t launch_attention_grouped(const void* q, const void* kc, const void* vc, const int32_t* idx,
+                                     const int* perm, int n_perm, int n_q, int k, int n_k, int hq, int dh,
+                                     float scale, void* out, float* lse, bool ungrouped, cudaStream_t st);
+
+// union of each group's index sets (two-stage rows: kept blocks + selection
+// bitmaps) as ascending key lists in whole chunks of 64, with per-key masks of
+// the group's queries; cap = list capacity per group (a multiple of 64)
+int group_union_cap(int k);
+cudaError_t launch_group_union(const int* kept, int keep, const uint32_t* sel, const int* perm, int n_perm, int n_q,
+                               int n_k, int cap, int* list, uint8_t* lmask, int* n_list, cudaStream_t st);
+
+// tcgen05 attention of the groups' union lists (attn_tc.cu), 16 heads x 128 dims
+bool tc_attention_supported(int hq, int dh);
+cudaError_t launch_attention_tc(const void* q, const void* kc, const void* vc, const int* list, const uint8_t* lmask,
+                                const int* n_list, const int* perm, int n_groups, int n_q, int cap, float scale,
+                                void* out, float* lse, uint32_t* status, long long budget, cudaStream_t st);
 
 cudaError_t launch_fill_upper(float* scores, int n_q, int n_k, long long ld, int q_pos0, cudaStream_t st);
 

@@ -37,7 +37,7 @@ struct TfShared {
 __global__ void __launch_bounds__(TF_THREADS)
     topk_fast_kernel(const float* __restrict__ scores, int n_rows, long long ld, int n_cols, int q_pos0,
                      const int* __restrict__ row_pos, const int* __restrict__ kept, int keep, int k,
-                     int32_t* __restrict__ idx) {
+                     int32_t* __restrict__ idx, uint32_t* __restrict__ sel) {
   __shared__ TfShared sh;
   const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool gathered = kept != nullptr;
@@ -111,8 +111,9 @@ __global__ void __launch_bounds__(TF_THREADS)
   }
   int32_t* out = idx + (long long)row * k;
   auto key_of = [&](int c) { return gathered ? sh.kb[c >> 6] * 64 + (c & 63) : c; };
-  // ordered emission of the positions whose flag is set (block scan over (thread, element))
-  auto emit_ordered = [&](auto flag, int base, int limit) {
+  // ordered emission of the positions whose flag is set (block scan over
+  // (thread, element)); returns the thread's emitted elements as a bit mask
+  auto emit_ordered = [&](auto flag, int base, int limit) -> uint32_t {
     int mine = 0;
 #pragma unroll
     for (int i = 0; i < TF_PER; ++i) mine += flag(i) ? 1 : 0;
@@ -130,15 +131,24 @@ __global__ void __launch_bounds__(TF_THREADS)
     for (int w = 0; w < TF_THREADS / 32; ++w)
       if (w < warp) before += sh.red[w];
     int p = base + before + x - mine;
+    uint32_t emitted = 0u;
 #pragma unroll
     for (int i = 0; i < TF_PER; ++i)
       if (flag(i)) {
-        if (p < limit) out[p] = key_of(c0 + i);
+        if (p < limit) {
+          out[p] = key_of(c0 + i);
+          emitted |= 1u << i;
+        }
         ++p;
       }
+    return emitted;
+  };
+  // selection bitmap of a gathered row: word tid covers columns [32 tid, 32 tid + 32)
+  auto put_sel = [&](uint32_t word) {
+    if (sel != nullptr && tid < keep * 2) sel[(long long)row * keep * 2 + tid] = word;
   };
   if (nv <= k) {
-    emit_ordered([&](int i) { return key[i] != 0u; }, 0, k);
+    put_sel(emit_ordered([&](int i) { return key[i] != 0u; }, 0, k));
     for (int j = nv + tid; j < k; j += TF_THREADS) out[j] = -1;
     return;
   }
@@ -216,29 +226,31 @@ __global__ void __launch_bounds__(TF_THREADS)
   }
   // every key strictly above the cut (or, for a bucket taken whole, at or above)
   int base = 0;
+  uint32_t word = 0u;
   {
     const bool whole = ties < 0;
-    int mine = 0;
 #pragma unroll
     for (int i = 0; i < TF_PER; ++i) {
       const uint32_t kk = key[i];
       const bool take = kk != 0u && (whole ? kk >= cut : kk > cut);
       if (take) {
         out[atomicAdd(&sh.n_out, 1)] = key_of(c0 + i);
-        ++mine;
+        word |= 1u << i;
       }
     }
     __syncthreads();
     base = sh.n_out;
   }
-  if (ties > 0) emit_ordered([&](int i) { return key[i] != 0u && key[i] == cut; }, base, base + ties);
+  if (ties > 0) word |= emit_ordered([&](int i) { return key[i] != 0u && key[i] == cut; }, base, base + ties);
+  put_sel(word);
 }
 
 cudaError_t launch_topk_fast(const float* scores, int n_rows, long long ld, int n_cols, int q_pos0, const int* row_pos,
-                             const int* kept, int keep, int k, int32_t* idx, cudaStream_t st) {
+                             const int* kept, int keep, int k, int32_t* idx, cudaStream_t st, uint32_t* sel) {
   if (n_rows <= 0) return cudaSuccess;
   if ((kept != nullptr ? keep * 64 : n_cols) > TF_MAXN) return cudaErrorNotSupported;
-  topk_fast_kernel<<<n_rows, TF_THREADS, 0, st>>>(scores, n_rows, ld, n_cols, q_pos0, row_pos, kept, keep, k, idx);
+  topk_fast_kernel<<<n_rows, TF_THREADS, 0, st>>>(scores, n_rows, ld, n_cols, q_pos0, row_pos, kept, keep, k, idx,
+                                                  kept != nullptr ? sel : nullptr);
   return cudaGetLastError();
 }
 

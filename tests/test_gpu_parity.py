@@ -267,6 +267,33 @@ def test_prefill_two_stage_small(sa):
     _check_two_stage(sa, wl, 3, rows, k=512)
 
 
+def test_prefill_attention_grouped_and_per_query_schedules(sa):
+    """The grouped prefill attention (runs of 8 queries sharing one gather of
+    their union of keys) and its one-query-at-a-time schedule both match the
+    oracle's attention over the same index rows, on a ragged two-stage chunking
+    (windows of queries that end mid-group) and on FLAT query order."""
+    wl = WORKLOADS["two_stage_t64k"].with_(T=6000, k=512)
+    inp = PrefillInputs(wl, "cuda", seed=8)
+    host = inp.to_host()
+    rows = sample_rows(wl.T, 60, seed=8, k=512, extra=(0, 1, 1499, 1500, 2047, 2048, 5999))
+    outs = {}
+    for name, hook, chunk in (("grouped", 0, 1500), ("per_query", sa.SA_HOOK_ATTN_UNGROUPED, 1500)):
+        pre = sa.Prefill(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, 512,
+                         mode="two_stage", chunk_rows=chunk, test_hook=hook)
+        out, lse, idx = pre()
+        torch.cuda.synchronize()
+        outs[name] = (out.float().cpu().numpy(), lse.cpu().numpy(), idx.cpu().numpy())
+    # the same index sets (the order inside a row is not specified)
+    assert np.array_equal(np.sort(outs["grouped"][2], axis=1), np.sort(outs["per_query"][2], axis=1))
+    att = attention_rows(host, {t: outs["grouped"][2][t] for t in rows})
+    for name, (out, lse, _) in outs.items():
+        for t in rows:
+            check_attention_row(out[t], att[t][0], lse[t], att[t][1], f"{name} row {t}")
+    wl = WORKLOADS["tiny_t512"]
+    _check_prefill(sa, wl, 9, range(0, wl.T, 7), hook=sa.SA_HOOK_ATTN_UNGROUPED)
+    _check_prefill(sa, wl, 9, range(0, wl.T, 7))
+
+
 def test_prefill_two_stage_equals_flat_below_64_blocks(sa):
     wl = WORKLOADS["two_stage_t64k"].with_(T=3000, k=256, topic_run=256)
     inp = PrefillInputs(wl, "cuda", seed=4)
