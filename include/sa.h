@@ -182,8 +182,9 @@ typedef struct {
 #define SA_HOOK_THETA_POS_INF 1   /* every row misses low -> whole-row fallback */
 #define SA_HOOK_THETA_NEG_INF 2   /* every key is a candidate -> overflow path */
 #define SA_HOOK_STALL_WAIT 3      /* a device wait that never completes -> SA_ERR_TIMEOUT */
-#define SA_HOOK_ATTN_UNGROUPED 4  /* prefill attention takes one query at a time, as for a group whose union of
-                                     selected keys does not fit the kernel's tables */
+#define SA_HOOK_ATTN_UNGROUPED 4  /* no query groups: the two-stage stage 2 scores each query's kept blocks on
+                                     its own and the prefill attention takes one query at a time, as for a
+                                     group whose union of selected keys does not fit the kernel's tables */
 
 /* Human-readable name of a status code (host, static storage). */
 const char* sa_status_string(sa_status s);

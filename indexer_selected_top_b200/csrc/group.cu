@@ -559,3 +559,90 @@ cudaError_t launch_group_union(const int* kept, int keep, const uint32_t* sel, c
 }
 
 }  // namespace sa
+
+namespace sa {
+
+// ------------------------------------------------- union of kept blocks
+// Per group: the blocks any of its queries kept, ascending, and for each the
+// slot (position in the query's kept list) of every query that kept it. The
+// two-stage stage 2 scores each union block once for the whole group.
+int group_blocks_cap() { return GA * 64; }
+
+__global__ void __launch_bounds__(256) group_blocks_kernel(const int* __restrict__ kept, int keep,
+                                                           const int* __restrict__ perm, int n_q, int n_k,
+                                                           int* __restrict__ gb_n, int* __restrict__ gb_blk,
+                                                           unsigned long long* __restrict__ gb_slot) {
+  constexpr int KB = 64, CAP = GA * KB;
+  __shared__ int qt[GA];
+  __shared__ int kb[GA][KB];
+  __shared__ uint32_t bits[GK_WORDS];
+  __shared__ int wpre[GK_WORDS];
+  __shared__ unsigned long long slots[CAP];
+  __shared__ int ub2blk[CAP];
+  __shared__ int s_nub;
+  const int g = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid < GA) {
+    const int j = g * GA + tid;
+    const int t = perm ? perm[j] : j;
+    qt[tid] = (t >= 0 && t < n_q) ? t : -1;
+  }
+  const int nwords = ((n_k + 63) / 64 + 31) / 32;
+  for (int i = tid; i < nwords; i += 256) bits[i] = 0u;
+  for (int i = tid; i < CAP; i += 256) slots[i] = ~0ull;
+  __syncthreads();
+  for (int i = tid; i < GA * KB; i += 256) {
+    const int qi = i / KB, c = i % KB, t = qt[qi];
+    const int b = (t >= 0 && c < keep) ? kept[(long long)t * keep + c] : -1;
+    kb[qi][c] = b;
+    if (b >= 0) atomicOr(&bits[b >> 5], 1u << (b & 31));
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int per = (nwords + 31) / 32;
+    const int lo = min(nwords, lane * per), hi = min(nwords, lo + per);
+    int cnt = 0;
+    for (int i = lo; i < hi; ++i) cnt += __popc(bits[i]);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int p = incl - cnt;
+    for (int i = lo; i < hi; ++i) {
+      wpre[i] = p;
+      uint32_t b = bits[i];
+      while (b) {
+        const int bit = __ffs(b) - 1;
+        b &= b - 1;
+        ub2blk[p++] = i * 32 + bit;
+      }
+    }
+    if (lane == 31) s_nub = incl;
+  }
+  __syncthreads();
+  // every query writes its own byte of each of its blocks' slot words
+  uint8_t* sb = reinterpret_cast<uint8_t*>(slots);
+  for (int i = tid; i < GA * KB; i += 256) {
+    const int qi = i / KB, c = i % KB, b = kb[qi][c];
+    if (b >= 0) sb[(wpre[b >> 5] + __popc(bits[b >> 5] & ((1u << (b & 31)) - 1u))) * 8 + qi] = (uint8_t)c;
+  }
+  __syncthreads();
+  const int n_ub = s_nub;
+  for (int u = tid; u < n_ub; u += 256) {
+    gb_blk[(long long)g * CAP + u] = ub2blk[u];
+    gb_slot[(long long)g * CAP + u] = slots[u];
+  }
+  if (tid == 0) gb_n[g] = n_ub;
+}
+
+cudaError_t launch_group_blocks(const int* kept, int keep, const int* perm, int n_perm, int n_q, int n_k, int* gb_n,
+                                int* gb_blk, unsigned long long* gb_slot, cudaStream_t st) {
+  if (n_q <= 0) return cudaSuccess;
+  if (keep <= 0 || keep > 64 || n_k > GK_MAX) return cudaErrorNotSupported;
+  const int n_groups = ((perm ? n_perm : n_q) + GA - 1) / GA;
+  group_blocks_kernel<<<n_groups, 256, 0, st>>>(kept, keep, perm, n_q, n_k, gb_n, gb_blk, gb_slot);
+  return cudaGetLastError();
+}
+
+}  // namespace sa

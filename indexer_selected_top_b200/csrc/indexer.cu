@@ -24,6 +24,10 @@
 //   IDX_DECODE   one query per sequence, a span of that sequence's key tiles
 //   IDX_GATHER   per query, the 64-key blocks it kept (two-stage stage 2);
 //                a tile = two kept blocks, N = H
+//   IDX_GROUPED  per group of 8 queries, the union of their kept blocks
+//                (two-stage stage 2): a tile = two union blocks, scored for
+//                QS queries at a time (N = 256); each score goes to the
+//                query's own candidate column if it kept the block
 // Output: the fp32 score of every (row, key) of the processed tiles, -inf
 // where the key is not visible, into a row-major table.
 #include <cstdio>
@@ -57,10 +61,16 @@ template <int H, int D, bool FP8, int MODE>
 struct IdxCfg {
   static constexpr int ESZ = FP8 ? 1 : 2;
   static constexpr int ROWB = D * ESZ;                       // bytes per index row
-  static constexpr int QS = (MODE == IDX_PREFILL) ? (SA_IDX_PREFILL_N / H) : 1;
+  static constexpr bool WIDE = MODE == IDX_PREFILL || MODE == IDX_GROUPED;   // N = QS queries x H heads
+  static constexpr int QS = WIDE ? (SA_IDX_PREFILL_N / H) : 1;
   static constexpr int N = QS * H;                           // MMA N
-  static constexpr int G = (MODE == IDX_PREFILL) ? (QS * 2 < 8 ? 8 / QS : 2) : 1;    // sub-tiles per CTA
-  static constexpr int NQ = (MODE == IDX_PREFILL) ? QS * G : (MODE == IDX_GATHER ? SA_IDX_GATHER_NQ : 1);
+  static constexpr int G = (MODE == IDX_PREFILL)   ? (QS * 2 < 8 ? 8 / QS : 2)
+                           : (MODE == IDX_GROUPED) ? (kGroupQueries / QS > 0 ? kGroupQueries / QS : 1)
+                                                   : 1;      // sub-tiles per CTA
+  static constexpr int NQ = (MODE == IDX_PREFILL)   ? QS * G
+                            : (MODE == IDX_GATHER)  ? SA_IDX_GATHER_NQ
+                            : (MODE == IDX_GROUPED) ? kGroupQueries
+                                                    : 1;
   static constexpr int NBUF = 512 / N;                       // TMEM accumulator buffers (fp32 columns)
   static constexpr int TEAMS = SA_IDX_TEAMS;
   static constexpr int THREADS = 64 + 128 * TEAMS;
@@ -70,13 +80,18 @@ struct IdxCfg {
   static constexpr int NS = (MODE == IDX_DECODE) ? 8 : SA_IDX_STAGES;    // key-tile stages
   static constexpr int KSTEPS = ROWB / 32;                   // 32-byte K slices per MMA
   static constexpr int KEEPMAX = 64;                          // gather: kept blocks per query
-  // gather: kept lists; other modes: the rows' thetas (candidate mode); 16-byte multiple
-  static constexpr int KEPT_BYTES = (MODE == IDX_GATHER) ? NQ * KEEPMAX * 4 : (NQ * 4 + 15) / 16 * 16;
+  static constexpr int GU = kGroupQueries * KEEPMAX;          // grouped: union blocks per group (at most)
+  // gather: kept lists; grouped: union blocks, their slot words and the
+  // group's queries; other modes: the rows' thetas (candidate mode); 16-byte multiple
+  static constexpr int KEPT_BYTES = (MODE == IDX_GATHER)    ? NQ * KEEPMAX * 4
+                                    : (MODE == IDX_GROUPED) ? GU * 8 + GU * 4 + 64
+                                                            : (NQ * 4 + 15) / 16 * 16;
   static constexpr int SMEM_USED =
       1024 + QBYTES + NS * KBYTES + NQ * H * 4 + KEPT_BYTES + (2 * NS + 1 + 2 * NBUF) * 8 + 16;
   // at least 120 KB: one CTA per SM, so two CTAs never contend for TMEM
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   static_assert(N <= 256 && N % 16 == 0, "MMA N");
+  static_assert(MODE != IDX_GROUPED || QS * G == kGroupQueries, "one group per CTA");
   static_assert(N % 32 == 0, "epilogue loads 32 columns at a time");
 };
 
@@ -126,6 +141,10 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
   float* sW = reinterpret_cast<float*>(sK + C::NS * C::KBYTES);
   int* sKept = reinterpret_cast<int*>(sW + C::NQ * H);         // gather: [NQ][KEEPMAX], -1 padded
   float* sTheta = reinterpret_cast<float*>(sKept);            // candidate mode: theta of the CTA's rows
+  // grouped: [GU] slot words, [GU] union blocks, [NQ] the group's queries
+  unsigned long long* sUSlot = reinterpret_cast<unsigned long long*>(sKept);
+  int* sUBlk = reinterpret_cast<int*>(sUSlot + C::GU);
+  int* sQt = sUBlk + C::GU;
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sKept) + C::KEPT_BYTES);
   uint64_t* kfull = bars;
   uint64_t* kempty = bars + C::NS;
@@ -156,6 +175,10 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
     tile0 = blockIdx.x * a.tiles_per_cta;
     ntiles = max(0, min(a.tiles_per_cta, total - tile0));
     njobs = ntiles;
+  } else if constexpr (MODE == IDX_GROUPED) {
+    q0 = blockIdx.x * C::NQ;       // the group's slice of perm
+    nq = C::NQ;
+    geff = C::G;                   // jobs are counted from the staged union below
   } else {
     q0 = blockIdx.x * C::NQ;
     nq = min(C::NQ, a.n_q - q0);   // jobs are counted from the staged kept lists below
@@ -179,8 +202,13 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
   for (int i = threadIdx.x; i < C::NQ * H; i += blockDim.x) {
     const int ql = i / H, h = i % H;
     float v = 0.f;
-    if (ql < nq) {
-      const long long r = (long long)(q0 + ql) * H + h;
+    int qrow = (ql < nq) ? q0 + ql : -1;
+    if constexpr (MODE == IDX_GROUPED) {
+      qrow = a.perm[q0 + ql];
+      if (qrow >= a.n_q) qrow = -1;
+    }
+    if (qrow >= 0) {
+      const long long r = (long long)qrow * H + h;
       v = a.w[r] * (a.q_scale ? a.q_scale[r] : 1.f);
     }
     sW[i] = SA_IDX_EPI_PACKED ? 0.5f * v : v;   // packed math sums (w / 2) * (a + |a|)
@@ -196,7 +224,27 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
       sKept[i] = (ql < nq && j < a.keep) ? a.kept[(long long)(q0 + ql) * a.keep + j] : -1;
     }
   }
+  if constexpr (MODE == IDX_GROUPED) {
+    // the group's queries and its union blocks with every query's slot
+    const int g = blockIdx.x;
+    const int nub = a.gb_n[g];
+    for (int i = threadIdx.x; i < C::NQ; i += blockDim.x) {
+      const int t = a.perm[q0 + i];
+      sQt[i] = (t >= 0 && t < a.n_q) ? t : -1;
+    }
+    for (int i = threadIdx.x; i < nub; i += blockDim.x) {
+      sUBlk[i] = a.gb_blk[(long long)g * a.gb_cap + i];
+      sUSlot[i] = a.gb_slot[(long long)g * a.gb_cap + i];
+    }
+    ntiles = (nub + 1) / 2;
+    njobs = ntiles * geff;
+  }
   __syncthreads();
+  if constexpr (MODE == IDX_GROUPED) {
+    bool any = false;
+    for (int ql = 0; ql < C::NQ; ++ql) any |= sQt[ql] >= 0;
+    if (!any) njobs = ntiles = 0;
+  }
   if constexpr (MODE == IDX_GATHER) {
     for (int ql = 0; ql < nq; ++ql) {
       int nb = 0;
@@ -218,6 +266,12 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
         mbar_arrive_expect_tx(qfull, geff * C::QS * H * C::ROWB);
         for (int g = 0; g < geff; ++g)
           tma_load_2d(sQ + g * C::QS * H * C::ROWB, &qmap, qfull, 0, (q0 + g * C::QS) * H);
+      } else if constexpr (MODE == IDX_GROUPED) {
+        int nv = 0;
+        for (int ql = 0; ql < C::NQ; ++ql) nv += sQt[ql] >= 0;
+        mbar_arrive_expect_tx(qfull, nv * H * C::ROWB);
+        for (int ql = 0; ql < C::NQ; ++ql)   // absent queries leave their rows unset: their scores are dropped
+          if (sQt[ql] >= 0) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, sQt[ql] * H);
       } else {
         mbar_arrive_expect_tx(qfull, nq * H * C::ROWB);
         for (int ql = 0; ql < nq; ++ql) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, (q0 + ql) * H);
@@ -236,6 +290,12 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
         } else if constexpr (MODE == IDX_DECODE) {
           mbar_arrive_expect_tx(&kfull[st], C::KBYTES);
           tma_load_2d(dst, &kmap, &kfull[st], 0, seq * a.n_k + (tile0 + i) * 128);
+        } else if constexpr (MODE == IDX_GROUPED) {
+          const int b0 = sUBlk[2 * i];
+          const int b1 = (2 * i + 1 < 2 * ntiles && 2 * i + 1 < a.gb_n[blockIdx.x]) ? sUBlk[2 * i + 1] : -1;
+          mbar_arrive_expect_tx(&kfull[st], (b1 >= 0 ? 2 : 1) * 64 * C::ROWB);
+          tma_load_2d(dst, &kmap, &kfull[st], 0, b0 * 64);
+          if (b1 >= 0) tma_load_2d(dst + 64 * C::ROWB, &kmap, &kfull[st], 0, b1 * 64);
         } else {
           const int* kr = gc.row();
           const int b0 = kr[2 * gc.pair];
@@ -263,7 +323,7 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
         if constexpr (MODE == IDX_GATHER) gc.init(sKept, C::KEEPMAX, 0, nq);
         for (int j = 0; j < njobs; ++j) {
           int tile, g;
-          if constexpr (MODE == IDX_PREFILL) {
+          if constexpr (C::WIDE) {
             tile = j / geff;
             g = j % geff;
           } else {
@@ -272,7 +332,7 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
           }
           const int st = tile % C::NS;
           const int buf = j % C::NBUF, ub = j / C::NBUF;
-          if (g == 0 || MODE != IDX_PREFILL) {
+          if (g == 0 || !C::WIDE) {
             if (!mbar_wait(&kfull[st], (tile / C::NS) & 1, wc, 3)) break;
           }
           if (!mbar_wait(&tempty[buf], (ub & 1) ^ 1, wc, 4)) break;
@@ -294,7 +354,7 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
               mma_bf16(d_tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
           }
           mma_commit(&tfull[buf]);
-          if (MODE != IDX_PREFILL || g == geff - 1) mma_commit(&kempty[st]);
+          if (!C::WIDE || g == geff - 1) mma_commit(&kempty[st]);
           if constexpr (MODE == IDX_GATHER) gc.next();
         }
       }
@@ -325,14 +385,20 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
       }
       k.ql = gc.ql;
       k.pair = gc.pair;
-      if constexpr (MODE == IDX_PREFILL) {
+      if constexpr (C::WIDE) {
         k.tile = jj / geff;
         k.g = jj % geff;
       } else {
         k.tile = jj;
         k.g = (MODE == IDX_GATHER) ? k.ql : 0;
       }
-      if constexpr (MODE == IDX_GATHER) {
+      if constexpr (MODE == IDX_GROUPED) {
+        const int ub = 2 * k.tile + (row >> 6);
+        const int blk = (jj < njobs && ub < a.gb_n[blockIdx.x]) ? sUBlk[ub] : -1;
+        k.s = blk * 64 + (row & 63);
+        k.kvalid = blk >= 0 && k.s < a.n_k;
+        k.col = ub;                          // the union block: each query's slot of it is looked up per query
+      } else if constexpr (MODE == IDX_GATHER) {
         const int slot = 2 * k.pair + (row >> 6);
         const int blk = (k.ql < nq) ? sKept[k.ql * C::KEEPMAX + slot] : -1;
         k.s = blk * 64 + (row & 63);
@@ -447,12 +513,21 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
 #pragma unroll
       for (int qq = 0; qq < C::QS; ++qq) {
         int t;
-        if constexpr (MODE == IDX_PREFILL)
+        int gcol = 0;                          // grouped: the query's candidate column of this key
+        if constexpr (MODE == IDX_PREFILL) {
           t = q0 + g * C::QS + qq;
-        else if constexpr (MODE == IDX_DECODE)
+        } else if constexpr (MODE == IDX_DECODE) {
           t = seq;
-        else
+        } else if constexpr (MODE == IDX_GROUPED) {
+          const int ql = g * C::QS + qq;
+          t = sQt[ql];
+          if (t < 0 || cur.s < 0) continue;    // absent query, or no union block in this half
+          const int slot = (int)((sUSlot[col] >> (8 * ql)) & 0xFFu);
+          if (slot == 0xFF) continue;          // the query did not keep this block
+          gcol = slot * 64 + (row & 63);
+        } else {
           t = q0 + ql;
+        }
         if (t >= a.n_q) continue;
         bool vis;
         if constexpr (MODE == IDX_DECODE)
@@ -490,6 +565,8 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
         }
         if constexpr (MODE == IDX_GATHER) {
           a.out[(long long)t * a.ld + col] = score;
+        } else if constexpr (MODE == IDX_GROUPED) {
+          a.out[(long long)t * a.ld + gcol] = score;
         } else {
           if (col < a.n_k) a.out[(long long)t * a.ld + col] = score;
         }
@@ -513,7 +590,7 @@ static cudaError_t launch_t(const void* q, const void* k, int q_rows, long long 
   const CUtensorMapDataType dt = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const CUtensorMapSwizzle sw = (C::ROWB == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   const uint32_t qbox = (MODE == IDX_PREFILL) ? C::QS * H : H;
-  const uint32_t kbox = (MODE == IDX_GATHER) ? 64 : 128;
+  const uint32_t kbox = (MODE == IDX_GATHER || MODE == IDX_GROUPED) ? 64 : 128;
   if (!make_tmap_2d(&qm, q, dt, D, (uint64_t)q_rows * H, C::ROWB, D, qbox, sw)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&km, k, dt, D, (uint64_t)k_rows, C::ROWB, D, kbox, sw)) return cudaErrorInvalidValue;
   auto kern = indexer_kernel<H, D, FP8, MODE>;
@@ -524,6 +601,8 @@ static cudaError_t launch_t(const void* q, const void* k, int q_rows, long long 
     grid = dim3((a.n_q + C::NQ - 1) / C::NQ);
   else if constexpr (MODE == IDX_DECODE)
     grid = dim3(((a.n_k + 127) / 128 + a.tiles_per_cta - 1) / a.tiles_per_cta, a.n_q);
+  else if constexpr (MODE == IDX_GROUPED)
+    grid = dim3(a.n_groups);
   else
     grid = dim3((a.n_q + C::NQ - 1) / C::NQ);
   if (grid.x == 0 || grid.y == 0) return cudaSuccess;
@@ -538,6 +617,7 @@ cudaError_t launch_indexer(int mode, int heads, int d, sa_dtype dt, const void* 
     if (mode == IDX_PREFILL) return launch_t<H_, D_, F_, IDX_PREFILL>(q, k, q_rows, k_rows, a, st); \
     if (mode == IDX_DECODE) return launch_t<H_, D_, F_, IDX_DECODE>(q, k, q_rows, k_rows, a, st);   \
     if (mode == IDX_GATHER) return launch_t<H_, D_, F_, IDX_GATHER>(q, k, q_rows, k_rows, a, st);   \
+    if (mode == IDX_GROUPED) return launch_t<H_, D_, F_, IDX_GROUPED>(q, k, q_rows, k_rows, a, st); \
   }
 #define SA_IDX_CASE_PREFILL(H_, D_, F_)                                                            \
   if (heads == H_ && d == D_ && (dt == SA_FP8_E4M3) == F_ && mode == IDX_PREFILL)                  \

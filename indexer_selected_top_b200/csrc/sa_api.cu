@@ -103,6 +103,7 @@ struct PrefillPlan {
   int m, n_s, cap, fb;   // stream: sample stride and count, list capacity, fallback rows per batch
   size_t off_table, off_idx, off_blk, off_blks, off_bsc, off_kept, off_cand, off_perm, total;
   size_t off_sel, off_ulist, off_umask, off_unl;   // two-stage: group union lists
+  size_t off_gbn, off_gbblk, off_gbslot;            // two-stage: group unions of kept blocks
   int n_groups, ucap;
   size_t off_ks, off_kss, off_stab, off_theta, off_cnt, off_list, off_miss, off_rows, off_count, off_pos;
   size_t off_fq, off_fqs, off_fw, off_ftab;
@@ -193,6 +194,12 @@ static bool plan_prefill(const sa_indexer_in* in, const sa_prefill_opts* o, Pref
     off += align256((size_t)p->n_groups * p->ucap * 4);
     p->off_umask = off;
     off += align256((size_t)p->n_groups * p->ucap);
+    p->off_gbn = off;
+    off += align256((size_t)p->n_groups * 4);
+    p->off_gbblk = off;
+    off += align256((size_t)p->n_groups * group_blocks_cap() * 4);
+    p->off_gbslot = off;
+    off += align256((size_t)p->n_groups * group_blocks_cap() * 8);
     p->off_unl = off;
     off += align256((size_t)p->n_groups * 4);
   }
@@ -570,10 +577,20 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
         e = launch_block_select(bsc, R, p.nb, std::max(p.nb, 1), ci.q_pos0, o->block_size, o->keep_blocks, kept,
                                 stream);
       if (e != cudaSuccess) return cuda_status(e);
-      // attention groups: queries that keep the same blocks side by side
-      e = launch_group_queries(kept, o->keep_blocks, R, ci.q_pos0, o->block_size,
-                               reinterpret_cast<int*>(w + p.off_perm), stream);
+      // groups of queries that keep the same blocks, and each group's union
+      // of kept blocks (stage 2 scores a union block once for the group)
+      int* perm = reinterpret_cast<int*>(w + p.off_perm);
+      int* gbn = reinterpret_cast<int*>(w + p.off_gbn);
+      int* gbblk = reinterpret_cast<int*>(w + p.off_gbblk);
+      unsigned long long* gbslot = reinterpret_cast<unsigned long long*>(w + p.off_gbslot);
+      e = launch_group_queries(kept, o->keep_blocks, R, ci.q_pos0, o->block_size, perm, stream);
       if (e != cudaSuccess) return cuda_status(e);
+      const bool grouped = o->test_hook != SA_HOOK_ATTN_UNGROUPED && in->n_k <= kUnionMaxKeys;
+      if (grouped) {
+        e = launch_group_blocks(kept, o->keep_blocks, perm, group_perm_len(R), R, in->n_k, gbn, gbblk, gbslot,
+                                stream);
+        if (e != cudaSuccess) return cuda_status(e);
+      }
       // stage 2: the visible keys of the kept blocks
       sm.mark(3, stream);
       IdxArgs a = base_args(&ci, status, o->test_hook);
@@ -581,7 +598,14 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
       a.ld = ncand;
       a.kept = kept;
       a.keep = o->keep_blocks;
-      e = launch_indexer(IDX_GATHER, in->n_heads, in->d_idx, in->dtype, ci.q, in->k, R, in->n_k, a, stream);
+      a.perm = perm;
+      a.gb_n = gbn;
+      a.gb_blk = gbblk;
+      a.gb_slot = gbslot;
+      a.gb_cap = group_blocks_cap();
+      a.n_groups = p.n_groups;
+      e = launch_indexer(grouped ? IDX_GROUPED : IDX_GATHER, in->n_heads, in->d_idx, in->dtype, ci.q, in->k, R,
+                         in->n_k, a, stream);
       if (e != cudaSuccess) return cuda_status(e);
       sm.mark(4, stream);
       uint32_t* sel = reinterpret_cast<uint32_t*>(w + p.off_sel);

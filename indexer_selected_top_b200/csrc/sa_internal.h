@@ -8,7 +8,7 @@
 
 namespace sa {
 
-enum IdxMode { IDX_PREFILL = 0, IDX_DECODE = 1, IDX_GATHER = 2 };
+enum IdxMode { IDX_PREFILL = 0, IDX_DECODE = 1, IDX_GATHER = 2, IDX_GROUPED = 3 };
 
 // Arguments of the indexer kernel (plain device pointers and sizes).
 struct IdxArgs {
@@ -25,6 +25,15 @@ struct IdxArgs {
   int tiles_per_cta;     // decode: key tiles per CTA
   const int* kept;       // gather: [n_q, keep] kept block ids, ascending, -1 padded
   int keep;
+  // grouped (two-stage stage 2 over groups of queries): the group's queries
+  // (perm), and per group its union blocks (ascending) with every query's
+  // slot of each (byte q of gb_slot; 0xFF: not kept), gb_cap entries per group
+  const int* perm;
+  const int* gb_n;
+  const int* gb_blk;
+  const unsigned long long* gb_slot;
+  int gb_cap;
+  int n_groups;
   uint32_t* status;      // device [error, site] or null
   long long budget;      // wait budget in clock cycles
   int hook;
@@ -95,6 +104,12 @@ cudaError_t launch_group_queries(const int* kept, int keep, int n_q, int q_pos0,
 cudaError_t launch_attention_grouped(const void* q, const void* kc, const void* vc, const int32_t* idx,
                                      const int* perm, int n_perm, int n_q, int k, int n_k, int hq, int dh,
                                      float scale, void* out, float* lse, bool ungrouped, cudaStream_t st);
+
+// union of the kept blocks of each group (ascending) with every query's slot
+// of each union block; cap = entries per group (kGroupQueries * keep at most)
+int group_blocks_cap();
+cudaError_t launch_group_blocks(const int* kept, int keep, const int* perm, int n_perm, int n_q, int n_k, int* gb_n,
+                                int* gb_blk, unsigned long long* gb_slot, cudaStream_t st);
 
 // union of each group's index sets (two-stage rows: kept blocks + selection
 // bitmaps) as ascending key lists in whole chunks of 64, with per-key masks of

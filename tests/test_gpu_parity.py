@@ -268,27 +268,37 @@ def test_prefill_two_stage_small(sa):
 
 
 def test_prefill_attention_grouped_and_per_query_schedules(sa):
-    """The grouped prefill attention (runs of 8 queries sharing one gather of
-    their union of keys) and its one-query-at-a-time schedule both match the
-    oracle's attention over the same index rows, on a ragged two-stage chunking
-    (windows of queries that end mid-group) and on FLAT query order."""
+    """The grouped two-stage schedule (stage 2 scoring each union block once
+    for 8 queries, attention over each group's union of keys on the tensor
+    cores) and the per-query schedule both give a valid exact top-k and the
+    oracle's attention over their own index rows, on a ragged chunking
+    (windows of queries that end mid-group); FLAT query order too. The two
+    schedules sum the heads in different orders, so near-ties at the cut may
+    resolve differently: each is judged against the oracle's scores."""
     wl = WORKLOADS["two_stage_t64k"].with_(T=6000, k=512)
     inp = PrefillInputs(wl, "cuda", seed=8)
     host = inp.to_host()
     rows = sample_rows(wl.T, 60, seed=8, k=512, extra=(0, 1, 1499, 1500, 2047, 2048, 5999))
-    outs = {}
-    for name, hook, chunk in (("grouped", 0, 1500), ("per_query", sa.SA_HOOK_ATTN_UNGROUPED, 1500)):
+    kept_gpu = _two_stage_kept_sets(sa, inp, 64 * 64)
+    ii = oracle.indexer.IndexerInputs(host)
+    sets = {}
+    for name, hook in (("grouped", 0), ("per_query", sa.SA_HOOK_ATTN_UNGROUPED)):
         pre = sa.Prefill(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, 512,
-                         mode="two_stage", chunk_rows=chunk, test_hook=hook)
+                         mode="two_stage", chunk_rows=1500, test_hook=hook)
         out, lse, idx = pre()
         torch.cuda.synchronize()
-        outs[name] = (out.float().cpu().numpy(), lse.cpu().numpy(), idx.cpu().numpy())
-    # the same index sets (the order inside a row is not specified)
-    assert np.array_equal(np.sort(outs["grouped"][2], axis=1), np.sort(outs["per_query"][2], axis=1))
-    att = attention_rows(host, {t: outs["grouped"][2][t] for t in rows})
-    for name, (out, lse, _) in outs.items():
+        out, lse, idx = out.float().cpu().numpy(), lse.cpu().numpy(), idx.cpu().numpy()
+        for t in rows:
+            cand = oracle.two_stage_candidates(kept_gpu[t], t, 64)
+            sc = oracle.scores_row(oracle.indexer.dequant(ii.q[t]), ii.sq[t], ii.kv[cand], ii.sk[cand], ii.w[t])
+            check_topk_row(idx[t], cand, sc, 512, f"{name} row {t}")
+        att = attention_rows(host, {t: idx[t] for t in rows})
         for t in rows:
             check_attention_row(out[t], att[t][0], lse[t], att[t][1], f"{name} row {t}")
+        sets[name] = np.sort(idx, axis=1)
+    # the schedules differ at most in near-ties, on few rows
+    n_diff = int((sets["grouped"] != sets["per_query"]).any(axis=1).sum())
+    assert n_diff <= wl.T // 50, n_diff
     wl = WORKLOADS["tiny_t512"]
     _check_prefill(sa, wl, 9, range(0, wl.T, 7), hook=sa.SA_HOOK_ATTN_UNGROUPED)
     _check_prefill(sa, wl, 9, range(0, wl.T, 7))
