@@ -3,26 +3,30 @@
 // A group of 8 queries x 16 query heads is one M = 128 tile: rows r =
 // 16 * query + head, so the two contractions of attention over the group's
 // shared keys are dense MMAs with the accumulators in tensor memory:
-//   S = Q K^T   (M 128 rows, N 64 keys, K 128 dims)   -> TMEM, two buffers
-//   O += P V    (M 128 rows, N 128 dims, K 64 keys)   -> TMEM
+//   S = Q K^T   (M 128 rows, N 128 keys, K 128 dims)  -> TMEM, two buffers
+//   O += P V    (M 128 rows, N 128 dims, K 128 keys)  -> TMEM
+// Q and P are the MMAs' A operands and live in tensor memory too (Q loaded
+// once per group, P written by the softmax over the S columns it has read),
+// so shared memory only carries the gathered K and V rows.
 // Every query still attends only to its own index set J_t (Latent Sparse
 // Attention section 3.2): the keys of a chunk come from the union of the
 // group's sets, and a per-key byte mask says which of the 8 queries selected
 // each one. The mask is applied by the tensor core itself (16 extra K dims,
 // see TC_MASK_BF16): keys a row's query did not select get a logit below
-// -2^99 and a softmax weight of exactly 0, so the row's softmax runs over J_t. The union lists (ascending keys, whole
-// chunks of 64, padded with -1 / mask 0) come from group_union_kernel.
+// -2^99 and a softmax weight of exactly 0, so the row's softmax runs over J_t.
+// The union lists (ascending keys, padded with -1 / mask 0 to whole chunks)
+// come from group_union_kernel.
 //
 // Roles (288 threads): warp 0 allocates TMEM and one lane issues the MMAs;
-// warps 1-4 gather whole chunks of K and V rows in turn (16-byte cp.async,
-// whole rows per 16 lanes) into 128-byte-swizzled tiles, publishing each on
-// an mbarrier that completes when the copies land; warps 5-8 run the
-// softmax, one thread per row (TMEM lane); P enters the MMA in bf16 while the row sum l
-// (and with it lse) is kept in fp32. The softmax keeps a running max per row and
-// rescales the O row in TMEM only when the max grows by more than 2^8, so P
-// stays below 256 and the final O / l uses one consistent reference.
+// warps 1-4 gather 32 keys each of every chunk (16-byte cp.async, whole rows
+// per 16 lanes) into 128-byte-swizzled tiles, publishing them on an mbarrier
+// that completes when the copies land; warps 5-8 run the softmax, one thread
+// per row (TMEM lane): a pass for the row max, then a pass writing P in bf16
+// while the row sum l (and with it lse) is kept in fp32. The running max is
+// lazy: the O row is rescaled in TMEM only when the max grows by more than
+// 2^8, so P stays below 256 and the final O / l uses one consistent reference.
 // K/V tiles: each 256-byte row is split into two 128-byte halves (dims 0-63,
-// 64-127), each half a [64 keys x 128 B] SW128 tile. For S the K tile is a
+// 64-127), each half a [128 keys x 128 B] SW128 tile. For S the K tile is a
 // K-major B operand; for O the same V tiles are an MN-major B operand (dims
 // contiguous), 8 keys per 1024-byte swizzle atom.
 #include <cuda_bf16.h>
@@ -37,13 +41,15 @@ constexpr int TC_GA = 8;               // queries per group
 constexpr int TC_HQ = 16;
 constexpr int TC_DH = 128;
 constexpr int TC_ROWS = TC_GA * TC_HQ; // 128
-constexpr int TC_CH = 64;              // keys per chunk
-constexpr int TC_ST = 4;               // K/V ring stages
-constexpr int TC_NSB = 3;              // S accumulators in TMEM (S = Q K^T runs ahead of O += P V)
-constexpr int TC_NPB = 3;              // P buffers in shared memory
-constexpr int TC_LW = 4;               // loader warps
+constexpr int TC_CH = kUnionChunk;     // keys per chunk (the union lists are padded to whole chunks)
+constexpr int TC_ST = 3;               // K/V ring stages
+constexpr int TC_LW = 4;               // loader warps (32 keys of every chunk each)
 constexpr int TC_THREADS = 32 * (1 + TC_LW + 4);
-constexpr int TC_O_COL = TC_NSB * TC_CH;   // TMEM column of O
+// tensor memory columns
+constexpr int TC_O_COL = 0;                        // O: 128 fp32 columns
+constexpr int TC_S_COL = TC_DH;                    // S buffers: 2 x 128 fp32 columns (P overwrites the first 64)
+constexpr int TC_Q_COL = TC_S_COL + 2 * TC_CH;     // Q: 128 dims as 64 columns of bf16 pairs
+constexpr int TC_QX_COL = TC_Q_COL + TC_DH / 2;    // Q mask dims: 16 dims as 8 columns
 constexpr float TC_RESCALE = 8.0f;     // log2 growth of the row max that forces a rescale
 // The mask enters S through the MMA: Q gets 16 extra dims holding a one-hot
 // of the row's query, K gets 16 extra dims holding -2^100 (bf16 0xF180) for
@@ -82,22 +88,17 @@ __device__ __forceinline__ uint64_t umma_desc_noswz(uint32_t saddr, uint32_t lbo
 }
 
 struct TcSmem {
-  static constexpr int Q_HALF = TC_ROWS * 128;            // 16 KB
-  static constexpr int KV_HALF = TC_CH * 128;             // 8 KB
-  static constexpr int QX = TC_ROWS * 32;                 // Q mask dims: [2 halves][128 rows][16 B]
-  static constexpr int KX = TC_CH * 32;                   // K mask dims: [2 halves][64 keys][16 B]
-  static constexpr int STAGE = 4 * KV_HALF + 1024 * ((KX + 1023) / 1024);   // K0 K1 V0 V1 KX
-  static constexpr int P_BYTES = TC_ROWS * 128;           // 128 rows x 64 keys bf16
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_QX = OFF_Q + 2 * Q_HALF;
-  static constexpr int OFF_KV = OFF_QX + 1024 * ((QX + 1023) / 1024);
-  static constexpr int OFF_P = OFF_KV + TC_ST * STAGE;
-  static constexpr int OFF_BAR = OFF_P + TC_NPB * P_BYTES;
-  // full[ST] empty[ST] sfull[NSB] sfree[NSB] pfull[NPB] pvdone[NPB] qfull drain
-  static constexpr int N_BAR = 2 * TC_ST + 2 * TC_NSB + 2 * TC_NPB + 2;
+  static constexpr int KV_HALF = TC_CH * 128;             // 16 KB: 128 keys x 64 dims
+  static constexpr int KX = TC_CH * 32;                   // K mask dims: [2 halves][128 keys][16 B]
+  static constexpr int STAGE = 4 * KV_HALF + KX;          // K0 K1 V0 V1 KX = 68 KB
+  static constexpr int OFF_KV = 0;
+  static constexpr int OFF_BAR = OFF_KV + TC_ST * STAGE;
+  // full[ST] empty[ST] sfull[2] pfull[2] pvdone[2] qfull drain
+  static constexpr int N_BAR = 2 * TC_ST + 8;
   static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
   static constexpr int SMEM = OFF_MISC + 64 + 1024;      // + slack for 1024-byte alignment
   static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
 };
 
 __global__ void __launch_bounds__(TC_THREADS, 1)
@@ -113,10 +114,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t* full = bars;
   uint64_t* empty = full + TC_ST;
   uint64_t* sfull = empty + TC_ST;
-  uint64_t* sfree = sfull + TC_NSB;
-  uint64_t* pfull = sfree + TC_NSB;
-  uint64_t* pvdone = pfull + TC_NPB;
-  uint64_t* qfull = pvdone + TC_NPB;
+  uint64_t* pfull = sfull + 2;
+  uint64_t* pvdone = pfull + 2;
+  uint64_t* qfull = pvdone + 2;
   uint64_t* drain = qfull + 1;
   uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L::OFF_MISC);
   uint32_t* tmem_slot = misc;
@@ -132,14 +132,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < TC_ST; ++s) {
-      mbar_init(&full[s], 32);
+      mbar_init(&full[s], 32 * TC_LW);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < TC_NSB; ++b) {
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&sfull[b], 1);
-      mbar_init(&sfree[b], 128);
-    }
-    for (int b = 0; b < TC_NPB; ++b) {
       mbar_init(&pfull[b], 128);
       mbar_init(&pvdone[b], 1);
     }
@@ -161,50 +158,49 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   if (warp == 0) {
     // ============================ MMA issuer ============================
-    // S = Q K^T of chunk i goes to S buffer i % NSB as soon as the chunk has
-    // landed and the softmax has read that buffer's previous chunk, so it
-    // runs up to NSB - 1 chunks ahead of O += P V
+    // S(i) = Q K^T of chunk i into S buffer i % 2 (Q and its mask dims read
+    // from tensor memory); O += P(j) V(j) with P read from the S buffer the
+    // softmax overwrote. S(j + 1) is issued before O += P(j) V(j), once the
+    // buffer's previous P has been consumed.
     if (lane == 0 && nch > 0) {
       constexpr uint32_t idesc_s = umma_idesc<1, 128, TC_CH>();
       constexpr uint32_t idesc_o = umma_idesc_bmn<1, 128, TC_DH>();
-      const uint32_t q_base = smem_u32(sm + L::OFF_Q);
-      const uint64_t qx_desc = umma_desc_noswz(smem_u32(sm + L::OFF_QX), L::QX / 2, 128);
-      int n_s = 0;                          // S products issued
-      auto issue_s = [&]() -> bool {
-        const int i = n_s, s = i % TC_ST, b = i % TC_NSB;
+      auto issue_s = [&](int i) -> bool {
+        const int s = i % TC_ST, b = i & 1;
         if (!mbar_wait(&full[s], (i / TC_ST) & 1, wc, 40)) return false;
-        if (i >= TC_NSB && !mbar_wait(&sfree[b], ((i / TC_NSB) - 1) & 1, wc, 41)) return false;
+        if (i >= 2 && !mbar_wait(&pvdone[b], ((i - 2) >> 1) & 1, wc, 41)) return false;
         tc_fence_after();
         const uint32_t k_base = smem_u32(sm + L::OFF_KV + s * L::STAGE);
+        const uint32_t d = tmem + TC_S_COL + b * TC_CH;
 #pragma unroll
         for (int kk = 0; kk < TC_DH / 16; ++kk) {
-          const uint64_t ad = umma_smem_desc<128>(q_base + (kk >> 2) * L::Q_HALF + (kk & 3) * 32);
           const uint64_t bd = umma_smem_desc<128>(k_base + (kk >> 2) * L::KV_HALF + (kk & 3) * 32);
-          mma_bf16(tmem + b * TC_CH, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          mma_bf16_ts(d, tmem + TC_Q_COL + kk * 8, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
         // the mask dims: one more K step adds the -2^100 bias where the row's query did not select the key
-        mma_bf16(tmem + b * TC_CH, qx_desc, umma_desc_noswz(k_base + 4 * L::KV_HALF, L::KX / 2, 128), idesc_s, 1u);
+        mma_bf16_ts(d, tmem + TC_QX_COL, umma_desc_noswz(k_base + 4 * L::KV_HALF, L::KX / 2, 128), idesc_s, 1u);
         mma_commit(&sfull[b]);
-        ++n_s;
         return true;
       };
       bool ok = mbar_wait(qfull, 0, wc, 42);
-      if (ok) tc_fence_after();
+      if (ok) {
+        tc_fence_after();
+        ok = issue_s(0);
+      }
       for (int j = 0; ok && j < nch; ++j) {
-        while (ok && n_s < nch && n_s < j + TC_NSB) ok = issue_s();
-        if (!ok || !mbar_wait(&pfull[j % TC_NPB], (j / TC_NPB) & 1, wc, 43)) break;
+        if (j + 1 < nch && !issue_s(j + 1)) break;
+        if (!mbar_wait(&pfull[j & 1], (j >> 1) & 1, wc, 43)) break;
         tc_fence_after();
         const uint32_t v_base = smem_u32(sm + L::OFF_KV + (j % TC_ST) * L::STAGE + 2 * L::KV_HALF);
-        const uint32_t p_base = smem_u32(sm + L::OFF_P + (j % TC_NPB) * L::P_BYTES);
+        const uint32_t p_col = tmem + TC_S_COL + (j & 1) * TC_CH;
 #pragma unroll
         for (int kk = 0; kk < TC_CH / 16; ++kk) {
-          const uint64_t ad = umma_smem_desc<128>(p_base + kk * 32);
-          // 16 keys = two 8-key atoms of 1024 B; the two 64-dim halves 8 KB apart
+          // 16 keys = two 8-key atoms of 1024 B; the two 64-dim halves 16 KB apart
           const uint64_t bd = umma_desc_sw128(v_base + kk * 2048, L::KV_HALF, 1024);
-          mma_bf16(tmem + TC_O_COL, ad, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + TC_O_COL, p_col + kk * 8, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&empty[j % TC_ST]);
-        mma_commit(&pvdone[j % TC_NPB]);
+        mma_commit(&pvdone[j & 1]);
       }
       // every MMA issued has completed before tensor memory is released
       mma_commit(drain);
@@ -212,67 +208,57 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
   } else if (warp <= TC_LW) {
     // ============================ K/V gather ============================
-    // loader warp lw owns chunks lw, lw + TC_LW, ...: it gathers a whole
-    // chunk, writes its mask dims, and publishes it without waiting (the
-    // barrier phase completes once the copies have landed). The next chunk's
-    // keys and masks are read before waiting for its ring stage.
+    // loader warp lw gathers keys [32 lw, 32 lw + 32) of every chunk and
+    // their mask dims, and publishes them without waiting (the barrier phase
+    // completes once all loaders' copies have landed). The next chunk's keys
+    // and masks are read before waiting for its ring stage.
     const int lw = warp - 1;
     const int seg = lane & 15, half = seg >> 3, c16 = seg & 7;
-    int k_lo = 0, k_hi = 0;
-    uint32_t m_lo = 0u, m_hi = 0u;
-    if (lw < nch) {
-      k_lo = glist[lw * TC_CH + lane];
-      k_hi = glist[lw * TC_CH + 32 + lane];
-      m_lo = gmask[lw * TC_CH + lane];
-      m_hi = gmask[lw * TC_CH + 32 + lane];
+    int key = 0;
+    uint32_t msk = 0u;
+    if (nch > 0) {
+      key = glist[lw * 32 + lane];
+      msk = gmask[lw * 32 + lane];
     }
-    for (int j = lw; j < nch; j += TC_LW) {
+    for (int j = 0; j < nch; ++j) {
       const int s = j % TC_ST;
-      const int jn = j + TC_LW;
-      int n_klo = 0, n_khi = 0;
-      uint32_t n_mlo = 0u, n_mhi = 0u;
-      if (jn < nch) {
-        n_klo = glist[jn * TC_CH + lane];
-        n_khi = glist[jn * TC_CH + 32 + lane];
-        n_mlo = gmask[jn * TC_CH + lane];
-        n_mhi = gmask[jn * TC_CH + 32 + lane];
+      int n_key = 0;
+      uint32_t n_msk = 0u;
+      if (j + 1 < nch) {
+        n_key = glist[(j + 1) * TC_CH + lw * 32 + lane];
+        n_msk = gmask[(j + 1) * TC_CH + lw * 32 + lane];
       }
       if (j >= TC_ST && !mbar_wait(&empty[s], ((j / TC_ST) - 1) & 1, wc, 44)) break;
-      k_lo = max(k_lo, 0);                    // padding (-1): any valid row, its mask byte is 0
-      k_hi = max(k_hi, 0);
+      const int kr = max(key, 0);                   // padding (-1): any valid row, its mask byte is 0
       uint8_t* st = sm + L::OFF_KV + s * L::STAGE;
-#pragma unroll 8
-      for (int i = 0; i < TC_CH / 2; ++i) {
-        const int r = 2 * i + (lane >> 4);
-        const int key = __shfl_sync(0xffffffffu, i < 16 ? k_lo : k_hi, r & 31);
-        const long long src = (long long)key * TC_DH + seg * 8;
+#pragma unroll 4
+      for (int i = 0; i < 16; ++i) {
+        const int rl = 2 * i + (lane >> 4);         // this warp's row
+        const int r = lw * 32 + rl;                 // row of the chunk
+        const long long src = (long long)__shfl_sync(0xffffffffu, kr, rl) * TC_DH + seg * 8;
         const uint32_t off = half * L::KV_HALF + r * 128 + ((c16 ^ (r & 7)) << 4);
         cp_async16(smem_u32(st + off), kc + src);
         cp_async16(smem_u32(st + 2 * L::KV_HALF + off), vc + src);
       }
-      // mask dims of keys lane and 32 + lane: dims 0-7 carry the bias for
-      // the queries that did not select the key, dims 8-15 are 0
-      uint8_t* kx = st + 4 * L::KV_HALF;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const uint32_t m = hh ? m_hi : m_lo;
+      // mask dims of this lane's key: dims 0-7 carry the bias for the
+      // queries that did not select it, dims 8-15 are 0
+      {
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const uint32_t lo = ((m >> (2 * e)) & 1u) ? 0u : TC_MASK_BF16;
-          const uint32_t hi = ((m >> (2 * e + 1)) & 1u) ? 0u : TC_MASK_BF16;
+          const uint32_t lo = ((msk >> (2 * e)) & 1u) ? 0u : TC_MASK_BF16;
+          const uint32_t hi = ((msk >> (2 * e + 1)) & 1u) ? 0u : TC_MASK_BF16;
           w[e] = lo | (hi << 16);
         }
-        const int key_row = hh * 32 + lane;
-        *reinterpret_cast<uint4*>(kx + key_row * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<uint4*>(kx + L::KX / 2 + key_row * 16) = make_uint4(0u, 0u, 0u, 0u);
+        uint8_t* kx = st + 4 * L::KV_HALF;
+        const int row = lw * 32 + lane;
+        *reinterpret_cast<uint4*>(kx + row * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(kx + L::KX / 2 + row * 16) = make_uint4(0u, 0u, 0u, 0u);
       }
       fence_proxy_async_smem();
       cp_async_publish(&full[s]);
-      k_lo = n_klo;
-      k_hi = n_khi;
-      m_lo = n_mlo;
-      m_hi = n_mhi;
+      key = n_key;
+      msk = n_msk;
     }
     cp_async_wait_all();   // no copy may land after the CTA has left
   } else {
@@ -283,51 +269,56 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int t = qt[qi];
     const uint32_t t_row = tmem + (uint32_t(qw * 32) << 16);
     {
-      // this row of the Q tile (two 128-byte halves, swizzled) and its mask dims
-      uint8_t* qa = sm + L::OFF_Q;
-      if (t >= 0) {
-        const __nv_bfloat16* src = q + ((long long)t * TC_HQ + h) * TC_DH;
+      // this row of Q (bf16 pairs: column c holds dims 2c, 2c + 1) and the
+      // one-hot of its query in the mask dims
+      uint32_t qv[32];
 #pragma unroll
-        for (int sg = 0; sg < 16; ++sg)
-          cp_async16(smem_u32(qa + (sg >> 3) * L::Q_HALF + r * 128 + (((sg & 7) ^ (r & 7)) << 4)), src + sg * 8);
-        cp_async_commit();
-        cp_async_wait<0>();
-      } else {
+      for (int hh = 0; hh < 2; ++hh) {
+        if (t >= 0) {
+          const uint4* src = reinterpret_cast<const uint4*>(q + ((long long)t * TC_HQ + h) * TC_DH + hh * 64);
 #pragma unroll
-        for (int sg = 0; sg < 16; ++sg)
-          *reinterpret_cast<uint4*>(qa + (sg >> 3) * L::Q_HALF + r * 128 + (((sg & 7) ^ (r & 7)) << 4)) =
-              make_uint4(0u, 0u, 0u, 0u);
+          for (int i = 0; i < 8; ++i) {
+            const uint4 v = src[i];
+            qv[4 * i] = v.x;
+            qv[4 * i + 1] = v.y;
+            qv[4 * i + 2] = v.z;
+            qv[4 * i + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) qv[i] = 0u;
+        }
+        tmem_st32(t_row + TC_Q_COL + hh * 32, *reinterpret_cast<const float(*)[32]>(qv));
       }
-      uint32_t w[4];
+      uint32_t qx[8];
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        w[e] = (qi == 2 * e ? 0x3F80u : 0u) | (qi == 2 * e + 1 ? 0x3F800000u : 0u);   // bf16 1.0 at dim qi
-      uint8_t* qx = sm + L::OFF_QX;
-      *reinterpret_cast<uint4*>(qx + r * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-      *reinterpret_cast<uint4*>(qx + L::QX / 2 + r * 16) = make_uint4(0u, 0u, 0u, 0u);
-      fence_proxy_async_smem();
+      for (int e = 0; e < 8; ++e)
+        qx[e] = (qi == 2 * e ? 0x3F80u : 0u) | (qi == 2 * e + 1 ? 0x3F800000u : 0u);   // bf16 1.0 at dim qi
+      tmem_st8(t_row + TC_QX_COL, qx);
+      tmem_st_wait();
+      tc_fence_before();
       mbar_arrive(qfull);
     }
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nch; ++j) {
-      const int b = j % TC_NSB, pb = j % TC_NPB;
-      ok = __all_sync(0xffffffffu, mbar_wait(&sfull[b], (j / TC_NSB) & 1, wc, 45));
+      const int b = j & 1;
+      const uint32_t s_row = t_row + TC_S_COL + b * TC_CH;
+      ok = __all_sync(0xffffffffu, mbar_wait(&sfull[b], (j >> 1) & 1, wc, 45));
       if (!ok) break;
       tc_fence_after();
-      float sv[TC_CH];
-      tmem_ld32(t_row + b * TC_CH, *reinterpret_cast<float(*)[32]>(sv));
-      tmem_ld32(t_row + b * TC_CH + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
-      tmem_ld_wait();
-      tmem_regs_ready(*reinterpret_cast<float(*)[32]>(sv));
-      tmem_regs_ready(*reinterpret_cast<float(*)[32]>(sv + 32));
-      tc_fence_before();
-      mbar_arrive(&sfree[b]);
-      // the row max over the chunk (masked keys sit below -2^99; the scale
-      // is positive, so it commutes with the max)
-      float mq[4] = {sv[0], sv[1], sv[2], sv[3]};
+      // pass 1: the row max over the chunk (masked keys sit below -2^99;
+      // the scale is positive, so it commutes with the max)
+      float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 4; c < TC_CH; ++c) mq[c & 3] = fmaxf(mq[c & 3], sv[c]);
+      for (int cb = 0; cb < TC_CH / 32; ++cb) {
+        float sv[32];
+        tmem_ld32(s_row + cb * 32, sv);
+        tmem_ld_wait();
+        tmem_regs_ready(sv);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) mq[c & 3] = fmaxf(mq[c & 3], sv[c]);
+      }
       float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
       mx = mx < TC_MASKED ? -INFINITY : mx * scale_log2;    // no key of the chunk is the row's
       const float m_new = fmaxf(m_used, mx);
@@ -335,8 +326,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (m_used == -INFINITY) m_used = m_new;          // the row's O is still 0
       if (__any_sync(0xffffffffu, resc)) {
         // O must hold every earlier chunk before it is rescaled in place
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(&pvdone[(j - 1) % TC_NPB], ((j - 1) / TC_NPB) & 1, wc, 47));
+        ok = __all_sync(0xffffffffu, mbar_wait(&pvdone[(j - 1) & 1], ((j - 1) >> 1) & 1, wc, 47));
         if (!ok) break;
         tc_fence_after();
         const float alpha = resc ? exp2f(m_used - m_new) : 1.f;
@@ -356,39 +346,37 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           m_used = m_new;
         }
       }
-      // P buffer pb is free once the O update of chunk j - NPB has completed
-      if (j >= TC_NPB) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&pvdone[pb], ((j / TC_NPB) - 1) & 1, wc, 48));
-        if (!ok) break;
-      }
-      uint8_t* prow = sm + L::OFF_P + pb * L::P_BYTES + (r >> 3) * 1024 + (r & 7) * 128;
-      // p = 2^(s * scale_log2 - m): one FMA and one ex2 per key; a masked
-      // key lands far below the normal range and gives exactly 0. A row with
-      // no valid key yet subtracts 0.
+      // pass 2: p = 2^(s * scale_log2 - m) (one FMA and one ex2 per key; a
+      // masked key lands far below the normal range and gives exactly 0),
+      // packed to bf16 pairs over the S columns already read: keys 32 cb ..
+      // 32 cb + 31 go to columns 16 cb .. 16 cb + 15
       const float msub = m_used == -INFINITY ? 0.f : m_used;
       float2 l2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int c8 = 0; c8 < TC_CH / 8; ++c8) {
-        uint32_t w[4];
+      for (int cb = 0; cb < TC_CH / 32; ++cb) {
+        float sv[32];
+        tmem_ld32(s_row + cb * 32, sv);
+        tmem_ld_wait();
+        tmem_regs_ready(sv);
+        uint32_t pw[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = ex2_approx(fmaf(sv[c8 * 8 + 2 * e], scale_log2, -msub));
-          const float p1 = ex2_approx(fmaf(sv[c8 * 8 + 2 * e + 1], scale_log2, -msub));
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2_approx(fmaf(sv[2 * e], scale_log2, -msub));
+          const float p1 = ex2_approx(fmaf(sv[2 * e + 1], scale_log2, -msub));
           const __nv_bfloat162 pv = __floats2bfloat162_rn(p0, p1);
           l2 = __fadd2_rn(l2, make_float2(p0, p1));      // the row sum in fp32, as lse needs
-          w[e] = *reinterpret_cast<const uint32_t*>(&pv);
+          pw[e] = *reinterpret_cast<const uint32_t*>(&pv);
         }
-        *reinterpret_cast<uint4*>(prow + ((c8 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        tmem_st16(s_row + cb * 16, pw);
       }
       l += l2.x + l2.y;
+      tmem_st_wait();
       tc_fence_before();
-      fence_proxy_async_smem();
-      mbar_arrive(&pfull[pb]);
+      mbar_arrive(&pfull[b]);
     }
     // epilogue: O / l in bf16, lse in natural log
     if (ok && nch > 0) {
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait(&pvdone[(nch - 1) % TC_NPB], ((nch - 1) / TC_NPB) & 1, wc, 49));
+      ok = __all_sync(0xffffffffu, mbar_wait(&pvdone[(nch - 1) & 1], ((nch - 1) >> 1) & 1, wc, 49));
       if (ok) {
         tc_fence_after();
         const float inv = l > 0.f ? 1.f / l : 0.f;

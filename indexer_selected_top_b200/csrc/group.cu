@@ -424,7 +424,7 @@ namespace sa {
 // The union of the group is built block-wise: the group's kept blocks in
 // ascending order (a bitmap over all blocks, ranked by popcount), a table of
 // each query's slot of every union block, then one mask byte per union key.
-int group_union_cap(int k) { return (GA * k + 63) / 64 * 64; }
+int group_union_cap(int k) { return (GA * k + kUnionChunk - 1) / kUnionChunk * kUnionChunk; }
 
 __global__ void __launch_bounds__(256) group_union_kernel(const int* __restrict__ kept, int keep,
                                                           const uint32_t* __restrict__ sel, const int* __restrict__ perm,
@@ -542,7 +542,7 @@ __global__ void __launch_bounds__(256) group_union_kernel(const int* __restrict_
       ++p;
     }
   }
-  for (int i = total + tid; i < (total + 63) / 64 * 64; i += 256) {
+  for (int i = total + tid; i < (total + kUnionChunk - 1) / kUnionChunk * kUnionChunk; i += 256) {
     gl[i] = -1;
     gm[i] = 0;
   }
@@ -552,7 +552,7 @@ __global__ void __launch_bounds__(256) group_union_kernel(const int* __restrict_
 cudaError_t launch_group_union(const int* kept, int keep, const uint32_t* sel, const int* perm, int n_perm, int n_q,
                                int n_k, int cap, int* list, uint8_t* lmask, int* n_list, cudaStream_t st) {
   if (n_q <= 0) return cudaSuccess;
-  if (keep <= 0 || keep > 64 || n_k > GK_MAX || cap % 64 != 0) return cudaErrorNotSupported;
+  if (keep <= 0 || keep > 64 || n_k > GK_MAX || cap % kUnionChunk != 0) return cudaErrorNotSupported;
   const int n_groups = ((perm ? n_perm : n_q) + GA - 1) / GA;
   group_union_kernel<<<n_groups, 256, 0, st>>>(kept, keep, sel, perm, n_q, n_k, cap, list, lmask, n_list);
   return cudaGetLastError();

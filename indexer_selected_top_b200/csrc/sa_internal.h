@@ -112,8 +112,10 @@ cudaError_t launch_group_blocks(const int* kept, int keep, const int* perm, int 
                                 int* gb_blk, unsigned long long* gb_slot, cudaStream_t st);
 
 // union of each group's index sets (two-stage rows: kept blocks + selection
-// bitmaps) as ascending key lists in whole chunks of 64, with per-key masks of
-// the group's queries; cap = list capacity per group (a multiple of 64)
+// bitmaps) as ascending key lists padded (-1, mask 0) to whole chunks of
+// kUnionChunk keys, with per-key masks of the group's queries; cap = list
+// capacity per group (a multiple of kUnionChunk)
+constexpr int kUnionChunk = 128;
 int group_union_cap(int k);
 cudaError_t launch_group_union(const int* kept, int keep, const uint32_t* sel, const int* perm, int n_perm, int n_q,
                                int n_k, int cap, int* list, uint8_t* lmask, int* n_list, cudaStream_t st);
