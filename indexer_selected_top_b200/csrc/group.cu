@@ -50,7 +50,12 @@ static __device__ __forceinline__ uint32_t block_hash(uint32_t b) {
 // order, -1 past n_q. The signature is the smallest hash over the query's
 // kept blocks, leaving out block 0 and the query's own block, which every
 // query keeps (HISA section 3: the first and the local block are always in).
-__global__ void __launch_bounds__(1024) group_queries_kernel(const int* __restrict__ kept, int keep, int n_q,
+// With `sel` (the top-k's selection bitmaps over the kept blocks' keys) only
+// the blocks holding at least min_sel selected keys count: the blocks a query
+// draws most of its keys from mark its neighbourhood better than the blocks
+// it kept at the margin.
+__global__ void __launch_bounds__(1024) group_queries_kernel(const int* __restrict__ kept, int keep,
+                                                             const uint32_t* __restrict__ sel, int min_sel, int n_q,
                                                              int q_pos0, int block, int* __restrict__ perm) {
   __shared__ unsigned long long key[GW];
   const int w0 = blockIdx.x * GW;
@@ -61,9 +66,11 @@ __global__ void __launch_bounds__(1024) group_queries_kernel(const int* __restri
       const int cur = (q_pos0 + t) / block;
       uint32_t h = 0xFFFFFFFFu;
       const int* kr = kept + (long long)t * keep;
+      const uint32_t* sr = sel ? sel + (long long)t * keep * 2 : nullptr;
       for (int j = 0; j < keep; ++j) {
         const int b = kr[j];
         if (b < 0) break;
+        if (sr != nullptr && __popc(sr[2 * j]) + __popc(sr[2 * j + 1]) < min_sel) continue;
         if (b != 0 && b != cur) h = min(h, block_hash((uint32_t)b));
       }
       k = ((unsigned long long)h << 32) | (uint32_t)t;
@@ -95,11 +102,11 @@ __global__ void __launch_bounds__(1024) group_queries_kernel(const int* __restri
 
 int group_perm_len(int n_q) { return (n_q + GW - 1) / GW * GW; }
 
-cudaError_t launch_group_queries(const int* kept, int keep, int n_q, int q_pos0, int block, int* perm,
-                                 cudaStream_t st) {
+cudaError_t launch_group_queries(const int* kept, int keep, const uint32_t* sel, int min_sel, int n_q, int q_pos0,
+                                 int block, int* perm, cudaStream_t st) {
   if (n_q <= 0) return cudaSuccess;
   if (keep <= 0 || block <= 0) return cudaErrorInvalidValue;
-  group_queries_kernel<<<(n_q + GW - 1) / GW, 1024, 0, st>>>(kept, keep, n_q, q_pos0, block, perm);
+  group_queries_kernel<<<(n_q + GW - 1) / GW, 1024, 0, st>>>(kept, keep, sel, min_sel, n_q, q_pos0, block, perm);
   return cudaGetLastError();
 }
 

@@ -104,6 +104,7 @@ struct PrefillPlan {
   size_t off_table, off_idx, off_blk, off_blks, off_bsc, off_kept, off_cand, off_perm, total;
   size_t off_sel, off_ulist, off_umask, off_unl;   // two-stage: group union lists
   size_t off_gbn, off_gbblk, off_gbslot;            // two-stage: group unions of kept blocks
+  size_t off_perm2;                                 // two-stage: attention groups (from the selections)
   int n_groups, ucap;
   size_t off_ks, off_kss, off_stab, off_theta, off_cnt, off_list, off_miss, off_rows, off_count, off_pos;
   size_t off_fq, off_fqs, off_fw, off_ftab;
@@ -184,6 +185,8 @@ static bool plan_prefill(const sa_indexer_in* in, const sa_prefill_opts* o, Pref
     p->off_cand = off;
     off += align256((size_t)R * o->keep_blocks * o->block_size * 4);
     p->off_perm = off;
+    off += align256((size_t)group_perm_len(R) * 4);
+    p->off_perm2 = off;
     off += align256((size_t)group_perm_len(R) * 4);
     // tensor-core attention of the groups' union lists
     p->n_groups = group_perm_len(R) / kGroupQueries;
@@ -583,7 +586,7 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
       int* gbn = reinterpret_cast<int*>(w + p.off_gbn);
       int* gbblk = reinterpret_cast<int*>(w + p.off_gbblk);
       unsigned long long* gbslot = reinterpret_cast<unsigned long long*>(w + p.off_gbslot);
-      e = launch_group_queries(kept, o->keep_blocks, R, ci.q_pos0, o->block_size, perm, stream);
+      e = launch_group_queries(kept, o->keep_blocks, nullptr, 0, R, ci.q_pos0, o->block_size, perm, stream);
       if (e != cudaSuccess) return cuda_status(e);
       const bool grouped = o->test_hook != SA_HOOK_ATTN_UNGROUPED && in->n_k <= kUnionMaxKeys;
       if (grouped) {
@@ -625,11 +628,18 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
       int* list = reinterpret_cast<int*>(w + p.off_ulist);
       uint8_t* lmask = reinterpret_cast<uint8_t*>(w + p.off_umask);
       int* nlist = reinterpret_cast<int*>(w + p.off_unl);
-      e = launch_group_union(reinterpret_cast<const int*>(w + p.off_kept), o->keep_blocks,
-                             reinterpret_cast<const uint32_t*>(w + p.off_sel), perm, group_perm_len(R), R, in->n_k,
-                             p.ucap, list, lmask, nlist, stream);
+      const int* kept = reinterpret_cast<const int*>(w + p.off_kept);
+      const uint32_t* sel = reinterpret_cast<const uint32_t*>(w + p.off_sel);
+      // attention groups: queries that draw most of their keys from the same
+      // blocks (a block counts when at least half of its keys were selected)
+      int* perm2 = reinterpret_cast<int*>(w + p.off_perm2);
+      e = launch_group_queries(kept, o->keep_blocks, sel, o->block_size / 2, R, ci.q_pos0, o->block_size, perm2,
+                               stream);
       if (e != cudaSuccess) return cuda_status(e);
-      e = launch_attention_tc(qa, at->k_cache, at->v_cache, list, lmask, nlist, perm, p.n_groups, R, p.ucap, scale,
+      e = launch_group_union(kept, o->keep_blocks, sel, perm2, group_perm_len(R), R, in->n_k, p.ucap, list, lmask,
+                             nlist, stream);
+      if (e != cudaSuccess) return cuda_status(e);
+      e = launch_attention_tc(qa, at->k_cache, at->v_cache, list, lmask, nlist, perm2, p.n_groups, R, p.ucap, scale,
                               oa, la, status, o->test_hook == SA_HOOK_STALL_WAIT ? kHookBudget : kWaitBudget,
                               stream);
     } else {
