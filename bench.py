@@ -113,6 +113,24 @@ def _isnum(s):
         return False
 
 
+# DRAM bytes per launch of a kernel from one ncu capture (read + write),
+# captured on the two-stage workload at T_cap rows and scaled to the run by
+# the number of candidate keys scored (the candidate scores are most of the
+# traffic). The capture and its command are summarised in profiles/; an entry
+# is removed when its kernel changes.
+MEASURED_DRAM = {
+    # stage2_indexer_two_stage.md: indexer_kernel<64, 128, 1, 3>, T = 16384
+    "stage2_indexer": {"bytes": 147.332352e6 + 188.291840e6, "T_cap": 16384},
+}
+
+
+def measured_traffic(kernel, wl):
+    m = MEASURED_DRAM.get(kernel)
+    if m is None or wl.mode != "two_stage":
+        return None
+    return round(m["bytes"] * two_stage_work(wl)["cand"] / two_stage_work(wl.with_(T=m["T_cap"]))["cand"])
+
+
 # ------------------------------------------------------- algorithmic work
 def two_stage_work(wl):
     """Data-independent algorithmic counts of the two-stage prefill."""
@@ -141,6 +159,7 @@ def flat_work(wl, streaming: bool):
         "indexer_flops": 2.0 * H * d * scores,
         "attn_pairs": pairs,
         "attn_bytes": pairs * 2 * wl.dh * 2,
+        "attn_flops": 4.0 * wl.Hq * wl.dh * pairs,
         # table path: the score table is read once by the selector (+ index rows written)
         "topk_bytes": 0 if streaming else scores * 4 + T * k * 4,
     }
@@ -323,8 +342,11 @@ def run_native(args, rank, world, local_rank):
             stages[n] = {"ms": round(ms, 4), "bound": "tensor", "achieved": work[flop_stage[n]] / s / 1e12,
                          "peak": fp8_peak, "unit": "TFLOP/s"}
         elif n == "attention":
-            stages[n] = {"ms": round(ms, 4), "bound": "hbm", "achieved": work["attn_bytes"] / s / 1e9,
-                         "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+            # the grouped kernels read each union key once per group of queries
+            # (from L2), so gathered bytes no longer bound them: the algorithmic
+            # work is the 4 Hq dh flops of every selected (query, key) pair
+            stages[n] = {"ms": round(ms, 4), "bound": "tensor", "achieved": work["attn_flops"] / s / 1e12,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
         elif n == "topk" and work["topk_bytes"] > 0:
             stages[n] = {"ms": round(ms, 4), "bound": "hbm", "achieved": work["topk_bytes"] / s / 1e9,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s"}
@@ -338,9 +360,9 @@ def run_native(args, rank, world, local_rank):
     roof = dict(stages[dom])
     roof.pop("ms")
     roof["kernel"] = dom
-    roof["traffic"] = None
-    roof["peak_source"] = (f"{peak_src}: " + ("2 x bf16 burst (nominal FP8/bf16 ratio)" if roof["unit"] == "TFLOP/s"
-                                              else "HBM copy"))
+    roof["traffic"] = measured_traffic(dom, wl)
+    roof["peak_source"] = (f"{peak_src}: " + ("2 x bf16 burst (nominal FP8/bf16 ratio)" if roof["peak"] == fp8_peak
+                                              else "bf16 burst" if roof["unit"] == "TFLOP/s" else "HBM copy"))
 
     decode = None
     if dec is not None:
@@ -399,7 +421,9 @@ def run_native(args, rank, world, local_rank):
                          f"attention), extrapolated to {wl.T} rows"}
 
     if wl.mode == "two_stage":
-        pre_launches = 6                       # pool, stage 1, keep, stage 2, top-k, attention
+        # pool, stage 1, keep, query groups, group block unions, stage 2, top-k,
+        # attention groups, group key unions, attention
+        pre_launches = 10
     elif wl.T <= 65536:
         pre_launches = 3                       # indexer (table), top-k, attention
     else:                                      # streaming: sample gathers once; per chunk sample scores,
