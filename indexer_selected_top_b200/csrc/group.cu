@@ -46,37 +46,42 @@ static __device__ __forceinline__ uint32_t block_hash(uint32_t b) {
   return x;
 }
 
+// The signature of query t: the smallest hash over its kept blocks, leaving
+// out block 0 and the query's own block, which every query keeps (HISA
+// section 3: the first and the local block are always in). With `sel` (the
+// top-k's selection bitmaps over the kept blocks' keys) only the blocks
+// holding at least min_sel selected keys count: the blocks a query draws most
+// of its keys from mark its neighbourhood better than the blocks it kept at
+// the margin. One warp per query: lane j reads kept slots j and j + 32.
+__global__ void __launch_bounds__(256) group_signature_kernel(const int* __restrict__ kept, int keep,
+                                                              const uint32_t* __restrict__ sel, int min_sel, int n_q,
+                                                              int q_pos0, int block,
+                                                              unsigned long long* __restrict__ sig) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (t >= n_q) return;
+  const int cur = (q_pos0 + t) / block;
+  uint32_t h = 0xFFFFFFFFu;
+  for (int j = lane; j < keep; j += 32) {
+    const int b = kept[(long long)t * keep + j];
+    bool use = b >= 0 && b != 0 && b != cur;
+    if (use && sel != nullptr) {
+      const uint32_t* sr = sel + (long long)t * keep * 2;
+      use = __popc(sr[2 * j]) + __popc(sr[2 * j + 1]) >= min_sel;
+    }
+    if (use) h = min(h, block_hash((uint32_t)b));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) h = min(h, __shfl_xor_sync(0xffffffffu, h, o));
+  if (lane == 0) sig[t] = ((unsigned long long)h << 32) | (uint32_t)t;
+}
+
 // perm[w * GW + i] = the query at rank i of window w in (signature, query)
-// order, -1 past n_q. The signature is the smallest hash over the query's
-// kept blocks, leaving out block 0 and the query's own block, which every
-// query keeps (HISA section 3: the first and the local block are always in).
-// With `sel` (the top-k's selection bitmaps over the kept blocks' keys) only
-// the blocks holding at least min_sel selected keys count: the blocks a query
-// draws most of its keys from mark its neighbourhood better than the blocks
-// it kept at the margin.
-__global__ void __launch_bounds__(1024) group_queries_kernel(const int* __restrict__ kept, int keep,
-                                                             const uint32_t* __restrict__ sel, int min_sel, int n_q,
-                                                             int q_pos0, int block, int* __restrict__ perm) {
+// order, -1 past n_q.
+__global__ void __launch_bounds__(1024) group_sort_kernel(const unsigned long long* __restrict__ sig, int n_q,
+                                                          int* __restrict__ perm) {
   __shared__ unsigned long long key[GW];
   const int w0 = blockIdx.x * GW;
-  for (int i = threadIdx.x; i < GW; i += 1024) {
-    const int t = w0 + i;
-    unsigned long long k = ~0ull;
-    if (t < n_q) {
-      const int cur = (q_pos0 + t) / block;
-      uint32_t h = 0xFFFFFFFFu;
-      const int* kr = kept + (long long)t * keep;
-      const uint32_t* sr = sel ? sel + (long long)t * keep * 2 : nullptr;
-      for (int j = 0; j < keep; ++j) {
-        const int b = kr[j];
-        if (b < 0) break;
-        if (sr != nullptr && __popc(sr[2 * j]) + __popc(sr[2 * j + 1]) < min_sel) continue;
-        if (b != 0 && b != cur) h = min(h, block_hash((uint32_t)b));
-      }
-      k = ((unsigned long long)h << 32) | (uint32_t)t;
-    }
-    key[i] = k;
-  }
+  for (int i = threadIdx.x; i < GW; i += 1024) key[i] = (w0 + i < n_q) ? sig[w0 + i] : ~0ull;
   __syncthreads();
   // bitonic sort, ascending
   for (int size = 2; size <= GW; size <<= 1) {
@@ -103,10 +108,13 @@ __global__ void __launch_bounds__(1024) group_queries_kernel(const int* __restri
 int group_perm_len(int n_q) { return (n_q + GW - 1) / GW * GW; }
 
 cudaError_t launch_group_queries(const int* kept, int keep, const uint32_t* sel, int min_sel, int n_q, int q_pos0,
-                                 int block, int* perm, cudaStream_t st) {
+                                 int block, unsigned long long* sig, int* perm, cudaStream_t st) {
   if (n_q <= 0) return cudaSuccess;
   if (keep <= 0 || block <= 0) return cudaErrorInvalidValue;
-  group_queries_kernel<<<(n_q + GW - 1) / GW, 1024, 0, st>>>(kept, keep, sel, min_sel, n_q, q_pos0, block, perm);
+  group_signature_kernel<<<(n_q + 7) / 8, 256, 0, st>>>(kept, keep, sel, min_sel, n_q, q_pos0, block, sig);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  group_sort_kernel<<<(n_q + GW - 1) / GW, 1024, 0, st>>>(sig, n_q, perm);
   return cudaGetLastError();
 }
 

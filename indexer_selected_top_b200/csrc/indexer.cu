@@ -45,12 +45,14 @@ namespace sa {
 #define SA_IDX_STAGES 6
 #endif
 // epilogue teams of 4 warps (2 or 4) and the prefill MMA N (256 or 128); a
-// team count above 2 needs N <= 128 so every team owns an accumulator
+// team count above 2 needs N <= 128 so every team owns an accumulator. Four
+// teams at N = 128 measured fastest for the grouped stage 2 (more epilogue
+// warps hide the TMEM-load latency) and on par for the flat prefill.
 #ifndef SA_IDX_TEAMS
-#define SA_IDX_TEAMS 2
+#define SA_IDX_TEAMS 4
 #endif
 #ifndef SA_IDX_PREFILL_N
-#define SA_IDX_PREFILL_N 256
+#define SA_IDX_PREFILL_N 128
 #endif
 // epilogue math: 1 = (w/2) * (a + |a|) accumulated with packed f32x2 FMAs
 #ifndef SA_IDX_EPI_PACKED

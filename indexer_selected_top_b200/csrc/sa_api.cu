@@ -105,6 +105,7 @@ struct PrefillPlan {
   size_t off_sel, off_ulist, off_umask, off_unl;   // two-stage: group union lists
   size_t off_gbn, off_gbblk, off_gbslot;            // two-stage: group unions of kept blocks
   size_t off_perm2;                                 // two-stage: attention groups (from the selections)
+  size_t off_sig;                                   // two-stage: grouping signatures
   int n_groups, ucap;
   size_t off_ks, off_kss, off_stab, off_theta, off_cnt, off_list, off_miss, off_rows, off_count, off_pos;
   size_t off_fq, off_fqs, off_fw, off_ftab;
@@ -188,6 +189,8 @@ static bool plan_prefill(const sa_indexer_in* in, const sa_prefill_opts* o, Pref
     off += align256((size_t)group_perm_len(R) * 4);
     p->off_perm2 = off;
     off += align256((size_t)group_perm_len(R) * 4);
+    p->off_sig = off;
+    off += align256((size_t)R * 8);
     // tensor-core attention of the groups' union lists
     p->n_groups = group_perm_len(R) / kGroupQueries;
     p->ucap = group_union_cap(o->k);
@@ -586,7 +589,8 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
       int* gbn = reinterpret_cast<int*>(w + p.off_gbn);
       int* gbblk = reinterpret_cast<int*>(w + p.off_gbblk);
       unsigned long long* gbslot = reinterpret_cast<unsigned long long*>(w + p.off_gbslot);
-      e = launch_group_queries(kept, o->keep_blocks, nullptr, 0, R, ci.q_pos0, o->block_size, perm, stream);
+      unsigned long long* sig = reinterpret_cast<unsigned long long*>(w + p.off_sig);
+      e = launch_group_queries(kept, o->keep_blocks, nullptr, 0, R, ci.q_pos0, o->block_size, sig, perm, stream);
       if (e != cudaSuccess) return cuda_status(e);
       const bool grouped = o->test_hook != SA_HOOK_ATTN_UNGROUPED && in->n_k <= kUnionMaxKeys;
       if (grouped) {
@@ -633,8 +637,8 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
       // attention groups: queries that draw most of their keys from the same
       // blocks (a block counts when at least half of its keys were selected)
       int* perm2 = reinterpret_cast<int*>(w + p.off_perm2);
-      e = launch_group_queries(kept, o->keep_blocks, sel, o->block_size / 2, R, ci.q_pos0, o->block_size, perm2,
-                               stream);
+      e = launch_group_queries(kept, o->keep_blocks, sel, o->block_size / 2, R, ci.q_pos0, o->block_size,
+                               reinterpret_cast<unsigned long long*>(w + p.off_sig), perm2, stream);
       if (e != cudaSuccess) return cuda_status(e);
       e = launch_group_union(kept, o->keep_blocks, sel, perm2, group_perm_len(R), R, in->n_k, p.ucap, list, lmask,
                              nlist, stream);

@@ -101,8 +101,9 @@ constexpr int kGroupQueries = 8;
 int group_perm_len(int n_q);
 // sel (nullable): the top-k's selection bitmaps; with it only kept blocks
 // holding at least min_sel selected keys enter the signature
+// holding at least min_sel selected keys enter the signature; sig = [n_q] scratch
 cudaError_t launch_group_queries(const int* kept, int keep, const uint32_t* sel, int min_sel, int n_q, int q_pos0,
-                                 int block, int* perm, cudaStream_t st);
+                                 int block, unsigned long long* sig, int* perm, cudaStream_t st);
 cudaError_t launch_attention_grouped(const void* q, const void* kc, const void* vc, const int32_t* idx,
                                      const int* perm, int n_perm, int n_q, int k, int n_k, int hq, int dh,
                                      float scale, void* out, float* lse, bool ungrouped, cudaStream_t st);

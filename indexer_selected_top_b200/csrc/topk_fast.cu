@@ -1,5 +1,5 @@
-// topk_fast.cu -- exact top-k of rows of at most 32 * TF_THREADS scores with
-// the keys held in registers (32 per thread), one CTA per row.
+// topk_fast.cu -- exact top-k of rows of at most 4096 scores with the keys
+// held in registers (TF_PER per thread), one CTA per row.
 //
 // Same order as topk.cu: higher score first, lower key index on ties (the
 // packed key of Latent Sparse Attention appendix F.1), found by radix select.
@@ -13,8 +13,17 @@
 
 namespace sa {
 
-constexpr int TF_THREADS = 128;
-constexpr int TF_PER = 32;                         // keys per thread
+// Tuning knobs: keys per thread (32 or 16; the CTA holds 4096 keys either way)
+// and resident CTAs per SM the registers are sized for. 16 keys x 256 threads
+// at 4 CTAs per SM measured fastest: the passes are latency-bound.
+#ifndef SA_TF_PER
+#define SA_TF_PER 16
+#endif
+#ifndef SA_TF_MINB
+#define SA_TF_MINB 4
+#endif
+constexpr int TF_PER = SA_TF_PER;                  // keys per thread
+constexpr int TF_THREADS = 4096 / TF_PER;
 constexpr int TF_MAXN = TF_THREADS * TF_PER;       // 4096
 
 static __device__ __forceinline__ uint32_t tf_key(float x) {
@@ -34,7 +43,7 @@ struct TfShared {
 // Row modes: 0 = causal table row (columns [0, min(n_cols, p + 1)) all valid,
 // key = column); 2 = two-stage candidate row (columns [0, 64 * #kept), key =
 // 64 * kept[c / 64] + c % 64, valid iff score > -inf).
-__global__ void __launch_bounds__(TF_THREADS)
+__global__ void __launch_bounds__(TF_THREADS, SA_TF_MINB)
     topk_fast_kernel(const float* __restrict__ scores, int n_rows, long long ld, int n_cols, int q_pos0,
                      const int* __restrict__ row_pos, const int* __restrict__ kept, int keep, int k,
                      int32_t* __restrict__ idx, uint32_t* __restrict__ sel) {
@@ -143,9 +152,15 @@ __global__ void __launch_bounds__(TF_THREADS)
       }
     return emitted;
   };
-  // selection bitmap of a gathered row: word tid covers columns [32 tid, 32 tid + 32)
+  // selection bitmap of a gathered row: word i covers columns [32 i, 32 i + 32)
   auto put_sel = [&](uint32_t word) {
-    if (sel != nullptr && tid < keep * 2) sel[(long long)row * keep * 2 + tid] = word;
+    if constexpr (TF_PER == 32) {
+      if (sel != nullptr && tid < keep * 2) sel[(long long)row * keep * 2 + tid] = word;
+    } else {
+      const uint32_t hi = __shfl_down_sync(0xffffffffu, word, 1);   // the next thread's 16 columns
+      if (sel != nullptr && (tid & 1) == 0 && tid / 2 < keep * 2)
+        sel[(long long)row * keep * 2 + tid / 2] = (word & 0xFFFFu) | (hi << 16);
+    }
   };
   if (nv <= k) {
     put_sel(emit_ordered([&](int i) { return key[i] != 0u; }, 0, k));
