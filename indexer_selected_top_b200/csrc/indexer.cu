@@ -54,6 +54,10 @@ namespace sa {
 #ifndef SA_IDX_PREFILL_N
 #define SA_IDX_PREFILL_N 128
 #endif
+// independent partial sums per query in the epilogue when N holds several queries
+#ifndef SA_IDX_NP_WIDE
+#define SA_IDX_NP_WIDE 2
+#endif
 // epilogue math: 1 = (w/2) * (a + |a|) accumulated with packed f32x2 FMAs
 #ifndef SA_IDX_EPI_PACKED
 #define SA_IDX_EPI_PACKED 1
@@ -433,7 +437,7 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
 
       // sum_h w'[h] * ReLU(acc[h]) in NP independent partial sums per query
       // (a single running sum would be a dependent FMA chain of H links)
-      constexpr int NPMAX = (C::QS > 1) ? 4 : 8;
+      constexpr int NPMAX = (C::QS > 1) ? SA_IDX_NP_WIDE : 8;
       constexpr int NP = (H / 4 < NPMAX) ? H / 4 : NPMAX;
       constexpr int NCH = C::N / 32;
       float acc[C::QS][NP];

@@ -15,12 +15,13 @@ namespace sa {
 
 // Tuning knobs: keys per thread (32 or 16; the CTA holds 4096 keys either way)
 // and resident CTAs per SM the registers are sized for. 16 keys x 256 threads
-// at 4 CTAs per SM measured fastest: the passes are latency-bound.
+// at 6 CTAs per SM measured fastest (the passes are latency-bound; the few
+// registers this leaves cost a small spill).
 #ifndef SA_TF_PER
 #define SA_TF_PER 16
 #endif
 #ifndef SA_TF_MINB
-#define SA_TF_MINB 4
+#define SA_TF_MINB 6
 #endif
 constexpr int TF_PER = SA_TF_PER;                  // keys per thread
 constexpr int TF_THREADS = 4096 / TF_PER;
