@@ -347,13 +347,15 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
             if constexpr (MODE == IDX_GATHER) gc.next();
             continue;
           }
-          const uint32_t a_base = smem_u32(sK + st * C::KBYTES);
-          const uint32_t b_base = smem_u32(sQ + g * (C::N * C::ROWB));
           const uint32_t d_tmem = tmem_base + buf * C::N;
+          // descriptors built once per job; a K step advances the start
+          // address field (16-byte units, bits 0-13: no carry below 256 KB)
+          const uint64_t ad0 = umma_smem_desc<C::ROWB>(smem_u32(sK + st * C::KBYTES));
+          const uint64_t bd0 = umma_smem_desc<C::ROWB>(smem_u32(sQ + g * (C::N * C::ROWB)));
 #pragma unroll
           for (int ks = 0; ks < C::KSTEPS; ++ks) {
-            const uint64_t ad = umma_smem_desc<C::ROWB>(a_base + ks * 32);
-            const uint64_t bd = umma_smem_desc<C::ROWB>(b_base + ks * 32);
+            const uint64_t ad = ad0 + uint64_t(ks * 32 / 16);
+            const uint64_t bd = bd0 + uint64_t(ks * 32 / 16);
             if constexpr (FP8)
               mma_f8(d_tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
             else
