@@ -377,6 +377,25 @@ def run_native(args, rank, world, local_rank):
                                            4),
                   "step_hbm_frac": round((dw["indexer_bytes"] + dw["topk_bytes"] + dw["attn_bytes"]) /
                                          (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)}
+        # the same step replayed from a CUDA graph (no per-kernel launch cost),
+        # each replay after the L2 flush, timed on the device like the eager steps
+        g = dec.graph()
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            g.replay()
+        gt = 0.0
+        for _ in range(K):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            b.synchronize()
+            gt += a.elapsed_time(b)
+        gus = reduce_max([gt / K * 1e3], device=dev)[0]
+        decode["graph_us_per_step"] = round(gus, 1)
+        decode["graph_us_per_token"] = round(gus / wd.batch, 3)
+        del g
 
     # ---------------- end to end through host buffers ----------------
     e2e = None

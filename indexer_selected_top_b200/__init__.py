@@ -282,6 +282,26 @@ class Decode:
                               _stream(stream)), "sa_decode")
         return self.out, self.lse, self.idx
 
+    def graph(self) -> "torch.cuda.CUDAGraph":
+        """This decode step captured as a CUDA graph. The step launches no
+        host synchronisation and no allocation, so every replay reruns it on the
+        same buffers (write the next token's inputs into them between replays).
+        The stage timer, if any, is not recorded by the graph."""
+        opts, self.opts = self.opts, DecodeOpts(k=self.opts.k, status=self.opts.status,
+                                                test_hook=self.opts.test_hook, stage_events=None, n_stage_events=0)
+        try:
+            s = torch.cuda.Stream()
+            s.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s):
+                self(s)                       # one eager run: first-launch setup stays out of the graph
+            torch.cuda.current_stream().wait_stream(s)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                self(s)
+        finally:
+            self.opts = opts
+        return g
+
 
 def decode(q, q_scale, k, k_scale, w, Q, K, V, seq_lens, k_top: int, **kw):
     return Decode(q, q_scale, k, k_scale, w, Q, K, V, seq_lens, k_top, **kw)()

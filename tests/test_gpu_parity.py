@@ -336,6 +336,31 @@ def _check_decode(sa, wl, seed, seqs=None, seq_lens=None, k=None, hook=0, status
         check_attention_row(out[b], o, lse[b], l, f"seq {b}")
 
 
+def test_decode_cuda_graph_replay(sa):
+    """One decode step captured as a CUDA graph and replayed: the replay
+    matches the oracle, and a replay after new inputs were written into the
+    same buffers matches the oracle on those inputs."""
+    k = 256
+    wl = WORKLOADS["decode_b64_l128k"].with_(batch=3, L=4000)
+    inp = DecodeInputs(wl, "cuda", seed=21)
+    dec = sa.Decode(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, inp.seq_lens, k)
+    g = dec.graph()
+    for seed in (21, 22):
+        nxt = DecodeInputs(wl, "cuda", seed=seed)
+        for name in ("q_idx", "q_scale", "k_idx", "k_scale", "w", "Q", "K", "V", "seq_lens"):
+            getattr(inp, name).copy_(getattr(nxt, name))
+        dec.out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        host = inp.to_host()
+        out, lse, idx = dec.out.float().cpu().numpy(), dec.lse.cpu().numpy(), dec.idx.cpu().numpy()
+        ref = oracle.decode_rows(host, range(wl.batch), k, attention=False)
+        for b in range(wl.batch):
+            check_topk_row(idx[b], ref[b]["cand"], ref[b]["scores"], k, f"seed {seed} seq {b}")
+            o, l = decode_attention_row(host, b, idx[b])
+            check_attention_row(out[b], o, lse[b], l, f"seed {seed} seq {b}")
+
+
 def test_decode_ragged_lengths(sa):
     wl = WORKLOADS["decode_b64_l128k"].with_(batch=4, L=5000)
     _check_decode(sa, wl, 0, seq_lens=[5000, 4097, 130, 2048], k=512)
