@@ -282,6 +282,26 @@ sa_status sa_sparse_attn_decode_noalloc(const sa_attn_in* in, const int32_t* idx
                                         float* lse, cudaStream_t stream);
 
 /*
+ * sa_quantize_rows_e4m3: the indexer's FP8 input encoding, on the device
+ * (Latent Sparse Attention section 2.1: the indexer runs in lower precision;
+ * the format is OCP FP8 e4m3, one fp32 scale per row), for example for the
+ * index key of each token a decode step appends.
+ *   x: device [n_rows, d] row-major, dtype SA_F32 or SA_BF16.
+ *   Per row: amax = max |x|; scale = amax / 448 in fp32 (1 for an all-zero
+ *   row); bytes = e4m3(x / scale) with the division in fp32 (IEEE round to
+ *   nearest) and the encoding rounding to nearest, ties to even, saturating
+ *   at +-448.
+ *   out: device [n_rows, d] uint8; scale: device [n_rows] fp32 (both
+ *   caller-owned). d in [1, 4096]; n_rows >= 0 (0 is a no-op). A negative
+ *   value that rounds to zero may encode as 0x80 (-0). NaN or infinite
+ *   inputs are not supported (their rows' results are unspecified).
+ *   SA_ERR_INVALID_ARGUMENT for null pointers or d out of range,
+ *   SA_ERR_UNSUPPORTED for other dtypes, SA_ERR_CUDA on a launch error.
+ */
+sa_status sa_quantize_rows_e4m3(const void* x, sa_dtype dtype, int64_t n_rows, int32_t d, uint8_t* out,
+                                float* scale, cudaStream_t stream);
+
+/*
  * sa_workspace_size: bytes of device workspace `op` needs for these operands
  * (host call, no device work). opts points to sa_prefill_opts (PREFILL),
  * sa_decode_opts (DECODE), an int32_t k (TOPK, SPARSE_ATTN) or NULL.

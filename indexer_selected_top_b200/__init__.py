@@ -33,7 +33,7 @@ SA_OP_INDEX_SCORES, SA_OP_TOPK, SA_OP_SPARSE_ATTN, SA_OP_PREFILL, SA_OP_DECODE =
 SA_HOOK_NONE, SA_HOOK_THETA_POS_INF, SA_HOOK_THETA_NEG_INF, SA_HOOK_STALL_WAIT, SA_HOOK_ATTN_UNGROUPED = range(5)
 
 EXPORTS = ("sa_status_string", "sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode",
-           "sa_workspace_size", "sa_sparse_attn_decode_noalloc")
+           "sa_workspace_size", "sa_sparse_attn_decode_noalloc", "sa_quantize_rows_e4m3")
 
 
 class IndexerIn(ctypes.Structure):
@@ -101,6 +101,7 @@ _lib.sa_prefill.argtypes = [ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), c
                             _P, _P, ctypes.c_size_t, _P]
 _lib.sa_decode.argtypes = [ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), ctypes.POINTER(DecodeOpts), _P, _P,
                            _P, _P, ctypes.c_size_t, _P]
+_lib.sa_quantize_rows_e4m3.argtypes = [_P, ctypes.c_int, ctypes.c_int64, ctypes.c_int32, _P, _P, _P]
 _lib.sa_workspace_size.argtypes = [ctypes.c_int, ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), _P,
                                    ctypes.POINTER(ctypes.c_size_t)]
 _lib.sa_sparse_attn_decode_noalloc.argtypes = [ctypes.POINTER(AttnIn), _P, ctypes.c_int32, _P, _P, _P]
@@ -305,6 +306,21 @@ class Decode:
 
 def decode(q, q_scale, k, k_scale, w, Q, K, V, seq_lens, k_top: int, **kw):
     return Decode(q, q_scale, k, k_scale, w, Q, K, V, seq_lens, k_top, **kw)()
+
+
+def quantize_rows_e4m3(x: torch.Tensor):
+    """Per-row FP8 e4m3 encoding on the device (sa_quantize_rows_e4m3):
+    returns (uint8 bytes shaped like x, fp32 scale per row)."""
+    if x.dtype not in (torch.float32, torch.bfloat16) or not x.is_cuda or x.dim() < 1:
+        raise ValueError("x: a CUDA float32 or bfloat16 tensor")
+    x = x.contiguous()
+    d = x.shape[-1]
+    n = x.numel() // max(d, 1)
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    _check(_lib.sa_quantize_rows_e4m3(_ptr(x), SA_F32 if x.dtype == torch.float32 else SA_BF16, n, d, _ptr(out),
+                                      _ptr(scale), _stream()), "sa_quantize_rows_e4m3")
+    return out, scale
 
 
 def new_status(device) -> torch.Tensor:

@@ -24,7 +24,7 @@ on the theflow "related" page (block-level coarse filter, then the token
 indexer inside the kept blocks) and LSA section 2.2 (a block scored by the mean
 of its keys, as in MoBA).
 """
-from .fp8 import e4m3_decode_table, e4m3_decode, e4m3_quantize_rne  # noqa: F401
+from .fp8 import e4m3_decode_table, e4m3_decode, e4m3_quantize_rne, quantize_rows  # noqa: F401
 from .indexer import scores_row, scores_rows  # noqa: F401
 from .topk import topk_row, topk_row_bruteforce  # noqa: F401
 from .attention import sparse_attention_row, dense_causal_attention_row  # noqa: F401

@@ -60,3 +60,16 @@ def e4m3_quantize_rne(x) -> np.ndarray:
     code = np.where(a == vhi, _POS_CODES[hi], np.where(pick_hi, _POS_CODES[hi], _POS_CODES[lo]))
     sign = (x < 0) & (code != 0)
     return (code | (sign.astype(np.uint8) << 7)).astype(np.uint8)
+
+
+def quantize_rows(x):
+    """Per-row encoding of the indexer's inputs (the input contract of the
+    lower-precision indexer, LSA section 2.1): scale = amax / 448 in fp32
+    (1 for an all-zero row), bytes = e4m3_quantize_rne(x / scale) with the
+    division in fp32 (IEEE round to nearest). Returns (uint8 bytes, fp32
+    scales)."""
+    x = np.asarray(x, dtype=np.float32)
+    amax = np.abs(x).max(axis=-1)
+    scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    y = (x / scale[..., None]).astype(np.float32)
+    return e4m3_quantize_rne(y), scale

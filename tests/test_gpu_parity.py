@@ -361,6 +361,31 @@ def test_decode_cuda_graph_replay(sa):
             check_attention_row(out[b], o, lse[b], l, f"seed {seed} seq {b}")
 
 
+def test_quantize_rows_e4m3_matches_oracle(sa):
+    """Device per-row FP8 encoding against the oracle's: identical scales, and
+    identical decoded values (bytes too wherever the value is not zero; a
+    negative value that rounds to zero may keep its sign)."""
+    g = torch.Generator(device="cuda").manual_seed(31)
+    x = torch.randn(200, 128, generator=g, device="cuda") * torch.logspace(-6, 3, 200, device="cuda")[:, None]
+    x[0] = 0.0                                                   # all-zero row: scale 1
+    x[1, 7] = 1.0e4                                              # one huge entry
+    x[2, :4] = torch.tensor([448.0, 1.0625, 1.1875, -1.0625], device="cuda")   # exact ties at scale 1
+    x[2, 4:] = 0.5
+    cases = [x, torch.randn(33, 37, generator=g, device="cuda"), torch.randn(4, 16, 128, generator=g, device="cuda")]
+    for xc in cases:
+        for dt in (torch.float32, torch.bfloat16):
+            xs = xc.to(dt)
+            b, s = sa.quantize_rows_e4m3(xs)
+            torch.cuda.synchronize()
+            ref_b, ref_s = oracle.quantize_rows(xs.float().cpu().numpy())
+            b = b.cpu().numpy()
+            assert np.array_equal(s.cpu().numpy(), ref_s), (dt, xc.shape)
+            dec, ref = oracle.e4m3_decode(b), oracle.e4m3_decode(ref_b)
+            assert np.array_equal(dec, ref), (dt, xc.shape)
+            nz = ref != 0
+            assert np.array_equal(b[nz], ref_b[nz]), (dt, xc.shape)
+
+
 def test_decode_ragged_lengths(sa):
     wl = WORKLOADS["decode_b64_l128k"].with_(batch=4, L=5000)
     _check_decode(sa, wl, 0, seq_lens=[5000, 4097, 130, 2048], k=512)

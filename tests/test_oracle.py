@@ -324,3 +324,20 @@ def test_generator_is_seeded_and_shaped():
     rows = sample_rows(5000, 40, seed=0, k=256)
     for must in (0, 1, 255, 256, 257, 4999):
         assert must in rows
+
+
+def test_quantize_rows_hand_values():
+    """Per-row e4m3 encoding, values worked out from the format's definition
+    (bias 7, 3 mantissa bits): 448 = 0x7E, 224 = 1.75 * 2^7 = 0x76, 1 = 0x38,
+    0.75 = 1.5 * 2^-1 = 0x34; 1.0625 lies halfway between 1 (0x38) and 1.125
+    (0x39) and 1.1875 halfway between 1.125 and 1.25 (0x3A): ties go to the
+    even byte."""
+    b, s = oracle.quantize_rows(np.array([[448.0, -224.0, 1.0, 0.0],
+                                          [896.0, 1.5, 0.0, -896.0],
+                                          [0.0, 0.0, 0.0, 0.0],
+                                          [448.0, 1.0625, 1.1875, -1.0625]], dtype=np.float32))
+    assert s.tolist() == [1.0, 2.0, 1.0, 1.0]
+    assert b.tolist() == [[0x7E, 0xF6, 0x38, 0x00],
+                          [0x7E, 0x34, 0x00, 0xFE],
+                          [0x00, 0x00, 0x00, 0x00],
+                          [0x7E, 0x38, 0x3A, 0xB8]]
