@@ -302,6 +302,24 @@ sa_status sa_quantize_rows_e4m3(const void* x, sa_dtype dtype, int64_t n_rows, i
                                 float* scale, cudaStream_t stream);
 
 /*
+ * sa_expand_sinks_window: the index rows attention serves around the k
+ * selected long-range keys (Latent Sparse Attention section 3.2 with its
+ * attention-sink and local-window keys: J_t = sinks + window + the selected
+ * keys those do not already cover).
+ *   idx: device [n_q, k] int32 selected keys (any order, -1 padded); row t
+ *   sits at position p = q_pos0 + t.
+ *   out: device [n_q, n_sink + n_window + k] int32, caller-owned. Row t lists
+ *   the sinks s < min(n_sink, p + 1) ascending, then the window keys
+ *   max(n_sink, p - n_window + 1) <= s <= p ascending, then the entries of
+ *   idx row t that are neither (in their order, -1 entries dropped), then -1.
+ *   n_sink >= 0, n_window >= 0, k >= 1, n_q >= 0 (0 is a no-op).
+ *   SA_ERR_INVALID_ARGUMENT for null pointers or negative sizes, SA_ERR_CUDA
+ *   on a launch error.
+ */
+sa_status sa_expand_sinks_window(const int32_t* idx, int32_t n_q, int32_t k, int32_t q_pos0, int32_t n_sink,
+                                 int32_t n_window, int32_t* out, cudaStream_t stream);
+
+/*
  * sa_workspace_size: bytes of device workspace `op` needs for these operands
  * (host call, no device work). opts points to sa_prefill_opts (PREFILL),
  * sa_decode_opts (DECODE), an int32_t k (TOPK, SPARSE_ATTN) or NULL.

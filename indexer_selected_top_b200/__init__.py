@@ -33,7 +33,8 @@ SA_OP_INDEX_SCORES, SA_OP_TOPK, SA_OP_SPARSE_ATTN, SA_OP_PREFILL, SA_OP_DECODE =
 SA_HOOK_NONE, SA_HOOK_THETA_POS_INF, SA_HOOK_THETA_NEG_INF, SA_HOOK_STALL_WAIT, SA_HOOK_ATTN_UNGROUPED = range(5)
 
 EXPORTS = ("sa_status_string", "sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode",
-           "sa_workspace_size", "sa_sparse_attn_decode_noalloc", "sa_quantize_rows_e4m3")
+           "sa_workspace_size", "sa_sparse_attn_decode_noalloc", "sa_quantize_rows_e4m3",
+           "sa_expand_sinks_window")
 
 
 class IndexerIn(ctypes.Structure):
@@ -102,6 +103,8 @@ _lib.sa_prefill.argtypes = [ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), c
 _lib.sa_decode.argtypes = [ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), ctypes.POINTER(DecodeOpts), _P, _P,
                            _P, _P, ctypes.c_size_t, _P]
 _lib.sa_quantize_rows_e4m3.argtypes = [_P, ctypes.c_int, ctypes.c_int64, ctypes.c_int32, _P, _P, _P]
+_lib.sa_expand_sinks_window.argtypes = [_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                        ctypes.c_int32, _P, _P]
 _lib.sa_workspace_size.argtypes = [ctypes.c_int, ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), _P,
                                    ctypes.POINTER(ctypes.c_size_t)]
 _lib.sa_sparse_attn_decode_noalloc.argtypes = [ctypes.POINTER(AttnIn), _P, ctypes.c_int32, _P, _P, _P]
@@ -321,6 +324,20 @@ def quantize_rows_e4m3(x: torch.Tensor):
     _check(_lib.sa_quantize_rows_e4m3(_ptr(x), SA_F32 if x.dtype == torch.float32 else SA_BF16, n, d, _ptr(out),
                                       _ptr(scale), _stream()), "sa_quantize_rows_e4m3")
     return out, scale
+
+
+def expand_sinks_window(idx: torch.Tensor, q_pos0: int, n_sink: int, n_window: int) -> torch.Tensor:
+    """Served index rows (sa_expand_sinks_window): per row the sinks, the local
+    window and the selected keys neither covers, -1 padded to
+    n_sink + n_window + k columns."""
+    if idx.dtype != torch.int32 or not idx.is_cuda or idx.dim() != 2:
+        raise ValueError("idx: a CUDA int32 tensor [n_q, k]")
+    idx = idx.contiguous()
+    n_q, k = idx.shape
+    out = torch.empty((n_q, n_sink + n_window + k), dtype=torch.int32, device=idx.device)
+    _check(_lib.sa_expand_sinks_window(_ptr(idx), n_q, k, q_pos0, n_sink, n_window, _ptr(out), _stream()),
+           "sa_expand_sinks_window")
+    return out
 
 
 def new_status(device) -> torch.Tensor:

@@ -94,3 +94,18 @@ def decode_attention_row(host, b: int, idx, scale=None):
     L = int(as_numpy(host["seq_lens"])[b])
     return sparse_attention_row(as_numpy(host["Q"][b]), as_numpy(host["K"][b, :L]),
                                 as_numpy(host["V"][b, :L]), np.asarray(idx), scale)
+
+
+def expand_sinks_window_row(idx, p: int, n_sink: int, n_window: int):
+    """The served index row of the query at position p (Latent Sparse
+    Attention section 3.2 with attention sinks and a local window): the sinks
+    0 .. min(n_sink, p + 1) - 1, then the window max(n_sink, p - n_window + 1)
+    .. p, then the selected keys (in their order) that neither covers, then -1
+    up to n_sink + n_window + len(idx)."""
+    idx = [int(s) for s in np.asarray(idx).tolist()]
+    sinks = list(range(min(n_sink, p + 1)))
+    w_lo = max(n_sink, p - n_window + 1)
+    window = list(range(w_lo, p + 1))
+    rest = [s for s in idx if s >= 0 and not (s < n_sink or s >= w_lo)]
+    row = sinks + window + rest
+    return np.array(row + [-1] * (n_sink + n_window + len(idx) - len(row)), dtype=np.int64)

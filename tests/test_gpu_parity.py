@@ -386,6 +386,43 @@ def test_quantize_rows_e4m3_matches_oracle(sa):
             assert np.array_equal(b[nz], ref_b[nz]), (dt, xc.shape)
 
 
+def test_expand_sinks_window_matches_oracle(sa):
+    """Served index rows (4 sinks, a 512-key window, the selected keys neither
+    covers) against the oracle row by row, on early rows (inside the sinks and
+    the window) and later ones, with -1 padding anywhere in the input rows; and
+    attention over the expanded rows against the oracle."""
+    from oracle.pipeline import expand_sinks_window_row
+    rng = np.random.default_rng(41)
+    n_q, k, q_pos0 = 300, 64, 400
+    idx = np.full((n_q, k), -1, dtype=np.int32)
+    for t in range(n_q):
+        p = q_pos0 + t
+        m = min(k, p + 1) if t % 4 else int(rng.integers(0, min(k, p + 1) + 1))
+        idx[t, :m] = rng.choice(p + 1, size=m, replace=False)
+        rng.shuffle(idx[t])
+    for n_sink, n_window, pos0 in ((4, 512, q_pos0), (4, 512, 0), (0, 32, q_pos0), (16, 0, q_pos0)):
+        out = sa.expand_sinks_window(torch.from_numpy(idx).cuda(), pos0, n_sink, n_window)
+        torch.cuda.synchronize()
+        out = out.cpu().numpy()
+        for t in range(n_q):
+            ref = expand_sinks_window_row(idx[t], pos0 + t, n_sink, n_window)
+            assert np.array_equal(out[t], ref), (n_sink, n_window, pos0, t)
+    # attention over the served rows
+    g = torch.Generator(device="cuda").manual_seed(42)
+    n_k = q_pos0 + n_q
+    K = (torch.randn(n_k, 128, generator=g, device="cuda") / np.sqrt(128)).bfloat16()
+    V = (torch.randn(n_k, 128, generator=g, device="cuda") / np.sqrt(128)).bfloat16()
+    Q = (torch.randn(n_q, 16, 128, generator=g, device="cuda") / np.sqrt(128)).bfloat16()
+    J = sa.expand_sinks_window(torch.from_numpy(idx).cuda(), q_pos0, 4, 512)
+    o, l = sa.sparse_attn(Q, K, V, J)
+    torch.cuda.synchronize()
+    o, l, J = o.float().cpu().numpy(), l.cpu().numpy(), J.cpu().numpy()
+    Qh, Kh, Vh = Q.double().cpu().numpy(), K.double().cpu().numpy(), V.double().cpu().numpy()
+    for t in range(0, n_q, 7):
+        ro, rl = oracle.sparse_attention_row(Qh[t], Kh, Vh, J[t])
+        check_attention_row(o[t], ro, l[t], rl, f"row {t}")
+
+
 def test_decode_ragged_lengths(sa):
     wl = WORKLOADS["decode_b64_l128k"].with_(batch=4, L=5000)
     _check_decode(sa, wl, 0, seq_lens=[5000, 4097, 130, 2048], k=512)

@@ -341,3 +341,16 @@ def test_quantize_rows_hand_values():
                           [0x7E, 0x34, 0x00, 0xFE],
                           [0x00, 0x00, 0x00, 0x00],
                           [0x7E, 0x38, 0x3A, 0xB8]]
+
+
+def test_expand_sinks_window_hand_rows():
+    """Position 10, two sinks, a window of three: sinks 0 1, window 8 9 10,
+    then the selected keys neither covers (5 and 7; 9, 0, 1 and 10 are
+    covered, -1 is dropped), then -1. Position 1: only the two sinks."""
+    from oracle.pipeline import expand_sinks_window_row
+    r = expand_sinks_window_row([9, 0, 5, -1, 7, 1, 10], 10, 2, 3)
+    assert r.tolist() == [0, 1, 8, 9, 10, 5, 7, -1, -1, -1, -1, -1]
+    r = expand_sinks_window_row([0, 1, -1], 1, 2, 3)
+    assert r.tolist() == [0, 1, -1, -1, -1, -1, -1, -1]
+    r = expand_sinks_window_row([3, 40, 2], 50, 0, 0)     # no sinks, no window: the selection unchanged
+    assert r.tolist() == [3, 40, 2]
