@@ -438,7 +438,8 @@ namespace sa {
 // bitmap over its kept blocks' candidates (column c = 64 * slot + offset).
 // The union of the group is built block-wise: the group's kept blocks in
 // ascending order (a bitmap over all blocks, ranked by popcount), a table of
-// each query's slot of every union block, then one mask byte per union key.
+// each query's slot of every union block, then one mask byte per union key
+// (8 keys at a time by an 8 x 8 bit transpose), compacted in key order.
 int group_union_cap(int k) { return (GA * k + kUnionChunk - 1) / kUnionChunk * kUnionChunk; }
 
 __global__ void __launch_bounds__(256) group_union_kernel(const int* __restrict__ kept, int keep,
@@ -455,6 +456,7 @@ __global__ void __launch_bounds__(256) group_union_kernel(const int* __restrict_
   __shared__ int ub2blk[GA * KB];
   __shared__ int red[8];
   __shared__ int s_nub;
+  extern __shared__ __align__(8) uint8_t ga_union_smem[];   // [GA * KB * 64] per-key query masks
   const int g = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid < GA) {
     const int j = g * GA + tid;
@@ -511,24 +513,35 @@ __global__ void __launch_bounds__(256) group_union_kernel(const int* __restrict_
     if (b >= 0) slot[qi][wpre[b >> 5] + __popc(bits[b >> 5] & ((1u << (b & 31)) - 1u))] = (signed char)c;
   }
   __syncthreads();
-  auto mask_of = [&](int e) -> uint32_t {
-    const int u = e >> 6, j = e & 63;
-    uint32_t m = 0u;
+  // per union key, the byte of the group's queries that selected it: for 8
+  // keys of a union block, byte q of `m` holds query q's selection bits of
+  // those keys; an 8 x 8 bit transpose turns it into one byte per key
+  uint8_t* mb = ga_union_smem;
+  for (int i = tid; i < n_ub * 8; i += 256) {
+    const int u = i >> 3, b8 = (i & 7) * 8;
+    unsigned long long m = 0ull;
 #pragma unroll
     for (int qi = 0; qi < GA; ++qi) {
-      const int s = slot[qi][u];
-      if (s >= 0) {
-        const int c = s * 64 + j;
-        m |= ((sw[qi][c >> 5] >> (c & 31)) & 1u) << qi;
+      const int sl = slot[qi][u];
+      if (sl >= 0) {
+        const int c = sl * 64 + b8;
+        m |= (unsigned long long)((sw[qi][c >> 5] >> (c & 31)) & 0xFFu) << (8 * qi);
       }
     }
-    return m;
-  };
+    unsigned long long t = (m ^ (m >> 7)) & 0x00AA00AA00AA00AAull;
+    m ^= t ^ (t << 7);
+    t = (m ^ (m >> 14)) & 0x0000CCCC0000CCCCull;
+    m ^= t ^ (t << 14);
+    t = (m ^ (m >> 28)) & 0x00000000F0F0F0F0ull;
+    m ^= t ^ (t << 28);
+    *reinterpret_cast<unsigned long long*>(mb + u * 64 + b8) = m;
+  }
+  __syncthreads();
   const int n_slot = n_ub * 64;
   const int per = (n_slot + 255) / 256;
   const int lo = min(n_slot, tid * per), hi = min(n_slot, lo + per);
   int cnt = 0;
-  for (int e = lo; e < hi; ++e) cnt += mask_of(e) != 0u;
+  for (int e = lo; e < hi; ++e) cnt += mb[e] != 0;
   int incl = cnt;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -548,11 +561,11 @@ __global__ void __launch_bounds__(256) group_union_kernel(const int* __restrict_
   uint8_t* gm = lmask + (long long)g * cap;
   int p = before + incl - cnt;
   for (int e = lo; e < hi; ++e) {
-    const uint32_t m = mask_of(e);
-    if (m != 0u) {
+    const uint8_t m = mb[e];
+    if (m != 0) {
       if (p < cap) {
         gl[p] = ub2blk[e >> 6] * 64 + (e & 63);
-        gm[p] = (uint8_t)m;
+        gm[p] = m;
       }
       ++p;
     }
@@ -569,7 +582,10 @@ cudaError_t launch_group_union(const int* kept, int keep, const uint32_t* sel, c
   if (n_q <= 0) return cudaSuccess;
   if (keep <= 0 || keep > 64 || n_k > GK_MAX || cap % kUnionChunk != 0) return cudaErrorNotSupported;
   const int n_groups = ((perm ? n_perm : n_q) + GA - 1) / GA;
-  group_union_kernel<<<n_groups, 256, 0, st>>>(kept, keep, sel, perm, n_q, n_k, cap, list, lmask, n_list);
+  constexpr int smem = GA * 64 * 64;   // one mask byte per key of up to GA * 64 union blocks
+  cudaError_t e = cudaFuncSetAttribute(group_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  group_union_kernel<<<n_groups, 256, smem, st>>>(kept, keep, sel, perm, n_q, n_k, cap, list, lmask, n_list);
   return cudaGetLastError();
 }
 
