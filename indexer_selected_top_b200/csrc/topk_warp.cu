@@ -197,11 +197,12 @@ constexpr int BW_MAXB = 4096;                 // blocks per row held in shared m
 
 __global__ void __launch_bounds__(TW_WARPS * 32)
     block_keep_warp_kernel(const float* __restrict__ bscores, int n_q, long long ld, int q_pos0, int block, int keep,
-                           int* __restrict__ kept) {
+                           int* __restrict__ kept, int cap) {
   extern __shared__ uint32_t bw_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint32_t* keys = bw_smem + warp * (BW_MAXB + 256 + BW_MAXB / 32);
-  uint32_t* hist = keys + BW_MAXB;
+  // per warp: cap block keys, a 256-bin histogram, cap / 32 flag words
+  uint32_t* keys = bw_smem + warp * (cap + 256 + cap / 32);
+  uint32_t* hist = keys + cap;
   uint32_t* flags = hist + 256;
   const int t = blockIdx.x * TW_WARPS + warp;
   if (t >= n_q) return;
@@ -286,11 +287,14 @@ cudaError_t launch_block_keep_warp(const float* bscores, int n_q, long long ld, 
                                    int* kept, cudaStream_t st) {
   if (n_q <= 0) return cudaSuccess;
   if ((q_pos0 + n_q - 1) / block >= BW_MAXB) return cudaErrorNotSupported;
-  const int smem = TW_WARPS * (BW_MAXB + 256 + BW_MAXB / 32) * 4;
+  // shared memory sized by the largest current block of the call (not the
+  // 4096-block maximum), so more CTAs fit per SM
+  const int cap = ((q_pos0 + n_q - 1) / block + 1 + 31) / 32 * 32;
+  const int smem = TW_WARPS * (cap + 256 + cap / 32) * 4;
   cudaError_t e = cudaFuncSetAttribute(block_keep_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   block_keep_warp_kernel<<<(n_q + TW_WARPS - 1) / TW_WARPS, TW_WARPS * 32, smem, st>>>(bscores, n_q, ld, q_pos0, block,
-                                                                                       keep, kept);
+                                                                                       keep, kept, cap);
   return cudaGetLastError();
 }
 
