@@ -91,3 +91,39 @@ def test_workspace_sizes_and_too_small(sa):
     assert sa.workspace_size(sa.SA_OP_DECODE, dind, datt, dopts) >= 64 * 131072 * 4
     assert sa.workspace_size(sa.SA_OP_SPARSE_ATTN, att=datt, opts=2048) > 0
     assert sa.workspace_size(sa.SA_OP_SPARSE_ATTN, att=att, opts=2048) == 0
+
+
+def test_new_entry_points_validate_on_the_host(sa):
+    lib = sa._lib
+    # sa_quantize_rows_e4m3(x, dtype, n_rows, d, out, scale, stream)
+    assert lib.sa_quantize_rows_e4m3(None, sa.SA_F32, 0, 128, None, None, None) == sa.SA_OK            # empty
+    assert lib.sa_quantize_rows_e4m3(None, sa.SA_F32, 4, 128, 256, 512, None) == sa.SA_ERR_INVALID_ARGUMENT
+    assert lib.sa_quantize_rows_e4m3(256, sa.SA_F32, 4, 0, 256, 512, None) == sa.SA_ERR_INVALID_ARGUMENT
+    assert lib.sa_quantize_rows_e4m3(256, sa.SA_F32, 4, 4097, 256, 512, None) == sa.SA_ERR_INVALID_ARGUMENT
+    assert lib.sa_quantize_rows_e4m3(256, sa.SA_F32, -1, 128, 256, 512, None) == sa.SA_ERR_INVALID_ARGUMENT
+    assert lib.sa_quantize_rows_e4m3(256, sa.SA_FP8_E4M3, 4, 128, 256, 512, None) == sa.SA_ERR_UNSUPPORTED
+    # sa_expand_sinks_window(idx, n_q, k, q_pos0, n_sink, n_window, out, stream)
+    assert lib.sa_expand_sinks_window(None, 0, 8, 0, 4, 16, None, None) == sa.SA_OK                    # empty
+    assert lib.sa_expand_sinks_window(None, 4, 8, 0, 4, 16, None, None) == sa.SA_ERR_INVALID_ARGUMENT
+    assert lib.sa_expand_sinks_window(256, 4, 0, 0, 4, 16, 512, None) == sa.SA_ERR_INVALID_ARGUMENT
+    assert lib.sa_expand_sinks_window(256, 4, 8, 0, -1, 16, 512, None) == sa.SA_ERR_INVALID_ARGUMENT
+    assert lib.sa_expand_sinks_window(256, 4, 8, -5, 4, 16, 512, None) == sa.SA_ERR_INVALID_ARGUMENT
+
+
+def test_two_stage_workspace_covers_the_group_tables(sa):
+    """The two-stage workspace grows with the query rows (per-row candidate
+    scores, selection bitmaps, group unions) and stays 256-byte sized."""
+    sizes = []
+    for n_q in (1000, 8192, 65536):
+        ind = sa.IndexerIn(n_q=n_q, n_k=65536, q_pos0=65536 - n_q, n_heads=64, d_idx=128, dtype=sa.SA_FP8_E4M3,
+                           q=256, q_scale=512, k=1024, k_scale=2048, w=4096, batch=0, seq_lens=None)
+        att = sa.AttnIn(q=256, k_cache=512, v_cache=1024, n_q=n_q, n_k=65536, n_q_heads=16, head_dim=128,
+                        softmax_scale=0.0, batch=0)
+        opts = sa.PrefillOpts(k=2048, mode=1, block_size=64, keep_blocks=64, chunk_rows=0, status=None,
+                              test_hook=0, stage_events=None, n_stage_events=0, flat_path=0)
+        sizes.append(sa.workspace_size(sa.SA_OP_PREFILL, ind, att, opts))
+    assert sizes[0] < sizes[1] < sizes[2]
+    # one chunk of at most 32768 rows: at least its candidate scores, index
+    # rows and group key lists (8 k entries of 4 + 1 bytes per group of 8)
+    R = 32768
+    assert sizes[2] >= R * (4096 * 4 + 2048 * 4) + R // 8 * 8 * 2048 * 5
