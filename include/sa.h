@@ -238,7 +238,10 @@ sa_status sa_sparse_attn(const sa_attn_in* in, const int32_t* idx, int32_t k, vo
  *   e4m3 with one scale per block); stage 1 scores complete blocks b <
  *   floor(p / block_size) and keeps block 0, the current block and the best
  *   keep_blocks - 2 others; stage 2 scores the visible keys of the kept
- *   blocks; then top-k and attention.
+ *   blocks; then top-k and attention. The two-stage path schedules its
+ *   queries in groups of 8 that keep (stage 2) or select (attention) mostly
+ *   the same keys, so a group's keys are loaded once; every query's scores,
+ *   selection and attention are its own, whatever its group.
  * Requires in->n_k == n_k of attn, q_pos0 + n_q <= n_k.
  * Host synchronisation: FLAT mode above the table size reads one counter per
  * chunk back to the host (the miss count, as the pages do in prefill).
