@@ -81,9 +81,6 @@ cudaError_t launch_compact_rows(const int* flags, int n_rows, int* rows, int* co
 cudaError_t launch_block_select(const float* bscores, int n_q, int nb, long long ld, int q_pos0, int block,
                                 int keep, int* kept, cudaStream_t st);
 
-cudaError_t launch_topk_rows_warp(const float* scores, int n_rows, long long ld, int n_cols, int q_pos0,
-                                  const int* kept, int keep, int k, int32_t* idx, cudaStream_t st);
-
 cudaError_t launch_block_keep_warp(const float* bscores, int n_q, long long ld, int q_pos0, int block, int keep,
                                    int* kept, cudaStream_t st);
 

@@ -1,22 +1,19 @@
-// topk_warp.cu -- exact top-k of short rows, one warp per row.
+// topk_warp.cu -- the stage-1 block keep: the best keep - 2 block scores of
+// each query row, one warp per row.
 //
-// Same order as topk.cu (higher score first, lower key index on ties; the
-// packed key of Latent Sparse Attention appendix F.1) and the same radix
-// select, restated for one warp: the row's order-preserving 32-bit score keys
-// sit in shared memory, each pass histograms the next 8-bit digit of the keys
-// that still match the prefix (per-instruction match aggregation keeps the
-// shared atomics low), and the pass stops early once the bucket holding the
-// cut is taken whole. Ties at the cut take the lowest positions by an ordered
-// ballot scan. Used for score-table rows of at most 4096 columns, for the
-// two-stage candidate rows (keep_blocks * 64 <= 4096 scores) and for the
-// stage-1 block keep (at most 4096 blocks).
+// Same order as topk.cu (higher score first, lower index on ties; the packed
+// key of Latent Sparse Attention appendix F.1) and the same radix select,
+// restated for one warp: the row's order-preserving 32-bit score keys sit in
+// shared memory, each pass histograms the next 8-bit digit of the keys that
+// still match the prefix (per-instruction match aggregation keeps the shared
+// atomics low), and the pass stops early once the bucket holding the cut is
+// taken whole. Ties at the cut take the lowest positions by an ordered ballot
+// scan. Rows of at most 4096 blocks (longer ones go to block_select_kernel).
 #include "sa_internal.h"
 
 namespace sa {
 
 constexpr int TW_WARPS = 4;
-constexpr int TW_MAXN = 4096;                 // candidate entries per row held in shared memory
-constexpr uint32_t TW_NEG_INF_KEY = 0x007FFFFFu;
 
 __device__ __forceinline__ uint32_t tw_key(float x) {
   uint32_t b = __float_as_uint(x);
@@ -103,96 +100,6 @@ __device__ void warp_cut(const uint32_t* keys, int n, int need, uint32_t* hist, 
   __syncwarp();
 }
 
-// Rows of a score table. With `kept`, row t is a two-stage candidate row of
-// keep * 64 scores whose column c scores key 64 * kept[t][c / 64] + c % 64 and
-// -inf marks an invisible key. Without, row t is a causal table row whose
-// columns s < min(n_cols, q_pos0 + t + 1) are its candidates (key = column).
-__global__ void __launch_bounds__(TW_WARPS * 32)
-    topk_rows_warp_kernel(const float* __restrict__ scores, int n_rows, long long ld, int n_cols, int q_pos0,
-                          const int* __restrict__ kept, int keep, int k, int32_t* __restrict__ idx) {
-  extern __shared__ uint32_t tw_smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint32_t* keys = tw_smem + warp * (TW_MAXN + 256 + 64);
-  uint32_t* hist = keys + TW_MAXN;
-  int* kb = reinterpret_cast<int*>(hist + 256);
-  const int row = blockIdx.x * TW_WARPS + warp;
-  if (row >= n_rows) return;
-  const bool gathered = kept != nullptr;
-  int n, nvalid = 0;
-  const float* srow = scores + row * ld;
-  if (gathered) {
-    const int* kr = kept + (long long)row * keep;
-    for (int j = lane; j < 64; j += 32) kb[j] = j < keep ? kr[j] : -1;
-    __syncwarp();
-    int nb = 0;
-    while (nb < keep && kb[nb] >= 0) ++nb;
-    n = nb * 64;
-    const float4* src = reinterpret_cast<const float4*>(srow);
-    for (int i = lane; i < n / 4; i += 32) {
-      const float4 v = src[i];
-      const uint32_t a = tw_key(v.x), b = tw_key(v.y), c = tw_key(v.z), d = tw_key(v.w);
-      keys[4 * i] = a;
-      keys[4 * i + 1] = b;
-      keys[4 * i + 2] = c;
-      keys[4 * i + 3] = d;
-      nvalid += (a != TW_NEG_INF_KEY) + (b != TW_NEG_INF_KEY) + (c != TW_NEG_INF_KEY) + (d != TW_NEG_INF_KEY);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) nvalid += __shfl_xor_sync(0xffffffffu, nvalid, o);
-  } else {
-    n = max(0, min(n_cols, q_pos0 + row + 1));
-    for (int i = lane; i < n; i += 32) keys[i] = tw_key(srow[i]);
-    nvalid = n;
-  }
-  __syncwarp();
-  int32_t* out = idx + (long long)row * k;
-  auto valid = [&](int i) { return !gathered || keys[i] != TW_NEG_INF_KEY; };
-  auto key_of = [&](int c) { return gathered ? kb[c >> 6] * 64 + (c & 63) : c; };
-  int pos = 0;
-  if (nvalid <= k) {
-    for (int i0 = 0; i0 < n; i0 += 32) {
-      const int i = i0 + lane;
-      const bool v = i < n && valid(i);
-      const unsigned b = __ballot_sync(0xffffffffu, v);
-      if (v) out[pos + __popc(b & ((1u << lane) - 1))] = key_of(i);
-      pos += __popc(b);
-    }
-  } else {
-    uint32_t cut;
-    int ties;
-    warp_cut(keys, n, k, hist, valid, cut, ties);
-    for (int i0 = 0; i0 < n; i0 += 32) {
-      const int i = i0 + lane;
-      bool take = false;
-      if (i < n && valid(i)) {
-        // bucket taken whole: every key at or above its prefix; otherwise the
-        // keys strictly above the cut, ties handled below
-        const uint32_t kk = keys[i];
-        take = (ties < 0) ? (kk >= cut) : (kk > cut);
-      }
-      const unsigned b = __ballot_sync(0xffffffffu, take);
-      if (take) out[pos + __popc(b & ((1u << lane) - 1))] = key_of(i);
-      pos += __popc(b);
-    }
-    if (ties > 0) {
-      for (int i0 = 0; i0 < n && ties > 0; i0 += 32) {
-        const int i = i0 + lane;
-        const bool eq = i < n && valid(i) && keys[i] == cut;
-        const unsigned b = __ballot_sync(0xffffffffu, eq);
-        const int r = __popc(b & ((1u << lane) - 1));
-        if (eq && r < ties) out[pos + r] = key_of(i);
-        const int took = min(ties, __popc(b));
-        pos += took;
-        ties -= took;
-      }
-    }
-  }
-  for (int j = pos + lane; j < k; j += 32) out[j] = -1;
-}
-
-// Stage-1 keep: block 0, the current block cur = (q_pos0 + t) / block, and the
-// best keep - 2 of blocks [1, cur - 1] by (score desc, block asc), written in
-// ascending block order, -1 padded to `keep`.
 constexpr int BW_MAXB = 4096;                 // blocks per row held in shared memory
 
 __global__ void __launch_bounds__(TW_WARPS * 32)
@@ -269,18 +176,6 @@ __global__ void __launch_bounds__(TW_WARPS * 32)
     pos += __shfl_sync(0xffffffffu, incl, 31);
   }
   for (int j = min(pos, keep) + lane; j < keep; j += 32) out[j] = -1;
-}
-
-cudaError_t launch_topk_rows_warp(const float* scores, int n_rows, long long ld, int n_cols, int q_pos0,
-                                  const int* kept, int keep, int k, int32_t* idx, cudaStream_t st) {
-  if (n_rows <= 0) return cudaSuccess;
-  if (kept != nullptr ? keep * 64 > TW_MAXN : n_cols > TW_MAXN) return cudaErrorNotSupported;
-  const int smem = TW_WARPS * (TW_MAXN + 256 + 64) * 4;
-  cudaError_t e = cudaFuncSetAttribute(topk_rows_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  topk_rows_warp_kernel<<<(n_rows + TW_WARPS - 1) / TW_WARPS, TW_WARPS * 32, smem, st>>>(scores, n_rows, ld, n_cols,
-                                                                                         q_pos0, kept, keep, k, idx);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_block_keep_warp(const float* bscores, int n_q, long long ld, int q_pos0, int block, int keep,
