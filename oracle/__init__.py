@@ -7,6 +7,9 @@ precision) that states what the hot path computes:
   (2) top-k     the k visible keys of largest score, ties to the lower index
   (3) attention softmax attention over the selected keys of one shared KV head
   (+) two-stage mean-pooled key blocks filter the keys before (1)-(2)
+  (+) LSA flat semantic search (``oracle.lsa``): unit keys pooled and
+      Ward-clustered into buckets per cluster block, queries score the
+      bucket centroids, and the top-p buckets expand into the index row
 
 Only tests/, the smoke check and the CPU-baseline leg of the benchmark may
 import this package; the product path (the CUDA library and its binding) never
