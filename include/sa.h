@@ -323,6 +323,102 @@ sa_status sa_expand_sinks_window(const int32_t* idx, int32_t n_q, int32_t k, int
                                  int32_t n_window, int32_t* out, cudaStream_t stream);
 
 /*
+ * LSA flat semantic search (Latent Sparse Attention section 3.1 "Semantic
+ * Clustering", section 3.2 "Semantic Search", appendix F.1 "Kernels"): index
+ * keys are clustered by content into buckets, once per cluster block of
+ * n_cluster consecutive keys, and each query expands its best buckets into
+ * its index row. Index keys and queries are bf16 rows of d_idx = 64.
+ *
+ *   n_pool           consecutive unit keys summed into one pool key (>= 1)
+ *   n_cluster        keys per cluster block, a multiple of n_pool, with
+ *                    n_cluster / n_pool <= 256 pool keys
+ *   n_buckets        m, buckets per cluster block (1 .. n_cluster / n_pool)
+ *   max_bucket_keys  n_b^max, a multiple of n_pool; unless m equals the
+ *                    pool keys per block it must be >= 2 n_cluster / m (a
+ *                    smaller cap can leave no pair that fits before m
+ *                    buckets remain)
+ * Violations are SA_ERR_INVALID_ARGUMENT; d_idx != 64 or more than 256 pool
+ * keys per block are SA_ERR_UNSUPPORTED.
+ */
+typedef struct {
+  int32_t d_idx;
+  int32_t n_pool;
+  int32_t n_cluster;
+  int32_t n_buckets;
+  int32_t max_bucket_keys;
+} sa_lsa_params;
+
+/*
+ * sa_lsa_build_buckets: the bucket cache of cluster blocks [block0, block0 +
+ *   n_blocks) of the index keys k_idx (device bf16 [n_k, 64]; block c holds
+ *   keys c * n_cluster .. (c + 1) * n_cluster - 1, so (block0 + n_blocks) *
+ *   n_cluster <= n_k). Per block (section 3.1): keys are L2 normalised,
+ *   summed n_pool at a time into pool keys, and clustered bottom up with
+ *   Ward's method -- every round, all pairs of buckets that are each other's
+ *   cheapest merge (among the merges that keep a bucket within n_b^max keys)
+ *   merge, until m buckets remain; a round that would overshoot merges its
+ *   cheapest pairs. The merge cost is n_a n_b / (n_a + n_b) |mu_a - mu_b|^2
+ *   over bucket means mu (counts in pool keys), computed in fp32 with one
+ *   rounding per operation and dimensions summed from 0 upward; cost ties go
+ *   to the lower index. Buckets of a block are numbered by their lowest pool
+ *   key; bucket b = c * m + r.
+ *   Outputs (device, caller-owned, indexed by absolute block so that later
+ *   blocks can be added by later calls):
+ *     centroids    bf16 [(block0 + n_blocks) * m, 64]: the bucket's key sum
+ *                  L2 normalised (fp32) and rounded to bf16 (nearest even)
+ *     bucket_off   int32 [(block0 + n_blocks) * m]: start of the bucket's key
+ *                  list in bucket_keys; the list ends at bucket_off[b + 1],
+ *                  or at (c + 1) * n_cluster for the block's last bucket
+ *     bucket_keys  int32 [(block0 + n_blocks) * n_cluster]: key positions,
+ *                  ascending within each bucket; block c fills [c * n_cluster,
+ *                  (c + 1) * n_cluster)
+ *   status (device, nullable) is zeroed by the call; error = SA_ERR_INTERNAL
+ *   if a block could not reach m buckets (excluded by the cap rule above).
+ *   k_idx and centroids must be 16-byte aligned. No workspace, no host
+ *   synchronisation. n_blocks = 0 is a no-op.
+ */
+sa_status sa_lsa_build_buckets(const sa_lsa_params* prm, const void* k_idx, int32_t n_k, int32_t block0,
+                               int32_t n_blocks, void* centroids, int32_t* bucket_off, int32_t* bucket_keys,
+                               sa_device_status* status, cudaStream_t stream);
+
+typedef struct {
+  int32_t p;          /* buckets kept per query, 1 .. 2048 */
+  int32_t k;          /* long-range keys per query, >= 1 */
+  int32_t n_sink;     /* attention-sink keys 0 .. n_sink - 1, >= 0 */
+  int32_t n_window;   /* most recent keys, >= 0 */
+  sa_device_status* status;   /* device, nullable; zeroed by the call */
+} sa_lsa_search_opts;
+
+/*
+ * sa_lsa_search: index rows of queries over a bucket cache (section 3.2).
+ *   q_idx: device bf16 [n_q, 64] index queries (not yet normalised); row i
+ *   sits at position pos = q_pos0 + i. The cache holds blocks 0 .. n_blocks
+ *   - 1 (from sa_lsa_build_buckets); the query scores the unit centroids of
+ *   blocks c < min(n_blocks, pos / n_cluster), s_b = c_b . q (q L2
+ *   normalised in fp32, rounded to bf16; products on the tensor cores with
+ *   fp32 accumulation), keeps the top p (ties: lower bucket id), and takes
+ *   their keys best first (score, then lower id; a bucket's keys in list
+ *   order) until k long-range keys are held, skipping keys among the sinks
+ *   (s < n_sink) or in the window (s >= max(n_sink, pos - n_window + 1)).
+ *   J: device int32 [n_q, n_sink + n_window + k], caller-owned. Row i: the
+ *   sinks ascending, the window ascending, the long-range keys (best bucket
+ *   first), then -1. Fewer than k long-range keys when the p buckets hold
+ *   fewer uncovered keys.
+ *   Scores are written to the workspace (the pages' short-context regime):
+ *   n_blocks * m must be <= 32768 (else SA_ERR_UNSUPPORTED). Workspace:
+ *   sa_lsa_search_workspace_size bytes, 256-byte aligned. No host
+ *   synchronisation; status error = SA_ERR_TIMEOUT if a bounded wait gave up.
+ */
+sa_status sa_lsa_search(const sa_lsa_params* prm, const sa_lsa_search_opts* opts, const void* q_idx, int32_t n_q,
+                        int32_t q_pos0, const void* centroids, const int32_t* bucket_off,
+                        const int32_t* bucket_keys, int32_t n_blocks, int32_t* J, void* ws, size_t ws_bytes,
+                        cudaStream_t stream);
+
+/* Workspace bytes of sa_lsa_search for these sizes (host call). */
+sa_status sa_lsa_search_workspace_size(const sa_lsa_params* prm, const sa_lsa_search_opts* opts, int32_t n_q,
+                                       int32_t q_pos0, int32_t n_blocks, size_t* bytes);
+
+/*
  * sa_workspace_size: bytes of device workspace `op` needs for these operands
  * (host call, no device work). opts points to sa_prefill_opts (PREFILL),
  * sa_decode_opts (DECODE), an int32_t k (TOPK, SPARSE_ATTN) or NULL.

@@ -34,7 +34,7 @@ SA_HOOK_NONE, SA_HOOK_THETA_POS_INF, SA_HOOK_THETA_NEG_INF, SA_HOOK_STALL_WAIT, 
 
 EXPORTS = ("sa_status_string", "sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode",
            "sa_workspace_size", "sa_sparse_attn_decode_noalloc", "sa_quantize_rows_e4m3",
-           "sa_expand_sinks_window")
+           "sa_expand_sinks_window", "sa_lsa_build_buckets", "sa_lsa_search", "sa_lsa_search_workspace_size")
 
 
 class IndexerIn(ctypes.Structure):
@@ -65,6 +65,16 @@ FLAT_PATHS = {"auto": SA_FLAT_AUTO, "table": SA_FLAT_TABLE, "stream": SA_FLAT_ST
 class DecodeOpts(ctypes.Structure):
     _fields_ = [("k", ctypes.c_int32), ("status", ctypes.c_void_p), ("test_hook", ctypes.c_int32),
                 ("stage_events", ctypes.c_void_p), ("n_stage_events", ctypes.c_int32)]
+
+
+class LsaParams(ctypes.Structure):
+    _fields_ = [("d_idx", ctypes.c_int32), ("n_pool", ctypes.c_int32), ("n_cluster", ctypes.c_int32),
+                ("n_buckets", ctypes.c_int32), ("max_bucket_keys", ctypes.c_int32)]
+
+
+class LsaSearchOpts(ctypes.Structure):
+    _fields_ = [("p", ctypes.c_int32), ("k", ctypes.c_int32), ("n_sink", ctypes.c_int32),
+                ("n_window", ctypes.c_int32), ("status", ctypes.c_void_p)]
 
 
 PREFILL_STAGES = {"flat": ("indexer", "topk", "attention"),
@@ -105,11 +115,19 @@ _lib.sa_decode.argtypes = [ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), ct
 _lib.sa_quantize_rows_e4m3.argtypes = [_P, ctypes.c_int, ctypes.c_int64, ctypes.c_int32, _P, _P, _P]
 _lib.sa_expand_sinks_window.argtypes = [_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                         ctypes.c_int32, _P, _P]
+_lib.sa_lsa_build_buckets.argtypes = [ctypes.POINTER(LsaParams), _P, ctypes.c_int32, ctypes.c_int32,
+                                      ctypes.c_int32, _P, _P, _P, _P, _P]
+_lib.sa_lsa_search.argtypes = [ctypes.POINTER(LsaParams), ctypes.POINTER(LsaSearchOpts), _P, ctypes.c_int32,
+                               ctypes.c_int32, _P, _P, _P, ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]
+_lib.sa_lsa_search_workspace_size.argtypes = [ctypes.POINTER(LsaParams), ctypes.POINTER(LsaSearchOpts),
+                                              ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                              ctypes.POINTER(ctypes.c_size_t)]
 _lib.sa_workspace_size.argtypes = [ctypes.c_int, ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), _P,
                                    ctypes.POINTER(ctypes.c_size_t)]
 _lib.sa_sparse_attn_decode_noalloc.argtypes = [ctypes.POINTER(AttnIn), _P, ctypes.c_int32, _P, _P, _P]
 for _f in ("sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode", "sa_workspace_size",
-           "sa_sparse_attn_decode_noalloc"):
+           "sa_sparse_attn_decode_noalloc", "sa_quantize_rows_e4m3", "sa_expand_sinks_window",
+           "sa_lsa_build_buckets", "sa_lsa_search", "sa_lsa_search_workspace_size"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -336,8 +354,62 @@ def expand_sinks_window(idx: torch.Tensor, q_pos0: int, n_sink: int, n_window: i
     n_q, k = idx.shape
     out = torch.empty((n_q, n_sink + n_window + k), dtype=torch.int32, device=idx.device)
     _check(_lib.sa_expand_sinks_window(_ptr(idx), n_q, k, q_pos0, n_sink, n_window, _ptr(out), _stream()),
-           "sa_expand_sinks_window")
+           "sa_expand_sinks_window", "sa_lsa_build_buckets", "sa_lsa_search", "sa_lsa_search_workspace_size")
     return out
+
+
+# ------------------------------------------------- LSA flat semantic search
+def lsa_params(n_pool: int = 4, n_cluster: int = 512, n_buckets: int = 64, max_bucket_keys: int = 32,
+               d_idx: int = 64) -> LsaParams:
+    """Clustering parameters of the bucket cache (sa_lsa_params)."""
+    return LsaParams(d_idx=d_idx, n_pool=n_pool, n_cluster=n_cluster, n_buckets=n_buckets,
+                     max_bucket_keys=max_bucket_keys)
+
+
+def lsa_build_buckets(k_idx: torch.Tensor, prm: LsaParams, n_blocks: int = None, block0: int = 0, out=None,
+                      status: torch.Tensor = None):
+    """Bucket cache of cluster blocks [block0, block0 + n_blocks) of the bf16
+    index keys k_idx [n_k, d_idx] (sa_lsa_build_buckets). Returns (centroids
+    bf16 [nb * m, d], bucket_off int32 [nb * m], bucket_keys int32
+    [nb * n_cluster]) with nb = block0 + n_blocks; `out` may pass those three
+    tensors to add blocks to an existing cache."""
+    if k_idx.dtype != torch.bfloat16 or not k_idx.is_cuda or k_idx.dim() != 2:
+        raise ValueError("k_idx: a CUDA bfloat16 tensor [n_k, d_idx]")
+    k_idx = k_idx.contiguous()
+    if n_blocks is None:
+        n_blocks = k_idx.shape[0] // prm.n_cluster - block0
+    nb = block0 + n_blocks
+    if out is None:
+        dev = k_idx.device
+        out = (torch.zeros((nb * prm.n_buckets, k_idx.shape[1]), dtype=torch.bfloat16, device=dev),
+               torch.zeros(nb * prm.n_buckets, dtype=torch.int32, device=dev),
+               torch.zeros(nb * prm.n_cluster, dtype=torch.int32, device=dev))
+    cent, off, keys = out
+    _check(_lib.sa_lsa_build_buckets(ctypes.byref(prm), _ptr(k_idx), k_idx.shape[0], block0, n_blocks, _ptr(cent),
+                                     _ptr(off), _ptr(keys), _ptr(status), _stream()), "sa_lsa_build_buckets")
+    return cent, off, keys
+
+
+def lsa_search(q_idx: torch.Tensor, prm: LsaParams, buckets, n_blocks: int, q_pos0: int, p: int, k: int,
+               n_sink: int = 0, n_window: int = 0, status: torch.Tensor = None) -> torch.Tensor:
+    """Index rows J [n_q, n_sink + n_window + k] int32 of the bf16 index
+    queries q_idx [n_q, d_idx] at positions q_pos0 + i over a bucket cache
+    from lsa_build_buckets holding n_blocks cluster blocks (sa_lsa_search)."""
+    if q_idx.dtype != torch.bfloat16 or not q_idx.is_cuda or q_idx.dim() != 2:
+        raise ValueError("q_idx: a CUDA bfloat16 tensor [n_q, d_idx]")
+    q_idx = q_idx.contiguous()
+    cent, off, keys = buckets
+    o = LsaSearchOpts(p=p, k=k, n_sink=n_sink, n_window=n_window, status=_ptr(status))
+    n_q = q_idx.shape[0]
+    nbytes = ctypes.c_size_t(0)
+    _check(_lib.sa_lsa_search_workspace_size(ctypes.byref(prm), ctypes.byref(o), n_q, q_pos0, n_blocks,
+                                             ctypes.byref(nbytes)), "sa_lsa_search_workspace_size")
+    ws = _workspace(nbytes.value, q_idx.device)
+    J = torch.empty((n_q, n_sink + n_window + k), dtype=torch.int32, device=q_idx.device)
+    _check(_lib.sa_lsa_search(ctypes.byref(prm), ctypes.byref(o), _ptr(q_idx), n_q, q_pos0, _ptr(cent), _ptr(off),
+                              _ptr(keys), n_blocks, _ptr(J), _aligned(ws), nbytes.value, _stream()),
+           "sa_lsa_search")
+    return J
 
 
 def new_status(device) -> torch.Tensor:

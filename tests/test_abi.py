@@ -127,3 +127,48 @@ def test_two_stage_workspace_covers_the_group_tables(sa):
     # rows and group key lists (8 k entries of 4 + 1 bytes per group of 8)
     R = 32768
     assert sizes[2] >= R * (4096 * 4 + 2048 * 4) + R // 8 * 8 * 2048 * 5
+
+
+def test_lsa_entry_points_validate_on_the_host(sa):
+    """sa_lsa_build_buckets / sa_lsa_search reject bad parameters before any
+    CUDA call, and an empty call is a no-op."""
+    lib = sa._lib
+    import ctypes
+    good = sa.lsa_params()
+    bad = [sa.lsa_params(n_pool=3),                       # n_cluster % n_pool
+           sa.lsa_params(max_bucket_keys=30),             # cap % n_pool
+           sa.lsa_params(n_buckets=129),                  # m > pool keys per block
+           sa.lsa_params(max_bucket_keys=12),             # cap < 2 n_cluster / m
+           sa.lsa_params(n_pool=0)]
+    for prm in bad:
+        assert lib.sa_lsa_build_buckets(ctypes.byref(prm), 256, 4096, 0, 1, 512, 768, 1024, None, None) \
+            == sa.SA_ERR_INVALID_ARGUMENT
+    # m equal to the pool keys per block needs no cap rule (no merges)
+    assert lib.sa_lsa_build_buckets(ctypes.byref(sa.lsa_params(n_buckets=128, max_bucket_keys=4)), None, 0, 0, 0,
+                                    None, None, None, None, None) == sa.SA_OK
+    assert lib.sa_lsa_build_buckets(ctypes.byref(sa.lsa_params(d_idx=128)), 256, 4096, 0, 1, 512, 768, 1024, None,
+                                    None) == sa.SA_ERR_UNSUPPORTED
+    assert lib.sa_lsa_build_buckets(ctypes.byref(sa.lsa_params(n_pool=1)), 256, 4096, 0, 1, 512, 768, 1024, None,
+                                    None) == sa.SA_ERR_UNSUPPORTED          # 512 pool keys per block
+    assert lib.sa_lsa_build_buckets(ctypes.byref(good), 256, 1000, 0, 2, 512, 768, 1024, None, None) \
+        == sa.SA_ERR_INVALID_ARGUMENT                                       # blocks beyond n_k
+    assert lib.sa_lsa_build_buckets(ctypes.byref(good), None, 4096, 0, 0, None, None, None, None, None) == sa.SA_OK
+    o = sa.LsaSearchOpts(p=512, k=2048, n_sink=4, n_window=512, status=None)
+    n = ctypes.c_size_t(0)
+    assert lib.sa_lsa_search_workspace_size(ctypes.byref(good), ctypes.byref(o), 65536, 0, 128, ctypes.byref(n)) \
+        == sa.SA_OK
+    # one chunk of 8192 rows: normalised queries, the score rows, lengths and top-p ids
+    assert n.value >= 8192 * (64 * 2 + 8192 * 4 + 4 + 512 * 4)
+    assert lib.sa_lsa_search(ctypes.byref(good), ctypes.byref(o), None, 0, 0, None, None, None, 128, None, None, 0,
+                             None) == sa.SA_OK
+    assert lib.sa_lsa_search(ctypes.byref(good), ctypes.byref(o), 256, 16, 0, 512, 768, 1024, 128, 2048, None, 0,
+                             None) == sa.SA_ERR_INVALID_ARGUMENT             # no workspace
+    for p, k, ns in [(0, 2048, 4), (512, 0, 4), (512, 2048, -1)]:
+        ob = sa.LsaSearchOpts(p=p, k=k, n_sink=ns, n_window=512, status=None)
+        assert lib.sa_lsa_search_workspace_size(ctypes.byref(good), ctypes.byref(ob), 16, 0, 8, ctypes.byref(n)) \
+            == sa.SA_ERR_INVALID_ARGUMENT
+    big_p = sa.LsaSearchOpts(p=4096, k=2048, n_sink=4, n_window=512, status=None)
+    assert lib.sa_lsa_search_workspace_size(ctypes.byref(good), ctypes.byref(big_p), 16, 0, 8, ctypes.byref(n)) \
+        == sa.SA_ERR_UNSUPPORTED
+    assert lib.sa_lsa_search_workspace_size(ctypes.byref(good), ctypes.byref(o), 16, 0, 513, ctypes.byref(n)) \
+        == sa.SA_ERR_UNSUPPORTED                                            # 32832 buckets: beyond the written-S regime

@@ -1,0 +1,238 @@
+"""Parity of the LSA flat semantic search (CUDA path through the C ABI) with
+the CPU oracle on the same seeded inputs. Needs a B200.
+
+Bucket caches are compared bit for bit: the clustering takes its merge
+decisions in fp32 with the oracle's rounding order, so centroids (bf16 bits),
+bucket offsets and key lists must be identical.
+
+Index rows: the sinks and the window are exact. The long-range part depends
+on the order of bucket scores, which the device accumulates in fp32 (tensor
+cores) and the oracle in fp64 over the same bf16 operands; the two differ by
+a few 1e-7 at d_idx = 64. A row must equal the oracle's unless the oracle's
+ranking has two scores within TIE of each other among its top p + 1 buckets,
+and at most 5 % of the rows may take that exception.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import lsa
+from workloads import LSA_WORKLOADS, LsaInputs
+from helpers import check_attention_row
+
+pytestmark = pytest.mark.gpu
+
+TIE = 1e-5
+
+
+@pytest.fixture(scope="module")
+def sa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from conftest import ensure_built
+    ensure_built()
+    import indexer_selected_top_b200 as m
+    return m
+
+
+def _params(sa, wl, **kw):
+    d = dict(n_pool=wl.n_pool, n_cluster=wl.n_cluster, n_buckets=wl.n_buckets, max_bucket_keys=wl.max_bucket_keys)
+    d.update(kw)
+    return sa.lsa_params(**d)
+
+
+def _build_both(sa, k_dev, prm, n_blocks=None):
+    cent, off, keys = sa.lsa_build_buckets(k_dev, prm, n_blocks=n_blocks)
+    torch.cuda.synchronize()
+    nb = off.numel() // prm.n_buckets
+    ref = lsa.build_buckets(k_dev.float().cpu().numpy(), prm.n_pool, prm.n_cluster, prm.n_buckets,
+                            prm.max_bucket_keys, nb)
+    return (cent, off, keys), ref, nb
+
+
+def _assert_same_cache(got, ref):
+    cent, off, keys = got
+    c_ref, o_ref, k_ref = ref
+    assert np.array_equal(off.cpu().numpy(), o_ref), "bucket offsets differ"
+    assert np.array_equal(keys.cpu().numpy(), k_ref), "bucket key lists differ"
+    g = cent.float().cpu().numpy()
+    assert np.array_equal(g.view(np.uint32), c_ref.astype(np.float32).view(np.uint32)), "centroid bits differ"
+
+
+@pytest.mark.parametrize("n_pool,n_cluster,m,cap,T", [
+    (4, 512, 64, 32, 8192),      # the pages' shape: 128 pool keys per block, two threads per bucket
+    (2, 512, 64, 32, 4096),      # 256 pool keys per block: one thread per bucket
+    (1, 64, 8, 16, 2048 + 37),   # small blocks, a ragged tail of keys past the last complete block
+    (4, 256, 32, 16, 4096),      # the tightest cap the rule allows (2 n_cluster / m)
+    (2, 128, 64, 2, 1024),       # m = pool keys per block: no merges
+])
+def test_bucket_cache_is_bit_exact(sa, n_pool, n_cluster, m, cap, T):
+    wl = LSA_WORKLOADS["lsa_t8k"].with_(T=T)
+    inp = LsaInputs(wl, "cuda", seed=1)
+    prm = sa.lsa_params(n_pool=n_pool, n_cluster=n_cluster, n_buckets=m, max_bucket_keys=cap)
+    status = sa.new_status("cuda")
+    cent, off, keys = sa.lsa_build_buckets(inp.k_idx, prm, status=status)
+    torch.cuda.synchronize()
+    assert status.cpu().tolist() == [0, 0, 0, 0]
+    nb = T // n_cluster
+    assert off.numel() == nb * m
+    ref = lsa.build_buckets(inp.k_idx.float().cpu().numpy(), n_pool, n_cluster, m, cap, nb)
+    _assert_same_cache((cent, off, keys), ref)
+
+
+def test_bucket_cache_grows_block_by_block(sa):
+    """Blocks added by later calls (as a decode appends cluster blocks) give
+    the cache one call over all of them gives."""
+    wl = LSA_WORKLOADS["lsa_t8k"]
+    inp = LsaInputs(wl, "cuda", seed=2)
+    prm = _params(sa, wl)
+    full = sa.lsa_build_buckets(inp.k_idx, prm)
+    part = sa.lsa_build_buckets(inp.k_idx, prm, n_blocks=5)
+    out = tuple(torch.zeros_like(t) for t in full)
+    for t, p in zip(out, part):
+        t[:p.numel() if t.dim() == 1 else p.shape[0]] = p
+    sa.lsa_build_buckets(inp.k_idx, prm, block0=5, n_blocks=16 - 5, out=out)
+    torch.cuda.synchronize()
+    for a, b in zip(full, out):
+        assert torch.equal(a, b)
+
+
+def _hand_cases():
+    with open(os.path.join(os.path.dirname(__file__), "golden", "lsa_hand.json")) as f:
+        return json.load(f)["cases"]
+
+
+@pytest.mark.parametrize("case", range(3))
+def test_hand_fixture_on_the_device(sa, case):
+    """The worked examples, with their 2-d keys and queries padded by zeros to
+    d_idx = 64 (zeros change no norm and no score)."""
+    c = _hand_cases()[case]
+    k = np.zeros((len(c["keys"]), 64), dtype=np.float32)
+    k[:, :c["d"]] = c["keys"]
+    k_dev = torch.from_numpy(k).to(torch.bfloat16).cuda()
+    prm = sa.lsa_params(n_pool=c["n_pool"], n_cluster=c["n_cluster"], n_buckets=c["m"],
+                        max_bucket_keys=c["max_bucket_keys"])
+    cent, off, keys = sa.lsa_build_buckets(k_dev, prm, n_blocks=c["n_blocks"])
+    torch.cuda.synchronize()
+    assert off.cpu().tolist() == c["bucket_off"]
+    assert keys.cpu().tolist() == c["bucket_keys"]
+    if "centroids" in c:
+        assert cent.float().cpu().numpy()[:, :c["d"]].tolist() == c["centroids"]
+        assert not cent.float().cpu().numpy()[:, c["d"]:].any()
+    for q in c["queries"]:
+        qv = np.zeros((1, 64), dtype=np.float32)
+        qv[0, :c["d"]] = q["q"]
+        J = sa.lsa_search(torch.from_numpy(qv).to(torch.bfloat16).cuda(), prm, (cent, off, keys), c["n_blocks"],
+                          q["pos"], q["p"], q["k"], c["n_sink"], c["n_window"])
+        torch.cuda.synchronize()
+        assert J.cpu().tolist()[0] == q["J"]
+
+
+def _tied(qn, pos, cent, n_blocks, wl, p):
+    """The oracle's ranking of the query's visible buckets has two scores
+    within TIE among its best p + 1."""
+    n_vis = min(n_blocks, pos // wl.n_cluster) * wl.n_buckets
+    if n_vis < 2:
+        return False
+    s = np.sort(lsa.bucket_scores(qn, cent, n_vis))[::-1][:p + 1]
+    return bool((np.diff(-s) < TIE).any())
+
+
+def _check_rows(J, rows, pos0, q_host, ref_cache, n_blocks, wl, p, k, n_sink, n_window):
+    cent, off, keys = ref_cache
+    qn = lsa.normalized_queries(q_host[rows])
+    exceptions = 0
+    for r, qv in zip(rows, qn):
+        pos = pos0 + r
+        want = lsa.search_row(qv, pos, cent, off, keys, n_blocks, wl.n_cluster, wl.n_buckets, p, k, n_sink,
+                              n_window)
+        got = J[r]
+        head = min(n_sink, pos + 1) + max(0, pos - max(n_sink, pos - n_window + 1) + 1)
+        assert np.array_equal(got[:head], want[:head]), f"row {pos}: sinks / window"
+        if np.array_equal(got, want):
+            continue
+        assert _tied(qv, pos, cent, n_blocks, wl, p), f"row {pos}: differs from the oracle without a score tie"
+        far = got[head:]
+        far = far[far >= 0]
+        assert len(set(far.tolist())) == len(far) and (far < (pos // wl.n_cluster) * wl.n_cluster).all()
+        exceptions += 1
+    assert exceptions <= 0.05 * len(rows), f"{exceptions} of {len(rows)} rows differ at score ties"
+    return exceptions
+
+
+def test_search_matches_oracle_t8k(sa):
+    """All 8,192 queries of the 8K workload; the oracle checks 400 rows,
+    among them the first and last rows of cluster blocks and rows that see no
+    bucket; a second call over rows 3000.. (q_pos0 = 3000, a ragged number of
+    rows) gives the same rows."""
+    wl = LSA_WORKLOADS["lsa_t8k"]
+    inp = LsaInputs(wl, "cuda", seed=3)
+    prm = _params(sa, wl)
+    cache, ref, nb = _build_both(sa, inp.k_idx, prm)
+    _assert_same_cache(cache, ref)
+    J = sa.lsa_search(inp.q_idx, prm, cache, nb, 0, wl.p, wl.k, wl.n_sink, wl.n_window)
+    J2 = sa.lsa_search(inp.q_idx[3000:], prm, cache, nb, 3000, wl.p, wl.k, wl.n_sink, wl.n_window)
+    torch.cuda.synchronize()
+    J, J2 = J.cpu().numpy(), J2.cpu().numpy()
+    assert np.array_equal(J[3000:], J2)
+    rng = np.random.default_rng(3)
+    nc = wl.n_cluster
+    edges = [0, 1, nc - 1, nc, nc + 1, 2 * nc - 1, 2 * nc, wl.T - 1]
+    rows = sorted(set(rng.choice(wl.T, 392, replace=False).tolist() + edges))
+    _check_rows(J, rows, 0, inp.q_idx.float().cpu().numpy(), ref, nb, wl, wl.p, wl.k, wl.n_sink, wl.n_window)
+
+
+@pytest.mark.parametrize("p,k,n_sink,n_window", [(100, 300, 0, 0), (7, 1000, 16, 64), (2048, 64, 4, 512),
+                                                 (1, 1, 1, 1)])
+def test_search_edge_parameters(sa, p, k, n_sink, n_window):
+    """p not a power of two, p above every row's bucket count, k above what
+    the buckets hold (short rows), no sinks or window, single entries."""
+    wl = LSA_WORKLOADS["lsa_t8k"].with_(T=4096)
+    inp = LsaInputs(wl, "cuda", seed=4)
+    prm = _params(sa, wl)
+    cache, ref, nb = _build_both(sa, inp.k_idx, prm)
+    q0, n_q = 700, 1000
+    J = sa.lsa_search(inp.q_idx[q0:q0 + n_q], prm, cache, nb, q0, p, k, n_sink, n_window)
+    torch.cuda.synchronize()
+    J = J.cpu().numpy()
+    assert J.shape == (n_q, n_sink + n_window + k)
+    rows = list(range(0, n_q, 7)) + [n_q - 1]
+    _check_rows(J, rows, q0, inp.q_idx[q0:q0 + n_q].float().cpu().numpy(), ref, nb, wl, p, k, n_sink, n_window)
+
+
+def test_search_full_size_t64k_with_attention(sa):
+    """The 64K workload as the benchmark runs it: 128 cluster blocks (bit-exact
+    cache), every query's row on the device, 64 rows checked by the oracle,
+    and sparse attention over the served rows of 8 of them."""
+    wl = LSA_WORKLOADS["lsa_t64k"]
+    inp = LsaInputs(wl, "cuda", seed=5)
+    prm = _params(sa, wl)
+    cache, ref, nb = _build_both(sa, inp.k_idx, prm)
+    _assert_same_cache(cache, ref)
+    status = sa.new_status("cuda")
+    J_dev = sa.lsa_search(inp.q_idx, prm, cache, nb, 0, wl.p, wl.k, wl.n_sink, wl.n_window, status=status)
+    torch.cuda.synchronize()
+    assert status.cpu().tolist() == [0, 0, 0, 0]
+    J = J_dev.cpu().numpy()
+    rng = np.random.default_rng(5)
+    rows = sorted(set(rng.choice(wl.T, 60, replace=False).tolist() + [511, 512, 40000, wl.T - 1]))
+    _check_rows(J, rows, 0, inp.q_idx.float().cpu().numpy(), ref, nb, wl, wl.p, wl.k, wl.n_sink, wl.n_window)
+    # every row: sinks and window first, then distinct earlier-block keys, then -1
+    far = J[:, wl.n_sink + wl.n_window:]
+    pos = np.arange(wl.T)
+    head_ok = (J[pos >= wl.n_window + wl.n_sink, :wl.n_sink] == np.arange(wl.n_sink)).all()
+    assert head_ok
+    assert (far < ((pos // wl.n_cluster) * wl.n_cluster)[:, None]).all()
+    Q, K, V = inp.attention_operands()
+    pick = rows[::8]
+    o, l = sa.sparse_attn(Q[pick], K, V, J_dev[pick].contiguous())
+    torch.cuda.synchronize()
+    o, l = o.float().cpu().numpy(), l.cpu().numpy()
+    Kh, Vh = K.double().cpu().numpy(), V.double().cpu().numpy()
+    for j, r in enumerate(pick):
+        ro, rl = oracle.sparse_attention_row(Q[r].double().cpu().numpy(), Kh, Vh, J[r])
+        check_attention_row(o[j], ro, l[j], rl, f"row {r}")

@@ -87,7 +87,7 @@ WORKLOADS = {
 # seeding: one independent stream per (seed, tensor, chunk)
 # ----------------------------------------------------------------------------
 _STREAMS = {"q": 1, "k": 2, "w": 3, "Q": 4, "K": 5, "V": 6, "dir": 7, "plant": 8,
-            "pnoise": 9, "topic": 10, "centroid": 11, "qtopic": 12}
+            "pnoise": 9, "topic": 10, "centroid": 11, "qtopic": 12, "runs": 13}
 
 
 def _mix(*vals: int) -> int:
@@ -343,3 +343,82 @@ def sample_rows(T: int, n: int, seed: int, k: int, extra=(), block: Optional[int
     picks = [int(rng.integers(edges[i], max(edges[i] + 1, edges[i + 1]))) for i in range(rest)]
     rows = sorted(set(must) | set(min(T - 1, p) for p in picks))
     return np.array(rows, dtype=np.int64)
+
+
+# ----------------------------------------------------------------------------
+# LSA semantic-search workloads
+# ----------------------------------------------------------------------------
+@dataclasses.dataclass(frozen=True)
+class LsaWorkload:
+    """Index keys and queries of the LSA flat semantic search (one bf16 head
+    of d_idx = 64), with the clustering and search parameters.
+
+    Keys follow topics that change every few tokens: ``topics`` centroids c ~
+    N(0, I_d); the sequence is cut into runs of geometric length (mean
+    ``run_mean``), each run takes a uniform topic, and its keys are c +
+    sigma N(0, I). The query at position t takes the topic of a uniformly drawn
+    position in [0, t] and is c + sigma N(0, I). Values are rounded to bf16;
+    normalisation is the method's own step, not the generator's."""
+    name: str
+    T: int
+    d: int = 64
+    n_pool: int = 4
+    n_cluster: int = 512
+    n_buckets: int = 64
+    max_bucket_keys: int = 32
+    p: int = 512
+    k: int = 2048
+    n_sink: int = 4
+    n_window: int = 512
+    topics: int = 256
+    run_mean: int = 16
+    sigma: float = 0.5
+    Hq: int = 16
+    dh: int = 128
+
+    def with_(self, **kw) -> "LsaWorkload":
+        return dataclasses.replace(self, **kw)
+
+
+LSA_WORKLOADS = {
+    # 8K tokens: 16 cluster blocks, 1,024 buckets; small enough for the oracle
+    "lsa_t8k": LsaWorkload("lsa_t8k", T=8192, p=128, k=512, topics=64),
+    # 64K tokens: 128 cluster blocks of 512 keys, 8,192 buckets of about 8 keys,
+    # p = 512 buckets for k = 2048 long-range keys, 4 sinks, a 512-key window
+    "lsa_t64k": LsaWorkload("lsa_t64k", T=65536),
+}
+
+
+class LsaInputs:
+    """k_idx [T, d] and q_idx [T, d] bf16 index keys / queries; Q [T, Hq, dh],
+    K, V [T, dh] bf16 attention operands (drawn on first use)."""
+
+    def __init__(self, wl: LsaWorkload, device="cpu", seed: int = 0):
+        self.wl, self.device, self.seed = wl, torch.device(device), seed
+        T, d, dev = wl.T, wl.d, self.device
+        rng = _np_rng(seed, "runs")
+        topic = np.empty(T, dtype=np.int64)
+        t = 0
+        while t < T:
+            n = int(rng.geometric(1.0 / wl.run_mean))
+            topic[t:t + n] = rng.integers(0, wl.topics)
+            t += n
+        src = np.minimum((_np_rng(seed, "qtopic").random(T) * (np.arange(T) + 1)).astype(np.int64), np.arange(T))
+        self.key_topic = topic
+        self.query_topic = topic[src]
+        cen = _randn((wl.topics, d), _gen(dev, seed, "centroid"), dev)
+        kt = torch.as_tensor(topic, device=dev)
+        qt = torch.as_tensor(self.query_topic, device=dev)
+        self.k_idx = (cen[kt] + wl.sigma * _randn((T, d), _gen(dev, seed, "k"), dev)).to(torch.bfloat16)
+        self.q_idx = (cen[qt] + wl.sigma * _randn((T, d), _gen(dev, seed, "q"), dev)).to(torch.bfloat16)
+        self._attn = None
+
+    def attention_operands(self):
+        if self._attn is None:
+            wl, dev, seed = self.wl, self.device, self.seed
+            std = 1.0 / math.sqrt(wl.dh)
+            Q = (_randn((wl.T, wl.Hq, wl.dh), _gen(dev, seed, "Q"), dev) * std).to(torch.bfloat16)
+            K = (_randn((wl.T, wl.dh), _gen(dev, seed, "K"), dev) * std).to(torch.bfloat16)
+            V = (_randn((wl.T, wl.dh), _gen(dev, seed, "V"), dev) * std).to(torch.bfloat16)
+            self._attn = (Q, K, V)
+        return self._attn
