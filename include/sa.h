@@ -333,10 +333,10 @@ sa_status sa_expand_sinks_window(const int32_t* idx, int32_t n_q, int32_t k, int
  *   n_cluster        keys per cluster block, a multiple of n_pool, with
  *                    n_cluster / n_pool <= 256 pool keys
  *   n_buckets        m, buckets per cluster block (1 .. n_cluster / n_pool)
- *   max_bucket_keys  n_b^max, a multiple of n_pool; unless m equals the
- *                    pool keys per block it must be >= 2 n_cluster / m (a
- *                    smaller cap can leave no pair that fits before m
- *                    buckets remain)
+ *   max_bucket_keys  n_b^max, a multiple of n_pool. With n_b^max >= 2
+ *                    n_cluster / m every block reaches m buckets; a smaller
+ *                    cap can leave no pair that fits before m buckets remain
+ *                    (sa_lsa_build_buckets then reports it, see there)
  * Violations are SA_ERR_INVALID_ARGUMENT; d_idx != 64 or more than 256 pool
  * keys per block are SA_ERR_UNSUPPORTED.
  */
@@ -373,7 +373,9 @@ typedef struct {
  *                  ascending within each bucket; block c fills [c * n_cluster,
  *                  (c + 1) * n_cluster)
  *   status (device, nullable) is zeroed by the call; error = SA_ERR_INTERNAL
- *   if a block could not reach m buckets (excluded by the cap rule above).
+ *   if a block could not reach m buckets because no remaining pair fits the
+ *   cap (only possible with n_b^max < 2 n_cluster / m); that block's outputs
+ *   are then left unwritten.
  *   k_idx and centroids must be 16-byte aligned. No workspace, no host
  *   synchronisation. n_blocks = 0 is a no-op.
  */

@@ -40,7 +40,6 @@ namespace sa {
 constexpr int TC_GA = 8;               // queries per group
 constexpr int TC_HQ = 16;
 constexpr int TC_DH = 128;
-constexpr int TC_ROWS = TC_GA * TC_HQ; // 128
 constexpr int TC_CH = kUnionChunk;     // keys per chunk (the union lists are padded to whole chunks)
 constexpr int TC_ST = 3;               // K/V ring stages
 constexpr int TC_LW = 4;               // loader warps (32 keys of every chunk each)

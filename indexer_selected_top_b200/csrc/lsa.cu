@@ -47,12 +47,6 @@ constexpr long long LSA_WAIT_BUDGET = 4000000000ll;
 
 // ------------------------------------------------------------ fp32 steps
 // One correctly rounded fp32 operation each; never contracted into an FMA.
-__device__ __forceinline__ float row_norm_f32(const float* x, int stride) {
-  float ss = __fmul_rn(x[0], x[0]);
-  for (int j = 1; j < LSA_D; ++j) ss = __fadd_rn(ss, __fmul_rn(x[j * stride], x[j * stride]));
-  return __fsqrt_rn(ss);
-}
-
 __device__ __forceinline__ void load_bf16_row(const __nv_bfloat16* src, float (&x)[LSA_D]) {
   const uint4* s4 = reinterpret_cast<const uint4*>(src);
 #pragma unroll
@@ -209,7 +203,7 @@ __global__ void __launch_bounds__(LSA_CT) lsa_cluster_kernel(ClusterArgs a) {
     }
     __syncthreads();
     const int M = sh.n_pairs, need = sh.n_alive - a.m;
-    if (M == 0) {                                  // no pair fits: excluded by the host's cap check
+    if (M == 0) {                                  // no pair fits (possible only when n_b^max < 2 n_cluster / m)
       if (tid == 0 && a.status != nullptr) atomicCAS(a.status, 0u, (uint32_t)SA_ERR_INTERNAL);
       sh.failed = 1;
       break;
@@ -490,9 +484,7 @@ static bool params_ok(const sa_lsa_params* prm) {
   if (np < 1 || nc < 1 || m < 1 || cap < 1) return false;
   if (nc % np != 0 || cap % np != 0) return false;
   const int P = nc / np;
-  if (m > P) return false;
-  if (m < P && (long long)cap * m < 2ll * nc) return false;     // progress needs n_b^max >= 2 n_cluster / m
-  return true;
+  return m <= P;
 }
 
 static bool params_supported(const sa_lsa_params* prm) {

@@ -138,7 +138,6 @@ def test_lsa_entry_points_validate_on_the_host(sa):
     bad = [sa.lsa_params(n_pool=3),                       # n_cluster % n_pool
            sa.lsa_params(max_bucket_keys=30),             # cap % n_pool
            sa.lsa_params(n_buckets=129),                  # m > pool keys per block
-           sa.lsa_params(max_bucket_keys=12),             # cap < 2 n_cluster / m
            sa.lsa_params(n_pool=0)]
     for prm in bad:
         assert lib.sa_lsa_build_buckets(ctypes.byref(prm), 256, 4096, 0, 1, 512, 768, 1024, None, None) \
