@@ -30,6 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "sparse-attn prefill tokens/s (indexer+top-k+attn) @64K k=2048; decode µs/token"
+LSA_METRIC = "LSA flat prefill tokens/s (clustering+bucket search+attn) @64K k=2048"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -175,6 +176,18 @@ def decode_work(wd):
     }
 
 
+def lsa_work(wl):
+    """Algorithmic counts of the LSA flat prefill over T tokens."""
+    T, nc, m = wl.T, wl.n_cluster, wl.n_buckets
+    nb = T // nc
+    vis = [min(nb, p // nc) * m for p in range(T)]             # buckets each query scores
+    return {
+        "scores": sum(vis),
+        "score_bytes": sum(vis) * 4,                             # S written once (read again by the top-p)
+        "score_flops": 2.0 * wl.d * sum(vis),
+    }
+
+
 # ------------------------------------------------------------- CPU oracle
 def oracle_two_stage_sample(host, wl, n_rows: int, seed: int):
     """Times the oracle on pooling (all blocks) + n_rows stratified rows of
@@ -201,6 +214,38 @@ def oracle_decode_sample(hostd, wd, n_seq: int):
     return dt / n_seq * wd.batch * 1e6, dt        # µs per decode step of the full batch
 
 
+def oracle_lsa_sample(k_host, q_host, attn_host, wl, n_rows: int, seed: int):
+    """Times the LSA oracle: the bucket cache of every cluster block, then
+    n_rows stratified query rows (search + attention); tokens/s extrapolated
+    to T rows."""
+    import numpy as np
+    import oracle
+    from oracle import lsa
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(wl.T, n_rows, replace=False))
+    t0 = time.perf_counter()
+    cent, off, keys = lsa.build_buckets(k_host, wl.n_pool, wl.n_cluster, wl.n_buckets, wl.max_bucket_keys)
+    t1 = time.perf_counter()
+    nb = wl.T // wl.n_cluster
+    qn = lsa.normalized_queries(q_host[rows])
+    Q, K, V = attn_host
+    for r, qv in zip(rows, qn):
+        J = lsa.search_row(qv, int(r), cent, off, keys, nb, wl.n_cluster, wl.n_buckets, wl.p, wl.k, wl.n_sink,
+                           wl.n_window)
+        oracle.sparse_attention_row(Q[r], K, V, J)
+    t2 = time.perf_counter()
+    full_s = (t1 - t0) + (t2 - t1) / len(rows) * wl.T
+    return wl.T / full_s, {"build_s": t1 - t0, "rows": len(rows), "rows_s": t2 - t1, "extrapolated_s": full_s}
+
+
+def lsa_host_inputs(wl, seed):
+    from workloads import LsaInputs
+    inp = LsaInputs(wl, "cpu", seed=seed)
+    Q, K, V = inp.attention_operands()
+    return (inp.k_idx.float().numpy(), inp.q_idx.float().numpy(),
+            (Q.double().numpy(), K.double().numpy(), V.double().numpy()))
+
+
 def blas_threads():
     try:
         import threadpoolctl
@@ -211,10 +256,40 @@ def blas_threads():
 
 
 # --------------------------------------------------------------- arms
+def run_reference_lsa(args):
+    """The LSA oracle as the reference arm (rank 0, host cores)."""
+    from workloads import LSA_WORKLOADS
+    wl = LSA_WORKLOADS[args.workload]
+    k_host, q_host, attn_host = lsa_host_inputs(wl, args.seed)
+    for i in range(args.warmup):
+        oracle_lsa_sample(k_host, q_host, attn_host, wl, args.ref_rows, seed=100 + i)
+    vals, infos = [], []
+    for i in range(args.steps):
+        v, info = oracle_lsa_sample(k_host, q_host, attn_host, wl, args.ref_rows, seed=200 + i)
+        vals.append(v)
+        infos.append(info)
+    value = statistics.mean(vals)
+    sample = (f"per step: the bucket cache of all {wl.T // wl.n_cluster} cluster blocks + {args.ref_rows} "
+              f"query rows (search, attention), extrapolated to {wl.T} rows")
+    line = {
+        "impl": "reference", "metric": LSA_METRIC, "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(statistics.mean(x["extrapolated_s"] for x in infos) * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 clustering, f64 scores",
+        "data": "synthetic", "config": {"workload": wl.name, "T": wl.T, "k": wl.k, "p": wl.p, "seed": args.seed},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args):
     """The oracle as the reference arm: rank 0 only, on host cores."""
     import torch
-    from workloads import WORKLOADS, PrefillInputs, DecodeInputs
+    from workloads import WORKLOADS, PrefillInputs, DecodeInputs, LSA_WORKLOADS
+    if args.workload in LSA_WORKLOADS:
+        return run_reference_lsa(args)
     wl = WORKLOADS[args.workload]
     wd = WORKLOADS["decode_b64_l128k"]
     inp = PrefillInputs(wl, "cpu", seed=args.seed)
@@ -250,9 +325,149 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_native_lsa(args, rank, world, local_rank):
+    """The LSA flat prefill: bucket cache of every cluster block, the index
+    rows of every query, attention over them."""
+    import torch
+    import torch.distributed as dist
+    import indexer_selected_top_b200 as sa
+    from workloads import LSA_WORKLOADS, LsaInputs
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = LSA_WORKLOADS[args.workload]
+    if args.T:
+        wl = wl.with_(T=args.T)
+    inp = LsaInputs(wl, dev, seed=rank_seed(args.seed, rank))
+    Q, K, V = inp.attention_operands()
+    prm = sa.lsa_params(n_pool=wl.n_pool, n_cluster=wl.n_cluster, n_buckets=wl.n_buckets,
+                        max_bucket_keys=wl.max_bucket_keys)
+    timer = sa.StageTimer(sa.LsaPrefill.STAGES)
+    status = sa.new_status(dev)
+    run = sa.LsaPrefill(inp.k_idx, inp.q_idx, Q, K, V, prm, wl.p, wl.k, wl.n_sink, wl.n_window, timer=timer,
+                        status=status)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        run()
+    torch.cuda.synchronize()
+    if status.cpu().tolist()[0] != 0:
+        raise RuntimeError(f"LSA prefill status {status.cpu().tolist()}")
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    tot, stage_ms = 0.0, {n: 0.0 for n in timer.names}
+    for _ in range(args.steps):
+        flush.fill_(1)                                   # evict L2, outside the timed events
+        run()
+        torch.cuda.synchronize()
+        for n, v in timer.ms().items():
+            stage_ms[n] += v
+        tot += timer.events[0].elapsed_time(timer.events[-1])
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    K_ = args.steps
+    tot = reduce_max([tot], device=dev)[0]
+    peaks, peak_src = load_peaks()
+    work = lsa_work(wl)
+    # attention work: the (query, key) pairs the served rows actually hold
+    work["attn_pairs"] = int((run.J >= 0).sum().item())
+    work["attn_flops"] = 4.0 * wl.Hq * wl.dh * work["attn_pairs"]
+    avg = {n: v / K_ for n, v in stage_ms.items()}
+    stages = {n: {"ms": round(v, 4)} for n, v in avg.items()}
+    # search: the score rows S are written once and read once by the top-p (HBM)
+    s_search = max(avg["search"], 1e-9) * 1e-3
+    stages["search"].update({"bound": "hbm", "achieved": round(2 * work["score_bytes"] / s_search / 1e9, 2),
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s"})
+    s_attn = max(avg["attention"], 1e-9) * 1e-3
+    stages["attention"].update({"bound": "tensor", "achieved": round(work["attn_flops"] / s_attn / 1e12, 2),
+                                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"})
+    for v in stages.values():
+        if "achieved" in v:
+            v["frac"] = round(v["achieved"] / v["peak"], 4)
+    dom = max((n for n in stages if "achieved" in stages[n]), key=lambda n: stages[n]["ms"])
+    roof = dict(stages[dom])
+    roof.pop("ms")
+    roof.update({"kernel": dom, "traffic": None,
+                 "peak_source": f"{peak_src}: " + ("bf16 burst" if roof["unit"] == "TFLOP/s" else "HBM copy")})
+    e2e = None
+    if not args.skip_e2e:
+        srcs = (inp.k_idx, inp.q_idx, Q, K, V)
+        hbuf = [t.cpu().pin_memory() for t in srcs]
+        hout = torch.empty(run.out.shape, dtype=run.out.dtype).pin_memory()
+        hlse = torch.empty(run.lse.shape, dtype=run.lse.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in hbuf)
+        d2h = hout.numel() * hout.element_size() + hlse.numel() * hlse.element_size()
+        ne = max(1, min(args.steps, args.e2e_steps))
+
+        def e2e_step():
+            for d_, h_ in zip(srcs, hbuf):
+                d_.copy_(h_, non_blocking=True)
+            run()
+            hout.copy_(run.out, non_blocking=True)
+            hlse.copy_(run.lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(ne):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        t_e2e = reduce_max([a.elapsed_time(b) / ne], device=dev)[0]
+        e2e = {"value": round(weak_scaling_value(world, 1, wl.T, t_e2e), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ne}
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+        k_host, q_host, attn_host = (inp.k_idx.float().cpu().numpy(), inp.q_idx.float().cpu().numpy(),
+                                     (Q.double().cpu().numpy(), K.double().cpu().numpy(), V.double().cpu().numpy()))
+        v, info = oracle_lsa_sample(k_host, q_host, attn_host, wl, args.lsa_cpu_rows, seed=7)
+        cpu = {"value": round(v, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"bucket cache of all {wl.T // wl.n_cluster} cluster blocks ({info['build_s']:.1f} s) + "
+                         f"{info['rows']} query rows ({info['rows_s']:.1f} s: search, attention), extrapolated "
+                         f"to {wl.T} rows"}
+    chunks = -(-wl.T // 8192)
+    launches = 1 + 5 * chunks + 1                      # clustering; per chunk qnorm, scores, lengths, top-p,
+    line = {                                           # expansion; attention
+        "metric": LSA_METRIC,
+        "value": round(weak_scaling_value(world, K_, wl.T, tot), 1),
+        "unit": "tokens/s", "n_gpus": world, "steps": K_, "warmup": args.warmup,
+        "ms_per_step": round(tot / K_, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 index (f32 clustering and accumulation), bf16 attention (f32 softmax)",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "d_idx": wl.d, "n_pool": wl.n_pool, "n_cluster": wl.n_cluster,
+                   "buckets_per_block": wl.n_buckets, "max_bucket_keys": wl.max_bucket_keys, "p": wl.p,
+                   "k": wl.k, "n_sink": wl.n_sink, "n_window": wl.n_window, "Hq": wl.Hq, "head_dim": wl.dh,
+                   "parallelism": f"replicas x{world}", "l2": "flushed (512 MB write) before every step"},
+        "roofline": roof, "stages": stages, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches * K_, "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_native(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
+    from workloads import LSA_WORKLOADS
+    if args.workload in LSA_WORKLOADS:
+        if rank == 0:
+            import importlib.util
+            spec = importlib.util.spec_from_file_location("_sa_build", os.path.join(ROOT, "indexer_selected_top_b200",
+                                                                                    "build.py"))
+            mod = importlib.util.module_from_spec(spec)
+            spec.loader.exec_module(mod)
+            mod.build()
+        if world > 1:
+            dist.barrier()
+        return run_native_lsa(args, rank, world, local_rank)
     if rank == 0:
         import importlib.util
         spec = importlib.util.spec_from_file_location("_sa_build", os.path.join(ROOT, "indexer_selected_top_b200",
@@ -481,7 +696,8 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("native", "reference"), default="native")
-    ap.add_argument("--workload", default="two_stage_t64k")
+    ap.add_argument("--workload", default="two_stage_t64k",
+                    help="two_stage_t64k (headline), another prefill workload, or lsa_t64k / lsa_t8k")
     ap.add_argument("--T", type=int, default=0, help="override the prefill length (profiling runs)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-decode", action="store_true")
@@ -490,6 +706,7 @@ def main():
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=96)
     ap.add_argument("--ref-rows", type=int, default=12)
+    ap.add_argument("--lsa-cpu-rows", type=int, default=2048, help="query rows of the LSA oracle baseline")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -412,6 +412,66 @@ def lsa_search(q_idx: torch.Tensor, prm: LsaParams, buckets, n_blocks: int, q_po
     return J
 
 
+class LsaPrefill:
+    """A prepared LSA flat prefill of one sequence: the bucket cache of its
+    complete cluster blocks (sa_lsa_build_buckets), the index rows of every
+    query (sa_lsa_search) and attention over them (sa_sparse_attn). Buffers
+    and workspaces are allocated once; stage i of a call runs between the
+    timer's events i and i + 1 (stages: cluster, search, attention)."""
+
+    STAGES = ("cluster", "search", "attention")
+
+    def __init__(self, k_idx, q_idx, Q, K, V, prm: LsaParams, p: int, k: int, n_sink: int = 4,
+                 n_window: int = 512, softmax_scale: float = 0.0, timer: "StageTimer" = None, status=None):
+        dev = Q.device
+        self.k_idx, self.q_idx = k_idx.contiguous(), q_idx.contiguous()
+        self.prm = prm
+        T = self.k_idx.shape[0]
+        self.n_blocks = T // prm.n_cluster
+        nb = self.n_blocks
+        self.cache = (torch.zeros((nb * prm.n_buckets, self.k_idx.shape[1]), dtype=torch.bfloat16, device=dev),
+                      torch.zeros(nb * prm.n_buckets, dtype=torch.int32, device=dev),
+                      torch.zeros(nb * prm.n_cluster, dtype=torch.int32, device=dev))
+        self.opts = LsaSearchOpts(p=p, k=k, n_sink=n_sink, n_window=n_window, status=_ptr(status))
+        n = ctypes.c_size_t(0)
+        _check(_lib.sa_lsa_search_workspace_size(ctypes.byref(prm), ctypes.byref(self.opts), self.q_idx.shape[0],
+                                                 0, nb, ctypes.byref(n)), "sa_lsa_search_workspace_size")
+        self.nws = n.value
+        self.ws = _workspace(self.nws, dev)
+        self.J = torch.empty((self.q_idx.shape[0], n_sink + n_window + k), dtype=torch.int32, device=dev)
+        self.att = attn_in(Q, K, V, softmax_scale)
+        self.nws_attn = workspace_size(SA_OP_SPARSE_ATTN, att=self.att, opts=self.J.shape[1])
+        self.ws_attn = _workspace(self.nws_attn, dev)
+        self.out = torch.empty_like(Q)
+        self.lse = torch.empty(Q.shape[:2], dtype=torch.float32, device=dev)
+        self.timer = timer
+        self.status = status
+        self._keep = (Q, K, V)
+
+    def __call__(self, stream=None):
+        st = _stream(stream)
+        ts = torch.cuda.current_stream() if stream is None else stream
+        ev = self.timer.events if self.timer else None
+        cent, off, keys = self.cache
+        if ev:
+            ev[0].record(ts)
+        _check(_lib.sa_lsa_build_buckets(ctypes.byref(self.prm), _ptr(self.k_idx), self.k_idx.shape[0], 0,
+                                         self.n_blocks, _ptr(cent), _ptr(off), _ptr(keys), _ptr(self.status), st),
+               "sa_lsa_build_buckets")
+        if ev:
+            ev[1].record(ts)
+        _check(_lib.sa_lsa_search(ctypes.byref(self.prm), ctypes.byref(self.opts), _ptr(self.q_idx),
+                                  self.q_idx.shape[0], 0, _ptr(cent), _ptr(off), _ptr(keys), self.n_blocks,
+                                  _ptr(self.J), _aligned(self.ws), self.nws, st), "sa_lsa_search")
+        if ev:
+            ev[2].record(ts)
+        _check(_lib.sa_sparse_attn(ctypes.byref(self.att), _ptr(self.J), self.J.shape[1], _ptr(self.out),
+                                   _ptr(self.lse), _aligned(self.ws_attn), self.nws_attn, st), "sa_sparse_attn")
+        if ev:
+            ev[3].record(ts)
+        return self.out, self.lse
+
+
 def new_status(device) -> torch.Tensor:
     """A zeroed device sa_device_status (4 x uint32, as int32)."""
     return torch.zeros(4, dtype=torch.int32, device=device)
