@@ -9,8 +9,8 @@ Index rows: the sinks and the window are exact. The long-range part depends
 on the order of bucket scores, which the device accumulates in fp32 (tensor
 cores) and the oracle in fp64 over the same bf16 operands; the two differ by
 a few 1e-7 at d_idx = 64. A row must equal the oracle's unless the oracle's
-ranking has two scores within TIE of each other among its top p + 1 buckets,
-and at most 5 % of the rows may take that exception.
+ranking has two scores within 1e-5 of each other among its top p + 1 buckets
+(tests/helpers.py), and at most 5 % of the rows may take that exception.
 """
 import json
 import os
@@ -22,11 +22,9 @@ import torch
 import oracle
 from oracle import lsa
 from workloads import LSA_WORKLOADS, LsaInputs
-from helpers import check_attention_row
+from helpers import check_attention_row, check_lsa_row
 
 pytestmark = pytest.mark.gpu
-
-TIE = 1e-5
 
 
 @pytest.fixture(scope="module")
@@ -132,16 +130,6 @@ def test_hand_fixture_on_the_device(sa, case):
         assert J.cpu().tolist()[0] == q["J"]
 
 
-def _tied(qn, pos, cent, n_blocks, wl, p):
-    """The oracle's ranking of the query's visible buckets has two scores
-    within TIE among its best p + 1."""
-    n_vis = min(n_blocks, pos // wl.n_cluster) * wl.n_buckets
-    if n_vis < 2:
-        return False
-    s = np.sort(lsa.bucket_scores(qn, cent, n_vis))[::-1][:p + 1]
-    return bool((np.diff(-s) < TIE).any())
-
-
 def _check_rows(J, rows, pos0, q_host, ref_cache, n_blocks, wl, p, k, n_sink, n_window):
     cent, off, keys = ref_cache
     qn = lsa.normalized_queries(q_host[rows])
@@ -150,16 +138,8 @@ def _check_rows(J, rows, pos0, q_host, ref_cache, n_blocks, wl, p, k, n_sink, n_
         pos = pos0 + r
         want = lsa.search_row(qv, pos, cent, off, keys, n_blocks, wl.n_cluster, wl.n_buckets, p, k, n_sink,
                               n_window)
-        got = J[r]
-        head = min(n_sink, pos + 1) + max(0, pos - max(n_sink, pos - n_window + 1) + 1)
-        assert np.array_equal(got[:head], want[:head]), f"row {pos}: sinks / window"
-        if np.array_equal(got, want):
-            continue
-        assert _tied(qv, pos, cent, n_blocks, wl, p), f"row {pos}: differs from the oracle without a score tie"
-        far = got[head:]
-        far = far[far >= 0]
-        assert len(set(far.tolist())) == len(far) and (far < (pos // wl.n_cluster) * wl.n_cluster).all()
-        exceptions += 1
+        exceptions += check_lsa_row(J[r], want, qv, pos, cent, n_blocks, wl.n_cluster, wl.n_buckets, p, n_sink,
+                                    n_window, f"row {pos}")
     assert exceptions <= 0.05 * len(rows), f"{exceptions} of {len(rows)} rows differ at score ties"
     return exceptions
 
