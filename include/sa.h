@@ -421,6 +421,36 @@ sa_status sa_lsa_search_workspace_size(const sa_lsa_params* prm, const sa_lsa_se
                                        int32_t q_pos0, int32_t n_blocks, size_t* bytes);
 
 /*
+ * sa_lsa_decode: one LSA decode step for `batch` sequences, each with its own
+ *   bucket cache (appendix F.1 "Flat decode": every request adds one query
+ *   per step, which scores the centroids of its request once, on the CUDA
+ *   cores -- at one flop per byte the scan is bound by HBM).
+ *   q_idx: device bf16 [batch, 64], the new index query of each sequence; it
+ *   sits at position seq_lens[b] - 1 (seq_lens: device int32 [batch], >= 1).
+ *   The caches are per-sequence slabs of what sa_lsa_build_buckets writes
+ *   for that sequence's keys: centroids bf16 [batch, max_blocks * m, 64],
+ *   bucket_off int32 [batch, max_blocks * m], bucket_keys int32 [batch,
+ *   max_blocks * n_cluster], positions within the sequence. n_blocks: device
+ *   int32 [batch], the cluster blocks each cache holds; the query scores the
+ *   buckets of blocks c < min(n_blocks[b], max_blocks, (seq_lens[b] - 1) /
+ *   n_cluster). Selection and the row layout are those of sa_lsa_search.
+ *   J: device int32 [batch, n_sink + n_window + k].
+ *   max_blocks * m <= 32768 (else SA_ERR_UNSUPPORTED). Workspace:
+ *   sa_lsa_decode_workspace_size bytes, 256-byte aligned. No host
+ *   synchronisation and no allocation, and every size is fixed by max_blocks
+ *   and batch (lengths are read on the device): the call can be captured in a
+ *   CUDA graph.
+ */
+sa_status sa_lsa_decode(const sa_lsa_params* prm, const sa_lsa_search_opts* opts, const void* q_idx, int32_t batch,
+                        const void* centroids, const int32_t* bucket_off, const int32_t* bucket_keys,
+                        int32_t max_blocks, const int32_t* n_blocks, const int32_t* seq_lens, int32_t* J, void* ws,
+                        size_t ws_bytes, cudaStream_t stream);
+
+/* Workspace bytes of sa_lsa_decode for these sizes (host call). */
+sa_status sa_lsa_decode_workspace_size(const sa_lsa_params* prm, const sa_lsa_search_opts* opts, int32_t batch,
+                                       int32_t max_blocks, size_t* bytes);
+
+/*
  * sa_workspace_size: bytes of device workspace `op` needs for these operands
  * (host call, no device work). opts points to sa_prefill_opts (PREFILL),
  * sa_decode_opts (DECODE), an int32_t k (TOPK, SPARSE_ATTN) or NULL.

@@ -34,7 +34,8 @@ SA_HOOK_NONE, SA_HOOK_THETA_POS_INF, SA_HOOK_THETA_NEG_INF, SA_HOOK_STALL_WAIT, 
 
 EXPORTS = ("sa_status_string", "sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode",
            "sa_workspace_size", "sa_sparse_attn_decode_noalloc", "sa_quantize_rows_e4m3",
-           "sa_expand_sinks_window", "sa_lsa_build_buckets", "sa_lsa_search", "sa_lsa_search_workspace_size")
+           "sa_expand_sinks_window", "sa_lsa_build_buckets", "sa_lsa_search", "sa_lsa_search_workspace_size", "sa_lsa_decode",
+           "sa_lsa_decode_workspace_size")
 
 
 class IndexerIn(ctypes.Structure):
@@ -122,12 +123,17 @@ _lib.sa_lsa_search.argtypes = [ctypes.POINTER(LsaParams), ctypes.POINTER(LsaSear
 _lib.sa_lsa_search_workspace_size.argtypes = [ctypes.POINTER(LsaParams), ctypes.POINTER(LsaSearchOpts),
                                               ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                               ctypes.POINTER(ctypes.c_size_t)]
+_lib.sa_lsa_decode.argtypes = [ctypes.POINTER(LsaParams), ctypes.POINTER(LsaSearchOpts), _P, ctypes.c_int32, _P,
+                               _P, _P, ctypes.c_int32, _P, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.sa_lsa_decode_workspace_size.argtypes = [ctypes.POINTER(LsaParams), ctypes.POINTER(LsaSearchOpts),
+                                              ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
 _lib.sa_workspace_size.argtypes = [ctypes.c_int, ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), _P,
                                    ctypes.POINTER(ctypes.c_size_t)]
 _lib.sa_sparse_attn_decode_noalloc.argtypes = [ctypes.POINTER(AttnIn), _P, ctypes.c_int32, _P, _P, _P]
 for _f in ("sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode", "sa_workspace_size",
            "sa_sparse_attn_decode_noalloc", "sa_quantize_rows_e4m3", "sa_expand_sinks_window",
-           "sa_lsa_build_buckets", "sa_lsa_search", "sa_lsa_search_workspace_size"):
+           "sa_lsa_build_buckets", "sa_lsa_search", "sa_lsa_search_workspace_size", "sa_lsa_decode",
+           "sa_lsa_decode_workspace_size"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -470,6 +476,53 @@ class LsaPrefill:
         if ev:
             ev[3].record(ts)
         return self.out, self.lse
+
+
+class LsaDecode:
+    """A prepared LSA decode step (sa_lsa_decode) for `batch` sequences with
+    per-sequence bucket caches: centroids [batch, max_blocks * m, 64] bf16,
+    bucket_off [batch, max_blocks * m] and bucket_keys [batch, max_blocks *
+    n_cluster] int32 (each slab as lsa_build_buckets writes it for that
+    sequence), n_blocks and seq_lens [batch] int32 on the device. Inputs are
+    read from the tensors given here at every call, so a captured graph
+    (graph()) replays over whatever they hold."""
+
+    def __init__(self, q_idx, prm: LsaParams, caches, n_blocks, seq_lens, p: int, k: int, n_sink: int = 4,
+                 n_window: int = 512, status=None):
+        self.q_idx, self.prm = q_idx, prm
+        self.cent, self.off, self.keys = caches
+        self.batch = q_idx.shape[0]
+        self.max_blocks = self.off.shape[1] // prm.n_buckets
+        self.n_blocks, self.seq_lens = n_blocks, seq_lens
+        self.opts = LsaSearchOpts(p=p, k=k, n_sink=n_sink, n_window=n_window, status=_ptr(status))
+        n = ctypes.c_size_t(0)
+        _check(_lib.sa_lsa_decode_workspace_size(ctypes.byref(prm), ctypes.byref(self.opts), self.batch,
+                                                 self.max_blocks, ctypes.byref(n)), "sa_lsa_decode_workspace_size")
+        self.nws = n.value
+        self.ws = _workspace(self.nws, q_idx.device)
+        self.J = torch.empty((self.batch, n_sink + n_window + k), dtype=torch.int32, device=q_idx.device)
+        self.status = status
+
+    def __call__(self, stream=None):
+        _check(_lib.sa_lsa_decode(ctypes.byref(self.prm), ctypes.byref(self.opts), _ptr(self.q_idx), self.batch,
+                                  _ptr(self.cent), _ptr(self.off), _ptr(self.keys), self.max_blocks,
+                                  _ptr(self.n_blocks), _ptr(self.seq_lens), _ptr(self.J), _aligned(self.ws),
+                                  self.nws, _stream(stream)), "sa_lsa_decode")
+        return self.J
+
+    def graph(self) -> "torch.cuda.CUDAGraph":
+        """The step captured as a CUDA graph, after one eager run (first-launch
+        setup stays out of the graph); every replay reruns it on the same
+        buffers."""
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self(s)
+        torch.cuda.current_stream().wait_stream(s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            self(s)
+        return g
 
 
 def new_status(device) -> torch.Tensor:

@@ -400,6 +400,38 @@ __global__ void lsa_rowlen_kernel(int rows, int pos0, int n_cluster, int m, int 
   if (i < rows) len[i] = visible_buckets(pos0 + i, n_cluster, m, n_blocks);
 }
 
+// ------------------------------------------------------- decode scores
+// One new query per sequence scores the centroids of its own cache on the
+// CUDA cores: a thread per bucket reads its 128-byte centroid once (the scan
+// is bound by HBM at one flop per byte, appendix F.1 "Flat decode").
+struct DecodeScoreArgs {
+  const __nv_bfloat16* cent;   // [batch, max_blocks * m, 64]
+  const __nv_bfloat16* qn;     // [batch, 64] unit queries
+  const int* n_blocks;         // [batch] cluster blocks in each cache
+  const int* seq_lens;         // [batch] the query sits at seq_lens[b] - 1
+  int n_cluster, m, max_blocks;
+  float* S;                    // [batch, ld]
+  long long ld;
+  int* len;                    // [batch] visible buckets
+};
+
+__global__ void __launch_bounds__(256) lsa_decode_score_kernel(DecodeScoreArgs a) {
+  const int sq = blockIdx.y;
+  const int pos = a.seq_lens[sq] - 1;
+  const int nb = max(0, min(min(a.n_blocks[sq], a.max_blocks), pos >= 0 ? pos / a.n_cluster : 0));
+  const int vis = nb * a.m;
+  if (blockIdx.x == 0 && threadIdx.x == 0) a.len[sq] = vis;
+  const int b = blockIdx.x * 256 + threadIdx.x;
+  if (b >= vis) return;
+  float q[LSA_D], x[LSA_D];
+  load_bf16_row(a.qn + (long long)sq * LSA_D, q);
+  load_bf16_row(a.cent + ((long long)sq * a.max_blocks * a.m + b) * LSA_D, x);
+  float acc = 0.f;
+#pragma unroll
+  for (int j = 0; j < LSA_D; ++j) acc = fmaf(q[j], x[j], acc);
+  a.S[(long long)sq * a.ld + b] = acc;
+}
+
 // ------------------------------------------------------------ expansion
 struct ExpandArgs {
   const float* S;              // [rows, ld]
@@ -408,8 +440,10 @@ struct ExpandArgs {
   int p, psort;                // psort: power of two >= p
   const int32_t* bucket_off;
   const int32_t* bucket_keys;
+  long long off_stride, keys_stride;   // per row (decode: every sequence has its own cache), else 0
   int n_cluster, m;
   int rows, pos0;
+  const int* seq_lens;         // decode: row i sits at seq_lens[i] - 1 (else at pos0 + i)
   int k, n_sink, n_window;
   int32_t* J;                  // [rows, n_sink + n_window + k]
 };
@@ -418,9 +452,11 @@ __global__ void __launch_bounds__(TK_THREADS) lsa_expand_kernel(ExpandArgs a) {
   __shared__ unsigned long long sig[LSA_PSORT_MAX];
   __shared__ int red[TK_THREADS / 32];
   const int i = blockIdx.x, tid = threadIdx.x;
-  const int pos = a.pos0 + i;
+  const int pos = a.seq_lens != nullptr ? a.seq_lens[i] - 1 : a.pos0 + i;
   const float* srow = a.S + (long long)i * a.ld;
   const int32_t* srl = a.sel + (long long)i * a.p;
+  const int32_t* boff = a.bucket_off + (long long)i * a.off_stride;
+  const int32_t* bkeys = a.bucket_keys + (long long)i * a.keys_stride;
   for (int j = tid; j < a.psort; j += TK_THREADS) {
     const int b = j < a.p ? srl[j] : -1;
     sig[j] = b >= 0 ? ((unsigned long long)score_key(srow[b]) << 32) | (uint32_t)~(uint32_t)b : 0ull;
@@ -458,17 +494,17 @@ __global__ void __launch_bounds__(TK_THREADS) lsa_expand_kernel(ExpandArgs a) {
     if (j < a.psort && sig[j] != 0ull) {
       const int b = (int)~(uint32_t)(sig[j] & 0xFFFFFFFFull);
       const int c = b / a.m;
-      lo = a.bucket_off[b];
-      hi = (b - c * a.m == a.m - 1) ? (c + 1) * a.n_cluster : a.bucket_off[b + 1];
+      lo = boff[b];
+      hi = (b - c * a.m == a.m - 1) ? (c + 1) * a.n_cluster : boff[b + 1];
       for (int e = lo; e < hi; ++e) {
-        const int s = a.bucket_keys[e];
+        const int s = bkeys[e];
         u += (s < a.n_sink || s >= w_lo) ? 0 : 1;
       }
     }
     int tot;
     const int at = run + block_excl_scan(u, red, &tot);
     for (int e = lo, w = at; e < hi && w < a.k; ++e) {
-      const int s = a.bucket_keys[e];
+      const int s = bkeys[e];
       if (s < a.n_sink || s >= w_lo) continue;
       far[w++] = s;
     }
@@ -636,6 +672,9 @@ extern "C" sa_status sa_lsa_search(const sa_lsa_params* prm, const sa_lsa_search
     ea.psort = pl.psort;
     ea.bucket_off = bucket_off;
     ea.bucket_keys = bucket_keys;
+    ea.off_stride = 0;
+    ea.keys_stride = 0;
+    ea.seq_lens = nullptr;
     ea.n_cluster = nc;
     ea.m = m;
     ea.rows = rows;
@@ -648,4 +687,116 @@ extern "C" sa_status sa_lsa_search(const sa_lsa_params* prm, const sa_lsa_search
     if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
   }
   return SA_OK;
+}
+
+// ------------------------------------------------------------- decode step
+namespace sa {
+
+struct DecodePlan {
+  long long ld;
+  int psort;
+  size_t off_qn, off_S, off_len, off_sel, total;
+};
+
+static DecodePlan plan_decode(const sa_lsa_params* prm, const sa_lsa_search_opts* o, int batch, int max_blocks) {
+  DecodePlan pl{};
+  const long long nb = (long long)max_blocks * prm->n_buckets;
+  pl.ld = ((nb > 0 ? nb : 1) + LSA_TILE - 1) / LSA_TILE * LSA_TILE;
+  pl.psort = 1;
+  while (pl.psort < o->p) pl.psort <<= 1;
+  size_t off = 0;
+  pl.off_qn = off;
+  off = up256(off + (size_t)batch * LSA_D * 2);
+  pl.off_S = off;
+  off = up256(off + (size_t)batch * pl.ld * 4);
+  pl.off_len = off;
+  off = up256(off + (size_t)batch * 4);
+  pl.off_sel = off;
+  off = up256(off + (size_t)batch * o->p * 4);
+  pl.total = off;
+  return pl;
+}
+
+static sa_status check_decode(const sa_lsa_params* prm, const sa_lsa_search_opts* o, int batch, int max_blocks) {
+  if (!params_ok(prm) || o == nullptr) return SA_ERR_INVALID_ARGUMENT;
+  if (batch < 0 || max_blocks < 0) return SA_ERR_INVALID_ARGUMENT;
+  if (o->p < 1 || o->k < 1 || o->n_sink < 0 || o->n_window < 0) return SA_ERR_INVALID_ARGUMENT;
+  if (!params_supported(prm) || o->p > LSA_PSORT_MAX) return SA_ERR_UNSUPPORTED;
+  if ((long long)max_blocks * prm->n_buckets > LSA_MAX_BUCKETS) return SA_ERR_UNSUPPORTED;
+  return SA_OK;
+}
+
+}  // namespace sa
+
+extern "C" sa_status sa_lsa_decode_workspace_size(const sa_lsa_params* prm, const sa_lsa_search_opts* o,
+                                                  int32_t batch, int32_t max_blocks, size_t* bytes) {
+  if (bytes == nullptr) return SA_ERR_INVALID_ARGUMENT;
+  const sa_status s = check_decode(prm, o, batch, max_blocks);
+  if (s != SA_OK) return s;
+  *bytes = batch == 0 ? 0 : plan_decode(prm, o, batch, max_blocks).total;
+  return SA_OK;
+}
+
+extern "C" sa_status sa_lsa_decode(const sa_lsa_params* prm, const sa_lsa_search_opts* o, const void* q_idx,
+                                   int32_t batch, const void* centroids, const int32_t* bucket_off,
+                                   const int32_t* bucket_keys, int32_t max_blocks, const int32_t* n_blocks,
+                                   const int32_t* seq_lens, int32_t* J, void* ws, size_t ws_bytes,
+                                   cudaStream_t stream) {
+  const sa_status s = check_decode(prm, o, batch, max_blocks);
+  if (s != SA_OK) return s;
+  if (o->status != nullptr && cudaMemsetAsync(o->status, 0, sizeof(sa_device_status), stream) != cudaSuccess)
+    return SA_ERR_CUDA;
+  if (batch == 0) return SA_OK;
+  if (q_idx == nullptr || J == nullptr || ws == nullptr || n_blocks == nullptr || seq_lens == nullptr)
+    return SA_ERR_INVALID_ARGUMENT;
+  if (max_blocks > 0 && (centroids == nullptr || bucket_off == nullptr || bucket_keys == nullptr))
+    return SA_ERR_INVALID_ARGUMENT;
+  if (!aligned16(q_idx) || (max_blocks > 0 && !aligned16(centroids))) return SA_ERR_INVALID_ARGUMENT;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return SA_ERR_INVALID_ARGUMENT;
+  const DecodePlan pl = plan_decode(prm, o, batch, max_blocks);
+  if (ws_bytes < pl.total) return SA_ERR_WORKSPACE_TOO_SMALL;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  __nv_bfloat16* qn = reinterpret_cast<__nv_bfloat16*>(w + pl.off_qn);
+  float* S = reinterpret_cast<float*>(w + pl.off_S);
+  int* len = reinterpret_cast<int*>(w + pl.off_len);
+  int32_t* sel = reinterpret_cast<int32_t*>(w + pl.off_sel);
+  const int m = prm->n_buckets, nc = prm->n_cluster;
+  const int nbmax = max_blocks * m;
+  lsa_qnorm_kernel<<<(batch + 255) / 256, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(q_idx), batch, qn);
+  DecodeScoreArgs da;
+  da.cent = static_cast<const __nv_bfloat16*>(centroids);
+  da.qn = qn;
+  da.n_blocks = n_blocks;
+  da.seq_lens = seq_lens;
+  da.n_cluster = nc;
+  da.m = m;
+  da.max_blocks = max_blocks;
+  da.S = S;
+  da.ld = pl.ld;
+  da.len = len;
+  const dim3 grid((unsigned)max(1, (nbmax + 255) / 256), (unsigned)batch);
+  lsa_decode_score_kernel<<<grid, 256, 0, stream>>>(da);
+  cudaError_t e = launch_topk_table(S, batch, max(nbmax, 1), pl.ld, 0, o->p, sel, 1, nullptr, 0, len, stream);
+  if (e != cudaSuccess) return SA_ERR_CUDA;
+  ExpandArgs ea;
+  ea.S = S;
+  ea.ld = pl.ld;
+  ea.sel = sel;
+  ea.p = o->p;
+  ea.psort = pl.psort;
+  ea.bucket_off = bucket_off;
+  ea.bucket_keys = bucket_keys;
+  ea.off_stride = (long long)max_blocks * m;
+  ea.keys_stride = (long long)max_blocks * nc;
+  ea.n_cluster = nc;
+  ea.m = m;
+  ea.rows = batch;
+  ea.pos0 = 0;
+  ea.seq_lens = seq_lens;
+  ea.k = o->k;
+  ea.n_sink = o->n_sink;
+  ea.n_window = o->n_window;
+  ea.J = J;
+  lsa_expand_kernel<<<batch, TK_THREADS, 0, stream>>>(ea);
+  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }

@@ -171,3 +171,26 @@ def test_lsa_entry_points_validate_on_the_host(sa):
         == sa.SA_ERR_UNSUPPORTED
     assert lib.sa_lsa_search_workspace_size(ctypes.byref(good), ctypes.byref(o), 16, 0, 513, ctypes.byref(n)) \
         == sa.SA_ERR_UNSUPPORTED                                            # 32832 buckets: beyond the written-S regime
+
+
+def test_lsa_decode_validates_on_the_host(sa):
+    import ctypes
+    lib = sa._lib
+    good = sa.lsa_params()
+    o = sa.LsaSearchOpts(p=512, k=2048, n_sink=4, n_window=512, status=None)
+    n = ctypes.c_size_t(0)
+    assert lib.sa_lsa_decode_workspace_size(ctypes.byref(good), ctypes.byref(o), 64, 256, ctypes.byref(n)) == sa.SA_OK
+    assert n.value >= 64 * (64 * 2 + 256 * 64 * 4 + 4 + 512 * 4)
+    assert lib.sa_lsa_decode_workspace_size(ctypes.byref(good), ctypes.byref(o), 64, 513, ctypes.byref(n)) \
+        == sa.SA_ERR_UNSUPPORTED
+    assert lib.sa_lsa_decode_workspace_size(ctypes.byref(sa.lsa_params(n_pool=3)), ctypes.byref(o), 64, 16,
+                                            ctypes.byref(n)) == sa.SA_ERR_INVALID_ARGUMENT
+    # batch 0: a no-op; missing lengths, caches or workspace: rejected before any launch
+    assert lib.sa_lsa_decode(ctypes.byref(good), ctypes.byref(o), None, 0, None, None, None, 16, None, None, None,
+                             None, 0, None) == sa.SA_OK
+    assert lib.sa_lsa_decode(ctypes.byref(good), ctypes.byref(o), 256, 4, 512, 768, 1024, 16, None, 2048, 4096,
+                             8192, 1 << 20, None) == sa.SA_ERR_INVALID_ARGUMENT
+    assert lib.sa_lsa_decode(ctypes.byref(good), ctypes.byref(o), 256, 4, None, 768, 1024, 16, 1280, 2048, 4096,
+                             8192, 1 << 20, None) == sa.SA_ERR_INVALID_ARGUMENT
+    assert lib.sa_lsa_decode(ctypes.byref(good), ctypes.byref(o), 256, 4, 512, 768, 1024, 16, 1280, 2048, 4096,
+                             8192, 256, None) == sa.SA_ERR_WORKSPACE_TOO_SMALL

@@ -216,3 +216,78 @@ def test_search_full_size_t64k_with_attention(sa):
     for j, r in enumerate(pick):
         ro, rl = oracle.sparse_attention_row(Q[r].double().cpu().numpy(), Kh, Vh, J[r])
         check_attention_row(o[j], ro, l[j], rl, f"row {r}")
+
+
+def _decode_setup(sa, lens, max_blocks, seed):
+    """Per-sequence caches (slabs written by lsa_build_buckets for each
+    sequence's own keys), the new queries, and the oracle's caches."""
+    wl = LSA_WORKLOADS["lsa_t8k"]
+    prm = _params(sa, wl)
+    B, m, nc = len(lens), wl.n_buckets, wl.n_cluster
+    cent = torch.zeros((B, max_blocks * m, 64), dtype=torch.bfloat16, device="cuda")
+    off = torch.zeros((B, max_blocks * m), dtype=torch.int32, device="cuda")
+    keys = torch.zeros((B, max_blocks * nc), dtype=torch.int32, device="cuda")
+    q = torch.empty((B, 64), dtype=torch.bfloat16, device="cuda")
+    refs, n_blocks = [], []
+    for b, L in enumerate(lens):
+        inp = LsaInputs(wl.with_(T=L), "cuda", seed=seed + b)
+        nb = min(max_blocks, L // nc)
+        sa.lsa_build_buckets(inp.k_idx, prm, n_blocks=nb, out=(cent[b], off[b], keys[b]))
+        q[b] = inp.q_idx[L - 1]
+        refs.append(lsa.build_buckets(inp.k_idx.float().cpu().numpy(), wl.n_pool, nc, m, wl.max_bucket_keys, nb))
+        n_blocks.append(nb)
+    torch.cuda.synchronize()
+    nbt = torch.tensor(n_blocks, dtype=torch.int32, device="cuda")
+    lt = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    return wl, prm, (cent, off, keys), q, nbt, lt, refs
+
+
+def _check_decode_rows(J, q, lens, refs, nbt, wl, p, k):
+    qn = lsa.normalized_queries(q.float().cpu().numpy())
+    for b, L in enumerate(lens):
+        cent, off, keys = refs[b]
+        nb = int(nbt[b])
+        want = lsa.search_row(qn[b], L - 1, cent, off, keys, nb, wl.n_cluster, wl.n_buckets, p, k, wl.n_sink,
+                              wl.n_window)
+        check_lsa_row(J[b], want, qn[b], L - 1, cent, nb, wl.n_cluster, wl.n_buckets, p, wl.n_sink, wl.n_window,
+                      f"sequence {b}")
+
+
+def test_decode_step_matches_oracle(sa):
+    """One decode step of 6 sequences of 8192, 5000, 4096, 600, 100 and 1
+    tokens over per-sequence caches of up to 16 cluster blocks (the longest
+    one with a cache one block short of its length): each new query's row
+    against the oracle's prefill row at that position."""
+    lens = [8192, 5000, 4096, 600, 100, 1]
+    wl, prm, caches, q, nbt, lt, refs = _decode_setup(sa, lens, 16, seed=20)
+    nbt[0] = 15                                      # a cache that lags its sequence by one block
+    status = sa.new_status("cuda")
+    dec = sa.LsaDecode(q, prm, caches, nbt, lt, wl.p, wl.k, wl.n_sink, wl.n_window, status=status)
+    J = dec().cpu().numpy()
+    torch.cuda.synchronize()
+    assert status.cpu().tolist() == [0, 0, 0, 0]
+    _check_decode_rows(J, q, lens, refs, nbt.cpu().numpy(), wl, wl.p, wl.k)
+
+
+def test_decode_step_replays_as_a_cuda_graph(sa):
+    """The step captured once, replayed after new queries and shorter lengths
+    are written into its input tensors, gives the eager rows."""
+    lens = [8192, 7000, 3000, 1500]
+    wl, prm, caches, q, nbt, lt, refs = _decode_setup(sa, lens, 16, seed=30)
+    dec = sa.LsaDecode(q, prm, caches, nbt, lt, wl.p, wl.k, wl.n_sink, wl.n_window)
+    g = dec.graph()
+    g.replay()
+    torch.cuda.synchronize()
+    first = dec.J.clone()
+    eager = dec().clone()
+    torch.cuda.synchronize()
+    assert torch.equal(first, eager)
+    new_lens = [6000, 7000, 2000, 1500]
+    gen = torch.Generator(device="cuda").manual_seed(31)
+    q.copy_(torch.randn(q.shape, generator=gen, device="cuda").to(torch.bfloat16))
+    lt.copy_(torch.tensor(new_lens, dtype=torch.int32))
+    g.replay()
+    torch.cuda.synchronize()
+    J = dec.J.cpu().numpy()
+    _check_decode_rows(J, q, new_lens, refs, nbt.cpu().numpy(), wl, wl.p, wl.k)
+    del g
