@@ -383,12 +383,27 @@ sa_status sa_lsa_build_buckets(const sa_lsa_params* prm, const void* k_idx, int3
                                int32_t n_blocks, void* centroids, int32_t* bucket_off, int32_t* bucket_keys,
                                sa_device_status* status, cudaStream_t stream);
 
+/* Search regimes (appendix F.1 "Flat prefill"): TABLE writes each query's
+ * bucket scores and selects its top p from them; STREAM never writes them:
+ * a threshold per query from about 8192 sampled centroids, a scan that lists
+ * the buckets at or above it (room for 3p), the top p of the list, and a
+ * whole-row rescoring for the rows whose list missed (fewer than p listed, or
+ * more than its room; their count is read back to the host once per chunk of
+ * 8192 queries). Both select the same buckets from the same scores. AUTO
+ * takes TABLE up to 32,768 buckets and STREAM beyond. */
+#define SA_LSA_AUTO 0
+#define SA_LSA_TABLE 1
+#define SA_LSA_STREAM 2
+
 typedef struct {
   int32_t p;          /* buckets kept per query, 1 .. 2048 */
   int32_t k;          /* long-range keys per query, >= 1 */
   int32_t n_sink;     /* attention-sink keys 0 .. n_sink - 1, >= 0 */
   int32_t n_window;   /* most recent keys, >= 0 */
-  sa_device_status* status;   /* device, nullable; zeroed by the call */
+  sa_device_status* status;   /* device, nullable; zeroed by the call (STREAM counts its fallback and
+                                 overflowed rows there) */
+  int32_t regime;     /* SA_LSA_AUTO, SA_LSA_TABLE or SA_LSA_STREAM (sa_lsa_search only) */
+  int32_t test_hook;  /* 0; SA_HOOK_THETA_POS_INF / _NEG_INF force every STREAM row to its fallback */
 } sa_lsa_search_opts;
 
 /*
@@ -406,10 +421,12 @@ typedef struct {
  *   sinks ascending, the window ascending, the long-range keys (best bucket
  *   first), then -1. Fewer than k long-range keys when the p buckets hold
  *   fewer uncovered keys.
- *   Scores are written to the workspace (the pages' short-context regime):
- *   n_blocks * m must be <= 32768 (else SA_ERR_UNSUPPORTED). Workspace:
- *   sa_lsa_search_workspace_size bytes, 256-byte aligned. No host
- *   synchronisation; status error = SA_ERR_TIMEOUT if a bounded wait gave up.
+ *   Regimes: see SA_LSA_*. TABLE needs n_blocks * m <= 32768 and STREAM
+ *   n_blocks * m <= 2^21 (else SA_ERR_UNSUPPORTED). Workspace:
+ *   sa_lsa_search_workspace_size bytes (for the same opts), 256-byte
+ *   aligned. TABLE does not synchronise the host; STREAM synchronises the
+ *   stream once per chunk of 8192 queries. status error = SA_ERR_TIMEOUT if
+ *   a bounded wait gave up.
  */
 sa_status sa_lsa_search(const sa_lsa_params* prm, const sa_lsa_search_opts* opts, const void* q_idx, int32_t n_q,
                         int32_t q_pos0, const void* centroids, const int32_t* bucket_off,

@@ -75,7 +75,12 @@ class LsaParams(ctypes.Structure):
 
 class LsaSearchOpts(ctypes.Structure):
     _fields_ = [("p", ctypes.c_int32), ("k", ctypes.c_int32), ("n_sink", ctypes.c_int32),
-                ("n_window", ctypes.c_int32), ("status", ctypes.c_void_p)]
+                ("n_window", ctypes.c_int32), ("status", ctypes.c_void_p), ("regime", ctypes.c_int32),
+                ("test_hook", ctypes.c_int32)]
+
+
+SA_LSA_AUTO, SA_LSA_TABLE, SA_LSA_STREAM = 0, 1, 2
+LSA_REGIMES = {"auto": SA_LSA_AUTO, "table": SA_LSA_TABLE, "stream": SA_LSA_STREAM}
 
 
 PREFILL_STAGES = {"flat": ("indexer", "topk", "attention"),
@@ -397,15 +402,19 @@ def lsa_build_buckets(k_idx: torch.Tensor, prm: LsaParams, n_blocks: int = None,
 
 
 def lsa_search(q_idx: torch.Tensor, prm: LsaParams, buckets, n_blocks: int, q_pos0: int, p: int, k: int,
-               n_sink: int = 0, n_window: int = 0, status: torch.Tensor = None) -> torch.Tensor:
+               n_sink: int = 0, n_window: int = 0, status: torch.Tensor = None, regime: str = "auto",
+               test_hook: int = 0) -> torch.Tensor:
     """Index rows J [n_q, n_sink + n_window + k] int32 of the bf16 index
     queries q_idx [n_q, d_idx] at positions q_pos0 + i over a bucket cache
-    from lsa_build_buckets holding n_blocks cluster blocks (sa_lsa_search)."""
+    from lsa_build_buckets holding n_blocks cluster blocks (sa_lsa_search).
+    regime: "auto", "table" (bucket scores written) or "stream" (threshold
+    scan, no score matrix)."""
     if q_idx.dtype != torch.bfloat16 or not q_idx.is_cuda or q_idx.dim() != 2:
         raise ValueError("q_idx: a CUDA bfloat16 tensor [n_q, d_idx]")
     q_idx = q_idx.contiguous()
     cent, off, keys = buckets
-    o = LsaSearchOpts(p=p, k=k, n_sink=n_sink, n_window=n_window, status=_ptr(status))
+    o = LsaSearchOpts(p=p, k=k, n_sink=n_sink, n_window=n_window, status=_ptr(status), regime=LSA_REGIMES[regime],
+                      test_hook=test_hook)
     n_q = q_idx.shape[0]
     nbytes = ctypes.c_size_t(0)
     _check(_lib.sa_lsa_search_workspace_size(ctypes.byref(prm), ctypes.byref(o), n_q, q_pos0, n_blocks,
@@ -428,7 +437,8 @@ class LsaPrefill:
     STAGES = ("cluster", "search", "attention")
 
     def __init__(self, k_idx, q_idx, Q, K, V, prm: LsaParams, p: int, k: int, n_sink: int = 4,
-                 n_window: int = 512, softmax_scale: float = 0.0, timer: "StageTimer" = None, status=None):
+                 n_window: int = 512, softmax_scale: float = 0.0, timer: "StageTimer" = None, status=None,
+                 regime: str = "auto"):
         dev = Q.device
         self.k_idx, self.q_idx = k_idx.contiguous(), q_idx.contiguous()
         self.prm = prm
@@ -438,7 +448,8 @@ class LsaPrefill:
         self.cache = (torch.zeros((nb * prm.n_buckets, self.k_idx.shape[1]), dtype=torch.bfloat16, device=dev),
                       torch.zeros(nb * prm.n_buckets, dtype=torch.int32, device=dev),
                       torch.zeros(nb * prm.n_cluster, dtype=torch.int32, device=dev))
-        self.opts = LsaSearchOpts(p=p, k=k, n_sink=n_sink, n_window=n_window, status=_ptr(status))
+        self.opts = LsaSearchOpts(p=p, k=k, n_sink=n_sink, n_window=n_window, status=_ptr(status),
+                                  regime=LSA_REGIMES[regime], test_hook=0)
         n = ctypes.c_size_t(0)
         _check(_lib.sa_lsa_search_workspace_size(ctypes.byref(prm), ctypes.byref(self.opts), self.q_idx.shape[0],
                                                  0, nb, ctypes.byref(n)), "sa_lsa_search_workspace_size")

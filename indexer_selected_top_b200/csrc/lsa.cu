@@ -315,14 +315,26 @@ __device__ __forceinline__ int visible_buckets(int pos, int n_cluster, int m, in
 struct ScoreArgs {
   const __nv_bfloat16* cent;   // [n_buckets, 64]
   const __nv_bfloat16* qn;     // [rows, 64] unit queries of the chunk
-  int n_buckets;               // buckets in the cache
+  int n_buckets;               // rows of cent
   int rows, pos0;              // chunk rows; position of row 0
+  const int* row_pos;          // position of every row (ascending), overriding pos0 + row when non-null
+  int col_stride;              // column b holds bucket b * col_stride (the sampled buckets of the estimate)
   int n_cluster, m, n_blocks;
-  float* S;                    // [rows, ld]
+  float* S;                    // table mode: [rows, ld]
   long long ld;
+  // candidate mode: every visible bucket b with score >= theta[row] is appended
+  // to the row's list as (score key << 32 | ~b); cnt[row] counts past cap
+  const float* theta;
+  unsigned long long* cand;    // [rows, cap]
+  int* cnt;                    // [rows]
+  int cap;
   uint32_t* status;
   long long budget;
 };
+
+__device__ __forceinline__ int row_position(const ScoreArgs& a, int i) {
+  return a.row_pos != nullptr ? a.row_pos[i] : a.pos0 + i;
+}
 
 // 128 rows x 64 bf16 (128 B each) into the 128-byte-swizzled K-major layout
 // of the MMA: row r's 16-byte chunk c at r * 128 + ((c ^ (r & 7)) << 4).
@@ -336,6 +348,7 @@ __device__ __forceinline__ void stage_rows_sw128(uint8_t* dst, const __nv_bfloat
   }
 }
 
+template <bool CAND>
 __global__ void __launch_bounds__(LSA_ST) lsa_score_kernel(ScoreArgs a) {
   extern __shared__ uint8_t lsa_score_raw[];
   __shared__ uint64_t bar;
@@ -343,7 +356,8 @@ __global__ void __launch_bounds__(LSA_ST) lsa_score_kernel(ScoreArgs a) {
   __shared__ uint32_t abort_flag;
   const int b0 = blockIdx.x * LSA_TILE, i0 = blockIdx.y * LSA_TILE;
   const int i_last = min(a.rows, i0 + LSA_TILE) - 1;
-  if (b0 >= visible_buckets(a.pos0 + i_last, a.n_cluster, a.m, a.n_blocks)) return;   // no query sees the tile
+  if ((long long)b0 * a.col_stride >= visible_buckets(row_position(a, i_last), a.n_cluster, a.m, a.n_blocks))
+    return;                                 // no query of the tile sees a bucket of it
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lsa_score_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = sm;                         // 128 buckets x 64 (16 KB)
   uint8_t* sB = sm + LSA_TILE * 128;        // 128 queries x 64 (16 KB)
@@ -383,10 +397,32 @@ __global__ void __launch_bounds__(LSA_ST) lsa_score_kernel(ScoreArgs a) {
       tmem_ld32(t_row + c0, v);
       tmem_ld_wait();
       tmem_regs_ready(v);
+      if constexpr (!CAND) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int i = i0 + c0 + j;
-        if (i < a.rows) a.S[(long long)i * a.ld + b] = v[j];
+        for (int j = 0; j < 32; ++j) {
+          const int i = i0 + c0 + j;
+          if (i < a.rows) a.S[(long long)i * a.ld + b] = v[j];
+        }
+      } else {
+        // threshold scan: one ballot per (warp, query), one atomic when a lane hits
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int i = i0 + c0 + j;
+          if (i < a.rows) {
+            const int vis = visible_buckets(row_position(a, i), a.n_cluster, a.m, a.n_blocks);
+            const bool hit = b < vis && v[j] >= a.theta[i];
+            const unsigned bal = __ballot_sync(0xffffffffu, hit);
+            if (bal != 0u) {
+              int base = 0;
+              if (lane == 0) base = atomicAdd(a.cnt + i, __popc(bal));
+              base = __shfl_sync(0xffffffffu, base, 0);
+              const int slot = base + __popc(bal & ((1u << lane) - 1u));
+              if (hit && slot < a.cap)
+                a.cand[(long long)i * a.cap + slot] =
+                    ((unsigned long long)score_key(v[j]) << 32) | (uint32_t)~(uint32_t)b;
+            }
+          }
+        }
       }
     }
   }
@@ -395,9 +431,112 @@ __global__ void __launch_bounds__(LSA_ST) lsa_score_kernel(ScoreArgs a) {
   if (warp == 0) tmem_dealloc<LSA_TILE>(tmem);
 }
 
-__global__ void lsa_rowlen_kernel(int rows, int pos0, int n_cluster, int m, int n_blocks, int* len) {
+__global__ void lsa_rowlen_kernel(int rows, int pos0, const int* row_pos, int n_cluster, int m, int n_blocks,
+                                  int* len) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < rows) len[i] = visible_buckets(pos0 + i, n_cluster, m, n_blocks);
+  if (i < rows) len[i] = visible_buckets(row_pos != nullptr ? row_pos[i] : pos0 + i, n_cluster, m, n_blocks);
+}
+
+// ------------------------------------------------ threshold regime pieces
+// Appendix F.1 "Selection by threshold": theta_i is set before the scan from
+// a sample of the row; the scan lists every bucket at or above it; only the
+// list is ranked; a row whose list holds fewer than p buckets, or more than
+// its room, falls back to its whole row. Here the sample is every stride-th
+// bucket (about 8192 of them); the query sees the n_vs samples below its
+// visible bucket count vis and takes the round(gamma p n_vs / vis)-th largest
+// sampled score, so that its list holds about gamma p buckets. Rows whose
+// visible buckets all fit in the list take theta = -inf.
+constexpr float LSA_GAMMA = 1.5f;   // list target gamma p, room 3p (twice the target, as the pages size it)
+constexpr int LSA_SAMPLES = 8192;
+
+__device__ __forceinline__ float lsa_key_to_float(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+__global__ void __launch_bounds__(TK_THREADS, 1)
+    lsa_theta_kernel(const float* __restrict__ stab, long long ld, int pos0, int n_cluster, int m, int n_blocks,
+                     int stride, int p, int cap, int hook, float* __restrict__ theta) {
+  extern __shared__ uint8_t lsa_th_raw[];
+  TkShared& sh = *reinterpret_cast<TkShared*>(lsa_th_raw);
+  const int t = blockIdx.x, tid = threadIdx.x;
+  const int vis = visible_buckets(pos0 + t, n_cluster, m, n_blocks);
+  float th;
+  if (hook == SA_HOOK_THETA_POS_INF) {
+    th = INFINITY;
+  } else if (hook == SA_HOOK_THETA_NEG_INF || vis <= cap) {
+    th = -INFINITY;
+  } else {
+    const int n_vs = (vis + stride - 1) / stride;
+    const long long want = llrintf(LSA_GAMMA * (float)p * (float)n_vs / (float)vis);
+    int need = (int)max(1ll, min((long long)n_vs, want));
+    const float* row = stab + (long long)t * ld;
+    uint32_t prefix = 0;
+    int pbits = 0;
+    while (pbits < 32) {                    // 12 + 12 + 8 bits: the exact need-th largest sample
+      const int db = (pbits == 24) ? 8 : TK_HBITS;
+      const int nbins = 1 << db;
+      for (int b = tid; b < nbins; b += TK_THREADS) sh.hist[b] = 0;
+      __syncthreads();
+      const int sdig = 32 - pbits - db;
+      for (int j = tid; j < n_vs; j += TK_THREADS) {
+        const uint32_t key = score_key(row[j]);
+        if (pbits == 0 || (key >> (32 - pbits)) == prefix) atomicAdd(&sh.hist[(key >> sdig) & (nbins - 1)], 1u);
+      }
+      __syncthreads();
+      find_bucket(sh, nbins, need);
+      need -= sh.above;
+      prefix = (prefix << db) | (uint32_t)sh.bucket;
+      pbits += db;
+      __syncthreads();
+    }
+    th = lsa_key_to_float(prefix);
+  }
+  if (tid == 0) theta[t] = th;
+}
+
+// The top-p of each row's list, written as packed keys (0 past the row's
+// min(p, vis) entries); rows whose list missed are flagged for the fallback.
+__global__ void __launch_bounds__(TK_THREADS, 1)
+    lsa_select_kernel(const unsigned long long* __restrict__ cand, const int* __restrict__ cnt, int cap, int pos0,
+                      int n_cluster, int m, int n_blocks, int p, unsigned long long* __restrict__ sig,
+                      int* __restrict__ miss, uint32_t* status) {
+  extern __shared__ uint8_t lsa_sel_raw[];
+  TkShared& sh = *reinterpret_cast<TkShared*>(lsa_sel_raw);
+  const int t = blockIdx.x, tid = threadIdx.x;
+  const int vis = visible_buckets(pos0 + t, n_cluster, m, n_blocks);
+  const int need = min(p, vis);
+  const int c = cnt[t];
+  const bool ok = c <= cap && c >= need;
+  if (tid == 0) {
+    miss[t] = ok ? 0 : 1;
+    if (status != nullptr) {
+      if (!ok) atomicAdd(status + 2, 1u);
+      if (c > cap) atomicAdd(status + 3, 1u);
+    }
+    sh.n_out = 0;
+  }
+  if (!ok) return;
+  const unsigned long long* row = cand + (long long)t * cap;
+  for (int j = tid; j < c; j += TK_THREADS) sh.cand[j] = row[j];
+  __syncthreads();
+  unsigned long long* out = sig + (long long)t * p;
+  smem_select64(sh, c, need, [&](uint64_t key) { out[atomicAdd(&sh.n_out, 1)] = key; });
+  for (int j = need + tid; j < p; j += TK_THREADS) out[j] = 0ull;
+}
+
+// Packed keys of the fallback rows from their rescored rows: fallback row f
+// (of n_f) is chunk row rows[f]; its top-p bucket ids sel[f] index S row f.
+__global__ void __launch_bounds__(256)
+    lsa_sig_from_table_kernel(const float* __restrict__ S, long long ld, const int32_t* __restrict__ sel, int p,
+                              const int* __restrict__ rows, int n_f, unsigned long long* __restrict__ sig) {
+  const int f = blockIdx.x;
+  if (f >= n_f) return;
+  unsigned long long* out = sig + (long long)rows[f] * p;
+  for (int j = threadIdx.x; j < p; j += 256) {
+    const int b = sel[(long long)f * p + j];
+    out[j] = b >= 0 ? ((unsigned long long)score_key(S[(long long)f * ld + b]) << 32) | (uint32_t)~(uint32_t)b
+                    : 0ull;
+  }
 }
 
 // ------------------------------------------------------- decode scores
@@ -434,6 +573,7 @@ __global__ void __launch_bounds__(256) lsa_decode_score_kernel(DecodeScoreArgs a
 
 // ------------------------------------------------------------ expansion
 struct ExpandArgs {
+  const unsigned long long* sig_in;   // [rows, p] packed keys of the top-p (0 = none), or null: from S and sel
   const float* S;              // [rows, ld]
   long long ld;
   const int32_t* sel;          // [rows, p] top-p bucket ids (any order, -1 padded)
@@ -458,8 +598,12 @@ __global__ void __launch_bounds__(TK_THREADS) lsa_expand_kernel(ExpandArgs a) {
   const int32_t* boff = a.bucket_off + (long long)i * a.off_stride;
   const int32_t* bkeys = a.bucket_keys + (long long)i * a.keys_stride;
   for (int j = tid; j < a.psort; j += TK_THREADS) {
-    const int b = j < a.p ? srl[j] : -1;
-    sig[j] = b >= 0 ? ((unsigned long long)score_key(srow[b]) << 32) | (uint32_t)~(uint32_t)b : 0ull;
+    if (a.sig_in != nullptr) {
+      sig[j] = j < a.p ? a.sig_in[(long long)i * a.p + j] : 0ull;
+    } else {
+      const int b = j < a.p ? srl[j] : -1;
+      sig[j] = b >= 0 ? ((unsigned long long)score_key(srow[b]) << 32) | (uint32_t)~(uint32_t)b : 0ull;
+    }
   }
   __syncthreads();
   // bitonic sort, descending: best bucket first (higher score, then lower id)
@@ -529,18 +673,33 @@ static bool params_supported(const sa_lsa_params* prm) {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+constexpr int LSA_MAX_BUCKETS_STREAM = 1 << 21;   // the threshold regime: up to 16M tokens at 8 keys a bucket
+
 struct SearchPlan {
+  bool stream;      // threshold regime (no score matrix)
   int R;            // query rows per chunk
   long long ld;     // score row stride (multiple of the tile)
   int psort;
-  size_t off_qn, off_S, off_len, off_sel, total;
+  // table regime
+  size_t off_qn, off_S, off_len, off_sel;
+  // threshold regime
+  int stride, n_s, cap, F;
+  long long ld_s;
+  size_t off_cs, off_stab, off_theta, off_cand, off_cnt, off_miss, off_frows, off_fpos, off_count, off_qnf, off_Sf,
+      off_lenf, off_self, off_sig;
+  size_t total;
 };
 
 static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
+static bool use_stream(const sa_lsa_search_opts* o, long long nb) {
+  return o->regime == SA_LSA_STREAM || (o->regime == SA_LSA_AUTO && nb > LSA_MAX_BUCKETS);
+}
+
 static SearchPlan plan_search(const sa_lsa_params* prm, const sa_lsa_search_opts* o, int n_q, int n_blocks) {
   SearchPlan pl{};
   const long long nb = (long long)n_blocks * prm->n_buckets;
+  pl.stream = use_stream(o, nb);
   pl.ld = ((nb > 0 ? nb : 1) + LSA_TILE - 1) / LSA_TILE * LSA_TILE;
   pl.R = max(1, min(n_q, 8192));
   pl.psort = 1;
@@ -548,12 +707,49 @@ static SearchPlan plan_search(const sa_lsa_params* prm, const sa_lsa_search_opts
   size_t off = 0;
   pl.off_qn = off;
   off = up256(off + (size_t)pl.R * LSA_D * 2);
-  pl.off_S = off;
-  off = up256(off + (size_t)pl.R * pl.ld * 4);
-  pl.off_len = off;
+  if (!pl.stream) {
+    pl.off_S = off;
+    off = up256(off + (size_t)pl.R * pl.ld * 4);
+    pl.off_len = off;
+    off = up256(off + (size_t)pl.R * 4);
+    pl.off_sel = off;
+    off = up256(off + (size_t)pl.R * o->p * 4);
+    pl.total = off;
+    return pl;
+  }
+  pl.stride = (int)max(1ll, (nb + LSA_SAMPLES - 1) / LSA_SAMPLES);
+  pl.n_s = (int)max(1ll, (nb + pl.stride - 1) / pl.stride);
+  pl.ld_s = ((long long)pl.n_s + LSA_TILE - 1) / LSA_TILE * LSA_TILE;
+  pl.cap = 3 * o->p;
+  pl.F = (int)max(16ll, min(1024ll, (512ll << 20) / (pl.ld * 4)));
+  pl.off_cs = off;
+  off = up256(off + (size_t)pl.n_s * LSA_D * 2);
+  pl.off_stab = off;
+  off = up256(off + (size_t)pl.R * pl.ld_s * 4);
+  pl.off_theta = off;
   off = up256(off + (size_t)pl.R * 4);
-  pl.off_sel = off;
-  off = up256(off + (size_t)pl.R * o->p * 4);
+  pl.off_cand = off;
+  off = up256(off + (size_t)pl.R * pl.cap * 8);
+  pl.off_cnt = off;
+  off = up256(off + (size_t)pl.R * 4);
+  pl.off_miss = off;
+  off = up256(off + (size_t)pl.R * 4);
+  pl.off_frows = off;
+  off = up256(off + (size_t)pl.R * 4);
+  pl.off_fpos = off;
+  off = up256(off + (size_t)pl.R * 4);
+  pl.off_count = off;
+  off = up256(off + 4);
+  pl.off_qnf = off;
+  off = up256(off + (size_t)pl.F * LSA_D * 2);
+  pl.off_Sf = off;
+  off = up256(off + (size_t)pl.F * pl.ld * 4);
+  pl.off_lenf = off;
+  off = up256(off + (size_t)pl.F * 4);
+  pl.off_self = off;
+  off = up256(off + (size_t)pl.F * o->p * 4);
+  pl.off_sig = off;
+  off = up256(off + (size_t)pl.R * o->p * 8);
   pl.total = off;
   return pl;
 }
@@ -563,8 +759,10 @@ static sa_status check_search(const sa_lsa_params* prm, const sa_lsa_search_opts
   if (!params_ok(prm) || o == nullptr) return SA_ERR_INVALID_ARGUMENT;
   if (n_q < 0 || q_pos0 < 0 || n_blocks < 0) return SA_ERR_INVALID_ARGUMENT;
   if (o->p < 1 || o->k < 1 || o->n_sink < 0 || o->n_window < 0) return SA_ERR_INVALID_ARGUMENT;
+  if (o->regime < SA_LSA_AUTO || o->regime > SA_LSA_STREAM) return SA_ERR_INVALID_ARGUMENT;
   if (!params_supported(prm) || o->p > LSA_PSORT_MAX) return SA_ERR_UNSUPPORTED;
-  if ((long long)n_blocks * prm->n_buckets > LSA_MAX_BUCKETS) return SA_ERR_UNSUPPORTED;
+  const long long nb = (long long)n_blocks * prm->n_buckets;
+  if (nb > (use_stream(o, nb) ? LSA_MAX_BUCKETS_STREAM : LSA_MAX_BUCKETS)) return SA_ERR_UNSUPPORTED;
   return SA_OK;
 }
 
@@ -630,44 +828,137 @@ extern "C" sa_status sa_lsa_search(const sa_lsa_params* prm, const sa_lsa_search
   if (ws_bytes < pl.total) return SA_ERR_WORKSPACE_TOO_SMALL;
   uint8_t* w = static_cast<uint8_t*>(ws);
   __nv_bfloat16* qn = reinterpret_cast<__nv_bfloat16*>(w + pl.off_qn);
-  float* S = reinterpret_cast<float*>(w + pl.off_S);
-  int* len = reinterpret_cast<int*>(w + pl.off_len);
-  int32_t* sel = reinterpret_cast<int32_t*>(w + pl.off_sel);
-  const int nc = prm->n_cluster, m = prm->n_buckets;
+  const int nc = prm->n_cluster, m = prm->n_buckets, nb_all = n_blocks * m;
   const long long width = (long long)o->n_sink + o->n_window + o->k;
-  if (cudaFuncSetAttribute(lsa_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LSA_SCORE_SMEM) !=
-      cudaSuccess)
+  const __nv_bfloat16* cent = static_cast<const __nv_bfloat16*>(centroids);
+  uint32_t* status = reinterpret_cast<uint32_t*>(o->status);
+  if (cudaFuncSetAttribute(lsa_score_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, LSA_SCORE_SMEM) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(lsa_score_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, LSA_SCORE_SMEM) !=
+          cudaSuccess)
     return SA_ERR_CUDA;
+  if (pl.stream) {
+    const int tks = (int)sizeof(TkShared);
+    if (cudaFuncSetAttribute(lsa_theta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tks) != cudaSuccess ||
+        cudaFuncSetAttribute(lsa_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tks) != cudaSuccess)
+      return SA_ERR_CUDA;
+  }
+  // the sampled centroids of the threshold estimate: every stride-th bucket
+  __nv_bfloat16* cs = pl.stream ? reinterpret_cast<__nv_bfloat16*>(w + pl.off_cs) : nullptr;
+  if (pl.stream && nb_all > 0 &&
+      launch_gather_rows(cent, cs, nullptr, pl.n_s, LSA_D * 2, pl.stride, LSA_D * 2, stream) != cudaSuccess)
+    return SA_ERR_CUDA;
+  ScoreArgs base{};
+  base.qn = qn;
+  base.n_cluster = nc;
+  base.m = m;
+  base.n_blocks = n_blocks;
+  base.col_stride = 1;
+  base.status = status;
+  base.budget = LSA_WAIT_BUDGET;
   for (int r0 = 0; r0 < n_q; r0 += pl.R) {
     const int rows = min(pl.R, n_q - r0), pos0 = q_pos0 + r0;
     lsa_qnorm_kernel<<<(rows + 255) / 256, 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(q_idx) + (long long)r0 * LSA_D, rows, qn);
     // buckets the chunk's last query sees (positions grow with the row)
     const int nbv = min(n_blocks, (pos0 + rows - 1) / nc) * m;
-    if (nbv > 0) {
-      ScoreArgs sa_;
-      sa_.cent = static_cast<const __nv_bfloat16*>(centroids);
-      sa_.qn = qn;
-      sa_.n_buckets = n_blocks * m;
-      sa_.rows = rows;
-      sa_.pos0 = pos0;
-      sa_.n_cluster = nc;
-      sa_.m = m;
-      sa_.n_blocks = n_blocks;
-      sa_.S = S;
-      sa_.ld = pl.ld;
-      sa_.status = reinterpret_cast<uint32_t*>(o->status);
-      sa_.budget = LSA_WAIT_BUDGET;
-      const dim3 grid((nbv + LSA_TILE - 1) / LSA_TILE, (rows + LSA_TILE - 1) / LSA_TILE);
-      lsa_score_kernel<<<grid, LSA_ST, LSA_SCORE_SMEM, stream>>>(sa_);
+    const dim3 grid((nbv + LSA_TILE - 1) / LSA_TILE, (rows + LSA_TILE - 1) / LSA_TILE);
+    base.rows = rows;
+    base.pos0 = pos0;
+    base.row_pos = nullptr;
+    ExpandArgs ea{};
+    if (!pl.stream) {
+      // table regime: S written, the top-p of each row by the radix select
+      float* S = reinterpret_cast<float*>(w + pl.off_S);
+      int* len = reinterpret_cast<int*>(w + pl.off_len);
+      int32_t* sel = reinterpret_cast<int32_t*>(w + pl.off_sel);
+      if (nbv > 0) {
+        ScoreArgs sa_ = base;
+        sa_.cent = cent;
+        sa_.n_buckets = nb_all;
+        sa_.S = S;
+        sa_.ld = pl.ld;
+        lsa_score_kernel<false><<<grid, LSA_ST, LSA_SCORE_SMEM, stream>>>(sa_);
+      }
+      lsa_rowlen_kernel<<<(rows + 255) / 256, 256, 0, stream>>>(rows, pos0, nullptr, nc, m, n_blocks, len);
+      if (launch_topk_table(S, rows, max(nbv, 1), pl.ld, pos0, o->p, sel, 1, nullptr, 0, len, stream) != cudaSuccess)
+        return SA_ERR_CUDA;
+      ea.sig_in = nullptr;
+      ea.S = S;
+      ea.ld = pl.ld;
+      ea.sel = sel;
+    } else {
+      // threshold regime (appendix F.1 "Selection by threshold"): no score matrix
+      float* stab = reinterpret_cast<float*>(w + pl.off_stab);
+      float* theta = reinterpret_cast<float*>(w + pl.off_theta);
+      unsigned long long* cand = reinterpret_cast<unsigned long long*>(w + pl.off_cand);
+      int* cnt = reinterpret_cast<int*>(w + pl.off_cnt);
+      int* miss = reinterpret_cast<int*>(w + pl.off_miss);
+      int* frows = reinterpret_cast<int*>(w + pl.off_frows);
+      int* fpos = reinterpret_cast<int*>(w + pl.off_fpos);
+      int* count = reinterpret_cast<int*>(w + pl.off_count);
+      unsigned long long* sig = reinterpret_cast<unsigned long long*>(w + pl.off_sig);
+      if (nbv > 0) {
+        ScoreArgs ss = base;              // sampled scores
+        ss.cent = cs;
+        ss.n_buckets = pl.n_s;
+        ss.col_stride = pl.stride;
+        ss.S = stab;
+        ss.ld = pl.ld_s;
+        const int nsv = (nbv + pl.stride - 1) / pl.stride;
+        lsa_score_kernel<false>
+            <<<dim3((nsv + LSA_TILE - 1) / LSA_TILE, grid.y), LSA_ST, LSA_SCORE_SMEM, stream>>>(ss);
+      }
+      lsa_theta_kernel<<<rows, TK_THREADS, sizeof(TkShared), stream>>>(stab, pl.ld_s, pos0, nc, m, n_blocks,
+                                                                       pl.stride, o->p, pl.cap, o->test_hook, theta);
+      if (cudaMemsetAsync(cnt, 0, (size_t)rows * 4, stream) != cudaSuccess) return SA_ERR_CUDA;
+      if (nbv > 0) {
+        ScoreArgs sc = base;              // the scan: compare with theta, list the hits
+        sc.cent = cent;
+        sc.n_buckets = nb_all;
+        sc.theta = theta;
+        sc.cand = cand;
+        sc.cnt = cnt;
+        sc.cap = pl.cap;
+        lsa_score_kernel<true><<<grid, LSA_ST, LSA_SCORE_SMEM, stream>>>(sc);
+      }
+      lsa_select_kernel<<<rows, TK_THREADS, sizeof(TkShared), stream>>>(cand, cnt, pl.cap, pos0, nc, m, n_blocks,
+                                                                        o->p, sig, miss, status);
+      if (launch_compact_rows(miss, rows, frows, count, pos0, fpos, stream) != cudaSuccess) return SA_ERR_CUDA;
+      // the fallback: the missed rows rescore their whole row (the host reads their count, as in the pages)
+      int n_miss = 0;
+      if (cudaMemcpyAsync(&n_miss, count, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+          cudaStreamSynchronize(stream) != cudaSuccess)
+        return SA_ERR_CUDA;
+      __nv_bfloat16* qnf = reinterpret_cast<__nv_bfloat16*>(w + pl.off_qnf);
+      float* Sf = reinterpret_cast<float*>(w + pl.off_Sf);
+      int* lenf = reinterpret_cast<int*>(w + pl.off_lenf);
+      int32_t* self = reinterpret_cast<int32_t*>(w + pl.off_self);
+      for (int f0 = 0; f0 < n_miss; f0 += pl.F) {
+        const int nf = min(pl.F, n_miss - f0);
+        if (launch_gather_rows(qn, qnf, frows + f0, nf, LSA_D * 2, 0, LSA_D * 2, stream) != cudaSuccess)
+          return SA_ERR_CUDA;
+        ScoreArgs sf = base;
+        sf.cent = cent;
+        sf.n_buckets = nb_all;
+        sf.qn = qnf;
+        sf.rows = nf;
+        sf.row_pos = fpos + f0;
+        sf.S = Sf;
+        sf.ld = pl.ld;
+        lsa_score_kernel<false>
+            <<<dim3(grid.x, (nf + LSA_TILE - 1) / LSA_TILE), LSA_ST, LSA_SCORE_SMEM, stream>>>(sf);
+        lsa_rowlen_kernel<<<(nf + 255) / 256, 256, 0, stream>>>(nf, 0, fpos + f0, nc, m, n_blocks, lenf);
+        if (launch_topk_table(Sf, nf, max(nbv, 1), pl.ld, 0, o->p, self, 1, nullptr, 0, lenf, stream) !=
+            cudaSuccess)
+          return SA_ERR_CUDA;
+        lsa_sig_from_table_kernel<<<nf, 256, 0, stream>>>(Sf, pl.ld, self, o->p, frows + f0, nf, sig);
+      }
+      ea.sig_in = sig;
+      ea.S = nullptr;
+      ea.ld = 0;
+      ea.sel = nullptr;
     }
-    lsa_rowlen_kernel<<<(rows + 255) / 256, 256, 0, stream>>>(rows, pos0, nc, m, n_blocks, len);
-    cudaError_t e = launch_topk_table(S, rows, max(nbv, 1), pl.ld, pos0, o->p, sel, 1, nullptr, 0, len, stream);
-    if (e != cudaSuccess) return SA_ERR_CUDA;
-    ExpandArgs ea;
-    ea.S = S;
-    ea.ld = pl.ld;
-    ea.sel = sel;
     ea.p = o->p;
     ea.psort = pl.psort;
     ea.bucket_off = bucket_off;
@@ -778,7 +1069,8 @@ extern "C" sa_status sa_lsa_decode(const sa_lsa_params* prm, const sa_lsa_search
   lsa_decode_score_kernel<<<grid, 256, 0, stream>>>(da);
   cudaError_t e = launch_topk_table(S, batch, max(nbmax, 1), pl.ld, 0, o->p, sel, 1, nullptr, 0, len, stream);
   if (e != cudaSuccess) return SA_ERR_CUDA;
-  ExpandArgs ea;
+  ExpandArgs ea{};
+  ea.sig_in = nullptr;
   ea.S = S;
   ea.ld = pl.ld;
   ea.sel = sel;

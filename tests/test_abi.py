@@ -169,8 +169,12 @@ def test_lsa_entry_points_validate_on_the_host(sa):
     big_p = sa.LsaSearchOpts(p=4096, k=2048, n_sink=4, n_window=512, status=None)
     assert lib.sa_lsa_search_workspace_size(ctypes.byref(good), ctypes.byref(big_p), 16, 0, 8, ctypes.byref(n)) \
         == sa.SA_ERR_UNSUPPORTED
+    # 32,832 buckets: beyond the written-S regime, so AUTO takes the threshold regime and TABLE refuses
     assert lib.sa_lsa_search_workspace_size(ctypes.byref(good), ctypes.byref(o), 16, 0, 513, ctypes.byref(n)) \
-        == sa.SA_ERR_UNSUPPORTED                                            # 32832 buckets: beyond the written-S regime
+        == sa.SA_OK
+    ot = sa.LsaSearchOpts(p=512, k=2048, n_sink=4, n_window=512, status=None, regime=sa.SA_LSA_TABLE, test_hook=0)
+    assert lib.sa_lsa_search_workspace_size(ctypes.byref(good), ctypes.byref(ot), 16, 0, 513, ctypes.byref(n)) \
+        == sa.SA_ERR_UNSUPPORTED
 
 
 def test_lsa_decode_validates_on_the_host(sa):
@@ -194,3 +198,29 @@ def test_lsa_decode_validates_on_the_host(sa):
                              8192, 1 << 20, None) == sa.SA_ERR_INVALID_ARGUMENT
     assert lib.sa_lsa_decode(ctypes.byref(good), ctypes.byref(o), 256, 4, 512, 768, 1024, 16, 1280, 2048, 4096,
                              8192, 256, None) == sa.SA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_lsa_search_regimes_validate_and_size(sa):
+    """TABLE is limited to 32,768 buckets, STREAM to 2^21; AUTO switches at
+    32,768; a STREAM workspace holds the lists (3p packed keys per row) and
+    no score matrix."""
+    import ctypes
+    lib = sa._lib
+    good = sa.lsa_params()
+    n = ctypes.c_size_t(0)
+
+    def size(regime, n_blocks, p=512):
+        o = sa.LsaSearchOpts(p=p, k=2048, n_sink=4, n_window=512, status=None, regime=regime, test_hook=0)
+        st = lib.sa_lsa_search_workspace_size(ctypes.byref(good), ctypes.byref(o), 65536, 0, n_blocks,
+                                              ctypes.byref(n))
+        return st, n.value
+
+    assert size(3, 16)[0] == sa.SA_ERR_INVALID_ARGUMENT
+    assert size(sa.SA_LSA_TABLE, 1024)[0] == sa.SA_ERR_UNSUPPORTED          # 65,536 buckets
+    st, auto_big = size(sa.SA_LSA_AUTO, 1024)
+    st2, stream_big = size(sa.SA_LSA_STREAM, 1024)
+    assert st == st2 == sa.SA_OK and auto_big == stream_big
+    assert stream_big >= 8192 * 3 * 512 * 8 + 8192 * 512 * 8                # lists and packed top-p
+    assert stream_big < 8192 * 65536 * 4                                     # no score matrix per chunk
+    assert size(sa.SA_LSA_STREAM, (1 << 21) // 64 + 1)[0] == sa.SA_ERR_UNSUPPORTED
+    assert size(sa.SA_LSA_AUTO, 128)[1] == size(sa.SA_LSA_TABLE, 128)[1]     # AUTO: TABLE below 32,768

@@ -291,3 +291,66 @@ def test_decode_step_replays_as_a_cuda_graph(sa):
     J = dec.J.cpu().numpy()
     _check_decode_rows(J, q, new_lens, refs, nbt.cpu().numpy(), wl, wl.p, wl.k)
     del g
+
+
+def test_threshold_regime_equals_the_table_regime(sa):
+    """Appendix F.1 "Selection by threshold": the scan computes the same
+    tensor-core scores as the table (same tiles), the list holds every bucket
+    at or above the threshold, and a missed row rescores its whole row, so
+    the threshold regime selects, orders and expands exactly as the table
+    regime: every row bit-exact, also when a hook sends every row to the
+    fallback (threshold +inf: no bucket listed; -inf: every list overflows)."""
+    wl = LSA_WORKLOADS["lsa_t8k"]
+    inp = LsaInputs(wl, "cuda", seed=6)
+    prm = _params(sa, wl)
+    cache, ref, nb = _build_both(sa, inp.k_idx, prm)
+    args = (inp.q_idx, prm, cache, nb, 0, wl.p, wl.k, wl.n_sink, wl.n_window)
+    J_table = sa.lsa_search(*args, regime="table")
+    st = sa.new_status("cuda")
+    J_stream = sa.lsa_search(*args, regime="stream", status=st)
+    torch.cuda.synchronize()
+    assert torch.equal(J_table, J_stream)
+    fallback, overflow = st.cpu().tolist()[2:]
+    assert fallback <= 0.05 * wl.T, f"{fallback} rows fell back"
+    vis_rows = wl.T - wl.n_cluster                    # rows that see at least one bucket
+    for hook, name in ((sa.SA_HOOK_THETA_POS_INF, "+inf"), (sa.SA_HOOK_THETA_NEG_INF, "-inf")):
+        st = sa.new_status("cuda")
+        J_hook = sa.lsa_search(*args, regime="stream", status=st, test_hook=hook)
+        torch.cuda.synchronize()
+        assert torch.equal(J_table, J_hook), name
+        fb, ov = st.cpu().tolist()[2:]
+        if hook == sa.SA_HOOK_THETA_POS_INF:
+            assert fb == vis_rows
+        else:
+            # rows whose visible buckets exceed the room 3p overflow
+            over = sum(1 for pos in range(wl.T) if min(nb, pos // wl.n_cluster) * wl.n_buckets > 3 * wl.p)
+            assert fb == ov == over
+
+
+def test_threshold_regime_at_512k_tokens(sa):
+    """2^19 tokens: 1,024 cluster blocks and 65,536 buckets, past the table
+    regime, so AUTO scans with thresholds. The bucket cache is bit-exact, 40
+    rows match the oracle (score-tie rule), and few rows fall back."""
+    wl = LSA_WORKLOADS["lsa_t64k"].with_(T=1 << 19)
+    inp = LsaInputs(wl, "cuda", seed=7)
+    prm = _params(sa, wl)
+    cache, ref, nb = _build_both(sa, inp.k_idx, prm)
+    _assert_same_cache(cache, ref)
+    rng = np.random.default_rng(7)
+    rows = sorted(set(rng.choice(wl.T, 36, replace=False).tolist() + [600, 70000, 300000, wl.T - 1]))
+    st = sa.new_status("cuda")
+    J = sa.lsa_search(inp.q_idx, prm, cache, nb, 0, wl.p, wl.k, wl.n_sink, wl.n_window, status=st)
+    torch.cuda.synchronize()
+    assert st.cpu().tolist()[0] == 0
+    assert st.cpu().tolist()[2] <= 0.05 * wl.T
+    Jr = J[rows].cpu().numpy()
+    del J
+    qn = lsa.normalized_queries(inp.q_idx.float().cpu().numpy()[rows])
+    cent, off, keys = ref
+    exceptions = 0
+    for j, (r, qv) in enumerate(zip(rows, qn)):
+        want = lsa.search_row(qv, r, cent, off, keys, nb, wl.n_cluster, wl.n_buckets, wl.p, wl.k, wl.n_sink,
+                              wl.n_window)
+        exceptions += check_lsa_row(Jr[j], want, qv, r, cent, nb, wl.n_cluster, wl.n_buckets, wl.p, wl.n_sink,
+                                    wl.n_window, f"row {r}")
+    assert exceptions <= 2
