@@ -396,6 +396,61 @@ def run_native_lsa(args, rank, world, local_rank):
     roof.pop("ms")
     roof.update({"kernel": dom, "traffic": None,
                  "peak_source": f"{peak_src}: " + ("bf16 burst" if roof["unit"] == "TFLOP/s" else "HBM copy")})
+    # ---------------- LSA decode step: 64 sequences, one new query each ----------------
+    decode = None
+    if not args.no_decode:
+        B, L = args.lsa_decode_batch, wl.T
+        nbl = L // wl.n_cluster
+        cent = torch.zeros((B, nbl * wl.n_buckets, wl.d), dtype=torch.bfloat16, device=dev)
+        boff = torch.zeros((B, nbl * wl.n_buckets), dtype=torch.int32, device=dev)
+        bkeys = torch.zeros((B, nbl * wl.n_cluster), dtype=torch.int32, device=dev)
+        qd = torch.empty((B, wl.d), dtype=torch.bfloat16, device=dev)
+        for b in range(B):                                 # every sequence its own index keys and cache
+            sb = LsaInputs(wl, dev, seed=rank_seed(args.seed, rank) + 10_000 + b)
+            sa.lsa_build_buckets(sb.k_idx, prm, n_blocks=nbl, out=(cent[b], boff[b], bkeys[b]))
+            qd[b] = sb.q_idx[L - 1]
+            del sb
+        g = torch.Generator(device=dev)
+        g.manual_seed(rank_seed(args.seed, rank) + 20_000)
+        std = 1.0 / math.sqrt(wl.dh)
+        Kd = (torch.randn((B, L, wl.dh), generator=g, device=dev) * std).to(torch.bfloat16)
+        Vd = (torch.randn((B, L, wl.dh), generator=g, device=dev) * std).to(torch.bfloat16)
+        Qd = (torch.randn((B, wl.Hq, wl.dh), generator=g, device=dev) * std).to(torch.bfloat16)
+        nbt = torch.full((B,), nbl, dtype=torch.int32, device=dev)
+        lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+        ldec = sa.LsaDecode(qd, prm, (cent, boff, bkeys), nbt, lens, wl.p, wl.k, wl.n_sink, wl.n_window)
+        out_d = torch.empty_like(Qd)
+        lse_d = torch.empty((B, wl.Hq), dtype=torch.float32, device=dev)
+
+        def dstep():
+            J = ldec()
+            sa.sparse_attn(Qd, Kd, Vd, J, out=out_d, lse=lse_d)
+
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            dstep()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        sel_ms = att_ms = 0.0
+        for _ in range(K_):
+            flush.fill_(1)
+            ev[0].record(stream)
+            J = ldec()
+            ev[1].record(stream)
+            sa.sparse_attn(Qd, Kd, Vd, J, out=out_d, lse=lse_d)
+            ev[2].record(stream)
+            torch.cuda.synchronize()
+            sel_ms += ev[0].elapsed_time(ev[1])
+            att_ms += ev[1].elapsed_time(ev[2])
+        sel_ms, att_ms = reduce_max([sel_ms / K_, att_ms / K_], device=dev)
+        cent_bytes = B * nbl * wl.n_buckets * (wl.d * 2 + 4)      # centroids read + row scores written
+        us = (sel_ms + att_ms) * 1e3
+        decode = {"us_per_step": round(us, 1), "us_per_token": round(us / B, 3), "batch": B, "L": L,
+                  "select_us": round(sel_ms * 1e3, 1), "attention_us": round(att_ms * 1e3, 1),
+                  "scan_hbm_bytes": cent_bytes,
+                  "select_hbm_frac": round(cent_bytes / (sel_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+        del Kd, Vd
+
     e2e = None
     if not args.skip_e2e:
         srcs = (inp.k_idx, inp.q_idx, Q, K, V)
@@ -446,7 +501,7 @@ def run_native_lsa(args, rank, world, local_rank):
                    "buckets_per_block": wl.n_buckets, "max_bucket_keys": wl.max_bucket_keys, "p": wl.p,
                    "k": wl.k, "n_sink": wl.n_sink, "n_window": wl.n_window, "Hq": wl.Hq, "head_dim": wl.dh,
                    "parallelism": f"replicas x{world}", "l2": "flushed (512 MB write) before every step"},
-        "roofline": roof, "stages": stages, "cpu_baseline": cpu, "e2e": e2e,
+        "roofline": roof, "stages": stages, "decode": decode, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches * K_, "clocks": clk,
     }
     if rank == 0:
@@ -707,6 +762,7 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=96)
     ap.add_argument("--ref-rows", type=int, default=12)
     ap.add_argument("--lsa-cpu-rows", type=int, default=2048, help="query rows of the LSA oracle baseline")
+    ap.add_argument("--lsa-decode-batch", type=int, default=64, help="sequences of the LSA decode step")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
