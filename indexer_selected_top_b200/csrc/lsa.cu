@@ -776,12 +776,14 @@ extern "C" sa_status sa_lsa_build_buckets(const sa_lsa_params* prm, const void* 
   if (!params_ok(prm) || n_k < 0 || block0 < 0 || n_blocks < 0) return SA_ERR_INVALID_ARGUMENT;
   if ((long long)(block0 + (long long)n_blocks) * prm->n_cluster > n_k) return SA_ERR_INVALID_ARGUMENT;
   if (!params_supported(prm)) return SA_ERR_UNSUPPORTED;
+  if (n_blocks > 0) {
+    if (k_idx == nullptr || centroids == nullptr || bucket_off == nullptr || bucket_keys == nullptr)
+      return SA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(k_idx) || !aligned16(centroids)) return SA_ERR_INVALID_ARGUMENT;
+  }
   if (status != nullptr && cudaMemsetAsync(status, 0, sizeof(sa_device_status), stream) != cudaSuccess)
     return SA_ERR_CUDA;
   if (n_blocks == 0) return SA_OK;
-  if (k_idx == nullptr || centroids == nullptr || bucket_off == nullptr || bucket_keys == nullptr)
-    return SA_ERR_INVALID_ARGUMENT;
-  if (!aligned16(k_idx) || !aligned16(centroids)) return SA_ERR_INVALID_ARGUMENT;
   ClusterArgs a;
   a.k = static_cast<const __nv_bfloat16*>(k_idx);
   a.block0 = block0;
@@ -816,16 +818,18 @@ extern "C" sa_status sa_lsa_search(const sa_lsa_params* prm, const sa_lsa_search
                                    size_t ws_bytes, cudaStream_t stream) {
   const sa_status s = check_search(prm, o, n_q, q_pos0, n_blocks);
   if (s != SA_OK) return s;
+  const SearchPlan pl = plan_search(prm, o, n_q, n_blocks);
+  if (n_q > 0) {
+    if (q_idx == nullptr || J == nullptr || ws == nullptr) return SA_ERR_INVALID_ARGUMENT;
+    if (n_blocks > 0 && (centroids == nullptr || bucket_off == nullptr || bucket_keys == nullptr))
+      return SA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q_idx) || (n_blocks > 0 && !aligned16(centroids))) return SA_ERR_INVALID_ARGUMENT;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return SA_ERR_INVALID_ARGUMENT;
+    if (ws_bytes < pl.total) return SA_ERR_WORKSPACE_TOO_SMALL;
+  }
   if (o->status != nullptr && cudaMemsetAsync(o->status, 0, sizeof(sa_device_status), stream) != cudaSuccess)
     return SA_ERR_CUDA;
   if (n_q == 0) return SA_OK;
-  if (q_idx == nullptr || J == nullptr || ws == nullptr) return SA_ERR_INVALID_ARGUMENT;
-  if (n_blocks > 0 && (centroids == nullptr || bucket_off == nullptr || bucket_keys == nullptr))
-    return SA_ERR_INVALID_ARGUMENT;
-  if (!aligned16(q_idx) || (n_blocks > 0 && !aligned16(centroids))) return SA_ERR_INVALID_ARGUMENT;
-  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return SA_ERR_INVALID_ARGUMENT;
-  const SearchPlan pl = plan_search(prm, o, n_q, n_blocks);
-  if (ws_bytes < pl.total) return SA_ERR_WORKSPACE_TOO_SMALL;
   uint8_t* w = static_cast<uint8_t*>(ws);
   __nv_bfloat16* qn = reinterpret_cast<__nv_bfloat16*>(w + pl.off_qn);
   const int nc = prm->n_cluster, m = prm->n_buckets, nb_all = n_blocks * m;
@@ -1035,17 +1039,19 @@ extern "C" sa_status sa_lsa_decode(const sa_lsa_params* prm, const sa_lsa_search
                                    cudaStream_t stream) {
   const sa_status s = check_decode(prm, o, batch, max_blocks);
   if (s != SA_OK) return s;
+  const DecodePlan pl = plan_decode(prm, o, batch, max_blocks);
+  if (batch > 0) {
+    if (q_idx == nullptr || J == nullptr || ws == nullptr || n_blocks == nullptr || seq_lens == nullptr)
+      return SA_ERR_INVALID_ARGUMENT;
+    if (max_blocks > 0 && (centroids == nullptr || bucket_off == nullptr || bucket_keys == nullptr))
+      return SA_ERR_INVALID_ARGUMENT;
+    if (!aligned16(q_idx) || (max_blocks > 0 && !aligned16(centroids))) return SA_ERR_INVALID_ARGUMENT;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return SA_ERR_INVALID_ARGUMENT;
+    if (ws_bytes < pl.total) return SA_ERR_WORKSPACE_TOO_SMALL;
+  }
   if (o->status != nullptr && cudaMemsetAsync(o->status, 0, sizeof(sa_device_status), stream) != cudaSuccess)
     return SA_ERR_CUDA;
   if (batch == 0) return SA_OK;
-  if (q_idx == nullptr || J == nullptr || ws == nullptr || n_blocks == nullptr || seq_lens == nullptr)
-    return SA_ERR_INVALID_ARGUMENT;
-  if (max_blocks > 0 && (centroids == nullptr || bucket_off == nullptr || bucket_keys == nullptr))
-    return SA_ERR_INVALID_ARGUMENT;
-  if (!aligned16(q_idx) || (max_blocks > 0 && !aligned16(centroids))) return SA_ERR_INVALID_ARGUMENT;
-  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return SA_ERR_INVALID_ARGUMENT;
-  const DecodePlan pl = plan_decode(prm, o, batch, max_blocks);
-  if (ws_bytes < pl.total) return SA_ERR_WORKSPACE_TOO_SMALL;
   uint8_t* w = static_cast<uint8_t*>(ws);
   __nv_bfloat16* qn = reinterpret_cast<__nv_bfloat16*>(w + pl.off_qn);
   float* S = reinterpret_cast<float*>(w + pl.off_S);

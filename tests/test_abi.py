@@ -224,3 +224,22 @@ def test_lsa_search_regimes_validate_and_size(sa):
     assert stream_big < 8192 * 65536 * 4                                     # no score matrix per chunk
     assert size(sa.SA_LSA_STREAM, (1 << 21) // 64 + 1)[0] == sa.SA_ERR_UNSUPPORTED
     assert size(sa.SA_LSA_AUTO, 128)[1] == size(sa.SA_LSA_TABLE, 128)[1]     # AUTO: TABLE below 32,768
+
+
+def test_lsa_calls_validate_before_touching_the_status_word(sa):
+    """A call that fails validation queues nothing, not even the zeroing of its
+    status word: with a (bogus) status pointer and a bad argument, the answer is
+    the validation error, not a CUDA error (there is no device here)."""
+    import ctypes
+    lib = sa._lib
+    good = sa.lsa_params()
+    bogus = 4096
+    assert lib.sa_lsa_build_buckets(ctypes.byref(good), None, 4096, 0, 1, 512, 768, 1024, bogus, None) \
+        == sa.SA_ERR_INVALID_ARGUMENT
+    o = sa.LsaSearchOpts(p=512, k=2048, n_sink=4, n_window=512, status=bogus, regime=0, test_hook=0)
+    assert lib.sa_lsa_search(ctypes.byref(good), ctypes.byref(o), None, 16, 0, 512, 768, 1024, 8, 2048, 8192,
+                             1 << 30, None) == sa.SA_ERR_INVALID_ARGUMENT
+    assert lib.sa_lsa_search(ctypes.byref(good), ctypes.byref(o), 256, 16, 0, 512, 768, 1024, 8, 2048, 8192, 256,
+                             None) == sa.SA_ERR_WORKSPACE_TOO_SMALL
+    assert lib.sa_lsa_decode(ctypes.byref(good), ctypes.byref(o), 256, 4, 512, 768, 1024, 16, None, 2048, 4096,
+                             8192, 1 << 20, None) == sa.SA_ERR_INVALID_ARGUMENT
