@@ -503,6 +503,8 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
     if (in->dtype != SA_FP8_E4M3) return SA_ERR_UNSUPPORTED;
     if ((in->q_pos0 + in->n_q - 1) / o->block_size >= kMaxBlocks) return SA_ERR_UNSUPPORTED;
   }
+  const int n_stages = o->mode == SA_MODE_FLAT ? SA_PREFILL_FLAT_STAGES : SA_PREFILL_TWO_STAGE_STAGES;
+  if (o->stage_events != nullptr && o->n_stage_events < n_stages + 1) return SA_ERR_INVALID_ARGUMENT;
   if (in->n_q == 0) return SA_OK;
   PrefillPlan p;
   plan_prefill(in, o, &p);
@@ -514,9 +516,6 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
   const float scale = attn_scale(at);
   const size_t qrow = (size_t)in->n_heads * in->d_idx * esize(in->dtype);
   cudaError_t e = cudaSuccess;
-
-  const int n_stages = o->mode == SA_MODE_FLAT ? SA_PREFILL_FLAT_STAGES : SA_PREFILL_TWO_STAGE_STAGES;
-  if (o->stage_events != nullptr && o->n_stage_events < n_stages + 1) return SA_ERR_INVALID_ARGUMENT;
   StageMarks sm{o->stage_events, o->n_stage_events, true};
 
   if (o->mode == SA_MODE_TWO_STAGE) {
@@ -668,10 +667,10 @@ sa_status sa_decode(const sa_indexer_in* in, const sa_attn_in* at, const sa_deco
   plan_decode(in, at, o->k, &p);
   if (ws == nullptr || ws_bytes < p.total) return SA_ERR_WORKSPACE_TOO_SMALL;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return SA_ERR_INVALID_ARGUMENT;
+  if (o->stage_events != nullptr && o->n_stage_events < SA_DECODE_STAGES + 1) return SA_ERR_INVALID_ARGUMENT;
   char* w = static_cast<char*>(ws);
   uint32_t* status = o->status ? reinterpret_cast<uint32_t*>(o->status) : nullptr;
   if (status && cudaMemsetAsync(status, 0, sizeof(sa_device_status), stream) != cudaSuccess) return SA_ERR_CUDA;
-  if (o->stage_events != nullptr && o->n_stage_events < SA_DECODE_STAGES + 1) return SA_ERR_INVALID_ARGUMENT;
   StageMarks sm{o->stage_events, o->n_stage_events, true};
   float* rows = reinterpret_cast<float*>(w + p.off_scores);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + p.off_idx);
