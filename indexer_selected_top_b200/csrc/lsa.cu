@@ -16,16 +16,23 @@
 // 0 upward: n_a n_b / (n_a + n_b) * |mu_a - mu_b|^2 with mu = sum / n, counts in
 // pool keys. Ties go to the lower index.
 //
-// Search (short context: the appendix's regime that writes the score matrix
-// S, below 32,768 buckets): queries are normalised to bf16; a tcgen05 kernel
-// computes S = C Q^T with 128 buckets on the MMA M dimension and 128 queries
-// on N (both operands bf16, K = d_idx = 64, fp32 accumulation in tensor
-// memory) and writes each query's row of S; the radix top-k of the library
-// keeps the p best buckets among the query's visible ones (the cluster blocks
-// before its own); one CTA per query sorts those p buckets by packed key
-// (score, then lower id), takes their keys best first into k long-range keys,
-// skipping keys of the sinks and the window, and writes the index row
-// [sinks | window | long-range keys | -1 ...].
+// Search: queries are normalised to bf16; a tcgen05 kernel scores 128 buckets
+// (MMA M dimension) against 128 queries (N), both operands bf16, K = d_idx =
+// 64, fp32 accumulation in tensor memory. Two regimes (appendix F.1 "Flat
+// prefill"): below 32,768 buckets the kernel writes each query's row of
+// scores S and the library's radix top-k keeps the p best of the query's
+// visible buckets (the cluster blocks before its own); beyond, S is never
+// written -- a threshold per query from sampled centroids, the same kernel
+// appending the buckets at or above it to the query's list in its epilogue,
+// a radix select over the list, and a whole-row rescoring for the rows whose
+// list missed ("Selection by threshold"). Either way one CTA per query sorts
+// its p buckets by packed key (score, then lower id), takes their keys best
+// first into k long-range keys, skipping keys of the sinks and the window, and
+// writes the index row [sinks | window | long-range keys | -1 ...].
+//
+// Decode ("Flat decode"): each sequence's new query scores the centroids of
+// its own bucket cache on the CUDA cores (one flop per byte: bound by HBM),
+// then the same top-p and expansion; fixed shapes, no host synchronisation.
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
