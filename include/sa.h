@@ -468,6 +468,31 @@ sa_status sa_lsa_decode_workspace_size(const sa_lsa_params* prm, const sa_lsa_se
                                        int32_t max_blocks, size_t* bytes);
 
 /*
+ * sa_lsa_attention: softmax attention over LSA index rows (section 3.2: one
+ *   row J_i per query, shared by all heads), on the tensor cores in two passes
+ *   whose results are merged by their log-sum-exp: the sinks and windows of
+ *   groups of 8 consecutive queries, and the long-range keys of groups of 8
+ *   queries whose long-range keys overlap (MinHash grouping). The result is
+ *   attention over the whole row, as sa_sparse_attn computes it.
+ *   J: device int32 [n_q, width] as sa_lsa_search writes it for these q_pos0,
+ *   n_sink and n_window (width = n_sink + n_window + k): row i holds the
+ *   sinks and window of position q_pos0 + i, then long-range keys, then -1.
+ *   attn: prefill operands (batch 0); out bf16 [n_q, n_q_heads, head_dim],
+ *   lse fp32 [n_q, n_q_heads] (nullable). Supported: 16 heads x 128 and
+ *   n_k <= 196608 (else SA_ERR_UNSUPPORTED: use sa_sparse_attn). status
+ *   (nullable) is zeroed by the call and reports a bounded wait that gave up.
+ *   Workspace: sa_lsa_attention_workspace_size bytes, 256-byte aligned. No
+ *   host synchronisation.
+ */
+sa_status sa_lsa_attention(const sa_attn_in* attn, const int32_t* J, int32_t width, int32_t q_pos0, int32_t n_sink,
+                           int32_t n_window, void* out, float* lse, sa_device_status* status, void* ws,
+                           size_t ws_bytes, cudaStream_t stream);
+
+/* Workspace bytes of sa_lsa_attention (host call). */
+sa_status sa_lsa_attention_workspace_size(const sa_attn_in* attn, int32_t width, int32_t q_pos0, int32_t n_sink,
+                                          int32_t n_window, size_t* bytes);
+
+/*
  * sa_workspace_size: bytes of device workspace `op` needs for these operands
  * (host call, no device work). opts points to sa_prefill_opts (PREFILL),
  * sa_decode_opts (DECODE), an int32_t k (TOPK, SPARSE_ATTN) or NULL.

@@ -35,7 +35,7 @@ SA_HOOK_NONE, SA_HOOK_THETA_POS_INF, SA_HOOK_THETA_NEG_INF, SA_HOOK_STALL_WAIT, 
 EXPORTS = ("sa_status_string", "sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode",
            "sa_workspace_size", "sa_sparse_attn_decode_noalloc", "sa_quantize_rows_e4m3",
            "sa_expand_sinks_window", "sa_lsa_build_buckets", "sa_lsa_search", "sa_lsa_search_workspace_size", "sa_lsa_decode",
-           "sa_lsa_decode_workspace_size")
+           "sa_lsa_decode_workspace_size", "sa_lsa_attention", "sa_lsa_attention_workspace_size")
 
 
 class IndexerIn(ctypes.Structure):
@@ -132,13 +132,17 @@ _lib.sa_lsa_decode.argtypes = [ctypes.POINTER(LsaParams), ctypes.POINTER(LsaSear
                                _P, _P, ctypes.c_int32, _P, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.sa_lsa_decode_workspace_size.argtypes = [ctypes.POINTER(LsaParams), ctypes.POINTER(LsaSearchOpts),
                                               ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+_lib.sa_lsa_attention.argtypes = [ctypes.POINTER(AttnIn), _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                  ctypes.c_int32, _P, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.sa_lsa_attention_workspace_size.argtypes = [ctypes.POINTER(AttnIn), ctypes.c_int32, ctypes.c_int32,
+                                                 ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
 _lib.sa_workspace_size.argtypes = [ctypes.c_int, ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), _P,
                                    ctypes.POINTER(ctypes.c_size_t)]
 _lib.sa_sparse_attn_decode_noalloc.argtypes = [ctypes.POINTER(AttnIn), _P, ctypes.c_int32, _P, _P, _P]
 for _f in ("sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode", "sa_workspace_size",
            "sa_sparse_attn_decode_noalloc", "sa_quantize_rows_e4m3", "sa_expand_sinks_window",
            "sa_lsa_build_buckets", "sa_lsa_search", "sa_lsa_search_workspace_size", "sa_lsa_decode",
-           "sa_lsa_decode_workspace_size"):
+           "sa_lsa_decode_workspace_size", "sa_lsa_attention", "sa_lsa_attention_workspace_size"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -430,7 +434,8 @@ def lsa_search(q_idx: torch.Tensor, prm: LsaParams, buckets, n_blocks: int, q_po
 class LsaPrefill:
     """A prepared LSA flat prefill of one sequence: the bucket cache of its
     complete cluster blocks (sa_lsa_build_buckets), the index rows of every
-    query (sa_lsa_search) and attention over them (sa_sparse_attn). Buffers
+    query (sa_lsa_search) and attention over them (sa_lsa_attention, or
+    sa_sparse_attn for shapes it does not take). Buffers
     and workspaces are allocated once; stage i of a call runs between the
     timer's events i and i + 1 (stages: cluster, search, attention)."""
 
@@ -456,11 +461,8 @@ class LsaPrefill:
         self.nws = n.value
         self.ws = _workspace(self.nws, dev)
         self.J = torch.empty((self.q_idx.shape[0], n_sink + n_window + k), dtype=torch.int32, device=dev)
-        self.att = attn_in(Q, K, V, softmax_scale)
-        self.nws_attn = workspace_size(SA_OP_SPARSE_ATTN, att=self.att, opts=self.J.shape[1])
-        self.ws_attn = _workspace(self.nws_attn, dev)
-        self.out = torch.empty_like(Q)
-        self.lse = torch.empty(Q.shape[:2], dtype=torch.float32, device=dev)
+        self.attn = LsaAttention(Q, K, V, self.J, 0, n_sink, n_window, softmax_scale, status)
+        self.out, self.lse = self.attn.out, self.attn.lse
         self.timer = timer
         self.status = status
         self._keep = (Q, K, V)
@@ -482,8 +484,7 @@ class LsaPrefill:
                                   _ptr(self.J), _aligned(self.ws), self.nws, st), "sa_lsa_search")
         if ev:
             ev[2].record(ts)
-        _check(_lib.sa_sparse_attn(ctypes.byref(self.att), _ptr(self.J), self.J.shape[1], _ptr(self.out),
-                                   _ptr(self.lse), _aligned(self.ws_attn), self.nws_attn, st), "sa_sparse_attn")
+        self.attn(stream)
         if ev:
             ev[3].record(ts)
         return self.out, self.lse
@@ -534,6 +535,54 @@ class LsaDecode:
         with torch.cuda.graph(g, stream=s):
             self(s)
         return g
+
+
+class LsaAttention:
+    """A prepared sa_lsa_attention call over index rows J [n_q, width] from
+    lsa_search (same q_pos0, n_sink, n_window): the sinks and windows of
+    consecutive queries and the long-range keys of queries grouped by overlap,
+    on the tensor cores, merged by log-sum-exp. `supported` is False for shapes
+    the tensor-core kernel does not take; calls then run sa_sparse_attn (the
+    per-query kernel) over the same rows."""
+
+    def __init__(self, Q, K, V, J, q_pos0: int = 0, n_sink: int = 4, n_window: int = 512,
+                 softmax_scale: float = 0.0, status=None):
+        self.att = attn_in(Q, K, V, softmax_scale)
+        self.J, self.q_pos0, self.n_sink, self.n_window = J, q_pos0, n_sink, n_window
+        self.width = J.shape[1]
+        n = ctypes.c_size_t(0)
+        code = _lib.sa_lsa_attention_workspace_size(ctypes.byref(self.att), self.width, q_pos0, n_sink, n_window,
+                                                    ctypes.byref(n))
+        self.supported = code == SA_OK
+        if code not in (SA_OK, SA_ERR_UNSUPPORTED):
+            _check(code, "sa_lsa_attention_workspace_size")
+        if not self.supported:
+            n.value = workspace_size(SA_OP_SPARSE_ATTN, att=self.att, opts=self.width)
+        self.nws = n.value
+        self.ws = _workspace(self.nws, Q.device)
+        self.out = torch.empty_like(Q)
+        self.lse = torch.empty(Q.shape[:2], dtype=torch.float32, device=Q.device)
+        self.status = status
+        self._keep = (Q, K, V)
+
+    def __call__(self, stream=None):
+        if self.supported:
+            _check(_lib.sa_lsa_attention(ctypes.byref(self.att), _ptr(self.J), self.width, self.q_pos0,
+                                         self.n_sink, self.n_window, _ptr(self.out), _ptr(self.lse),
+                                         _ptr(self.status), _aligned(self.ws), self.nws, _stream(stream)),
+                   "sa_lsa_attention")
+        else:
+            _check(_lib.sa_sparse_attn(ctypes.byref(self.att), _ptr(self.J), self.width, _ptr(self.out),
+                                       _ptr(self.lse), _aligned(self.ws), self.nws, _stream(stream)),
+                   "sa_sparse_attn")
+        return self.out, self.lse
+
+
+def lsa_attention(Q, K, V, J, q_pos0: int = 0, n_sink: int = 4, n_window: int = 512, softmax_scale: float = 0.0,
+                  status=None):
+    """Attention over LSA index rows (sa_lsa_attention; the per-query kernel
+    for shapes it does not take). Returns (out, lse)."""
+    return LsaAttention(Q, K, V, J, q_pos0, n_sink, n_window, softmax_scale, status)()
 
 
 def new_status(device) -> torch.Tensor:

@@ -10,7 +10,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["sa_api.cu", "indexer.cu", "topk.cu", "attn.cu", "pool.cu", "noalloc.cu", "topk_warp.cu", "stream.cu", "topk_fast.cu", "group.cu", "attn_tc.cu", "quant.cu", "expand.cu", "lsa.cu"]
+SOURCES = ["sa_api.cu", "indexer.cu", "topk.cu", "attn.cu", "pool.cu", "noalloc.cu", "topk_warp.cu", "stream.cu", "topk_fast.cu", "group.cu", "attn_tc.cu", "quant.cu", "expand.cu", "lsa.cu", "lsa_attn.cu"]
 LIB = os.path.join(HERE, "libsa.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -118,6 +118,14 @@ cudaError_t launch_group_queries(const int* kept, int keep, const uint32_t* sel,
   return cudaGetLastError();
 }
 
+cudaError_t launch_group_sort(const unsigned long long* sig, int n_q, int* perm, cudaStream_t st) {
+  if (n_q <= 0) return cudaSuccess;
+  group_sort_kernel<<<(n_q + GW - 1) / GW, 1024, 0, st>>>(sig, n_q, perm);
+  return cudaGetLastError();
+}
+
+int group_window() { return GW; }
+
 // ------------------------------------------------------- grouped attention
 template <int DH>
 struct GaCfg {

@@ -122,6 +122,10 @@ cudaError_t launch_group_union(const int* kept, int keep, const uint32_t* sel, c
 
 // tcgen05 attention of the groups' union lists (attn_tc.cu), 16 heads x 128 dims
 bool tc_attention_supported(int hq, int dh);
+// perm[w * W + i] = the query of rank i in window w of W queries (W =
+// group_window()) by the 64-bit key sig[t] (ascending), -1 past n_q
+cudaError_t launch_group_sort(const unsigned long long* sig, int n_q, int* perm, cudaStream_t st);
+int group_window();
 cudaError_t launch_attention_tc(const void* q, const void* kc, const void* vc, const int* list, const uint8_t* lmask,
                                 const int* n_list, const int* perm, int n_groups, int n_q, int cap, float scale,
                                 void* out, float* lse, uint32_t* status, long long budget, cudaStream_t st);

@@ -354,3 +354,41 @@ def test_threshold_regime_at_512k_tokens(sa):
         exceptions += check_lsa_row(Jr[j], want, qv, r, cent, nb, wl.n_cluster, wl.n_buckets, wl.p, wl.n_sink,
                                     wl.n_window, f"row {r}")
     assert exceptions <= 2
+
+
+def test_lsa_attention_matches_the_oracle_and_the_per_query_kernel(sa):
+    """Attention over LSA index rows in two tensor-core passes (sinks and
+    windows of consecutive queries; long-range keys of queries grouped by
+    overlap) merged by log-sum-exp, against the oracle over the same rows, and
+    against the per-query kernel on every row; also a ragged chunk that starts
+    at q_pos0 = 3000."""
+    wl = LSA_WORKLOADS["lsa_t8k"]
+    inp = LsaInputs(wl, "cuda", seed=8)
+    prm = _params(sa, wl)
+    cache, ref, nb = _build_both(sa, inp.k_idx, prm)
+    J = sa.lsa_search(inp.q_idx, prm, cache, nb, 0, wl.p, wl.k, wl.n_sink, wl.n_window)
+    Q, K, V = inp.attention_operands()
+    st = sa.new_status("cuda")
+    att = sa.LsaAttention(Q, K, V, J, 0, wl.n_sink, wl.n_window, status=st)
+    assert att.supported
+    o, l = att()
+    o2, l2 = sa.sparse_attn(Q, K, V, J)
+    torch.cuda.synchronize()
+    assert st.cpu().tolist()[0] == 0
+    o, l, o2, l2 = o.float(), l, o2.float(), l2
+    scale = o2.abs().max().item()
+    assert (o - o2).abs().max().item() <= 1e-2 * scale + 1e-4
+    assert torch.allclose(l, l2, atol=2e-3, rtol=0)
+    Jh = J.cpu().numpy()
+    Kh, Vh = K.double().cpu().numpy(), V.double().cpu().numpy()
+    oh, lh = o.cpu().numpy(), l.cpu().numpy()
+    for r in [0, 3, 511, 512, 515, 516, 1023, 1024, 4000, wl.T - 1]:
+        ro, rl = oracle.sparse_attention_row(Q[r].double().cpu().numpy(), Kh, Vh, Jh[r])
+        check_attention_row(oh[r], ro, lh[r], rl, f"row {r}")
+    q0 = 3000
+    J3 = sa.lsa_search(inp.q_idx[q0:], prm, cache, nb, q0, wl.p, wl.k, wl.n_sink, wl.n_window)
+    o3, l3 = sa.lsa_attention(Q[q0:].contiguous(), K, V, J3, q0, wl.n_sink, wl.n_window)
+    torch.cuda.synchronize()
+    assert torch.equal(J3, J[q0:])
+    assert (o3.float() - o[q0:]).abs().max().item() <= 1e-2 * scale + 1e-4
+    assert torch.allclose(l3, l[q0:], atol=2e-3, rtol=0)
