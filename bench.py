@@ -489,15 +489,20 @@ def run_native_lsa(args, rank, world, local_rank):
                          f"{info['rows']} query rows ({info['rows_s']:.1f} s: search, attention), extrapolated "
                          f"to {wl.T} rows"}
     chunks = -(-wl.T // 8192)
-    launches = 1 + 5 * chunks + 1                      # clustering; per chunk qnorm, scores, lengths, top-p,
-    line = {                                           # expansion; attention
+    # clustering; per 8192-query chunk: unit queries, scores, lengths, top-p, expansion; attention: per
+    # 16384-query chunk local union, local pass, signatures, sort, long-range union, long-range pass, merge
+    # (one launch on the per-query kernel)
+    attn_launches = 7 * -(-wl.T // 16384) if run.attn.supported else 1
+    launches = 1 + 5 * chunks + attn_launches
+    line = {
         "metric": LSA_METRIC,
         "value": round(weak_scaling_value(world, K_, wl.T, tot), 1),
         "unit": "tokens/s", "n_gpus": world, "steps": K_, "warmup": args.warmup,
         "ms_per_step": round(tot / K_, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16 index (f32 clustering and accumulation), bf16 attention (f32 softmax)",
         "data": "synthetic",
-        "config": {"workload": wl.name, "T": wl.T, "d_idx": wl.d, "n_pool": wl.n_pool, "n_cluster": wl.n_cluster,
+        "config": {"workload": wl.name, "T": wl.T, "d_idx": wl.d,
+                   "attention": "tensor-core local + long-range passes" if run.attn.supported else "per-query", "n_pool": wl.n_pool, "n_cluster": wl.n_cluster,
                    "buckets_per_block": wl.n_buckets, "max_bucket_keys": wl.max_bucket_keys, "p": wl.p,
                    "k": wl.k, "n_sink": wl.n_sink, "n_window": wl.n_window, "Hq": wl.Hq, "head_dim": wl.dh,
                    "parallelism": f"replicas x{world}", "l2": "flushed (512 MB write) before every step"},
