@@ -477,7 +477,8 @@ sa_status sa_lsa_decode_workspace_size(const sa_lsa_params* prm, const sa_lsa_se
  *   J: device int32 [n_q, width] as sa_lsa_search writes it for these q_pos0,
  *   n_sink and n_window (width = n_sink + n_window + k): row i holds the
  *   sinks and window of position q_pos0 + i, then long-range keys, then -1.
- *   attn: prefill operands (batch 0); out bf16 [n_q, n_q_heads, head_dim],
+ *   attn: prefill operands (batch 0), with q_pos0 + n_q <= n_k (the local part
+ *   reads the keys up to each query's own position); out bf16 [n_q, n_q_heads, head_dim],
  *   lse fp32 [n_q, n_q_heads] (nullable). Supported: 16 heads x 128 and
  *   n_k <= 196608 (else SA_ERR_UNSUPPORTED: use sa_sparse_attn). status
  *   (nullable) is zeroed by the call and reports a bounded wait that gave up.

@@ -243,6 +243,7 @@ static sa_status la_check(const sa_attn_in* at, int width, int q_pos0, int n_sin
   if (at == nullptr || at->batch != 0 || at->n_q < 0 || at->n_k <= 0) return SA_ERR_INVALID_ARGUMENT;
   if (width < 1 || q_pos0 < 0 || n_sink < 0 || n_window < 0 || n_sink + (long long)n_window > width)
     return SA_ERR_INVALID_ARGUMENT;
+  if (q_pos0 + (long long)at->n_q > at->n_k) return SA_ERR_INVALID_ARGUMENT;   // every query's own key is cached
   if (!tc_attention_supported(at->n_q_heads, at->head_dim) || at->n_k > LA_MAX_KEYS) return SA_ERR_UNSUPPORTED;
   return SA_OK;
 }

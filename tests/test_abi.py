@@ -243,3 +243,29 @@ def test_lsa_calls_validate_before_touching_the_status_word(sa):
                              None) == sa.SA_ERR_WORKSPACE_TOO_SMALL
     assert lib.sa_lsa_decode(ctypes.byref(good), ctypes.byref(o), 256, 4, 512, 768, 1024, 16, None, 2048, 4096,
                              8192, 1 << 20, None) == sa.SA_ERR_INVALID_ARGUMENT
+
+
+def test_lsa_attention_validates_on_the_host(sa):
+    import ctypes
+    lib = sa._lib
+    n = ctypes.c_size_t(0)
+    att = sa.AttnIn(n_q=1000, n_k=4096, n_q_heads=16, head_dim=128, softmax_scale=0.0, q=256, k_cache=512,
+                    v_cache=768, batch=0)
+    assert lib.sa_lsa_attention_workspace_size(ctypes.byref(att), 2564, 0, 4, 512, ctypes.byref(n)) == sa.SA_OK
+    assert n.value > 0
+    # the queries' own keys must be in the cache
+    assert lib.sa_lsa_attention_workspace_size(ctypes.byref(att), 2564, 3500, 4, 512, ctypes.byref(n)) \
+        == sa.SA_ERR_INVALID_ARGUMENT
+    assert lib.sa_lsa_attention_workspace_size(ctypes.byref(att), 100, 0, 4, 512, ctypes.byref(n)) \
+        == sa.SA_ERR_INVALID_ARGUMENT                                       # width below sinks + window
+    other = sa.AttnIn(n_q=1000, n_k=4096, n_q_heads=8, head_dim=64, softmax_scale=0.0, q=256, k_cache=512,
+                      v_cache=768, batch=0)
+    assert lib.sa_lsa_attention_workspace_size(ctypes.byref(other), 2564, 0, 4, 512, ctypes.byref(n)) \
+        == sa.SA_ERR_UNSUPPORTED
+    big = sa.AttnIn(n_q=1000, n_k=1 << 20, n_q_heads=16, head_dim=128, softmax_scale=0.0, q=256, k_cache=512,
+                    v_cache=768, batch=0)
+    assert lib.sa_lsa_attention_workspace_size(ctypes.byref(big), 2564, 0, 4, 512, ctypes.byref(n)) \
+        == sa.SA_ERR_UNSUPPORTED
+    # rejected before any device work, even with a (bogus) status pointer
+    assert lib.sa_lsa_attention(ctypes.byref(att), None, 2564, 0, 4, 512, 1024, None, 4096, 8192, 1 << 30, None) \
+        == sa.SA_ERR_INVALID_ARGUMENT
