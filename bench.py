@@ -342,17 +342,15 @@ def run_native_lsa(args, rank, world, local_rank):
     prm = sa.lsa_params(n_pool=wl.n_pool, n_cluster=wl.n_cluster, n_buckets=wl.n_buckets,
                         max_bucket_keys=wl.max_bucket_keys)
     timer = sa.StageTimer(sa.LsaPrefill.STAGES)
-    status = sa.new_status(dev)
-    run = sa.LsaPrefill(inp.k_idx, inp.q_idx, Q, K, V, prm, wl.p, wl.k, wl.n_sink, wl.n_window, timer=timer,
-                        status=status)
+    run = sa.LsaPrefill(inp.k_idx, inp.q_idx, Q, K, V, prm, wl.p, wl.k, wl.n_sink, wl.n_window, timer=timer)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
         flush.fill_(1)
         run()
     torch.cuda.synchronize()
-    if status.cpu().tolist()[0] != 0:
-        raise RuntimeError(f"LSA prefill status {status.cpu().tolist()}")
+    if run.stage_status[:, 0].any():
+        raise RuntimeError(f"LSA prefill status {run.stage_status.cpu().tolist()}")
     clocks = ClockSampler(local_rank)
     if world > 1:
         dist.barrier()

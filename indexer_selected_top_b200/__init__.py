@@ -437,14 +437,18 @@ class LsaPrefill:
     query (sa_lsa_search) and attention over them (sa_lsa_attention, or
     sa_sparse_attn for shapes it does not take). Buffers
     and workspaces are allocated once; stage i of a call runs between the
-    timer's events i and i + 1 (stages: cluster, search, attention)."""
+    timer's events i and i + 1 (stages: cluster, search, attention). Each
+    stage reports to its own row of `stage_status` ([3, 4] int32 on the
+    device, sa_device_status words), which every call rewrites."""
 
     STAGES = ("cluster", "search", "attention")
 
     def __init__(self, k_idx, q_idx, Q, K, V, prm: LsaParams, p: int, k: int, n_sink: int = 4,
-                 n_window: int = 512, softmax_scale: float = 0.0, timer: "StageTimer" = None, status=None,
+                 n_window: int = 512, softmax_scale: float = 0.0, timer: "StageTimer" = None,
                  regime: str = "auto"):
         dev = Q.device
+        self.stage_status = torch.zeros((3, 4), dtype=torch.int32, device=dev)
+        status = self.stage_status[1]
         self.k_idx, self.q_idx = k_idx.contiguous(), q_idx.contiguous()
         self.prm = prm
         T = self.k_idx.shape[0]
@@ -461,10 +465,9 @@ class LsaPrefill:
         self.nws = n.value
         self.ws = _workspace(self.nws, dev)
         self.J = torch.empty((self.q_idx.shape[0], n_sink + n_window + k), dtype=torch.int32, device=dev)
-        self.attn = LsaAttention(Q, K, V, self.J, 0, n_sink, n_window, softmax_scale, status)
+        self.attn = LsaAttention(Q, K, V, self.J, 0, n_sink, n_window, softmax_scale, self.stage_status[2])
         self.out, self.lse = self.attn.out, self.attn.lse
         self.timer = timer
-        self.status = status
         self._keep = (Q, K, V)
 
     def __call__(self, stream=None):
@@ -475,8 +478,8 @@ class LsaPrefill:
         if ev:
             ev[0].record(ts)
         _check(_lib.sa_lsa_build_buckets(ctypes.byref(self.prm), _ptr(self.k_idx), self.k_idx.shape[0], 0,
-                                         self.n_blocks, _ptr(cent), _ptr(off), _ptr(keys), _ptr(self.status), st),
-               "sa_lsa_build_buckets")
+                                         self.n_blocks, _ptr(cent), _ptr(off), _ptr(keys),
+                                         _ptr(self.stage_status[0]), st), "sa_lsa_build_buckets")
         if ev:
             ev[1].record(ts)
         _check(_lib.sa_lsa_search(ctypes.byref(self.prm), ctypes.byref(self.opts), _ptr(self.q_idx),
