@@ -308,3 +308,39 @@ def test_ward_partner_ties_go_to_the_lower_index():
     assert lsa.ward_cost(pts[0], 1, pts[1], 1) == lsa.ward_cost(pts[1], 1, pts[2], 1) == np.float32(0.5)
     bucket, _, counts = lsa.ward_block(pts, 2, 3)
     assert bucket.tolist() == [0, 0, 1] and counts.tolist() == [2, 1]
+
+
+def test_ward_properties_on_random_blocks():
+    """Many random small blocks: exactly m buckets, none above the cap, every
+    pool key in one bucket, buckets numbered by their lowest pool key, sums
+    equal to their members' sums; with no cap and m = 1, the clusters formed
+    are those of scipy's Ward linkage."""
+    from hypothesis import given, settings, strategies as st
+    from scipy.cluster.hierarchy import linkage
+
+    @settings(max_examples=60, deadline=None, derandomize=True, database=None)
+    @given(P=st.integers(2, 24), dim=st.integers(1, 5), m_frac=st.floats(0.05, 1.0), extra=st.integers(0, 4),
+           seed=st.integers(0, 2 ** 31 - 1))
+    def check(P, dim, m_frac, extra, seed):
+        pts = np.random.default_rng(seed).standard_normal((P, dim)).astype(np.float32)
+        m = max(1, min(P, int(round(m_frac * P))))
+        cap = -(-2 * P // m) + extra
+        bucket, sums, counts = lsa.ward_block(pts, m, cap)
+        assert len(counts) == m and counts.max() <= max(cap, 1) and counts.sum() == P
+        assert sorted(set(bucket.tolist())) == list(range(m))
+        lows = [int(np.flatnonzero(bucket == r)[0]) for r in range(m)]
+        assert lows == sorted(lows)
+        assert np.allclose(sums, np.stack([pts[bucket == r].astype(np.float64).sum(0) for r in range(m)]),
+                           atol=1e-4)
+        if P >= 3:
+            _, _, _, rounds = lsa.ward_block(pts, 1, P, record=True)
+            formed, _ = _clusters_from_rounds(P, rounds)
+            Z = linkage(pts.astype(np.float64), method="ward")
+            members = {g: frozenset([g]) for g in range(P)}
+            ref = set()
+            for i, (u, v, _, _) in enumerate(Z):
+                members[P + i] = members[int(u)] | members[int(v)]
+                ref.add(members[P + i])
+            assert formed == ref
+
+    check()
