@@ -494,6 +494,21 @@ sa_status sa_lsa_attention_workspace_size(const sa_attn_in* attn, int32_t width,
                                           int32_t n_window, size_t* bytes);
 
 /*
+ * sa_debug_errors: invariant checks of the debug build (compiled with
+ *   -DSA_DEBUG_CHECKS: `build.py --debug-checks` writes libsa_debug.so). A
+ *   failed check records its site and value in device memory and the kernel
+ *   carries on without the guarded access (an attention index beyond the
+ *   cache is skipped, as in the release build); nothing traps. This call
+ *   reads the record: out (host uint32 [4]) = {first failed site
+ *   (SA_DBG_* in the library's debug.cuh), its value, number of failed
+ *   checks, 0}; reset != 0 clears it. Synchronous (device -> host copies);
+ *   call it after the stream's work has finished. The record is global to the
+ *   process: concurrent calls share it. Release builds return
+ *   SA_ERR_UNSUPPORTED and check nothing.
+ */
+sa_status sa_debug_errors(uint32_t* out, int32_t reset);
+
+/*
  * sa_workspace_size: bytes of device workspace `op` needs for these operands
  * (host call, no device work). opts points to sa_prefill_opts (PREFILL),
  * sa_decode_opts (DECODE), an int32_t k (TOPK, SPARSE_ATTN) or NULL.

@@ -35,7 +35,8 @@ SA_HOOK_NONE, SA_HOOK_THETA_POS_INF, SA_HOOK_THETA_NEG_INF, SA_HOOK_STALL_WAIT, 
 EXPORTS = ("sa_status_string", "sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode",
            "sa_workspace_size", "sa_sparse_attn_decode_noalloc", "sa_quantize_rows_e4m3",
            "sa_expand_sinks_window", "sa_lsa_build_buckets", "sa_lsa_search", "sa_lsa_search_workspace_size", "sa_lsa_decode",
-           "sa_lsa_decode_workspace_size", "sa_lsa_attention", "sa_lsa_attention_workspace_size")
+           "sa_lsa_decode_workspace_size", "sa_lsa_attention", "sa_lsa_attention_workspace_size",
+           "sa_debug_errors")
 
 
 class IndexerIn(ctypes.Structure):
@@ -136,13 +137,15 @@ _lib.sa_lsa_attention.argtypes = [ctypes.POINTER(AttnIn), _P, ctypes.c_int32, ct
                                   ctypes.c_int32, _P, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.sa_lsa_attention_workspace_size.argtypes = [ctypes.POINTER(AttnIn), ctypes.c_int32, ctypes.c_int32,
                                                  ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+_lib.sa_debug_errors.argtypes = [_P, ctypes.c_int32]
 _lib.sa_workspace_size.argtypes = [ctypes.c_int, ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), _P,
                                    ctypes.POINTER(ctypes.c_size_t)]
 _lib.sa_sparse_attn_decode_noalloc.argtypes = [ctypes.POINTER(AttnIn), _P, ctypes.c_int32, _P, _P, _P]
 for _f in ("sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode", "sa_workspace_size",
            "sa_sparse_attn_decode_noalloc", "sa_quantize_rows_e4m3", "sa_expand_sinks_window",
            "sa_lsa_build_buckets", "sa_lsa_search", "sa_lsa_search_workspace_size", "sa_lsa_decode",
-           "sa_lsa_decode_workspace_size", "sa_lsa_attention", "sa_lsa_attention_workspace_size"):
+           "sa_lsa_decode_workspace_size", "sa_lsa_attention", "sa_lsa_attention_workspace_size",
+           "sa_debug_errors"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -586,6 +589,22 @@ def lsa_attention(Q, K, V, J, q_pos0: int = 0, n_sink: int = 4, n_window: int = 
     """Attention over LSA index rows (sa_lsa_attention; the per-query kernel
     for shapes it does not take). Returns (out, lse)."""
     return LsaAttention(Q, K, V, J, q_pos0, n_sink, n_window, softmax_scale, status)()
+
+
+DEBUG_SITES = {1: "attention index beyond the cache", 2: "two-stage group union beyond its list",
+               3: "LSA bucket the query cannot see", 4: "LSA long-range key outside [0, position]",
+               5: "LSA long-range union beyond its list", 6: "LSA bucket list entry outside its block"}
+
+
+def debug_errors(reset: bool = True):
+    """The debug build's record of failed invariant checks (sa_debug_errors):
+    None when nothing failed, else (site name, value, count). Raises SaError
+    with SA_ERR_UNSUPPORTED on a release build."""
+    out = (ctypes.c_uint32 * 4)()
+    _check(_lib.sa_debug_errors(ctypes.cast(out, ctypes.c_void_p), 1 if reset else 0), "sa_debug_errors")
+    if out[0] == 0:
+        return None
+    return DEBUG_SITES.get(out[0], str(out[0])), out[1], out[2]
 
 
 def new_status(device) -> torch.Tensor:

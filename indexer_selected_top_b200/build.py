@@ -1,5 +1,6 @@
 """Builds libsa.so (the CUDA library behind include/sa.h) in-tree with nvcc
 for sm_100a. Usage: python indexer_selected_top_b200/build.py [--force]
+[--debug-checks: libsa_debug.so, with device-side invariant checks]
 
 Run it by path (or load it with load_build below): importing the package
 itself loads libsa.so, which must already exist."""
@@ -57,5 +58,19 @@ def build(force: bool = False, verbose: bool = False, out: str = None, defines=(
     return lib
 
 
+DEBUG_LIB = os.path.join(HERE, "libsa_debug.so")
+
+
+def build_debug(verbose: bool = False) -> str:
+    """The debug build: the same sources with -DSA_DEBUG_CHECKS (device-side
+    invariant checks that record errors for sa_debug_errors), as
+    libsa_debug.so beside libsa.so. Load it with SA_LIB=<path>."""
+    return build(force=True, verbose=verbose, out=DEBUG_LIB, defines=("SA_DEBUG_CHECKS",),
+                 bdir=os.path.join(HERE, "_build_debug"))
+
+
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    if "--debug-checks" in sys.argv:
+        print(build_debug(verbose=True))
+    else:
+        print(build(force="--force" in sys.argv, verbose=True))

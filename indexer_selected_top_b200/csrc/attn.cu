@@ -20,6 +20,7 @@
 #include <cuda_bf16.h>
 
 #include "attn_common.cuh"
+#include "debug.cuh"
 #include "ptx.cuh"
 #include "sa_internal.h"
 
@@ -80,6 +81,7 @@ __global__ void __launch_bounds__(AT_WARPS * 32)
   const int nchunks = (j_hi > j_lo) ? (j_hi - j_lo + AT_CHUNK - 1) / AT_CHUNK : 0;
   for (int j = threadIdx.x; j < nchunks * AT_CHUNK; j += AT_WARPS * 32) {
     int s = (j_lo + j < j_hi) ? irow[j_lo + j] : -1;
+    SA_DBG_CHECK(s < n_k, SA_DBG_ATTN_INDEX, s);
     sidx[j] = (s >= 0 && s < n_k) ? s : -1;
   }
   __syncthreads();
@@ -229,4 +231,8 @@ cudaError_t launch_attention(const void* q, const void* kc, const void* vc, cons
   return cudaErrorNotSupported;
 }
 
+}  // namespace sa
+
+namespace sa {
+SA_DEBUG_UNIT(dbg_read_attn)
 }  // namespace sa

@@ -22,6 +22,7 @@
 #include <cuda_bf16.h>
 
 #include "attn_common.cuh"
+#include "debug.cuh"
 #include "ptx.cuh"
 #include "sa_internal.h"
 
@@ -564,6 +565,7 @@ __global__ void __launch_bounds__(256) group_union_kernel(const int* __restrict_
     before += (w < warp) ? red[w] : 0;
     total += red[w];
   }
+  if (tid == 0) SA_DBG_CHECK(total <= cap, SA_DBG_GROUP_UNION, total);
   total = min(total, cap);                        // cannot bind: each query selects at most k keys
   int* gl = list + (long long)g * cap;
   uint8_t* gm = lmask + (long long)g * cap;
@@ -684,4 +686,8 @@ cudaError_t launch_group_blocks(const int* kept, int keep, const int* perm, int 
   return cudaGetLastError();
 }
 
+}  // namespace sa
+
+namespace sa {
+SA_DEBUG_UNIT(dbg_read_group)
 }  // namespace sa

@@ -35,6 +35,7 @@
 // then the same top-p and expansion; fixed shapes, no host synchronisation.
 #include <cuda_bf16.h>
 
+#include "debug.cuh"
 #include "ptx.cuh"
 #include "radix.cuh"
 #include "sa_internal.h"
@@ -270,6 +271,7 @@ __global__ void __launch_bounds__(LSA_CT) lsa_cluster_kernel(ClusterArgs a) {
     const int r = sh.root[g];
     int before = 0;
     for (int x = 0; x < g; ++x) before += sh.root[x] == r ? 1 : 0;
+    SA_DBG_CHECK(sh.koff[r] + (before + 1) * a.n_pool <= a.n_cluster, SA_DBG_LSA_CLUSTER, g);
     int32_t* dst = a.bucket_keys + kbase + sh.koff[r] + before * a.n_pool;
     for (int e = 0; e < a.n_pool; ++e) dst[e] = (int32_t)(kbase + (long long)g * a.n_pool + e);
     if (sh.alive[g]) {
@@ -645,6 +647,7 @@ __global__ void __launch_bounds__(TK_THREADS) lsa_expand_kernel(ExpandArgs a) {
     if (j < a.psort && sig[j] != 0ull) {
       const int b = (int)~(uint32_t)(sig[j] & 0xFFFFFFFFull);
       const int c = b / a.m;
+      SA_DBG_CHECK(b >= 0 && c < max(0, pos) / a.n_cluster, SA_DBG_LSA_BUCKET, b);
       lo = boff[b];
       hi = (b - c * a.m == a.m - 1) ? (c + 1) * a.n_cluster : boff[b + 1];
       for (int e = lo; e < hi; ++e) {
@@ -657,6 +660,7 @@ __global__ void __launch_bounds__(TK_THREADS) lsa_expand_kernel(ExpandArgs a) {
     for (int e = lo, w = at; e < hi && w < a.k; ++e) {
       const int s = bkeys[e];
       if (s < a.n_sink || s >= w_lo) continue;
+      SA_DBG_CHECK(s >= 0 && s <= pos, SA_DBG_LSA_KEY, s);
       far[w++] = s;
     }
     run += tot;
@@ -1105,3 +1109,7 @@ extern "C" sa_status sa_lsa_decode(const sa_lsa_params* prm, const sa_lsa_search
   lsa_expand_kernel<<<batch, TK_THREADS, 0, stream>>>(ea);
   return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
+
+namespace sa {
+SA_DEBUG_UNIT(dbg_read_lsa)
+}  // namespace sa

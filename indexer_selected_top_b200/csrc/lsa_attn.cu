@@ -19,6 +19,7 @@
 //           the sum: softmax over the disjoint union of the two parts.
 #include <cuda_bf16.h>
 
+#include "debug.cuh"
 #include "radix.cuh"
 #include "sa_internal.h"
 
@@ -136,6 +137,7 @@ __global__ void __launch_bounds__(TK_THREADS)
   }
   int tot;
   int o = block_excl_scan(cnt, red, &tot);
+  if (tid == 0) SA_DBG_CHECK(tot <= cap, SA_DBG_LSA_FAR_UNION, tot);
   const int total = min(tot, cap);
   int* gl = list + (long long)g * cap;
   uint8_t* gm = lmask + (long long)g * cap;
@@ -327,3 +329,7 @@ extern "C" sa_status sa_lsa_attention(const sa_attn_in* attn, const int32_t* J, 
   }
   return SA_OK;
 }
+
+namespace sa {
+SA_DEBUG_UNIT(dbg_read_lsa_attn)
+}  // namespace sa

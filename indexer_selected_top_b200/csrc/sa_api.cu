@@ -715,3 +715,37 @@ sa_status sa_decode(const sa_indexer_in* in, const sa_attn_in* at, const sa_deco
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------ debug build
+#ifdef SA_DEBUG_CHECKS
+namespace sa {
+int dbg_read_attn(uint32_t* out, int reset);
+int dbg_read_group(uint32_t* out, int reset);
+int dbg_read_lsa(uint32_t* out, int reset);
+int dbg_read_lsa_attn(uint32_t* out, int reset);
+}  // namespace sa
+#endif
+
+extern "C" sa_status sa_debug_errors(uint32_t* out, int32_t reset) {
+#ifdef SA_DEBUG_CHECKS
+  if (out == nullptr) return SA_ERR_INVALID_ARGUMENT;
+  int (*const readers[])(uint32_t*, int) = {sa::dbg_read_attn, sa::dbg_read_group, sa::dbg_read_lsa,
+                                            sa::dbg_read_lsa_attn};
+  uint32_t acc[4] = {0u, 0u, 0u, 0u};
+  for (auto rd : readers) {
+    uint32_t w[4];
+    if (rd(w, reset) != 0) return SA_ERR_CUDA;
+    if (acc[0] == 0u && w[0] != 0u) {
+      acc[0] = w[0];
+      acc[1] = w[1];
+    }
+    acc[2] += w[2];
+  }
+  std::memcpy(out, acc, sizeof(acc));
+  return SA_OK;
+#else
+  (void)out;
+  (void)reset;
+  return SA_ERR_UNSUPPORTED;
+#endif
+}

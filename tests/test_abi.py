@@ -269,3 +269,24 @@ def test_lsa_attention_validates_on_the_host(sa):
     # rejected before any device work, even with a (bogus) status pointer
     assert lib.sa_lsa_attention(ctypes.byref(att), None, 2564, 0, 4, 512, 1024, None, 4096, 8192, 1 << 30, None) \
         == sa.SA_ERR_INVALID_ARGUMENT
+
+
+def test_debug_checks_build_and_the_release_refusal(sa):
+    """Release builds check nothing and say so; the debug build (the same
+    sources with -DSA_DEBUG_CHECKS) compiles, exports the same calls, and its
+    reader reaches for the device record (no device here: a CUDA error)."""
+    import ctypes
+    import importlib.util
+    out = (ctypes.c_uint32 * 4)()
+    assert sa._lib.sa_debug_errors(ctypes.cast(out, ctypes.c_void_p), 0) == sa.SA_ERR_UNSUPPORTED
+    spec = importlib.util.spec_from_file_location("_sa_build", os.path.join(ROOT, "indexer_selected_top_b200",
+                                                                            "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    path = mod.build_debug()
+    dbg = ctypes.CDLL(path)
+    for name in sa.EXPORTS:
+        assert hasattr(dbg, name), name
+    dbg.sa_debug_errors.argtypes = [ctypes.c_void_p, ctypes.c_int32]
+    assert dbg.sa_debug_errors(None, 0) == sa.SA_ERR_INVALID_ARGUMENT
+    assert dbg.sa_debug_errors(ctypes.cast(out, ctypes.c_void_p), 0) in (sa.SA_OK, sa.SA_ERR_CUDA)

@@ -392,3 +392,62 @@ def test_lsa_attention_matches_the_oracle_and_the_per_query_kernel(sa):
     assert torch.equal(J3, J[q0:])
     assert (o3.float() - o[q0:]).abs().max().item() <= 1e-2 * scale + 1e-4
     assert torch.allclose(l3, l[q0:], atol=2e-3, rtol=0)
+
+
+_DEBUG_CHILD = r"""
+import os, sys, json
+import torch
+sys.path.insert(0, os.environ["SA_ROOT"])
+import indexer_selected_top_b200 as sa
+from workloads import LSA_WORKLOADS, LsaInputs
+res = {}
+# an attention index beyond the cache: recorded, and skipped as in the release build
+g = torch.Generator(device="cuda").manual_seed(9)
+n_k = 300
+K = (torch.randn(n_k, 128, generator=g, device="cuda") / 11.3).bfloat16()
+V = (torch.randn(n_k, 128, generator=g, device="cuda") / 11.3).bfloat16()
+Q = (torch.randn(4, 16, 128, generator=g, device="cuda") / 11.3).bfloat16()
+idx = torch.tensor([[1, 2, 3, n_k + 5], [4, 5, -1, -1], [7, 8, 9, 10], [11, -1, -1, -1]], dtype=torch.int32,
+                   device="cuda")
+sa.debug_errors(reset=True)
+o, l = sa.sparse_attn(Q, K, V, idx)
+o2, l2 = sa.sparse_attn(Q, K, V, torch.where(idx >= n_k, torch.full_like(idx, -1), idx))
+torch.cuda.synchronize()
+res["bad_index"] = sa.debug_errors(reset=True)
+res["same_as_skipped"] = bool(torch.equal(o, o2))
+# a valid LSA pipeline records nothing
+wl = LSA_WORKLOADS["lsa_t8k"].with_(T=2048)
+inp = LsaInputs(wl, "cuda", seed=10)
+prm = sa.lsa_params(n_pool=wl.n_pool, n_cluster=wl.n_cluster, n_buckets=wl.n_buckets,
+                    max_bucket_keys=wl.max_bucket_keys)
+cache = sa.lsa_build_buckets(inp.k_idx, prm)
+J = sa.lsa_search(inp.q_idx, prm, cache, wl.T // wl.n_cluster, 0, wl.p, wl.k, wl.n_sink, wl.n_window)
+Qa, Ka, Va = inp.attention_operands()
+sa.lsa_attention(Qa, Ka, Va, J, 0, wl.n_sink, wl.n_window)
+torch.cuda.synchronize()
+res["lsa"] = sa.debug_errors(reset=True)
+print(json.dumps(res))
+"""
+
+
+def test_debug_build_records_a_bad_index_and_nothing_on_valid_work(sa):
+    """The debug build (device-side invariant checks) in a child process: an
+    attention index beyond the cache is recorded with its value and skipped
+    (the result equals the row without it); a valid LSA pipeline (clustering,
+    search, attention) records nothing."""
+    import subprocess
+    import sys
+    import importlib.util
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location("_sa_build", os.path.join(root, "indexer_selected_top_b200",
+                                                                            "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    lib = mod.build_debug()
+    env = dict(os.environ, SA_LIB=lib, SA_ROOT=root, PYTHONPATH=root)
+    r = subprocess.run([sys.executable, "-c", _DEBUG_CHILD], capture_output=True, text=True, timeout=600, env=env)
+    assert r.returncode == 0, r.stderr[-3000:]
+    res = json.loads(r.stdout.strip().splitlines()[-1])
+    assert res["bad_index"] is not None and res["bad_index"][0] == "attention index beyond the cache"
+    assert res["bad_index"][1] == 305 and res["same_as_skipped"]
+    assert res["lsa"] is None
