@@ -447,7 +447,22 @@ def run_native_lsa(args, rank, world, local_rank):
                   "select_us": round(sel_ms * 1e3, 1), "attention_us": round(att_ms * 1e3, 1),
                   "scan_hbm_bytes": cent_bytes,
                   "select_hbm_frac": round(cent_bytes / (sel_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
-        del Kd, Vd
+        # the selection replayed from a CUDA graph (no per-kernel launch cost), after the L2 flush
+        g = ldec.graph()
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            g.replay()
+        gt = 0.0
+        for _ in range(K_):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            b.synchronize()
+            gt += a.elapsed_time(b)
+        decode["graph_select_us"] = round(reduce_max([gt / K_ * 1e3], device=dev)[0], 1)
+        del g, Kd, Vd
 
     e2e = None
     if not args.skip_e2e:
