@@ -520,6 +520,8 @@ def run_native_lsa(args, rank, world, local_rank):
                    "k": wl.k, "n_sink": wl.n_sink, "n_window": wl.n_window, "Hq": wl.Hq, "head_dim": wl.dh,
                    "parallelism": f"replicas x{world}", "l2": "flushed (512 MB write) before every step"},
         "roofline": roof, "stages": stages, "decode": decode, "cpu_baseline": cpu, "e2e": e2e,
+        # per stage (cluster, search, attention): error, wait site, fallback rows, overflowed rows
+        "status": run.stage_status.cpu().tolist(),
         "gpu_launches": launches * K_, "clocks": clk,
     }
     if rank == 0:
