@@ -372,7 +372,7 @@ def expand_sinks_window(idx: torch.Tensor, q_pos0: int, n_sink: int, n_window: i
     n_q, k = idx.shape
     out = torch.empty((n_q, n_sink + n_window + k), dtype=torch.int32, device=idx.device)
     _check(_lib.sa_expand_sinks_window(_ptr(idx), n_q, k, q_pos0, n_sink, n_window, _ptr(out), _stream()),
-           "sa_expand_sinks_window", "sa_lsa_build_buckets", "sa_lsa_search", "sa_lsa_search_workspace_size")
+           "sa_expand_sinks_window")
     return out
 
 
@@ -475,8 +475,8 @@ class LsaPrefill:
 
     def __call__(self, stream=None):
         st = _stream(stream)
-        ts = torch.cuda.current_stream() if stream is None else stream
         ev = self.timer.events if self.timer else None
+        ts = (torch.cuda.current_stream() if stream is None else stream) if ev else None
         cent, off, keys = self.cache
         if ev:
             ev[0].record(ts)

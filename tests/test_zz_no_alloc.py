@@ -6,7 +6,8 @@ device memory, or a decode loop that may not call the CUDA allocator once it
 is running). It keeps its split-K partial results in a fixed array inside the
 library instead. These checks call it through the C ABI twice in a row, with
 different shapes so the second call runs on the first call's leftovers, and
-compare each result with sa_sparse_attn given its own workspace. The file
+compare each result with sa_sparse_attn given its own workspace and with the
+oracle's fp64 attention over the same index rows. The file
 sorts last so a run that stops at the first failure has run everything else.
 """
 import ctypes
@@ -53,9 +54,17 @@ def _call_noalloc(sa, Q, K, V, idx):
     return out, lse
 
 
-def test_noalloc_matches_workspace_path_twice(sa):
-    cases = [(64, 4096, 16, 128, 2048, 1, 1.0 / np.sqrt(128)),   # decode-sized batch, k = 2048
-             (3, 900, 16, 128, 700, 2, 1.0)]                     # smaller and sharper, on leftovers
+@pytest.mark.parametrize("cases", [
+    # decode-sized batch at k = 2048, then a smaller, sharper call on its leftovers
+    [(64, 4096, 16, 128, 2048, 1, 1.0 / np.sqrt(128)), (3, 900, 16, 128, 700, 2, 1.0)],
+    # the other head shape: 8 heads of 64, k not a multiple of the 256-key split
+    [(5, 3000, 8, 64, 1000, 4, 1.0 / 8.0), (2, 700, 8, 64, 300, 5, 1.0)],
+])
+def test_noalloc_matches_workspace_path_twice(sa, cases):
+    """Two calls in a row: each result equals sa_sparse_attn's (same
+    tolerance as every attention parity test), and both equal the oracle's
+    fp64 softmax attention over the same index rows."""
+    from oracle import sparse_attention_row
     for B, L, hq, dh, k, seed, std in cases:
         Q, K, V, idx = _case(B, L, hq, dh, k, seed, std)
         ref_out, ref_lse = sa.sparse_attn(Q, K, V, idx)
@@ -63,8 +72,12 @@ def test_noalloc_matches_workspace_path_twice(sa):
         torch.cuda.synchronize()
         ro, rl = ref_out.float().cpu().numpy(), ref_lse.cpu().numpy()
         go, gl = out.float().cpu().numpy(), lse.cpu().numpy()
+        Qh, Kh, Vh, ih = Q.double().cpu().numpy(), K.double().cpu().numpy(), V.double().cpu().numpy(), \
+            idx.cpu().numpy()
         for b in range(B):
-            check_attention_row(go[b], ro[b], gl[b], rl[b], f"B={B} seq {b}")
+            check_attention_row(go[b], ro[b], gl[b], rl[b], f"B={B} seq {b} vs sa_sparse_attn")
+            o, l = sparse_attention_row(Qh[b], Kh[b], Vh[b], ih[b])
+            check_attention_row(go[b], o, gl[b], l, f"B={B} seq {b} vs oracle")
 
 
 def test_noalloc_rejects_sizes_beyond_its_array(sa):
