@@ -114,13 +114,12 @@ def _isnum(s):
         return False
 
 
-# DRAM bytes per launch of a kernel from one ncu capture (read + write),
-# captured on the two-stage workload at T_cap rows and scaled to the run by
-# the number of candidate keys scored (the candidate scores are most of the
-# traffic). The capture and its command are summarised in profiles/; an entry
-# is removed when its kernel changes.
+# DRAM bytes per launch of a kernel from one ncu capture (dram__bytes_read.sum
+# + dram__bytes_write.sum), captured on the two-stage workload at T_cap rows
+# and scaled to the run by the number of candidate keys scored (the candidate
+# scores are most of the traffic). An entry is removed when its kernel changes.
 MEASURED_DRAM = {
-    # stage2_indexer_two_stage.md: indexer_kernel<64, 128, 1, 3>, T = 16384
+    # the stage-2 indexer_kernel<64, 128, 1, 3> (grouped mode), two-stage workload at T = 16384
     "stage2_indexer": {"bytes": 147.324672e6 + 184.366592e6, "T_cap": 16384},
 }
 
@@ -189,21 +188,33 @@ def lsa_work(wl):
 
 
 # ------------------------------------------------------------- CPU oracle
-def oracle_two_stage_sample(host, wl, n_rows: int, seed: int):
-    """Times the oracle on pooling (all blocks) + n_rows stratified rows of
-    the two-stage prefill; returns (tokens/s extrapolated to T rows, info)."""
+def timing_rows(T: int, n: int, seed: int = 0):
+    """n evenly spaced query rows, t_i = floor((i + f) T / n), with the
+    offset f in [0, 1) drawn from the seed: every stratum of [0, T) once, so
+    the mean cost per row estimates the mean over all rows."""
+    import numpy as np
+    f = (0.5 + seed * 0.6180339887498949) % 1.0
+    return np.minimum(T - 1, ((np.arange(n) + f) * T / n).astype(np.int64))
+
+
+def oracle_two_stage_sample(host, wl, n_rows: int, seed: int = 0):
+    """Times the oracle on pooling (all blocks) + n_rows evenly spaced rows of
+    the two-stage prefill; returns (tokens/s extrapolated to T rows, info).
+    info["cores"] is the process CPU time over the wall time: the host cores
+    the oracle kept busy (its row loop is serial; numpy's BLAS threads the
+    products)."""
     import oracle
     from oracle.two_stage import pool_block_keys
-    from workloads import sample_rows
-    rows = sample_rows(wl.T, n_rows, seed=seed, k=wl.k)
-    t0 = time.perf_counter()
+    rows = timing_rows(wl.T, n_rows, seed)
+    c0, t0 = time.process_time(), time.perf_counter()
     blocks = pool_block_keys(host["k_idx"].numpy(), host["k_scale"].numpy(), wl.block_size)
     t1 = time.perf_counter()
     oracle.prefill_rows(host, rows, wl.k, mode="two_stage", keep=wl.keep_blocks, blocks=blocks)
-    t2 = time.perf_counter()
+    c2, t2 = time.process_time(), time.perf_counter()
     per_row = (t2 - t1) / len(rows)
     full_s = (t1 - t0) + per_row * wl.T
-    return wl.T / full_s, {"pool_s": t1 - t0, "rows": len(rows), "rows_s": t2 - t1, "extrapolated_s": full_s}
+    return wl.T / full_s, {"pool_s": t1 - t0, "rows": len(rows), "rows_s": t2 - t1, "extrapolated_s": full_s,
+                           "measured_s": t2 - t0, "cores": round((c2 - c0) / max(t2 - t0, 1e-9), 2)}
 
 
 def oracle_decode_sample(hostd, wd, n_seq: int):
@@ -291,6 +302,8 @@ def run_reference(args):
     if args.workload in LSA_WORKLOADS:
         return run_reference_lsa(args)
     wl = WORKLOADS[args.workload]
+    if args.T:
+        wl = wl.with_(T=args.T)
     wd = WORKLOADS["decode_b64_l128k"]
     inp = PrefillInputs(wl, "cpu", seed=args.seed)
     host = inp.to_host()
@@ -306,18 +319,25 @@ def run_reference(args):
     dec_us, _ = oracle_decode_sample(hostd, wd.with_(batch=2), 1)
     dec_us = dec_us / 2 * wd.batch
     value = statistics.mean(vals)
+    measured_s = statistics.mean(x["measured_s"] for x in infos)
     sec_per_step = statistics.mean(x["extrapolated_s"] for x in infos)
-    sample = (f"per step: mean-pooling of all {wl.T // wl.block_size} blocks + {args.ref_rows} stratified "
-              f"query rows (both indexer stages, top-k, attention), extrapolated to {wl.T} rows")
+    cores = round(statistics.mean(x["cores"] for x in infos), 2)
+    sample = (f"per step: mean-pooling of all {wl.T // wl.block_size} blocks + {args.ref_rows} evenly spaced "
+              f"query rows (both indexer stages, top-k, attention); value = {wl.T} rows over the extrapolated "
+              f"time of all rows; cores = process CPU time / wall time")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(sec_per_step * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        # the measured wall time of one step (its sample); the full workload's
+        # time is an extrapolation and is reported apart
+        "ms_per_step": round(measured_s * 1e3, 3),
+        "extrapolated_full_step_ms": round(sec_per_step * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "k": wl.k, "mode": "two_stage", "block": wl.block_size,
-                   "keep_blocks": wl.keep_blocks, "seed": args.seed},
-        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                         "sample": sample},
+                   "keep_blocks": wl.keep_blocks, "seed": args.seed, "rows_per_step": args.ref_rows},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "threads": blas_threads(),
+                         "kind": "oracle", "sample": sample},
         "decode": {"us_per_step": round(dec_us, 1), "us_per_token": round(dec_us / wd.batch, 2),
                    "sample": "1 sequence of 131072 keys, scaled to the 64-sequence step"},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -528,56 +548,155 @@ def run_native_lsa(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def _build_library():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_sa_build", os.path.join(ROOT, "indexer_selected_top_b200",
+                                                                            "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
+def measure_fp8_peak(dev, n: int = 8192, reps: int = 10):
+    """Dense FP8 e4m3 tensor throughput of this GPU, measured the way the bf16
+    peak in MEASURED_PEAKS.json is: one n^3 product (torch._scaled_mm, cuBLAS,
+    bf16 output), best of `reps` CUDA-event timings, 2 n^3 flops."""
+    import torch
+    a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()
+    one = torch.tensor(1.0, device=dev)
+    for _ in range(3):
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        e1.record()
+        e1.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    del a, b
+    return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+
+
+def prefill_roofline(wl, stages_ms: dict, peaks: dict, fp8_peak: float, traffic_known: bool = True):
+    """Per-stage roofline of a prefill (algorithmic work over the stage's
+    device time, summed over chunks) and the dominant stage's entry."""
+    streaming = wl.mode != "two_stage" and wl.T > 65536
+    work = two_stage_work(wl) if wl.mode == "two_stage" else flat_work(wl, streaming)
+    idx_peak = fp8_peak if wl.idx_dtype == "fp8" else peaks["bf16_tflops"]
+    flop_stage = {"stage2_indexer": "stage2_flops", "stage1_indexer": "stage1_flops", "indexer": "indexer_flops"}
+    stages = {}
+    for n, ms in stages_ms.items():
+        s = max(ms, 1e-9) * 1e-3
+        if n in flop_stage:
+            stages[n] = {"ms": round(ms, 4), "bound": "tensor", "achieved": work[flop_stage[n]] / s / 1e12,
+                         "peak": idx_peak, "unit": "TFLOP/s"}
+        elif n == "attention":
+            # the grouped kernels read each union key once per group of queries
+            # (from L2), so gathered bytes do not bound them: the algorithmic
+            # work is the 4 Hq dh flops of every selected (query, key) pair
+            stages[n] = {"ms": round(ms, 4), "bound": "tensor", "achieved": work["attn_flops"] / s / 1e12,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+        elif n == "topk" and work["topk_bytes"] > 0 and ms > 0:
+            stages[n] = {"ms": round(ms, 4), "bound": "hbm", "achieved": work["topk_bytes"] / s / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        else:
+            stages[n] = {"ms": round(ms, 4)}
+    for v in stages.values():
+        if "achieved" in v:
+            v["achieved"] = round(v["achieved"], 2)
+            v["peak"] = round(v["peak"], 1)
+            v["frac"] = round(v["achieved"] / v["peak"], 4)
+    dom = max((n for n in stages if "achieved" in stages[n]), key=lambda n: stages[n]["ms"])
+    roof = dict(stages[dom])
+    roof.pop("ms")
+    roof["kernel"] = dom
+    roof["traffic"] = measured_traffic(dom, wl) if traffic_known else None
+    return stages, roof
+
+
+def time_prefill(sa, wl, dev, seed: int, warmup: int, steps: int, flush, mode=None):
+    """A prepared sa_prefill over one seeded input of `wl`, timed on the
+    device (CUDA events, L2 flushed before every step outside the events).
+    Returns (ms per step, stage ms per step summed over chunks, status words,
+    prepared call, inputs)."""
+    import torch
+    from workloads import PrefillInputs
+    inp = PrefillInputs(wl, dev, seed=seed)
+    status = sa.new_status(dev)
+    mode = mode or wl.mode
+    # the library's default chunking; two-stage tables for all rows at once
+    chunk = wl.T if mode == "two_stage" else 0
+    pre = sa.Prefill(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, wl.k, mode=mode,
+                     keep_blocks=wl.keep_blocks, chunk_rows=chunk, status=status, timed=True)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        flush.fill_(1)
+        pre()
+    torch.cuda.synchronize()
+    tot, stage_ms = 0.0, {n: 0.0 for n in pre.timer.names}
+    words = [0, 0, 0, 0]
+    for _ in range(steps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        pre()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1)
+        for n, v in pre.timer.ms().items():
+            stage_ms[n] += v
+        w = status.cpu().tolist()
+        if w[0] != 0:
+            raise RuntimeError(f"{wl.name}: device status {w}")
+        words = [max(a, b) for a, b in zip(words, w)]
+    return tot / steps, {n: v / steps for n, v in stage_ms.items()}, words, pre, inp
+
+
 def run_native(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     from workloads import LSA_WORKLOADS
-    if args.workload in LSA_WORKLOADS:
-        if rank == 0:
-            import importlib.util
-            spec = importlib.util.spec_from_file_location("_sa_build", os.path.join(ROOT, "indexer_selected_top_b200",
-                                                                                    "build.py"))
-            mod = importlib.util.module_from_spec(spec)
-            spec.loader.exec_module(mod)
-            mod.build()
-        if world > 1:
-            dist.barrier()
-        return run_native_lsa(args, rank, world, local_rank)
     if rank == 0:
-        import importlib.util
-        spec = importlib.util.spec_from_file_location("_sa_build", os.path.join(ROOT, "indexer_selected_top_b200",
-                                                                                "build.py"))
-        mod = importlib.util.module_from_spec(spec)
-        spec.loader.exec_module(mod)
-        mod.build()
+        _build_library()
     if world > 1:
         dist.barrier()
+    if args.workload in LSA_WORKLOADS:
+        return run_native_lsa(args, rank, world, local_rank)
     import indexer_selected_top_b200 as sa
-    from workloads import WORKLOADS, PrefillInputs, DecodeInputs
+    from workloads import WORKLOADS, DecodeInputs
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    fp8_peak = measure_fp8_peak(dev)
     wl = WORKLOADS[args.workload]
     if args.T:
         wl = wl.with_(T=args.T)
     wd = WORKLOADS["decode_b64_l128k"]
     seed = rank_seed(args.seed, rank)
-    inp = PrefillInputs(wl, dev, seed=seed)
-    ptimer = sa.StageTimer(sa.PREFILL_STAGES[wl.mode])
-    # one chunk for the two-stage and table paths (stage events cover the whole step)
-    chunk = wl.T if (wl.mode == "two_stage" or wl.T <= 65536) else 0
-    pre = sa.Prefill(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, wl.k, mode=wl.mode,
-                     keep_blocks=wl.keep_blocks, chunk_rows=chunk, timer=ptimer)
-    dec = None
-    if not args.no_decode:
-        dinp = DecodeInputs(wd, dev, seed=seed)
-        dtimer = sa.StageTimer(sa.DECODE_STAGES)
-        dec = sa.Decode(dinp.q_idx, dinp.q_scale, dinp.k_idx, dinp.k_scale, dinp.w, dinp.Q, dinp.K, dinp.V,
-                        dinp.seq_lens, wd.k, timer=dtimer)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(timed):
+    # ---------------- the headline prefill, the decode step ----------------
+    from workloads import PrefillInputs
+    inp = PrefillInputs(wl, dev, seed=seed)
+    pstatus = sa.new_status(dev)
+    chunk = wl.T if wl.mode == "two_stage" else 0
+    pre = sa.Prefill(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, wl.k, mode=wl.mode,
+                     keep_blocks=wl.keep_blocks, chunk_rows=chunk, status=pstatus, timed=True)
+    ptimer = pre.timer
+    dec = dstatus = None
+    if not args.no_decode:
+        dinp = DecodeInputs(wd, dev, seed=seed)
+        dtimer = sa.StageTimer(sa.DECODE_STAGES)
+        dstatus = sa.new_status(dev)
+        dec = sa.Decode(dinp.q_idx, dinp.q_scale, dinp.k_idx, dinp.k_scale, dinp.w, dinp.Q, dinp.K, dinp.V,
+                        dinp.seq_lens, wd.k, timer=dtimer, status=dstatus)
+
+    def step():
         flush.fill_(1)                                   # evict L2, outside the timed events
         e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
         e0.record(stream)
@@ -588,9 +707,15 @@ def run_native(args, rank, world, local_rank):
         e2.record(stream)
         return e0, e1, e2
 
+    def check_status():
+        for name, st in (("prefill", pstatus), ("decode", dstatus)):
+            if st is not None and st[0].item() != 0:
+                raise RuntimeError(f"{name}: device status {st.cpu().tolist()}")
+
     for _ in range(args.warmup):
-        step(False)
+        step()
     torch.cuda.synchronize()
+    check_status()
     clocks = ClockSampler(local_rank)
     if world > 1:
         dist.barrier()
@@ -602,14 +727,19 @@ def run_native(args, rank, world, local_rank):
     recs = []
     stage_ms = {n: 0.0 for n in ptimer.names}
     dstage_ms = {n: 0.0 for n in sa.DECODE_STAGES}
+    words = {"prefill": [0, 0, 0, 0], "decode": [0, 0, 0, 0]}
     for _ in range(args.steps):
-        recs.append(step(True))
-        torch.cuda.synchronize()                         # read this step's stage events
+        recs.append(step())
+        torch.cuda.synchronize()                         # read this step's stage events and status words
+        check_status()
         for n, v in ptimer.ms().items():
             stage_ms[n] += v
         if dec is not None:
             for n, v in dtimer.ms().items():
                 dstage_ms[n] += v
+        for name, st in (("prefill", pstatus), ("decode", dstatus)):
+            if st is not None:
+                words[name] = [max(a, b) for a, b in zip(words[name], st.cpu().tolist())]
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -619,40 +749,12 @@ def run_native(args, rank, world, local_rank):
     pre_ms, dec_ms, all_ms = reduce_max([pre_ms, dec_ms, pre_ms + dec_ms], device=dev)
     K = args.steps
 
-    # ---------------- roofline of the dominant prefill kernel ----------------
-    peaks, peak_src = load_peaks()
-    fp8_peak = 2.0 * peaks["bf16_tflops"]                # dense FP8 = 2 x measured bf16 (nominal ratio)
-    work = two_stage_work(wl) if wl.mode == "two_stage" else flat_work(wl, wl.T > 65536)
     avg = {n: v / K for n, v in stage_ms.items()}
-    flop_stage = {"stage2_indexer": "stage2_flops", "stage1_indexer": "stage1_flops", "indexer": "indexer_flops"}
-    stages = {}
-    for n, ms in avg.items():
-        s = max(ms, 1e-9) * 1e-3
-        if n in flop_stage:
-            stages[n] = {"ms": round(ms, 4), "bound": "tensor", "achieved": work[flop_stage[n]] / s / 1e12,
-                         "peak": fp8_peak, "unit": "TFLOP/s"}
-        elif n == "attention":
-            # the grouped kernels read each union key once per group of queries
-            # (from L2), so gathered bytes no longer bound them: the algorithmic
-            # work is the 4 Hq dh flops of every selected (query, key) pair
-            stages[n] = {"ms": round(ms, 4), "bound": "tensor", "achieved": work["attn_flops"] / s / 1e12,
-                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
-        elif n == "topk" and work["topk_bytes"] > 0:
-            stages[n] = {"ms": round(ms, 4), "bound": "hbm", "achieved": work["topk_bytes"] / s / 1e9,
-                         "peak": peaks["hbm_gbs"], "unit": "GB/s"}
-        else:
-            stages[n] = {"ms": round(ms, 4)}
-    for v in stages.values():
-        if "achieved" in v:
-            v["achieved"] = round(v["achieved"], 2)
-            v["frac"] = round(v["achieved"] / v["peak"], 4)
-    dom = max((n for n in stages if "achieved" in stages[n]), key=lambda n: stages[n]["ms"])
-    roof = dict(stages[dom])
-    roof.pop("ms")
-    roof["kernel"] = dom
-    roof["traffic"] = measured_traffic(dom, wl)
-    roof["peak_source"] = (f"{peak_src}: " + ("2 x bf16 burst (nominal FP8/bf16 ratio)" if roof["peak"] == fp8_peak
-                                              else "bf16 burst" if roof["unit"] == "TFLOP/s" else "HBM copy"))
+    stages, roof = prefill_roofline(wl, avg, peaks, fp8_peak)
+    roof["peak_source"] = (f"FP8 e4m3: measured in this run (cuBLAS _scaled_mm 8192^3, best of 10); "
+                           f"2 x the bf16 burst of MEASURED_PEAKS.json would be {2 * peaks['bf16_tflops']:.1f}"
+                           if roof["unit"] == "TFLOP/s" and roof["peak"] == round(fp8_peak, 1)
+                           else f"{peak_src}: " + ("bf16 burst" if roof["unit"] == "TFLOP/s" else "HBM copy"))
 
     decode = None
     if dec is not None:
@@ -666,7 +768,8 @@ def run_native(args, rank, world, local_rank):
                   "gather_hbm_frac": round(dw["attn_bytes"] / (davg["attention"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                            4),
                   "step_hbm_frac": round((dw["indexer_bytes"] + dw["topk_bytes"] + dw["attn_bytes"]) /
-                                         (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)}
+                                         (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+                  "status": words["decode"]}
         # the same step replayed from a CUDA graph (no per-kernel launch cost),
         # each replay after the L2 flush, timed on the device like the eager steps
         g = dec.graph()
@@ -682,6 +785,7 @@ def run_native(args, rank, world, local_rank):
             b.record()
             b.synchronize()
             gt += a.elapsed_time(b)
+        check_status()
         gus = reduce_max([gt / K * 1e3], device=dev)[0]
         decode["graph_us_per_step"] = round(gus, 1)
         decode["graph_us_per_token"] = round(gus / wd.batch, 3)
@@ -715,6 +819,7 @@ def run_native(args, rank, world, local_rank):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
+        check_status()
         t_e2e = reduce_max([a.elapsed_time(b) / ne], device=dev)[0]
         e2e = {"value": round(weak_scaling_value(world, 1, wl.T, t_e2e), 1), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ne}
@@ -723,22 +828,52 @@ def run_native(args, rank, world, local_rank):
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
         host = inp.to_host()
-        v, info = oracle_two_stage_sample(host, wl, args.cpu_rows, seed=7)
-        cpu = {"value": round(v, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+        v, info = oracle_two_stage_sample(host, wl, args.cpu_rows)
+        cpu = {"value": round(v, 3), "unit": "tokens/s", "cores": info["cores"], "kind": "oracle",
+               "threads": blas_threads(),
                "sample": f"mean-pooling of all {wl.T // wl.block_size} blocks ({info['pool_s']:.1f} s) + "
-                         f"{info['rows']} stratified rows ({info['rows_s']:.1f} s: both indexer stages, top-k, "
-                         f"attention), extrapolated to {wl.T} rows"}
-
+                         f"{info['rows']} evenly spaced rows ({info['rows_s']:.1f} s: both indexer stages, top-k, "
+                         f"attention), extrapolated to {wl.T} rows; cores = process CPU time / wall time"}
     if wl.mode == "two_stage":
         # pool, stage 1, keep, query groups, group block unions, stage 2, top-k,
         # attention groups, group key unions, attention
-        pre_launches = 10
+        pre_launches = 10 * pre.chunks
     elif wl.T <= 65536:
-        pre_launches = 3                       # indexer (table), top-k, attention
+        pre_launches = 3 * pre.chunks          # indexer (table), top-k, attention
     else:                                      # streaming: sample gathers once; per chunk sample scores,
-        n_chunks = -(-wl.T // 16384)           # thresholds, scan, list select, compaction, attention
-        pre_launches = 2 + 6 * n_chunks        # (+ 5 per fallback batch, normally none)
+        pre_launches = 2 + 6 * pre.chunks      # thresholds, scan, list select, compaction, attention
     launches_per_step = pre_launches + (4 if dec is not None else 0)
+    headline_cfg = {"workload": wl.name, "T": wl.T, "H": wl.H, "d_idx": wl.d, "k": wl.k, "mode": wl.mode,
+                    "block": wl.block_size, "keep_blocks": wl.keep_blocks, "Hq": wl.Hq, "head_dim": wl.dh,
+                    "decode": None if dec is None else {"workload": wd.name, "batch": wd.batch, "L": wd.L},
+                    "parallelism": f"replicas x{world}", "l2": "flushed (512 MB write) before every step",
+                    "prefill_ms_per_step": round(pre_ms / K, 4), "status": words["prefill"]}
+    del pre, inp
+    if dec is not None:
+        del dec, dinp
+    torch.cuda.empty_cache()
+
+    # ---------------- the other configurations, one line each ----------------
+    configs = {}
+    if not args.headline_only:
+        for name, mode, w_c, k_c in (("tiny_t512", None, 3, 20), ("prefill_t16k", None, 3, 5),
+                                     ("two_stage_t64k", "flat", 2, 3), ("prefill_t1m", None, 1, 1)):
+            c = WORKLOADS[name]
+            if mode:
+                c = c.with_(mode=mode)
+            ms, sms, st, pc, ci = time_prefill(sa, c, dev, seed, w_c, k_c, flush)
+            ms = reduce_max([ms], device=dev)[0]
+            cst, croof = prefill_roofline(c, sms, peaks, fp8_peak, traffic_known=False)
+            configs[name + ("_flat" if mode else "")] = {
+                "tokens_per_s": round(weak_scaling_value(world, 1, c.T, ms), 1), "ms_per_step": round(ms, 4),
+                "T": c.T, "k": c.k, "mode": c.mode, "idx_dtype": c.idx_dtype,
+                "path": ("two-stage" if c.mode == "two_stage" else
+                         "flat, score table" if c.T <= 65536 else "flat, streaming threshold (no table)"),
+                "chunks": pc.chunks, "warmup": w_c, "steps": k_c, "stages": cst, "roofline": croof,
+                "status": st}
+            del pc, ci
+            torch.cuda.empty_cache()
+
     line = {
         "metric": METRIC,
         "value": round(weak_scaling_value(world, K, wl.T, pre_ms), 1),
@@ -748,14 +883,13 @@ def run_native(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp8-e4m3 indexer (f32 accumulate), bf16 attention (f32 softmax)",
         "data": "synthetic",
-        "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "d_idx": wl.d, "k": wl.k, "mode": wl.mode,
-                   "block": wl.block_size, "keep_blocks": wl.keep_blocks, "Hq": wl.Hq, "head_dim": wl.dh,
-                   "decode": None if dec is None else {"workload": wd.name, "batch": wd.batch, "L": wd.L},
-                   "parallelism": f"replicas x{world}", "l2": "flushed (512 MB write) before every step",
-                   "prefill_ms_per_step": round(pre_ms / K, 4)},
+        "config": headline_cfg,
         "roofline": roof,
         "stages": stages,
         "decode": decode,
+        "configs": configs,
+        "peaks": {"fp8_tflops_measured": round(fp8_peak, 1), "bf16_tflops": peaks["bf16_tflops"],
+                  "hbm_gbs": peaks["hbm_gbs"], "source": peak_src},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches_per_step * K,
@@ -776,10 +910,12 @@ def main():
     ap.add_argument("--T", type=int, default=0, help="override the prefill length (profiling runs)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the other configurations (16K, 1M, 64K flat, tiny) on the JSON line")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=96)
+    ap.add_argument("--cpu-rows", type=int, default=4096, help="rows of the oracle baseline (about 4 ms each)")
     ap.add_argument("--ref-rows", type=int, default=12)
     ap.add_argument("--lsa-cpu-rows", type=int, default=2048, help="query rows of the LSA oracle baseline")
     ap.add_argument("--lsa-decode-batch", type=int, default=64, help="sequences of the LSA decode step")

@@ -133,13 +133,21 @@ typedef struct {
   uint32_t overflow_rows;  /* rows whose candidate list overflowed */
 } sa_device_status;
 
-/* Optional stage timing: when stage_events is non-NULL the call records
- * stage_events[i] on `stream` before stage i of its FIRST chunk and
- * stage_events[n] after its last stage (n_stage_events must be >= n + 1).
+/* Optional stage timing: when stage_events is non-NULL the call records,
+ * for every chunk c of its rows (sa_prefill_chunk_rows gives the chunk
+ * size; decode has one chunk), stage_events[c * (n + 1) + i] on `stream`
+ * before stage i of that chunk and stage_events[c * (n + 1) + n] after its
+ * last stage. n_stage_events must be >= n + 1; chunks whose events lie past
+ * n_stage_events are not recorded. The time of stage i summed over the
+ * recorded chunks is then the sum of the elapsed times between events
+ * c * (n + 1) + i and c * (n + 1) + i + 1.
  * Stages (n): FLAT = indexer, top-k, attention (3); TWO_STAGE = pooling,
  * stage-1 indexer, block keep, stage-2 indexer, top-k, attention (6);
- * decode = indexer, top-k, attention (3). Events are created by the caller;
- * an event that cannot be recorded makes the call return
+ * decode = indexer, top-k, attention (3). The two-stage pooling runs once,
+ * in the first chunk (later chunks record an empty pooling stage); the FLAT
+ * path without a score table (SA_FLAT_STREAM) scores and selects inside its
+ * indexer stage (its top-k stage is empty). Events are created by the
+ * caller; an event that cannot be recorded makes the call return
  * SA_ERR_INVALID_ARGUMENT after its work has been queued. */
 #define SA_PREFILL_FLAT_STAGES 3
 #define SA_PREFILL_TWO_STAGE_STAGES 6
@@ -516,6 +524,16 @@ sa_status sa_debug_errors(uint32_t* out, int32_t reset);
  */
 sa_status sa_workspace_size(sa_op op, const sa_indexer_in* in, const sa_attn_in* attn,
                             const void* opts, size_t* bytes);
+
+/*
+ * sa_prefill_chunk_rows: the number of query rows sa_prefill processes per
+ * chunk for these operands and options (host call, no device work): the
+ * call's rows are taken in ceil(n_q / rows) consecutive chunks, each with
+ * its own stage events (see stage_events above). It follows the same plan as
+ * sa_workspace_size (SA_OP_PREFILL). SA_ERR_INVALID_ARGUMENT for a NULL
+ * argument or invalid options.
+ */
+sa_status sa_prefill_chunk_rows(const sa_indexer_in* in, const sa_prefill_opts* opts, int32_t* rows);
 
 #ifdef __cplusplus
 }

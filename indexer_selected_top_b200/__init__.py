@@ -36,7 +36,7 @@ EXPORTS = ("sa_status_string", "sa_index_scores", "sa_topk", "sa_sparse_attn", "
            "sa_workspace_size", "sa_sparse_attn_decode_noalloc", "sa_quantize_rows_e4m3",
            "sa_expand_sinks_window", "sa_lsa_build_buckets", "sa_lsa_search", "sa_lsa_search_workspace_size", "sa_lsa_decode",
            "sa_lsa_decode_workspace_size", "sa_lsa_attention", "sa_lsa_attention_workspace_size",
-           "sa_debug_errors")
+           "sa_debug_errors", "sa_prefill_chunk_rows")
 
 
 class IndexerIn(ctypes.Structure):
@@ -90,12 +90,15 @@ DECODE_STAGES = ("indexer", "topk", "attention")
 
 
 class StageTimer:
-    """torch.cuda.Events handed to the library; stage i runs between events i
-    and i+1 (first chunk only)."""
+    """torch.cuda.Events handed to the library: chunk c's stage i runs between
+    events c * (n + 1) + i and c * (n + 1) + i + 1 (n stages). ms() sums each
+    stage over the chunks (a prepared Prefill sizes its timer for all of its
+    chunks)."""
 
-    def __init__(self, names):
+    def __init__(self, names, chunks: int = 1):
         self.names = names
-        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+        self.chunks = max(1, chunks)
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range((len(names) + 1) * self.chunks)]
         for e in self.events:          # torch creates the CUDA event on first record
             e.record()
         self._arr = (ctypes.c_void_p * len(self.events))(*[e.cuda_event for e in self.events])
@@ -105,7 +108,13 @@ class StageTimer:
         return ctypes.cast(self._arr, ctypes.c_void_p)
 
     def ms(self) -> dict:
-        return {n: self.events[i].elapsed_time(self.events[i + 1]) for i, n in enumerate(self.names)}
+        n = len(self.names) + 1
+        return {name: sum(self.events[c * n + i].elapsed_time(self.events[c * n + i + 1])
+                          for c in range(self.chunks)) for i, name in enumerate(self.names)}
+
+    def total_ms(self) -> float:
+        """First event to last: the whole call, every chunk."""
+        return self.events[0].elapsed_time(self.events[-1])
 
 
 _P = ctypes.c_void_p
@@ -141,11 +150,13 @@ _lib.sa_debug_errors.argtypes = [_P, ctypes.c_int32]
 _lib.sa_workspace_size.argtypes = [ctypes.c_int, ctypes.POINTER(IndexerIn), ctypes.POINTER(AttnIn), _P,
                                    ctypes.POINTER(ctypes.c_size_t)]
 _lib.sa_sparse_attn_decode_noalloc.argtypes = [ctypes.POINTER(AttnIn), _P, ctypes.c_int32, _P, _P, _P]
+_lib.sa_prefill_chunk_rows.argtypes = [ctypes.POINTER(IndexerIn), ctypes.POINTER(PrefillOpts),
+                                       ctypes.POINTER(ctypes.c_int32)]
 for _f in ("sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode", "sa_workspace_size",
            "sa_sparse_attn_decode_noalloc", "sa_quantize_rows_e4m3", "sa_expand_sinks_window",
            "sa_lsa_build_buckets", "sa_lsa_search", "sa_lsa_search_workspace_size", "sa_lsa_decode",
            "sa_lsa_decode_workspace_size", "sa_lsa_attention", "sa_lsa_attention_workspace_size",
-           "sa_debug_errors"):
+           "sa_debug_errors", "sa_prefill_chunk_rows"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -270,15 +281,25 @@ class Prefill:
 
     def __init__(self, q, q_scale, k, k_scale, w, Q, K, V, k_top: int, mode: str = "flat", block_size=64,
                  keep_blocks=64, chunk_rows=0, q_pos0=0, softmax_scale=0.0, want_idx=True, want_lse=True,
-                 status=None, test_hook=0, timer: "StageTimer" = None, flat_path: str = "auto"):
+                 status=None, test_hook=0, timer: "StageTimer" = None, flat_path: str = "auto",
+                 timed: bool = False):
+        """timed=True: the call records its stages on a StageTimer of its
+        own (self.timer), sized for every chunk; or pass `timer`."""
         self.ind = indexer_in(q, q_scale, k, k_scale, w, q_pos0)
         self.att = attn_in(Q, K, V, softmax_scale)
         self.opts = PrefillOpts(k=k_top, mode=SA_MODE_TWO_STAGE if mode == "two_stage" else SA_MODE_FLAT,
                                 block_size=block_size, keep_blocks=keep_blocks, chunk_rows=chunk_rows,
-                                status=_ptr(status), test_hook=test_hook,
-                                stage_events=timer.ptr if timer else None,
-                                n_stage_events=len(timer.events) if timer else 0,
-                                flat_path=FLAT_PATHS[flat_path])
+                                status=_ptr(status), test_hook=test_hook, flat_path=FLAT_PATHS[flat_path])
+        rows = ctypes.c_int32(0)
+        _check(_lib.sa_prefill_chunk_rows(ctypes.byref(self.ind), ctypes.byref(self.opts), ctypes.byref(rows)),
+               "sa_prefill_chunk_rows")
+        self.chunk_rows = rows.value
+        self.chunks = -(-q.shape[0] // max(rows.value, 1))
+        if timed and timer is None:
+            timer = StageTimer(PREFILL_STAGES[mode], self.chunks)
+        if timer is not None:
+            self.opts.stage_events = timer.ptr
+            self.opts.n_stage_events = len(timer.events)
         self.timer = timer
         self.nws = workspace_size(SA_OP_PREFILL, self.ind, self.att, self.opts)
         self.ws = _workspace(self.nws, Q.device)

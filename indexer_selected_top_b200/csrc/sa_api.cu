@@ -273,14 +273,15 @@ static IdxArgs base_args(const sa_indexer_in* in, uint32_t* status, int hook) {
 
 static size_t esize(sa_dtype d) { return d == SA_FP8_E4M3 ? 1 : 2; }
 
-// Records stage_events[i] (first chunk only) when the caller asked for them.
+// Records stage_events[base + i] when the caller asked for them; base is the
+// first event of the current chunk (chunk * (stages + 1)).
 struct StageMarks {
   cudaEvent_t* ev;
   int n;
-  bool on;
+  int base = 0;
   bool ok = true;
   void mark(int i, cudaStream_t st) {
-    if (on && ev != nullptr && i < n && cudaEventRecord(ev[i], st) != cudaSuccess) {
+    if (ev != nullptr && base + i < n && cudaEventRecord(ev[base + i], st) != cudaSuccess) {
       (void)cudaGetLastError();   // do not let a bad event handle surface as a launch error
       ok = false;
     }
@@ -435,6 +436,16 @@ sa_status sa_workspace_size(sa_op op, const sa_indexer_in* in, const sa_attn_in*
   return SA_ERR_INVALID_ARGUMENT;
 }
 
+sa_status sa_prefill_chunk_rows(const sa_indexer_in* in, const sa_prefill_opts* o, int32_t* rows) {
+  if (in == nullptr || o == nullptr || rows == nullptr) return SA_ERR_INVALID_ARGUMENT;
+  if (o->k <= 0 || o->block_size <= 0 || o->keep_blocks <= 0 || in->n_q < 0 || in->n_k <= 0)
+    return SA_ERR_INVALID_ARGUMENT;
+  PrefillPlan p;
+  plan_prefill(in, o, &p);
+  *rows = p.R;
+  return SA_OK;
+}
+
 sa_status sa_index_scores(const sa_indexer_in* in, float* scores, int64_t ld, void* ws, size_t ws_bytes,
                           cudaStream_t stream) {
   (void)ws;
@@ -516,7 +527,7 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
   const float scale = attn_scale(at);
   const size_t qrow = (size_t)in->n_heads * in->d_idx * esize(in->dtype);
   cudaError_t e = cudaSuccess;
-  StageMarks sm{o->stage_events, o->n_stage_events, true};
+  StageMarks sm{o->stage_events, o->n_stage_events};
 
   if (o->mode == SA_MODE_TWO_STAGE) {
     uint8_t* blk = reinterpret_cast<uint8_t*>(w + p.off_blk);
@@ -535,7 +546,8 @@ sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* at, const sa_pre
     ci.q_scale = in->q_scale ? in->q_scale + (size_t)r0 * in->n_heads : nullptr;
     ci.w = in->w + (size_t)r0 * in->n_heads;
     int32_t* idx = idx_out ? idx_out + (size_t)r0 * o->k : reinterpret_cast<int32_t*>(w + p.off_idx);
-    sm.on = (r0 == 0);
+    sm.base = (r0 / p.R) * (n_stages + 1);
+    if (o->mode == SA_MODE_TWO_STAGE && r0 > 0) sm.mark(0, stream);   // pooling ran in the first chunk
     if (o->mode == SA_MODE_FLAT && p.stream) {
       sm.mark(0, stream);
       sa_status fs = stream_select_chunk(in, &ci, o, p, w, r0 == 0, idx, status, stream);
@@ -671,7 +683,7 @@ sa_status sa_decode(const sa_indexer_in* in, const sa_attn_in* at, const sa_deco
   char* w = static_cast<char*>(ws);
   uint32_t* status = o->status ? reinterpret_cast<uint32_t*>(o->status) : nullptr;
   if (status && cudaMemsetAsync(status, 0, sizeof(sa_device_status), stream) != cudaSuccess) return SA_ERR_CUDA;
-  StageMarks sm{o->stage_events, o->n_stage_events, true};
+  StageMarks sm{o->stage_events, o->n_stage_events};
   float* rows = reinterpret_cast<float*>(w + p.off_scores);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + p.off_idx);
   IdxArgs a = base_args(in, status, o->test_hook);

@@ -52,3 +52,29 @@ def test_lsa_reference_arm_prints_one_json_line():
     assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["config"]["workload"] == "lsa_t8k"
+
+
+def test_timing_rows_cover_every_stratum_once():
+    import bench
+    for T, n in ((65536, 96), (1000, 7), (64, 64)):
+        for seed in (0, 3):
+            r = bench.timing_rows(T, n, seed)
+            assert len(r) == n and (r >= 0).all() and (r < T).all()
+            assert (((r * n) // T) == list(range(n))).all(), (T, n, seed)
+
+
+def test_two_stage_reference_arm_reports_measured_and_extrapolated_time():
+    """The reference arm's ms_per_step is the wall time it measured; the full
+    workload's time is an extrapolation, reported apart and larger."""
+    env = dict(os.environ, PYTHONPATH=ROOT)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--T", "4096",
+                        "--steps", "1", "--warmup", "0", "--ref-rows", "4"],
+                       capture_output=True, text=True, timeout=600, env=env, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["config"]["T"] == 4096 and d["config"]["rows_per_step"] == 4
+    assert 0 < d["ms_per_step"] < d["extrapolated_full_step_ms"]
+    assert abs(d["value"] - 4096 / (d["extrapolated_full_step_ms"] * 1e-3)) <= 1e-3 * d["value"] + 1e-3
+    assert d["cpu_baseline"]["cores"] > 0 and d["cpu_baseline"]["value"] == d["value"]

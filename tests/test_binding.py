@@ -5,9 +5,9 @@ status code into SaError. A wrapper whose call or status check is malformed
 (wrong arity, a wrong argument type, a bad _check call) would only show on a
 GPU. Here the library handle is replaced by a proxy that checks each call
 against the real function's declared argtypes (count, and the conversion ctypes
-itself applies), answers workspace-size queries on the host, and returns
-SA_ERR_INVALID_ARGUMENT for every other entry point: each wrapper must then
-raise SaError naming that entry point. No compute entry point of the library
+itself applies), answers the size queries (workspace bytes, chunk rows) on
+the host, and returns SA_ERR_INVALID_ARGUMENT for every other entry point:
+each wrapper must then raise SaError naming that entry point. No compute entry point of the library
 is called, and every tensor stays in host memory."""
 import ctypes
 
@@ -50,8 +50,8 @@ class _Proxy:
             for a, t in zip(args, fn.argtypes):
                 t.from_param(a)                      # raises as ctypes would on a wrong type
             self._calls.append(name)
-            if name.endswith("workspace_size"):
-                out = args[-1]._obj                  # byref(c_size_t)
+            if name.endswith("workspace_size") or name == "sa_prefill_chunk_rows":
+                out = args[-1]._obj                  # byref(c_size_t) / byref(c_int32)
                 out.value = 4096
                 return 0
             return 1                                 # SA_ERR_INVALID_ARGUMENT
@@ -112,6 +112,24 @@ def test_core_wrappers_reach_their_status_check(proxied):
     _raises(sa, calls, "sa_decode", sa.decode, dq, dqs, dk, dks, dw, dQ, dK, dV, lens, 32)
     _raises(sa, calls, "sa_sparse_attn_decode_noalloc", sa.sparse_attn_decode_noalloc, dQ, dK, dV,
             torch.zeros((2, 32), dtype=torch.int32))
+
+
+def test_chunk_rows_query_wrapper_reaches_its_status_check(sa, monkeypatch):
+    calls = []
+
+    class _Fail(_Proxy):
+        def __getattr__(self, name):
+            inner = super().__getattr__(name)
+            if name != "sa_prefill_chunk_rows":
+                return inner
+
+            def call(*args):
+                inner(*args)
+                return 1
+            return call
+    monkeypatch.setattr(sa, "_lib", _Fail(sa._lib, calls))
+    q, qs, k, ks, w, Q, K, V = _prefill_inputs()
+    _raises(sa, calls, "sa_prefill_chunk_rows", sa.Prefill, q, qs, k, ks, w, Q, K, V, 32)
 
 
 def test_workspace_query_wrapper_reaches_its_status_check(sa, monkeypatch):
