@@ -12,11 +12,17 @@
 // are positive: ReLU(sq*sk*a) = sq*sk*ReLU(a).
 //
 // Roles: warp 0 = TMA producer (one lane), warp 1 = MMA issuer (one lane)
-// and TMEM owner, warps 2.. = TEAMS epilogue teams of 4 warps. The 512 TMEM
-// columns hold 512 / N fp32 accumulators (2 at N = 256, 8 at N = 64) used as
-// a ring; team b % TEAMS drains buffer b, so the epilogue of one
-// accumulator overlaps the MMAs into the others (the pages' bucket scan also
-// overlaps its epilogue with its products: appendix F.1, "Flat prefill").
+// and TMEM owner, warps 2..17 = epilogue teams. The 512 TMEM columns hold
+// 512 / N fp32 accumulators (2 at N = 256, 8 at N = 64) used as a ring; team
+// b % TEAMS drains buffer b, so the epilogue of one accumulator overlaps the
+// MMAs into the others (the pages' bucket scan also overlaps its epilogue
+// with its products: appendix F.1, "Flat prefill"). A team has 4 warps per
+// accumulator column slice, one per TMEM lane quarter: the wide modes (N =
+// 256 = 4 queries x 64 heads) run 2 teams of 8 warps, each warp draining one
+// 128-column slice (2 queries); the narrow modes (N = 64, one query) run 4
+// teams of 4 warps. On sm_100a one M = 128, K = 32 FP8 MMA costs about the
+// same ~97 cycles for any N up to 128 and ~128 cycles at N = 256, so N = 256
+// doubles the work per instruction for a third more time.
 //
 // Key sources (template MODE):
 //   IDX_PREFILL  keys [0, lim] of one sequence, NQ consecutive query rows per
@@ -44,16 +50,16 @@ namespace sa {
 #ifndef SA_IDX_STAGES
 #define SA_IDX_STAGES 6
 #endif
-// epilogue teams of 4 warps (2 or 4) and the prefill MMA N (256 or 128); a
-// team count above 2 needs N <= 128 so every team owns an accumulator. Four
-// teams at N = 128 measured fastest for the grouped stage 2 (more epilogue
-// warps hide the TMEM-load latency) and on par for the flat prefill.
-#ifndef SA_IDX_TEAMS
-#define SA_IDX_TEAMS 4
-#endif
+// the wide modes' MMA N (256 or 128) and their epilogue teams (16 warps in
+// 2 or 4 teams; every team owns whole accumulators, so 4 teams need N = 128)
 #ifndef SA_IDX_PREFILL_N
-#define SA_IDX_PREFILL_N 128
+#define SA_IDX_PREFILL_N 256
 #endif
+#ifndef SA_IDX_TEAMS_WIDE
+#define SA_IDX_TEAMS_WIDE 2
+#endif
+constexpr int kIdxEpiWarps = 16;                              // epilogue warps of every mode
+constexpr int kIdxThreads = 64 + 32 * kIdxEpiWarps;
 // independent partial sums per query in the epilogue when N holds several queries
 #ifndef SA_IDX_NP_WIDE
 #define SA_IDX_NP_WIDE 2
@@ -78,9 +84,14 @@ struct IdxCfg {
                             : (MODE == IDX_GROUPED) ? kGroupQueries
                                                     : 1;
   static constexpr int NBUF = 512 / N;                       // TMEM accumulator buffers (fp32 columns)
-  static constexpr int TEAMS = SA_IDX_TEAMS;
-  static constexpr int THREADS = 64 + 128 * TEAMS;
+  static constexpr int TEAMS = WIDE ? SA_IDX_TEAMS_WIDE : 4;
+  static constexpr int WPT = kIdxEpiWarps / TEAMS;           // warps per team
+  static constexpr int SLICES = WPT / 4;                      // column slices of an accumulator
+  static constexpr int SCOLS = N / SLICES;                    // columns one warp drains per job
+  static constexpr int QSW = QS / SLICES;                     // queries one warp drains per job
+  static constexpr int THREADS = kIdxThreads;
   static_assert(NBUF % TEAMS == 0, "every team owns whole accumulators");
+  static_assert(WPT % 4 == 0 && QS % SLICES == 0 && SCOLS == QSW * H, "a warp drains whole queries");
   static constexpr int QBYTES = NQ * H * ROWB;
   static constexpr int KBYTES = 128 * ROWB;
   static constexpr int NS = (MODE == IDX_DECODE) ? 8 : SA_IDX_STAGES;    // key-tile stages
@@ -98,7 +109,7 @@ struct IdxCfg {
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   static_assert(N <= 256 && N % 16 == 0, "MMA N");
   static_assert(MODE != IDX_GROUPED || QS * G == kGroupQueries, "one group per CTA");
-  static_assert(N % 32 == 0, "epilogue loads 32 columns at a time");
+  static_assert(SCOLS % 32 == 0, "epilogue loads 32 columns at a time");
 };
 
 __device__ __forceinline__ int vis_limit(int t, const IdxArgs& a) {
@@ -136,7 +147,7 @@ struct GatherCursor {
 };
 
 template <int H, int D, bool FP8, int MODE>
-__global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
+__global__ void __launch_bounds__(kIdxThreads, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                    const IdxArgs a) {
   using C = IdxCfg<H, D, FP8, MODE>;
@@ -199,7 +210,7 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
     mbar_init(qfull, 1);
     for (int b = 0; b < C::NBUF; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], C::WPT);
     }
     *abort_flag = 0u;
     fence_barrier_init();
@@ -369,7 +380,8 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
     }
   } else {
     // ======================= epilogue teams =======================
-    const int team = (warp - 2) >> 2;        // jobs j with j % TEAMS == team
+    const int team = (warp - 2) / C::WPT;    // jobs j with j % TEAMS == team
+    const int slice = ((warp - 2) % C::WPT) >> 2;   // the accumulator columns [slice * SCOLS, +SCOLS)
     const int lq = warp & 3;                 // TMEM lane quarter this warp may access
     const int row = lq * 32 + lane;          // key row of the tile (TMEM lane)
     // job -> (tile, sub-tile / query, this thread's key, its scale); the scale
@@ -441,20 +453,20 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
       // (a single running sum would be a dependent FMA chain of H links)
       constexpr int NPMAX = (C::QS > 1) ? SA_IDX_NP_WIDE : 8;
       constexpr int NP = (H / 4 < NPMAX) ? H / 4 : NPMAX;
-      constexpr int NCH = C::N / 32;
-      float acc[C::QS][NP];
+      constexpr int NCH = C::SCOLS / 32;
+      float acc[C::QSW][NP];
 #pragma unroll
-      for (int qq = 0; qq < C::QS; ++qq)
+      for (int qq = 0; qq < C::QSW; ++qq)
 #pragma unroll
         for (int p = 0; p < NP; ++p) acc[qq][p] = 0.f;
-      const uint32_t t_addr = tmem_base + (uint32_t(lq * 32) << 16) + buf * C::N;
-      const float* wrow = sW + g * C::N;
+      const uint32_t t_addr = tmem_base + (uint32_t(lq * 32) << 16) + buf * C::N + slice * C::SCOLS;
+      const float* wrow = sW + g * C::N + slice * C::SCOLS;
 #if SA_IDX_EPI_PACKED
       // w * ReLU(a) = (w / 2) * (a + |a|): a + |a| is exact (2a or +0) and one
       // FADD; the halved weights sit in sW, pairs accumulate with f32x2 FMAs
-      float2 acc2[C::QS][NP];
+      float2 acc2[C::QSW][NP];
 #pragma unroll
-      for (int qq = 0; qq < C::QS; ++qq)
+      for (int qq = 0; qq < C::QSW; ++qq)
 #pragma unroll
         for (int p = 0; p < NP; ++p) acc2[qq][p] = make_float2(0.f, 0.f);
       auto consume = [&](const float (&v)[32], int c) {
@@ -519,15 +531,16 @@ __global__ void __launch_bounds__(64 + 128 * SA_IDX_TEAMS, 1)
       }
       // outputs
 #pragma unroll
-      for (int qq = 0; qq < C::QS; ++qq) {
+      for (int qq = 0; qq < C::QSW; ++qq) {
         int t;
         int gcol = 0;                          // grouped: the query's candidate column of this key
+        const int qj = slice * C::QSW + qq;    // the query's place among the job's QS
         if constexpr (MODE == IDX_PREFILL) {
-          t = q0 + g * C::QS + qq;
+          t = q0 + g * C::QS + qj;
         } else if constexpr (MODE == IDX_DECODE) {
           t = seq;
         } else if constexpr (MODE == IDX_GROUPED) {
-          const int ql = g * C::QS + qq;
+          const int ql = g * C::QS + qj;
           t = sQt[ql];
           if (t < 0 || cur.s < 0) continue;    // absent query, or no union block in this half
           const int slot = (int)((sUSlot[col] >> (8 * ql)) & 0xFFu);
