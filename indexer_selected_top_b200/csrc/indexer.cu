@@ -175,6 +175,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 
   // ---------------- work unit (identical in every role) ----------------
   int q0 = 0, nq = 0, seq = 0, tile0 = 0, ntiles = 0, geff = 1, njobs = 0, seq_len = a.n_k;
+  int n_ub = 0;                    // grouped: the group's union blocks
   if constexpr (MODE == IDX_PREFILL) {
     const int unit = gridDim.x - 1 - blockIdx.x;            // heaviest (latest rows) first
     q0 = unit * C::NQ;
@@ -245,6 +246,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     // the group's queries and its union blocks with every query's slot
     const int g = blockIdx.x;
     const int nub = a.gb_n[g];
+    n_ub = nub;
     for (int i = threadIdx.x; i < C::NQ; i += blockDim.x) {
       const int t = a.perm[q0 + i];
       sQt[i] = (t >= 0 && t < a.n_q) ? t : -1;
@@ -309,7 +311,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           tma_load_2d(dst, &kmap, &kfull[st], 0, seq * a.n_k + (tile0 + i) * 128);
         } else if constexpr (MODE == IDX_GROUPED) {
           const int b0 = sUBlk[2 * i];
-          const int b1 = (2 * i + 1 < 2 * ntiles && 2 * i + 1 < a.gb_n[blockIdx.x]) ? sUBlk[2 * i + 1] : -1;
+          const int b1 = (2 * i + 1 < n_ub) ? sUBlk[2 * i + 1] : -1;
           mbar_arrive_expect_tx(&kfull[st], (b1 >= 0 ? 2 : 1) * 64 * C::ROWB);
           tma_load_2d(dst, &kmap, &kfull[st], 0, b0 * 64);
           if (b1 >= 0) tma_load_2d(dst + 64 * C::ROWB, &kmap, &kfull[st], 0, b1 * 64);
@@ -338,11 +340,16 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         tc_fence_after();
         GatherCursor gc;
         if constexpr (MODE == IDX_GATHER) gc.init(sKept, C::KEEPMAX, 0, nq);
+        int wtile = 0, wg = 0;             // wide modes: job j = tile * geff + g, advanced without division
         for (int j = 0; j < njobs; ++j) {
           int tile, g;
           if constexpr (C::WIDE) {
-            tile = j / geff;
-            g = j % geff;
+            tile = wtile;
+            g = wg;
+            if (++wg == geff) {
+              wg = 0;
+              ++wtile;
+            }
           } else {
             tile = j;
             g = (MODE == IDX_GATHER) ? gc.ql : 0;
@@ -383,7 +390,16 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     const int team = (warp - 2) / C::WPT;    // jobs j with j % TEAMS == team
     const int slice = ((warp - 2) % C::WPT) >> 2;   // the accumulator columns [slice * SCOLS, +SCOLS)
     const int lq = warp & 3;                 // TMEM lane quarter this warp may access
-    const int row = lq * 32 + lane;          // key row of the tile (TMEM lane)
+    // FP8 modes drain TMEM with the 16x256b shape: thread (quad r = lane / 4,
+    // place c = lane % 4) reads lanes r + 8a + 16h of its quarter and the
+    // columns 8i + 2c + e of each 32-column chunk, so it needs the weights of
+    // a fixed quarter of the columns only (held in registers) and sums its 16
+    // heads of a query per lane; a reduce-scatter over the quad then leaves it
+    // the full sums of lane 8c + r. The bf16 modes (4 or 8 heads) read one
+    // lane per thread (32x32b) with the weights from shared memory.
+    constexpr bool QUAD = FP8;
+    const int qr = lane >> 2, qc = lane & 3;
+    const int row = lq * 32 + (QUAD ? qr + 8 * qc : lane);   // key row of the tile this thread scores
     // job -> (tile, sub-tile / query, this thread's key, its scale); the scale
     // of the team's next job is loaded one job ahead so its global-load
     // latency hides behind the current job
@@ -395,6 +411,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     GatherCursor gc = {};                    // gather: cursor at the job being loaded
     int jq = 0;
     if constexpr (MODE == IDX_GATHER) gc.init(sKept, C::KEEPMAX, 0, nq);
+    // wide modes: (tile, sub-tile) of the job job_key is asked for next; the
+    // team's jobs advance by TEAMS, which moves these without a division
+    int ktile = C::WIDE ? team / geff : 0, kg = C::WIDE ? team % geff : 0;
     auto job_key = [&](int jj) {
       JobKey k;
       if constexpr (MODE == IDX_GATHER) {
@@ -406,15 +425,20 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       k.ql = gc.ql;
       k.pair = gc.pair;
       if constexpr (C::WIDE) {
-        k.tile = jj / geff;
-        k.g = jj % geff;
+        k.tile = ktile;
+        k.g = kg;
+        kg += C::TEAMS;
+        while (kg >= geff) {
+          kg -= geff;
+          ++ktile;
+        }
       } else {
         k.tile = jj;
         k.g = (MODE == IDX_GATHER) ? k.ql : 0;
       }
       if constexpr (MODE == IDX_GROUPED) {
         const int ub = 2 * k.tile + (row >> 6);
-        const int blk = (jj < njobs && ub < a.gb_n[blockIdx.x]) ? sUBlk[ub] : -1;
+        const int blk = (jj < njobs && ub < n_ub) ? sUBlk[ub] : -1;
         k.s = blk * 64 + (row & 63);
         k.kvalid = blk >= 0 && k.s < a.n_k;
         k.col = ub;                          // the union block: each query's slot of it is looked up per query
@@ -438,6 +462,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         k.sk = a.k_scale[(long long)seq * a.n_k * (MODE == IDX_DECODE) + k.s];
       return k;
     };
+    float2 wq[QUAD ? C::SCOLS / 32 : 1][4];   // 16x256b path: this thread's weights (halved), per chunk and group
+    int wg = -1;                             // the sub-tile / query they belong to
     JobKey nxt = job_key(team);
     for (int j = team; j < njobs; j += C::TEAMS) {
       const JobKey cur = nxt;
@@ -449,6 +475,85 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       if (!mbar_wait(&tfull[buf], ub & 1, wc, 5)) break;
       tc_fence_after();
 
+      float qsum[C::QSW];                      // sum_h w'[h] * ReLU(acc[h]) of this thread's key row, per query
+      auto release = [&]() {   // every column of this accumulator is in registers
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf]);
+      };
+      if constexpr (QUAD) {
+        constexpr int NCC = C::SCOLS / 32;     // 32-column chunks of the warp's slice (each within one query)
+        constexpr int NLD = 2 * NCC;           // loads: (lane half h, chunk)
+        static_assert(H % 32 == 0, "a chunk holds heads of one query");
+        if (g != wg) {                         // the job's queries changed: their weights of this thread's columns
+          const float* wrow = sW + g * C::N + slice * C::SCOLS + 2 * qc;
+#pragma unroll
+          for (int cc = 0; cc < NCC; ++cc)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) wq[cc][i] = *reinterpret_cast<const float2*>(wrow + cc * 32 + 8 * i);
+          wg = g;
+        }
+        // w * ReLU(a) = (w / 2) * (a + |a|): a + |a| is exact (2a or +0) and one
+        // FADD; the halved weights sit in sW, pairs of heads accumulate with
+        // f32x2 FMAs. acc2[L][qq]: lane 8L + r, query qq.
+        float2 acc2[4][C::QSW];
+#pragma unroll
+        for (int L = 0; L < 4; ++L)
+#pragma unroll
+          for (int qq = 0; qq < C::QSW; ++qq) acc2[L][qq] = make_float2(0.f, 0.f);
+        const uint32_t t0 = tmem_base + buf * C::N + slice * C::SCOLS;
+        auto addr = [&](int n) {
+          return t0 + (uint32_t(lq * 32 + 16 * (n / NCC)) << 16) + uint32_t((n % NCC) * 32);
+        };
+        auto consume = [&](const uint32_t (&v)[16], int n) {
+          const int h = n / NCC, cc = n % NCC, qq = cc * 32 / H;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int a2 = 0; a2 < 2; ++a2) {
+              const float x0 = __uint_as_float(v[4 * i + 2 * a2]), x1 = __uint_as_float(v[4 * i + 2 * a2 + 1]);
+              acc2[2 * h + a2][qq] =
+                  __ffma2_rn(wq[cc][i], make_float2(x0 + fabsf(x0), x1 + fabsf(x1)), acc2[2 * h + a2][qq]);
+            }
+        };
+        // double-buffered loads: load n + 1 is in flight while load n is consumed
+        uint32_t va[16], vb[16];
+        tmem_ld16x256b_x4(addr(0), va);
+        tmem_ld_wait();
+        tmem_regs_ready(va);
+#pragma unroll
+        for (int n = 0; n < NLD; n += 2) {
+          if (n + 1 < NLD) tmem_ld16x256b_x4(addr(n + 1), vb);
+          if (n + 1 >= NLD) release();
+          consume(va, n);
+          if (n + 1 < NLD) {
+            tmem_ld_wait();
+            tmem_regs_ready(vb);
+            if (n + 2 < NLD) tmem_ld16x256b_x4(addr(n + 2), va);
+            if (n + 2 >= NLD) release();
+            consume(vb, n + 1);
+            if (n + 2 < NLD) {
+              tmem_ld_wait();
+              tmem_regs_ready(va);
+            }
+          }
+        }
+        // reduce-scatter over the quad: the lane pair {0,1} or {2,3} by bit 1
+        // of c, then one lane by bit 0; thread c keeps lane c (row 8c + r)
+#pragma unroll
+        for (int qq = 0; qq < C::QSW; ++qq) {
+          float sl[4];
+#pragma unroll
+          for (int L = 0; L < 4; ++L) sl[L] = acc2[L][qq].x + acc2[L][qq].y;
+          const bool hi2 = (qc & 2) != 0, hi1 = (qc & 1) != 0;
+          float k0 = hi2 ? sl[2] : sl[0], k1 = hi2 ? sl[3] : sl[1];
+          const float o0 = hi2 ? sl[0] : sl[2], o1 = hi2 ? sl[1] : sl[3];
+          k0 += __shfl_xor_sync(0xffffffffu, o0, 2);
+          k1 += __shfl_xor_sync(0xffffffffu, o1, 2);
+          const float kk = hi1 ? k1 : k0, oo = hi1 ? k0 : k1;
+          qsum[qq] = kk + __shfl_xor_sync(0xffffffffu, oo, 1);
+        }
+      } else {
       // sum_h w'[h] * ReLU(acc[h]) in NP independent partial sums per query
       // (a single running sum would be a dependent FMA chain of H links)
       constexpr int NPMAX = (C::QS > 1) ? SA_IDX_NP_WIDE : 8;
@@ -501,11 +606,6 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         }
       };
 #endif
-      auto release = [&]() {   // every column of this accumulator is in registers
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[buf]);
-      };
       // double-buffered TMEM loads: chunk c + 1 is in flight while chunk c is
       // consumed (one wait::ld covers it)
       float va[32], vb[32];
@@ -528,6 +628,19 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             tmem_regs_ready(va);
           }
         }
+      }
+#pragma unroll
+      for (int qq = 0; qq < C::QSW; ++qq) {
+        float sum = 0.f;
+#if SA_IDX_EPI_PACKED
+#pragma unroll
+        for (int p = 0; p < NP; ++p) sum += acc2[qq][p].x + acc2[qq][p].y;
+#else
+#pragma unroll
+        for (int p = 0; p < NP; ++p) sum += acc[qq][p];
+#endif
+        qsum[qq] = sum;
+      }
       }
       // outputs
 #pragma unroll
@@ -555,15 +668,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           vis = kvalid;
         else
           vis = kvalid && s <= vis_limit(t, a);
-        float sum = 0.f;
-#if SA_IDX_EPI_PACKED
-#pragma unroll
-        for (int p = 0; p < NP; ++p) sum += acc2[qq][p].x + acc2[qq][p].y;
-#else
-#pragma unroll
-        for (int p = 0; p < NP; ++p) sum += acc[qq][p];
-#endif
-        const float score = vis ? sum * sk : -__int_as_float(0x7f800000);
+        const float score = vis ? qsum[qq] * sk : -__int_as_float(0x7f800000);
         if constexpr (MODE == IDX_PREFILL) {
           if (a.cand != nullptr) {
             // candidate mode: warp-aggregated append of keys at or above theta
