@@ -50,6 +50,10 @@ namespace sa {
 #ifndef SA_IDX_STAGES
 #define SA_IDX_STAGES 6
 #endif
+// FP8 prefill: sub-tiles of QS queries per CTA (each key tile serves G jobs)
+#ifndef SA_IDX_PREFILL_G
+#define SA_IDX_PREFILL_G 2
+#endif
 // the wide modes' MMA N (256 or 128) and their epilogue teams (16 warps in
 // 2 or 4 teams; every team owns whole accumulators, so 4 teams need N = 128)
 #ifndef SA_IDX_PREFILL_N
@@ -68,6 +72,11 @@ constexpr int kIdxThreads = 64 + 32 * kIdxEpiWarps;
 #ifndef SA_IDX_EPI_PACKED
 #define SA_IDX_EPI_PACKED 1
 #endif
+// FP8 (16x256b) epilogue math per head: 0 = (w/2)(a + |a|) in packed f32x2
+// FMAs, 1 = the same in scalar FMAs, 2 = w * max(a, 0) in scalar FMAs
+#ifndef SA_IDX_QUAD_MATH
+#define SA_IDX_QUAD_MATH 0
+#endif
 
 template <int H, int D, bool FP8, int MODE>
 struct IdxCfg {
@@ -76,7 +85,7 @@ struct IdxCfg {
   static constexpr bool WIDE = MODE == IDX_PREFILL || MODE == IDX_GROUPED;   // N = QS queries x H heads
   static constexpr int QS = WIDE ? (SA_IDX_PREFILL_N / H) : 1;
   static constexpr int N = QS * H;                           // MMA N
-  static constexpr int G = (MODE == IDX_PREFILL)   ? (QS * 2 < 8 ? 8 / QS : 2)
+  static constexpr int G = (MODE == IDX_PREFILL)   ? (QS * 2 < 8 ? 8 / QS : SA_IDX_PREFILL_G)
                            : (MODE == IDX_GROUPED) ? (kGroupQueries / QS > 0 ? kGroupQueries / QS : 1)
                                                    : 1;      // sub-tiles per CTA
   static constexpr int NQ = (MODE == IDX_PREFILL)   ? QS * G
@@ -490,7 +499,12 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 #pragma unroll
           for (int cc = 0; cc < NCC; ++cc)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) wq[cc][i] = *reinterpret_cast<const float2*>(wrow + cc * 32 + 8 * i);
+            for (int i = 0; i < 4; ++i) {
+              wq[cc][i] = *reinterpret_cast<const float2*>(wrow + cc * 32 + 8 * i);
+#if SA_IDX_QUAD_MATH == 2
+              wq[cc][i] = make_float2(2.f * wq[cc][i].x, 2.f * wq[cc][i].y);
+#endif
+            }
           wg = g;
         }
         // w * ReLU(a) = (w / 2) * (a + |a|): a + |a| is exact (2a or +0) and one
@@ -512,8 +526,16 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 #pragma unroll
             for (int a2 = 0; a2 < 2; ++a2) {
               const float x0 = __uint_as_float(v[4 * i + 2 * a2]), x1 = __uint_as_float(v[4 * i + 2 * a2 + 1]);
-              acc2[2 * h + a2][qq] =
-                  __ffma2_rn(wq[cc][i], make_float2(x0 + fabsf(x0), x1 + fabsf(x1)), acc2[2 * h + a2][qq]);
+              float2& acc = acc2[2 * h + a2][qq];
+#if SA_IDX_QUAD_MATH == 0
+              acc = __ffma2_rn(wq[cc][i], make_float2(x0 + fabsf(x0), x1 + fabsf(x1)), acc);
+#elif SA_IDX_QUAD_MATH == 1
+              acc.x = fmaf(wq[cc][i].x, x0 + fabsf(x0), acc.x);
+              acc.y = fmaf(wq[cc][i].y, x1 + fabsf(x1), acc.y);
+#else
+              acc.x = fmaf(wq[cc][i].x, fmaxf(x0, 0.f), acc.x);   // the weights hold w, not w / 2
+              acc.y = fmaf(wq[cc][i].y, fmaxf(x1, 0.f), acc.y);
+#endif
             }
         };
         // double-buffered loads: load n + 1 is in flight while load n is consumed
