@@ -251,8 +251,11 @@ sa_status sa_sparse_attn(const sa_attn_in* in, const int32_t* idx, int32_t k, vo
  *   the same keys, so a group's keys are loaded once; every query's scores,
  *   selection and attention are its own, whatever its group.
  * Requires in->n_k == n_k of attn, q_pos0 + n_q <= n_k.
- * Host synchronisation: FLAT mode above the table size reads one counter per
- * chunk back to the host (the miss count, as the pages do in prefill).
+ * No host synchronisation and no allocation in any mode: the rows whose
+ * candidate list missed are queued on the device and re-selected from their
+ * whole rows by kernels sized for the chunk's worst case that skip the rows
+ * past the queue's length, so the call is stream-ordered throughout and can
+ * be captured in a CUDA graph.
  */
 sa_status sa_prefill(const sa_indexer_in* in, const sa_attn_in* attn, const sa_prefill_opts* opts,
                      int32_t* idx_out, void* out, float* lse, void* ws, size_t ws_bytes,

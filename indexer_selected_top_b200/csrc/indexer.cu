@@ -185,10 +185,12 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   // ---------------- work unit (identical in every role) ----------------
   int q0 = 0, nq = 0, seq = 0, tile0 = 0, ntiles = 0, geff = 1, njobs = 0, seq_len = a.n_k;
   int n_ub = 0;                    // grouped: the group's union blocks
+  const int n_rows = (a.row_count != nullptr) ? min(a.n_q, *a.row_count - a.row_base) : a.n_q;
   if constexpr (MODE == IDX_PREFILL) {
     const int unit = gridDim.x - 1 - blockIdx.x;            // heaviest (latest rows) first
     q0 = unit * C::NQ;
-    nq = min(C::NQ, a.n_q - q0);
+    nq = min(C::NQ, n_rows - q0);
+    if (nq <= 0) return;                                    // past the rows flagged on the device (uniform)
     geff = (nq + C::QS - 1) / C::QS;
     const int lim = min(vis_limit(q0 + nq - 1, a), a.n_k - 1);
     ntiles = (lim < 0) ? 0 : (lim / 128 + 1);
@@ -229,7 +231,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   for (int i = threadIdx.x; i < C::NQ * H; i += blockDim.x) {
     const int ql = i / H, h = i % H;
     float v = 0.f;
-    int qrow = (ql < nq) ? q0 + ql : -1;
+    int qrow = (ql < nq) ? (a.q_rows != nullptr ? a.q_rows[q0 + ql] : q0 + ql) : -1;
     if constexpr (MODE == IDX_GROUPED) {
       qrow = a.perm[q0 + ql];
       if (qrow >= a.n_q) qrow = -1;
@@ -291,9 +293,14 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       prefetch_tmap(&qmap);
       prefetch_tmap(&kmap);
       if constexpr (MODE == IDX_PREFILL) {
-        mbar_arrive_expect_tx(qfull, geff * C::QS * H * C::ROWB);
-        for (int g = 0; g < geff; ++g)
-          tma_load_2d(sQ + g * C::QS * H * C::ROWB, &qmap, qfull, 0, (q0 + g * C::QS) * H);
+        if (a.q_rows != nullptr) {           // listed rows: one box of H rows per query (rows past nq stay unset)
+          mbar_arrive_expect_tx(qfull, nq * H * C::ROWB);
+          for (int ql = 0; ql < nq; ++ql) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, a.q_rows[q0 + ql] * H);
+        } else {
+          mbar_arrive_expect_tx(qfull, geff * C::QS * H * C::ROWB);
+          for (int g = 0; g < geff; ++g)
+            tma_load_2d(sQ + g * C::QS * H * C::ROWB, &qmap, qfull, 0, (q0 + g * C::QS) * H);
+        }
       } else if constexpr (MODE == IDX_GROUPED) {
         int nv = 0;
         for (int ql = 0; ql < C::NQ; ++ql) nv += sQt[ql] >= 0;
@@ -684,7 +691,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         } else {
           t = q0 + ql;
         }
-        if (t >= a.n_q) continue;
+        if (t >= n_rows) continue;
         bool vis;
         if constexpr (MODE == IDX_DECODE)
           vis = kvalid;
@@ -737,7 +744,7 @@ static cudaError_t launch_t(const void* q, const void* k, int q_rows, long long 
   CUtensorMap qm, km;
   const CUtensorMapDataType dt = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const CUtensorMapSwizzle sw = (C::ROWB == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  const uint32_t qbox = (MODE == IDX_PREFILL) ? C::QS * H : H;
+  const uint32_t qbox = (MODE == IDX_PREFILL && a.q_rows == nullptr) ? C::QS * H : H;
   const uint32_t kbox = (MODE == IDX_GATHER || MODE == IDX_GROUPED) ? 64 : 128;
   if (!make_tmap_2d(&qm, q, dt, D, (uint64_t)q_rows * H, C::ROWB, D, qbox, sw)) return cudaErrorInvalidValue;
   if (!make_tmap_2d(&km, k, dt, D, (uint64_t)k_rows, C::ROWB, D, kbox, sw)) return cudaErrorInvalidValue;

@@ -88,7 +88,10 @@ static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 constexpr long long kWaitBudget = 4000000000ll;     // ~2 s of SM clock
 constexpr long long kHookBudget = 20000000ll;       // ~10 ms: the stall hook
-constexpr int kDecodeSplitKeys = 256;               // keys per decode attention split
+#ifndef SA_DECODE_SPLIT_KEYS
+#define SA_DECODE_SPLIT_KEYS 256
+#endif
+constexpr int kDecodeSplitKeys = SA_DECODE_SPLIT_KEYS;   // keys per decode attention split
 constexpr int kDecodeTilesPerCta = 64;              // 8192 keys per decode indexer CTA
 constexpr int kDecodeSamples = 8192;                // sampled scores per sequence for the decode threshold
 constexpr int kMaxBlocks = 16384;                   // two-stage: blocks per sequence
@@ -108,7 +111,7 @@ struct PrefillPlan {
   size_t off_sig;                                   // two-stage: grouping signatures
   int n_groups, ucap;
   size_t off_ks, off_kss, off_stab, off_theta, off_cnt, off_list, off_miss, off_rows, off_count, off_pos;
-  size_t off_fq, off_fqs, off_fw, off_ftab;
+  size_t off_ftab;
 };
 
 constexpr int kStreamSamples = 16384;      // sampled keys per row for the threshold (at most)
@@ -138,7 +141,6 @@ static bool plan_prefill(const sa_indexer_in* in, const sa_prefill_opts* o, Pref
     while (R > 1 && ((long long)R * p->n_s * 4ll > (2ll << 30) || (long long)R * p->cap * 8ll > (2ll << 30)))
       R = (R + 1) / 2;
     p->fb = (int)std::max<long long>(1, std::min<long long>(R, (1ll << 30) / ((long long)in->n_k * 4)));
-    const size_t qrow = (size_t)in->n_heads * in->d_idx * (in->dtype == SA_FP8_E4M3 ? 1 : 2);
     p->off_ks = off;
     off += align256((size_t)p->n_s * in->d_idx * (in->dtype == SA_FP8_E4M3 ? 1 : 2));
     p->off_kss = off;
@@ -159,12 +161,6 @@ static bool plan_prefill(const sa_indexer_in* in, const sa_prefill_opts* o, Pref
     off += 256;
     p->off_pos = off;
     off += align256((size_t)R * 4);
-    p->off_fq = off;
-    off += align256((size_t)p->fb * qrow);
-    p->off_fqs = off;
-    off += align256((size_t)p->fb * in->n_heads * 4);
-    p->off_fw = off;
-    off += align256((size_t)p->fb * in->n_heads * 4);
     p->off_ftab = off;
     off += align256((size_t)p->fb * in->n_k * 4);
   } else if (o->mode == SA_MODE_FLAT) {
@@ -290,14 +286,14 @@ struct StageMarks {
 
 // Streaming FLAT selection of one chunk (rows ci->q_pos0 ...): sampled
 // thresholds, the appending scan, the exact list select, then the whole-row
-// fallback for the rows whose list missed (one counter read on the host).
+// fallback for the rows whose list missed (queued on the device; no host
+// synchronisation).
 static sa_status stream_select_chunk(const sa_indexer_in* in, const sa_indexer_in* ci, const sa_prefill_opts* o,
                                      const PrefillPlan& p, char* w, bool first, int32_t* idx, uint32_t* status,
                                      cudaStream_t stream) {
   const int R = ci->n_q;
   const size_t esz = esize(in->dtype);
   const int krow = in->d_idx * (int)esz;
-  const int qrow = in->n_heads * in->d_idx * (int)esz;
   uint8_t* ks = reinterpret_cast<uint8_t*>(w + p.off_ks);
   float* kss = reinterpret_cast<float*>(w + p.off_kss);
   float* stab = reinterpret_cast<float*>(w + p.off_stab);
@@ -344,39 +340,30 @@ static sa_status stream_select_chunk(const sa_indexer_in* in, const sa_indexer_i
     e = launch_indexer(IDX_PREFILL, in->n_heads, in->d_idx, in->dtype, ci->q, in->k, R, in->n_k, a, stream);
     if (e != cudaSuccess) return cuda_status(e);
   }
-  // 4. exact select of each list; flag the misses
+  // 4. exact select of each list; flag the misses and queue them (ascending)
   e = launch_select_cand(list, cnt, theta, R, p.cap, ci->q_pos0, in->n_k, o->k, idx, miss, status, stream);
   if (e == cudaSuccess) e = launch_compact_rows(miss, R, rows, count, ci->q_pos0, pos, stream);
   if (e != cudaSuccess) return cuda_status(e);
-  int n_miss = 0;
-  if (cudaMemcpyAsync(&n_miss, count, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
-      cudaStreamSynchronize(stream) != cudaSuccess)
-    return SA_ERR_CUDA;
-  // 5. whole-row fallback of the missed rows, in batches
-  uint8_t* fq = reinterpret_cast<uint8_t*>(w + p.off_fq);
-  float* fqs = reinterpret_cast<float*>(w + p.off_fqs);
-  float* fw = reinterpret_cast<float*>(w + p.off_fw);
+  // 5. whole-row fallback of the queued rows, in batches of p.fb sized for
+  // the worst case (every row of the chunk); the kernels read the queue's
+  // length on the device and skip the rows past it, so the host never waits
+  // for the count (the call stays stream-ordered and can be captured)
   float* ftab = reinterpret_cast<float*>(w + p.off_ftab);
-  for (int b0 = 0; b0 < n_miss; b0 += p.fb) {
-    const int nb = std::min(p.fb, n_miss - b0);
-    e = launch_gather_rows(ci->q, fq, rows + b0, nb, qrow, 0, qrow, stream);
-    if (e == cudaSuccess && ci->q_scale)
-      e = launch_gather_rows(ci->q_scale, fqs, rows + b0, nb, in->n_heads * 4, 0, in->n_heads * 4, stream);
-    if (e == cudaSuccess) e = launch_gather_rows(ci->w, fw, rows + b0, nb, in->n_heads * 4, 0, in->n_heads * 4, stream);
-    if (e != cudaSuccess) return cuda_status(e);
+  for (int b0 = 0; b0 < R; b0 += p.fb) {
+    const int nb = std::min(p.fb, R - b0);
     sa_indexer_in fi = *ci;
     fi.n_q = nb;
-    fi.q = fq;
-    fi.q_scale = ci->q_scale ? fqs : nullptr;
-    fi.w = fw;
     IdxArgs a = base_args(&fi, status, o->test_hook);
     a.row_pos = pos + b0;
+    a.q_rows = rows + b0;
+    a.row_count = count;
+    a.row_base = b0;
     a.out = ftab;
     a.ld = in->n_k;
-    e = launch_indexer(IDX_PREFILL, in->n_heads, in->d_idx, in->dtype, fq, in->k, nb, in->n_k, a, stream);
+    e = launch_indexer(IDX_PREFILL, in->n_heads, in->d_idx, in->dtype, ci->q, in->k, R, in->n_k, a, stream);
     if (e == cudaSuccess)
       e = launch_topk_table(ftab, nb, in->n_k, in->n_k, 0, o->k, idx, 0, nullptr, 0, nullptr, stream, pos + b0,
-                            rows + b0);
+                            rows + b0, nullptr, count, b0);
     if (e != cudaSuccess) return cuda_status(e);
   }
   return SA_OK;

@@ -40,6 +40,13 @@ struct IdxArgs {
   // prefill: absolute position of every query row (ascending), overriding
   // q_pos0 + t when non-null
   const int* row_pos;
+  // prefill: query row t of this launch is row q_rows[t] of q (and of w,
+  // q_scale) when non-null; rows t >= *row_count - row_base (a count on the
+  // device) are skipped, so a launch sized for the worst case does only the
+  // rows a previous kernel flagged
+  const int* q_rows;
+  const int* row_count;
+  int row_base;
   // candidate mode (prefill): instead of writing the table, append every
   // visible key with score >= theta[t] to row t's list as the packed key
   // (order-preserving score bits << 32 | ~key); counts may exceed cap
@@ -56,7 +63,7 @@ cudaError_t launch_indexer(int mode, int heads, int d, sa_dtype dt, const void* 
 cudaError_t launch_topk_table(const float* scores, int n_rows, int n_cols, long long ld, int q_pos0, int k,
                               int32_t* idx, int vis_mode, const int* kept, int keep, const int* seq_lens,
                               cudaStream_t st, const int* row_pos = nullptr, const int* out_rows = nullptr,
-                              const int* only_flagged = nullptr);
+                              const int* only_flagged = nullptr, const int* row_count = nullptr, int row_base = 0);
 
 // sel (gathered rows only, nullable): per row keep * 2 words, bit c of the
 // row's bitmap set iff candidate column c was selected

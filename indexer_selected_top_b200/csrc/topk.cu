@@ -127,11 +127,12 @@ __device__ void topk_row(TkShared& sh, const RowView& rv, int k, int32_t* out) {
 __global__ void __launch_bounds__(TK_THREADS, 1)
     topk_table_kernel(const float* scores, int n_rows, int n_cols, long long ld, int q_pos0, int k, int32_t* idx,
                       int vis_mode, const int* kept, int keep, const int* seq_lens, const int* row_pos,
-                      const int* out_rows, const int* only_flagged) {
+                      const int* out_rows, const int* only_flagged, const int* row_count, int row_base) {
   extern __shared__ uint8_t tk_raw[];
   TkShared& sh = *reinterpret_cast<TkShared*>(tk_raw);
   const int row = blockIdx.x;
   if (only_flagged != nullptr && only_flagged[row] == 0) return;   // this row was selected already
+  if (row_count != nullptr && row >= *row_count - row_base) return;  // past the rows flagged on the device
   RowView rv;
   rv.s = scores + (long long)row * ld;
   rv.vis_mode = vis_mode;
@@ -152,13 +153,15 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
 
 cudaError_t launch_topk_table(const float* scores, int n_rows, int n_cols, long long ld, int q_pos0, int k,
                               int32_t* idx, int vis_mode, const int* kept, int keep, const int* seq_lens,
-                              cudaStream_t st, const int* row_pos, const int* out_rows, const int* only_flagged) {
+                              cudaStream_t st, const int* row_pos, const int* out_rows, const int* only_flagged,
+                              const int* row_count, int row_base) {
   if (n_rows <= 0) return cudaSuccess;
   const int smem = (int)sizeof(TkShared);
   cudaError_t e = cudaFuncSetAttribute(topk_table_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   topk_table_kernel<<<n_rows, TK_THREADS, smem, st>>>(scores, n_rows, n_cols, ld, q_pos0, k, idx, vis_mode, kept,
-                                                       keep, seq_lens, row_pos, out_rows, only_flagged);
+                                                       keep, seq_lens, row_pos, out_rows, only_flagged, row_count,
+                                                       row_base);
   return cudaGetLastError();
 }
 

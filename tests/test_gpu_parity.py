@@ -213,6 +213,52 @@ def test_prefill_flat_streaming_forced_fallbacks(sa):
     assert s[3] == wl.T - 512 and s[2] == wl.T - 512, s
 
 
+def test_prefill_flat_streaming_fallback_in_device_batches(sa):
+    # theta = +inf: every row of every chunk is queued for the whole-row
+    # fallback; at 40,000 keys a batch holds 1 GiB / (4 n_k) = 6710 rows, so
+    # each 16,000-row chunk runs three batches gated by the queue's length on
+    # the device. Rows around the batch edges are checked against the oracle.
+    wl = WORKLOADS["prefill_t16k"].with_(T=40000, k=256)
+    rows = sample_rows(wl.T, 40, seed=8, k=256,
+                       extra=(6709, 6710, 13419, 13420, 15999, 16000, 22709, 22710, 32000, 39999))
+    st = sa.new_status("cuda")
+    _check_prefill(sa, wl, 8, rows, k=256, flat_path="stream", chunk_rows=16000, hook=sa.SA_HOOK_THETA_POS_INF,
+                   status=st)
+    s = st.cpu().tolist()
+    assert s[0] == 0 and s[2] == wl.T, s
+
+
+def test_prefill_flat_streaming_replays_as_a_cuda_graph(sa):
+    """The streaming FLAT prefill (sampled thresholds, appending scan, list
+    select, device-queued fallback) makes no host round trip, so it can be
+    captured in a CUDA graph; the replay selects the same key sets and gives
+    the same attention as the eager call."""
+    wl = WORKLOADS["prefill_t16k"].with_(T=20000, k=256)
+    inp = PrefillInputs(wl, "cuda", seed=9)
+    st = sa.new_status("cuda")
+    pre = sa.Prefill(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, wl.k,
+                     flat_path="stream", chunk_rows=8000, status=st)
+    out, lse, idx = pre()
+    torch.cuda.synchronize()
+    ref_idx = np.sort(idx.cpu().numpy(), axis=1)
+    ref_out, ref_lse = out.float().cpu().numpy(), lse.cpu().numpy()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        pre(s)
+    idx.fill_(-7)
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert st.cpu().tolist()[0] == 0
+    assert np.array_equal(np.sort(idx.cpu().numpy(), axis=1), ref_idx)
+    go, gl = out.float().cpu().numpy(), lse.cpu().numpy()
+    for t in range(0, wl.T, 997):
+        check_attention_row(go[t], ref_out[t], gl[t], ref_lse[t], f"replayed row {t}")
+    del g
+
+
 def _two_stage_kept_sets(sa, inp, k_all):
     """Kept blocks of every row, read through the public API: with k = keep *
     64 every visible key of the kept blocks is selected."""
