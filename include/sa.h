@@ -190,6 +190,8 @@ typedef struct {
 #define SA_HOOK_THETA_POS_INF 1   /* every row misses low -> whole-row fallback */
 #define SA_HOOK_THETA_NEG_INF 2   /* every key is a candidate -> overflow path */
 #define SA_HOOK_STALL_WAIT 3      /* a device wait that never completes -> SA_ERR_TIMEOUT */
+#define SA_HOOK_THETA_RUNNING 5    /* every threshold starts at -inf and the streaming scan runs in key phases of
+                                     cap - k keys, so only the running threshold keeps the lists in bounds */
 #define SA_HOOK_ATTN_UNGROUPED 4  /* no query groups: the two-stage stage 2 scores each query's kept blocks on
                                      its own and the prefill attention takes one query at a time, as for a
                                      group whose union of selected keys does not fit the kernel's tables */

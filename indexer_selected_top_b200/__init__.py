@@ -30,7 +30,8 @@ SA_OK, SA_ERR_INVALID_ARGUMENT, SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE_TOO_SMALL, 
 SA_BF16, SA_FP8_E4M3, SA_F32 = 0, 1, 2
 SA_MODE_FLAT, SA_MODE_TWO_STAGE = 0, 1
 SA_OP_INDEX_SCORES, SA_OP_TOPK, SA_OP_SPARSE_ATTN, SA_OP_PREFILL, SA_OP_DECODE = range(5)
-SA_HOOK_NONE, SA_HOOK_THETA_POS_INF, SA_HOOK_THETA_NEG_INF, SA_HOOK_STALL_WAIT, SA_HOOK_ATTN_UNGROUPED = range(5)
+SA_HOOK_NONE, SA_HOOK_THETA_POS_INF, SA_HOOK_THETA_NEG_INF, SA_HOOK_STALL_WAIT, SA_HOOK_ATTN_UNGROUPED, \
+    SA_HOOK_THETA_RUNNING = range(6)
 
 EXPORTS = ("sa_status_string", "sa_index_scores", "sa_topk", "sa_sparse_attn", "sa_prefill", "sa_decode",
            "sa_workspace_size", "sa_sparse_attn_decode_noalloc", "sa_quantize_rows_e4m3",

@@ -193,7 +193,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     if (nq <= 0) return;                                    // past the rows flagged on the device (uniform)
     geff = (nq + C::QS - 1) / C::QS;
     const int lim = min(vis_limit(q0 + nq - 1, a), a.n_k - 1);
-    ntiles = (lim < 0) ? 0 : (lim / 128 + 1);
+    tile0 = a.tile_lo;                                      // the key tiles [tile_lo, min(tile_hi, lim / 128 + 1))
+    ntiles = (lim < 0) ? 0 : max(0, min(lim / 128 + 1, a.tile_hi) - tile0);
     njobs = ntiles * geff;
   } else if constexpr (MODE == IDX_DECODE) {
     seq = blockIdx.y;
@@ -321,7 +322,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         uint8_t* dst = sK + st * C::KBYTES;
         if constexpr (MODE == IDX_PREFILL) {
           mbar_arrive_expect_tx(&kfull[st], C::KBYTES);
-          tma_load_2d(dst, &kmap, &kfull[st], 0, i * 128);
+          tma_load_2d(dst, &kmap, &kfull[st], 0, (tile0 + i) * 128);
         } else if constexpr (MODE == IDX_DECODE) {
           mbar_arrive_expect_tx(&kfull[st], C::KBYTES);
           tma_load_2d(dst, &kmap, &kfull[st], 0, seq * a.n_k + (tile0 + i) * 128);
@@ -469,7 +470,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         k.kvalid = k.s < seq_len;
         k.col = k.s;
       } else {
-        k.s = k.tile * 128 + row;
+        k.s = (tile0 + k.tile) * 128 + row;
         k.kvalid = k.s < a.n_k;
         k.col = k.s;
       }

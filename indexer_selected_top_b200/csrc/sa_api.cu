@@ -117,6 +117,8 @@ struct PrefillPlan {
 constexpr int kStreamSamples = 16384;      // sampled keys per row for the threshold (at most)
 constexpr float kStreamGamma = 2.0f;       // target list length = gamma * k
 constexpr int kTableMaxKeys = 65536;       // FLAT auto: table path up to this many keys
+constexpr int kStreamPhases = 4;           // streaming scan: key phases (running threshold between them) ...
+constexpr int kStreamPhaseTilesMin = 2048; // ... of at least this many 128-key tiles
 constexpr int kUnionMaxKeys = 1 << 20;     // block bitmap of the group union kernel
 
 static bool flat_streams(const sa_indexer_in* in, const sa_prefill_opts* o) {
@@ -264,6 +266,8 @@ static IdxArgs base_args(const sa_indexer_in* in, uint32_t* status, int hook) {
   a.status = status;
   a.budget = hook == SA_HOOK_STALL_WAIT ? kHookBudget : kWaitBudget;
   a.hook = hook;
+  a.tile_lo = 0;
+  a.tile_hi = 1 << 30;
   return a;
 }
 
@@ -329,16 +333,27 @@ static sa_status stream_select_chunk(const sa_indexer_in* in, const sa_indexer_i
   e = launch_theta(stab, R, p.n_s, p.n_s, ci->q_pos0, p.m, in->n_k, o->k, p.cap, kStreamGamma, o->test_hook, theta,
                    stream);
   if (e != cudaSuccess) return cuda_status(e);
-  // 3. the scan appends candidates
+  // 3. the scan appends candidates, in key phases; between phases each list
+  // holding more than k keys is cut to its k best and its threshold raised
+  // to the k-th (a running threshold: later phases list fewer keys)
   if (cudaMemsetAsync(cnt, 0, (size_t)R * 4, stream) != cudaSuccess) return SA_ERR_CUDA;
   {
-    IdxArgs a = base_args(ci, status, o->test_hook);
-    a.theta = theta;
-    a.cand = list;
-    a.cand_cnt = cnt;
-    a.cap = p.cap;
-    e = launch_indexer(IDX_PREFILL, in->n_heads, in->d_idx, in->dtype, ci->q, in->k, R, in->n_k, a, stream);
-    if (e != cudaSuccess) return cuda_status(e);
+    const int n_tiles = (ci->q_pos0 + R - 1) / 128 + 1;            // key tiles the chunk's last row sees
+    int per = (n_tiles + kStreamPhases - 1) / kStreamPhases;
+    per = std::max(per, std::min(n_tiles, kStreamPhaseTilesMin));
+    if (o->test_hook == SA_HOOK_THETA_RUNNING) per = std::max(1, (p.cap - o->k) / 128);
+    for (int lo = 0; lo < n_tiles; lo += per) {
+      IdxArgs a = base_args(ci, status, o->test_hook);
+      a.theta = theta;
+      a.cand = list;
+      a.cand_cnt = cnt;
+      a.cap = p.cap;
+      a.tile_lo = lo;
+      a.tile_hi = std::min(n_tiles, lo + per);
+      e = launch_indexer(IDX_PREFILL, in->n_heads, in->d_idx, in->dtype, ci->q, in->k, R, in->n_k, a, stream);
+      if (e == cudaSuccess && lo + per < n_tiles) e = launch_raise_theta(list, cnt, theta, R, p.cap, o->k, stream);
+      if (e != cudaSuccess) return cuda_status(e);
+    }
   }
   // 4. exact select of each list; flag the misses and queue them (ascending)
   e = launch_select_cand(list, cnt, theta, R, p.cap, ci->q_pos0, in->n_k, o->k, idx, miss, status, stream);

@@ -47,6 +47,8 @@ struct IdxArgs {
   const int* q_rows;
   const int* row_count;
   int row_base;
+  // prefill: only the key tiles [tile_lo, tile_hi) of 128 keys are scored
+  int tile_lo, tile_hi;
   // candidate mode (prefill): instead of writing the table, append every
   // visible key with score >= theta[t] to row t's list as the packed key
   // (order-preserving score bits << 32 | ~key); counts may exceed cap
@@ -82,6 +84,12 @@ cudaError_t launch_select_cand(const unsigned long long* cand, const int* cnt, c
                                cudaStream_t st, int decode = 0, const int* seq_lens = nullptr);
 cudaError_t launch_collect_cand(const float* rows, int batch, long long ld, int n_k, const int* seq_lens,
                                 const float* theta, unsigned long long* cand, int* cnt, int cap, cudaStream_t st);
+// Running threshold between the key phases of the streaming scan: every
+// row whose list holds more than k and at most cap entries keeps exactly its
+// k best packed keys (compacted to the front, count = k), and its threshold
+// rises to the score of the k-th.
+cudaError_t launch_raise_theta(unsigned long long* cand, int* cnt, float* theta, int n_rows, int cap, int k,
+                               cudaStream_t st);
 cudaError_t launch_compact_rows(const int* flags, int n_rows, int* rows, int* count, int q_pos0, int* pos,
                                 cudaStream_t st);
 

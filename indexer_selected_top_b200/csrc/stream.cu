@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
   float th;
   if (hook == SA_HOOK_THETA_POS_INF) {
     th = INFINITY;
-  } else if (hook == SA_HOOK_THETA_NEG_INF || n_vis <= cap) {
+  } else if (hook == SA_HOOK_THETA_NEG_INF || hook == SA_HOOK_THETA_RUNNING || n_vis <= cap) {
     th = -INFINITY;
   } else {
     const int n_vs = decode ? (n_vis + m - 1) / m : min(n_s, p / m + 1);
@@ -189,6 +189,52 @@ cudaError_t launch_collect_cand(const float* rows, int batch, long long ld, int 
   if (batch <= 0) return cudaSuccess;
   const int chunks = (n_k + COLLECT_CHUNK - 1) / COLLECT_CHUNK;
   collect_cand_kernel<<<dim3(chunks, batch), 256, 0, st>>>(rows, ld, n_k, seq_lens, theta, cand, cnt, cap);
+  return cudaGetLastError();
+}
+
+// Running threshold (Latent Sparse Attention appendix F.1, "Selection by
+// threshold": any k listed keys lower-bound the k-th best, so a key below the
+// k-th best listed so far is never selected). One CTA per row: a list of c
+// entries, k < c <= cap, is cut to its k best packed keys, written back to
+// the front of the list, and the row's threshold rises to the score of the
+// k-th. A list that overflowed (c > cap) lost entries and is left alone; its
+// row falls back later.
+__global__ void __launch_bounds__(TK_THREADS, 1)
+    raise_theta_kernel(unsigned long long* __restrict__ cand, int* __restrict__ cnt, float* __restrict__ theta,
+                       int cap, int k) {
+  extern __shared__ uint8_t rt_raw[];
+  TkShared& sh = *reinterpret_cast<TkShared*>(rt_raw);
+  __shared__ unsigned long long kmin;
+  const int t = blockIdx.x, tid = threadIdx.x;
+  const int c = cnt[t];
+  if (c <= k || c > cap) return;
+  unsigned long long* row = cand + (long long)t * cap;
+  for (int j = tid; j < c; j += TK_THREADS) sh.cand[j] = row[j];
+  if (tid == 0) {
+    sh.n_out = 0;
+    kmin = ~0ull;
+  }
+  __syncthreads();
+  smem_select64(sh, c, k, [&](uint64_t key) {
+    row[atomicAdd(&sh.n_out, 1)] = key;
+    atomicMin(&kmin, (unsigned long long)key);
+  });
+  if (tid == 0) {
+    cnt[t] = k;
+    const uint32_t hk = (uint32_t)(kmin >> 32);            // the k-th key's score bits, order-preserving
+    const uint32_t b = (hk & 0x80000000u) ? (hk & 0x7FFFFFFFu) : ~hk;
+    theta[t] = fmaxf(theta[t], __uint_as_float(b));
+  }
+}
+
+cudaError_t launch_raise_theta(unsigned long long* cand, int* cnt, float* theta, int n_rows, int cap, int k,
+                               cudaStream_t st) {
+  if (n_rows <= 0) return cudaSuccess;
+  if (cap > TK_CAP) return cudaErrorNotSupported;
+  const int smem = (int)sizeof(TkShared);
+  cudaError_t e = cudaFuncSetAttribute(raise_theta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  raise_theta_kernel<<<n_rows, TK_THREADS, smem, st>>>(cand, cnt, theta, cap, k);
   return cudaGetLastError();
 }
 

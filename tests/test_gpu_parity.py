@@ -213,6 +213,21 @@ def test_prefill_flat_streaming_forced_fallbacks(sa):
     assert s[3] == wl.T - 512 and s[2] == wl.T - 512, s
 
 
+@pytest.mark.parametrize("T,k,chunk", [(3000, 128, 0), (20000, 256, 7000)])
+def test_prefill_flat_streaming_running_threshold(sa, T, k, chunk):
+    # every threshold starts at -inf and the scan runs in phases of cap - k
+    # keys: without the running threshold every row with more than cap = 4k
+    # visible keys would overflow its list; with it, each list is cut to its
+    # k best between phases, no row overflows or falls back, and the rows
+    # still match the oracle exactly
+    wl = WORKLOADS["prefill_t16k"].with_(T=T, k=k)
+    rows = sample_rows(wl.T, 48, seed=7, k=k, extra=(4 * k - 1, 4 * k, 4 * k + 1))
+    st = sa.new_status("cuda")
+    _check_prefill(sa, wl, 7, rows, k=k, flat_path="stream", chunk_rows=chunk, hook=sa.SA_HOOK_THETA_RUNNING,
+                   status=st)
+    assert st.cpu().tolist() == [0, 0, 0, 0]
+
+
 def test_prefill_flat_streaming_fallback_in_device_batches(sa):
     # theta = +inf: every row of every chunk is queued for the whole-row
     # fallback; at 40,000 keys a batch holds 1 GiB / (4 n_k) = 6710 rows, so
