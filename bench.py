@@ -617,6 +617,55 @@ def prefill_roofline(wl, stages_ms: dict, peaks: dict, fp8_peak: float, traffic_
     return stages, roof
 
 
+def time_lsa_prefill(sa, wl, dev, seed: int, warmup: int, steps: int, flush, peaks):
+    """The LSA flat prefill of `wl` (bucket cache of every cluster block, the
+    index rows of every query, attention over them), timed on the device like
+    time_prefill. Returns a dict for the JSON line (tokens/s, stage times,
+    roofline of the dominant stage, status words)."""
+    import torch
+    from workloads import LsaInputs
+    inp = LsaInputs(wl, dev, seed=seed)
+    Q, K, V = inp.attention_operands()
+    prm = sa.lsa_params(n_pool=wl.n_pool, n_cluster=wl.n_cluster, n_buckets=wl.n_buckets,
+                        max_bucket_keys=wl.max_bucket_keys)
+    timer = sa.StageTimer(sa.LsaPrefill.STAGES)
+    run = sa.LsaPrefill(inp.k_idx, inp.q_idx, Q, K, V, prm, wl.p, wl.k, wl.n_sink, wl.n_window, timer=timer)
+    for _ in range(warmup):
+        flush.fill_(1)
+        run()
+    torch.cuda.synchronize()
+    tot, stage_ms = 0.0, {n: 0.0 for n in timer.names}
+    for _ in range(steps):
+        flush.fill_(1)
+        run()
+        torch.cuda.synchronize()
+        if run.stage_status[:, 0].any():
+            raise RuntimeError(f"LSA prefill status {run.stage_status.cpu().tolist()}")
+        for n, v in timer.ms().items():
+            stage_ms[n] += v
+        tot += timer.total_ms()
+    work = lsa_work(wl)
+    pairs = int((run.J >= 0).sum().item())
+    avg = {n: v / steps for n, v in stage_ms.items()}
+    stages = {n: {"ms": round(v, 4)} for n, v in avg.items()}
+    stages["search"].update({"bound": "hbm", "achieved": round(2 * work["score_bytes"] / (avg["search"] * 1e-3) / 1e9,
+                                                                2), "peak": peaks["hbm_gbs"], "unit": "GB/s"})
+    stages["attention"].update({"bound": "tensor", "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                "achieved": round(4.0 * wl.Hq * wl.dh * pairs / (avg["attention"] * 1e-3) / 1e12, 2)})
+    for v in stages.values():
+        if "achieved" in v:
+            v["frac"] = round(v["achieved"] / v["peak"], 4)
+    dom = max((n for n in stages if "achieved" in stages[n]), key=lambda n: stages[n]["ms"])
+    roof = dict(stages[dom])
+    roof.pop("ms")
+    roof.update({"kernel": dom, "traffic": None})
+    ms = tot / steps
+    return {"tokens_per_s": round(wl.T / (ms * 1e-3), 1), "ms_per_step": round(ms, 4), "T": wl.T, "p": wl.p,
+            "k": wl.k, "n_sink": wl.n_sink, "n_window": wl.n_window, "warmup": warmup, "steps": steps,
+            "attention": "tensor-core local + long-range passes" if run.attn.supported else "per-query",
+            "stages": stages, "roofline": roof, "status": run.stage_status.cpu().tolist()}
+
+
 def time_prefill(sa, wl, dev, seed: int, warmup: int, steps: int, flush, mode=None):
     """A prepared sa_prefill over one seeded input of `wl`, timed on the
     device (CUDA events, L2 flushed before every step outside the events).
@@ -873,6 +922,13 @@ def run_native(args, rank, world, local_rank):
                 "status": st}
             del pc, ci
             torch.cuda.empty_cache()
+        # the LSA flat semantic search of the same length (clustering, bucket search, attention)
+        from workloads import LSA_WORKLOADS
+        lsa_line = time_lsa_prefill(sa, LSA_WORKLOADS["lsa_t64k"], dev, seed, 3, 5, flush, peaks)
+        lsa_line["tokens_per_s"] = round(weak_scaling_value(world, 1, lsa_line["T"],
+                                                            reduce_max([lsa_line["ms_per_step"]], device=dev)[0]), 1)
+        configs["lsa_t64k"] = lsa_line
+        torch.cuda.empty_cache()
 
     line = {
         "metric": METRIC,

@@ -75,28 +75,72 @@ def check_attention_row(o_gpu, o_ref, lse_gpu=None, lse_ref=None, where=""):
 LSA_TIE = 1e-5
 
 
-def lsa_row_tied(qn, pos, cent, n_blocks, n_cluster, m, p):
-    """True when two of the query's best p + 1 bucket scores (oracle, fp64)
-    lie within LSA_TIE: the only case in which its row may differ."""
-    from oracle import lsa
-    n_vis = min(n_blocks, pos // n_cluster) * m
-    if n_vis < 2:
-        return False
-    s = np.sort(lsa.bucket_scores(qn, cent, n_vis))[::-1][:p + 1]
-    return bool((np.diff(-s) < LSA_TIE).any())
+def _bucket_end(b, off, m, n_cluster):
+    c, r = divmod(b, m)
+    return (c + 1) * n_cluster if r == m - 1 else int(off[b + 1])
 
 
-def check_lsa_row(got, want, qn, pos, cent, n_blocks, n_cluster, m, p, n_sink, n_window, where=""):
-    """Sinks and window exact; the rest equal to the oracle's row unless a
-    score tie allows another order (then: distinct keys of earlier blocks).
+def check_lsa_row(got, want, qn, pos, cache, n_blocks, n_cluster, m, p, n_sink, n_window, where=""):
+    """An LSA index row against the oracle's. Sinks and window must be exact.
+    The long-range part must equal the oracle's, or else differ only by the
+    order of buckets whose fp64 scores lie within LSA_TIE (the device ranks by
+    fp32 tensor-core sums): the device's bucket sequence is recovered from its
+    keys, and then (a) every bucket's keys come as one run, in list order,
+    skipping the keys the sinks or the window hold, all of them except in the
+    last bucket when the row is full; (b) consecutive buckets are in score
+    order up to LSA_TIE; (c) every bucket used could be among the top p (its
+    score at least the p-th best minus LSA_TIE); (d) no bucket scoring more
+    than LSA_TIE above the last one used, with a key to give, was skipped, and
+    a row with room left used every bucket above the p-th best plus LSA_TIE.
     Returns True when the row needed the tie exception."""
+    from oracle import lsa
+    cent, off, keys = cache
     got = np.asarray(got)
     head = min(n_sink, pos + 1) + max(0, pos - max(n_sink, pos - n_window + 1) + 1)
     assert np.array_equal(got[:head], want[:head]), f"{where}: sinks / window"
     if np.array_equal(got, want):
         return False
-    assert lsa_row_tied(qn, pos, cent, n_blocks, n_cluster, m, p), f"{where}: differs without a score tie"
+    k = len(got) - n_sink - n_window
+    w_lo = max(n_sink, pos - n_window + 1)
     far = got[head:]
-    far = far[far >= 0]
-    assert len(set(far.tolist())) == len(far) and (far < (pos // n_cluster) * n_cluster).all(), where
+    assert (far[(far >= 0).sum():] == -1).all(), f"{where}: -1 not at the tail"
+    far = far[far >= 0].tolist()
+    n_vis = min(n_blocks, pos // n_cluster) * m
+    s = lsa.bucket_scores(qn, cent, n_vis)
+    order = np.lexsort((np.arange(n_vis), -s))
+    theta_p = s[order[min(p, n_vis) - 1]] if n_vis else np.inf
+    uncovered = {}
+    def free_keys(b):
+        if b not in uncovered:
+            lst = keys[off[b]:_bucket_end(b, off, m, n_cluster)]
+            uncovered[b] = [int(x) for x in lst if not (int(x) < n_sink or int(x) >= w_lo)]
+        return uncovered[b]
+    key2b = {}
+    for c in sorted({x // n_cluster for x in far}):
+        assert c < min(n_blocks, pos // n_cluster), f"{where}: key of an invisible block"
+        for b in range(c * m, c * m + m):
+            for x in keys[off[b]:_bucket_end(b, off, m, n_cluster)]:
+                key2b[int(x)] = b
+    seq, i = [], 0
+    while i < len(far):
+        b = key2b[far[i]]
+        assert b not in seq, f"{where}: bucket {b} in two runs"
+        run = free_keys(b)
+        n = min(len(run), len(far) - i)
+        assert far[i:i + n] == run[:n], f"{where}: bucket {b} keys out of list order"
+        last_partial = n < len(run)
+        i += n
+        assert not last_partial or i == k, f"{where}: bucket {b} cut short before the row is full"
+        seq.append(b)
+    assert len(far) == len(set(far)), f"{where}: duplicate keys"
+    for a, b in zip(seq, seq[1:]):
+        assert s[a] >= s[b] - LSA_TIE, f"{where}: bucket {b} ({s[b]:.7f}) after {a} ({s[a]:.7f})"
+    for b in seq:
+        assert s[b] >= theta_p - LSA_TIE, f"{where}: bucket {b} is not among the top {p}"
+    used = set(seq)
+    floor = s[seq[-1]] + LSA_TIE if seq else -np.inf
+    if len(far) < k:
+        floor = min(floor, theta_p + LSA_TIE)
+    skipped = [int(b) for b in order[:p] if b not in used and s[b] > floor and free_keys(int(b))]
+    assert not skipped, f"{where}: better buckets {skipped[:4]} skipped"
     return True

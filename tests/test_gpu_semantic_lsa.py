@@ -138,7 +138,7 @@ def _check_rows(J, rows, pos0, q_host, ref_cache, n_blocks, wl, p, k, n_sink, n_
         pos = pos0 + r
         want = lsa.search_row(qv, pos, cent, off, keys, n_blocks, wl.n_cluster, wl.n_buckets, p, k, n_sink,
                               n_window)
-        exceptions += check_lsa_row(J[r], want, qv, pos, cent, n_blocks, wl.n_cluster, wl.n_buckets, p, n_sink,
+        exceptions += check_lsa_row(J[r], want, qv, pos, ref_cache, n_blocks, wl.n_cluster, wl.n_buckets, p, n_sink,
                                     n_window, f"row {pos}")
     assert exceptions <= 0.05 * len(rows), f"{exceptions} of {len(rows)} rows differ at score ties"
     return exceptions
@@ -249,7 +249,7 @@ def _check_decode_rows(J, q, lens, refs, nbt, wl, p, k):
         nb = int(nbt[b])
         want = lsa.search_row(qn[b], L - 1, cent, off, keys, nb, wl.n_cluster, wl.n_buckets, p, k, wl.n_sink,
                               wl.n_window)
-        check_lsa_row(J[b], want, qn[b], L - 1, cent, nb, wl.n_cluster, wl.n_buckets, p, wl.n_sink, wl.n_window,
+        check_lsa_row(J[b], want, qn[b], L - 1, refs[b], nb, wl.n_cluster, wl.n_buckets, p, wl.n_sink, wl.n_window,
                       f"sequence {b}")
 
 
@@ -351,7 +351,7 @@ def test_threshold_regime_at_512k_tokens(sa):
     for j, (r, qv) in enumerate(zip(rows, qn)):
         want = lsa.search_row(qv, r, cent, off, keys, nb, wl.n_cluster, wl.n_buckets, wl.p, wl.k, wl.n_sink,
                               wl.n_window)
-        exceptions += check_lsa_row(Jr[j], want, qv, r, cent, nb, wl.n_cluster, wl.n_buckets, wl.p, wl.n_sink,
+        exceptions += check_lsa_row(Jr[j], want, qv, r, ref, nb, wl.n_cluster, wl.n_buckets, wl.p, wl.n_sink,
                                     wl.n_window, f"row {r}")
     # each exception was already checked to sit at a score tie; they stay rare
     assert exceptions <= max(2, len(rows) // 10)
