@@ -118,10 +118,7 @@ def _isnum(s):
 # + dram__bytes_write.sum), captured on the two-stage workload at T_cap rows
 # and scaled to the run by the number of candidate keys scored (the candidate
 # scores are most of the traffic). An entry is removed when its kernel changes.
-MEASURED_DRAM = {
-    # the stage-2 indexer_kernel<64, 128, 1, 3> (grouped mode), two-stage workload at T = 16384
-    "stage2_indexer": {"bytes": 147.324672e6 + 184.366592e6, "T_cap": 16384},
-}
+MEASURED_DRAM = {}
 
 
 def measured_traffic(kernel, wl):
@@ -725,6 +722,8 @@ def run_native(args, rank, world, local_rank):
     if args.T:
         wl = wl.with_(T=args.T)
     wd = WORKLOADS["decode_b64_l128k"]
+    if args.decode_L:
+        wd = wd.with_(L=args.decode_L)
     seed = rank_seed(args.seed, rank)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -839,6 +838,7 @@ def run_native(args, rank, world, local_rank):
         decode["graph_us_per_step"] = round(gus, 1)
         decode["graph_us_per_token"] = round(gus / wd.batch, 3)
         del g
+        decode["gather_gbs"] = round(dw["attn_bytes"] / (davg["attention"] * 1e-3) / 1e9, 1)
 
     # ---------------- end to end through host buffers ----------------
     e2e = None
@@ -964,6 +964,7 @@ def main():
     ap.add_argument("--workload", default="two_stage_t64k",
                     help="two_stage_t64k (headline), another prefill workload, or lsa_t64k / lsa_t8k")
     ap.add_argument("--T", type=int, default=0, help="override the prefill length (profiling runs)")
+    ap.add_argument("--decode-L", type=int, default=0, help="override the decode cache length (profiling runs)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--headline-only", action="store_true",
