@@ -118,7 +118,10 @@ def _isnum(s):
 # + dram__bytes_write.sum), captured on the two-stage workload at T_cap rows
 # and scaled to the run by the number of candidate keys scored (the candidate
 # scores are most of the traffic). An entry is removed when its kernel changes.
-MEASURED_DRAM = {}
+MEASURED_DRAM = {
+    # the stage-2 indexer_kernel<64, 128, 1, 3> (grouped mode), two-stage workload at T = 16384
+    "stage2_indexer": {"bytes": 147.400448e6 + 185.557248e6, "T_cap": 16384},
+}
 
 
 def measured_traffic(kernel, wl):
@@ -839,6 +842,32 @@ def run_native(args, rank, world, local_rank):
         decode["graph_us_per_token"] = round(gus / wd.batch, 3)
         del g
         decode["gather_gbs"] = round(dw["attn_bytes"] / (davg["attention"] * 1e-3) / 1e9, 1)
+        # graphs per context-length bucket: every sequence at the bucket's
+        # length, the narrowest bucket's graph replayed after the L2 flush
+        graphs = sa.DecodeGraphs(dec, wd.L)
+        saved = dinp.seq_lens.clone()
+        per_bucket = {}
+        for b in graphs.buckets:
+            if b < 16384:
+                continue
+            dinp.seq_lens.fill_(b)
+            for _ in range(args.warmup):
+                flush.fill_(1)
+                graphs.replay(b)
+            bt = 0.0
+            for _ in range(K):
+                flush.fill_(1)
+                a, e_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                graphs.replay(b)
+                e_.record()
+                e_.synchronize()
+                bt += a.elapsed_time(e_)
+            check_status()
+            per_bucket[str(b)] = round(reduce_max([bt / K * 1e3], device=dev)[0], 1)
+        dinp.seq_lens.copy_(saved)
+        decode["graph_us_per_bucket"] = per_bucket
+        del graphs
 
     # ---------------- end to end through host buffers ----------------
     e2e = None

@@ -182,6 +182,11 @@ typedef struct {
   int32_t test_hook;
   cudaEvent_t* stage_events;  /* host array, nullable (see above) */
   int32_t n_stage_events;
+  int32_t max_len;       /* 0, or the longest context this call serves (<= n_k): the kernels' grids cover
+                            max_len keys per sequence instead of the cache's n_k, so a CUDA graph captured
+                            for a context-length bucket does only that bucket's work; a sequence longer
+                            than max_len sets status->error = SA_ERR_INVALID_ARGUMENT and is read up to
+                            max_len only */
 } sa_decode_opts;
 
 /* test hooks: force the threshold of the streaming selector, a stalled wait,

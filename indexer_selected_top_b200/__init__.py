@@ -67,7 +67,7 @@ FLAT_PATHS = {"auto": SA_FLAT_AUTO, "table": SA_FLAT_TABLE, "stream": SA_FLAT_ST
 
 class DecodeOpts(ctypes.Structure):
     _fields_ = [("k", ctypes.c_int32), ("status", ctypes.c_void_p), ("test_hook", ctypes.c_int32),
-                ("stage_events", ctypes.c_void_p), ("n_stage_events", ctypes.c_int32)]
+                ("stage_events", ctypes.c_void_p), ("n_stage_events", ctypes.c_int32), ("max_len", ctypes.c_int32)]
 
 
 class LsaParams(ctypes.Structure):
@@ -324,12 +324,14 @@ class Decode:
     """A prepared sa_decode call (one decode step of a batch of sequences)."""
 
     def __init__(self, q, q_scale, k, k_scale, w, Q, K, V, seq_lens, k_top: int, softmax_scale=0.0,
-                 want_idx=True, want_lse=True, status=None, test_hook=0, timer: "StageTimer" = None):
+                 want_idx=True, want_lse=True, status=None, test_hook=0, timer: "StageTimer" = None,
+                 max_len: int = 0):
+        """max_len: 0, or the longest context the calls serve (sa_decode_opts.max_len)."""
         self.ind = indexer_in(q, q_scale, k, k_scale, w, 0, seq_lens)
         self.att = attn_in(Q, K, V, softmax_scale)
         self.opts = DecodeOpts(k=k_top, status=_ptr(status), test_hook=test_hook,
                                stage_events=timer.ptr if timer else None,
-                               n_stage_events=len(timer.events) if timer else 0)
+                               n_stage_events=len(timer.events) if timer else 0, max_len=max_len)
         self.timer = timer
         self.nws = workspace_size(SA_OP_DECODE, self.ind, self.att, self.opts)
         self.ws = _workspace(self.nws, Q.device)
@@ -344,13 +346,16 @@ class Decode:
                               _stream(stream)), "sa_decode")
         return self.out, self.lse, self.idx
 
-    def graph(self) -> "torch.cuda.CUDAGraph":
+    def graph(self, max_len: int = None) -> "torch.cuda.CUDAGraph":
         """This decode step captured as a CUDA graph. The step launches no
         host synchronisation and no allocation, so every replay reruns it on the
         same buffers (write the next token's inputs into them between replays).
+        max_len (default: the call's own) bounds the contexts the graph serves.
         The stage timer, if any, is not recorded by the graph."""
+        ml = self.opts.max_len if max_len is None else max_len
         opts, self.opts = self.opts, DecodeOpts(k=self.opts.k, status=self.opts.status,
-                                                test_hook=self.opts.test_hook, stage_events=None, n_stage_events=0)
+                                                test_hook=self.opts.test_hook, stage_events=None, n_stage_events=0,
+                                                max_len=ml)
         try:
             s = torch.cuda.Stream()
             s.wait_stream(torch.cuda.current_stream())
@@ -363,6 +368,51 @@ class Decode:
         finally:
             self.opts = opts
         return g
+
+
+def context_buckets(capacity: int, smallest: int = 4096):
+    """Context-length bounds of the decode graphs: ceil(1.125 * 2^e) rounded
+    up to whole 128-key tiles for every e whose bound is at least `smallest`
+    and below `capacity`, then `capacity` (the pages capture their decode
+    graphs for context ranges of this form, LSA appendix F.1 "CUDA graphs")."""
+    out, e = [], 0
+    while True:
+        b = -(-(9 << e) // 8)
+        b = -(-b // 128) * 128
+        if b >= capacity:
+            break
+        if b >= smallest:
+            out.append(b)
+        e += 1
+    return out + [capacity]
+
+
+class DecodeGraphs:
+    """One CUDA graph of a prepared Decode per context-length bucket
+    (context_buckets). replay(longest) replays the graph of the narrowest
+    bucket that holds the batch's longest sequence, so a step over short
+    contexts launches grids sized for them. Graphs are captured on first use
+    (after one eager run of that bucket); inputs are read from the Decode's
+    tensors at every replay."""
+
+    def __init__(self, dec: Decode, capacity: int, smallest: int = 4096):
+        self.dec = dec
+        self.buckets = context_buckets(capacity, smallest)
+        self.graphs = {}
+
+    def bucket(self, longest: int) -> int:
+        for b in self.buckets:
+            if longest <= b:
+                return b
+        raise ValueError(f"context {longest} beyond the capacity {self.buckets[-1]}")
+
+    def replay(self, longest: int) -> int:
+        b = self.bucket(longest)
+        g = self.graphs.get(b)
+        if g is None:
+            g = self.graphs[b] = self.dec.graph(max_len=b)
+        g.replay()
+        return b
 
 
 def decode(q, q_scale, k, k_scale, w, Q, K, V, seq_lens, k_top: int, **kw):

@@ -200,7 +200,10 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     seq = blockIdx.y;
     q0 = seq;
     nq = 1;
-    seq_len = a.seq_lens ? min(a.seq_lens[seq], a.n_k) : a.n_k;
+    seq_len = a.seq_lens ? min(a.seq_lens[seq], a.span) : a.span;
+    if (a.seq_lens != nullptr && a.seq_lens[seq] > a.span && blockIdx.x == 0 && threadIdx.x == 0 &&
+        a.status != nullptr)
+      atomicCAS(a.status, 0u, 1u /* SA_ERR_INVALID_ARGUMENT: a sequence longer than the call's max_len */);
     const int total = (seq_len + 127) / 128;
     tile0 = blockIdx.x * a.tiles_per_cta;
     ntiles = max(0, min(a.tiles_per_cta, total - tile0));
@@ -756,7 +759,7 @@ static cudaError_t launch_t(const void* q, const void* k, int q_rows, long long 
   if constexpr (MODE == IDX_PREFILL)
     grid = dim3((a.n_q + C::NQ - 1) / C::NQ);
   else if constexpr (MODE == IDX_DECODE)
-    grid = dim3(((a.n_k + 127) / 128 + a.tiles_per_cta - 1) / a.tiles_per_cta, a.n_q);
+    grid = dim3(((a.span + 127) / 128 + a.tiles_per_cta - 1) / a.tiles_per_cta, a.n_q);
   else if constexpr (MODE == IDX_GROUPED)
     grid = dim3(a.n_groups);
   else

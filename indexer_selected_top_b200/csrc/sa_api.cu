@@ -268,6 +268,7 @@ static IdxArgs base_args(const sa_indexer_in* in, uint32_t* status, int hook) {
   a.hook = hook;
   a.tile_lo = 0;
   a.tile_hi = 1 << 30;
+  a.span = in->n_k;
   return a;
 }
 
@@ -682,6 +683,8 @@ sa_status sa_decode(const sa_indexer_in* in, const sa_attn_in* at, const sa_deco
   if (ws == nullptr || ws_bytes < p.total) return SA_ERR_WORKSPACE_TOO_SMALL;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return SA_ERR_INVALID_ARGUMENT;
   if (o->stage_events != nullptr && o->n_stage_events < SA_DECODE_STAGES + 1) return SA_ERR_INVALID_ARGUMENT;
+  if (o->max_len < 0) return SA_ERR_INVALID_ARGUMENT;
+  const int span = o->max_len > 0 ? std::min(o->max_len, in->n_k) : in->n_k;   // keys per sequence the grids cover
   char* w = static_cast<char*>(ws);
   uint32_t* status = o->status ? reinterpret_cast<uint32_t*>(o->status) : nullptr;
   if (status && cudaMemsetAsync(status, 0, sizeof(sa_device_status), stream) != cudaSuccess) return SA_ERR_CUDA;
@@ -692,6 +695,7 @@ sa_status sa_decode(const sa_indexer_in* in, const sa_attn_in* at, const sa_deco
   a.out = rows;
   a.ld = in->n_k;
   a.tiles_per_cta = kDecodeTilesPerCta;
+  a.span = span;
   sm.mark(0, stream);
   cudaError_t e = launch_indexer(IDX_DECODE, in->n_heads, in->d_idx, in->dtype, in->q, in->k, in->batch,
                                  (long long)in->batch * in->n_k, a, stream);
@@ -706,16 +710,16 @@ sa_status sa_decode(const sa_indexer_in* in, const sa_attn_in* at, const sa_deco
     int* cnt = reinterpret_cast<int*>(w + p.off_cnt);
     auto* list = reinterpret_cast<unsigned long long*>(w + p.off_list);
     int* miss = reinterpret_cast<int*>(w + p.off_miss);
-    e = launch_theta(rows, in->batch, 0, in->n_k, 0, p.m, in->n_k, o->k, p.cap, kStreamGamma, o->test_hook, theta,
+    e = launch_theta(rows, in->batch, 0, in->n_k, 0, p.m, span, o->k, p.cap, kStreamGamma, o->test_hook, theta,
                      stream, 1, in->seq_lens);
     if (e == cudaSuccess && cudaMemsetAsync(cnt, 0, (size_t)in->batch * 4, stream) != cudaSuccess) e = cudaErrorUnknown;
     if (e == cudaSuccess)
-      e = launch_collect_cand(rows, in->batch, in->n_k, in->n_k, in->seq_lens, theta, list, cnt, p.cap, stream);
+      e = launch_collect_cand(rows, in->batch, in->n_k, span, in->seq_lens, theta, list, cnt, p.cap, stream);
     if (e == cudaSuccess)
-      e = launch_select_cand(list, cnt, theta, in->batch, p.cap, 0, in->n_k, o->k, idx, miss, status, stream, 1,
+      e = launch_select_cand(list, cnt, theta, in->batch, p.cap, 0, span, o->k, idx, miss, status, stream, 1,
                              in->seq_lens);
     if (e == cudaSuccess)
-      e = launch_topk_table(rows, in->batch, in->n_k, in->n_k, 0, o->k, idx, 1, nullptr, 0, in->seq_lens, stream,
+      e = launch_topk_table(rows, in->batch, span, in->n_k, 0, o->k, idx, 1, nullptr, 0, in->seq_lens, stream,
                             nullptr, nullptr, miss);
     if (e != cudaSuccess) return cuda_status(e);
   }

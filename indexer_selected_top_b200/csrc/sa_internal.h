@@ -49,6 +49,8 @@ struct IdxArgs {
   int row_base;
   // prefill: only the key tiles [tile_lo, tile_hi) of 128 keys are scored
   int tile_lo, tile_hi;
+  // decode: keys per sequence the grid covers (<= n_k, the cache's row stride)
+  int span;
   // candidate mode (prefill): instead of writing the table, append every
   // visible key with score >= theta[t] to row t's list as the packed key
   // (order-preserving score bits << 32 | ~key); counts may exceed cap

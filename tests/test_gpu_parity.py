@@ -397,6 +397,40 @@ def _check_decode(sa, wl, seed, seqs=None, seq_lens=None, k=None, hook=0, status
         check_attention_row(out[b], o, lse[b], l, f"seq {b}")
 
 
+def test_decode_graphs_per_context_bucket(sa):
+    """Decode graphs captured per context-length bucket (1.125 * 2^e keys):
+    each replay runs the narrowest bucket that holds the batch's longest
+    sequence, over mixed lengths, and matches the oracle; a call whose
+    max_len is shorter than a sequence reports it in the status word."""
+    k = 256
+    wl = WORKLOADS["decode_b64_l128k"].with_(batch=4, L=8192)
+    inp = DecodeInputs(wl, "cuda", seed=12)
+    st = sa.new_status("cuda")
+    dec = sa.Decode(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, inp.seq_lens, k,
+                    status=st)
+    graphs = sa.DecodeGraphs(dec, wl.L, smallest=1024)
+    assert graphs.buckets == [1152, 2304, 4608, 8192]
+    for lens, bucket in (([1000, 2000, 300, 2300], 2304), ([8000, 5000, 100, 7000], 8192),
+                         ([1100, 50, 900, 1152], 1152), ([4608, 4000, 1, 2305], 4608)):
+        inp.seq_lens.copy_(torch.tensor(lens, dtype=torch.int32))
+        assert graphs.replay(max(lens)) == bucket
+        torch.cuda.synchronize()
+        assert st.cpu().tolist()[0] == 0
+        host = inp.to_host()
+        idx, out, lse = dec.idx.cpu().numpy(), dec.out.float().cpu().numpy(), dec.lse.cpu().numpy()
+        ref = oracle.decode_rows(host, range(wl.batch), k, attention=False)
+        for b in range(wl.batch):
+            check_topk_row(idx[b], ref[b]["cand"], ref[b]["scores"], k, f"bucket {bucket} seq {b}")
+            o, l = decode_attention_row(host, b, idx[b])
+            check_attention_row(out[b], o, lse[b], l, f"bucket {bucket} seq {b}")
+    inp.seq_lens.copy_(torch.tensor([1000, 2000, 300, 100], dtype=torch.int32))
+    short = sa.Decode(inp.q_idx, inp.q_scale, inp.k_idx, inp.k_scale, inp.w, inp.Q, inp.K, inp.V, inp.seq_lens, k,
+                      status=st, max_len=1152)
+    short()
+    torch.cuda.synchronize()
+    assert st.cpu().tolist()[0] == sa.SA_ERR_INVALID_ARGUMENT
+
+
 def test_decode_cuda_graph_replay(sa):
     """One decode step captured as a CUDA graph and replayed: the replay
     matches the oracle, and a replay after new inputs were written into the
