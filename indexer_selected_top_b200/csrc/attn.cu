@@ -73,6 +73,8 @@ __global__ void __launch_bounds__(AT_WARPS * 32)
   const __nv_bfloat16* kbase = kc + (batch ? (long long)t * n_k * DH : 0ll);
   const __nv_bfloat16* vbase = vc + (batch ? (long long)t * n_k * DH : 0ll);
   const int32_t* irow = idx + (long long)t * k;
+  pdl_launch_dependents();
+  pdl_wait();                 // decode chain: the index rows come from the previous kernel
 
   // this CTA's slice of the index row, in chunks of 16, staged in shared
   // memory once (invalid entries become -1)
@@ -176,6 +178,7 @@ __global__ void __launch_bounds__(DH) attn_combine_kernel(const float* __restric
                                                           const float* __restrict__ part_lse, int n_q, int splits,
                                                           __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
   const int t = blockIdx.x / HQ, h = blockIdx.x % HQ, col = threadIdx.x;
+  pdl_wait();
   float M = -INFINITY;
   for (int s = 0; s < splits; ++s) M = fmaxf(M, part_lse[((long long)t * splits + s) * HQ + h]);
   float L = 0.f, acc = 0.f;
@@ -193,7 +196,7 @@ __global__ void __launch_bounds__(DH) attn_combine_kernel(const float* __restric
 template <int HQ, int DH>
 static cudaError_t launch_attn_t(const void* q, const void* kc, const void* vc, const int32_t* idx, int n_q, int k,
                                  int n_k, float scale, int batch, void* out, float* lse, float* part_o,
-                                 float* part_lse, int splits, uint32_t* status, cudaStream_t st) {
+                                 float* part_lse, int splits, uint32_t* status, cudaStream_t st, bool pdl) {
   using C = AtCfg<HQ, DH>;
   auto kern = sparse_attn_kernel<HQ, DH>;
   const int smem = C::SMEM + at_slice(k, splits) * 4;
@@ -203,31 +206,30 @@ static cudaError_t launch_attn_t(const void* q, const void* kc, const void* vc, 
   e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   const float scale_log2 = scale * 1.4426950408889634f;
-  kern<<<dim3(n_q, splits), AT_WARPS * 32, smem, st>>>(
-      (const __nv_bfloat16*)q, (const __nv_bfloat16*)kc, (const __nv_bfloat16*)vc, idx, n_q, k, n_k, scale_log2,
-      batch, (__nv_bfloat16*)out, lse, part_o, part_lse, splits, status);
-  e = cudaGetLastError();
+  e = launch_k(kern, dim3(n_q, splits), dim3(AT_WARPS * 32), smem, st, pdl, (const __nv_bfloat16*)q,
+               (const __nv_bfloat16*)kc, (const __nv_bfloat16*)vc, idx, n_q, k, n_k, scale_log2, batch,
+               (__nv_bfloat16*)out, lse, part_o, part_lse, splits, status);
   if (e != cudaSuccess || splits == 1) return e;
-  attn_combine_kernel<HQ, DH><<<n_q * HQ, DH, 0, st>>>(part_o, part_lse, n_q, splits, (__nv_bfloat16*)out, lse);
-  return cudaGetLastError();
+  return launch_k(attn_combine_kernel<HQ, DH>, dim3(n_q * HQ), dim3(DH), 0, st, pdl, (const float*)part_o,
+                  (const float*)part_lse, n_q, splits, (__nv_bfloat16*)out, lse);
 }
 
 cudaError_t launch_attention(const void* q, const void* kc, const void* vc, const int32_t* idx, int n_q, int k,
                              int n_k, int hq, int dh, float scale, int batch, void* out, float* lse, float* part_o,
-                             float* part_lse, int splits, cudaStream_t st, uint32_t* status) {
+                             float* part_lse, int splits, cudaStream_t st, uint32_t* status, bool pdl) {
   if (n_q <= 0) return cudaSuccess;
   if (hq == 16 && dh == 128)
     return launch_attn_t<16, 128>(q, kc, vc, idx, n_q, k, n_k, scale, batch, out, lse, part_o, part_lse, splits,
-                                  status, st);
+                                  status, st, pdl);
   if (hq == 8 && dh == 128)
     return launch_attn_t<8, 128>(q, kc, vc, idx, n_q, k, n_k, scale, batch, out, lse, part_o, part_lse, splits,
-                                 status, st);
+                                 status, st, pdl);
   if (hq == 16 && dh == 64)
     return launch_attn_t<16, 64>(q, kc, vc, idx, n_q, k, n_k, scale, batch, out, lse, part_o, part_lse, splits,
-                                 status, st);
+                                 status, st, pdl);
   if (hq == 8 && dh == 64)
     return launch_attn_t<8, 64>(q, kc, vc, idx, n_q, k, n_k, scale, batch, out, lse, part_o, part_lse, splits,
-                                status, st);
+                                status, st, pdl);
   return cudaErrorNotSupported;
 }
 

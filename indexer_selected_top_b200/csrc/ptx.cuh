@@ -95,6 +95,15 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   }
 }
 
+// ------------------------------------------------ programmatic dependent launch
+// In a kernel launched with programmatic stream serialization, pdl_wait()
+// blocks until the previous kernel in the stream has completed and its memory
+// is visible; pdl_launch_dependents() lets the next such kernel be launched
+// before this one ends (its CTAs then wait in pdl_wait). Both are no-ops in a
+// kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // --------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t x,
                                             int32_t y) {

@@ -710,23 +710,25 @@ sa_status sa_decode(const sa_indexer_in* in, const sa_attn_in* at, const sa_deco
     int* cnt = reinterpret_cast<int*>(w + p.off_cnt);
     auto* list = reinterpret_cast<unsigned long long*>(w + p.off_list);
     int* miss = reinterpret_cast<int*>(w + p.off_miss);
+    // the selection kernels and the attention run as a chain of programmatic
+    // dependent launches: each is launched while its predecessor runs and
+    // waits for it on the device (the threshold kernel also empties the lists)
     e = launch_theta(rows, in->batch, 0, in->n_k, 0, p.m, span, o->k, p.cap, kStreamGamma, o->test_hook, theta,
-                     stream, 1, in->seq_lens);
-    if (e == cudaSuccess && cudaMemsetAsync(cnt, 0, (size_t)in->batch * 4, stream) != cudaSuccess) e = cudaErrorUnknown;
+                     stream, 1, in->seq_lens, cnt, true);
     if (e == cudaSuccess)
-      e = launch_collect_cand(rows, in->batch, in->n_k, span, in->seq_lens, theta, list, cnt, p.cap, stream);
+      e = launch_collect_cand(rows, in->batch, in->n_k, span, in->seq_lens, theta, list, cnt, p.cap, stream, true);
     if (e == cudaSuccess)
       e = launch_select_cand(list, cnt, theta, in->batch, p.cap, 0, span, o->k, idx, miss, status, stream, 1,
-                             in->seq_lens);
+                             in->seq_lens, true);
     if (e == cudaSuccess)
       e = launch_topk_table(rows, in->batch, span, in->n_k, 0, o->k, idx, 1, nullptr, 0, in->seq_lens, stream,
-                            nullptr, nullptr, miss);
+                            nullptr, nullptr, miss, nullptr, 0, true);
     if (e != cudaSuccess) return cuda_status(e);
   }
   sm.mark(2, stream);
   e = launch_attention(at->q, at->k_cache, at->v_cache, idx, in->batch, o->k, at->n_k, at->n_q_heads, at->head_dim,
                        attn_scale(at), in->batch, out, lse, reinterpret_cast<float*>(w + p.off_po),
-                       reinterpret_cast<float*>(w + p.off_pl), p.splits, stream, status);
+                       reinterpret_cast<float*>(w + p.off_pl), p.splits, stream, status, true);
   if (e != cudaSuccess) return cuda_status(e);
   sm.mark(3, stream);
   return sm.ok ? SA_OK : SA_ERR_INVALID_ARGUMENT;

@@ -60,14 +60,35 @@ struct IdxArgs {
   int cap;
 };
 
-// Host launchers (return cudaError_t of the launch).
+// A kernel launch, with programmatic stream serialization when `pdl` is set
+// (the kernel may then be launched before the previous one in the stream
+// ends; it waits for it in pdl_wait()).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// Host launchers (return cudaError_t of the launch). `pdl`: launched as a
+// programmatic dependent of the previous kernel in the stream (decode chain).
 cudaError_t launch_indexer(int mode, int heads, int d, sa_dtype dt, const void* q, const void* k, int q_rows,
                            long long k_rows, const IdxArgs& a, cudaStream_t st);
 
 cudaError_t launch_topk_table(const float* scores, int n_rows, int n_cols, long long ld, int q_pos0, int k,
                               int32_t* idx, int vis_mode, const int* kept, int keep, const int* seq_lens,
                               cudaStream_t st, const int* row_pos = nullptr, const int* out_rows = nullptr,
-                              const int* only_flagged = nullptr, const int* row_count = nullptr, int row_base = 0);
+                              const int* only_flagged = nullptr, const int* row_count = nullptr, int row_base = 0,
+                              bool pdl = false);
 
 // sel (gathered rows only, nullable): per row keep * 2 words, bit c of the
 // row's bitmap set iff candidate column c was selected
@@ -80,12 +101,13 @@ cudaError_t launch_gather_rows(const void* src, void* dst, const int* rows, int 
                                int m_stride, int row_bytes, cudaStream_t st);
 cudaError_t launch_theta(const float* stab, int n_rows, int n_s, long long ld, int q_pos0, int m, int n_k, int k,
                          int cap, float gamma, int hook, float* theta, cudaStream_t st, int decode = 0,
-                         const int* seq_lens = nullptr);
+                         const int* seq_lens = nullptr, int* zero_cnt = nullptr, bool pdl = false);
 cudaError_t launch_select_cand(const unsigned long long* cand, const int* cnt, const float* theta, int n_rows,
                                int cap, int q_pos0, int n_k, int k, int32_t* idx, int* miss_flag, uint32_t* status,
-                               cudaStream_t st, int decode = 0, const int* seq_lens = nullptr);
+                               cudaStream_t st, int decode = 0, const int* seq_lens = nullptr, bool pdl = false);
 cudaError_t launch_collect_cand(const float* rows, int batch, long long ld, int n_k, const int* seq_lens,
-                                const float* theta, unsigned long long* cand, int* cnt, int cap, cudaStream_t st);
+                                const float* theta, unsigned long long* cand, int* cnt, int cap, cudaStream_t st,
+                                bool pdl = false);
 // Running threshold between the key phases of the streaming scan: every
 // row whose list holds more than k and at most cap entries keeps exactly its
 // k best packed keys (compacted to the front, count = k), and its threshold
@@ -107,7 +129,7 @@ cudaError_t launch_pool_blocks(const uint8_t* k, const float* k_scale, int n_blo
 cudaError_t launch_attention(const void* q, const void* kc, const void* vc, const int32_t* idx, int n_q, int k,
                              int n_k, int hq, int dh, float scale, int batch, void* out, float* lse,
                              float* part_o, float* part_lse, int splits, cudaStream_t st,
-                             uint32_t* status = nullptr);
+                             uint32_t* status = nullptr, bool pdl = false);
 
 // grouped prefill attention (group.cu): perm orders the queries so that runs
 // of kGroupQueries share keys (nullptr: query order); n_perm = its length

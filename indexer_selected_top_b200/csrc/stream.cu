@@ -17,6 +17,7 @@
 // score, n_theta = round(gamma * k * n_vs / n_vis). Rows whose visible keys
 // all fit in the list take theta = -inf.
 #include "radix.cuh"
+#include "ptx.cuh"
 #include "sa_internal.h"
 
 namespace sa {
@@ -51,10 +52,14 @@ static __device__ __forceinline__ float key_to_float(uint32_t key) {
 // are every m-th visible score (n_vis = seq_lens[t], or n_k).
 __global__ void __launch_bounds__(TK_THREADS, 1)
     theta_kernel(const float* __restrict__ stab, int n_s, long long ld, int q_pos0, int m, int n_k, int k, int cap,
-                 float gamma, int hook, float* __restrict__ theta, int decode, const int* seq_lens) {
+                 float gamma, int hook, float* __restrict__ theta, int decode, const int* seq_lens,
+                 int* __restrict__ zero_cnt) {
   extern __shared__ uint8_t th_raw[];
   TkShared& sh = *reinterpret_cast<TkShared*>(th_raw);
   const int t = blockIdx.x, tid = threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
+  if (zero_cnt != nullptr && tid == 0) zero_cnt[t] = 0;      // the row's list starts empty
   const int p = decode ? ((seq_lens ? min(seq_lens[t], n_k) : n_k) - 1) : q_pos0 + t;
   const int n_vis = min(n_k, p + 1);
   const int sstride = decode ? m : 1;
@@ -94,14 +99,13 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
 
 cudaError_t launch_theta(const float* stab, int n_rows, int n_s, long long ld, int q_pos0, int m, int n_k, int k,
                          int cap, float gamma, int hook, float* theta, cudaStream_t st, int decode,
-                         const int* seq_lens) {
+                         const int* seq_lens, int* zero_cnt, bool pdl) {
   if (n_rows <= 0) return cudaSuccess;
   const int smem = (int)sizeof(TkShared);
   cudaError_t e = cudaFuncSetAttribute(theta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  theta_kernel<<<n_rows, TK_THREADS, smem, st>>>(stab, n_s, ld, q_pos0, m, n_k, k, cap, gamma, hook, theta, decode,
-                                                 seq_lens);
-  return cudaGetLastError();
+  return launch_k(theta_kernel, dim3(n_rows), dim3(TK_THREADS), smem, st, pdl, stab, n_s, ld, q_pos0, m, n_k, k, cap,
+                  gamma, hook, theta, decode, seq_lens, zero_cnt);
 }
 
 // Exact top-k of each row's candidate list; rows whose list missed (fewer
@@ -114,6 +118,8 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
   extern __shared__ uint8_t sc_raw[];
   TkShared& sh = *reinterpret_cast<TkShared*>(sc_raw);
   const int t = blockIdx.x, tid = threadIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
   const int n_vis = decode ? (seq_lens ? min(seq_lens[t], n_k) : n_k) : min(n_k, q_pos0 + t + 1);
   const int need = min(k, n_vis);
   const int c = cnt[t];
@@ -139,16 +145,15 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
 
 cudaError_t launch_select_cand(const unsigned long long* cand, const int* cnt, const float* theta, int n_rows,
                                int cap, int q_pos0, int n_k, int k, int32_t* idx, int* miss_flag, uint32_t* status,
-                               cudaStream_t st, int decode, const int* seq_lens) {
+                               cudaStream_t st, int decode, const int* seq_lens, bool pdl) {
   (void)theta;
   if (n_rows <= 0) return cudaSuccess;
   if (cap > TK_CAP) return cudaErrorNotSupported;
   const int smem = (int)sizeof(TkShared);
   cudaError_t e = cudaFuncSetAttribute(select_cand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  select_cand_kernel<<<n_rows, TK_THREADS, smem, st>>>(cand, cnt, cap, q_pos0, n_k, k, idx, miss_flag, status,
-                                                       decode, seq_lens);
-  return cudaGetLastError();
+  return launch_k(select_cand_kernel, dim3(n_rows), dim3(TK_THREADS), smem, st, pdl, cand, cnt, cap, q_pos0, n_k, k,
+                  idx, miss_flag, status, decode, seq_lens);
 }
 
 // Decode lists from the written score rows: every visible score >= theta[b]
@@ -165,6 +170,8 @@ __global__ void __launch_bounds__(256)
   __shared__ unsigned long long hits[COLLECT_CHUNK];
   __shared__ int n_hit, base;
   const int b = blockIdx.y;
+  pdl_launch_dependents();
+  pdl_wait();
   const int n_vis = seq_lens ? min(seq_lens[b], n_k) : n_k;
   const float th = theta[b];
   const float* row = rows + (long long)b * ld;
@@ -185,11 +192,12 @@ __global__ void __launch_bounds__(256)
 }
 
 cudaError_t launch_collect_cand(const float* rows, int batch, long long ld, int n_k, const int* seq_lens,
-                                const float* theta, unsigned long long* cand, int* cnt, int cap, cudaStream_t st) {
+                                const float* theta, unsigned long long* cand, int* cnt, int cap, cudaStream_t st,
+                                bool pdl) {
   if (batch <= 0) return cudaSuccess;
   const int chunks = (n_k + COLLECT_CHUNK - 1) / COLLECT_CHUNK;
-  collect_cand_kernel<<<dim3(chunks, batch), 256, 0, st>>>(rows, ld, n_k, seq_lens, theta, cand, cnt, cap);
-  return cudaGetLastError();
+  return launch_k(collect_cand_kernel, dim3(chunks, batch), dim3(256), 0, st, pdl, rows, ld, n_k, seq_lens, theta,
+                  cand, cnt, cap);
 }
 
 // Running threshold (Latent Sparse Attention appendix F.1, "Selection by

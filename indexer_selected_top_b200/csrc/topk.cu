@@ -15,6 +15,7 @@
 // select over the packed 64-bit keys finishes. A bucket of identical scores
 // larger than shared memory is resolved by an ordered scan (lowest indices).
 #include "radix.cuh"
+#include "ptx.cuh"
 #include "sa_internal.h"
 
 namespace sa {
@@ -131,6 +132,8 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
   extern __shared__ uint8_t tk_raw[];
   TkShared& sh = *reinterpret_cast<TkShared*>(tk_raw);
   const int row = blockIdx.x;
+  pdl_launch_dependents();
+  pdl_wait();
   if (only_flagged != nullptr && only_flagged[row] == 0) return;   // this row was selected already
   if (row_count != nullptr && row >= *row_count - row_base) return;  // past the rows flagged on the device
   RowView rv;
@@ -154,15 +157,14 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
 cudaError_t launch_topk_table(const float* scores, int n_rows, int n_cols, long long ld, int q_pos0, int k,
                               int32_t* idx, int vis_mode, const int* kept, int keep, const int* seq_lens,
                               cudaStream_t st, const int* row_pos, const int* out_rows, const int* only_flagged,
-                              const int* row_count, int row_base) {
+                              const int* row_count, int row_base, bool pdl) {
   if (n_rows <= 0) return cudaSuccess;
   const int smem = (int)sizeof(TkShared);
   cudaError_t e = cudaFuncSetAttribute(topk_table_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  topk_table_kernel<<<n_rows, TK_THREADS, smem, st>>>(scores, n_rows, n_cols, ld, q_pos0, k, idx, vis_mode, kept,
-                                                       keep, seq_lens, row_pos, out_rows, only_flagged, row_count,
-                                                       row_base);
-  return cudaGetLastError();
+  return launch_k(topk_table_kernel, dim3(n_rows), dim3(TK_THREADS), smem, st, pdl, scores, n_rows, n_cols, ld,
+                  q_pos0, k, idx, vis_mode, kept, keep, seq_lens, row_pos, out_rows, only_flagged, row_count,
+                  row_base);
 }
 
 // ------------------------------------------------------------ stage-1 keep
