@@ -53,10 +53,13 @@ __global__ void __launch_bounds__(TF_THREADS, SA_TF_MINB)
   const bool gathered = kept != nullptr;
   int n;
   if (gathered) {
-    if (tid < 64) sh.kb[tid] = tid < keep ? kept[(long long)row * keep + tid] : -1;
-    __syncthreads();
-    int nb = 0;
-    while (nb < keep && sh.kb[nb] >= 0) ++nb;
+    // kept lists are -1 padded at the tail: the kept count is one block count
+    int kbv = -1;
+    if (tid < 64) {
+      kbv = tid < keep ? kept[(long long)row * keep + tid] : -1;
+      sh.kb[tid] = kbv;
+    }
+    const int nb = __syncthreads_count(kbv >= 0);
     n = min(n_cols, nb * 64);
   } else {
     n = max(0, min(n_cols, (row_pos ? row_pos[row] : q_pos0 + row) + 1));
@@ -120,7 +123,11 @@ __global__ void __launch_bounds__(TF_THREADS, SA_TF_MINB)
     ork |= sh.redu[1][w];
   }
   int32_t* out = idx + (long long)row * k;
-  auto key_of = [&](int c) { return gathered ? sh.kb[c >> 6] * 64 + (c & 63) : c; };
+  // the thread's TF_PER columns lie in one 64-key block: its first key id
+  // (gathered rows: the block's key base) is looked up once
+  static_assert(64 % TF_PER == 0, "a thread's columns share one kept block");
+  const int key0 = gathered ? (c0 < 64 * 64 ? sh.kb[c0 >> 6] * 64 + (c0 & 63) : 0) : c0;
+  auto key_of = [&](int c) { return key0 + (c - c0); };
   // ordered emission of the positions whose flag is set (block scan over
   // (thread, element)); returns the thread's emitted elements as a bit mask
   auto emit_ordered = [&](auto flag, int base, int limit) -> uint32_t {
