@@ -231,6 +231,32 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     *abort_flag = 0u;
     fence_barrier_init();
   }
+  // prefill and decode: the TMA lane (thread 0) issues the query tile and the
+  // first ring of key tiles right away, so their latency overlaps the rest of
+  // the setup (the weights' global loads, the TMEM allocation)
+  if constexpr (MODE == IDX_PREFILL || MODE == IDX_DECODE) {
+    if (threadIdx.x == 0 && njobs > 0) {
+      prefetch_tmap(&qmap);
+      prefetch_tmap(&kmap);
+      if (MODE == IDX_PREFILL && a.q_rows != nullptr) {   // listed rows: one box of H rows per query
+        mbar_arrive_expect_tx(qfull, nq * H * C::ROWB);
+        for (int ql = 0; ql < nq; ++ql) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, a.q_rows[q0 + ql] * H);
+      } else if (MODE == IDX_PREFILL) {
+        mbar_arrive_expect_tx(qfull, geff * C::QS * H * C::ROWB);
+        for (int g = 0; g < geff; ++g)
+          tma_load_2d(sQ + g * C::QS * H * C::ROWB, &qmap, qfull, 0, (q0 + g * C::QS) * H);
+      } else {
+        mbar_arrive_expect_tx(qfull, nq * H * C::ROWB);
+        for (int ql = 0; ql < nq; ++ql) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, (q0 + ql) * H);
+      }
+      const int n0 = min(ntiles, C::NS);   // the ring starts empty: no wait
+      for (int i = 0; i < n0; ++i) {
+        mbar_arrive_expect_tx(&kfull[i], C::KBYTES);
+        const long long row0 = (MODE == IDX_DECODE) ? (long long)seq * a.n_k : 0ll;
+        tma_load_2d(sK + i * C::KBYTES, &kmap, &kfull[i], 0, (int)(row0 + (tile0 + i) * 128));
+      }
+    }
+  }
   if (warp == 1) tmem_alloc<512>(tmem_slot);
   for (int i = threadIdx.x; i < C::NQ * H; i += blockDim.x) {
     const int ql = i / H, h = i % H;
@@ -294,31 +320,28 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   if (warp == 0) {
     // ======================= TMA producer =======================
     if (lane == 0 && njobs > 0) {
-      prefetch_tmap(&qmap);
-      prefetch_tmap(&kmap);
-      if constexpr (MODE == IDX_PREFILL) {
-        if (a.q_rows != nullptr) {           // listed rows: one box of H rows per query (rows past nq stay unset)
-          mbar_arrive_expect_tx(qfull, nq * H * C::ROWB);
-          for (int ql = 0; ql < nq; ++ql) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, a.q_rows[q0 + ql] * H);
-        } else {
-          mbar_arrive_expect_tx(qfull, geff * C::QS * H * C::ROWB);
-          for (int g = 0; g < geff; ++g)
-            tma_load_2d(sQ + g * C::QS * H * C::ROWB, &qmap, qfull, 0, (q0 + g * C::QS) * H);
-        }
+      if constexpr (MODE == IDX_PREFILL || MODE == IDX_DECODE) {
+        // the query tile and the first key tiles went out during the setup
       } else if constexpr (MODE == IDX_GROUPED) {
+        prefetch_tmap(&qmap);
+        prefetch_tmap(&kmap);
         int nv = 0;
         for (int ql = 0; ql < C::NQ; ++ql) nv += sQt[ql] >= 0;
         mbar_arrive_expect_tx(qfull, nv * H * C::ROWB);
         for (int ql = 0; ql < C::NQ; ++ql)   // absent queries leave their rows unset: their scores are dropped
           if (sQt[ql] >= 0) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, sQt[ql] * H);
       } else {
+        prefetch_tmap(&qmap);
+        prefetch_tmap(&kmap);
         mbar_arrive_expect_tx(qfull, nq * H * C::ROWB);
         for (int ql = 0; ql < nq; ++ql) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, (q0 + ql) * H);
       }
       GatherCursor gc;
       if constexpr (MODE == IDX_GATHER) gc.init(sKept, C::KEEPMAX, 0, nq);
-      int issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
+      // prefill and decode: the setup issued the first min(ntiles, NS) tiles
+      const int early = (MODE == IDX_PREFILL || MODE == IDX_DECODE) ? min(ntiles, C::NS) : 0;
+      int issued = early;
+      for (int i = early; i < ntiles; ++i) {
         const int st = i % C::NS, u = i / C::NS;
         if (!mbar_wait(&kempty[st], (u & 1) ^ 1, wc, 1)) break;
         ++issued;
