@@ -507,6 +507,25 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     };
     float2 wq[QUAD ? C::SCOLS / 32 : 1][4];   // 16x256b path: this thread's weights (halved), per chunk and group
     int wg = -1;                             // the sub-tile / query they belong to
+    // per query of the warp's slice, fixed while the job's queries are: its
+    // output row (-1: none) and its causal limit (the last visible key); the
+    // FP8 modes (one or two queries per warp) keep them in registers, the
+    // bf16 modes (up to 32 queries per warp) recompute them per job
+    constexpr bool HOIST = QUAD;
+    int tq[HOIST ? C::QSW : 1], limq[HOIST ? C::QSW : 1];
+    auto query_row = [&](int g_, int ql_, int qq) {
+      const int qj = slice * C::QSW + qq;    // the query's place among the job's QS
+      int t;
+      if constexpr (MODE == IDX_PREFILL)
+        t = q0 + g_ * C::QS + qj;
+      else if constexpr (MODE == IDX_DECODE)
+        t = seq;
+      else if constexpr (MODE == IDX_GROUPED)
+        t = sQt[g_ * C::QS + qj];
+      else
+        t = q0 + ql_;
+      return (t >= n_rows) ? -1 : t;
+    };
     JobKey nxt = job_key(team);
     for (int j = team; j < njobs; j += C::TEAMS) {
       const JobKey cur = nxt;
@@ -519,6 +538,14 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       tc_fence_after();
 
       float qsum[C::QSW];                      // sum_h w'[h] * ReLU(acc[h]) of this thread's key row, per query
+      if (HOIST && g != wg) {                  // the job's queries changed
+#pragma unroll
+        for (int qq = 0; qq < (HOIST ? C::QSW : 0); ++qq) {
+          const int t = query_row(g, ql, qq);
+          tq[qq] = t;
+          limq[qq] = (MODE == IDX_DECODE || t < 0) ? 0 : vis_limit(t, a);
+        }
+      }
       auto release = [&]() {   // every column of this accumulator is in registers
         tc_fence_before();
         __syncwarp();
@@ -539,7 +566,6 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
               wq[cc][i] = make_float2(2.f * wq[cc][i].x, 2.f * wq[cc][i].y);
 #endif
             }
-          wg = g;
         }
         // w * ReLU(a) = (w / 2) * (a + |a|): a + |a| is exact (2a or +0) and one
         // FADD; the halved weights sit in sW, pairs of heads accumulate with
@@ -698,32 +724,25 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         qsum[qq] = sum;
       }
       }
+      wg = g;
       // outputs
 #pragma unroll
       for (int qq = 0; qq < C::QSW; ++qq) {
-        int t;
+        const int t = HOIST ? tq[HOIST ? qq : 0] : query_row(g, ql, qq);
+        if (t < 0) continue;                   // absent query, or a row past the last
         int gcol = 0;                          // grouped: the query's candidate column of this key
-        const int qj = slice * C::QSW + qq;    // the query's place among the job's QS
-        if constexpr (MODE == IDX_PREFILL) {
-          t = q0 + g * C::QS + qj;
-        } else if constexpr (MODE == IDX_DECODE) {
-          t = seq;
-        } else if constexpr (MODE == IDX_GROUPED) {
-          const int ql = g * C::QS + qj;
-          t = sQt[ql];
-          if (t < 0 || cur.s < 0) continue;    // absent query, or no union block in this half
+        if constexpr (MODE == IDX_GROUPED) {
+          if (cur.s < 0) continue;             // no union block in this half
+          const int ql = g * C::QS + slice * C::QSW + qq;
           const int slot = (int)((sUSlot[col] >> (8 * ql)) & 0xFFu);
           if (slot == 0xFF) continue;          // the query did not keep this block
           gcol = slot * 64 + (row & 63);
-        } else {
-          t = q0 + ql;
         }
-        if (t >= n_rows) continue;
         bool vis;
         if constexpr (MODE == IDX_DECODE)
           vis = kvalid;
         else
-          vis = kvalid && s <= vis_limit(t, a);
+          vis = kvalid && s <= (HOIST ? limq[HOIST ? qq : 0] : vis_limit(t, a));
         const float score = vis ? qsum[qq] * sk : -__int_as_float(0x7f800000);
         if constexpr (MODE == IDX_PREFILL) {
           if (a.cand != nullptr) {
