@@ -108,7 +108,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                    uint32_t* status, long long budget) {
   using L = TcSmem;
   extern __shared__ uint8_t tc_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tc_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sm = smem_align1024(tc_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
   uint64_t* full = bars;
   uint64_t* empty = full + TC_ST;

@@ -121,6 +121,12 @@ struct IdxCfg {
   static_assert(SCOLS % 32 == 0, "epilogue loads 32 columns at a time");
 };
 
+// a compile-time int passed as a value (selects a drain's load range)
+template <int V>
+struct IntC {
+  static constexpr int value = V;
+};
+
 __device__ __forceinline__ int vis_limit(int t, const IdxArgs& a) {
   const int p = a.row_pos ? a.row_pos[t] : a.q_pos0 + t;
   return (a.div == 1) ? (p - a.off) : (p / a.div - a.off);
@@ -161,7 +167,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
                    const IdxArgs a) {
   using C = IdxCfg<H, D, FP8, MODE>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_align1024(smem_raw);
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + C::QBYTES;
   float* sW = reinterpret_cast<float*>(sK + C::NS * C::KBYTES);
@@ -231,29 +237,62 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     *abort_flag = 0u;
     fence_barrier_init();
   }
-  // prefill and decode: the TMA lane (thread 0) issues the query tile and the
-  // first ring of key tiles right away, so their latency overlaps the rest of
-  // the setup (the weights' global loads, the TMEM allocation)
-  if constexpr (MODE == IDX_PREFILL || MODE == IDX_DECODE) {
-    if (threadIdx.x == 0 && njobs > 0) {
-      prefetch_tmap(&qmap);
-      prefetch_tmap(&kmap);
-      if (MODE == IDX_PREFILL && a.q_rows != nullptr) {   // listed rows: one box of H rows per query
-        mbar_arrive_expect_tx(qfull, nq * H * C::ROWB);
-        for (int ql = 0; ql < nq; ++ql) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, a.q_rows[q0 + ql] * H);
-      } else if (MODE == IDX_PREFILL) {
-        mbar_arrive_expect_tx(qfull, geff * C::QS * H * C::ROWB);
-        for (int g = 0; g < geff; ++g)
-          tma_load_2d(sQ + g * C::QS * H * C::ROWB, &qmap, qfull, 0, (q0 + g * C::QS) * H);
-      } else {
-        mbar_arrive_expect_tx(qfull, nq * H * C::ROWB);
-        for (int ql = 0; ql < nq; ++ql) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, (q0 + ql) * H);
+  // the TMA lane (thread 0) issues the query tile and the first ring of key
+  // tiles right away, so their latency overlaps the rest of the setup (the
+  // weights' global loads, the staging of the group's lists, the TMEM
+  // allocation); grouped CTAs read their queries and first union blocks from
+  // global memory for it, by the same rules the staging below applies
+  int early = 0;                   // key tiles issued during the setup (thread 0)
+  if (threadIdx.x == 0) {
+    if constexpr (MODE == IDX_PREFILL || MODE == IDX_DECODE) {
+      if (njobs > 0) {
+        prefetch_tmap(&qmap);
+        prefetch_tmap(&kmap);
+        if (MODE == IDX_PREFILL && a.q_rows != nullptr) {   // listed rows: one box of H rows per query
+          mbar_arrive_expect_tx(qfull, nq * H * C::ROWB);
+          for (int ql = 0; ql < nq; ++ql) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, a.q_rows[q0 + ql] * H);
+        } else if (MODE == IDX_PREFILL) {
+          mbar_arrive_expect_tx(qfull, geff * C::QS * H * C::ROWB);
+          for (int g = 0; g < geff; ++g)
+            tma_load_2d(sQ + g * C::QS * H * C::ROWB, &qmap, qfull, 0, (q0 + g * C::QS) * H);
+        } else {
+          mbar_arrive_expect_tx(qfull, nq * H * C::ROWB);
+          for (int ql = 0; ql < nq; ++ql) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, (q0 + ql) * H);
+        }
+        early = min(ntiles, C::NS);   // the ring starts empty: no wait
+        for (int i = 0; i < early; ++i) {
+          mbar_arrive_expect_tx(&kfull[i], C::KBYTES);
+          const long long row0 = (MODE == IDX_DECODE) ? (long long)seq * a.n_k : 0ll;
+          tma_load_2d(sK + i * C::KBYTES, &kmap, &kfull[i], 0, (int)(row0 + (tile0 + i) * 128));
+        }
       }
-      const int n0 = min(ntiles, C::NS);   // the ring starts empty: no wait
-      for (int i = 0; i < n0; ++i) {
-        mbar_arrive_expect_tx(&kfull[i], C::KBYTES);
-        const long long row0 = (MODE == IDX_DECODE) ? (long long)seq * a.n_k : 0ll;
-        tma_load_2d(sK + i * C::KBYTES, &kmap, &kfull[i], 0, (int)(row0 + (tile0 + i) * 128));
+    } else if constexpr (MODE == IDX_GROUPED) {
+      int qt[C::NQ], nv = 0;
+#pragma unroll
+      for (int ql = 0; ql < C::NQ; ++ql) {
+        const int t = a.perm[q0 + ql];
+        qt[ql] = (t >= 0 && t < a.n_q) ? t : -1;
+        nv += qt[ql] >= 0;
+      }
+      const int nub = a.gb_n[blockIdx.x];
+      const int nt = (nub + 1) / 2;
+      if (nv > 0 && nt > 0) {          // else the CTA has no jobs
+        prefetch_tmap(&qmap);
+        prefetch_tmap(&kmap);
+        mbar_arrive_expect_tx(qfull, nv * H * C::ROWB);
+#pragma unroll
+        for (int ql = 0; ql < C::NQ; ++ql)   // absent queries leave their rows unset: their scores are dropped
+          if (qt[ql] >= 0) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, qt[ql] * H);
+        early = min(nt, C::NS);
+        const int* blk = a.gb_blk + (long long)blockIdx.x * a.gb_cap;
+        for (int i = 0; i < early; ++i) {
+          const int b0 = blk[2 * i];
+          const int b1 = (2 * i + 1 < nub) ? blk[2 * i + 1] : -1;
+          uint8_t* dst = sK + i * C::KBYTES;
+          mbar_arrive_expect_tx(&kfull[i], (b1 >= 0 ? 2 : 1) * 64 * C::ROWB);
+          tma_load_2d(dst, &kmap, &kfull[i], 0, b0 * 64);
+          if (b1 >= 0) tma_load_2d(dst + 64 * C::ROWB, &kmap, &kfull[i], 0, b1 * 64);
+        }
       }
     }
   }
@@ -320,16 +359,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   if (warp == 0) {
     // ======================= TMA producer =======================
     if (lane == 0 && njobs > 0) {
-      if constexpr (MODE == IDX_PREFILL || MODE == IDX_DECODE) {
+      if constexpr (MODE == IDX_PREFILL || MODE == IDX_DECODE || MODE == IDX_GROUPED) {
         // the query tile and the first key tiles went out during the setup
-      } else if constexpr (MODE == IDX_GROUPED) {
-        prefetch_tmap(&qmap);
-        prefetch_tmap(&kmap);
-        int nv = 0;
-        for (int ql = 0; ql < C::NQ; ++ql) nv += sQt[ql] >= 0;
-        mbar_arrive_expect_tx(qfull, nv * H * C::ROWB);
-        for (int ql = 0; ql < C::NQ; ++ql)   // absent queries leave their rows unset: their scores are dropped
-          if (sQt[ql] >= 0) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, sQt[ql] * H);
       } else {
         prefetch_tmap(&qmap);
         prefetch_tmap(&kmap);
@@ -338,9 +369,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       }
       GatherCursor gc;
       if constexpr (MODE == IDX_GATHER) gc.init(sKept, C::KEEPMAX, 0, nq);
-      // prefill and decode: the setup issued the first min(ntiles, NS) tiles
-      const int early = (MODE == IDX_PREFILL || MODE == IDX_DECODE) ? min(ntiles, C::NS) : 0;
-      int issued = early;
+      int issued = early;              // the setup issued tiles [0, early)
       for (int i = early; i < ntiles; ++i) {
         const int st = i % C::NS, u = i / C::NS;
         if (!mbar_wait(&kempty[st], (u & 1) ^ 1, wc, 1)) break;
@@ -508,11 +537,13 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     float2 wq[QUAD ? C::SCOLS / 32 : 1][4];   // 16x256b path: this thread's weights (halved), per chunk and group
     int wg = -1;                             // the sub-tile / query they belong to
     // per query of the warp's slice, fixed while the job's queries are: its
-    // output row (-1: none) and its causal limit (the last visible key); the
-    // FP8 modes (one or two queries per warp) keep them in registers, the
-    // bf16 modes (up to 32 queries per warp) recompute them per job
+    // causal limit (the last visible key) and, grouped, its output row (-1:
+    // none). The FP8 modes (one or two queries per warp) keep them in
+    // registers; the bf16 modes (up to 32 queries per warp) recompute them per
+    // job, as every mode but grouped does the row (a few integer operations)
     constexpr bool HOIST = QUAD;
-    int tq[HOIST ? C::QSW : 1], limq[HOIST ? C::QSW : 1];
+    constexpr bool HOIST_T = QUAD && MODE == IDX_GROUPED;
+    int tq[HOIST_T ? C::QSW : 1], limq[HOIST ? C::QSW : 1];
     auto query_row = [&](int g_, int ql_, int qq) {
       const int qj = slice * C::QSW + qq;    // the query's place among the job's QS
       int t;
@@ -542,7 +573,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 #pragma unroll
         for (int qq = 0; qq < (HOIST ? C::QSW : 0); ++qq) {
           const int t = query_row(g, ql, qq);
-          tq[qq] = t;
+          if constexpr (HOIST_T) tq[qq] = t;
           limq[qq] = (MODE == IDX_DECODE || t < 0) ? 0 : vis_limit(t, a);
         }
       }
@@ -567,6 +598,25 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 #endif
             }
         }
+        // the warp's queries this job scores (bit qq). A grouped job skips a
+        // query that did not keep the block of the warp's rows (its 32 rows lie
+        // in one 64-key block): the accumulator columns of that query are
+        // neither read nor summed, and its scores are not written.
+        constexpr uint32_t FULL = (1u << C::QSW) - 1u;
+        constexpr bool SPLIT = MODE == IDX_GROUPED && C::QSW == 2;   // per-query load ranges below
+        uint32_t need = FULL;
+        if constexpr (SPLIT) {
+          if (s < 0) {
+            need = 0u;                         // no union block in this half of the tile
+          } else {
+            const unsigned long long wslot = sUSlot[col];
+#pragma unroll
+            for (int qq = 0; qq < C::QSW; ++qq) {
+              const int qlq = g * C::QS + slice * C::QSW + qq;
+              if (tq[qq] < 0 || ((wslot >> (8 * qlq)) & 0xFFull) == 0xFFull) need &= ~(1u << qq);
+            }
+          }
+        }
         // w * ReLU(a) = (w / 2) * (a + |a|): a + |a| is exact (2a or +0) and one
         // FADD; the halved weights sit in sW, pairs of heads accumulate with
         // f32x2 FMAs. acc2[L][qq]: lane 8L + r, query qq.
@@ -575,12 +625,29 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         for (int L = 0; L < 4; ++L)
 #pragma unroll
           for (int qq = 0; qq < C::QSW; ++qq) acc2[L][qq] = make_float2(0.f, 0.f);
+        // load n covers lane half h and 32-column chunk cc: in query-major
+        // order (n = qq * LPQ + h * CPQ + chunk of the query) when a job may
+        // skip one of the warp's queries, else lane-half-major (n = h * NCC + cc)
+        constexpr int CPQ = NCC / C::QSW;      // 32-column chunks per query
+        constexpr int LPQ = 2 * CPQ;           // loads per query
+        static_assert(CPQ * C::QSW == NCC && CPQ * 32 == H, "a query's heads fill whole chunks");
+        struct LoadAt {
+          int qq, h, cc;
+        };
+        auto load_at = [](int n) {
+          if constexpr (SPLIT)
+            return LoadAt{n / LPQ, (n % LPQ) / CPQ, (n / LPQ) * CPQ + n % CPQ};
+          else
+            return LoadAt{(n % NCC) / CPQ, n / NCC, n % NCC};
+        };
         const uint32_t t0 = tmem_base + buf * C::N + slice * C::SCOLS;
         auto addr = [&](int n) {
-          return t0 + (uint32_t(lq * 32 + 16 * (n / NCC)) << 16) + uint32_t((n % NCC) * 32);
+          const LoadAt l = load_at(n);
+          return t0 + (uint32_t(lq * 32 + 16 * l.h) << 16) + uint32_t(l.cc * 32);
         };
         auto consume = [&](const uint32_t (&v)[16], int n) {
-          const int h = n / NCC, cc = n % NCC, qq = cc * 32 / H;
+          const LoadAt l = load_at(n);
+          const int qq = l.qq, h = l.h, cc = l.cc;
 #pragma unroll
           for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -598,32 +665,50 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 #endif
             }
         };
-        // double-buffered loads: load n + 1 is in flight while load n is consumed
-        uint32_t va[16], vb[16];
-        tmem_ld16x256b_x4(addr(0), va);
-        tmem_ld_wait();
-        tmem_regs_ready(va);
+        // loads [LO, HI), double-buffered: load n + 1 is in flight while load n
+        // is consumed; the accumulator is released once its last load is issued
+        auto drain = [&](auto lo_c, auto hi_c) {
+          constexpr int LO = decltype(lo_c)::value, HI = decltype(hi_c)::value;
+          uint32_t va[16], vb[16];
+          tmem_ld16x256b_x4(addr(LO), va);
+          tmem_ld_wait();
+          tmem_regs_ready(va);
 #pragma unroll
-        for (int n = 0; n < NLD; n += 2) {
-          if (n + 1 < NLD) tmem_ld16x256b_x4(addr(n + 1), vb);
-          if (n + 1 >= NLD) release();
-          consume(va, n);
-          if (n + 1 < NLD) {
-            tmem_ld_wait();
-            tmem_regs_ready(vb);
-            if (n + 2 < NLD) tmem_ld16x256b_x4(addr(n + 2), va);
-            if (n + 2 >= NLD) release();
-            consume(vb, n + 1);
-            if (n + 2 < NLD) {
+          for (int n = LO; n < HI; n += 2) {
+            if (n + 1 < HI) tmem_ld16x256b_x4(addr(n + 1), vb);
+            if (n + 1 >= HI) release();
+            consume(va, n);
+            if (n + 1 < HI) {
               tmem_ld_wait();
-              tmem_regs_ready(va);
+              tmem_regs_ready(vb);
+              if (n + 2 < HI) tmem_ld16x256b_x4(addr(n + 2), va);
+              if (n + 2 >= HI) release();
+              consume(vb, n + 1);
+              if (n + 2 < HI) {
+                tmem_ld_wait();
+                tmem_regs_ready(va);
+              }
             }
           }
+        };
+        if constexpr (SPLIT) {
+          if (need == FULL)
+            drain(IntC<0>{}, IntC<NLD>{});
+          else if (need == 1u)
+            drain(IntC<0>{}, IntC<LPQ>{});
+          else if (need == 2u)
+            drain(IntC<LPQ>{}, IntC<NLD>{});
+          else
+            release();
+        } else {
+          drain(IntC<0>{}, IntC<NLD>{});
         }
         // reduce-scatter over the quad: the lane pair {0,1} or {2,3} by bit 1
         // of c, then one lane by bit 0; thread c keeps lane c (row 8c + r)
 #pragma unroll
         for (int qq = 0; qq < C::QSW; ++qq) {
+          qsum[qq] = 0.f;
+          if (SPLIT && !((need >> qq) & 1u)) continue;   // warp-uniform
           float sl[4];
 #pragma unroll
           for (int L = 0; L < 4; ++L) sl[L] = acc2[L][qq].x + acc2[L][qq].y;
@@ -728,7 +813,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       // outputs
 #pragma unroll
       for (int qq = 0; qq < C::QSW; ++qq) {
-        const int t = HOIST ? tq[HOIST ? qq : 0] : query_row(g, ql, qq);
+        const int t = HOIST_T ? tq[HOIST_T ? qq : 0] : query_row(g, ql, qq);
         if (t < 0) continue;                   // absent query, or a row past the last
         int gcol = 0;                          // grouped: the query's candidate column of this key
         if constexpr (MODE == IDX_GROUPED) {

@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(LSA_ST) lsa_score_kernel(ScoreArgs a) {
   const int i_last = min(a.rows, i0 + LSA_TILE) - 1;
   if ((long long)b0 * a.col_stride >= visible_buckets(row_position(a, i_last), a.n_cluster, a.m, a.n_blocks))
     return;                                 // no query of the tile sees a bucket of it
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lsa_score_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sm = smem_align1024(lsa_score_raw);
   uint8_t* sA = sm;                         // 128 buckets x 64 (16 KB)
   uint8_t* sB = sm + LSA_TILE * 128;        // 128 queries x 64 (16 KB)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

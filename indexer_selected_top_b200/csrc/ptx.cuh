@@ -10,6 +10,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte aligned byte of a dynamic shared-memory array. The
+// pointer is the array plus an offset (no round trip through an integer), so
+// the compiler still knows it addresses shared memory and accesses through it
+// compile to shared-memory loads and stores rather than generic ones.
+__device__ __forceinline__ uint8_t* smem_align1024(uint8_t* raw) {
+  return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ bool elect_one_lane() {
   return (threadIdx.x & 31) == 0;
 }
