@@ -569,6 +569,10 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       tc_fence_after();
 
       float qsum[C::QSW];                      // sum_h w'[h] * ReLU(acc[h]) of this thread's key row, per query
+      // grouped, two queries per warp: the jobs skip queries per warp below,
+      // and the slot bytes read for that serve the outputs too
+      constexpr bool SPLIT = QUAD && MODE == IDX_GROUPED && C::QSW == 2;
+      uint32_t slots2 = 0xFFFFu;
       if (HOIST && g != wg) {                  // the job's queries changed
 #pragma unroll
         for (int qq = 0; qq < (HOIST ? C::QSW : 0); ++qq) {
@@ -603,23 +607,22 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         // in one 64-key block): the accumulator columns of that query are
         // neither read nor summed, and its scores are not written.
         constexpr uint32_t FULL = (1u << C::QSW) - 1u;
-        constexpr bool SPLIT = MODE == IDX_GROUPED && C::QSW == 2;   // per-query load ranges below
         uint32_t need = FULL;
         if constexpr (SPLIT) {
           if (s < 0) {
             need = 0u;                         // no union block in this half of the tile
           } else {
-            const unsigned long long wslot = sUSlot[col];
+            // the slot bytes of the warp's two queries (adjacent in the slot word)
+            slots2 = (uint32_t)(sUSlot[col] >> (8 * (g * C::QS + slice * C::QSW))) & 0xFFFFu;
 #pragma unroll
-            for (int qq = 0; qq < C::QSW; ++qq) {
-              const int qlq = g * C::QS + slice * C::QSW + qq;
-              if (tq[qq] < 0 || ((wslot >> (8 * qlq)) & 0xFFull) == 0xFFull) need &= ~(1u << qq);
-            }
+            for (int qq = 0; qq < C::QSW; ++qq)
+              if (tq[qq] < 0 || ((slots2 >> (8 * qq)) & 0xFFu) == 0xFFu) need &= ~(1u << qq);
           }
         }
         // w * ReLU(a) = (w / 2) * (a + |a|): a + |a| is exact (2a or +0) and one
         // FADD; the halved weights sit in sW, pairs of heads accumulate with
-        // f32x2 FMAs. acc2[L][qq]: lane 8L + r, query qq.
+        // f32x2 FMAs. acc2[L][qq]: lane 8L + r, query qq (two accumulators per
+        // lane and query, alternating over the column groups, measured slower)
         float2 acc2[4][C::QSW];
 #pragma unroll
         for (int L = 0; L < 4; ++L)
@@ -819,7 +822,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         if constexpr (MODE == IDX_GROUPED) {
           if (cur.s < 0) continue;             // no union block in this half
           const int ql = g * C::QS + slice * C::QSW + qq;
-          const int slot = (int)((sUSlot[col] >> (8 * ql)) & 0xFFu);
+          const int slot = SPLIT ? (int)((slots2 >> (8 * qq)) & 0xFFu) : (int)((sUSlot[col] >> (8 * ql)) & 0xFFu);
           if (slot == 0xFF) continue;          // the query did not keep this block
           gcol = slot * 64 + (row & 63);
         }
