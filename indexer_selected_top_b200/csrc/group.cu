@@ -6,8 +6,9 @@
 // Queries that attend to nearly the same keys can share those reads. In the
 // two-stage method the queries that keep the same key blocks (HISA section 3)
 // select mostly the same keys; the grouping kernel below sorts every window
-// of GW consecutive queries by a MinHash of its kept-block set, so runs of GA
-// queries in that order tend to keep the same blocks. The grouped kernel then
+// of GW consecutive queries by three MinHashes of its kept-block set
+// (lexicographically), so runs of GA queries in that order tend to keep the
+// same blocks. The grouped kernel then
 // takes GA queries per CTA (one warp each), forms the union of their index
 // sets with a per-key mask of the queries that chose the key, gathers each
 // union key once into a ring shared by the CTA, and lets every warp attend
@@ -29,6 +30,7 @@
 namespace sa {
 
 constexpr int GW = 2048;             // queries per grouping window
+static_assert(GW == 2048, "the sort key holds a query's index in its window in 11 bits");
 constexpr int GA = kGroupQueries;    // queries per attention group (one warp each)
 constexpr int GT = GA * 32;          // threads per grouped CTA
 constexpr int GCH = 64;              // keys per ring stage
@@ -47,13 +49,22 @@ static __device__ __forceinline__ uint32_t block_hash(uint32_t b) {
   return x;
 }
 
-// The signature of query t: the smallest hash over its kept blocks, leaving
-// out block 0 and the query's own block, which every query keeps (HISA
-// section 3: the first and the local block are always in). With `sel` (the
-// top-k's selection bitmaps over the kept blocks' keys) only the blocks
-// holding at least min_sel selected keys count: the blocks a query draws most
-// of its keys from mark its neighbourhood better than the blocks it kept at
-// the margin. One warp per query: lane j reads kept slots j and j + 32.
+// The signature of query t: the smallest hash over its kept blocks under
+// three hash functions, leaving out block 0 and the query's own block, which
+// every query keeps (HISA section 3: the first and the local block are always
+// in). Two queries agree on one MinHash with probability equal to the Jaccard
+// similarity of their block sets; sorting by the first, then the second, then
+// the third keeps a run of equal first hashes ordered by how much more its
+// members share, so fewer groups straddle two runs (on the 64K two-stage
+// workload an 8-query group's union of kept blocks is 1.08 x its queries' mean
+// kept count, against 1.32 with one MinHash). With `sel` (the top-k's
+// selection bitmaps over the kept blocks' keys) only the blocks holding at
+// least min_sel selected keys count: the blocks a query draws most of its keys
+// from mark its neighbourhood better than the blocks it kept at the margin.
+// The sort key packs the three minima (17, 18 and 18 high bits) above the
+// query's index in its window (11 bits); the first field stops at 0x1FFFE so
+// no key equals the empty slot's all-ones. One warp per query: lane j reads
+// kept slots j and j + 32.
 __global__ void __launch_bounds__(256) group_signature_kernel(const int* __restrict__ kept, int keep,
                                                               const uint32_t* __restrict__ sel, int min_sel, int n_q,
                                                               int q_pos0, int block,
@@ -61,7 +72,7 @@ __global__ void __launch_bounds__(256) group_signature_kernel(const int* __restr
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (t >= n_q) return;
   const int cur = (q_pos0 + t) / block;
-  uint32_t h = 0xFFFFFFFFu;
+  uint32_t h1 = 0xFFFFFFFFu, h2 = 0xFFFFFFFFu, h3 = 0xFFFFFFFFu;
   for (int j = lane; j < keep; j += 32) {
     const int b = kept[(long long)t * keep + j];
     bool use = b >= 0 && b != 0 && b != cur;
@@ -69,15 +80,27 @@ __global__ void __launch_bounds__(256) group_signature_kernel(const int* __restr
       const uint32_t* sr = sel + (long long)t * keep * 2;
       use = __popc(sr[2 * j]) + __popc(sr[2 * j + 1]) >= min_sel;
     }
-    if (use) h = min(h, block_hash((uint32_t)b));
+    if (use) {
+      h1 = min(h1, block_hash(3u * (uint32_t)b));
+      h2 = min(h2, block_hash(3u * (uint32_t)b + 1u));
+      h3 = min(h3, block_hash(3u * (uint32_t)b + 2u));
+    }
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) h = min(h, __shfl_xor_sync(0xffffffffu, h, o));
-  if (lane == 0) sig[t] = ((unsigned long long)h << 32) | (uint32_t)t;
+  for (int o = 16; o > 0; o >>= 1) {
+    h1 = min(h1, __shfl_xor_sync(0xffffffffu, h1, o));
+    h2 = min(h2, __shfl_xor_sync(0xffffffffu, h2, o));
+    h3 = min(h3, __shfl_xor_sync(0xffffffffu, h3, o));
+  }
+  if (lane == 0)
+    sig[t] = ((unsigned long long)min(h1 >> 15, 0x1FFFEu) << 47) | ((unsigned long long)(h2 >> 14) << 29) |
+             ((unsigned long long)(h3 >> 14) << 11) | (unsigned long long)(t & (GW - 1));
 }
 
 // perm[w * GW + i] = the query at rank i of window w in (signature, query)
-// order, -1 past n_q.
+// order, -1 past n_q. A key's low 11 bits are its query's index in the window
+// (the keys of the two-stage grouping above, and (hash << 32 | t) keys, whose
+// t has those bits).
 __global__ void __launch_bounds__(1024) group_sort_kernel(const unsigned long long* __restrict__ sig, int n_q,
                                                           int* __restrict__ perm) {
   __shared__ unsigned long long key[GW];
@@ -102,7 +125,7 @@ __global__ void __launch_bounds__(1024) group_sort_kernel(const unsigned long lo
   }
   for (int i = threadIdx.x; i < GW; i += 1024) {
     const unsigned long long k = key[i];
-    perm[w0 + i] = (k == ~0ull) ? -1 : (int)(uint32_t)(k & 0xFFFFFFFFu);
+    perm[w0 + i] = (k == ~0ull) ? -1 : w0 + (int)(k & (unsigned long long)(GW - 1));
   }
 }
 
