@@ -41,6 +41,10 @@ cudaError_t launch_gather_rows(const void* src, void* dst, const int* rows, int 
   return cudaGetLastError();
 }
 
+// sample keys a theta thread holds in registers (TH_REG * TK_THREADS = 16,384
+// samples, the most a row of the library's plans has)
+constexpr int TH_REG = 32;
+
 static __device__ __forceinline__ float key_to_float(uint32_t key) {
   const uint32_t b = (key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key;
   return __uint_as_float(b);
@@ -73,6 +77,18 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
     const long long want = llrintf(gamma * (float)k * (float)n_vs / (float)n_vis);
     int need = (int)max(1ll, min((long long)n_vs, want));
     const float* row = stab + (long long)t * ld;
+    // the samples' keys, read once (all loads in flight together) and kept in
+    // registers for the three passes; a longer sample row (not planned by the
+    // library) is re-read from memory in every pass
+    uint32_t kr[TH_REG];
+    const bool in_regs = n_vs <= TH_REG * TK_THREADS;
+    if (in_regs) {
+#pragma unroll
+      for (int i = 0; i < TH_REG; ++i) {
+        const int j = tid + i * TK_THREADS;
+        kr[i] = (j < n_vs) ? score_key(row[(long long)j * sstride]) : 0u;
+      }
+    }
     uint32_t prefix = 0;
     int pbits = 0;
     while (pbits < 32) {                    // 12 + 12 + 8 bits: the exact n_theta-th key
@@ -81,9 +97,15 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
       for (int b = tid; b < nbins; b += TK_THREADS) sh.hist[b] = 0;
       __syncthreads();
       const int sdig = 32 - pbits - db;
-      for (int j = tid; j < n_vs; j += TK_THREADS) {
-        const uint32_t key = score_key(row[(long long)j * sstride]);
+      auto count = [&](uint32_t key) {
         if (pbits == 0 || (key >> (32 - pbits)) == prefix) atomicAdd(&sh.hist[(key >> sdig) & (nbins - 1)], 1u);
+      };
+      if (in_regs) {
+#pragma unroll
+        for (int i = 0; i < TH_REG; ++i)
+          if (tid + i * TK_THREADS < n_vs) count(kr[i]);
+      } else {
+        for (int j = tid; j < n_vs; j += TK_THREADS) count(score_key(row[(long long)j * sstride]));
       }
       __syncthreads();
       find_bucket(sh, nbins, need);
@@ -178,9 +200,25 @@ __global__ void __launch_bounds__(256)
   const int lo = blockIdx.x * COLLECT_CHUNK, hi = min(n_vis, lo + COLLECT_CHUNK);
   if (threadIdx.x == 0) n_hit = 0;
   __syncthreads();
-  for (int s = lo + threadIdx.x; s < hi; s += 256) {
-    const float sc = row[s];
+  auto take = [&](float sc, int s) {
     if (sc >= th) hits[atomicAdd(&n_hit, 1)] = ((unsigned long long)score_key(sc) << 32) | (uint32_t)(~(uint32_t)s);
+  };
+  if (hi - lo == COLLECT_CHUNK && (ld & 3) == 0 && (reinterpret_cast<uintptr_t>(row) & 15u) == 0) {
+    // a whole chunk: four 16-byte loads per thread, all in flight together
+    float4 v[COLLECT_CHUNK / 1024];
+#pragma unroll
+    for (int i = 0; i < COLLECT_CHUNK / 1024; ++i)
+      v[i] = *reinterpret_cast<const float4*>(row + lo + 4 * (threadIdx.x + 256 * i));
+#pragma unroll
+    for (int i = 0; i < COLLECT_CHUNK / 1024; ++i) {
+      const int s = lo + 4 * (threadIdx.x + 256 * i);
+      take(v[i].x, s);
+      take(v[i].y, s + 1);
+      take(v[i].z, s + 2);
+      take(v[i].w, s + 3);
+    }
+  } else {
+    for (int s = lo + threadIdx.x; s < hi; s += 256) take(row[s], s);
   }
   __syncthreads();
   const int n = n_hit;
