@@ -12,7 +12,11 @@
 // are positive: ReLU(sq*sk*a) = sq*sk*ReLU(a).
 //
 // Roles: warp 0 = TMA producer (one lane), warp 1 = MMA issuer (one lane)
-// and TMEM owner, warps 2..17 = epilogue teams. The 512 TMEM columns hold
+// and TMEM owner, warps 2..17 = epilogue teams, warp 18 = metadata stager.
+// Prefill and grouped CTAs are persistent (one per SM): each loops over its
+// work units with two query buffers and two metadata buffers, so the next
+// unit's query tile (TMA) and weights (the stager) load while one runs and
+// no unit pays a CTA's setup and drain. The 512 TMEM columns hold
 // 512 / N fp32 accumulators (2 at N = 256, 8 at N = 64) used as a ring; team
 // b % TEAMS drains buffer b, so the epilogue of one accumulator overlaps the
 // MMAs into the others (the pages' bucket scan also overlaps its epilogue
@@ -50,6 +54,11 @@ namespace sa {
 #ifndef SA_IDX_STAGES
 #define SA_IDX_STAGES 6
 #endif
+// key-tile ring depth of the persistent modes (their two query buffers take
+// the shared memory of the other stages)
+#ifndef SA_IDX_STAGES_PERSIST
+#define SA_IDX_STAGES_PERSIST 5
+#endif
 // FP8 prefill: sub-tiles of QS queries per CTA (each key tile serves G jobs)
 #ifndef SA_IDX_PREFILL_G
 #define SA_IDX_PREFILL_G 2
@@ -63,7 +72,7 @@ namespace sa {
 #define SA_IDX_TEAMS_WIDE 2
 #endif
 constexpr int kIdxEpiWarps = 16;                              // epilogue warps of every mode
-constexpr int kIdxThreads = 64 + 32 * kIdxEpiWarps;
+constexpr int kIdxThreads = 64 + 32 * kIdxEpiWarps + 32;      // + the staging warp of the persistent modes
 // independent partial sums per query in the epilogue when N holds several queries
 #ifndef SA_IDX_NP_WIDE
 #define SA_IDX_NP_WIDE 2
@@ -101,9 +110,14 @@ struct IdxCfg {
   static constexpr int THREADS = kIdxThreads;
   static_assert(NBUF % TEAMS == 0, "every team owns whole accumulators");
   static_assert(WPT % 4 == 0 && QS % SLICES == 0 && SCOLS == QSW * H, "a warp drains whole queries");
+  // prefill and grouped CTAs are persistent: each loops over work units (a
+  // block of NQ rows, a query group) with two query buffers and two metadata
+  // buffers, so the next unit's queries and weights load while one runs
+  static constexpr bool PERSIST = MODE == IDX_PREFILL || MODE == IDX_GROUPED;
+  static constexpr int QB = PERSIST ? 2 : 1;                  // query / metadata buffers
   static constexpr int QBYTES = NQ * H * ROWB;
   static constexpr int KBYTES = 128 * ROWB;
-  static constexpr int NS = (MODE == IDX_DECODE) ? 8 : SA_IDX_STAGES;    // key-tile stages
+  static constexpr int NS = (MODE == IDX_DECODE) ? 8 : PERSIST ? SA_IDX_STAGES_PERSIST : SA_IDX_STAGES;
   static constexpr int KSTEPS = ROWB / 32;                   // 32-byte K slices per MMA
   static constexpr int KEEPMAX = 64;                          // gather: kept blocks per query
   static constexpr int GU = kGroupQueries * KEEPMAX;          // grouped: union blocks per group (at most)
@@ -112,8 +126,12 @@ struct IdxCfg {
   static constexpr int KEPT_BYTES = (MODE == IDX_GATHER)    ? NQ * KEEPMAX * 4
                                     : (MODE == IDX_GROUPED) ? GU * 8 + GU * 4 + 64
                                                             : (NQ * 4 + 15) / 16 * 16;
-  static constexpr int SMEM_USED =
-      1024 + QBYTES + NS * KBYTES + NQ * H * 4 + KEPT_BYTES + (2 * NS + 1 + 2 * NBUF) * 8 + 16;
+  static constexpr int WBYTES = NQ * H * 4;                    // the unit's weights
+  static constexpr int META = WBYTES + KEPT_BYTES;              // one metadata buffer
+  static constexpr int NBAR = 2 * NS + 4 * QB + 2 * NBUF;
+  static constexpr int SMEM_USED = 1024 + QB * QBYTES + NS * KBYTES + QB * META + NBAR * 8 + 16;
+  static_assert(SMEM_USED <= 227 * 1024, "shared memory");
+  static_assert(WBYTES % 16 == 0 && KEPT_BYTES % 16 == 0, "metadata alignment");
   // at least 120 KB: one CTA per SM, so two CTAs never contend for TMEM
   static constexpr int SMEM = SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024;
   static_assert(N <= 256 && N % 16 == 0, "MMA N");
@@ -166,62 +184,280 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                    const IdxArgs a) {
   using C = IdxCfg<H, D, FP8, MODE>;
+  constexpr bool PERSIST = C::PERSIST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_align1024(smem_raw);
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + C::QBYTES;
-  float* sW = reinterpret_cast<float*>(sK + C::NS * C::KBYTES);
-  int* sKept = reinterpret_cast<int*>(sW + C::NQ * H);         // gather: [NQ][KEEPMAX], -1 padded
-  float* sTheta = reinterpret_cast<float*>(sKept);            // candidate mode: theta of the CTA's rows
-  // grouped: [GU] slot words, [GU] union blocks, [NQ] the group's queries
-  unsigned long long* sUSlot = reinterpret_cast<unsigned long long*>(sKept);
-  int* sUBlk = reinterpret_cast<int*>(sUSlot + C::GU);
-  int* sQt = sUBlk + C::GU;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sKept) + C::KEPT_BYTES);
+  uint8_t* sQ0 = smem;                                        // [QB] query tiles
+  uint8_t* sK = sQ0 + C::QB * C::QBYTES;                       // [NS] key tiles
+  uint8_t* sMeta0 = sK + C::NS * C::KBYTES;                    // [QB] per-unit metadata
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sMeta0 + C::QB * C::META);
   uint64_t* kfull = bars;
-  uint64_t* kempty = bars + C::NS;
-  uint64_t* qfull = bars + 2 * C::NS;
-  uint64_t* tfull = qfull + 1;
+  uint64_t* kempty = kfull + C::NS;
+  uint64_t* qfull = kempty + C::NS;    // [QB] the unit's query tile landed
+  uint64_t* qempty = qfull + C::QB;    // [QB] the MMAs of the unit that read the buffer are done
+  uint64_t* mfull = qempty + C::QB;    // [QB] the unit's metadata is staged
+  uint64_t* mempty = mfull + C::QB;    // [QB] the epilogue is done with it
+  uint64_t* tfull = mempty + C::QB;
   uint64_t* tempty = tfull + C::NBUF;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + C::NBUF);
   volatile uint32_t* abort_flag = tmem_slot + 1;
+  // metadata buffer b: the weights (halved: the packed math sums (w / 2) *
+  // (a + |a|)), then gather: kept lists [NQ][KEEPMAX], -1 padded; grouped: [GU]
+  // slot words, [GU] union blocks, [NQ] the group's queries; prefill: the
+  // rows' thetas (candidate mode)
+  struct Meta {
+    float* w;
+    int* kept;
+    float* theta;
+    unsigned long long* uslot;
+    int* ublk;
+    int* qt;
+  };
+  auto meta = [&](int b) {
+    uint8_t* m = sMeta0 + b * C::META;
+    Meta r;
+    r.w = reinterpret_cast<float*>(m);
+    r.kept = reinterpret_cast<int*>(m + C::WBYTES);
+    r.theta = reinterpret_cast<float*>(m + C::WBYTES);
+    r.uslot = reinterpret_cast<unsigned long long*>(m + C::WBYTES);
+    r.ublk = reinterpret_cast<int*>(r.uslot + C::GU);
+    r.qt = r.ublk + C::GU;
+    return r;
+  };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kStagerWarp = 2 + kIdxEpiWarps;
 
-  // ---------------- work unit (identical in every role) ----------------
-  int q0 = 0, nq = 0, seq = 0, tile0 = 0, ntiles = 0, geff = 1, njobs = 0, seq_len = a.n_k;
-  int n_ub = 0;                    // grouped: the group's union blocks
+  // ---------------- work units (identical in every role) ----------------
   const int n_rows = (a.row_count != nullptr) ? min(a.n_q, *a.row_count - a.row_base) : a.n_q;
-  if constexpr (MODE == IDX_PREFILL) {
-    const int unit = gridDim.x - 1 - blockIdx.x;            // heaviest (latest rows) first
-    q0 = unit * C::NQ;
-    nq = min(C::NQ, n_rows - q0);
-    if (nq <= 0) return;                                    // past the rows flagged on the device (uniform)
-    geff = (nq + C::QS - 1) / C::QS;
-    const int lim = min(vis_limit(q0 + nq - 1, a), a.n_k - 1);
-    tile0 = a.tile_lo;                                      // the key tiles [tile_lo, min(tile_hi, lim / 128 + 1))
-    ntiles = (lim < 0) ? 0 : max(0, min(lim / 128 + 1, a.tile_hi) - tile0);
-    njobs = ntiles * geff;
-  } else if constexpr (MODE == IDX_DECODE) {
-    seq = blockIdx.y;
-    q0 = seq;
-    nq = 1;
-    seq_len = a.seq_lens ? min(a.seq_lens[seq], a.span) : a.span;
-    if (a.seq_lens != nullptr && a.seq_lens[seq] > a.span && blockIdx.x == 0 && threadIdx.x == 0 &&
-        a.status != nullptr)
-      atomicCAS(a.status, 0u, 1u /* SA_ERR_INVALID_ARGUMENT: a sequence longer than the call's max_len */);
-    const int total = (seq_len + 127) / 128;
-    tile0 = blockIdx.x * a.tiles_per_cta;
-    ntiles = max(0, min(a.tiles_per_cta, total - tile0));
-    njobs = ntiles;
-  } else if constexpr (MODE == IDX_GROUPED) {
-    q0 = blockIdx.x * C::NQ;       // the group's slice of perm
-    nq = C::NQ;
-    geff = C::G;                   // jobs are counted from the staged union below
-  } else {
-    q0 = blockIdx.x * C::NQ;
-    nq = min(C::NQ, a.n_q - q0);   // jobs are counted from the staged kept lists below
-  }
+  int n_units = 1;
+  if constexpr (MODE == IDX_PREFILL) n_units = (a.n_q + C::NQ - 1) / C::NQ;
+  if constexpr (MODE == IDX_GROUPED) n_units = a.n_groups;
+  // the it-th unit of this CTA (-1: none left). Persistent CTAs take units
+  // round-robin, prefill in descending row order (the latest rows see the most
+  // keys) and alternating direction per round, which evens out their work
+  auto unit_at = [&](int it) -> int {
+    if constexpr (PERSIST) {
+      const int pos = (MODE == IDX_PREFILL && (it & 1)) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x;
+      const long long idx = (long long)it * gridDim.x + pos;
+      if (idx >= n_units) return -1;
+      return MODE == IDX_PREFILL ? n_units - 1 - (int)idx : (int)idx;
+    } else {
+      return it == 0 ? (int)blockIdx.x : -1;
+    }
+  };
+  struct UnitP {
+    int q0, nq, seq, tile0, ntiles, geff, njobs, n_ub, seq_len;
+  };
+  int gather_njobs = 0;                // gather: counted from the staged kept lists
+  auto unit_params = [&](int unit) {
+    UnitP u;
+    u.q0 = 0;
+    u.nq = 0;
+    u.seq = 0;
+    u.tile0 = 0;
+    u.ntiles = 0;
+    u.geff = 1;
+    u.njobs = 0;
+    u.n_ub = 0;
+    u.seq_len = a.n_k;
+    if constexpr (MODE == IDX_PREFILL) {
+      u.q0 = unit * C::NQ;
+      u.nq = min(C::NQ, n_rows - u.q0);
+      if (u.nq > 0) {                  // else past the rows flagged on the device
+        u.geff = (u.nq + C::QS - 1) / C::QS;
+        const int lim = min(vis_limit(u.q0 + u.nq - 1, a), a.n_k - 1);
+        u.tile0 = a.tile_lo;           // the key tiles [tile_lo, min(tile_hi, lim / 128 + 1))
+        u.ntiles = (lim < 0) ? 0 : max(0, min(lim / 128 + 1, a.tile_hi) - u.tile0);
+        u.njobs = u.ntiles * u.geff;
+      }
+    } else if constexpr (MODE == IDX_DECODE) {
+      u.seq = blockIdx.y;
+      u.q0 = u.seq;
+      u.nq = 1;
+      u.seq_len = a.seq_lens ? min(a.seq_lens[u.seq], a.span) : a.span;
+      const int total = (u.seq_len + 127) / 128;
+      u.tile0 = blockIdx.x * a.tiles_per_cta;
+      u.ntiles = max(0, min(a.tiles_per_cta, total - u.tile0));
+      u.njobs = u.ntiles;
+    } else if constexpr (MODE == IDX_GROUPED) {
+      u.q0 = unit * C::NQ;             // the group's slice of perm
+      u.nq = C::NQ;
+      u.geff = C::G;
+      int nv = 0;
+      for (int ql = 0; ql < C::NQ; ++ql) {
+        const int t = a.perm[u.q0 + ql];
+        nv += (t >= 0 && t < a.n_q) ? 1 : 0;
+      }
+      u.n_ub = a.gb_n[unit];
+      u.ntiles = (nv > 0) ? (u.n_ub + 1) / 2 : 0;   // absent queries only: no jobs
+      u.njobs = u.ntiles * u.geff;
+    } else {
+      u.q0 = unit * C::NQ;
+      u.nq = min(C::NQ, a.n_q - u.q0);
+      u.njobs = u.ntiles = gather_njobs;
+    }
+    return u;
+  };
+  // a unit's metadata into buffer m by one warp (the stager): the query rows
+  // first (one load per query, shared by shuffles), then every weight and
+  // scale load of the lane issued before any is used, so a unit costs about
+  // two load latencies however many weights it has
+  auto stage_warp = [&](const UnitP& u, const Meta& m) {
+    static_assert(C::NQ <= 32 || MODE != IDX_GROUPED, "one query row per lane");
+    constexpr int NWI = (C::NQ * H + 31) / 32;
+    int myrow = -1;                    // the row of query `lane` (lanes < NQ; NQ <= 32 here)
+    if (lane < C::NQ) {
+      if constexpr (MODE == IDX_GROUPED) {
+        const int t = a.perm[u.q0 + lane];
+        myrow = (t >= 0 && t < a.n_q) ? t : -1;
+      } else {
+        myrow = (lane < u.nq) ? (a.q_rows != nullptr ? a.q_rows[u.q0 + lane] : u.q0 + lane) : -1;
+      }
+    }
+    float wv[NWI], sv[NWI];
+#pragma unroll
+    for (int k = 0; k < NWI; ++k) {
+      const int i = lane + 32 * k, ql = i / H, h = i % H;
+      int qrow = (C::NQ <= 32) ? __shfl_sync(0xffffffffu, myrow, ql & 31) : -1;
+      if constexpr (C::NQ > 32)        // bf16 prefill with many queries per unit: rows by arithmetic
+        qrow = (ql < u.nq) ? (a.q_rows != nullptr ? a.q_rows[u.q0 + ql] : u.q0 + ql) : -1;
+      wv[k] = 0.f;
+      sv[k] = 1.f;
+      if (i < C::NQ * H && qrow >= 0) {
+        const long long r = (long long)qrow * H + h;
+        wv[k] = a.w[r];
+        if (a.q_scale) sv[k] = a.q_scale[r];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < NWI; ++k) {
+      const int i = lane + 32 * k;
+      const float v = wv[k] * sv[k];
+      if (i < C::NQ * H) m.w[i] = SA_IDX_EPI_PACKED ? 0.5f * v : v;
+    }
+    if constexpr (MODE == IDX_PREFILL) {
+      if (a.cand != nullptr)
+        for (int i = lane; i < C::NQ; i += 32) m.theta[i] = (i < u.nq) ? a.theta[u.q0 + i] : 0.f;
+    }
+    if constexpr (MODE == IDX_GROUPED) {
+      if (lane < C::NQ) m.qt[lane] = myrow;
+      const int gi = u.q0 / C::NQ;
+      const int* blk = a.gb_blk + (long long)gi * a.gb_cap;
+      const unsigned long long* slot = a.gb_slot + (long long)gi * a.gb_cap;
+      for (int i0 = 0; i0 < u.n_ub; i0 += 32 * 8) {   // eight loads of each list in flight per lane
+        int bv[8];
+        unsigned long long svv[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int i = i0 + lane + 32 * k;
+          bv[k] = (i < u.n_ub) ? blk[i] : 0;
+          svv[k] = (i < u.n_ub) ? slot[i] : 0ull;
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int i = i0 + lane + 32 * k;
+          if (i < u.n_ub) {
+            m.ublk[i] = bv[k];
+            m.uslot[i] = svv[k];
+          }
+        }
+      }
+    }
+  };
+  // a unit's metadata into buffer m, by threads tid = 0.. of nthr
+  auto stage = [&](const UnitP& u, const Meta& m, int tid, int nthr) {
+    for (int i = tid; i < C::NQ * H; i += nthr) {
+      const int ql = i / H, h = i % H;
+      float v = 0.f;
+      int qrow = (ql < u.nq) ? (a.q_rows != nullptr ? a.q_rows[u.q0 + ql] : u.q0 + ql) : -1;
+      if constexpr (MODE == IDX_GROUPED) {
+        qrow = a.perm[u.q0 + ql];
+        if (qrow >= a.n_q) qrow = -1;
+      }
+      if (qrow >= 0) {
+        const long long r = (long long)qrow * H + h;
+        v = a.w[r] * (a.q_scale ? a.q_scale[r] : 1.f);
+      }
+      m.w[i] = SA_IDX_EPI_PACKED ? 0.5f * v : v;
+    }
+    if constexpr (MODE == IDX_PREFILL) {
+      if (a.cand != nullptr)
+        for (int i = tid; i < C::NQ; i += nthr) m.theta[i] = (i < u.nq) ? a.theta[u.q0 + i] : 0.f;
+    }
+    if constexpr (MODE == IDX_GATHER) {
+      for (int i = tid; i < C::NQ * C::KEEPMAX; i += nthr) {
+        const int ql = i / C::KEEPMAX, j = i % C::KEEPMAX;
+        m.kept[i] = (ql < u.nq && j < a.keep) ? a.kept[(long long)(u.q0 + ql) * a.keep + j] : -1;
+      }
+    }
+    if constexpr (MODE == IDX_GROUPED) {
+      const int gi = u.q0 / C::NQ;
+      for (int i = tid; i < C::NQ; i += nthr) {
+        const int t = a.perm[u.q0 + i];
+        m.qt[i] = (t >= 0 && t < a.n_q) ? t : -1;
+      }
+      for (int i = tid; i < u.n_ub; i += nthr) {
+        m.ublk[i] = a.gb_blk[(long long)gi * a.gb_cap + i];
+        m.uslot[i] = a.gb_slot[(long long)gi * a.gb_cap + i];
+      }
+    }
+  };
+  // the key tile i of unit u into ring stage st (the TMA lane)
+  auto load_tile = [&](const UnitP& u, int i, int st, GatherCursor& gc) {
+    uint8_t* dst = sK + st * C::KBYTES;
+    if constexpr (MODE == IDX_PREFILL) {
+      mbar_arrive_expect_tx(&kfull[st], C::KBYTES);
+      tma_load_2d(dst, &kmap, &kfull[st], 0, (u.tile0 + i) * 128);
+    } else if constexpr (MODE == IDX_DECODE) {
+      mbar_arrive_expect_tx(&kfull[st], C::KBYTES);
+      tma_load_2d(dst, &kmap, &kfull[st], 0, (int)((long long)u.seq * a.n_k + (u.tile0 + i) * 128));
+    } else if constexpr (MODE == IDX_GROUPED) {
+      const int* blk = a.gb_blk + (long long)(u.q0 / C::NQ) * a.gb_cap;   // the union, read from global memory
+      const int b0 = blk[2 * i];
+      const int b1 = (2 * i + 1 < u.n_ub) ? blk[2 * i + 1] : -1;
+      mbar_arrive_expect_tx(&kfull[st], (b1 >= 0 ? 2 : 1) * 64 * C::ROWB);
+      tma_load_2d(dst, &kmap, &kfull[st], 0, b0 * 64);
+      if (b1 >= 0) tma_load_2d(dst + 64 * C::ROWB, &kmap, &kfull[st], 0, b1 * 64);
+    } else {
+      const int* kr = gc.row();
+      const int b0 = kr[2 * gc.pair];
+      const int b1 = kr[2 * gc.pair + 1];
+      mbar_arrive_expect_tx(&kfull[st], (b1 >= 0 ? 2 : 1) * 64 * C::ROWB);
+      tma_load_2d(dst, &kmap, &kfull[st], 0, b0 * 64);
+      if (b1 >= 0) tma_load_2d(dst + 64 * C::ROWB, &kmap, &kfull[st], 0, b1 * 64);
+      gc.next();
+    }
+  };
+  // the query tile of unit u into buffer b (the TMA lane)
+  auto load_q = [&](const UnitP& u, int b) {
+    uint8_t* q = sQ0 + b * C::QBYTES;
+    if constexpr (MODE == IDX_PREFILL) {
+      if (a.q_rows != nullptr) {       // listed rows: one box of H rows per query
+        mbar_arrive_expect_tx(&qfull[b], u.nq * H * C::ROWB);
+        for (int ql = 0; ql < u.nq; ++ql) tma_load_2d(q + ql * H * C::ROWB, &qmap, &qfull[b], 0, a.q_rows[u.q0 + ql] * H);
+      } else {
+        mbar_arrive_expect_tx(&qfull[b], u.geff * C::QS * H * C::ROWB);
+        for (int g = 0; g < u.geff; ++g)
+          tma_load_2d(q + g * C::QS * H * C::ROWB, &qmap, &qfull[b], 0, (u.q0 + g * C::QS) * H);
+      }
+    } else if constexpr (MODE == IDX_GROUPED) {
+      int qt[C::NQ], nv = 0;
+#pragma unroll
+      for (int ql = 0; ql < C::NQ; ++ql) {
+        const int t = a.perm[u.q0 + ql];
+        qt[ql] = (t >= 0 && t < a.n_q) ? t : -1;
+        nv += qt[ql] >= 0;
+      }
+      mbar_arrive_expect_tx(&qfull[b], nv * H * C::ROWB);
+#pragma unroll
+      for (int ql = 0; ql < C::NQ; ++ql)   // absent queries leave their rows unset: their scores are dropped
+        if (qt[ql] >= 0) tma_load_2d(q + ql * H * C::ROWB, &qmap, &qfull[b], 0, qt[ql] * H);
+    } else {
+      mbar_arrive_expect_tx(&qfull[b], u.nq * H * C::ROWB);
+      for (int ql = 0; ql < u.nq; ++ql) tma_load_2d(q + ql * H * C::ROWB, &qmap, &qfull[b], 0, (u.q0 + ql) * H);
+    }
+  };
 
   // ---------------- setup ----------------
   if (threadIdx.x == 0) {
@@ -229,128 +465,61 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       mbar_init(&kfull[s], 1);
       mbar_init(&kempty[s], 1);
     }
-    mbar_init(qfull, 1);
+    for (int b = 0; b < C::QB; ++b) {
+      mbar_init(&qfull[b], 1);
+      mbar_init(&qempty[b], 1);
+      mbar_init(&mfull[b], 32);
+      mbar_init(&mempty[b], kIdxEpiWarps);
+    }
     for (int b = 0; b < C::NBUF; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], C::WPT);
     }
     *abort_flag = 0u;
     fence_barrier_init();
+    if constexpr (MODE == IDX_DECODE) {
+      const int seq = blockIdx.y;
+      if (a.seq_lens != nullptr && a.seq_lens[seq] > a.span && blockIdx.x == 0 && a.status != nullptr)
+        atomicCAS(a.status, 0u, 1u /* SA_ERR_INVALID_ARGUMENT: a sequence longer than the call's max_len */);
+    }
   }
-  // the TMA lane (thread 0) issues the query tile and the first ring of key
-  // tiles right away, so their latency overlaps the rest of the setup (the
-  // weights' global loads, the staging of the group's lists, the TMEM
-  // allocation); grouped CTAs read their queries and first union blocks from
-  // global memory for it, by the same rules the staging below applies
-  int early = 0;                   // key tiles issued during the setup (thread 0)
-  if (threadIdx.x == 0) {
-    if constexpr (MODE == IDX_PREFILL || MODE == IDX_DECODE) {
-      if (njobs > 0) {
+  // the TMA lane (thread 0) issues the first unit's query tile and first ring
+  // of key tiles right away, so their latency overlaps the rest of the setup
+  // (the staging of the weights and lists, the TMEM allocation)
+  int early_it = -1, early = 0;        // the unit (its `it`) and key tiles issued during the setup (thread 0)
+  if constexpr (MODE != IDX_GATHER) {
+    if (threadIdx.x == 0) {
+      for (int it = 0;; ++it) {
+        const int unit = unit_at(it);
+        if (unit < 0) break;
+        const UnitP u = unit_params(unit);
+        if (u.njobs == 0) continue;
         prefetch_tmap(&qmap);
         prefetch_tmap(&kmap);
-        if (MODE == IDX_PREFILL && a.q_rows != nullptr) {   // listed rows: one box of H rows per query
-          mbar_arrive_expect_tx(qfull, nq * H * C::ROWB);
-          for (int ql = 0; ql < nq; ++ql) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, a.q_rows[q0 + ql] * H);
-        } else if (MODE == IDX_PREFILL) {
-          mbar_arrive_expect_tx(qfull, geff * C::QS * H * C::ROWB);
-          for (int g = 0; g < geff; ++g)
-            tma_load_2d(sQ + g * C::QS * H * C::ROWB, &qmap, qfull, 0, (q0 + g * C::QS) * H);
-        } else {
-          mbar_arrive_expect_tx(qfull, nq * H * C::ROWB);
-          for (int ql = 0; ql < nq; ++ql) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, (q0 + ql) * H);
-        }
-        early = min(ntiles, C::NS);   // the ring starts empty: no wait
-        for (int i = 0; i < early; ++i) {
-          mbar_arrive_expect_tx(&kfull[i], C::KBYTES);
-          const long long row0 = (MODE == IDX_DECODE) ? (long long)seq * a.n_k : 0ll;
-          tma_load_2d(sK + i * C::KBYTES, &kmap, &kfull[i], 0, (int)(row0 + (tile0 + i) * 128));
-        }
-      }
-    } else if constexpr (MODE == IDX_GROUPED) {
-      int qt[C::NQ], nv = 0;
-#pragma unroll
-      for (int ql = 0; ql < C::NQ; ++ql) {
-        const int t = a.perm[q0 + ql];
-        qt[ql] = (t >= 0 && t < a.n_q) ? t : -1;
-        nv += qt[ql] >= 0;
-      }
-      const int nub = a.gb_n[blockIdx.x];
-      const int nt = (nub + 1) / 2;
-      if (nv > 0 && nt > 0) {          // else the CTA has no jobs
-        prefetch_tmap(&qmap);
-        prefetch_tmap(&kmap);
-        mbar_arrive_expect_tx(qfull, nv * H * C::ROWB);
-#pragma unroll
-        for (int ql = 0; ql < C::NQ; ++ql)   // absent queries leave their rows unset: their scores are dropped
-          if (qt[ql] >= 0) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, qt[ql] * H);
-        early = min(nt, C::NS);
-        const int* blk = a.gb_blk + (long long)blockIdx.x * a.gb_cap;
-        for (int i = 0; i < early; ++i) {
-          const int b0 = blk[2 * i];
-          const int b1 = (2 * i + 1 < nub) ? blk[2 * i + 1] : -1;
-          uint8_t* dst = sK + i * C::KBYTES;
-          mbar_arrive_expect_tx(&kfull[i], (b1 >= 0 ? 2 : 1) * 64 * C::ROWB);
-          tma_load_2d(dst, &kmap, &kfull[i], 0, b0 * 64);
-          if (b1 >= 0) tma_load_2d(dst + 64 * C::ROWB, &kmap, &kfull[i], 0, b1 * 64);
-        }
+        load_q(u, 0);
+        early = min(u.ntiles, C::NS);  // the ring starts empty: no wait
+        GatherCursor gc = {};
+        for (int i = 0; i < early; ++i) load_tile(u, i, i, gc);
+        early_it = it;
+        break;
       }
     }
   }
   if (warp == 1) tmem_alloc<512>(tmem_slot);
-  for (int i = threadIdx.x; i < C::NQ * H; i += blockDim.x) {
-    const int ql = i / H, h = i % H;
-    float v = 0.f;
-    int qrow = (ql < nq) ? (a.q_rows != nullptr ? a.q_rows[q0 + ql] : q0 + ql) : -1;
-    if constexpr (MODE == IDX_GROUPED) {
-      qrow = a.perm[q0 + ql];
-      if (qrow >= a.n_q) qrow = -1;
-    }
-    if (qrow >= 0) {
-      const long long r = (long long)qrow * H + h;
-      v = a.w[r] * (a.q_scale ? a.q_scale[r] : 1.f);
-    }
-    sW[i] = SA_IDX_EPI_PACKED ? 0.5f * v : v;   // packed math sums (w / 2) * (a + |a|)
-  }
-  if constexpr (MODE == IDX_PREFILL) {
-    if (a.cand != nullptr)
-      for (int i = threadIdx.x; i < C::NQ; i += blockDim.x) sTheta[i] = (i < nq) ? a.theta[q0 + i] : 0.f;
-  }
-  if constexpr (MODE == IDX_GATHER) {
-    // the CTA's kept-block lists, staged once: every role walks them per job
-    for (int i = threadIdx.x; i < C::NQ * C::KEEPMAX; i += blockDim.x) {
-      const int ql = i / C::KEEPMAX, j = i % C::KEEPMAX;
-      sKept[i] = (ql < nq && j < a.keep) ? a.kept[(long long)(q0 + ql) * a.keep + j] : -1;
-    }
-  }
-  if constexpr (MODE == IDX_GROUPED) {
-    // the group's queries and its union blocks with every query's slot
-    const int g = blockIdx.x;
-    const int nub = a.gb_n[g];
-    n_ub = nub;
-    for (int i = threadIdx.x; i < C::NQ; i += blockDim.x) {
-      const int t = a.perm[q0 + i];
-      sQt[i] = (t >= 0 && t < a.n_q) ? t : -1;
-    }
-    for (int i = threadIdx.x; i < nub; i += blockDim.x) {
-      sUBlk[i] = a.gb_blk[(long long)g * a.gb_cap + i];
-      sUSlot[i] = a.gb_slot[(long long)g * a.gb_cap + i];
-    }
-    ntiles = (nub + 1) / 2;
-    njobs = ntiles * geff;
+  if constexpr (!PERSIST) {
+    // one unit per CTA: every thread stages it
+    const int unit = unit_at(0);
+    stage(unit_params(unit), meta(0), threadIdx.x, blockDim.x);
   }
   __syncthreads();
-  if constexpr (MODE == IDX_GROUPED) {
-    bool any = false;
-    for (int ql = 0; ql < C::NQ; ++ql) any |= sQt[ql] >= 0;
-    if (!any) njobs = ntiles = 0;
-  }
   if constexpr (MODE == IDX_GATHER) {
-    for (int ql = 0; ql < nq; ++ql) {
+    const UnitP u = unit_params(unit_at(0));
+    const int* kept = meta(0).kept;
+    for (int ql = 0; ql < u.nq; ++ql) {
       int nb = 0;
-      while (nb < C::KEEPMAX && sKept[ql * C::KEEPMAX + nb] >= 0) ++nb;
-      njobs += (nb + 1) / 2;
+      while (nb < C::KEEPMAX && kept[ql * C::KEEPMAX + nb] >= 0) ++nb;
+      gather_njobs += (nb + 1) / 2;
     }
-    ntiles = njobs;
   }
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
@@ -358,67 +527,77 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 
   if (warp == 0) {
     // ======================= TMA producer =======================
-    if (lane == 0 && njobs > 0) {
-      if constexpr (MODE == IDX_PREFILL || MODE == IDX_DECODE || MODE == IDX_GROUPED) {
-        // the query tile and the first key tiles went out during the setup
-      } else {
-        prefetch_tmap(&qmap);
-        prefetch_tmap(&kmap);
-        mbar_arrive_expect_tx(qfull, nq * H * C::ROWB);
-        for (int ql = 0; ql < nq; ++ql) tma_load_2d(sQ + ql * H * C::ROWB, &qmap, qfull, 0, (q0 + ql) * H);
-      }
-      GatherCursor gc;
-      if constexpr (MODE == IDX_GATHER) gc.init(sKept, C::KEEPMAX, 0, nq);
-      int issued = early;              // the setup issued tiles [0, early)
-      for (int i = early; i < ntiles; ++i) {
-        const int st = i % C::NS, u = i / C::NS;
-        if (!mbar_wait(&kempty[st], (u & 1) ^ 1, wc, 1)) break;
-        ++issued;
-        uint8_t* dst = sK + st * C::KBYTES;
-        if constexpr (MODE == IDX_PREFILL) {
-          mbar_arrive_expect_tx(&kfull[st], C::KBYTES);
-          tma_load_2d(dst, &kmap, &kfull[st], 0, (tile0 + i) * 128);
-        } else if constexpr (MODE == IDX_DECODE) {
-          mbar_arrive_expect_tx(&kfull[st], C::KBYTES);
-          tma_load_2d(dst, &kmap, &kfull[st], 0, seq * a.n_k + (tile0 + i) * 128);
-        } else if constexpr (MODE == IDX_GROUPED) {
-          const int b0 = sUBlk[2 * i];
-          const int b1 = (2 * i + 1 < n_ub) ? sUBlk[2 * i + 1] : -1;
-          mbar_arrive_expect_tx(&kfull[st], (b1 >= 0 ? 2 : 1) * 64 * C::ROWB);
-          tma_load_2d(dst, &kmap, &kfull[st], 0, b0 * 64);
-          if (b1 >= 0) tma_load_2d(dst + 64 * C::ROWB, &kmap, &kfull[st], 0, b1 * 64);
-        } else {
-          const int* kr = gc.row();
-          const int b0 = kr[2 * gc.pair];
-          const int b1 = kr[2 * gc.pair + 1];
-          mbar_arrive_expect_tx(&kfull[st], (b1 >= 0 ? 2 : 1) * 64 * C::ROWB);
-          tma_load_2d(dst, &kmap, &kfull[st], 0, b0 * 64);
-          if (b1 >= 0) tma_load_2d(dst + 64 * C::ROWB, &kmap, &kfull[st], 0, b1 * 64);
-          gc.next();
+    if (lane == 0) {
+      int kc = early;                  // key tiles issued (ring position)
+      int qn[C::QB];                   // query tiles issued per buffer
+#pragma unroll
+      for (int b = 0; b < C::QB; ++b) qn[b] = 0;
+      int bi = 0;                      // buffer uses
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        const int unit = unit_at(it);
+        if (unit < 0) break;
+        const UnitP u = unit_params(unit);
+        if (u.njobs == 0) continue;
+        const int b = bi % C::QB, use = bi / C::QB;
+        ++bi;
+        const bool first = it == early_it;
+        if (!first) {
+          if (use > 0 && !mbar_wait(&qempty[b], (use - 1) & 1, wc, 6)) break;
+          if constexpr (MODE == IDX_GATHER) {
+            prefetch_tmap(&qmap);
+            prefetch_tmap(&kmap);
+          }
+          load_q(u, b);
+        }
+        ++qn[b];
+        GatherCursor gc = {};
+        if constexpr (MODE == IDX_GATHER) gc.init(meta(0).kept, C::KEEPMAX, 0, u.nq);
+        for (int i = first ? early : 0; i < u.ntiles; ++i) {
+          const int st = kc % C::NS;
+          if (kc >= C::NS && !mbar_wait(&kempty[st], ((kc / C::NS) - 1) & 1, wc, 1)) {
+            ok = false;
+            break;
+          }
+          load_tile(u, i, st, gc);
+          ++kc;
         }
       }
       // never leave with copies in flight (matters only after an abort):
       // wait, bounded and regardless of the abort flag, for the last loads
       const WaitCtx drain{abort_flag, nullptr, a.budget};
-      for (int i = max(0, issued - C::NS); i < issued; ++i)
-        mbar_wait_drain(&kfull[i % C::NS], (i / C::NS) & 1, drain);
-      mbar_wait_drain(qfull, 0, drain);
+      for (int i = max(0, kc - C::NS); i < kc; ++i) mbar_wait_drain(&kfull[i % C::NS], (i / C::NS) & 1, drain);
+#pragma unroll
+      for (int b = 0; b < C::QB; ++b)
+        if (qn[b] > 0) mbar_wait_drain(&qfull[b], (qn[b] - 1) & 1, drain);
     }
   } else if (warp == 1) {
     // ======================= MMA issuer =======================
-    if (lane == 0 && njobs > 0) {
+    if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc<FP8 ? 0 : 1, 128, C::N>();
-      if (mbar_wait(qfull, 0, wc, 2)) {
+      int kt0 = 0;                     // key tiles of the earlier units (ring position of the unit's first)
+      int J = 0;                       // jobs of the earlier units (accumulator ring position)
+      int bi = 0;
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        const int unit = unit_at(it);
+        if (unit < 0) break;
+        const UnitP u = unit_params(unit);
+        if (u.njobs == 0) continue;
+        const int b = bi % C::QB, use = bi / C::QB;
+        ++bi;
+        if (!mbar_wait(&qfull[b], use & 1, wc, 2)) break;
         tc_fence_after();
+        const uint8_t* sQ = sQ0 + b * C::QBYTES;
         GatherCursor gc;
-        if constexpr (MODE == IDX_GATHER) gc.init(sKept, C::KEEPMAX, 0, nq);
-        int wtile = 0, wg = 0;             // wide modes: job j = tile * geff + g, advanced without division
-        for (int j = 0; j < njobs; ++j) {
+        if constexpr (MODE == IDX_GATHER) gc.init(meta(0).kept, C::KEEPMAX, 0, u.nq);
+        int wtile = 0, wg = 0;         // wide modes: job j = tile * geff + g, advanced without division
+        for (int j = 0; j < u.njobs; ++j, ++J) {
           int tile, g;
           if constexpr (C::WIDE) {
             tile = wtile;
             g = wg;
-            if (++wg == geff) {
+            if (++wg == u.geff) {
               wg = 0;
               ++wtile;
             }
@@ -426,14 +605,21 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             tile = j;
             g = (MODE == IDX_GATHER) ? gc.ql : 0;
           }
-          const int st = tile % C::NS;
-          const int buf = j % C::NBUF, ub = j / C::NBUF;
+          const int kt = kt0 + tile;
+          const int st = kt % C::NS;
+          const int buf = J % C::NBUF, ub = J / C::NBUF;
           if (g == 0 || !C::WIDE) {
-            if (!mbar_wait(&kfull[st], (tile / C::NS) & 1, wc, 3)) break;
+            if (!mbar_wait(&kfull[st], (kt / C::NS) & 1, wc, 3)) {
+              ok = false;
+              break;
+            }
           }
-          if (!mbar_wait(&tempty[buf], (ub & 1) ^ 1, wc, 4)) break;
+          if (!mbar_wait(&tempty[buf], (ub & 1) ^ 1, wc, 4)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          if (a.hook == SA_HOOK_STALL_WAIT && j == 0) {            // test hook: never signal job 0
+          if (a.hook == SA_HOOK_STALL_WAIT && J == 0) {            // test hook: never signal job 0
             if constexpr (MODE == IDX_GATHER) gc.next();
             continue;
           }
@@ -452,14 +638,17 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
               mma_bf16(d_tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
           }
           mma_commit(&tfull[buf]);
-          if (!C::WIDE || g == geff - 1) mma_commit(&kempty[st]);
+          if (!C::WIDE || g == u.geff - 1) mma_commit(&kempty[st]);
           if constexpr (MODE == IDX_GATHER) gc.next();
         }
+        if (!ok) break;
+        mma_commit(&qempty[b]);        // the buffer is free once this unit's MMAs are done
+        kt0 += u.ntiles;
       }
     }
-  } else {
+  } else if (warp < kStagerWarp) {
     // ======================= epilogue teams =======================
-    const int team = (warp - 2) / C::WPT;    // jobs j with j % TEAMS == team
+    const int team = (warp - 2) / C::WPT;    // jobs J with J % TEAMS == team
     const int slice = ((warp - 2) % C::WPT) >> 2;   // the accumulator columns [slice * SCOLS, +SCOLS)
     const int lq = warp & 3;                 // TMEM lane quarter this warp may access
     // FP8 modes drain TMEM with the 16x256b shape: thread (quad r = lane / 4,
@@ -480,12 +669,19 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       bool kvalid;
       float sk;
     };
+    // the current unit, as the job lambdas below read it
+    int q0 = 0, nq = 0, seq = 0, tile0 = 0, geff = 1, njobs = 0, n_ub = 0, seq_len = a.n_k;
+    const float* sW = nullptr;
+    const int* sKept = nullptr;
+    const float* sTheta = nullptr;
+    const unsigned long long* sUSlot = nullptr;
+    const int* sUBlk = nullptr;
+    const int* sQt = nullptr;
     GatherCursor gc = {};                    // gather: cursor at the job being loaded
     int jq = 0;
-    if constexpr (MODE == IDX_GATHER) gc.init(sKept, C::KEEPMAX, 0, nq);
     // wide modes: (tile, sub-tile) of the job job_key is asked for next; the
     // team's jobs advance by TEAMS, which moves these without a division
-    int ktile = C::WIDE ? team / geff : 0, kg = C::WIDE ? team % geff : 0;
+    int ktile = 0, kg = 0;
     auto job_key = [&](int jj) {
       JobKey k;
       if constexpr (MODE == IDX_GATHER) {
@@ -557,16 +753,58 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         t = q0 + ql_;
       return (t >= n_rows) ? -1 : t;
     };
-    JobKey nxt = job_key(team);
-    for (int j = team; j < njobs; j += C::TEAMS) {
-      const JobKey cur = nxt;
-      nxt = job_key(j + C::TEAMS);
-      const int ql = cur.ql, g = cur.g, s = cur.s, col = cur.col;
-      const bool kvalid = cur.kvalid;
-      const float sk = cur.sk;
-      const int buf = j % C::NBUF, ub = j / C::NBUF;    // buffer buf is always drained by team buf % TEAMS
-      if (!mbar_wait(&tfull[buf], ub & 1, wc, 5)) break;
-      tc_fence_after();
+    int J0 = 0;                              // jobs of the earlier units
+    int bi = 0;
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+      const int unit = unit_at(it);
+      if (unit < 0) break;
+      const UnitP u = unit_params(unit);
+      if (u.njobs == 0) continue;
+      const int bm = bi % C::QB, usem = bi / C::QB;
+      ++bi;
+      if (PERSIST && !mbar_wait(&mfull[bm], usem & 1, wc, 7)) break;
+      const Meta m = meta(bm);
+      sW = m.w;
+      sKept = m.kept;
+      sTheta = m.theta;
+      sUSlot = m.uslot;
+      sUBlk = m.ublk;
+      sQt = m.qt;
+      q0 = u.q0;
+      nq = u.nq;
+      seq = u.seq;
+      tile0 = u.tile0;
+      geff = u.geff;
+      njobs = u.njobs;
+      n_ub = u.n_ub;
+      seq_len = u.seq_len;
+      wg = -1;                               // new weights and limits
+      // this team's first job of the unit: the smallest local j with
+      // (J0 + j) % TEAMS == team
+      const int jfirst = ((team - J0) % C::TEAMS + C::TEAMS) % C::TEAMS;
+      if constexpr (C::WIDE) {
+        ktile = jfirst / geff;
+        kg = jfirst % geff;
+      }
+      if constexpr (MODE == IDX_GATHER) {
+        gc.init(sKept, C::KEEPMAX, 0, nq);
+        jq = 0;
+      }
+      JobKey nxt = job_key(jfirst);
+      for (int j = jfirst; j < njobs; j += C::TEAMS) {
+        const JobKey cur = nxt;
+        nxt = job_key(j + C::TEAMS);
+        const int ql = cur.ql, g = cur.g, s = cur.s, col = cur.col;
+        const bool kvalid = cur.kvalid;
+        const float sk = cur.sk;
+        const int Jg = J0 + j;
+        const int buf = Jg % C::NBUF, ub = Jg / C::NBUF;   // buffer buf is always drained by team buf % TEAMS
+        if (!mbar_wait(&tfull[buf], ub & 1, wc, 5)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
 
       float qsum[C::QSW];                      // sum_h w'[h] * ReLU(acc[h]) of this thread's key row, per query
       // grouped, two queries per warp: the jobs skip queries per warp below,
@@ -860,6 +1098,30 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           if (col < a.n_k) a.out[(long long)t * a.ld + col] = score;
         }
       }
+      }
+      J0 += njobs;
+      if constexpr (PERSIST) {                 // this warp is done with the unit's metadata
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&mempty[bm]);
+      }
+    }
+  } else {
+    // ======================= metadata stager =======================
+    // persistent modes: stages each unit's weights and lists into the
+    // metadata buffer its epilogue reads, up to two units ahead
+    if constexpr (PERSIST) {
+      int bi = 0;
+      for (int it = 0;; ++it) {
+        const int unit = unit_at(it);
+        if (unit < 0) break;
+        const UnitP u = unit_params(unit);
+        if (u.njobs == 0) continue;
+        const int b = bi % C::QB, use = bi / C::QB;
+        ++bi;
+        if (use > 0 && !mbar_wait(&mempty[b], (use - 1) & 1, wc, 8)) break;
+        stage_warp(u, meta(b));
+        mbar_arrive(&mfull[b]);                // each lane after its own stores
+      }
     }
   }
 
@@ -886,14 +1148,19 @@ static cudaError_t launch_t(const void* q, const void* k, int q_rows, long long 
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid;
-  if constexpr (MODE == IDX_PREFILL)
-    grid = dim3((a.n_q + C::NQ - 1) / C::NQ);
-  else if constexpr (MODE == IDX_DECODE)
+  if constexpr (C::PERSIST) {
+    // one persistent CTA per SM (at most one per unit)
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int units = (MODE == IDX_PREFILL) ? (a.n_q + C::NQ - 1) / C::NQ : a.n_groups;
+    grid = dim3(units < sms ? units : sms);
+  } else if constexpr (MODE == IDX_DECODE) {
     grid = dim3(((a.span + 127) / 128 + a.tiles_per_cta - 1) / a.tiles_per_cta, a.n_q);
-  else if constexpr (MODE == IDX_GROUPED)
-    grid = dim3(a.n_groups);
-  else
+  } else {
     grid = dim3((a.n_q + C::NQ - 1) / C::NQ);
+  }
   if (grid.x == 0 || grid.y == 0) return cudaSuccess;
   kern<<<grid, C::THREADS, C::SMEM, st>>>(qm, km, a);
   return cudaGetLastError();
