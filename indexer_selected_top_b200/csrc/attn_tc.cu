@@ -17,6 +17,10 @@
 // The union lists (ascending keys, padded with -1 / mask 0 to whole chunks)
 // come from group_union_kernel.
 //
+// One persistent CTA per SM loops over its groups; chunks are counted across
+// groups, so the K/V ring and the S buffers run on from one group to the
+// next, and the next group's first S products overlap the O write-back of
+// the one before (its first O += P V waits until that O has been read).
 // Roles (288 threads): warp 0 allocates TMEM and one lane issues the MMAs;
 // warps 1-4 gather 32 keys each of every chunk (16-byte cp.async, whole rows
 // per 16 lanes) into 128-byte-swizzled tiles, publishing them on an mbarrier
@@ -92,8 +96,8 @@ struct TcSmem {
   static constexpr int STAGE = 4 * KV_HALF + KX;          // K0 K1 V0 V1 KX = 68 KB
   static constexpr int OFF_KV = 0;
   static constexpr int OFF_BAR = OFF_KV + TC_ST * STAGE;
-  // full[ST] empty[ST] sfull[2] pfull[2] pvdone[2] qfull drain
-  static constexpr int N_BAR = 2 * TC_ST + 8;
+  // full[ST] empty[ST] sfull[2] pfull[2] pvdone[2] qfull drain ofree
+  static constexpr int N_BAR = 2 * TC_ST + 9;
   static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
   static constexpr int SMEM = OFF_MISC + 64 + 1024;      // + slack for 1024-byte alignment
   static_assert(SMEM <= 227 * 1024, "shared memory");
@@ -104,8 +108,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
                    const __nv_bfloat16* __restrict__ vc, const int* __restrict__ list,
                    const uint8_t* __restrict__ lmask, const int* __restrict__ n_list, const int* __restrict__ perm,
-                   int n_q, int cap, float scale_log2, __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
-                   uint32_t* status, long long budget) {
+                   int n_groups, int n_q, int cap, float scale_log2, __nv_bfloat16* __restrict__ out,
+                   float* __restrict__ lse, uint32_t* status, long long budget) {
   using L = TcSmem;
   extern __shared__ uint8_t tc_raw[];
   uint8_t* sm = smem_align1024(tc_raw);
@@ -117,17 +121,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t* pvdone = pfull + 2;
   uint64_t* qfull = pvdone + 2;
   uint64_t* drain = qfull + 1;
+  uint64_t* ofree = drain + 1;                   // the softmax has read the group's O
   uint32_t* misc = reinterpret_cast<uint32_t*>(sm + L::OFF_MISC);
   uint32_t* tmem_slot = misc;
   volatile uint32_t* abort_flag = misc + 1;
-  int* qt = reinterpret_cast<int*>(misc + 2);     // [TC_GA]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = blockIdx.x;
-  const int nl = n_list[g];
-  const int nch = (nl + TC_CH - 1) / TC_CH;
-  const int* glist = list + (long long)g * cap;
-  const uint8_t* gmask = lmask + (long long)g * cap;
+  // the CTA's groups: blockIdx.x, + gridDim.x, ... (one CTA per SM). Chunks
+  // are counted across them (c), so the K/V ring, the two S buffers and their
+  // barrier phases run on from one group to the next; a group with no keys
+  // touches none of them
+  auto group_at = [&](int it) -> int {
+    const long long g = (long long)it * gridDim.x + blockIdx.x;
+    return g < n_groups ? (int)g : -1;
+  };
+  auto n_chunks = [&](int g) { return (n_list[g] + TC_CH - 1) / TC_CH; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < TC_ST; ++s) {
@@ -141,13 +149,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     mbar_init(qfull, 128);
     mbar_init(drain, 1);
+    mbar_init(ofree, 128);
     *abort_flag = 0u;
     fence_barrier_init();
-  }
-  if (threadIdx.x < TC_GA) {
-    const int j = g * TC_GA + threadIdx.x;
-    const int t = perm ? perm[j] : j;
-    qt[threadIdx.x] = (t >= 0 && t < n_q) ? t : -1;
   }
   if (warp == 0) tmem_alloc<512>(tmem_slot);
   __syncthreads();
@@ -157,17 +161,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   if (warp == 0) {
     // ============================ MMA issuer ============================
-    // S(i) = Q K^T of chunk i into S buffer i % 2 (Q and its mask dims read
-    // from tensor memory); O += P(j) V(j) with P read from the S buffer the
-    // softmax overwrote. S(j + 1) is issued before O += P(j) V(j), once the
-    // buffer's previous P has been consumed.
-    if (lane == 0 && nch > 0) {
+    // S(c) = Q K^T of chunk c into S buffer c % 2 (Q and its mask dims read
+    // from tensor memory); O += P(c) V(c) with P read from the S buffer the
+    // softmax overwrote. S(c + 1) is issued before O += P(c) V(c), once the
+    // buffer's previous P has been consumed; a group's first O += P V (which
+    // starts O afresh) waits until the softmax has read the previous group's O.
+    if (lane == 0) {
       constexpr uint32_t idesc_s = umma_idesc<1, 128, TC_CH>();
       constexpr uint32_t idesc_o = umma_idesc_bmn<1, 128, TC_DH>();
-      auto issue_s = [&](int i) -> bool {
-        const int s = i % TC_ST, b = i & 1;
-        if (!mbar_wait(&full[s], (i / TC_ST) & 1, wc, 40)) return false;
-        if (i >= 2 && !mbar_wait(&pvdone[b], ((i - 2) >> 1) & 1, wc, 41)) return false;
+      auto issue_s = [&](int c) -> bool {
+        const int s = c % TC_ST, b = c & 1;
+        if (!mbar_wait(&full[s], (c / TC_ST) & 1, wc, 40)) return false;
+        if (c >= 2 && !mbar_wait(&pvdone[b], ((c - 2) >> 1) & 1, wc, 41)) return false;
         tc_fence_after();
         const uint32_t k_base = smem_u32(sm + L::OFF_KV + s * L::STAGE);
         const uint32_t d = tmem + TC_S_COL + b * TC_CH;
@@ -181,25 +186,45 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         mma_commit(&sfull[b]);
         return true;
       };
-      bool ok = mbar_wait(qfull, 0, wc, 42);
-      if (ok) {
+      int c0 = 0, gi = 0;                // chunks and non-empty groups before this one
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        const int g = group_at(it);
+        if (g < 0) break;
+        const int nch = n_chunks(g);
+        if (nch == 0) continue;
+        ok = mbar_wait(qfull, gi & 1, wc, 42);
+        if (!ok) break;
         tc_fence_after();
-        ok = issue_s(0);
-      }
-      for (int j = 0; ok && j < nch; ++j) {
-        if (j + 1 < nch && !issue_s(j + 1)) break;
-        if (!mbar_wait(&pfull[j & 1], (j >> 1) & 1, wc, 43)) break;
-        tc_fence_after();
-        const uint32_t v_base = smem_u32(sm + L::OFF_KV + (j % TC_ST) * L::STAGE + 2 * L::KV_HALF);
-        const uint32_t p_col = tmem + TC_S_COL + (j & 1) * TC_CH;
+        ok = issue_s(c0);
+        for (int j = 0; ok && j < nch; ++j) {
+          const int c = c0 + j;
+          if (j + 1 < nch && !issue_s(c + 1)) {
+            ok = false;
+            break;
+          }
+          if (!mbar_wait(&pfull[c & 1], (c >> 1) & 1, wc, 43)) {
+            ok = false;
+            break;
+          }
+          if (j == 0 && gi > 0 && !mbar_wait(ofree, (gi - 1) & 1, wc, 48)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t v_base = smem_u32(sm + L::OFF_KV + (c % TC_ST) * L::STAGE + 2 * L::KV_HALF);
+          const uint32_t p_col = tmem + TC_S_COL + (c & 1) * TC_CH;
 #pragma unroll
-        for (int kk = 0; kk < TC_CH / 16; ++kk) {
-          // 16 keys = two 8-key atoms of 1024 B; the two 64-dim halves 16 KB apart
-          const uint64_t bd = umma_desc_sw128(v_base + kk * 2048, L::KV_HALF, 1024);
-          mma_bf16_ts(tmem + TC_O_COL, p_col + kk * 8, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < TC_CH / 16; ++kk) {
+            // 16 keys = two 8-key atoms of 1024 B; the two 64-dim halves 16 KB apart
+            const uint64_t bd = umma_desc_sw128(v_base + kk * 2048, L::KV_HALF, 1024);
+            mma_bf16_ts(tmem + TC_O_COL, p_col + kk * 8, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[c % TC_ST]);
+          mma_commit(&pvdone[c & 1]);
         }
-        mma_commit(&empty[j % TC_ST]);
-        mma_commit(&pvdone[j & 1]);
+        c0 += nch;
+        ++gi;
       }
       // every MMA issued has completed before tensor memory is released
       mma_commit(drain);
@@ -213,51 +238,60 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // and masks are read before waiting for its ring stage.
     const int lw = warp - 1;
     const int seg = lane & 15, half = seg >> 3, c16 = seg & 7;
-    int key = 0;
-    uint32_t msk = 0u;
-    if (nch > 0) {
-      key = glist[lw * 32 + lane];
-      msk = gmask[lw * 32 + lane];
-    }
-    for (int j = 0; j < nch; ++j) {
-      const int s = j % TC_ST;
-      int n_key = 0;
-      uint32_t n_msk = 0u;
-      if (j + 1 < nch) {
-        n_key = glist[(j + 1) * TC_CH + lw * 32 + lane];
-        n_msk = gmask[(j + 1) * TC_CH + lw * 32 + lane];
-      }
-      if (j >= TC_ST && !mbar_wait(&empty[s], ((j / TC_ST) - 1) & 1, wc, 44)) break;
-      const int kr = max(key, 0);                   // padding (-1): any valid row, its mask byte is 0
-      uint8_t* st = sm + L::OFF_KV + s * L::STAGE;
-#pragma unroll 4
-      for (int i = 0; i < 16; ++i) {
-        const int rl = 2 * i + (lane >> 4);         // this warp's row
-        const int r = lw * 32 + rl;                 // row of the chunk
-        const long long src = (long long)__shfl_sync(0xffffffffu, kr, rl) * TC_DH + seg * 8;
-        const uint32_t off = half * L::KV_HALF + r * 128 + ((c16 ^ (r & 7)) << 4);
-        cp_async16(smem_u32(st + off), kc + src);
-        cp_async16(smem_u32(st + 2 * L::KV_HALF + off), vc + src);
-      }
-      // mask dims of this lane's key: dims 0-7 carry the bias for the
-      // queries that did not select it, dims 8-15 are 0
-      {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t lo = ((msk >> (2 * e)) & 1u) ? 0u : TC_MASK_BF16;
-          const uint32_t hi = ((msk >> (2 * e + 1)) & 1u) ? 0u : TC_MASK_BF16;
-          w[e] = lo | (hi << 16);
+    int c = 0;                               // chunks of the earlier groups
+    bool ok = true;
+    for (int it = 0; ok; ++it) {
+      const int g = group_at(it);
+      if (g < 0) break;
+      const int nch = n_chunks(g);
+      if (nch == 0) continue;
+      const int* glist = list + (long long)g * cap;
+      const uint8_t* gmask = lmask + (long long)g * cap;
+      int key = glist[lw * 32 + lane];
+      uint32_t msk = gmask[lw * 32 + lane];
+      for (int j = 0; j < nch; ++j, ++c) {
+        const int s = c % TC_ST;
+        int n_key = 0;
+        uint32_t n_msk = 0u;
+        if (j + 1 < nch) {
+          n_key = glist[(j + 1) * TC_CH + lw * 32 + lane];
+          n_msk = gmask[(j + 1) * TC_CH + lw * 32 + lane];
         }
-        uint8_t* kx = st + 4 * L::KV_HALF;
-        const int row = lw * 32 + lane;
-        *reinterpret_cast<uint4*>(kx + row * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<uint4*>(kx + L::KX / 2 + row * 16) = make_uint4(0u, 0u, 0u, 0u);
+        if (c >= TC_ST && !mbar_wait(&empty[s], ((c / TC_ST) - 1) & 1, wc, 44)) {
+          ok = false;
+          break;
+        }
+        const int kr = max(key, 0);                   // padding (-1): any valid row, its mask byte is 0
+        uint8_t* st = sm + L::OFF_KV + s * L::STAGE;
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const int rl = 2 * i + (lane >> 4);         // this warp's row
+          const int r = lw * 32 + rl;                 // row of the chunk
+          const long long src = (long long)__shfl_sync(0xffffffffu, kr, rl) * TC_DH + seg * 8;
+          const uint32_t off = half * L::KV_HALF + r * 128 + ((c16 ^ (r & 7)) << 4);
+          cp_async16(smem_u32(st + off), kc + src);
+          cp_async16(smem_u32(st + 2 * L::KV_HALF + off), vc + src);
+        }
+        // mask dims of this lane's key: dims 0-7 carry the bias for the
+        // queries that did not select it, dims 8-15 are 0
+        {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t lo = ((msk >> (2 * e)) & 1u) ? 0u : TC_MASK_BF16;
+            const uint32_t hi = ((msk >> (2 * e + 1)) & 1u) ? 0u : TC_MASK_BF16;
+            w[e] = lo | (hi << 16);
+          }
+          uint8_t* kx = st + 4 * L::KV_HALF;
+          const int row = lw * 32 + lane;
+          *reinterpret_cast<uint4*>(kx + row * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(kx + L::KX / 2 + row * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+        cp_async_publish(&full[s]);
+        key = n_key;
+        msk = n_msk;
       }
-      fence_proxy_async_smem();
-      cp_async_publish(&full[s]);
-      key = n_key;
-      msk = n_msk;
     }
     cp_async_wait_all();   // no copy may land after the CTA has left
   } else {
@@ -265,148 +299,162 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int qw = warp & 3;                  // TMEM lane quarter of this warp
     const int r = qw * 32 + lane;             // row = 16 * query + head
     const int qi = r >> 4, h = r & 15;
-    const int t = qt[qi];
     const uint32_t t_row = tmem + (uint32_t(qw * 32) << 16);
-    {
-      // this row of Q (bf16 pairs: column c holds dims 2c, 2c + 1) and the
-      // one-hot of its query in the mask dims
-      uint32_t qv[32];
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        if (t >= 0) {
-          const uint4* src = reinterpret_cast<const uint4*>(q + ((long long)t * TC_HQ + h) * TC_DH + hh * 64);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint4 v = src[i];
-            qv[4 * i] = v.x;
-            qv[4 * i + 1] = v.y;
-            qv[4 * i + 2] = v.z;
-            qv[4 * i + 3] = v.w;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) qv[i] = 0u;
-        }
-        tmem_st32(t_row + TC_Q_COL + hh * 32, *reinterpret_cast<const float(*)[32]>(qv));
-      }
-      uint32_t qx[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        qx[e] = (qi == 2 * e ? 0x3F80u : 0u) | (qi == 2 * e + 1 ? 0x3F800000u : 0u);   // bf16 1.0 at dim qi
-      tmem_st8(t_row + TC_QX_COL, qx);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(qfull);
-    }
-    float m_used = -INFINITY, l = 0.f;
+    int c0 = 0, gi = 0;                       // chunks and non-empty groups before this one
     bool ok = true;
-    for (int j = 0; j < nch; ++j) {
-      const int b = j & 1;
-      const uint32_t s_row = t_row + TC_S_COL + b * TC_CH;
-      ok = __all_sync(0xffffffffu, mbar_wait(&sfull[b], (j >> 1) & 1, wc, 45));
-      if (!ok) break;
-      tc_fence_after();
-      // pass 1: the row max over the chunk (masked keys sit below -2^99;
-      // the scale is positive, so it commutes with the max)
-      float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int cb = 0; cb < TC_CH / 32; ++cb) {
-        float sv[32];
-        tmem_ld32(s_row + cb * 32, sv);
-        tmem_ld_wait();
-        tmem_regs_ready(sv);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) mq[c & 3] = fmaxf(mq[c & 3], sv[c]);
+    for (int it = 0; ok; ++it) {
+      const int g = group_at(it);
+      if (g < 0) break;
+      const int nch = n_chunks(g);
+      const int tq = perm ? perm[g * TC_GA + qi] : g * TC_GA + qi;
+      const int t = (tq >= 0 && tq < n_q) ? tq : -1;
+      if (nch == 0) {                         // no keys: a zero row and lse = -inf
+        if (t >= 0) {
+          __nv_bfloat16* dst = out + ((long long)t * TC_HQ + h) * TC_DH;
+          for (int i = 0; i < TC_DH; i += 8) *reinterpret_cast<uint4*>(dst + i) = make_uint4(0u, 0u, 0u, 0u);
+          if (lse != nullptr) lse[(long long)t * TC_HQ + h] = -INFINITY;
+        }
+        continue;
       }
-      float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-      mx = mx < TC_MASKED ? -INFINITY : mx * scale_log2;    // no key of the chunk is the row's
-      const float m_new = fmaxf(m_used, mx);
-      const bool resc = m_used != -INFINITY && m_new > m_used + TC_RESCALE;
-      if (m_used == -INFINITY) m_used = m_new;          // the row's O is still 0
-      if (__any_sync(0xffffffffu, resc)) {
-        // O must hold every earlier chunk before it is rescaled in place
-        ok = __all_sync(0xffffffffu, mbar_wait(&pvdone[(j - 1) & 1], ((j - 1) >> 1) & 1, wc, 47));
+      {
+        // this row of Q (bf16 pairs: column c holds dims 2c, 2c + 1) and the
+        // one-hot of its query in the mask dims; every S product of the
+        // previous group has completed (this thread waited for the last)
+        uint32_t qv[32];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          if (t >= 0) {
+            const uint4* src = reinterpret_cast<const uint4*>(q + ((long long)t * TC_HQ + h) * TC_DH + hh * 64);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint4 v = src[i];
+              qv[4 * i] = v.x;
+              qv[4 * i + 1] = v.y;
+              qv[4 * i + 2] = v.z;
+              qv[4 * i + 3] = v.w;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) qv[i] = 0u;
+          }
+          tmem_st32(t_row + TC_Q_COL + hh * 32, *reinterpret_cast<const float(*)[32]>(qv));
+        }
+        uint32_t qx[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          qx[e] = (qi == 2 * e ? 0x3F80u : 0u) | (qi == 2 * e + 1 ? 0x3F800000u : 0u);   // bf16 1.0 at dim qi
+        tmem_st8(t_row + TC_QX_COL, qx);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(qfull);
+      }
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < nch; ++j) {
+        const int c = c0 + j, b = c & 1;
+        const uint32_t s_row = t_row + TC_S_COL + b * TC_CH;
+        ok = __all_sync(0xffffffffu, mbar_wait(&sfull[b], (c >> 1) & 1, wc, 45));
         if (!ok) break;
         tc_fence_after();
-        const float alpha = resc ? exp2f(m_used - m_new) : 1.f;
+        // pass 1: the row max over the chunk (masked keys sit below -2^99;
+        // the scale is positive, so it commutes with the max)
+        float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int cb = 0; cb < TC_DH / 32; ++cb) {
-          float ov[32];
-          tmem_ld32(t_row + TC_O_COL + cb * 32, ov);
+        for (int cb = 0; cb < TC_CH / 32; ++cb) {
+          float sv[32];
+          tmem_ld32(s_row + cb * 32, sv);
           tmem_ld_wait();
-          tmem_regs_ready(ov);
+          tmem_regs_ready(sv);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-          tmem_st32(t_row + TC_O_COL + cb * 32, ov);
+          for (int cc = 0; cc < 32; ++cc) mq[cc & 3] = fmaxf(mq[cc & 3], sv[cc]);
         }
+        float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+        mx = mx < TC_MASKED ? -INFINITY : mx * scale_log2;    // no key of the chunk is the row's
+        const float m_new = fmaxf(m_used, mx);
+        const bool resc = m_used != -INFINITY && m_new > m_used + TC_RESCALE;
+        if (m_used == -INFINITY) m_used = m_new;          // the row's O is still 0
+        if (__any_sync(0xffffffffu, resc)) {
+          // O must hold every earlier chunk of the group before it is rescaled in place
+          ok = __all_sync(0xffffffffu, mbar_wait(&pvdone[(c - 1) & 1], ((c - 1) >> 1) & 1, wc, 47));
+          if (!ok) break;
+          tc_fence_after();
+          const float alpha = resc ? exp2f(m_used - m_new) : 1.f;
+#pragma unroll
+          for (int cb = 0; cb < TC_DH / 32; ++cb) {
+            float ov[32];
+            tmem_ld32(t_row + TC_O_COL + cb * 32, ov);
+            tmem_ld_wait();
+            tmem_regs_ready(ov);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+            tmem_st32(t_row + TC_O_COL + cb * 32, ov);
+          }
+          tmem_st_wait();
+          if (resc) {
+            l *= alpha;
+            m_used = m_new;
+          }
+        }
+        // pass 2: p = 2^(s * scale_log2 - m) (one FMA and one ex2 per key; a
+        // masked key lands far below the normal range and gives exactly 0),
+        // packed to bf16 pairs over the S columns already read: keys 32 cb ..
+        // 32 cb + 31 go to columns 16 cb .. 16 cb + 15
+        const float msub = m_used == -INFINITY ? 0.f : m_used;
+        float2 l2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int cb = 0; cb < TC_CH / 32; ++cb) {
+          float sv[32];
+          tmem_ld32(s_row + cb * 32, sv);
+          tmem_ld_wait();
+          tmem_regs_ready(sv);
+          uint32_t pw[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2_approx(fmaf(sv[2 * e], scale_log2, -msub));
+            const float p1 = ex2_approx(fmaf(sv[2 * e + 1], scale_log2, -msub));
+            const __nv_bfloat162 pv = __floats2bfloat162_rn(p0, p1);
+            l2 = __fadd2_rn(l2, make_float2(p0, p1));      // the row sum in fp32, as lse needs
+            pw[e] = *reinterpret_cast<const uint32_t*>(&pv);
+          }
+          tmem_st16(s_row + cb * 16, pw);
+        }
+        l += l2.x + l2.y;
         tmem_st_wait();
-        if (resc) {
-          l *= alpha;
-          m_used = m_new;
-        }
+        tc_fence_before();
+        mbar_arrive(&pfull[b]);
       }
-      // pass 2: p = 2^(s * scale_log2 - m) (one FMA and one ex2 per key; a
-      // masked key lands far below the normal range and gives exactly 0),
-      // packed to bf16 pairs over the S columns already read: keys 32 cb ..
-      // 32 cb + 31 go to columns 16 cb .. 16 cb + 15
-      const float msub = m_used == -INFINITY ? 0.f : m_used;
-      float2 l2 = make_float2(0.f, 0.f);
+      if (!ok) break;
+      // epilogue: O / l in bf16, lse in natural log; then O is free for the
+      // next group's first O += P V
+      const int cl = c0 + nch - 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&pvdone[cl & 1], (cl >> 1) & 1, wc, 49));
+      if (!ok) break;
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* dst = out + ((long long)(t < 0 ? 0 : t) * TC_HQ + h) * TC_DH;
 #pragma unroll
-      for (int cb = 0; cb < TC_CH / 32; ++cb) {
-        float sv[32];
-        tmem_ld32(s_row + cb * 32, sv);
+      for (int cb = 0; cb < TC_DH / 32; ++cb) {
+        float ov[32];
+        tmem_ld32(t_row + TC_O_COL + cb * 32, ov);
         tmem_ld_wait();
-        tmem_regs_ready(sv);
-        uint32_t pw[16];
+        tmem_regs_ready(ov);
+        if (t >= 0) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2_approx(fmaf(sv[2 * e], scale_log2, -msub));
-          const float p1 = ex2_approx(fmaf(sv[2 * e + 1], scale_log2, -msub));
-          const __nv_bfloat162 pv = __floats2bfloat162_rn(p0, p1);
-          l2 = __fadd2_rn(l2, make_float2(p0, p1));      // the row sum in fp32, as lse needs
-          pw[e] = *reinterpret_cast<const uint32_t*>(&pv);
-        }
-        tmem_st16(s_row + cb * 16, pw);
-      }
-      l += l2.x + l2.y;
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&pfull[b]);
-    }
-    // epilogue: O / l in bf16, lse in natural log
-    if (ok && nch > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&pvdone[(nch - 1) & 1], ((nch - 1) >> 1) & 1, wc, 49));
-      if (ok) {
-        tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        __nv_bfloat16* dst = out + ((long long)(t < 0 ? 0 : t) * TC_HQ + h) * TC_DH;
-#pragma unroll
-        for (int cb = 0; cb < TC_DH / 32; ++cb) {
-          float ov[32];
-          tmem_ld32(t_row + TC_O_COL + cb * 32, ov);
-          tmem_ld_wait();
-          tmem_regs_ready(ov);
-          if (t >= 0) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              uint4 pk;
-              pk.x = pack_bf16(ov[i] * inv, ov[i + 1] * inv);
-              pk.y = pack_bf16(ov[i + 2] * inv, ov[i + 3] * inv);
-              pk.z = pack_bf16(ov[i + 4] * inv, ov[i + 5] * inv);
-              pk.w = pack_bf16(ov[i + 6] * inv, ov[i + 7] * inv);
-              *reinterpret_cast<uint4*>(dst + cb * 32 + i) = pk;
-            }
+          for (int i = 0; i < 32; i += 8) {
+            uint4 pk;
+            pk.x = pack_bf16(ov[i] * inv, ov[i + 1] * inv);
+            pk.y = pack_bf16(ov[i + 2] * inv, ov[i + 3] * inv);
+            pk.z = pack_bf16(ov[i + 4] * inv, ov[i + 5] * inv);
+            pk.w = pack_bf16(ov[i + 6] * inv, ov[i + 7] * inv);
+            *reinterpret_cast<uint4*>(dst + cb * 32 + i) = pk;
           }
         }
       }
-    }
-    if (t >= 0 && (ok || nch == 0)) {
-      if (nch == 0) {
-        __nv_bfloat16* dst = out + ((long long)t * TC_HQ + h) * TC_DH;
-        for (int i = 0; i < TC_DH; i += 8) *reinterpret_cast<uint4*>(dst + i) = make_uint4(0u, 0u, 0u, 0u);
-      }
-      if (lse != nullptr)
+      tc_fence_before();
+      mbar_arrive(ofree);
+      if (t >= 0 && lse != nullptr)
         lse[(long long)t * TC_HQ + h] = l > 0.f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      c0 += nch;
+      ++gi;
     }
   }
 
@@ -427,9 +475,15 @@ cudaError_t launch_attention_tc(const void* q, const void* kc, const void* vc, c
   cudaError_t e =
       cudaFuncSetAttribute(tc_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TcSmem::SMEM);
   if (e != cudaSuccess) return e;
-  tc_attn_kernel<<<n_groups, TC_THREADS, TcSmem::SMEM, st>>>(
-      (const __nv_bfloat16*)q, (const __nv_bfloat16*)kc, (const __nv_bfloat16*)vc, list, lmask, n_list, perm, n_q,
-      cap, scale * 1.4426950408889634f, (__nv_bfloat16*)out, lse, status, budget);
+  // one persistent CTA per SM (at most one per group)
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int grid = n_groups < sms ? n_groups : sms;
+  tc_attn_kernel<<<grid, TC_THREADS, TcSmem::SMEM, st>>>(
+      (const __nv_bfloat16*)q, (const __nv_bfloat16*)kc, (const __nv_bfloat16*)vc, list, lmask, n_list, perm,
+      n_groups, n_q, cap, scale * 1.4426950408889634f, (__nv_bfloat16*)out, lse, status, budget);
   return cudaGetLastError();
 }
 
