@@ -127,7 +127,20 @@ __global__ void __launch_bounds__(TW_WARPS * 32)
   if (n_other <= keep - 2) {
     for (int b = 1 + lane; b <= n_other; b += 32) atomicOr(&flags[b >> 5], 1u << (b & 31));
   } else {
-    for (int i = lane; i < n_other; i += 32) keys[i] = tw_key(row[1 + i]);
+    // the row's scores, eight loads per lane in flight before any is stored
+    for (int i0 = 0; i0 < n_other; i0 += 32 * 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + lane + 32 * u;
+        v[u] = (i < n_other) ? row[1 + i] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + lane + 32 * u;
+        if (i < n_other) keys[i] = tw_key(v[u]);
+      }
+    }
     __syncwarp();
     uint32_t cut;
     int ties;
