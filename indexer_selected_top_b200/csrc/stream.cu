@@ -91,8 +91,13 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
     }
     uint32_t prefix = 0;
     int pbits = 0;
-    while (pbits < 32) {                    // 12 + 12 + 8 bits: the exact n_theta-th key
-      const int db = (pbits == 24) ? 8 : TK_HBITS;
+    // two 12-bit passes fix the n_theta-th key to its top 24 bits; theta is
+    // the smallest key with that prefix, so it lists at least the exact
+    // threshold's keys (any threshold keeps the selection exact; a third pass
+    // for the last 8 bits would shorten the list by the few samples within
+    // 2^-15 of it)
+    while (pbits < 24) {
+      const int db = TK_HBITS;
       const int nbins = 1 << db;
       for (int b = tid; b < nbins; b += TK_THREADS) sh.hist[b] = 0;
       __syncthreads();
@@ -114,7 +119,8 @@ __global__ void __launch_bounds__(TK_THREADS, 1)
       pbits += db;
       __syncthreads();
     }
-    th = key_to_float(prefix);
+    // the bucket below every finite score is -inf's (its other keys are NaN patterns)
+    th = ((prefix << 8) < 0x00800000u) ? -INFINITY : key_to_float(prefix << 8);
   }
   if (tid == 0) theta[t] = th;
 }
