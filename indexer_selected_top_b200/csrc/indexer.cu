@@ -365,7 +365,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       }
     }
   };
-  // a unit's metadata into buffer m, by threads tid = 0.. of nthr
+  // a unit's metadata into buffer m, by threads tid = 0.. of nthr (the
+  // one-unit modes: every thread of the CTA, before the setup barrier)
   auto stage = [&](const UnitP& u, const Meta& m, int tid, int nthr) {
     for (int i = tid; i < C::NQ * H; i += nthr) {
       const int ql = i / H, h = i % H;
